@@ -1,0 +1,220 @@
+"""Seeded synthetic workloads for the Qwen-Image-2.1 single-stream DiT step.
+
+This module holds shapes, seeds and value distributions only; it performs none
+of the method's arithmetic.  Both the CUDA path (through the tests and the
+benchmark) and the CPU oracle receive the tensors drawn here, so the two sides
+see bit-identical inputs.
+
+Draws use torch's CPU generator (``torch.Generator``, one per named tensor,
+seeded from the workload seed and the tensor's name), the same kind of draw the
+RGBA-Image-2.1 Core AI port describes for its initial noise ("Use it":
+``torch.randn`` on a CPU generator seeded with ``--seed``).  Weights are random-init: no trained checkpoint is
+involved anywhere.
+
+Value distributions (fixed for every workload):
+  * Linear weights N(0, 0.02) in fp32 (quantized later for W8A8 Linears, cast
+    to bf16 for BF16 Linears), biases N(0, 0.02) as bf16,
+  * Q/K RMSNorm weights 1 + N(0, 0.1) as bf16,
+  * latents N(0, 1) fp32, text features N(0, 1) bf16,
+  * block-level modulation tables N(0, 0.5) bf16 (block tests only; the full
+    step derives them from the timestep embedding).
+"""
+from __future__ import annotations
+
+import dataclasses
+import zlib
+from typing import Optional, Sequence, Tuple
+
+import torch
+
+__all__ = [
+    "Group", "DitConfig", "TINY", "BLOCK512", "STEP1024", "EDIT1024", "GEN2048",
+    "CONFIGS", "gen", "linear_weight", "bias", "norm_weight", "latents",
+    "text_features", "ref_latents", "hidden_states", "mod_table", "block_weights", "model_weights",
+]
+
+
+@dataclasses.dataclass(frozen=True)
+class Group:
+    """One contiguous token group of the joint sequence."""
+    kind: str                                  # "text" or "image"
+    tokens: int
+    grid: Optional[Tuple[int, int]] = None     # (h, w) for image groups
+
+
+@dataclasses.dataclass(frozen=True)
+class DitConfig:
+    name: str
+    hidden: int
+    heads: int
+    head_dim: int
+    mlp: int
+    blocks: int
+    patch: int
+    groups: Tuple[Group, ...]                  # last group = target latent tokens
+    eps: float = 1e-6
+    weight_seed: int = 0
+    input_seed: int = 1
+    latent_seed: int = 1
+    steps: int = 1
+    t: Optional[float] = None                  # fixed timestep for block-only workloads
+
+    @property
+    def tokens(self) -> int:
+        return sum(g.tokens for g in self.groups)
+
+    @property
+    def prefix_tokens(self) -> int:
+        return sum(g.tokens for g in self.groups[:-1])
+
+    @property
+    def target_tokens(self) -> int:
+        return self.groups[-1].tokens
+
+    @property
+    def text_tokens(self) -> int:
+        return sum(g.tokens for g in self.groups if g.kind == "text")
+
+    def group_sizes(self) -> Tuple[int, ...]:
+        return tuple(g.tokens for g in self.groups)
+
+    def group_row_sets(self) -> Tuple[int, ...]:
+        """Modulation row set per group: 0 for conditioning prefix groups, 1 for the target."""
+        return tuple(0 if i < len(self.groups) - 1 else 1 for i in range(len(self.groups)))
+
+    def replace(self, **kw) -> "DitConfig":
+        return dataclasses.replace(self, **kw)
+
+
+_TEXT = "text"
+_IMAGE = "image"
+
+# 16 text + 64 image tokens (8x8 grid of 2x2-patched 64-channel latents), one block.
+TINY = DitConfig("tiny_h256_1block", 256, 2, 128, 1024, 1, 256,
+                 (Group(_TEXT, 16), Group(_IMAGE, 64, (8, 8))),
+                 weight_seed=0, input_seed=0, latent_seed=0, t=0.5)
+# One full-width block at 512x512: 256 text + 1024 image tokens.
+BLOCK512 = DitConfig("block_512px", 4096, 32, 128, 16384, 1, 64,
+                     (Group(_TEXT, 256), Group(_IMAGE, 1024, (32, 32))), t=0.5)
+# Full 32-block step at 1024x1024: 512 text + 4096 image tokens.
+STEP1024 = DitConfig("step_1024px", 4096, 32, 128, 16384, 32, 64,
+                     (Group(_TEXT, 512), Group(_IMAGE, 4096, (64, 64))))
+# Edit step: 256 text + 1024 reference + 4096 target tokens.
+EDIT1024 = DitConfig("edit_1024px", 4096, 32, 128, 16384, 32, 64,
+                     (Group(_TEXT, 256), Group(_IMAGE, 1024, (32, 32)),
+                      Group(_IMAGE, 4096, (64, 64))))
+# 40-step denoise at 2048x2048: 512 text + 16384 image tokens.
+GEN2048 = DitConfig("denoise40_2048px", 4096, 32, 128, 16384, 32, 64,
+                    (Group(_TEXT, 512), Group(_IMAGE, 16384, (128, 128))),
+                    steps=40, latent_seed=42)
+
+CONFIGS = {c.name: c for c in (TINY, BLOCK512, STEP1024, EDIT1024, GEN2048)}
+
+
+def gen(seed: int, *tags) -> torch.Generator:
+    """A CPU generator whose seed is a stable function of ``seed`` and ``tags``."""
+    key = repr((seed,) + tuple(tags)).encode()
+    return torch.Generator().manual_seed((seed * 0x9E3779B1 + zlib.crc32(key)) % (2 ** 63))
+
+
+def _normal(shape, std, g, device="cpu") -> torch.Tensor:
+    t = torch.randn(*shape, generator=g, dtype=torch.float32)
+    t.mul_(std)
+    return t.to(device)
+
+
+def linear_weight(seed, tag, n, k, device="cpu") -> torch.Tensor:
+    """fp32 [n, k] ~ N(0, 0.02)."""
+    return _normal((n, k), 0.02, gen(seed, "w", tag), device)
+
+
+def bias(seed, tag, n, device="cpu") -> torch.Tensor:
+    """bf16 [n] ~ N(0, 0.02)."""
+    return _normal((n,), 0.02, gen(seed, "b", tag), device).to(torch.bfloat16)
+
+
+def norm_weight(seed, tag, d, device="cpu") -> torch.Tensor:
+    """bf16 [d] ~ 1 + N(0, 0.1)."""
+    return (1.0 + _normal((d,), 0.1, gen(seed, "n", tag), device)).to(torch.bfloat16)
+
+
+def latents(cfg: DitConfig, device="cpu") -> torch.Tensor:
+    """fp32 [target_tokens, patch] ~ N(0, 1)."""
+    return _normal((cfg.target_tokens, cfg.patch), 1.0, gen(cfg.latent_seed, "latents"), device)
+
+
+def ref_latents(cfg: DitConfig, device="cpu"):
+    """fp32 [reference_tokens, patch] ~ N(0, 1) for edit sequences, else None."""
+    ref = [g for g in cfg.groups[:-1] if g.kind == "image"]
+    if not ref:
+        return None
+    n = sum(g.tokens for g in ref)
+    return _normal((n, cfg.patch), 1.0, gen(cfg.latent_seed, "ref_latents"), device)
+
+
+def text_features(cfg: DitConfig, device="cpu") -> torch.Tensor:
+    """bf16 [text_tokens, hidden] ~ N(0, 1): the encoder's last hidden state stand-in."""
+    return _normal((cfg.text_tokens, cfg.hidden), 1.0,
+                   gen(cfg.input_seed, "txt"), device).to(torch.bfloat16)
+
+
+def hidden_states(cfg: DitConfig, tokens: int, device="cpu", tag="x") -> torch.Tensor:
+    """fp32 [tokens, hidden] ~ N(0, 1): a block-level residual-stream input."""
+    return _normal((tokens, cfg.hidden), 1.0, gen(cfg.input_seed, tag), device)
+
+
+def mod_table(cfg: DitConfig, rows: int = 2, device="cpu", tag="mod") -> torch.Tensor:
+    """bf16 [rows, 6, hidden] ~ N(0, 0.5): block-level modulation rows."""
+    return _normal((rows, 6, cfg.hidden), 0.5, gen(cfg.input_seed, tag), device).to(torch.bfloat16)
+
+
+def block_weights(cfg: DitConfig, layer: int, device="cpu") -> dict:
+    """Random-init weights of one block.
+
+    W8A8 Linears come as fp32 (``qkv`` [3H, H], ``out`` [H, H], ``up`` [F, H],
+    ``down`` [H, F]); each side quantizes them itself.  ``mod`` is the block's
+    adaLN Linear [6H, H] as bf16.
+    """
+    s, H, F, d = cfg.weight_seed, cfg.hidden, cfg.mlp, cfg.head_dim
+    L = ("blk", layer)
+    return {
+        "qkv": linear_weight(s, L + ("qkv",), 3 * H, H, device),
+        "qkv_b": bias(s, L + ("qkv",), 3 * H, device),
+        "out": linear_weight(s, L + ("out",), H, H, device),
+        "out_b": bias(s, L + ("out",), H, device),
+        "up": linear_weight(s, L + ("up",), F, H, device),
+        "up_b": bias(s, L + ("up",), F, device),
+        "down": linear_weight(s, L + ("down",), H, F, device),
+        "down_b": bias(s, L + ("down",), H, device),
+        "norm_q": norm_weight(s, L + ("nq",), d, device),
+        "norm_k": norm_weight(s, L + ("nk",), d, device),
+        "mod": linear_weight(s, L + ("mod",), 6 * H, H, device).to(torch.bfloat16),
+        "mod_b": bias(s, L + ("mod",), 6 * H, device),
+    }
+
+
+def model_weights(cfg: DitConfig, device="cpu") -> dict:
+    """Random-init weights of the step-level BF16 Linears (no blocks)."""
+    s, H, P = cfg.weight_seed, cfg.hidden, cfg.patch
+
+    def lin(tag, n, k):
+        return linear_weight(s, ("g", tag), n, k, device).to(torch.bfloat16)
+
+    return {
+        "t1": lin("t1", H, 256), "t1_b": bias(s, ("g", "t1"), H, device),
+        "t2": lin("t2", H, H), "t2_b": bias(s, ("g", "t2"), H, device),
+        "img_in": lin("img_in", H, P), "img_in_b": bias(s, ("g", "img_in"), H, device),
+        "txt_in": lin("txt_in", H, H), "txt_in_b": bias(s, ("g", "txt_in"), H, device),
+        "final_mod": lin("final_mod", 2 * H, H),
+        "final_mod_b": bias(s, ("g", "final_mod"), 2 * H, device),
+        "proj_out": lin("proj_out", P, H), "proj_out_b": bias(s, ("g", "proj_out"), P, device),
+    }
+
+
+def group_layout(sizes: Sequence[int]):
+    """Cumulative group ends for a list of group sizes (pure bookkeeping)."""
+    ends, acc = [], 0
+    for n in sizes:
+        acc += int(n)
+        ends.append(acc)
+    return ends
