@@ -1,0 +1,878 @@
+// C ABI of libqi (declared in include/qi.h): host-side validation, workspace
+// carving and the orchestration of the block and of the denoising step.
+// Every argument check runs before the first launch of a call.
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <string>
+
+#include "qi.h"
+#include "qi_common.cuh"
+#include "qi_internal.h"
+
+struct qi_ctx {
+  int device;
+  int num_sms;
+  int* status;   // device status word
+};
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int cuda_fail(const char* what) {
+  const cudaError_t e = cudaGetLastError();
+  return fail(QI_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+cudaStream_t S(void* s) { return static_cast<cudaStream_t>(s); }
+
+// Validate a group table against a sequence length; fill the device-side copy.
+int check_groups(const qi_groups* g, int total, qi::GroupTable* out) {
+  if (!g) return fail(QI_ERR_INVALID_ARG, "groups is NULL");
+  if (g->n < 1 || g->n > QI_MAX_GROUPS)
+    return fail(QI_ERR_INVALID_ARG, "groups->n = %d outside 1..%d", g->n, QI_MAX_GROUPS);
+  int prev = 0;
+  for (int i = 0; i < g->n; ++i) {
+    if (g->end[i] <= prev)
+      return fail(QI_ERR_INVALID_ARG, "group ends must be strictly ascending and positive");
+    if (g->row_set[i] < 0) return fail(QI_ERR_INVALID_ARG, "negative row set");
+    prev = g->end[i];
+  }
+  if (total >= 0 && prev != total)
+    return fail(QI_ERR_INVALID_ARG, "groups->end[n-1] = %d but the sequence has %d tokens", prev,
+                total);
+  if (out) {
+    memset(out, 0, sizeof(*out));
+    out->n = g->n;
+    for (int i = 0; i < g->n; ++i) {
+      out->end[i] = g->end[i];
+      out->row_set[i] = g->row_set[i];
+    }
+  }
+  return QI_OK;
+}
+
+int check_dims(const qi_dims* d) {
+  if (!d) return fail(QI_ERR_INVALID_ARG, "dims is NULL");
+  if (d->head_dim != 128) return fail(QI_ERR_UNSUPPORTED_SHAPE, "head_dim must be 128");
+  if (d->heads < 1 || d->hidden != d->heads * d->head_dim)
+    return fail(QI_ERR_INVALID_ARG, "hidden must equal heads * head_dim");
+  if (d->hidden % 256 != 0 || d->hidden > 16384)
+    return fail(QI_ERR_UNSUPPORTED_SHAPE, "hidden must be a multiple of 256, at most 16384");
+  if (d->mlp % 128 != 0 || d->mlp < 128 || d->mlp > 16384)
+    return fail(QI_ERR_UNSUPPORTED_SHAPE, "mlp must be a multiple of 128 in 128..16384");
+  if (d->patch % 64 != 0 || d->patch < 64)
+    return fail(QI_ERR_UNSUPPORTED_SHAPE, "patch must be a positive multiple of 64");
+  if (d->blocks < 1 || d->blocks > 64)
+    return fail(QI_ERR_UNSUPPORTED_SHAPE, "blocks must be in 1..64");
+  if (!(d->eps >= 0.f)) return fail(QI_ERR_INVALID_ARG, "eps must be >= 0");
+  return QI_OK;
+}
+
+int check_w8(const qi_w8* w, const char* name, int n, int k) {
+  if (!w || !w->q || !w->s || !w->rowsum)
+    return fail(QI_ERR_INVALID_ARG, "W8A8 weight %s has a NULL pointer", name);
+  if ((n >= 0 && w->n != n) || (k >= 0 && w->k != k))
+    return fail(QI_ERR_UNSUPPORTED_SHAPE, "W8A8 weight %s is [%d, %d], expected [%d, %d]", name,
+                w->n, w->k, n, k);
+  if (w->k % 128 != 0 || w->k < 128)
+    return fail(QI_ERR_UNSUPPORTED_SHAPE, "W8A8 weight %s: k = %d is not a multiple of 128", name,
+                w->k);
+  if (w->n % 16 != 0 || w->n < 16)
+    return fail(QI_ERR_UNSUPPORTED_SHAPE, "W8A8 weight %s: n = %d is not a multiple of 16", name,
+                w->n);
+  if (!aligned16(w->q) || !aligned16(w->s) || !aligned16(w->rowsum) ||
+      (w->bias && !aligned16(w->bias)))
+    return fail(QI_ERR_ALIGNMENT, "W8A8 weight %s: pointers must be 16-byte aligned", name);
+  return QI_OK;
+}
+
+int check_bf16_linear(const qi_linear_bf16* w, const char* name, int n, int k) {
+  if (!w || !w->w) return fail(QI_ERR_INVALID_ARG, "BF16 weight %s is NULL", name);
+  if ((n >= 0 && w->n != n) || (k >= 0 && w->k != k))
+    return fail(QI_ERR_UNSUPPORTED_SHAPE, "BF16 weight %s is [%d, %d], expected [%d, %d]", name,
+                w->n, w->k, n, k);
+  if (!aligned16(w->w) || (w->bias && !aligned16(w->bias)))
+    return fail(QI_ERR_ALIGNMENT, "BF16 weight %s: pointers must be 16-byte aligned", name);
+  return QI_OK;
+}
+
+// Bump allocator over the caller's workspace (256-byte aligned pieces).
+struct Carve {
+  uint8_t* base;
+  size_t cap, off;
+  template <class T>
+  T* take(size_t count) {
+    off = (off + 255) & ~static_cast<size_t>(255);
+    T* p = reinterpret_cast<T*>(base ? base + off : nullptr);
+    off += count * sizeof(T);
+    return p;
+  }
+};
+
+struct BlockBufs {
+  int8_t* uq;       // [T, max(H, F)]
+  float* sa;        // [T]
+  int32_t* zp;      // [T]
+  uint16_t* qkv;    // [T, 3H]
+  uint16_t* q;      // [T, H]
+  uint16_t* o;      // [T, H]
+  uint16_t* g;      // [T, F]
+};
+
+BlockBufs carve_block(Carve& c, const qi_dims& d, int T) {
+  BlockBufs b;
+  const size_t H = d.hidden, F = d.mlp, W = H > F ? H : F;
+  b.uq = c.take<int8_t>(static_cast<size_t>(T) * W);
+  b.sa = c.take<float>(T);
+  b.zp = c.take<int32_t>(T);
+  b.qkv = c.take<uint16_t>(static_cast<size_t>(T) * 3 * H);
+  b.q = c.take<uint16_t>(static_cast<size_t>(T) * H);
+  b.o = c.take<uint16_t>(static_cast<size_t>(T) * H);
+  b.g = c.take<uint16_t>(static_cast<size_t>(T) * F);
+  return b;
+}
+
+size_t block_bytes(const qi_dims& d, int T) {
+  Carve c{nullptr, 0, 0};
+  carve_block(c, d, T);
+  return c.off + 256;
+}
+
+struct StepBufs {
+  float* x;             // [S, H] fp32 residual stream
+  float* emb;           // [2, 256]
+  float* h1;            // [2, H]
+  float* temb;          // [2, H]
+  uint16_t* block_mod;  // [blocks][2][6H]
+  uint16_t* final_mod;  // [2][2H]
+  uint16_t* lat_bf16;   // [S, P] bf16 copies of the latents fed to img_in
+  uint16_t* u_final;    // [S, H]
+  uint16_t* kv;         // [blocks][2][S][H] when the caller passes no cache
+  uint8_t* block_ws;
+  size_t block_ws_bytes;
+};
+
+StepBufs carve_step(Carve& c, const qi_dims& d, int Sq, int S, bool own_kv) {
+  StepBufs b;
+  const size_t H = d.hidden, P = d.patch;
+  b.x = c.take<float>(static_cast<size_t>(Sq) * H);
+  b.emb = c.take<float>(2 * 256);
+  b.h1 = c.take<float>(2 * H);
+  b.temb = c.take<float>(2 * H);
+  b.block_mod = c.take<uint16_t>(static_cast<size_t>(d.blocks) * 2 * 6 * H);
+  b.final_mod = c.take<uint16_t>(2 * 2 * H);
+  b.lat_bf16 = c.take<uint16_t>(static_cast<size_t>(S) * P);
+  b.u_final = c.take<uint16_t>(static_cast<size_t>(S) * H);
+  b.kv = own_kv ? c.take<uint16_t>(static_cast<size_t>(d.blocks) * 2 * S * H) : nullptr;
+  b.block_ws_bytes = block_bytes(d, Sq);
+  b.block_ws = c.take<uint8_t>(b.block_ws_bytes);
+  return b;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------- TMA encode
+
+namespace qi {
+
+bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, uint64_t inner,
+                  uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner,
+                  uint32_t box_outer) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  if (!encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+      return false;
+    encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_stride_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = encode(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace qi
+
+// ---------------------------------------------------------------- internal ops
+
+namespace {
+
+int run_quant(qi_ctx* ctx, const void* x, bool xbf16, int M, int K, int ldx,
+              const uint16_t* shift, const uint16_t* scale, int mod_ld, const qi::GroupTable& gt,
+              int row0, float eps, int8_t* q, float* s, int32_t* zp, uint16_t* u_bf16,
+              cudaStream_t st) {
+  (void)ctx;
+  qi::QuantParams p;
+  p.x = x;
+  p.x_bf16 = xbf16 ? 1 : 0;
+  p.M = M;
+  p.K = K;
+  p.ldx = ldx;
+  p.ln = shift ? 1 : 0;
+  p.shift = shift;
+  p.scale = scale;
+  p.mod_ld = mod_ld;
+  p.groups = gt;
+  p.row0 = row0;
+  p.eps = eps;
+  p.q = q;
+  p.ldq = K;
+  p.s = s;
+  p.zp = zp;
+  p.u_bf16 = u_bf16;
+  if (qi::launch_quant(p, st) != 0) return cuda_fail("quantize launch");
+  return QI_OK;
+}
+
+int run_w8a8(qi_ctx* ctx, const int8_t* qa, const float* sa, const int32_t* zp, int M,
+             const qi_w8& w, int epi, uint16_t* y, int ldy, float* res, int ldr,
+             const uint16_t* gate, int gate_ld, const qi::GroupTable& gt, int row0,
+             int32_t* acc_debug, cudaStream_t st) {
+  if (M == 0) return QI_OK;
+  qi::GemmParams p;
+  memset(&p, 0, sizeof(p));
+  p.M = M;
+  p.N = w.n;
+  p.K = w.k;
+  p.num_kb = w.k / 128;
+  p.s_a = sa;
+  p.zp_a = zp;
+  p.s_w = w.s;
+  p.rowsum = w.rowsum;
+  p.bias = w.bias;
+  p.y = y;
+  p.ldy = ldy;
+  p.yf = res;
+  p.ldyf = ldr;
+  p.gate = gate;
+  p.gate_ld = gate_ld;
+  p.groups = gt;
+  p.row0 = row0;
+  p.acc_debug = acc_debug;
+  p.status = ctx->status;
+  const int r = qi::launch_gemm(true, epi, qa, w.k, w.q, w.k, p, ctx->num_sms, st);
+  if (r == -2) return fail(QI_ERR_CUDA, "cuTensorMapEncodeTiled failed (W8A8 operands)");
+  if (r != 0) return cuda_fail("W8A8 GEMM launch");
+  return QI_OK;
+}
+
+int run_bf16_linear(qi_ctx* ctx, const uint16_t* a, int M, int lda, const qi_linear_bf16& w,
+                    int epi, float* yf, int ldyf, float dt, float* v_out, cudaStream_t st) {
+  if (M == 0) return QI_OK;
+  qi::GemmParams p;
+  memset(&p, 0, sizeof(p));
+  p.M = M;
+  p.N = w.n;
+  p.K = w.k;
+  p.num_kb = w.k / 64;
+  p.bias = w.bias;
+  p.yf = yf;
+  p.ldyf = ldyf;
+  p.dt = dt;
+  p.v_out = v_out;
+  p.status = ctx->status;
+  const int r = qi::launch_gemm(false, epi, a, lda, w.w, w.k, p, ctx->num_sms, st);
+  if (r == -2) return fail(QI_ERR_CUDA, "cuTensorMapEncodeTiled failed (BF16 operands)");
+  if (r != 0) return cuda_fail("BF16 GEMM launch");
+  return QI_OK;
+}
+
+int run_block(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, float* x, int T, int row0,
+              const uint16_t* mod, const qi::GroupTable& gt, int S, const float* cs,
+              const float* sn, uint16_t* kl, uint16_t* vl, uint8_t* ws, size_t ws_bytes,
+              cudaStream_t st) {
+  const int H = d.hidden, F = d.mlp;
+  Carve c{ws, ws_bytes, 0};
+  BlockBufs b = carve_block(c, d, T);
+  const int mld = 6 * H;
+  int r;
+  // attention half
+  if ((r = run_quant(ctx, x, false, T, H, H, mod + 0 * H, mod + 1 * H, mld, gt, row0, d.eps,
+                     b.uq, b.sa, b.zp, nullptr, st)))
+    return r;
+  if ((r = run_w8a8(ctx, b.uq, b.sa, b.zp, T, w.qkv, qi::EPI_BF16, b.qkv, 3 * H, nullptr, 0,
+                    nullptr, 0, gt, row0, nullptr, st)))
+    return r;
+  qi::QkNormRopeParams np;
+  np.qkv = b.qkv;
+  np.ldqkv = 3 * H;
+  np.T = T;
+  np.heads = d.heads;
+  np.d = d.head_dim;
+  np.wq = w.norm_q;
+  np.wk = w.norm_k;
+  np.cos = cs;
+  np.sin = sn;
+  np.eps = d.eps;
+  np.q_out = b.q;
+  np.k_out = kl + static_cast<size_t>(row0) * H;
+  np.v_out = vl + static_cast<size_t>(row0) * H;
+  np.ldo = H;
+  if (qi::launch_qk_norm_rope(np, st) != 0) return cuda_fail("qk norm/rope launch");
+  qi::AttnParams ap;
+  ap.q = b.q;
+  ap.k = kl;
+  ap.v = vl;
+  ap.o = b.o;
+  ap.ldq = H;
+  ap.ldkv = H;
+  ap.ldo = H;
+  ap.Sq = T;
+  ap.Sk = S;
+  ap.heads = d.heads;
+  ap.q_offset = row0;
+  ap.sm_scale = 1.0f / sqrtf(static_cast<float>(d.head_dim));
+  ap.groups = gt;
+  if (qi::launch_attention(ap, st) != 0) return cuda_fail("attention launch");
+  if ((r = run_quant(ctx, b.o, true, T, H, H, nullptr, nullptr, 0, gt, row0, d.eps, b.uq, b.sa,
+                     b.zp, nullptr, st)))
+    return r;
+  if ((r = run_w8a8(ctx, b.uq, b.sa, b.zp, T, w.out, qi::EPI_GATED, nullptr, 0, x, H,
+                    mod + 2 * H, mld, gt, row0, nullptr, st)))
+    return r;
+  // MLP half
+  if ((r = run_quant(ctx, x, false, T, H, H, mod + 3 * H, mod + 4 * H, mld, gt, row0, d.eps,
+                     b.uq, b.sa, b.zp, nullptr, st)))
+    return r;
+  if ((r = run_w8a8(ctx, b.uq, b.sa, b.zp, T, w.up, qi::EPI_GELU, b.g, F, nullptr, 0, nullptr, 0,
+                    gt, row0, nullptr, st)))
+    return r;
+  if ((r = run_quant(ctx, b.g, true, T, F, F, nullptr, nullptr, 0, gt, row0, d.eps, b.uq, b.sa,
+                     b.zp, nullptr, st)))
+    return r;
+  if ((r = run_w8a8(ctx, b.uq, b.sa, b.zp, T, w.down, qi::EPI_GATED, nullptr, 0, x, H,
+                    mod + 5 * H, mld, gt, row0, nullptr, st)))
+    return r;
+  return QI_OK;
+}
+
+int check_block_weights(const qi_dims& d, const qi_block_weights* w) {
+  if (!w) return fail(QI_ERR_INVALID_ARG, "block weights are NULL");
+  const int H = d.hidden, F = d.mlp;
+  int r;
+  if ((r = check_w8(&w->qkv, "qkv", 3 * H, H))) return r;
+  if ((r = check_w8(&w->out, "out", H, H))) return r;
+  if ((r = check_w8(&w->up, "up", F, H))) return r;
+  if ((r = check_w8(&w->down, "down", H, F))) return r;
+  if (!w->norm_q || !w->norm_k) return fail(QI_ERR_INVALID_ARG, "norm_q / norm_k is NULL");
+  if (!aligned16(w->norm_q) || !aligned16(w->norm_k))
+    return fail(QI_ERR_ALIGNMENT, "norm_q / norm_k must be 16-byte aligned");
+  return QI_OK;
+}
+
+int run_time_conditioning(qi_ctx* ctx, const qi_model& m, float sigma, uint16_t* block_mod,
+                          uint16_t* final_mod, StepBufs& b, cudaStream_t st) {
+  const qi_dims& d = m.dims;
+  const int H = d.hidden;
+  // t = 0 for the conditioning prefix, t = sigma for the target.
+  if (qi::launch_timestep_embedding(0.0f, sigma, b.emb, st) != 0)
+    return cuda_fail("timestep embedding launch");
+  qi::GemvParams g;
+  memset(&g, 0, sizeof(g));
+  g.x = b.emb;
+  g.R = 2;
+  g.k = 256;
+  g.silu_in = 0;
+  g.y_bf16 = 0;
+  g.n_jobs = 1;
+  g.jobs[0] = {m.t1.w, m.t1.bias, b.h1, H, H};
+  if (qi::launch_gemv(g, st) != 0) return cuda_fail("timestep MLP 1 launch");
+  g.x = b.h1;
+  g.k = H;
+  g.silu_in = 1;
+  g.jobs[0] = {m.t2.w, m.t2.bias, b.temb, H, H};
+  if (qi::launch_gemv(g, st) != 0) return cuda_fail("timestep MLP 2 launch");
+  g.x = b.temb;
+  g.silu_in = 1;
+  g.y_bf16 = 1;
+  g.n_jobs = 0;
+  for (int l = 0; l < d.blocks; ++l)
+    g.jobs[g.n_jobs++] = {m.blocks[l].mod.w, m.blocks[l].mod.bias,
+                          block_mod + static_cast<size_t>(l) * 2 * 6 * H, 6 * H, 6 * H};
+  g.jobs[g.n_jobs++] = {m.final_mod.w, m.final_mod.bias, final_mod, 2 * H, 2 * H};
+  if (qi::launch_gemv(g, st) != 0) return cuda_fail("adaLN rows launch");
+  return QI_OK;
+}
+
+int check_model(const qi_model* m) {
+  if (!m) return fail(QI_ERR_INVALID_ARG, "model is NULL");
+  int r;
+  if ((r = check_dims(&m->dims))) return r;
+  const qi_dims& d = m->dims;
+  const int H = d.hidden, P = d.patch;
+  if (!m->blocks) return fail(QI_ERR_INVALID_ARG, "model->blocks is NULL");
+  for (int l = 0; l < d.blocks; ++l) {
+    if ((r = check_block_weights(d, &m->blocks[l]))) return r;
+    if ((r = check_bf16_linear(&m->blocks[l].mod, "block mod", 6 * H, H))) return r;
+  }
+  if ((r = check_bf16_linear(&m->t1, "t1", H, 256))) return r;
+  if ((r = check_bf16_linear(&m->t2, "t2", H, H))) return r;
+  if ((r = check_bf16_linear(&m->img_in, "img_in", H, P))) return r;
+  if ((r = check_bf16_linear(&m->txt_in, "txt_in", H, H))) return r;
+  if ((r = check_bf16_linear(&m->final_mod, "final_mod", 2 * H, H))) return r;
+  if ((r = check_bf16_linear(&m->proj_out, "proj_out", P, H))) return r;
+  return QI_OK;
+}
+
+}  // namespace
+
+// ================================================================= C ABI
+
+extern "C" {
+
+int qi_ctx_create(int device, qi_ctx** out) {
+  if (!out) return fail(QI_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (cudaSetDevice(device) != cudaSuccess) return cuda_fail("cudaSetDevice");
+  int major = 0, minor = 0, sms = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, device);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device);
+  if (major != 10 || minor != 0)
+    return fail(QI_ERR_UNSUPPORTED_SHAPE, "device %d is sm_%d%d; libqi is built for sm_100a",
+                device, major, minor);
+  qi_ctx* c = new qi_ctx;
+  c->device = device;
+  c->num_sms = sms;
+  c->status = nullptr;
+  if (cudaMalloc(&c->status, 256) != cudaSuccess) {
+    delete c;
+    return cuda_fail("cudaMalloc(status)");
+  }
+  if (cudaMemset(c->status, 0, 256) != cudaSuccess) {
+    cudaFree(c->status);
+    delete c;
+    return cuda_fail("cudaMemset(status)");
+  }
+  *out = c;
+  return QI_OK;
+}
+
+int qi_ctx_destroy(qi_ctx* ctx) {
+  if (!ctx) return QI_OK;
+  cudaFree(ctx->status);
+  delete ctx;
+  return QI_OK;
+}
+
+int qi_ctx_check(qi_ctx* ctx, void* stream) {
+  if (!ctx) return fail(QI_ERR_INVALID_ARG, "ctx is NULL");
+  if (cudaStreamSynchronize(S(stream)) != cudaSuccess) return cuda_fail("stream synchronize");
+  int st = 0;
+  if (cudaMemcpy(&st, ctx->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return cuda_fail("status read");
+  if (st != 0) {
+    cudaMemset(ctx->status, 0, sizeof(int));
+    return fail(QI_ERR_TIMEOUT, "a kernel recorded device status %d (bounded wait expired)", st);
+  }
+  return QI_OK;
+}
+
+int qi_last_error(char* buf, size_t n) {
+  if (!buf || n == 0) return QI_ERR_INVALID_ARG;
+  snprintf(buf, n, "%s", g_last_error.c_str());
+  return QI_OK;
+}
+
+int qi_prepare_w8(qi_ctx* ctx, const float* w, int n, int k, int8_t* q, float* s,
+                  int32_t* rowsum, void* stream) {
+  if (!ctx || !w || !q || !s || !rowsum) return fail(QI_ERR_INVALID_ARG, "NULL argument");
+  if (n < 0 || k < 8 || k % 8 != 0) return fail(QI_ERR_UNSUPPORTED_SHAPE, "need k % 8 == 0");
+  if (qi::launch_prepare_w8(w, n, k, q, s, rowsum, S(stream)) != 0)
+    return cuda_fail("prepare_w8 launch");
+  return QI_OK;
+}
+
+int qi_quantize_act(qi_ctx* ctx, const void* x, int x_dtype, int M, int K, int ldx,
+                    const uint16_t* shift, const uint16_t* scale, int mod_ld,
+                    const qi_groups* groups, int row0, float eps, int8_t* q, float* s_a,
+                    int32_t* zp_a, void* stream) {
+  if (!ctx || !x || !q || !s_a || !zp_a) return fail(QI_ERR_INVALID_ARG, "NULL argument");
+  if (x_dtype != QI_F32 && x_dtype != QI_BF16) return fail(QI_ERR_INVALID_ARG, "bad x_dtype");
+  if (M < 0 || K < 8 || K % 8 != 0 || K > 16384 || ldx < K || ldx % 8 != 0)
+    return fail(QI_ERR_UNSUPPORTED_SHAPE, "quantize: need 8 <= K <= 16384, K %% 8 == 0, ldx %% 8 == 0");
+  if (!aligned16(x) || !aligned16(q)) return fail(QI_ERR_ALIGNMENT, "x / q must be 16-byte aligned");
+  qi::GroupTable gt;
+  memset(&gt, 0, sizeof(gt));
+  gt.n = 1;
+  gt.end[0] = 1 << 30;
+  if (shift || scale) {
+    if (!shift || !scale) return fail(QI_ERR_INVALID_ARG, "shift and scale go together");
+    if (!aligned16(shift) || !aligned16(scale) || mod_ld % 8 != 0)
+      return fail(QI_ERR_ALIGNMENT, "shift / scale rows must be 16-byte aligned");
+    int r;
+    if ((r = check_groups(groups, -1, &gt))) return r;
+    if (row0 < 0 || row0 + M > gt.end[gt.n - 1])
+      return fail(QI_ERR_INVALID_ARG, "rows row0..row0+M-1 fall outside the groups");
+  }
+  return run_quant(ctx, x, x_dtype == QI_BF16, M, K, ldx, shift, scale, mod_ld, gt, row0, eps, q,
+                   s_a, zp_a, nullptr, S(stream));
+}
+
+int qi_w8a8_linear(qi_ctx* ctx, const int8_t* qa, const float* s_a, const int32_t* zp_a, int M,
+                   const qi_w8* w, const qi_epilogue* ep, uint16_t* y, int ldy,
+                   int32_t* acc_debug, void* stream) {
+  if (!ctx || !qa || !s_a || !zp_a) return fail(QI_ERR_INVALID_ARG, "NULL argument");
+  if (M < 0) return fail(QI_ERR_INVALID_ARG, "M < 0");
+  int r;
+  if ((r = check_w8(w, "w", -1, -1))) return r;
+  if (!aligned16(qa)) return fail(QI_ERR_ALIGNMENT, "qa must be 16-byte aligned");
+  const int kind = ep ? ep->kind : QI_EPI_STORE;
+  qi::GroupTable gt;
+  memset(&gt, 0, sizeof(gt));
+  gt.n = 1;
+  gt.end[0] = 1 << 30;
+  if (kind == QI_EPI_STORE || kind == QI_EPI_GELU_TANH) {
+    if (!y) return fail(QI_ERR_INVALID_ARG, "y is NULL");
+    if (!aligned16(y) || ldy < w->n || ldy % 8 != 0)
+      return fail(QI_ERR_ALIGNMENT, "y must be 16-byte aligned with ldy %% 8 == 0, ldy >= n");
+    return run_w8a8(ctx, qa, s_a, zp_a, M, *w, kind == QI_EPI_STORE ? qi::EPI_BF16 : qi::EPI_GELU,
+                    y, ldy, nullptr, 0, nullptr, 0, gt, 0, acc_debug, S(stream));
+  }
+  if (kind != QI_EPI_GATED_RESIDUAL) return fail(QI_ERR_INVALID_ARG, "bad epilogue kind");
+  if (!ep->residual || !ep->gate) return fail(QI_ERR_INVALID_ARG, "residual / gate is NULL");
+  if (ep->ld_residual < w->n) return fail(QI_ERR_INVALID_ARG, "ld_residual < n");
+  if ((r = check_groups(ep->groups, -1, &gt))) return r;
+  if (ep->row0 < 0 || ep->row0 + M > gt.end[gt.n - 1])
+    return fail(QI_ERR_INVALID_ARG, "rows row0..row0+M-1 fall outside the groups");
+  return run_w8a8(ctx, qa, s_a, zp_a, M, *w, qi::EPI_GATED, nullptr, 0, ep->residual,
+                  ep->ld_residual, ep->gate, ep->gate_ld, gt, ep->row0, acc_debug, S(stream));
+}
+
+int qi_bf16_linear(qi_ctx* ctx, const uint16_t* a, int M, int lda, const qi_linear_bf16* w,
+                   float* y, int ldy, void* stream) {
+  if (!ctx || !a || !y) return fail(QI_ERR_INVALID_ARG, "NULL argument");
+  int r;
+  if ((r = check_bf16_linear(w, "w", -1, -1))) return r;
+  if (M < 0 || w->k % 64 != 0 || w->k < 64 || w->n % 16 != 0 || lda < w->k || lda % 8 != 0 ||
+      ldy < w->n)
+    return fail(QI_ERR_UNSUPPORTED_SHAPE, "bf16 linear: need k %% 64 == 0, n %% 16 == 0, lda %% 8 == 0");
+  if (!aligned16(a)) return fail(QI_ERR_ALIGNMENT, "a must be 16-byte aligned");
+  return run_bf16_linear(ctx, a, M, lda, *w, qi::EPI_F32, y, ldy, 0.f, nullptr, S(stream));
+}
+
+int qi_qk_norm_rope(qi_ctx* ctx, const uint16_t* qkv, int T, int heads, int head_dim,
+                    const uint16_t* wq, const uint16_t* wk, const float* rope_cos,
+                    const float* rope_sin, float eps, uint16_t* q_out, uint16_t* k_out,
+                    uint16_t* v_out, int ldo, void* stream) {
+  if (!ctx || !qkv || !wq || !wk || !rope_cos || !rope_sin || !q_out || !k_out || !v_out)
+    return fail(QI_ERR_INVALID_ARG, "NULL argument");
+  if (head_dim != 128) return fail(QI_ERR_UNSUPPORTED_SHAPE, "head_dim must be 128");
+  if (T < 0 || heads < 1 || ldo < heads * head_dim)
+    return fail(QI_ERR_INVALID_ARG, "bad T / heads / ldo");
+  qi::QkNormRopeParams p;
+  p.qkv = qkv;
+  p.ldqkv = 3 * heads * head_dim;
+  p.T = T;
+  p.heads = heads;
+  p.d = head_dim;
+  p.wq = wq;
+  p.wk = wk;
+  p.cos = rope_cos;
+  p.sin = rope_sin;
+  p.eps = eps;
+  p.q_out = q_out;
+  p.k_out = k_out;
+  p.v_out = v_out;
+  p.ldo = ldo;
+  if (qi::launch_qk_norm_rope(p, S(stream)) != 0) return cuda_fail("qk norm/rope launch");
+  return QI_OK;
+}
+
+int qi_attn_block_causal(qi_ctx* ctx, const uint16_t* q, int ldq, int Sq, int q_offset,
+                         const uint16_t* k, const uint16_t* v, int ldkv, int Sk, int heads,
+                         int head_dim, const qi_groups* groups, float sm_scale, uint16_t* o,
+                         int ldo, void* stream) {
+  if (!ctx || !q || !k || !v || !o) return fail(QI_ERR_INVALID_ARG, "NULL argument");
+  if (head_dim != 128) return fail(QI_ERR_UNSUPPORTED_SHAPE, "head_dim must be 128");
+  if (Sq < 0 || Sk < 1 || q_offset < 0 || q_offset + Sq > Sk || heads < 1)
+    return fail(QI_ERR_INVALID_ARG, "need 0 <= q_offset, q_offset + Sq <= Sk");
+  const int W = heads * head_dim;
+  if (ldq < W || ldkv < W || ldo < W || ldq % 8 || ldkv % 8 || ldo % 8)
+    return fail(QI_ERR_ALIGNMENT, "leading dimensions must be >= heads*128 and multiples of 8");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return fail(QI_ERR_ALIGNMENT, "q/k/v/o must be 16-byte aligned");
+  qi::GroupTable gt;
+  int r;
+  if ((r = check_groups(groups, Sk, &gt))) return r;
+  qi::AttnParams p;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.o = o;
+  p.ldq = ldq;
+  p.ldkv = ldkv;
+  p.ldo = ldo;
+  p.Sq = Sq;
+  p.Sk = Sk;
+  p.heads = heads;
+  p.q_offset = q_offset;
+  p.sm_scale = sm_scale;
+  p.groups = gt;
+  if (qi::launch_attention(p, S(stream)) != 0) return cuda_fail("attention launch");
+  return QI_OK;
+}
+
+int qi_block_workspace_bytes(const qi_dims* dims, int T, size_t* bytes) {
+  int r;
+  if ((r = check_dims(dims))) return r;
+  if (!bytes || T < 0) return fail(QI_ERR_INVALID_ARG, "bad arguments");
+  *bytes = block_bytes(*dims, T);
+  return QI_OK;
+}
+
+int qi_dit_block_forward(qi_ctx* ctx, const qi_dims* dims, const qi_block_weights* w, float* x,
+                         int T, int row0, const uint16_t* mod, const qi_groups* groups,
+                         const float* rope_cos, const float* rope_sin, uint16_t* k_layer,
+                         uint16_t* v_layer, int kv_mode, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  int r;
+  if (!ctx || !x || !mod || !rope_cos || !rope_sin || !k_layer || !v_layer || !workspace)
+    return fail(QI_ERR_INVALID_ARG, "NULL argument");
+  if ((r = check_dims(dims))) return r;
+  if ((r = check_block_weights(*dims, w))) return r;
+  qi::GroupTable gt;
+  if ((r = check_groups(groups, -1, &gt))) return r;
+  const int S_total = gt.end[gt.n - 1];
+  if (T < 1 || row0 < 0 || row0 + T != S_total)
+    return fail(QI_ERR_INVALID_ARG, "rows row0..row0+T-1 must end the sequence (row0 + T == S)");
+  if (kv_mode == QI_KV_NONE || kv_mode == QI_KV_WRITE_PREFIX) {
+    if (row0 != 0) return fail(QI_ERR_INVALID_ARG, "this kv_mode processes every token (row0 == 0)");
+  } else if (kv_mode == QI_KV_READ_PREFIX) {
+    if (row0 == 0) return fail(QI_ERR_INVALID_ARG, "READ_PREFIX needs row0 > 0");
+  } else {
+    return fail(QI_ERR_INVALID_ARG, "bad kv_mode");
+  }
+  for (int g = 0; g < gt.n; ++g)
+    if (gt.row_set[g] > 1) return fail(QI_ERR_INVALID_ARG, "row sets must be 0 or 1");
+  if (!aligned16(x) || !aligned16(mod) || !aligned16(k_layer) || !aligned16(v_layer) ||
+      !aligned16(workspace) || !aligned16(rope_cos) || !aligned16(rope_sin))
+    return fail(QI_ERR_ALIGNMENT, "pointers must be 16-byte aligned");
+  if (workspace_bytes < block_bytes(*dims, T))
+    return fail(QI_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", workspace_bytes,
+                block_bytes(*dims, T));
+  return run_block(ctx, *dims, *w, x, T, row0, mod, gt, S_total, rope_cos, rope_sin, k_layer,
+                   v_layer, static_cast<uint8_t*>(workspace), workspace_bytes, S(stream));
+}
+
+int qi_step_workspace_bytes(const qi_dims* dims, int S_tokens, size_t* bytes) {
+  int r;
+  if ((r = check_dims(dims))) return r;
+  if (!bytes || S_tokens < 1) return fail(QI_ERR_INVALID_ARG, "bad arguments");
+  Carve c{nullptr, 0, 0};
+  carve_step(c, *dims, S_tokens, S_tokens, true);
+  *bytes = c.off + 256;
+  return QI_OK;
+}
+
+int qi_time_conditioning(qi_ctx* ctx, const qi_model* model, float sigma, uint16_t* block_mod,
+                         uint16_t* final_mod, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+  int r;
+  if (!ctx || !block_mod || !final_mod || !workspace) return fail(QI_ERR_INVALID_ARG, "NULL argument");
+  if ((r = check_model(model))) return r;
+  Carve c{static_cast<uint8_t*>(workspace), workspace_bytes, 0};
+  StepBufs b = carve_step(c, model->dims, 1, 1, false);
+  if (c.off > workspace_bytes) return fail(QI_ERR_WORKSPACE, "workspace too small");
+  return run_time_conditioning(ctx, *model, sigma, block_mod, final_mod, b, S(stream));
+}
+
+int qi_denoise_step(qi_ctx* ctx, const qi_model* model, float* latents, const uint16_t* txt,
+                    int text_tokens, const float* ref_latents, const qi_groups* groups,
+                    const float* rope_cos, const float* rope_sin, float sigma, float sigma_next,
+                    int kv_mode, uint16_t* kv_cache, float* v_out, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  int r;
+  if (!ctx || !latents || !rope_cos || !rope_sin || !workspace)
+    return fail(QI_ERR_INVALID_ARG, "NULL argument");
+  if ((r = check_model(model))) return r;
+  const qi_dims& d = model->dims;
+  qi::GroupTable gt;
+  if ((r = check_groups(groups, -1, &gt))) return r;
+  if (gt.n < 2) return fail(QI_ERR_INVALID_ARG, "a step needs a conditioning prefix and a target group");
+  for (int g = 0; g < gt.n; ++g)
+    if (gt.row_set[g] != (g == gt.n - 1 ? 1 : 0))
+      return fail(QI_ERR_INVALID_ARG, "row sets must be 0 for prefix groups and 1 for the target");
+  const int S_tok = gt.end[gt.n - 1];
+  const int P_tok = gt.end[gt.n - 2];
+  const int N = S_tok - P_tok;
+  const int R_ref = P_tok - text_tokens;
+  if (text_tokens < 1 || R_ref < 0) return fail(QI_ERR_INVALID_ARG, "text_tokens outside the prefix");
+  if (R_ref > 0 && !ref_latents && kv_mode != QI_KV_READ_PREFIX)
+    return fail(QI_ERR_INVALID_ARG, "the prefix holds reference tokens but ref_latents is NULL");
+  const int row0 = kv_mode == QI_KV_READ_PREFIX ? P_tok : 0;
+  if (kv_mode != QI_KV_NONE && kv_mode != QI_KV_WRITE_PREFIX && kv_mode != QI_KV_READ_PREFIX)
+    return fail(QI_ERR_INVALID_ARG, "bad kv_mode");
+  if (kv_mode != QI_KV_READ_PREFIX && !txt) return fail(QI_ERR_INVALID_ARG, "txt is NULL");
+  if (kv_mode != QI_KV_NONE && !kv_cache)
+    return fail(QI_ERR_INVALID_ARG, "kv_cache is required with prefix caching");
+  if (!aligned16(latents) || (txt && !aligned16(txt)) || (ref_latents && !aligned16(ref_latents)) ||
+      (kv_cache && !aligned16(kv_cache)) || !aligned16(workspace) || (v_out && !aligned16(v_out)))
+    return fail(QI_ERR_ALIGNMENT, "pointers must be 16-byte aligned");
+  size_t need = 0;
+  {
+    Carve c{nullptr, 0, 0};
+    carve_step(c, d, S_tok, S_tok, kv_cache == nullptr);
+    need = c.off + 256;
+  }
+  if (workspace_bytes < need)
+    return fail(QI_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", workspace_bytes, need);
+
+  cudaStream_t st = S(stream);
+  const int H = d.hidden, P = d.patch, T = S_tok - row0;
+  Carve c{static_cast<uint8_t*>(workspace), workspace_bytes, 0};
+  StepBufs b = carve_step(c, d, S_tok, S_tok, kv_cache == nullptr);
+  uint16_t* kv = kv_cache ? kv_cache : b.kv;
+
+  if ((r = run_time_conditioning(ctx, *model, sigma, b.block_mod, b.final_mod, b, st))) return r;
+
+  // residual stream rows row0 .. S-1
+  float* x = b.x;
+  if (row0 == 0) {
+    if ((r = run_bf16_linear(ctx, txt, text_tokens, H, model->txt_in, qi::EPI_F32, x, H, 0.f,
+                             nullptr, st)))
+      return r;
+    if (R_ref > 0) {
+      if (qi::launch_f32_to_bf16(ref_latents, b.lat_bf16, static_cast<int64_t>(R_ref) * P, st))
+        return cuda_fail("cast launch");
+      if ((r = run_bf16_linear(ctx, b.lat_bf16, R_ref, P, model->img_in, qi::EPI_F32,
+                               x + static_cast<size_t>(text_tokens) * H, H, 0.f, nullptr, st)))
+        return r;
+    }
+  }
+  uint16_t* lat_t = b.lat_bf16 + static_cast<size_t>(R_ref > 0 ? R_ref : 0) * P;
+  if (qi::launch_f32_to_bf16(latents, lat_t, static_cast<int64_t>(N) * P, st))
+    return cuda_fail("cast launch");
+  float* x_tgt = x + static_cast<size_t>(P_tok - row0) * H;
+  if ((r = run_bf16_linear(ctx, lat_t, N, P, model->img_in, qi::EPI_F32, x_tgt, H, 0.f, nullptr,
+                           st)))
+    return r;
+
+  for (int l = 0; l < d.blocks; ++l) {
+    uint16_t* kl = kv + static_cast<size_t>(l) * 2 * S_tok * H;
+    uint16_t* vl = kl + static_cast<size_t>(S_tok) * H;
+    if ((r = run_block(ctx, d, model->blocks[l], x, T, row0,
+                       b.block_mod + static_cast<size_t>(l) * 2 * 6 * H, gt, S_tok,
+                       rope_cos + static_cast<size_t>(row0) * 64,
+                       rope_sin + static_cast<size_t>(row0) * 64, kl, vl, b.block_ws,
+                       b.block_ws_bytes, st)))
+      return r;
+  }
+
+  // final adaLN (row set of the target: row 1 of final_mod) + proj_out + Euler
+  qi::GroupTable one;
+  memset(&one, 0, sizeof(one));
+  one.n = 1;
+  one.end[0] = N;
+  const uint16_t* fm = b.final_mod + 2 * H;   // row 1 (the step's sigma)
+  if ((r = run_quant(ctx, x_tgt, false, N, H, H, fm, fm + H, 0, one, 0, d.eps, nullptr, nullptr,
+                     nullptr, b.u_final, st)))
+    return r;
+  const float dt = sigma_next - sigma;
+  if ((r = run_bf16_linear(ctx, b.u_final, N, H, model->proj_out, qi::EPI_EULER, latents, P, dt,
+                           v_out, st)))
+    return r;
+  return QI_OK;
+}
+
+int qi_euler_update(qi_ctx* ctx, float* x, const float* v, int64_t n, float sigma,
+                    float sigma_next, void* stream) {
+  if (!ctx || !x || !v || n < 0) return fail(QI_ERR_INVALID_ARG, "bad arguments");
+  const float dt = sigma_next - sigma;
+  if (qi::launch_euler(x, v, n, dt, S(stream)) != 0) return cuda_fail("euler launch");
+  return QI_OK;
+}
+
+int qi_rope_tables(int n_groups, const int32_t* kinds, const int32_t* tokens,
+                   const int32_t* grid_h, const int32_t* grid_w, float* rope_cos,
+                   float* rope_sin) {
+  if (n_groups < 1 || n_groups > QI_MAX_GROUPS || !kinds || !tokens || !rope_cos || !rope_sin)
+    return fail(QI_ERR_INVALID_ARG, "bad arguments");
+  int L = 0;
+  for (int g = 0; g < n_groups; ++g)
+    if (kinds[g] == 0) L += tokens[g];
+  static const int pairs[3] = {8, 28, 28};
+  int t = 0, ti = 0, k = 0;
+  for (int g = 0; g < n_groups; ++g) {
+    if (kinds[g] != 0 && (!grid_h || !grid_w || grid_h[g] * grid_w[g] != tokens[g]))
+      return fail(QI_ERR_INVALID_ARG, "image group %d: grid does not match its token count", g);
+    for (int i = 0; i < tokens[g]; ++i, ++t) {
+      int pos[3];
+      if (kinds[g] == 0) {
+        pos[0] = pos[1] = pos[2] = ti++;
+      } else {
+        const int h = grid_h[g], w = grid_w[g], y = i / w, xx = i % w;
+        pos[0] = L + k;
+        pos[1] = y - (h - h / 2);
+        pos[2] = xx - (w - w / 2);
+      }
+      int j = 0;
+      for (int a = 0; a < 3; ++a)
+        for (int p = 0; p < pairs[a]; ++p, ++j) {
+          const double f = pow(10000.0, -static_cast<double>(p) / pairs[a]);
+          const double ang = pos[a] * f;
+          rope_cos[static_cast<size_t>(t) * 64 + j] = static_cast<float>(cos(ang));
+          rope_sin[static_cast<size_t>(t) * 64 + j] = static_cast<float>(sin(ang));
+        }
+    }
+    if (kinds[g] != 0) ++k;
+  }
+  return QI_OK;
+}
+
+int qi_sigma_schedule(int steps, int image_tokens, float* sigmas) {
+  if (steps < 1 || image_tokens < 1 || !sigmas) return fail(QI_ERR_INVALID_ARG, "bad arguments");
+  const double base_len = 256, max_len = 8192, base_shift = 0.5, max_shift = 0.9, terminal = 0.02;
+  const double slope = (max_shift - base_shift) / (max_len - base_len);
+  const double mu = image_tokens * slope + (base_shift - slope * base_len);
+  const double em = exp(mu);
+  double* one_minus = new double[steps];
+  for (int i = 0; i < steps; ++i) {
+    const double base = steps == 1 ? 1.0 : 1.0 + (1.0 / steps - 1.0) * i / (steps - 1);
+    const double shifted = em / (em + (1.0 / base - 1.0));
+    one_minus[i] = 1.0 - shifted;
+  }
+  const double stretch = one_minus[steps - 1] / (1.0 - terminal);
+  for (int i = 0; i < steps; ++i)
+    sigmas[i] = static_cast<float>(stretch > 0 ? 1.0 - one_minus[i] / stretch : 1.0);
+  sigmas[steps] = 0.0f;
+  delete[] one_minus;
+  return QI_OK;
+}
+
+int qi_debug_timeout_probe(qi_ctx* ctx, uint64_t limit_ns, void* stream) {
+  if (!ctx) return fail(QI_ERR_INVALID_ARG, "ctx is NULL");
+  if (limit_ns < 1000ull || limit_ns > 5000000000ull)
+    return fail(QI_ERR_INVALID_ARG, "limit_ns outside 1e3 .. 5e9");
+  if (qi::launch_timeout_probe(limit_ns, ctx->status, S(stream)) != 0)
+    return cuda_fail("probe launch");
+  return QI_OK;
+}
+
+}  // extern "C"

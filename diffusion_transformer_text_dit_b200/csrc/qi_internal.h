@@ -1,0 +1,132 @@
+// Internal (non-exported) declarations shared by the kernel files and the
+// C-ABI layer.  Nothing here is part of the public interface in include/qi.h.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "qi_common.cuh"
+
+namespace qi {
+
+enum GemmEpilogue {
+  EPI_BF16 = 0,    // y (bf16) = value
+  EPI_GELU = 1,    // y (bf16) = GELU_tanh(bf16(value))
+  EPI_GATED = 2,   // yf (fp32) += gate[row set] * bf16(value)
+  EPI_F32 = 3,     // yf (fp32) = value
+  EPI_EULER = 4,   // v = value; yf (fp32 latents) += dt * v
+};
+
+struct GemmParams {
+  int M, N, K;       // K in elements
+  int num_kb;        // K / (128 bytes / element size)
+  // W8A8 dequantization
+  const float* s_a;
+  const int32_t* zp_a;
+  const float* s_w;
+  const int32_t* rowsum;
+  const uint16_t* bias;   // bf16 [N] or null
+  // outputs
+  uint16_t* y;            // bf16 [M, ldy]
+  int ldy;
+  float* yf;              // fp32 [M, ldyf]: output, residual or latents
+  int ldyf;
+  const uint16_t* gate;   // bf16: gate of row set r at gate + r * gate_ld
+  int gate_ld;
+  GroupTable groups;      // row sets of global tokens
+  int row0;               // global token index of row 0
+  int32_t* acc_debug;     // optional raw int32 accumulators [M, N]
+  float dt;               // Euler: sigma_next - sigma
+  float* v_out;           // Euler: optional velocity [M, ldyf]
+  int* status;            // device status word
+};
+
+// TMA descriptor for a row-major 2-D tensor [outer, inner] with a 128-byte
+// swizzled box of box_inner x box_outer elements.
+bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, uint64_t inner,
+                  uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner,
+                  uint32_t box_outer);
+
+int pick_block_n(int N);
+int launch_gemm(bool int8, int epi, const void* A, int lda, const void* B, int ldb,
+                const GemmParams& p, int num_sms, cudaStream_t st);
+
+// Per-row quantization (optionally fused with LayerNorm + adaLN modulate).
+struct QuantParams {
+  const void* x;          // [M, ldx], fp32 or bf16
+  int x_bf16;
+  int M, K, ldx;
+  int ln;                 // 1: LayerNorm + modulate before quantizing
+  const uint16_t* shift;  // bf16 row of set r at shift + r * mod_ld
+  const uint16_t* scale;
+  int mod_ld;
+  GroupTable groups;
+  int row0;
+  float eps;
+  int8_t* q;              // [M, ldq]
+  int ldq;
+  float* s;               // [M]
+  int32_t* zp;            // [M]
+  uint16_t* u_bf16;       // if non-null: write bf16(u) [M, ldq] instead of quantizing
+};
+int launch_quant(const QuantParams& p, cudaStream_t st);
+
+int launch_prepare_w8(const float* w, int n, int k, int8_t* q, float* s, int32_t* rowsum,
+                      cudaStream_t st);
+
+// Q/K RMSNorm (cast before scale) + 3-axis RoPE on a fused QKV row block.
+struct QkNormRopeParams {
+  const uint16_t* qkv;    // [T, ldqkv] bf16: q | k | v, each heads*d wide
+  int ldqkv;
+  int T, heads, d;
+  const uint16_t* wq;     // [d] bf16
+  const uint16_t* wk;
+  const float* cos;       // [T, d/2]
+  const float* sin;
+  float eps;
+  uint16_t* q_out;        // [T, ldo]
+  uint16_t* k_out;        // [T, ldo]
+  uint16_t* v_out;        // [T, ldo]
+  int ldo;
+};
+int launch_qk_norm_rope(const QkNormRopeParams& p, cudaStream_t st);
+
+// Block-causal attention.
+struct AttnParams {
+  const uint16_t* q;      // [Sq, ldq]
+  const uint16_t* k;      // [Sk, ldkv]
+  const uint16_t* v;
+  uint16_t* o;            // [Sq, ldo]
+  int ldq, ldkv, ldo;
+  int Sq, Sk, heads, q_offset;
+  float sm_scale;
+  GroupTable groups;
+};
+int launch_attention(const AttnParams& p, cudaStream_t st);
+
+// Thin GEMV for M <= 2 rows (timestep MLP, adaLN rows).
+struct GemvJob {
+  const uint16_t* w;      // [n, k] bf16
+  const uint16_t* b;      // [n] bf16 or null
+  void* y;                // [R, ldy] (fp32 or bf16)
+  int n;
+  int ldy;
+};
+constexpr int GEMV_MAX_JOBS = 80;
+struct GemvParams {
+  const float* x;         // [R, k] fp32 input rows
+  int R, k;
+  int silu_in;            // apply SiLU to x
+  int y_bf16;
+  int n_jobs;
+  GemvJob jobs[GEMV_MAX_JOBS];
+};
+int launch_gemv(const GemvParams& p, cudaStream_t st);
+
+int launch_timestep_embedding(float t0, float t1, float* out, cudaStream_t st);
+int launch_timeout_probe(uint64_t limit_ns, int* status, cudaStream_t st);
+int launch_f32_to_bf16(const float* x, uint16_t* y, int64_t n, cudaStream_t st);
+int launch_euler(float* x, const float* v, int64_t n, float dt, cudaStream_t st);
+
+}  // namespace qi

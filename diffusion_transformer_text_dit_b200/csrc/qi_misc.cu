@@ -1,0 +1,234 @@
+// Bandwidth-bound kernels of the step:
+//  * Q/K RMSNorm with the cast ordering of "Qwen Image 2.1 native qualification"
+//    (Numerical checks: the normalized activation is cast to the scale's dtype
+//    before the scale multiplies) fused with 3-axis RoPE ("RGBA-Image-2.1 - Core
+//    AI port of Qwen-Image-2.1", Graph contracts / RoPE: 64 rotation pairs per
+//    128-wide head from per-token cos/sin tables);
+//  * the thin GEMV behind the timestep MLP and the adaLN modulation rows
+//    (qwen-image-mnn, "What runs where": modulation rows), M <= 2 rows;
+//  * the sinusoidal timestep embedding, fp32 -> bf16 casts and the FlowMatch
+//    Euler update x += (sigma_next - sigma) * v (Core AI port, Sampler).
+#include <math.h>
+
+#include "qi_common.cuh"
+#include "qi_internal.h"
+
+namespace qi {
+
+// ---------------------------------------------------------------- Q/K norm + RoPE
+
+// One CTA per token, 8 warps; warp w handles head slots w, w+8, ... of the
+// 3*heads slots (q heads, k heads, v heads).  Lane l holds elements 4l..4l+3
+// of the 128-wide head, i.e. rotation pairs 2l and 2l+1.
+// Arithmetic is fp32 with explicitly rounded operations (no contraction):
+//   r = 1 / sqrt(sum(x^2)/128 + eps);  n = bf16(x * r);  y = bf16(n * w)
+//   (a, b) -> (bf16(a c - b s), bf16(a s + b c))
+__global__ void __launch_bounds__(256) qk_norm_rope_kernel(const QkNormRopeParams p) {
+  const int t = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int H = p.heads * p.d;
+  const uint16_t* row = p.qkv + static_cast<int64_t>(t) * p.ldqkv;
+  const float2 cs = *reinterpret_cast<const float2*>(p.cos + static_cast<int64_t>(t) * (p.d / 2) + 2 * lane);
+  const float2 sn = *reinterpret_cast<const float2*>(p.sin + static_cast<int64_t>(t) * (p.d / 2) + 2 * lane);
+  for (int hs = warp; hs < 3 * p.heads; hs += 8) {
+    const int which = hs / p.heads, h = hs - which * p.heads;
+    const uint2 raw = *reinterpret_cast<const uint2*>(row + which * H + h * p.d + lane * 4);
+    uint16_t* dst = (which == 0 ? p.q_out : (which == 1 ? p.k_out : p.v_out)) +
+                    static_cast<int64_t>(t) * p.ldo + h * p.d + lane * 4;
+    if (which == 2) {
+      *reinterpret_cast<uint2*>(dst) = raw;
+      continue;
+    }
+    float x[4] = {__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xFFFF0000u),
+                  __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xFFFF0000u)};
+    float ss = __fadd_rn(__fadd_rn(__fmul_rn(x[0], x[0]), __fmul_rn(x[1], x[1])),
+                         __fadd_rn(__fmul_rn(x[2], x[2]), __fmul_rn(x[3], x[3])));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, o));
+    const float ms = __fdiv_rn(ss, static_cast<float>(p.d));
+    const float r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, p.eps)));
+    const uint2 wraw = *reinterpret_cast<const uint2*>((which == 0 ? p.wq : p.wk) + lane * 4);
+    const float w[4] = {__uint_as_float(wraw.x << 16), __uint_as_float(wraw.x & 0xFFFF0000u),
+                        __uint_as_float(wraw.y << 16), __uint_as_float(wraw.y & 0xFFFF0000u)};
+    float y[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) y[i] = bf16_round_f(__fmul_rn(bf16_round_f(__fmul_rn(x[i], r)), w[i]));
+    const float c0 = cs.x, c1 = cs.y, s0 = sn.x, s1 = sn.y;
+    const float o0 = __fsub_rn(__fmul_rn(y[0], c0), __fmul_rn(y[1], s0));
+    const float o1 = __fadd_rn(__fmul_rn(y[0], s0), __fmul_rn(y[1], c0));
+    const float o2 = __fsub_rn(__fmul_rn(y[2], c1), __fmul_rn(y[3], s1));
+    const float o3 = __fadd_rn(__fmul_rn(y[2], s1), __fmul_rn(y[3], c1));
+    *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(o0, o1), pack_bf16x2(o2, o3));
+  }
+}
+
+int launch_qk_norm_rope(const QkNormRopeParams& p, cudaStream_t st) {
+  if (p.T == 0) return 0;
+  if (p.d != 128) return -1;
+  qk_norm_rope_kernel<<<p.T, 256, 0, st>>>(p);
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+// ---------------------------------------------------------------- GEMV
+
+// y[r][j] = sum_k act(x[r][k]) * W[j][k] + b[j] for every row j of every job.
+// x (R <= 2 rows) is staged in shared memory as fp32 (SiLU applied on load
+// when requested); one warp per output row, 16-byte weight loads.
+constexpr int GEMV_THREADS = 256;
+
+__global__ void __launch_bounds__(GEMV_THREADS) gemv_kernel(const GemvParams p) {
+  extern __shared__ float xs[];
+  const int total_in = p.R * p.k;
+  for (int i = threadIdx.x; i < total_in; i += GEMV_THREADS) {
+    float v = p.x[i];
+    if (p.silu_in) v = v / (1.0f + expf(-v));
+    xs[i] = v;
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int gwarp = (blockIdx.x * GEMV_THREADS + threadIdx.x) >> 5;
+  const int nwarps = (gridDim.x * GEMV_THREADS) >> 5;
+  int total_rows = 0;
+  for (int j = 0; j < p.n_jobs; ++j) total_rows += p.jobs[j].n;
+  for (int g = gwarp; g < total_rows; g += nwarps) {
+    int job = 0, row = g;
+    while (row >= p.jobs[job].n) {
+      row -= p.jobs[job].n;
+      ++job;
+    }
+    const GemvJob& J = p.jobs[job];
+    const uint16_t* wr = J.w + static_cast<int64_t>(row) * p.k;
+    float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll 4
+    for (int kk = lane * 8; kk < p.k; kk += 256) {
+      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(wr + kk));
+      const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float w0 = __uint_as_float(wv[i] << 16), w1 = __uint_as_float(wv[i] & 0xFFFF0000u);
+        acc0 = fmaf(w0, xs[kk + 2 * i], fmaf(w1, xs[kk + 2 * i + 1], acc0));
+        if (p.R > 1)
+          acc1 = fmaf(w0, xs[p.k + kk + 2 * i], fmaf(w1, xs[p.k + kk + 2 * i + 1], acc1));
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      acc0 += __shfl_xor_sync(0xffffffffu, acc0, o);
+      acc1 += __shfl_xor_sync(0xffffffffu, acc1, o);
+    }
+    if (lane == 0) {
+      const float b = J.b ? bf16_bits_to_float(J.b[row]) : 0.f;
+      const float out[2] = {acc0 + b, acc1 + b};
+      for (int r = 0; r < p.R; ++r) {
+        if (p.y_bf16) {
+          __nv_bfloat16 h = __float2bfloat16_rn(out[r]);
+          static_cast<uint16_t*>(J.y)[static_cast<int64_t>(r) * J.ldy + row] =
+              *reinterpret_cast<uint16_t*>(&h);
+        } else {
+          static_cast<float*>(J.y)[static_cast<int64_t>(r) * J.ldy + row] = out[r];
+        }
+      }
+    }
+  }
+}
+
+int launch_gemv(const GemvParams& p, cudaStream_t st) {
+  if (p.R < 1 || p.R > 2 || p.k % 256 != 0 || p.n_jobs > GEMV_MAX_JOBS) return -1;
+  int total_rows = 0;
+  for (int j = 0; j < p.n_jobs; ++j) total_rows += p.jobs[j].n;
+  if (total_rows == 0) return 0;
+  const size_t smem = static_cast<size_t>(p.R) * p.k * sizeof(float);
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(gemv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024) !=
+        cudaSuccess)
+      return -1;
+    attr = true;
+  }
+  if (smem > 64 * 1024) return -1;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int rows_per_cta = GEMV_THREADS / 32;
+  int grid = (total_rows + rows_per_cta - 1) / rows_per_cta;
+  const int max_grid = sms * 6;
+  if (grid > max_grid) grid = max_grid;
+  gemv_kernel<<<grid, GEMV_THREADS, smem, st>>>(p);
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+// ---------------------------------------------------------------- small kernels
+
+// out[r] = [cos(1000 t_r f_i), sin(1000 t_r f_i)], f_i = exp(-ln(1e4) i / 128), i < 128,
+// for the two timesteps t_0 (row 0) and t_1 (row 1).  Evaluated in double.
+__global__ void timestep_embedding_kernel(float t0, float t1, float* out) {
+  const int r = blockIdx.x;
+  const int i = threadIdx.x;   // 0..127
+  const double f = exp(-log(10000.0) * static_cast<double>(i) / 128.0);
+  const double a = 1000.0 * static_cast<double>(r == 0 ? t0 : t1) * f;
+  out[r * 256 + i] = static_cast<float>(cos(a));
+  out[r * 256 + 128 + i] = static_cast<float>(sin(a));
+}
+
+int launch_timestep_embedding(float t0, float t1, float* out, cudaStream_t st) {
+  timestep_embedding_kernel<<<2, 128, 0, st>>>(t0, t1, out);
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+__global__ void f32_to_bf16_kernel(const float* __restrict__ x, uint16_t* __restrict__ y, int64_t n) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    __nv_bfloat16 h = __float2bfloat16_rn(x[i]);
+    y[i] = *reinterpret_cast<uint16_t*>(&h);
+  }
+}
+
+int launch_f32_to_bf16(const float* x, uint16_t* y, int64_t n, cudaStream_t st) {
+  if (n == 0) return 0;
+  int64_t g = (n + 255) / 256;
+  if (g > 148 * 16) g = 148 * 16;
+  f32_to_bf16_kernel<<<static_cast<int>(g), 256, 0, st>>>(x, y, n);
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+// x += dt * v in fp32, one rounding per operation (no fused multiply-add).
+__global__ void euler_kernel(float* __restrict__ x, const float* __restrict__ v, int64_t n, float dt) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    x[i] = __fadd_rn(x[i], __fmul_rn(dt, v[i]));
+}
+
+int launch_euler(float* x, const float* v, int64_t n, float dt, cudaStream_t st) {
+  if (n == 0) return 0;
+  int64_t g = (n + 255) / 256;
+  if (g > 148 * 16) g = 148 * 16;
+  euler_kernel<<<static_cast<int>(g), 256, 0, st>>>(x, v, n, dt);
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+// Failure-detection probe: wait on an mbarrier that nothing ever arrives on,
+// bounded by limit_ns; the expiry is recorded in the status word.
+__global__ void timeout_probe_kernel(uint64_t limit_ns, int* status) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(&bar, 0)) {
+      if (globaltimer_ns() - t0 > limit_ns) {
+        set_error(status, QI_DEV_ERR_TIMEOUT);
+        break;
+      }
+    }
+  }
+}
+
+int launch_timeout_probe(uint64_t limit_ns, int* status, cudaStream_t st) {
+  timeout_probe_kernel<<<1, 32, 0, st>>>(limit_ns, status);
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+}  // namespace qi

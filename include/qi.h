@@ -1,0 +1,312 @@
+/*
+ * qi.h - C ABI of libqi: one denoising step of the Qwen-Image-2.1
+ * single-stream diffusion transformer with W8A8 Linears, for NVIDIA B200
+ * (sm_100a).
+ *
+ * Sources (cited by page title and section):
+ *   [W8]   FlagRelease "Qwen-Image-2.1-W8A8-arm-FlagOS", "Quantization and
+ *          validation": symmetric INT8 weights per output channel (zero point 0,
+ *          FP32 scales); dynamic asymmetric INT8 activations per token/row
+ *          (FP32 scales); INT32 accumulation, FP32 scaling, BF16 output.
+ *   [QN]   "Qwen Image 2.1 native qualification", "Numerical checks": Q/K
+ *          RMSNorm casts the normalized activation to the scale's dtype
+ *          before scaling.
+ *   [GC]   "RGBA-Image-2.1 - Core AI port of Qwen-Image-2.1", intro and
+ *          "Graph contracts": 32-block single-stream DiT with block-causal
+ *          attention; joint sequence [text | image] with one image token per
+ *          16x16 px tile; 3-axis RoPE positions; 64 rotation pairs per head;
+ *          shifted sigmas and the Euler update x += (sigma_next - sigma) * v.
+ *   [MNN]  qwen-image-mnn, "What runs where": 3-axis RoPE, block-causal mask
+ *          and modulation rows as the joint-sequence bookkeeping.
+ *   [PX]   EliovpAI "Qwen_Image-2.1-MXFP4-Paiton-RDNA4", "Runtime precision and
+ *          quality" / "Tested operating limits": cached text-prefix pass
+ *          (prefix KV reuse); unsupported settings rejected before GPU work.
+ *
+ * Conventions (all entry points):
+ *   - Every call returns a qi_status.  Arguments are validated on the host
+ *     before anything is launched; a rejected call launches nothing.
+ *     qi_last_error() returns a text description of the last failure on the
+ *     calling thread.
+ *   - Tensor pointers are device pointers owned by the caller unless stated
+ *     otherwise; all must be 16-byte aligned.  Matrices are row-major
+ *     [rows, ld] with ld in elements.  bf16 values are passed as uint16_t bit
+ *     patterns.  Weights are [out, in] (K-major).
+ *   - Every device call is asynchronous on the given CUDA stream
+ *     (cudaStream_t passed as void*; NULL = the legacy default stream).
+ *     Nothing synchronizes except qi_ctx_check().
+ *   - The library never allocates device memory in a compute call.  Scratch
+ *     comes from a caller-owned workspace whose size the *_workspace_bytes
+ *     functions return; qi_ctx_create() allocates only a 256-byte device
+ *     status word.
+ *   - Kernels never trap.  A pipeline wait that does not complete within 2 s
+ *     records QI_ERR_TIMEOUT in the context's status word and the kernel
+ *     returns; qi_ctx_check() reports it.
+ */
+#ifndef QI_H_
+#define QI_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct qi_ctx qi_ctx;
+
+typedef enum {
+  QI_OK = 0,
+  QI_ERR_INVALID_ARG = 1,       /* null pointer, negative size, bad enum, bad group table */
+  QI_ERR_UNSUPPORTED_SHAPE = 2, /* shape outside what the kernels support (see each call) */
+  QI_ERR_ALIGNMENT = 3,         /* pointer or leading dimension not 16-byte aligned */
+  QI_ERR_CUDA = 4,              /* a CUDA runtime / driver call failed */
+  QI_ERR_TIMEOUT = 5,           /* a kernel's bounded wait expired (device status word) */
+  QI_ERR_WORKSPACE = 6          /* workspace smaller than the *_workspace_bytes size */
+} qi_status;
+
+typedef enum { QI_F32 = 0, QI_BF16 = 1 } qi_dtype;
+
+/* Joint-sequence groups ([MNN] "block-causal mask"; [GC] Sequence).
+ * Groups are contiguous and ordered: group g holds global tokens
+ * [end[g-1], end[g]) (end[-1] = 0).  A token attends to every token of its
+ * own group and of all earlier groups.  row_set[g] selects which modulation
+ * row set (adaLN rows) the group's tokens use.  Passed by host pointer. */
+#define QI_MAX_GROUPS 16
+typedef struct qi_groups {
+  int32_t n;                        /* 1..QI_MAX_GROUPS */
+  int32_t end[QI_MAX_GROUPS];       /* strictly ascending; end[n-1] = sequence length */
+  int32_t row_set[QI_MAX_GROUPS];   /* >= 0 */
+} qi_groups;
+
+/* One W8A8 Linear prepared by qi_prepare_w8 ([W8]). */
+typedef struct qi_w8 {
+  const int8_t* q;         /* [n, k] int8 codes, K-major */
+  const float* s;          /* [n] per-output-channel scale */
+  const int32_t* rowsum;   /* [n] sum_k q[n, k] (zero-point correction) */
+  const uint16_t* bias;    /* [n] bf16, or NULL */
+  int32_t n, k;
+} qi_w8;
+
+/* One BF16 Linear: y = x W^T + b. */
+typedef struct qi_linear_bf16 {
+  const uint16_t* w;       /* [n, k] bf16 */
+  const uint16_t* bias;    /* [n] bf16, or NULL */
+  int32_t n, k;
+} qi_linear_bf16;
+
+typedef enum {
+  QI_EPI_STORE = 0,           /* y = bf16(Linear(x)) */
+  QI_EPI_GELU_TANH = 1,       /* y = bf16(GELU_tanh(bf16(Linear(x)))) */
+  QI_EPI_GATED_RESIDUAL = 2   /* residual += gate[row set] * bf16(Linear(x)), fp32 */
+} qi_epilogue_kind;
+
+typedef struct qi_epilogue {
+  int32_t kind;                /* qi_epilogue_kind */
+  float* residual;             /* GATED_RESIDUAL: fp32 [M, ld_residual], updated in place */
+  int32_t ld_residual;
+  const uint16_t* gate;        /* GATED_RESIDUAL: bf16 gate row of set r at gate + r * gate_ld */
+  int32_t gate_ld;
+  const qi_groups* groups;     /* GATED_RESIDUAL: row set of each row (host pointer) */
+  int32_t row0;                /* global token index of row 0 */
+} qi_epilogue;
+
+typedef struct qi_dims {
+  int32_t hidden;     /* H = heads * head_dim */
+  int32_t heads;
+  int32_t head_dim;   /* must be 128 */
+  int32_t mlp;        /* F */
+  int32_t patch;      /* P: latent token width (64, or 256 with 2x2 packing) */
+  int32_t blocks;
+  float eps;          /* LayerNorm / RMSNorm epsilon (1e-6) */
+} qi_dims;
+
+typedef struct qi_block_weights {
+  qi_w8 qkv;               /* n = 3H: rows [0,H) = q, [H,2H) = k, [2H,3H) = v */
+  qi_w8 out;               /* n = H, k = H */
+  qi_w8 up;                /* n = F, k = H */
+  qi_w8 down;              /* n = H, k = F */
+  const uint16_t* norm_q;  /* [head_dim] bf16 RMSNorm scale */
+  const uint16_t* norm_k;
+  qi_linear_bf16 mod;      /* adaLN: n = 6H, k = H (used by the step-level calls) */
+} qi_block_weights;
+
+typedef struct qi_model {
+  qi_dims dims;
+  const qi_block_weights* blocks;   /* host array of dims.blocks entries */
+  qi_linear_bf16 t1;                /* timestep MLP 1: n = H, k = 256 */
+  qi_linear_bf16 t2;                /* timestep MLP 2: n = H, k = H */
+  qi_linear_bf16 img_in;            /* n = H, k = P */
+  qi_linear_bf16 txt_in;            /* n = H, k = H */
+  qi_linear_bf16 final_mod;         /* final adaLN: n = 2H (shift, scale), k = H */
+  qi_linear_bf16 proj_out;          /* n = P, k = H */
+} qi_model;
+
+typedef enum {
+  QI_KV_NONE = 0,          /* every token processed; K/V buffers are scratch */
+  QI_KV_WRITE_PREFIX = 1,  /* every token processed; the prefix K/V stay in the buffers */
+  QI_KV_READ_PREFIX = 2    /* only the target rows processed; prefix K/V read from the buffers */
+} qi_kv_mode;
+
+/* ------------------------------------------------------------------ context */
+
+/* Create a context on CUDA device `device`.  Allocates one 256-byte device
+ * status word (cudaMalloc, outside any compute call).  *out is owned by the
+ * caller and released with qi_ctx_destroy. */
+int qi_ctx_create(int device, qi_ctx** out);
+int qi_ctx_destroy(qi_ctx* ctx);
+
+/* Synchronize `stream`, then read and clear the device status word.
+ * Returns QI_ERR_TIMEOUT if a kernel recorded an expired wait, QI_ERR_CUDA if
+ * the stream reported an error, else QI_OK. */
+int qi_ctx_check(qi_ctx* ctx, void* stream);
+
+/* Copy the calling thread's last error text into buf (NUL-terminated). */
+int qi_last_error(char* buf, size_t n);
+
+/* ------------------------------------------------------------------ W8A8 ([W8]) */
+
+/* Quantize fp32 weights w [n, k] symmetrically per output channel:
+ * s[n] = max|w[n,:]| / 127 (1 for an all-zero row), q = clamp(rint(w / s), -127, 127),
+ * rowsum[n] = sum_k q[n, k].  Requires k % 8 == 0 (8 <= k). */
+int qi_prepare_w8(qi_ctx* ctx, const float* w, int n, int k, int8_t* q, float* s,
+                  int32_t* rowsum, void* stream);
+
+/* Per-token dynamic asymmetric int8 quantization of x [M, K] (ld ldx):
+ *   lo = min(min_k u, 0), hi = max(max_k u, 0), s = (hi - lo)/255,
+ *   zp = clamp(rint(-128 - lo/s), -128, 127), q = clamp(rint(u/s) + zp, -128, 127)
+ * (fp32 IEEE operations; an all-zero row gets s = 1, zp = 0).
+ * If shift != NULL the quantized value is u = LN(x)(1 + scale) + shift, with a
+ * non-affine LayerNorm (eps) and the bf16 shift/scale row of the token's row
+ * set (shift + r * mod_ld, scale + r * mod_ld; groups/row0 map rows to global
+ * tokens); else u = x.  x_dtype is QI_F32 or QI_BF16.
+ * Outputs: q [M, K] int8 (ld K), s_a [M] fp32, zp_a [M] int32.
+ * Requires K % 8 == 0 and K <= 16384; ldx % 8 == 0. */
+int qi_quantize_act(qi_ctx* ctx, const void* x, int x_dtype, int M, int K, int ldx,
+                    const uint16_t* shift, const uint16_t* scale, int mod_ld,
+                    const qi_groups* groups, int row0, float eps, int8_t* q, float* s_a,
+                    int32_t* zp_a, void* stream);
+
+/* W8A8 Linear on tcgen05 tensor cores (int8 x int8 -> int32 in TMEM):
+ *   acc[m, n] = sum_k qa[m, k] w.q[n, k]
+ *   val = (acc - zp_a[m] * w.rowsum[n]) * s_a[m] * w.s[n] + w.bias[n]   (fp32)
+ * then the epilogue ep (NULL = QI_EPI_STORE) writes y [M, w.n] bf16 (ld ldy) or
+ * updates ep->residual.  acc_debug, if not NULL, receives the raw int32
+ * accumulators [M, w.n].  Requires w.k % 128 == 0, w.n % 16 == 0, ldy % 8 == 0. */
+int qi_w8a8_linear(qi_ctx* ctx, const int8_t* qa, const float* s_a, const int32_t* zp_a, int M,
+                   const qi_w8* w, const qi_epilogue* ep, uint16_t* y, int ldy,
+                   int32_t* acc_debug, void* stream);
+
+/* BF16 Linear on tcgen05 tensor cores: y [M, w.n] fp32 (ld ldy) = a [M, w.k] W^T + b.
+ * Requires w.k % 64 == 0, w.n % 16 == 0, lda % 8 == 0. */
+int qi_bf16_linear(qi_ctx* ctx, const uint16_t* a, int M, int lda, const qi_linear_bf16* w,
+                   float* y, int ldy, void* stream);
+
+/* ------------------------------------------------------------------ attention path */
+
+/* Q/K RMSNorm + 3-axis RoPE on a fused QKV block qkv [T, 3H] bf16 ([QN], [GC] RoPE):
+ *   r = 1/sqrt(mean(x^2) + eps); n = bf16(x r); y = bf16(n w)   (cast BEFORE the scale)
+ *   pair j = (y[2j], y[2j+1]) -> (bf16(a c - b s), bf16(a s + b c)), c/s = cos/sin[t, j]
+ * applied per head to q (wq) and k (wk); v is copied.  Outputs q_out, k_out,
+ * v_out [T, ldo] bf16.  cos/sin: [T, head_dim/2] fp32.  head_dim must be 128. */
+int qi_qk_norm_rope(qi_ctx* ctx, const uint16_t* qkv, int T, int heads, int head_dim,
+                    const uint16_t* wq, const uint16_t* wk, const float* rope_cos,
+                    const float* rope_sin, float eps, uint16_t* q_out, uint16_t* k_out,
+                    uint16_t* v_out, int ldo, void* stream);
+
+/* Block-causal attention ([GC], [MNN]):  O = softmax(Q K^T sm_scale + M) V per head,
+ * M(i, j) = 0 iff group(j) <= group(q_offset + i), else -inf.
+ * q [Sq, ldq], k/v [Sk, ldkv], o [Sq, ldo] bf16; head h occupies columns
+ * [h*128, (h+1)*128).  Queries are global tokens q_offset .. q_offset+Sq-1;
+ * keys are global tokens 0 .. Sk-1 (Sk = groups->end[n-1]).  Key tiles that
+ * no query of a tile may see are skipped.  head_dim must be 128. */
+int qi_attn_block_causal(qi_ctx* ctx, const uint16_t* q, int ldq, int Sq, int q_offset,
+                         const uint16_t* k, const uint16_t* v, int ldkv, int Sk, int heads,
+                         int head_dim, const qi_groups* groups, float sm_scale, uint16_t* o,
+                         int ldo, void* stream);
+
+/* ------------------------------------------------------------------ block */
+
+/* Workspace bytes needed by qi_dit_block_forward for T processed rows. */
+int qi_block_workspace_bytes(const qi_dims* dims, int T, size_t* bytes);
+
+/* One single-stream block on rows row0 .. row0+T-1 of the joint sequence:
+ *   u1 = LN(x)(1 + scale1) + shift1 -> W8A8 QKV -> Q/K RMSNorm + RoPE
+ *   x += gate1 * W8A8_out(attention)          (block-causal, keys 0 .. end of row's group)
+ *   u2 = LN(x)(1 + scale2) + shift2 -> W8A8 up -> GELU-tanh -> W8A8 down
+ *   x += gate2 * down
+ * x: fp32 residual rows [T, H] (in/out).  mod: bf16 [R, 6, H] rows
+ * (shift1, scale1, gate1, shift2, scale2, gate2) per row set.  rope_cos/sin:
+ * [T, 64] fp32 tables of the processed rows.  k_layer / v_layer: this layer's
+ * bf16 [S, H] key and value buffers (S = groups->end[n-1]); the call writes
+ * rows row0 .. row0+T-1 and attends over rows 0 .. S-1 within the mask.
+ * kv_mode NONE / WRITE_PREFIX need row0 == 0 and T == S; READ_PREFIX needs
+ * row0 + T == S with rows 0 .. row0-1 already written by an earlier call
+ * ([PX] cached prefix pass). */
+int qi_dit_block_forward(qi_ctx* ctx, const qi_dims* dims, const qi_block_weights* w, float* x,
+                         int T, int row0, const uint16_t* mod, const qi_groups* groups,
+                         const float* rope_cos, const float* rope_sin, uint16_t* k_layer,
+                         uint16_t* v_layer, int kv_mode, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------ step */
+
+/* Timestep conditioning of a step: temb_r = t2(SiLU(t1(sinusoid(1000 t_r))))
+ * for t_0 = 0 (conditioning prefix rows) and t_1 = sigma (target rows);
+ * block_mod [blocks][2][6H] bf16 = mod_l(SiLU(temb_r)); final_mod [2H] bf16 =
+ * final_mod(SiLU(temb_1)) as (shift, scale).  Workspace: qi_step_workspace_bytes. */
+int qi_time_conditioning(qi_ctx* ctx, const qi_model* model, float sigma, uint16_t* block_mod,
+                         uint16_t* final_mod, void* workspace, size_t workspace_bytes,
+                         void* stream);
+
+/* Workspace bytes needed by qi_denoise_step for a sequence of S tokens. */
+int qi_step_workspace_bytes(const qi_dims* dims, int S, size_t* bytes);
+
+/* One FlowMatch Euler denoising step ([GC] Graph contracts / Sampler):
+ *   x = [txt_in(txt) | img_in(ref_latents) | img_in(latents)]
+ *   x = blocks(x) with the time conditioning above
+ *   v = proj_out(LN(x_target)(1 + scale) + shift);   latents += (sigma_next - sigma) v
+ * latents [N, P] fp32 (in/out); txt [L, H] bf16 with L = text_tokens (NULL in
+ * READ_PREFIX mode); ref_latents [R, P] fp32 for an edit sequence (NULL if
+ * none; R = prefix tokens - L).  groups: the joint sequence, target last.
+ * rope_cos/sin [S, 64] fp32 for the whole sequence.  kv_cache: bf16
+ * [blocks][2][S][H] (K then V per block) holding the prefix K/V across steps;
+ * may be NULL in QI_KV_NONE mode (workspace used).  v_out [N, P] fp32 gets the
+ * velocity if not NULL. */
+int qi_denoise_step(qi_ctx* ctx, const qi_model* model, float* latents, const uint16_t* txt,
+                    int text_tokens, const float* ref_latents, const qi_groups* groups,
+                    const float* rope_cos, const float* rope_sin, float sigma, float sigma_next,
+                    int kv_mode, uint16_t* kv_cache, float* v_out, void* workspace,
+                    size_t workspace_bytes, void* stream);
+
+/* x += (sigma_next - sigma) * v over n fp32 values, one rounding per operation
+ * (no fused multiply-add); sigma_next - sigma is rounded to fp32 first ([GC] Sampler). */
+int qi_euler_update(qi_ctx* ctx, float* x, const float* v, int64_t n, float sigma,
+                    float sigma_next, void* stream);
+
+/* ------------------------------------------------------------------ host helpers */
+
+/* RoPE tables ([GC] RoPE): text token i at (i, i, i); image token (y, x) of the
+ * k-th image group (h x w grid, raster order) at (L + k, y - (h - h/2), x - (w - w/2)),
+ * L = number of text tokens.  Rotation pairs 0..7 use the frame axis, 8..35 the
+ * h axis, 36..63 the w axis; pair i of an axis with n pairs has frequency
+ * 10000^(-i/n).  kinds[g]: 0 text, 1 image.  Writes HOST arrays cos/sin [S, 64]. */
+int qi_rope_tables(int n_groups, const int32_t* kinds, const int32_t* tokens,
+                   const int32_t* grid_h, const int32_t* grid_w, float* rope_cos,
+                   float* rope_sin);
+
+/* Shifted FlowMatch sigmas ([GC] Sampler): linspace(1, 1/steps, steps) shifted by
+ * e^mu / (e^mu + 1/sigma - 1), mu linear in image_tokens (0.5 at 256 tokens,
+ * 0.9 at 8192), tail stretched to 0.02, then 0 appended.  Writes HOST sigmas[steps+1]. */
+int qi_sigma_schedule(int steps, int image_tokens, float* sigmas);
+
+/* Failure-detection probe: launch one CTA that waits on an mbarrier nothing
+ * arrives on, bounded by limit_ns (1e3 .. 5e9).  The wait expires, the kernel
+ * records QI_ERR_TIMEOUT in the status word and returns; the context stays
+ * usable.  Read the result with qi_ctx_check(). */
+int qi_debug_timeout_probe(qi_ctx* ctx, uint64_t limit_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QI_H_ */

@@ -316,9 +316,9 @@ def dit_block(x, pw: dict, mod, row_set, q_group, k_group, cos, sin, heads, head
 
     Steps (reading of the pages' block; see the design notes):
       u1 = LN(x)(1 + scale1) + shift1 -> W8A8 QKV -> Q/K RMSNorm (cast first) -> RoPE
-      o  = block-causal attention
+      o  = bf16(block-causal attention)
       x += gate1 * W8A8 out(o)
-      u2 = LN(x)(1 + scale2) + shift2 -> W8A8 up -> GELU-tanh -> W8A8 down
+      u2 = LN(x)(1 + scale2) + shift2 -> W8A8 up -> bf16(GELU-tanh) -> W8A8 down
       x += gate2 * down
     Returns the new x (and the (K, V) of the processed rows if return_kv).
     """
@@ -341,11 +341,16 @@ def dit_block(x, pw: dict, mod, row_set, q_group, k_group, cos, sin, heads, head
     else:
         k_all, v_all = k, v
     o = attention_block_causal(q, k_all, v_all, q_group, k_group, 1.0 / math.sqrt(head_dim))
-    o = o.reshape(T, H)
+    # The attention output and the GELU output are activation tensors of the
+    # BF16 transformer (FlagOS card: the Linears outside the W8A8 set and the
+    # activations stay BF16), so the per-token quantizer sees them as bf16
+    # values: the code decision is taken on the same bf16 input precision as
+    # the CUDA path.
+    o = bf16_round(o.reshape(T, H))
 
     x = x + gate1 * w8a8_apply(o, pw["out"])
     u2 = modulate(layer_norm(x, eps), shift2, scale2)
-    g = gelu_tanh(w8a8_apply(u2, pw["up"]))
+    g = bf16_round(gelu_tanh(w8a8_apply(u2, pw["up"])))
     x = x + gate2 * w8a8_apply(g, pw["down"])
     if return_kv:
         return x, (k, v)

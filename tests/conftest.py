@@ -27,3 +27,15 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+@pytest.fixture(scope="session")
+def ctx():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from diffusion_transformer_text_dit_b200 import build_lib, qi
+    build_lib.build()
+    c = qi.Context()
+    yield c
+    c.close()

@@ -1,0 +1,101 @@
+"""Block-level parity: qi_dit_block_forward against the oracle's block, and the
+cached-prefix invariant (target rows computed with prefix K/V read from the
+cache equal the uncached computation bit for bit)."""
+import numpy as np
+import pytest
+import torch
+
+from diffusion_transformer_text_dit_b200 import qi, synth
+from oracle import qi_oracle as O
+from tests._util import bf16_np, cuda, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+
+def oracle_block_weights(wts):
+    return O.prepare_block({k: v.float().numpy() for k, v in wts.items()})
+
+
+def run_block(ctx, cfg, wts, x, mod, sizes, kv=None, row0=0, mode=qi.QI_KV_NONE, bw=None):
+    H = cfg.hidden
+    ends = list(np.cumsum(sizes))
+    S = ends[-1]
+    g = qi.groups_struct(ends, [0] * (len(sizes) - 1) + [1])
+    gd = [(gr.kind, gr.tokens, gr.grid) for gr in cfg.groups] if cfg.groups and sum(
+        gg.tokens for gg in cfg.groups) == S else [("text", sizes[0], None)] + [
+        ("image", n, (1, n)) for n in sizes[1:]]
+    cos, sin = qi.qi_rope_tables(gd)
+    dims = qi.dims_struct(H, cfg.heads, cfg.mlp, cfg.patch, 1)
+    bw = bw or qi.BlockWeights(ctx, wts)
+    if kv is None:
+        kv = (torch.zeros((S, H), dtype=torch.bfloat16, device="cuda"),
+              torch.zeros((S, H), dtype=torch.bfloat16, device="cuda"))
+    T = S - row0
+    ws = torch.empty(qi.qi_block_workspace_bytes(dims, T), dtype=torch.uint8, device="cuda")
+    xg = cuda(x)
+    qi.qi_dit_block_forward(ctx, dims, bw.struct, xg, row0, cuda(mod), g,
+                            cuda(cos[row0:].contiguous()), cuda(sin[row0:].contiguous()),
+                            kv[0], kv[1], mode, ws)
+    ctx.check()
+    return xg, kv, bw, gd
+
+
+def oracle_block(cfg, wts, x, mod, sizes, gd):
+    ends = list(np.cumsum(sizes))
+    gid = O.group_ids(ends)
+    rs = np.where(gid < len(sizes) - 1, 0, 1)
+    cos, sin = O.rope_tables(O.rope_positions(gd))
+    return O.dit_block(x.numpy(), oracle_block_weights(wts), bf16_np(mod), rs, gid, gid, cos, sin,
+                       cfg.heads, cfg.head_dim, cfg.eps)
+
+
+@pytest.mark.parametrize("cfg", [synth.TINY, synth.TINY.replace(
+    name="tiny_ragged", groups=(synth.Group("text", 21), synth.Group("image", 35, (5, 7))))],
+    ids=["tiny", "ragged"])
+def test_block_tiny_vs_oracle(ctx, cfg):
+    wts = synth.block_weights(cfg, 0)
+    sizes = cfg.group_sizes()
+    x = synth.hidden_states(cfg, cfg.tokens)
+    mod = synth.mod_table(cfg)
+    xg, _, _, gd = run_block(ctx, cfg, wts, x, mod, sizes)
+    ref = oracle_block(cfg, wts, x, mod, sizes, gd)
+    out = xg.cpu().numpy()
+    assert np.all(np.isfinite(out))
+    assert rel_l2(out, ref) < 1e-2
+    assert rel_l2(out - x.numpy(), ref - x.numpy()) < 1e-2   # the block's own contribution
+
+
+def test_block_512px_vs_oracle(ctx):
+    cfg = synth.BLOCK512
+    wts = synth.block_weights(cfg, 0)
+    sizes = cfg.group_sizes()
+    x = synth.hidden_states(cfg, cfg.tokens)
+    mod = synth.mod_table(cfg)
+    xg, _, _, gd = run_block(ctx, cfg, wts, x, mod, sizes)
+    ref = oracle_block(cfg, wts, x, mod, sizes, gd)
+    out = xg.cpu().numpy()
+    assert rel_l2(out, ref) < 1e-2
+    assert rel_l2(out - x.numpy(), ref - x.numpy()) < 1e-2
+
+
+@pytest.mark.parametrize("sizes", [[128, 64, 192], [16, 64], [21, 35, 30]])
+def test_block_cached_prefix_bit_identical(ctx, sizes):
+    cfg = synth.TINY
+    wts = synth.block_weights(cfg, 1)
+    S = sum(sizes)
+    x = synth.hidden_states(cfg, S, tag="xc")
+    mod = synth.mod_table(cfg, tag="modc")
+    full, kv, bw, _ = run_block(ctx, cfg, wts, x, mod, sizes, mode=qi.QI_KV_WRITE_PREFIX)
+    P = S - sizes[-1]
+    part, _, _, _ = run_block(ctx, cfg, wts, x[P:].contiguous(), mod, sizes, kv=kv, row0=P,
+                              mode=qi.QI_KV_READ_PREFIX, bw=bw)
+    assert torch.equal(full[P:], part)
+
+
+def test_block_rejects_bad_arguments(ctx):
+    cfg = synth.TINY
+    wts = synth.block_weights(cfg, 0)
+    with pytest.raises(qi.QiError) as e:
+        run_block(ctx, cfg, wts, synth.hidden_states(cfg, 80), synth.mod_table(cfg), [16, 64],
+                  row0=16, mode=qi.QI_KV_NONE)
+    assert e.value.code == qi.QI_ERR_INVALID_ARG
