@@ -92,9 +92,10 @@ __device__ __forceinline__ int key_limit(const GroupTable& g, int t) {
 
 __global__ void __launch_bounds__(AT_THREADS, 2) attn_kernel(const AttnParams p) {
   extern __shared__ __align__(128) uint8_t at_smem[];
+  // layout: Q | K0 | V0 | K1 | V1  (5 x 16 KB); stage b: K at 16K + 32K b, V at 32K + 32K b
   const uint32_t sQ = smem_u32(at_smem);
   const uint32_t sK0 = sQ + AT_TILE_BYTES;
-  const uint32_t sV0 = sQ + 3 * AT_TILE_BYTES;
+  const uint32_t sV0 = sQ + 2 * AT_TILE_BYTES;
 
   const int n_qtiles = (p.Sq + AT_BM - 1) / AT_BM;
   const int qt = n_qtiles - 1 - static_cast<int>(blockIdx.x);   // heavy tiles first
@@ -236,6 +237,8 @@ __global__ void __launch_bounds__(AT_THREADS, 2) attn_kernel(const AttnParams p)
     }
     __syncthreads();
   }
+
+  cp_async_wait<0>();
 
   // full row sums across the quad, normalise, store
 #pragma unroll
