@@ -13,10 +13,21 @@
 #include "qi_common.cuh"
 #include "qi_internal.h"
 
+// Optional per-launch timing: when enabled, every kernel launch of the library
+// is bracketed by a pair of CUDA events on its stream; durations are summed per
+// kernel class when read back.  Launches are counted per class either way.
+constexpr int QI_PROF_CLASSES = 8;
+constexpr int QI_PROF_MAX_PAIRS = 16384;
+
 struct qi_ctx {
   int device;
   int num_sms;
   int* status;   // device status word
+  bool prof_on;
+  int prof_used;
+  cudaEvent_t* prof_ev;          // [2 * QI_PROF_MAX_PAIRS]
+  int* prof_cls;                 // [QI_PROF_MAX_PAIRS]
+  long long launches[QI_PROF_CLASSES];
 };
 
 namespace {
@@ -42,6 +53,24 @@ int cuda_fail(const char* what) {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 cudaStream_t S(void* s) { return static_cast<cudaStream_t>(s); }
+
+struct Prof {
+  qi_ctx* c;
+  int slot;
+  cudaStream_t st;
+  Prof(qi_ctx* ctx, int cls, cudaStream_t s) : c(ctx), slot(-1), st(s) {
+    if (!c) return;
+    c->launches[cls] += 1;
+    if (c->prof_on && c->prof_used < QI_PROF_MAX_PAIRS) {
+      slot = c->prof_used++;
+      c->prof_cls[slot] = cls;
+      cudaEventRecord(c->prof_ev[2 * slot], st);
+    }
+  }
+  ~Prof() {
+    if (slot >= 0) cudaEventRecord(c->prof_ev[2 * slot + 1], st);
+  }
+};
 
 // Validate a group table against a sequence length; fill the device-side copy.
 int check_groups(const qi_groups* g, int total, qi::GroupTable* out) {
@@ -246,6 +275,7 @@ int run_quant(qi_ctx* ctx, const void* x, bool xbf16, int M, int K, int ldx,
   p.s = s;
   p.zp = zp;
   p.u_bf16 = u_bf16;
+  Prof pr(ctx, QI_KCLASS_QUANT, st);
   if (qi::launch_quant(p, st) != 0) return cuda_fail("quantize launch");
   return QI_OK;
 }
@@ -276,6 +306,7 @@ int run_w8a8(qi_ctx* ctx, const int8_t* qa, const float* sa, const int32_t* zp, 
   p.row0 = row0;
   p.acc_debug = acc_debug;
   p.status = ctx->status;
+  Prof pr(ctx, QI_KCLASS_GEMM_I8, st);
   const int r = qi::launch_gemm(true, epi, qa, w.k, w.q, w.k, p, ctx->num_sms, st);
   if (r == -2) return fail(QI_ERR_CUDA, "cuTensorMapEncodeTiled failed (W8A8 operands)");
   if (r != 0) return cuda_fail("W8A8 GEMM launch");
@@ -297,6 +328,7 @@ int run_bf16_linear(qi_ctx* ctx, const uint16_t* a, int M, int lda, const qi_lin
   p.dt = dt;
   p.v_out = v_out;
   p.status = ctx->status;
+  Prof pr(ctx, QI_KCLASS_GEMM_BF16, st);
   const int r = qi::launch_gemm(false, epi, a, lda, w.w, w.k, p, ctx->num_sms, st);
   if (r == -2) return fail(QI_ERR_CUDA, "cuTensorMapEncodeTiled failed (BF16 operands)");
   if (r != 0) return cuda_fail("BF16 GEMM launch");
@@ -334,7 +366,10 @@ int run_block(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, float* x
   np.k_out = kl + static_cast<size_t>(row0) * H;
   np.v_out = vl + static_cast<size_t>(row0) * H;
   np.ldo = H;
-  if (qi::launch_qk_norm_rope(np, st) != 0) return cuda_fail("qk norm/rope launch");
+  {
+    Prof pr(ctx, QI_KCLASS_QKNORM, st);
+    if (qi::launch_qk_norm_rope(np, st) != 0) return cuda_fail("qk norm/rope launch");
+  }
   qi::AttnParams ap;
   ap.q = b.q;
   ap.k = kl;
@@ -349,7 +384,10 @@ int run_block(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, float* x
   ap.q_offset = row0;
   ap.sm_scale = 1.0f / sqrtf(static_cast<float>(d.head_dim));
   ap.groups = gt;
-  if (qi::launch_attention(ap, st) != 0) return cuda_fail("attention launch");
+  {
+    Prof pr(ctx, QI_KCLASS_ATTN, st);
+    if (qi::launch_attention(ap, st) != 0) return cuda_fail("attention launch");
+  }
   if ((r = run_quant(ctx, b.o, true, T, H, H, nullptr, nullptr, 0, gt, row0, d.eps, b.uq, b.sa,
                      b.zp, nullptr, st)))
     return r;
@@ -391,8 +429,11 @@ int run_time_conditioning(qi_ctx* ctx, const qi_model& m, float sigma, uint16_t*
   const qi_dims& d = m.dims;
   const int H = d.hidden;
   // t = 0 for the conditioning prefix, t = sigma for the target.
-  if (qi::launch_timestep_embedding(0.0f, sigma, b.emb, st) != 0)
-    return cuda_fail("timestep embedding launch");
+  {
+    Prof pr(ctx, QI_KCLASS_OTHER, st);
+    if (qi::launch_timestep_embedding(0.0f, sigma, b.emb, st) != 0)
+      return cuda_fail("timestep embedding launch");
+  }
   qi::GemvParams g;
   memset(&g, 0, sizeof(g));
   g.x = b.emb;
@@ -402,12 +443,18 @@ int run_time_conditioning(qi_ctx* ctx, const qi_model& m, float sigma, uint16_t*
   g.y_bf16 = 0;
   g.n_jobs = 1;
   g.jobs[0] = {m.t1.w, m.t1.bias, b.h1, H, H};
-  if (qi::launch_gemv(g, st) != 0) return cuda_fail("timestep MLP 1 launch");
+  {
+    Prof pr(ctx, QI_KCLASS_GEMV, st);
+    if (qi::launch_gemv(g, st) != 0) return cuda_fail("timestep MLP 1 launch");
+  }
   g.x = b.h1;
   g.k = H;
   g.silu_in = 1;
   g.jobs[0] = {m.t2.w, m.t2.bias, b.temb, H, H};
-  if (qi::launch_gemv(g, st) != 0) return cuda_fail("timestep MLP 2 launch");
+  {
+    Prof pr(ctx, QI_KCLASS_GEMV, st);
+    if (qi::launch_gemv(g, st) != 0) return cuda_fail("timestep MLP 2 launch");
+  }
   g.x = b.temb;
   g.silu_in = 1;
   g.y_bf16 = 1;
@@ -416,7 +463,10 @@ int run_time_conditioning(qi_ctx* ctx, const qi_model& m, float sigma, uint16_t*
     g.jobs[g.n_jobs++] = {m.blocks[l].mod.w, m.blocks[l].mod.bias,
                           block_mod + static_cast<size_t>(l) * 2 * 6 * H, 6 * H, 6 * H};
   g.jobs[g.n_jobs++] = {m.final_mod.w, m.final_mod.bias, final_mod, 2 * H, 2 * H};
-  if (qi::launch_gemv(g, st) != 0) return cuda_fail("adaLN rows launch");
+  {
+    Prof pr(ctx, QI_KCLASS_GEMV, st);
+    if (qi::launch_gemv(g, st) != 0) return cuda_fail("adaLN rows launch");
+  }
   return QI_OK;
 }
 
@@ -461,6 +511,11 @@ int qi_ctx_create(int device, qi_ctx** out) {
   c->device = device;
   c->num_sms = sms;
   c->status = nullptr;
+  c->prof_on = false;
+  c->prof_used = 0;
+  c->prof_ev = nullptr;
+  c->prof_cls = nullptr;
+  for (int i = 0; i < QI_PROF_CLASSES; ++i) c->launches[i] = 0;
   if (cudaMalloc(&c->status, 256) != cudaSuccess) {
     delete c;
     return cuda_fail("cudaMalloc(status)");
@@ -476,6 +531,11 @@ int qi_ctx_create(int device, qi_ctx** out) {
 
 int qi_ctx_destroy(qi_ctx* ctx) {
   if (!ctx) return QI_OK;
+  if (ctx->prof_ev) {
+    for (int i = 0; i < 2 * QI_PROF_MAX_PAIRS; ++i) cudaEventDestroy(ctx->prof_ev[i]);
+    delete[] ctx->prof_ev;
+    delete[] ctx->prof_cls;
+  }
   cudaFree(ctx->status);
   delete ctx;
   return QI_OK;
@@ -759,6 +819,7 @@ int qi_denoise_step(qi_ctx* ctx, const qi_model* model, float* latents, const ui
                              nullptr, st)))
       return r;
     if (R_ref > 0) {
+      Prof pr(ctx, QI_KCLASS_OTHER, st);
       if (qi::launch_f32_to_bf16(ref_latents, b.lat_bf16, static_cast<int64_t>(R_ref) * P, st))
         return cuda_fail("cast launch");
       if ((r = run_bf16_linear(ctx, b.lat_bf16, R_ref, P, model->img_in, qi::EPI_F32,
@@ -767,8 +828,11 @@ int qi_denoise_step(qi_ctx* ctx, const qi_model* model, float* latents, const ui
     }
   }
   uint16_t* lat_t = b.lat_bf16 + static_cast<size_t>(R_ref > 0 ? R_ref : 0) * P;
-  if (qi::launch_f32_to_bf16(latents, lat_t, static_cast<int64_t>(N) * P, st))
-    return cuda_fail("cast launch");
+  {
+    Prof pr(ctx, QI_KCLASS_OTHER, st);
+    if (qi::launch_f32_to_bf16(latents, lat_t, static_cast<int64_t>(N) * P, st))
+      return cuda_fail("cast launch");
+  }
   float* x_tgt = x + static_cast<size_t>(P_tok - row0) * H;
   if ((r = run_bf16_linear(ctx, lat_t, N, P, model->img_in, qi::EPI_F32, x_tgt, H, 0.f, nullptr,
                            st)))
@@ -863,6 +927,41 @@ int qi_sigma_schedule(int steps, int image_tokens, float* sigmas) {
     sigmas[i] = static_cast<float>(stretch > 0 ? 1.0 - one_minus[i] / stretch : 1.0);
   sigmas[steps] = 0.0f;
   delete[] one_minus;
+  return QI_OK;
+}
+
+int qi_ctx_profile(qi_ctx* ctx, int enable) {
+  if (!ctx) return fail(QI_ERR_INVALID_ARG, "ctx is NULL");
+  if (enable && !ctx->prof_ev) {
+    ctx->prof_ev = new cudaEvent_t[2 * QI_PROF_MAX_PAIRS];
+    ctx->prof_cls = new int[QI_PROF_MAX_PAIRS];
+    for (int i = 0; i < 2 * QI_PROF_MAX_PAIRS; ++i)
+      if (cudaEventCreate(&ctx->prof_ev[i]) != cudaSuccess) return cuda_fail("cudaEventCreate");
+  }
+  ctx->prof_on = enable != 0;
+  ctx->prof_used = 0;
+  for (int i = 0; i < QI_PROF_CLASSES; ++i) ctx->launches[i] = 0;
+  return QI_OK;
+}
+
+int qi_ctx_profile_read(qi_ctx* ctx, int kernel_class, long long* launches, int* timed,
+                        double* total_ms) {
+  if (!ctx || kernel_class < 0 || kernel_class >= QI_PROF_CLASSES || !launches || !timed ||
+      !total_ms)
+    return fail(QI_ERR_INVALID_ARG, "bad arguments");
+  *launches = ctx->launches[kernel_class];
+  *timed = 0;
+  *total_ms = 0.0;
+  for (int i = 0; i < ctx->prof_used; ++i) {
+    if (ctx->prof_cls[i] != kernel_class) continue;
+    if (cudaEventSynchronize(ctx->prof_ev[2 * i + 1]) != cudaSuccess)
+      return cuda_fail("cudaEventSynchronize");
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, ctx->prof_ev[2 * i], ctx->prof_ev[2 * i + 1]) != cudaSuccess)
+      return cuda_fail("cudaEventElapsedTime");
+    *total_ms += ms;
+    *timed += 1;
+  }
   return QI_OK;
 }
 

@@ -121,7 +121,12 @@ _SIGS = {
                        C.POINTER(C.c_int32), C.POINTER(C.c_int32), C.c_void_p, C.c_void_p],
     "qi_sigma_schedule": [C.c_int, C.c_int, C.c_void_p],
     "qi_debug_timeout_probe": [C.c_void_p, C.c_uint64, C.c_void_p],
+    "qi_ctx_profile": [C.c_void_p, C.c_int],
+    "qi_ctx_profile_read": [C.c_void_p, C.c_int, C.POINTER(C.c_longlong), C.POINTER(C.c_int),
+                            C.POINTER(C.c_double)],
 }
+
+KERNEL_CLASSES = ("gemm_i8", "gemm_bf16", "attention", "quant", "qk_norm_rope", "gemv", "other")
 
 EXPORTED = tuple(_SIGS)
 
@@ -195,6 +200,19 @@ class Context:
 
     def check(self, stream=None):
         check(lib().qi_ctx_check(self.handle, stream_ptr(stream)))
+
+    def profile(self, enable: bool):
+        """Reset launch counters; time every launch with CUDA events if enable."""
+        check(lib().qi_ctx_profile(self.handle, 1 if enable else 0))
+
+    def profile_read(self) -> dict:
+        """{class: (launches, timed launches, total ms)} since the last profile() call."""
+        out = {}
+        for i, name in enumerate(KERNEL_CLASSES):
+            n, t, ms = C.c_longlong(), C.c_int(), C.c_double()
+            check(lib().qi_ctx_profile_read(self.handle, i, C.byref(n), C.byref(t), C.byref(ms)))
+            out[name] = (n.value, t.value, ms.value)
+        return out
 
     def close(self):
         if self.handle:

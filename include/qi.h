@@ -163,6 +163,29 @@ int qi_ctx_check(qi_ctx* ctx, void* stream);
 /* Copy the calling thread's last error text into buf (NUL-terminated). */
 int qi_last_error(char* buf, size_t n);
 
+/* Kernel classes counted (and optionally timed) per context. */
+typedef enum {
+  QI_KCLASS_GEMM_I8 = 0,    /* tcgen05 kind::i8 W8A8 GEMMs */
+  QI_KCLASS_GEMM_BF16 = 1,  /* tcgen05 kind::f16 BF16 GEMMs */
+  QI_KCLASS_ATTN = 2,       /* block-causal attention */
+  QI_KCLASS_QUANT = 3,      /* LayerNorm/modulate/int8 quantization */
+  QI_KCLASS_QKNORM = 4,     /* Q/K RMSNorm + RoPE */
+  QI_KCLASS_GEMV = 5,       /* timestep MLP / adaLN rows */
+  QI_KCLASS_OTHER = 6       /* embeddings, casts */
+} qi_kernel_class;
+
+/* Reset the per-class launch counters and switch per-launch timing on or off.
+ * When on, every launch is bracketed by two CUDA events recorded on its
+ * stream (at most 16384 launches are timed until the next reset).  The first
+ * call with enable != 0 creates the events (host-side, not in a compute call). */
+int qi_ctx_profile(qi_ctx* ctx, int enable);
+
+/* Launches of `kernel_class` since the last qi_ctx_profile() call, how many of
+ * them were timed, and their summed device duration in milliseconds (waits for
+ * the recorded events). */
+int qi_ctx_profile_read(qi_ctx* ctx, int kernel_class, long long* launches, int* timed,
+                        double* total_ms);
+
 /* ------------------------------------------------------------------ W8A8 ([W8]) */
 
 /* Quantize fp32 weights w [n, k] symmetrically per output channel:
