@@ -7,6 +7,7 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <mutex>
 #include <string>
 
 #include "qi.h"
@@ -492,6 +493,40 @@ int check_model(const qi_model* m) {
 
 }  // namespace
 
+// ================================================================= fixed scratch
+
+// Scratch for qi_dit_block_forward_noalloc: a fixed array inside the library,
+// so that callers which may not allocate device memory can still run a block.
+// Every GPU that loads the library holds these bytes until the process exits.
+#define QI_NOALLOC_SCRATCH_BYTES (16u << 20)
+static __device__ __align__(256) uint8_t qi_noalloc_scratch[QI_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int QI_NOALLOC_MAX_DEVICES = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[QI_NOALLOC_MAX_DEVICES] = {};
+
+// Device address of the scratch array on the current device.  The array's
+// name is only a host-side stand-in, so the address is looked up once per
+// device (with that device current) and cached.
+int noalloc_scratch(int device, void** out) {
+  if (device < 0 || device >= QI_NOALLOC_MAX_DEVICES)
+    return fail(QI_ERR_INVALID_ARG, "device %d outside 0..%d", device, QI_NOALLOC_MAX_DEVICES - 1);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_addr[device]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, qi_noalloc_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(QI_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
+    g_noalloc_addr[device] = p;
+  }
+  *out = g_noalloc_addr[device];
+  return QI_OK;
+}
+
+}  // namespace
+
 // ================================================================= C ABI
 
 extern "C" {
@@ -739,6 +774,35 @@ int qi_dit_block_forward(qi_ctx* ctx, const qi_dims* dims, const qi_block_weight
                 block_bytes(*dims, T));
   return run_block(ctx, *dims, *w, x, T, row0, mod, gt, S_total, rope_cos, rope_sin, k_layer,
                    v_layer, static_cast<uint8_t*>(workspace), workspace_bytes, S(stream));
+}
+
+int qi_dit_block_forward_noalloc(qi_ctx* ctx, const qi_dims* dims, const qi_block_weights* w,
+                                 float* x, int T, int row0, const uint16_t* mod,
+                                 const qi_groups* groups, const float* rope_cos,
+                                 const float* rope_sin, uint16_t* k_layer, uint16_t* v_layer,
+                                 int kv_mode, void* stream) {
+  if (!ctx) return fail(QI_ERR_INVALID_ARG, "ctx is NULL");
+  int r;
+  if ((r = check_dims(dims))) return r;
+  if (T < 1) return fail(QI_ERR_INVALID_ARG, "T must be >= 1");
+  const size_t need = block_bytes(*dims, T);
+  if (need > QI_NOALLOC_SCRATCH_BYTES)
+    return fail(QI_ERR_WORKSPACE,
+                "qi_dit_block_forward_noalloc: %d rows at hidden %d / mlp %d need %zu scratch "
+                "bytes, more than the library's fixed %u; use qi_dit_block_forward with a "
+                "caller-owned workspace",
+                T, dims->hidden, dims->mlp, need, QI_NOALLOC_SCRATCH_BYTES);
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess) return cuda_fail("cudaGetDevice");
+  if (cur != ctx->device)
+    return fail(QI_ERR_INVALID_ARG, "the current device (%d) is not the context's device (%d)",
+                cur, ctx->device);
+  void* scratch = nullptr;
+  if ((r = noalloc_scratch(cur, &scratch))) return r;
+  // Every region of the block's scratch is written before it is read, so
+  // nothing has to be cleared between calls.
+  return qi_dit_block_forward(ctx, dims, w, x, T, row0, mod, groups, rope_cos, rope_sin, k_layer,
+                              v_layer, kv_mode, scratch, QI_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 int qi_step_workspace_bytes(const qi_dims* dims, int S_tokens, size_t* bytes) {

@@ -108,6 +108,10 @@ _SIGS = {
                              C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.POINTER(qi_groups),
                              C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int,
                              C.c_void_p, C.c_size_t, C.c_void_p],
+    "qi_dit_block_forward_noalloc": [C.c_void_p, C.POINTER(qi_dims), C.POINTER(qi_block_weights),
+                                     C.c_void_p, C.c_int, C.c_int, C.c_void_p,
+                                     C.POINTER(qi_groups), C.c_void_p, C.c_void_p, C.c_void_p,
+                                     C.c_void_p, C.c_int, C.c_void_p],
     "qi_time_conditioning": [C.c_void_p, C.POINTER(qi_model), C.c_float, C.c_void_p, C.c_void_p,
                              C.c_void_p, C.c_size_t, C.c_void_p],
     "qi_step_workspace_bytes": [C.POINTER(qi_dims), C.c_int, C.POINTER(C.c_size_t)],
@@ -338,6 +342,17 @@ def qi_dit_block_forward(ctx: Context, dims: qi_dims, bw: qi_block_weights, x, r
                                      ptr(mod), C.byref(groups), ptr(cos), ptr(sin), ptr(k_layer),
                                      ptr(v_layer), kv_mode, ptr(workspace), workspace.numel(),
                                      stream_ptr(stream)))
+
+
+def qi_dit_block_forward_noalloc(ctx: Context, dims: qi_dims, bw: qi_block_weights, x, row0, mod,
+                                 groups: qi_groups, cos, sin, k_layer, v_layer, kv_mode,
+                                 stream=None):
+    """qi_dit_block_forward without a workspace: the library's fixed scratch is used."""
+    T = x.shape[0]
+    check(lib().qi_dit_block_forward_noalloc(ctx.handle, C.byref(dims), C.byref(bw), ptr(x), T,
+                                             row0, ptr(mod), C.byref(groups), ptr(cos), ptr(sin),
+                                             ptr(k_layer), ptr(v_layer), kv_mode,
+                                             stream_ptr(stream)))
 
 
 def qi_time_conditioning(ctx: Context, model: "Model", sigma: float, block_mod, final_mod,

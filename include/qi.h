@@ -271,6 +271,31 @@ int qi_dit_block_forward(qi_ctx* ctx, const qi_dims* dims, const qi_block_weight
                          uint16_t* v_layer, int kv_mode, void* workspace,
                          size_t workspace_bytes, void* stream);
 
+/* Same block as qi_dit_block_forward, for callers that cannot allocate device
+ * memory: a program that only receives input and output buffers from its host
+ * framework, or one that runs under a fixed device-memory budget and must not
+ * grow it at an unpredictable moment.  It takes no workspace argument and calls
+ * no cudaMalloc, cudaFree or other allocating routine; its scratch is a fixed
+ * 16 MiB array inside the library (every GPU that loads the library holds it
+ * until the process exits).  The pages describe no such call; it has no
+ * counterpart there.
+ *   - Sizes whose scratch (qi_block_workspace_bytes) exceeds 16 MiB are rejected
+ *     with QI_ERR_WORKSPACE before anything is launched (at hidden 256 / mlp
+ *     1024 up to 2,974 rows fit; at hidden 4096 / mlp 16384 up to 186 rows).
+ *   - The first call on a device looks up the array's device address (once,
+ *     with that device current; the current device must be the context's).
+ *     Make that first call before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents;
+ *     every region is written before it is read, so nothing needs clearing.
+ *     Calls whose kernels overlap on the GPU (different streams, or several
+ *     host threads) race on it: serialize them.
+ * Arguments and results are those of qi_dit_block_forward. */
+int qi_dit_block_forward_noalloc(qi_ctx* ctx, const qi_dims* dims, const qi_block_weights* w,
+                                 float* x, int T, int row0, const uint16_t* mod,
+                                 const qi_groups* groups, const float* rope_cos,
+                                 const float* rope_sin, uint16_t* k_layer, uint16_t* v_layer,
+                                 int kv_mode, void* stream);
+
 /* ------------------------------------------------------------------ step */
 
 /* Timestep conditioning of a step: temb_r = t2(SiLU(t1(sinusoid(1000 t_r))))
