@@ -9,7 +9,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libqi.so")
-SOURCES = ["qi_api.cu", "qi_gemm.cu", "qi_quant.cu", "qi_misc.cu", "qi_attn.cu"]
+SOURCES = ["qi_api.cu", "qi_gemm.cu", "qi_quant.cu", "qi_misc.cu", "qi_attn_tc.cu"]
 HEADERS = ["qi_common.cuh", "qi_internal.h"]
 
 

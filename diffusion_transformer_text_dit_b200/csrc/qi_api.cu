@@ -385,9 +385,12 @@ int run_block(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, float* x
   ap.q_offset = row0;
   ap.sm_scale = 1.0f / sqrtf(static_cast<float>(d.head_dim));
   ap.groups = gt;
+  ap.status = ctx->status;
   {
     Prof pr(ctx, QI_KCLASS_ATTN, st);
-    if (qi::launch_attention(ap, st) != 0) return cuda_fail("attention launch");
+    const int r2 = qi::launch_attention(ap, st);
+    if (r2 == -2) return fail(QI_ERR_CUDA, "cuTensorMapEncodeTiled failed (attention operands)");
+    if (r2 != 0) return cuda_fail("attention launch");
   }
   if ((r = run_quant(ctx, b.o, true, T, H, H, nullptr, nullptr, 0, gt, row0, d.eps, b.uq, b.sa,
                      b.zp, nullptr, st)))
@@ -730,7 +733,13 @@ int qi_attn_block_causal(qi_ctx* ctx, const uint16_t* q, int ldq, int Sq, int q_
   p.q_offset = q_offset;
   p.sm_scale = sm_scale;
   p.groups = gt;
-  if (qi::launch_attention(p, S(stream)) != 0) return cuda_fail("attention launch");
+  p.status = ctx->status;
+  {
+    Prof pr(ctx, QI_KCLASS_ATTN, S(stream));
+    const int r2 = qi::launch_attention(p, S(stream));
+    if (r2 == -2) return fail(QI_ERR_CUDA, "cuTensorMapEncodeTiled failed (attention operands)");
+    if (r2 != 0) return cuda_fail("attention launch");
+  }
   return QI_OK;
 }
 

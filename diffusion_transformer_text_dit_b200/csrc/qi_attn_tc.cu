@@ -1,0 +1,379 @@
+// Block-causal flash attention on tcgen05 tensor cores (sm_100a), head_dim 128,
+// bf16 in / bf16 out, fp32 softmax.
+//
+// Mask (RGBA-Image-2.1 Core AI port: "block-causal attention"; qwen-image-mnn:
+// "block-causal mask"): the joint sequence is a list of contiguous groups
+// [text | (reference) | target]; a token sees every token of its own group and
+// of all earlier groups, so the keys of a query at global position t are
+// exactly [0, end(group(t))) - a per-query key limit.  Key tiles at or past the
+// largest limit of the CTA's queries are never loaded; tiles entirely below
+// the smallest limit are not masked.  Queries may be a suffix of the sequence
+// (q_offset > 0: the cached-prefix step processes only the target rows while
+// keys/values cover the whole sequence).
+//
+// One CTA = one head x 256 queries, as two 128-row tiles A and B that share
+// the key/value stream.  TMEM (512 columns): S_A | S_B | O_A | O_B, 128 fp32
+// columns each.  Per key tile j of 128 keys:
+//   S_X = Q_X K_j^T         tcgen05.mma kind::f16, A = Q (smem), B = K (smem), both K-major
+//   softmax warps of X read S_X (one query row per thread), write P_X as bf16
+//   into the first 64 columns of S_X
+//   O_X += P_X V_j          tcgen05.mma with A = P from TMEM, B = V (smem, MN-major)
+// Issue order (one thread): S_A0 S_B0 | PV_A(j) S_A(j+1) PV_B(j) S_B(j+1) ...
+// so each tile's softmax overlaps the other tile's MMAs.  The softmax keeps a
+// per-row reference maximum and rescales O (TMEM load / store) only when the
+// running maximum exceeds it by more than 8 (base 2): P <= 256 in between,
+// exact in value because the final normalisation divides by the same sum.
+//
+// Warps: 0-3 softmax of tile A (TMEM lanes 0-127), 4-7 softmax of tile B,
+// 8 TMA producer, 9 TMEM allocator + MMA issuer.  K/V stream through a 2-stage
+// ring; every barrier wait is bounded (qi_common.cuh).
+#include "qi_common.cuh"
+#include "qi_internal.h"
+
+namespace qi {
+
+constexpr int FA_ROWS = 128;                   // rows per Q tile, keys per K/V tile
+constexpr int FA_THREADS = 320;
+constexpr int FA_TILE = 128 * 128 * 2;         // 32 KB: 128 rows x 128 bf16
+constexpr int FA_HALF = FA_TILE / 2;           // one 64-column (128-byte) swizzle region
+constexpr int FA_SMEM = 1024 + 6 * FA_TILE + 256;
+
+// MN-major operand with the 128-byte swizzle: 64 elements (128 B) contiguous
+// along N, K rows 128 B apart inside an 8-row group, 8-row groups 1024 B
+// apart (stride offset), 64-element column blocks lbo_bytes apart (leading
+// offset).
+__device__ __forceinline__ uint64_t umma_desc_mnmajor_sw128(uint32_t saddr, uint32_t lbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>(1024u >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(2u) << 61;
+  return d;
+}
+
+// D (TMEM) += A (TMEM, K-major) x B (smem descriptor), kind::f16.
+__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ int fa_key_limit(const GroupTable& g, int t) {
+  return g.end[group_of(g, t)];
+}
+
+__global__ void __launch_bounds__(FA_THREADS, 1)
+    fa_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+              const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+  int* status = p.status;
+  extern __shared__ uint8_t fa_smem_raw[];
+  const uint32_t raw_addr = smem_u32(fa_smem_raw);
+  uint8_t* smem = fa_smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  uint8_t* sQ = smem;                      // [2][FA_TILE]: tile A, tile B
+  uint8_t* sK = smem + 2 * FA_TILE;        // [2 stages][FA_TILE]
+  uint8_t* sV = smem + 4 * FA_TILE;        // [2 stages][FA_TILE]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 6 * FA_TILE);
+  uint64_t* q_full = bars + 0;
+  uint64_t* k_full = bars + 1;      // [2]
+  uint64_t* v_full = bars + 3;      // [2]
+  uint64_t* kv_empty = bars + 5;    // [2]
+  uint64_t* s_full = bars + 7;      // [2] per Q tile
+  uint64_t* p_full = bars + 9;      // [2] per Q tile
+  uint64_t* o_full = bars + 11;
+  uint64_t* drain = bars + 12;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_ctiles = (p.Sq + 2 * FA_ROWS - 1) / (2 * FA_ROWS);
+  const int ct = n_ctiles - 1 - static_cast<int>(blockIdx.x);   // heavy tiles first
+  const int h = blockIdx.y;
+  const int q0 = ct * 2 * FA_ROWS;
+  const int q_last = min(q0 + 2 * FA_ROWS, p.Sq) - 1;
+  const int kv_end = min(fa_key_limit(p.groups, p.q_offset + q_last), p.Sk);
+  const int kv_min = min(fa_key_limit(p.groups, p.q_offset + q0), p.Sk);
+  const int n_kv = (kv_end + FA_ROWS - 1) / FA_ROWS;
+  const int hc = h * 128;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&p_full[s], 128);
+    }
+    mbar_init(o_full, 1);
+    mbar_init(drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 8 && lane == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+  }
+  if (warp == 9) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(q_full, 2 * FA_TILE);
+      for (int t = 0; t < 2; ++t)
+        for (int half = 0; half < 2; ++half)
+          tma_load_2d(&tmQ, q_full, sQ + t * FA_TILE + half * FA_HALF, hc + 64 * half,
+                      q0 + t * FA_ROWS);
+      bool ok = true;
+      int j = 0;
+      for (; j < n_kv; ++j) {
+        const int st = j & 1;
+        if (!mbar_wait(&kv_empty[st], ((j >> 1) & 1) ^ 1u, status)) { ok = false; break; }
+        mbar_arrive_expect_tx(&k_full[st], FA_TILE);
+        for (int half = 0; half < 2; ++half)
+          tma_load_2d(&tmK, &k_full[st], sK + st * FA_TILE + half * FA_HALF, hc + 64 * half,
+                      j * FA_ROWS);
+        mbar_arrive_expect_tx(&v_full[st], FA_TILE);
+        for (int half = 0; half < 2; ++half)
+          tma_load_2d(&tmV, &v_full[st], sV + st * FA_TILE + half * FA_HALF, hc + 64 * half,
+                      j * FA_ROWS);
+      }
+      if (!ok) {
+        // bounded drain of the loads already armed (Q and the last two K/V tiles)
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(q_full, 0) && globaltimer_ns() - t0 < QI_WAIT_NS) {
+        }
+        for (int jj = j - 2; jj < j; ++jj) {
+          if (jj < 0) continue;
+          const int st = jj & 1;
+          const uint32_t par = (jj >> 1) & 1;
+          const uint64_t t1 = globaltimer_ns();
+          while (!(mbar_try_wait(&k_full[st], par) && mbar_try_wait(&v_full[st], par)) &&
+                 globaltimer_ns() - t1 < QI_WAIT_NS) {
+          }
+        }
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = umma_idesc(false, 128, 128);
+      constexpr uint32_t idesc_pv = umma_idesc(false, 128, 128) | (1u << 16);   // B MN-major
+      bool ok = mbar_wait(q_full, 0, status);
+      auto issue_s = [&](int X, int jj) -> bool {
+        const int st = jj & 1;
+        if (!mbar_wait(&k_full[st], (jj >> 1) & 1, status)) return false;
+        tc_fence_after();
+        const uint32_t qa = smem_u32(sQ + X * FA_TILE), kb = smem_u32(sK + st * FA_TILE);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * FA_HALF + (kk & 3) * 32;
+          umma_f16(tmem_base + X * 128, umma_desc_kmajor_sw128(qa + off),
+                   umma_desc_kmajor_sw128(kb + off), idesc_s, kk > 0);
+        }
+        umma_commit(&s_full[X]);
+        return true;
+      };
+      auto issue_pv = [&](int X, int jj) -> bool {
+        const int st = jj & 1;
+        if (!mbar_wait(&v_full[st], (jj >> 1) & 1, status)) return false;
+        if (!mbar_wait(&p_full[X], jj & 1, status)) return false;
+        tc_fence_after();
+        const uint32_t vb = smem_u32(sV + st * FA_TILE);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)   // 16 keys per instruction: two 8-row groups
+          umma_f16_ts(tmem_base + 256 + X * 128, tmem_base + X * 128 + kk * 8,
+                      umma_desc_mnmajor_sw128(vb + kk * 2048, FA_HALF), idesc_pv,
+                      (jj > 0 || kk > 0) ? 1u : 0u);
+        return true;
+      };
+      if (ok && n_kv > 0) ok = issue_s(0, 0) && issue_s(1, 0);
+      for (int j = 0; ok && j < n_kv; ++j) {
+        ok = issue_pv(0, j);
+        if (ok && j + 1 < n_kv) ok = issue_s(0, j + 1);
+        if (ok) ok = issue_pv(1, j);
+        if (ok) umma_commit(&kv_empty[j & 1]);
+        if (ok && j + 1 < n_kv) ok = issue_s(1, j + 1);
+      }
+      if (ok) {
+        umma_commit(o_full);
+      } else {
+        umma_commit(drain);
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < QI_WAIT_NS) {
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int X = warp >> 2;
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_bits = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem_base + lane_bits + X * 128;
+    const uint32_t tO = tmem_base + lane_bits + 256 + X * 128;
+    const int qrow = q0 + X * FA_ROWS + row;
+    const int lim = qrow < p.Sq ? min(fa_key_limit(p.groups, p.q_offset + qrow), p.Sk) : p.Sk;
+    const float sl2 = p.sm_scale * 1.4426950408889634f;
+    float m_ref = -INFINITY;   // reference maximum, base-2 scaled
+    float l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_kv; ++j) {
+      if (!mbar_wait_warp(&s_full[X], j & 1, status)) { ok = false; break; }
+      tc_fence_after();
+      const int k0 = j * FA_ROWS;
+      const bool masked = k0 + FA_ROWS > kv_min;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tS + c * 32, r);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          float s = __uint_as_float(r[i]);
+          if (masked && k0 + c * 32 + i >= lim) s = -INFINITY;
+          mx = fmaxf(mx, s);
+        }
+      }
+      const float mx2 = mx * sl2;
+      // New reference maximum for this row if it grew by more than 8 (base 2).
+      const bool grow = (j == 0) || (mx2 > m_ref + 8.0f);
+      float f = 1.0f;
+      if (grow) {
+        const float m_new = fmaxf(m_ref, mx2);
+        if (j > 0) f = exp2f(m_ref - m_new);
+        l *= f;
+        m_ref = m_new;
+      }
+      // The O rescale uses warp-collective TMEM loads/stores, so the decision
+      // is taken per warp: if any row of the warp moved its reference, the
+      // whole warp rescales (factor 1 for the rows that did not).  O is
+      // complete up to tile j-1: the commit that released S_X(j) covers every
+      // earlier MMA.
+      if (__any_sync(0xffffffffu, grow && j > 0)) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tO + c * 32, r);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * f);
+          tmem_st32(tO + c * 32, r);
+        }
+        tmem_st_wait();
+      }
+      float sum = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tS + c * 32, r);
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float s0 = __uint_as_float(r[2 * i]), s1 = __uint_as_float(r[2 * i + 1]);
+          float p0 = exp2f(fmaf(s0, sl2, -m_ref));
+          float p1 = exp2f(fmaf(s1, sl2, -m_ref));
+          if (masked) {
+            if (k0 + c * 32 + 2 * i >= lim) p0 = 0.f;
+            if (k0 + c * 32 + 2 * i + 1 >= lim) p1 = 0.f;
+          }
+          sum += p0 + p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(tS + c * 16, pk);   // P overwrites S columns already read
+      }
+      l += sum;
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&p_full[X]);
+    }
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok && n_kv > 0 && mbar_wait_warp(o_full, 0, status)) {
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.0f / l : 0.f;
+      // every lane of the warp takes part in the (warp-wide) TMEM loads
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tO + c * 32, r);
+        if (qrow < p.Sq) {
+          uint4* dst = reinterpret_cast<uint4*>(p.o + static_cast<int64_t>(qrow) * p.ldo + hc + c * 32);
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            dst[v] = make_uint4(
+                pack_bf16x2(__uint_as_float(r[8 * v + 0]) * inv, __uint_as_float(r[8 * v + 1]) * inv),
+                pack_bf16x2(__uint_as_float(r[8 * v + 2]) * inv, __uint_as_float(r[8 * v + 3]) * inv),
+                pack_bf16x2(__uint_as_float(r[8 * v + 4]) * inv, __uint_as_float(r[8 * v + 5]) * inv),
+                pack_bf16x2(__uint_as_float(r[8 * v + 6]) * inv, __uint_as_float(r[8 * v + 7]) * inv));
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+int launch_attention(const AttnParams& p, cudaStream_t st) {
+  if (p.Sq == 0) return 0;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(fa_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, FA_SMEM) !=
+        cudaSuccess)
+      return -1;
+    attr = true;
+  }
+  const int W = p.heads * 128;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap_2d(&tq, p.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, p.Sq,
+                    static_cast<uint64_t>(p.ldq) * 2, 64, FA_ROWS) ||
+      !make_tmap_2d(&tk, p.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, p.Sk,
+                    static_cast<uint64_t>(p.ldkv) * 2, 64, FA_ROWS) ||
+      !make_tmap_2d(&tv, p.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, p.Sk,
+                    static_cast<uint64_t>(p.ldkv) * 2, 64, FA_ROWS))
+    return -2;
+  dim3 grid((p.Sq + 2 * FA_ROWS - 1) / (2 * FA_ROWS), p.heads);
+  fa_kernel<<<grid, FA_THREADS, FA_SMEM, st>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+}  // namespace qi

@@ -92,6 +92,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
   }
 }
 
+// Warp-uniform form of mbar_wait for code that issues warp-collective
+// (.sync.aligned) tcgen05 instructions after the wait: every lane of the warp
+// returns the same answer, so no lane can leave while the others go on to a
+// collective instruction.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, int* status) {
+  const bool ok = mbar_wait(bar, parity, status);
+  return __all_sync(0xffffffffu, ok);
+}
+
 // ---------------------------------------------------------------- TMA
 
 // 2-D tiled bulk tensor load into shared memory, completing on `bar`.

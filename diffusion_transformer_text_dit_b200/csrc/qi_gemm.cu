@@ -175,7 +175,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       const int m0 = (tile % m_tiles) * GEMM_BM;
       const int n0 = (tile / m_tiles) * BN;
-      if (!mbar_wait(&tfull[acc], acc_phase, p.status)) break;
+      if (!mbar_wait_warp(&tfull[acc], acc_phase, p.status)) break;
       tc_fence_after();
       const int m = m0 + row_in_tile;
       const bool row_ok = m < p.M;

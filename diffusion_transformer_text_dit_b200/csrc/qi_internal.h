@@ -102,6 +102,7 @@ struct AttnParams {
   int Sq, Sk, heads, q_offset;
   float sm_scale;
   GroupTable groups;
+  int* status;            // device status word
 };
 int launch_attention(const AttnParams& p, cudaStream_t st);
 

@@ -258,7 +258,7 @@ def _attn_case(sizes, heads, seed):
     q = _bf16((S, heads * 128), seed, 1.0)
     k = _bf16((S, heads * 128), seed + 1, 1.0)
     v = _bf16((S, heads * 128), seed + 2, 1.0)
-    ends = list(np.cumsum(sizes))
+    ends = [int(e) for e in np.cumsum(sizes)]
     return q, k, v, ends
 
 
@@ -349,3 +349,20 @@ def test_timeout_probe_reports_and_context_survives(ctx):
     x = torch.randn(4, 256, device="cuda")
     qi.qi_quantize_act(ctx, x)
     ctx.check()
+
+
+def test_attention_growing_scores_rescale_path(ctx):
+    # later keys are scaled up so each key tile's row maximum exceeds the
+    # previous one by a wide margin: the running-maximum rescale of O is taken,
+    # in some lanes of a warp and not in others
+    sizes = [128, 640]
+    heads = 2
+    q, k, v, ends = _attn_case(sizes, heads, 91)
+    S = sum(sizes)
+    ramp = torch.linspace(0.5, 6.0, S).reshape(S, 1)
+    k = (k.float() * ramp).to(torch.bfloat16)
+    g = qi.groups_struct(ends, [0, 1])
+    o = qi.qi_attn_block_causal(ctx, cuda(q), cuda(k), cuda(v), g)
+    ctx.check()
+    ref = _oracle_attn(q, k, v, ends, heads)
+    assert rel_l2(bf16_np(o), ref) < 4e-3
