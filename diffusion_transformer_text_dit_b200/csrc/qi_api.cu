@@ -349,27 +349,36 @@ int run_block(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, float* x
   if ((r = run_quant(ctx, x, false, T, H, H, mod + 0 * H, mod + 1 * H, mld, gt, row0, d.eps,
                      b.uq, b.sa, b.zp, nullptr, st)))
     return r;
-  if ((r = run_w8a8(ctx, b.uq, b.sa, b.zp, T, w.qkv, qi::EPI_BF16, b.qkv, 3 * H, nullptr, 0,
-                    nullptr, 0, gt, row0, nullptr, st)))
-    return r;
-  qi::QkNormRopeParams np;
-  np.qkv = b.qkv;
-  np.ldqkv = 3 * H;
-  np.T = T;
-  np.heads = d.heads;
-  np.d = d.head_dim;
-  np.wq = w.norm_q;
-  np.wk = w.norm_k;
-  np.cos = cs;
-  np.sin = sn;
-  np.eps = d.eps;
-  np.q_out = b.q;
-  np.k_out = kl + static_cast<size_t>(row0) * H;
-  np.v_out = vl + static_cast<size_t>(row0) * H;
-  np.ldo = H;
+  // QKV projection with Q/K RMSNorm + RoPE fused into its epilogue: q goes to
+  // the block's q buffer, k and v straight into this layer's K/V rows.
   {
-    Prof pr(ctx, QI_KCLASS_QKNORM, st);
-    if (qi::launch_qk_norm_rope(np, st) != 0) return cuda_fail("qk norm/rope launch");
+    qi::GemmParams p;
+    memset(&p, 0, sizeof(p));
+    p.M = T;
+    p.N = w.qkv.n;
+    p.K = w.qkv.k;
+    p.num_kb = w.qkv.k / 128;
+    p.s_a = b.sa;
+    p.zp_a = b.zp;
+    p.s_w = w.qkv.s;
+    p.rowsum = w.qkv.rowsum;
+    p.bias = w.qkv.bias;
+    p.H = H;
+    p.eps = d.eps;
+    p.wq = w.norm_q;
+    p.wk = w.norm_k;
+    p.rcos = cs;
+    p.rsin = sn;
+    p.q_out = b.q;
+    p.k_out = kl + static_cast<size_t>(row0) * H;
+    p.v_out_bf16 = vl + static_cast<size_t>(row0) * H;
+    p.ldo = H;
+    p.status = ctx->status;
+    Prof pr(ctx, QI_KCLASS_GEMM_I8, st);
+    const int rr = qi::launch_gemm(true, qi::EPI_QKV, b.uq, w.qkv.k, w.qkv.q, w.qkv.k, p,
+                                   ctx->num_sms, st);
+    if (rr == -2) return fail(QI_ERR_CUDA, "cuTensorMapEncodeTiled failed (QKV operands)");
+    if (rr != 0) return cuda_fail("QKV GEMM launch");
   }
   qi::AttnParams ap;
   ap.q = b.q;
@@ -652,6 +661,47 @@ int qi_w8a8_linear(qi_ctx* ctx, const int8_t* qa, const float* s_a, const int32_
       return fail(QI_ERR_ALIGNMENT, "y must be 16-byte aligned with ldy %% 8 == 0, ldy >= n");
     return run_w8a8(ctx, qa, s_a, zp_a, M, *w, kind == QI_EPI_STORE ? qi::EPI_BF16 : qi::EPI_GELU,
                     y, ldy, nullptr, 0, nullptr, 0, gt, 0, acc_debug, S(stream));
+  }
+  if (kind == QI_EPI_QKV_NORM_ROPE) {
+    const int H = ep->hidden;
+    if (H < 128 || H % 128 != 0 || w->n != 3 * H)
+      return fail(QI_ERR_UNSUPPORTED_SHAPE, "QKV epilogue: need hidden %% 128 == 0 and n == 3 * hidden");
+    if (!ep->norm_q || !ep->norm_k || !ep->rope_cos || !ep->rope_sin || !ep->q_out ||
+        !ep->k_out || !ep->v_out)
+      return fail(QI_ERR_INVALID_ARG, "QKV epilogue: NULL pointer");
+    if (ep->ld_out < H || ep->ld_out % 8 != 0 || !aligned16(ep->q_out) || !aligned16(ep->k_out) ||
+        !aligned16(ep->v_out) || !aligned16(ep->rope_cos) || !aligned16(ep->rope_sin) ||
+        !aligned16(ep->norm_q) || !aligned16(ep->norm_k))
+      return fail(QI_ERR_ALIGNMENT, "QKV epilogue: pointers must be 16-byte aligned, ld_out %% 8 == 0");
+    if (M == 0) return QI_OK;
+    qi::GemmParams p;
+    memset(&p, 0, sizeof(p));
+    p.M = M;
+    p.N = w->n;
+    p.K = w->k;
+    p.num_kb = w->k / 128;
+    p.s_a = s_a;
+    p.zp_a = zp_a;
+    p.s_w = w->s;
+    p.rowsum = w->rowsum;
+    p.bias = w->bias;
+    p.H = H;
+    p.eps = ep->eps;
+    p.wq = ep->norm_q;
+    p.wk = ep->norm_k;
+    p.rcos = ep->rope_cos;
+    p.rsin = ep->rope_sin;
+    p.q_out = ep->q_out;
+    p.k_out = ep->k_out;
+    p.v_out_bf16 = ep->v_out;
+    p.ldo = ep->ld_out;
+    p.status = ctx->status;
+    Prof pr(ctx, QI_KCLASS_GEMM_I8, S(stream));
+    const int rr = qi::launch_gemm(true, qi::EPI_QKV, qa, w->k, w->q, w->k, p, ctx->num_sms,
+                                   S(stream));
+    if (rr == -2) return fail(QI_ERR_CUDA, "cuTensorMapEncodeTiled failed (QKV operands)");
+    if (rr != 0) return fail(QI_ERR_UNSUPPORTED_SHAPE, "QKV epilogue launch failed (tile/head layout)");
+    return QI_OK;
   }
   if (kind != QI_EPI_GATED_RESIDUAL) return fail(QI_ERR_INVALID_ARG, "bad epilogue kind");
   if (!ep->residual || !ep->gate) return fail(QI_ERR_INVALID_ARG, "residual / gate is NULL");

@@ -9,10 +9,12 @@
 //  * kind::f16 : bf16 x bf16 -> fp32 (the BF16 Linears: in/out projections).
 //      y = acc + bias[n]
 //
-// Warp roles in a 192-thread CTA (one CTA per SM, persistent over tiles):
+// Warp roles in a 320-thread CTA (one CTA per SM, persistent over tiles):
 //   warp 0      TMA producer (one thread)
 //   warp 1      TMEM allocator + MMA issuer (one thread)
-//   warps 2..5  epilogue: warp w reads TMEM lanes 32*(w%4) .. +31
+//   warps 2..9  epilogue: warp w reads TMEM lanes 32*(w%4) .. +31; warps 2-5
+//               take the first half of the tile's columns, warps 6-9 the second
+//               (two warps per SM sub-partition hide the epilogue's latencies)
 // Tiles are 128 x BN; the accumulator is double-buffered in TMEM (2*BN
 // columns) so the epilogue of tile i overlaps the MMAs of tile i+1.
 #include "qi_common.cuh"
@@ -22,7 +24,8 @@ namespace qi {
 
 constexpr int GEMM_BM = 128;
 constexpr int GEMM_BK_BYTES = 128;      // one 128-byte swizzle row per stage
-constexpr int GEMM_THREADS = 192;
+constexpr int GEMM_THREADS = 320;
+constexpr int GEMM_EPI_WARPS = 8;
 
 template <int BN>
 struct GemmCfg {
@@ -39,6 +42,97 @@ __device__ __forceinline__ float gelu_tanh_f(float x) {
   const float k0 = 0.7978845608028654f;   // sqrt(2/pi)
   const float k1 = 0.044715f;
   return 0.5f * x * (1.0f + tanhf(k0 * (x + k1 * x * x * x)));
+}
+
+// W8A8 dequantization of 32 accumulator columns starting at column nb,
+// rounded to bf16 (the Linear's output dtype).
+__device__ __forceinline__ void dequant32_bf16(const GemmParams& p, const uint32_t (&r)[32], int nb,
+                                               float sa, int32_t zp, float (&y)[32]) {
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const int n = nb + j;
+    const float b = p.bias ? bf16_bits_to_float(__ldg(p.bias + n)) : 0.f;
+    const int32_t corr = static_cast<int32_t>(r[j]) - zp * __ldg(p.rowsum + n);
+    y[j] = bf16_round_f(fmaf(static_cast<float>(corr) * sa, __ldg(p.s_w + n), b));
+  }
+}
+
+// Fused epilogue of the QKV projection: the W columns handled by one epilogue
+// warp are W/128 whole heads of q, k or v.  For q and k each head row is read from TMEM
+// twice: once for the sum of squares of its bf16 values, once to apply
+//   r = 1/sqrt(mean + eps), n = bf16(y r), y' = bf16(n w)     (cast before scale)
+//   (a, b) -> (bf16(a c - b s), bf16(a s + b c))              (RoPE, pair = column/2)
+// with explicitly rounded fp32 operations; v is stored as bf16(y).
+template <int W>
+__device__ __forceinline__ void qkv_epilogue(const GemmParams& p, uint32_t t_row, int m,
+                                             bool row_ok, float sa, int32_t zp, int n0, int lane,
+                                             uint64_t* tempty_bar) {
+  const int which = n0 / p.H;
+  const int col0 = n0 - which * p.H;
+  uint16_t* out = which == 0 ? p.q_out : (which == 1 ? p.k_out : p.v_out_bf16);
+  const uint16_t* w = which == 0 ? p.wq : p.wk;
+#pragma unroll 1
+  for (int hh = 0; hh < W / 128; ++hh) {
+    float rs = 1.0f;
+    if (which < 2) {
+      float ss = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld32(t_row + hh * 128 + c * 32, r);
+        if (row_ok) {
+          float y[32];
+          dequant32_bf16(p, r, n0 + hh * 128 + c * 32, sa, zp, y);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) ss = __fadd_rn(ss, __fmul_rn(y[j], y[j]));
+        }
+      }
+      rs = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(ss, 128.0f), p.eps)));
+    }
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      uint32_t r[32];
+      tmem_ld32(t_row + hh * 128 + c * 32, r);
+      if (hh == W / 128 - 1 && c == 3) {   // this warp's last TMEM read of the accumulator
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tempty_bar);
+      }
+      if (!row_ok) continue;
+      float y[32];
+      dequant32_bf16(p, r, n0 + hh * 128 + c * 32, sa, zp, y);
+      uint32_t pk[16];
+      if (which < 2) {
+        const float4* c4 = reinterpret_cast<const float4*>(p.rcos + static_cast<size_t>(m) * 64 + c * 16);
+        const float4* s4 = reinterpret_cast<const float4*>(p.rsin + static_cast<size_t>(m) * 64 + c * 16);
+        const uint4* w4 = reinterpret_cast<const uint4*>(w + c * 32);
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const float4 cc = __ldg(c4 + g), sn = __ldg(s4 + g);
+          const uint4 wv = __ldg(w4 + g);
+          const float cs[4] = {cc.x, cc.y, cc.z, cc.w}, si[4] = {sn.x, sn.y, sn.z, sn.w};
+          const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const int i = 4 * g + t;   // pair index in the chunk
+            const float a = bf16_round_f(__fmul_rn(bf16_round_f(__fmul_rn(y[2 * i], rs)),
+                                                   __uint_as_float(ww[t] << 16)));
+            const float b = bf16_round_f(__fmul_rn(bf16_round_f(__fmul_rn(y[2 * i + 1], rs)),
+                                                   __uint_as_float(ww[t] & 0xFFFF0000u)));
+            pk[i] = pack_bf16x2(__fsub_rn(__fmul_rn(a, cs[t]), __fmul_rn(b, si[t])),
+                                __fadd_rn(__fmul_rn(a, si[t]), __fmul_rn(b, cs[t])));
+          }
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(y[2 * i], y[2 * i + 1]);
+      }
+      uint4* dst = reinterpret_cast<uint4*>(out + static_cast<size_t>(m) * p.ldo + col0 +
+                                            hh * 128 + c * 32);
+#pragma unroll
+      for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+    }
+  }
 }
 
 template <bool I8, int BN, int EPI>
@@ -73,7 +167,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 4);
+      mbar_init(&tempty[a], GEMM_EPI_WARPS);
     }
     mbar_init(drain, 1);
     fence_mbar_init();
@@ -169,6 +263,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;          // 0: warps 2-5, 1: warps 6-9
     const int row_in_tile = quarter * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -191,11 +286,18 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       }
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
+      if constexpr (EPI == EPI_QKV) {
+        qkv_epilogue<BN / 2>(p, t_row + half * (BN / 2), m, row_ok, sa, zp, n0 + half * (BN / 2),
+                             lane, &tempty[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+        continue;
+      }
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = half * (BN / 64); c < (half + 1) * (BN / 64); ++c) {
         uint32_t r[32];
         tmem_ld32(t_row + c * 32, r);
-        if (c == BN / 32 - 1) {
+        if (c == (half + 1) * (BN / 64) - 1) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -364,6 +466,9 @@ int launch_gemm(bool int8, int epi, const void* A, int lda, const void* B, int l
       case EPI_BF16: return launch_gemm_bn<true, EPI_BF16>(bn, ta, tb, p, num_sms, st);
       case EPI_GELU: return launch_gemm_bn<true, EPI_GELU>(bn, ta, tb, p, num_sms, st);
       case EPI_GATED: return launch_gemm_bn<true, EPI_GATED>(bn, ta, tb, p, num_sms, st);
+      case EPI_QKV:   // each epilogue half-tile must hold a whole head of one of q, k, v
+        if (bn == 256 && p.H % 256 == 0) return launch_gemm_t<true, 256, EPI_QKV>(ta, tb, p, num_sms, st);
+        return -1;
     }
   } else {
     switch (epi) {

@@ -16,6 +16,7 @@ enum GemmEpilogue {
   EPI_GATED = 2,   // yf (fp32) += gate[row set] * bf16(value)
   EPI_F32 = 3,     // yf (fp32) = value
   EPI_EULER = 4,   // v = value; yf (fp32 latents) += dt * v
+  EPI_QKV = 5,     // q, k: RMSNorm (cast first) + RoPE of bf16(value); v: bf16(value)
 };
 
 struct GemmParams {
@@ -39,6 +40,17 @@ struct GemmParams {
   int32_t* acc_debug;     // optional raw int32 accumulators [M, N]
   float dt;               // Euler: sigma_next - sigma
   float* v_out;           // Euler: optional velocity [M, ldyf]
+  // fused QKV epilogue (N = 3H; a tile holds whole heads of one of q, k, v)
+  int H;
+  float eps;
+  const uint16_t* wq;     // [128] bf16 RMSNorm scales
+  const uint16_t* wk;
+  const float* rcos;      // [M, 64] tables of the rows of this GEMM
+  const float* rsin;
+  uint16_t* q_out;        // [M, H] rows of this GEMM
+  uint16_t* k_out;
+  uint16_t* v_out_bf16;
+  int ldo;
   int* status;            // device status word
 };
 

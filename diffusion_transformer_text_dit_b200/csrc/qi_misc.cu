@@ -73,11 +73,29 @@ int launch_qk_norm_rope(const QkNormRopeParams& p, cudaStream_t st) {
 
 // y[r][j] = sum_k act(x[r][k]) * W[j][k] + b[j] for every row j of every job.
 // x (R <= 2 rows) is staged in shared memory as fp32 (SiLU applied on load
-// when requested); one warp per output row, 16-byte weight loads.
+// when requested).  One warp handles 4 consecutive weight rows at a time:
+// every lane streams 4 x 16 bytes of weights per step and reuses the x values
+// it read from shared memory for all 4 rows; 8 independent accumulators keep
+// the FMA chains short.  The weights are read once: the kernel is bound by
+// HBM bandwidth (6.4 GB of adaLN weights per 32-block step).
 constexpr int GEMV_THREADS = 256;
+constexpr int GEMV_ROWS = 4;
+
+__device__ __forceinline__ float dot8(const uint4 w, const float4 a, const float4 b, float acc) {
+  acc = fmaf(__uint_as_float(w.x << 16), a.x, acc);
+  acc = fmaf(__uint_as_float(w.x & 0xFFFF0000u), a.y, acc);
+  acc = fmaf(__uint_as_float(w.y << 16), a.z, acc);
+  acc = fmaf(__uint_as_float(w.y & 0xFFFF0000u), a.w, acc);
+  acc = fmaf(__uint_as_float(w.z << 16), b.x, acc);
+  acc = fmaf(__uint_as_float(w.z & 0xFFFF0000u), b.y, acc);
+  acc = fmaf(__uint_as_float(w.w << 16), b.z, acc);
+  acc = fmaf(__uint_as_float(w.w & 0xFFFF0000u), b.w, acc);
+  return acc;
+}
 
 __global__ void __launch_bounds__(GEMV_THREADS) gemv_kernel(const GemvParams p) {
-  extern __shared__ float xs[];
+  extern __shared__ float4 xs4[];
+  float* xs = reinterpret_cast<float*>(xs4);
   const int total_in = p.R * p.k;
   for (int i = threadIdx.x; i < total_in; i += GEMV_THREADS) {
     float v = p.x[i];
@@ -88,45 +106,56 @@ __global__ void __launch_bounds__(GEMV_THREADS) gemv_kernel(const GemvParams p) 
   const int lane = threadIdx.x & 31;
   const int gwarp = (blockIdx.x * GEMV_THREADS + threadIdx.x) >> 5;
   const int nwarps = (gridDim.x * GEMV_THREADS) >> 5;
-  int total_rows = 0;
-  for (int j = 0; j < p.n_jobs; ++j) total_rows += p.jobs[j].n;
-  for (int g = gwarp; g < total_rows; g += nwarps) {
-    int job = 0, row = g;
-    while (row >= p.jobs[job].n) {
-      row -= p.jobs[job].n;
+  int total = 0;
+  for (int j = 0; j < p.n_jobs; ++j) total += p.jobs[j].n / GEMV_ROWS;
+  const int k4 = p.k / 4;
+  for (int g = gwarp; g < total; g += nwarps) {
+    int job = 0, grp = g;
+    while (grp >= p.jobs[job].n / GEMV_ROWS) {
+      grp -= p.jobs[job].n / GEMV_ROWS;
       ++job;
     }
     const GemvJob& J = p.jobs[job];
-    const uint16_t* wr = J.w + static_cast<int64_t>(row) * p.k;
-    float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll 4
+    const int row0 = grp * GEMV_ROWS;
+    const uint16_t* w0 = J.w + static_cast<int64_t>(row0) * p.k;
+    float a0[GEMV_ROWS] = {0.f, 0.f, 0.f, 0.f}, a1[GEMV_ROWS] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 2
     for (int kk = lane * 8; kk < p.k; kk += 256) {
-      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(wr + kk));
-      const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
+      uint4 w[GEMV_ROWS];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float w0 = __uint_as_float(wv[i] << 16), w1 = __uint_as_float(wv[i] & 0xFFFF0000u);
-        acc0 = fmaf(w0, xs[kk + 2 * i], fmaf(w1, xs[kk + 2 * i + 1], acc0));
-        if (p.R > 1)
-          acc1 = fmaf(w0, xs[p.k + kk + 2 * i], fmaf(w1, xs[p.k + kk + 2 * i + 1], acc1));
+      for (int i = 0; i < GEMV_ROWS; ++i)
+        w[i] = __ldg(reinterpret_cast<const uint4*>(w0 + static_cast<int64_t>(i) * p.k + kk));
+      const float4 xa = xs4[kk / 4], xb = xs4[kk / 4 + 1];
+#pragma unroll
+      for (int i = 0; i < GEMV_ROWS; ++i) a0[i] = dot8(w[i], xa, xb, a0[i]);
+      if (p.R > 1) {
+        const float4 ya = xs4[k4 + kk / 4], yb = xs4[k4 + kk / 4 + 1];
+#pragma unroll
+        for (int i = 0; i < GEMV_ROWS; ++i) a1[i] = dot8(w[i], ya, yb, a1[i]);
       }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-      acc0 += __shfl_xor_sync(0xffffffffu, acc0, o);
-      acc1 += __shfl_xor_sync(0xffffffffu, acc1, o);
+#pragma unroll
+      for (int i = 0; i < GEMV_ROWS; ++i) {
+        a0[i] += __shfl_xor_sync(0xffffffffu, a0[i], o);
+        a1[i] += __shfl_xor_sync(0xffffffffu, a1[i], o);
+      }
     }
-    if (lane == 0) {
-      const float b = J.b ? bf16_bits_to_float(J.b[row]) : 0.f;
-      const float out[2] = {acc0 + b, acc1 + b};
-      for (int r = 0; r < p.R; ++r) {
-        if (p.y_bf16) {
-          __nv_bfloat16 h = __float2bfloat16_rn(out[r]);
-          static_cast<uint16_t*>(J.y)[static_cast<int64_t>(r) * J.ldy + row] =
-              *reinterpret_cast<uint16_t*>(&h);
-        } else {
-          static_cast<float*>(J.y)[static_cast<int64_t>(r) * J.ldy + row] = out[r];
-        }
+    if (lane < GEMV_ROWS * p.R) {
+      const int i = lane % GEMV_ROWS, r = lane / GEMV_ROWS;
+      float out = 0.f;
+#pragma unroll
+      for (int t = 0; t < GEMV_ROWS; ++t)
+        if (t == i) out = r == 0 ? a0[t] : a1[t];
+      const int row = row0 + i;
+      out += J.b ? bf16_bits_to_float(J.b[row]) : 0.f;
+      if (p.y_bf16) {
+        __nv_bfloat16 hv = __float2bfloat16_rn(out);
+        static_cast<uint16_t*>(J.y)[static_cast<int64_t>(r) * J.ldy + row] =
+            *reinterpret_cast<uint16_t*>(&hv);
+      } else {
+        static_cast<float*>(J.y)[static_cast<int64_t>(r) * J.ldy + row] = out;
       }
     }
   }
@@ -134,9 +163,12 @@ __global__ void __launch_bounds__(GEMV_THREADS) gemv_kernel(const GemvParams p) 
 
 int launch_gemv(const GemvParams& p, cudaStream_t st) {
   if (p.R < 1 || p.R > 2 || p.k % 256 != 0 || p.n_jobs > GEMV_MAX_JOBS) return -1;
-  int total_rows = 0;
-  for (int j = 0; j < p.n_jobs; ++j) total_rows += p.jobs[j].n;
-  if (total_rows == 0) return 0;
+  int total = 0;
+  for (int j = 0; j < p.n_jobs; ++j) {
+    if (p.jobs[j].n % GEMV_ROWS != 0) return -1;
+    total += p.jobs[j].n / GEMV_ROWS;
+  }
+  if (total == 0) return 0;
   const size_t smem = static_cast<size_t>(p.R) * p.k * sizeof(float);
   static bool attr = false;
   if (!attr) {
@@ -149,9 +181,9 @@ int launch_gemv(const GemvParams& p, cudaStream_t st) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int rows_per_cta = GEMV_THREADS / 32;
-  int grid = (total_rows + rows_per_cta - 1) / rows_per_cta;
-  const int max_grid = sms * 6;
+  const int per_cta = GEMV_THREADS / 32;
+  int grid = (total + per_cta - 1) / per_cta;
+  const int max_grid = sms * 8;
   if (grid > max_grid) grid = max_grid;
   gemv_kernel<<<grid, GEMV_THREADS, smem, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? 0 : -1;

@@ -12,16 +12,15 @@
 // Weight scheme (same section: symmetric INT8 per output channel, zero point
 // 0, FP32 scales): s = max|w| / 127 (1 for a zero row), q = clamp(rint(w/s), +-127).
 //
-// One 256-thread CTA per row; the row lives in registers (8 elements per
-// chunk, up to 8 chunks per thread: K <= 16384), so the input is read once
-// from HBM and the int8 codes written once.
+// One CTA per row; the row lives in registers (one thread per 32 values), so
+// the input is read once from HBM and the int8 codes are written once.
 #include "qi_common.cuh"
 #include "qi_internal.h"
 
 namespace qi {
 
-constexpr int QT = 256;        // threads per row
-constexpr int QMAXC = 8;       // max chunks of 8 elements per thread
+constexpr int QT = 256;        // threads per row of the weight-preparation kernel
+constexpr int QCH = 4;         // chunks of 8 elements per thread (32 values)
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -39,7 +38,7 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
-// Block-wide reduction of one value over QT threads (8 warps).
+// Block-wide reduction of one value over QT threads (weight preparation).
 template <int OP>   // 0 sum, 1 min, 2 max
 __device__ __forceinline__ float block_reduce(float v, float* red) {
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
@@ -52,6 +51,37 @@ __device__ __forceinline__ float block_reduce(float v, float* red) {
   for (int i = 1; i < QT / 32; ++i)
     r = OP == 0 ? r + red[i] : (OP == 1 ? fminf(r, red[i]) : fmaxf(r, red[i]));
   return r;
+}
+
+// Block-wide reduction of a pair over blockDim.x threads: (sum, sum) or
+// (min, max).  `red` holds 2 x 32 floats.
+template <bool MINMAX>
+__device__ __forceinline__ float2 block_reduce2(float a, float b, float* red) {
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31, nw = blockDim.x >> 5;
+  if (MINMAX) {
+    a = warp_min(a);
+    b = warp_max(b);
+  } else {
+    a = warp_sum(a);
+    b = warp_sum(b);
+  }
+  __syncthreads();
+  if (l == 0) {
+    red[w] = a;
+    red[32 + w] = b;
+  }
+  __syncthreads();
+  float ra = red[0], rb = red[32];
+  for (int i = 1; i < nw; ++i) {
+    if (MINMAX) {
+      ra = fminf(ra, red[i]);
+      rb = fmaxf(rb, red[32 + i]);
+    } else {
+      ra += red[i];
+      rb += red[32 + i];
+    }
+  }
+  return make_float2(ra, rb);
 }
 
 template <bool XBF16>
@@ -72,45 +102,46 @@ __device__ __forceinline__ void load8(const void* base, int64_t off, float* v) {
   }
 }
 
+// One CTA per row with blockDim.x = max(32, K / 32) threads, each holding up
+// to QCH chunks of 8 consecutive elements: chunk c of thread t covers
+// [8 (t + c blockDim), +8), so each load instruction of a warp reads one
+// contiguous segment of the row.
 template <bool XBF16, bool LN>
-__global__ void __launch_bounds__(QT) quant_kernel(const QuantParams p) {
-  __shared__ float red[QT / 32];
+__global__ void __launch_bounds__(1024) quant_kernel(const QuantParams p) {
+  __shared__ float red[64];
   const int row = blockIdx.x;
   const int tid = threadIdx.x;
+  const int nt = blockDim.x;
   const int nchunk = p.K >> 3;
-  float v[QMAXC][8];
+  float v[QCH][8];
 
 #pragma unroll
-  for (int c = 0; c < QMAXC; ++c) {
-    const int ch = tid + c * QT;
+  for (int c = 0; c < QCH; ++c) {
+    const int ch = tid + c * nt;
     if (ch < nchunk) load8<XBF16>(p.x, static_cast<int64_t>(row) * p.ldx + ch * 8, v[c]);
   }
 
   if (LN) {
-    float s = 0.f;
+    float s = 0.f, ss = 0.f;
 #pragma unroll
-    for (int c = 0; c < QMAXC; ++c)
-      if (tid + c * QT < nchunk)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) s += v[c][i];
-    const float mean = block_reduce<0>(s, red) / static_cast<float>(p.K);
-    float ss = 0.f;
-#pragma unroll
-    for (int c = 0; c < QMAXC; ++c)
-      if (tid + c * QT < nchunk)
+    for (int c = 0; c < QCH; ++c)
+      if (tid + c * nt < nchunk)
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const float d = v[c][i] - mean;
-          ss += d * d;
+          s += v[c][i];
+          ss = fmaf(v[c][i], v[c][i], ss);
         }
-    const float var = block_reduce<0>(ss, red) / static_cast<float>(p.K);
+    const float2 t = block_reduce2<false>(s, ss, red);
+    const float inv_k = 1.0f / static_cast<float>(p.K);
+    const float mean = t.x * inv_k;
+    const float var = fmaxf(t.y * inv_k - mean * mean, 0.0f);
     const float rstd = 1.0f / sqrtf(var + p.eps);
     const int rs = p.groups.row_set[group_of(p.groups, p.row0 + row)];
     const uint16_t* sh = p.shift + static_cast<int64_t>(rs) * p.mod_ld;
     const uint16_t* sc = p.scale + static_cast<int64_t>(rs) * p.mod_ld;
 #pragma unroll
-    for (int c = 0; c < QMAXC; ++c) {
-      const int ch = tid + c * QT;
+    for (int c = 0; c < QCH; ++c) {
+      const int ch = tid + c * nt;
       if (ch < nchunk) {
         float fsh[8], fsc[8];
         load8<true>(sh, ch * 8, fsh);
@@ -122,8 +153,8 @@ __global__ void __launch_bounds__(QT) quant_kernel(const QuantParams p) {
     }
     if (p.u_bf16) {   // modulated activation for a BF16 Linear
 #pragma unroll
-      for (int c = 0; c < QMAXC; ++c) {
-        const int ch = tid + c * QT;
+      for (int c = 0; c < QCH; ++c) {
+        const int ch = tid + c * nt;
         if (ch < nchunk) {
           uint4 o;
           o.x = pack_bf16x2(v[c][0], v[c][1]);
@@ -139,15 +170,16 @@ __global__ void __launch_bounds__(QT) quant_kernel(const QuantParams p) {
 
   float lo = 0.f, hi = 0.f;
 #pragma unroll
-  for (int c = 0; c < QMAXC; ++c)
-    if (tid + c * QT < nchunk)
+  for (int c = 0; c < QCH; ++c)
+    if (tid + c * nt < nchunk)
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         lo = fminf(lo, v[c][i]);
         hi = fmaxf(hi, v[c][i]);
       }
-  lo = block_reduce<1>(lo, red);
-  hi = block_reduce<2>(hi, red);
+  const float2 mm = block_reduce2<true>(lo, hi, red);
+  lo = mm.x;
+  hi = mm.y;
   float s = __fdiv_rn(__fsub_rn(hi, lo), 255.0f);
   int zp;
   if (s == 0.0f) {
@@ -158,8 +190,8 @@ __global__ void __launch_bounds__(QT) quant_kernel(const QuantParams p) {
     zp = static_cast<int>(fminf(fmaxf(z, -128.0f), 127.0f));
   }
 #pragma unroll
-  for (int c = 0; c < QMAXC; ++c) {
-    const int ch = tid + c * QT;
+  for (int c = 0; c < QCH; ++c) {
+    const int ch = tid + c * nt;
     if (ch < nchunk) {
       uint32_t packed[2] = {0u, 0u};
 #pragma unroll
@@ -180,8 +212,11 @@ __global__ void __launch_bounds__(QT) quant_kernel(const QuantParams p) {
 
 int launch_quant(const QuantParams& p, cudaStream_t st) {
   if (p.M == 0) return 0;
-  if (p.K % 8 != 0 || p.K > QT * 8 * QMAXC) return -1;
-  dim3 grid(p.M), block(QT);
+  if (p.K % 8 != 0 || p.K > 1024 * 8 * QCH) return -1;
+  int nt = (p.K / 8 + QCH - 1) / QCH;   // threads so that each holds <= QCH chunks
+  nt = ((nt + 31) / 32) * 32;
+  if (nt < 32) nt = 32;
+  dim3 grid(p.M), block(nt);
   if (p.x_bf16) {
     if (p.ln) quant_kernel<true, true><<<grid, block, 0, st>>>(p);
     else quant_kernel<true, false><<<grid, block, 0, st>>>(p);

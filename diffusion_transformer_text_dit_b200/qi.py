@@ -27,7 +27,7 @@ QI_ERR_TIMEOUT = 5
 QI_ERR_WORKSPACE = 6
 
 QI_F32, QI_BF16 = 0, 1
-QI_EPI_STORE, QI_EPI_GELU_TANH, QI_EPI_GATED_RESIDUAL = 0, 1, 2
+QI_EPI_STORE, QI_EPI_GELU_TANH, QI_EPI_GATED_RESIDUAL, QI_EPI_QKV_NORM_ROPE = 0, 1, 2, 3
 QI_KV_NONE, QI_KV_WRITE_PREFIX, QI_KV_READ_PREFIX = 0, 1, 2
 QI_MAX_GROUPS = 16
 
@@ -57,7 +57,10 @@ class qi_linear_bf16(C.Structure):
 class qi_epilogue(C.Structure):
     _fields_ = [("kind", C.c_int32), ("residual", C.c_void_p), ("ld_residual", C.c_int32),
                 ("gate", C.c_void_p), ("gate_ld", C.c_int32), ("groups", C.POINTER(qi_groups)),
-                ("row0", C.c_int32)]
+                ("row0", C.c_int32), ("hidden", C.c_int32), ("eps", C.c_float),
+                ("norm_q", C.c_void_p), ("norm_k", C.c_void_p), ("rope_cos", C.c_void_p),
+                ("rope_sin", C.c_void_p), ("q_out", C.c_void_p), ("k_out", C.c_void_p),
+                ("v_out", C.c_void_p), ("ld_out", C.c_int32)]
 
 
 class qi_dims(C.Structure):

@@ -97,7 +97,10 @@ typedef struct qi_linear_bf16 {
 typedef enum {
   QI_EPI_STORE = 0,           /* y = bf16(Linear(x)) */
   QI_EPI_GELU_TANH = 1,       /* y = bf16(GELU_tanh(bf16(Linear(x)))) */
-  QI_EPI_GATED_RESIDUAL = 2   /* residual += gate[row set] * bf16(Linear(x)), fp32 */
+  QI_EPI_GATED_RESIDUAL = 2,  /* residual += gate[row set] * bf16(Linear(x)), fp32 */
+  QI_EPI_QKV_NORM_ROPE = 3    /* fused QKV projection: y = bf16(Linear(x)) split into q | k | v
+                                 (n = 3 * hidden); q and k get the Q/K RMSNorm (cast before
+                                 scale) and RoPE of qi_qk_norm_rope, v is stored as is */
 } qi_epilogue_kind;
 
 typedef struct qi_epilogue {
@@ -108,6 +111,17 @@ typedef struct qi_epilogue {
   int32_t gate_ld;
   const qi_groups* groups;     /* GATED_RESIDUAL: row set of each row (host pointer) */
   int32_t row0;                /* global token index of row 0 */
+  /* QKV_NORM_ROPE: hidden % 128 == 0 (a GEMM tile holds whole heads), head_dim 128 */
+  int32_t hidden;
+  float eps;
+  const uint16_t* norm_q;      /* [128] bf16 */
+  const uint16_t* norm_k;
+  const float* rope_cos;       /* [M, 64] fp32 tables of the M rows */
+  const float* rope_sin;
+  uint16_t* q_out;             /* [M, ld_out] bf16 */
+  uint16_t* k_out;
+  uint16_t* v_out;
+  int32_t ld_out;
 } qi_epilogue;
 
 typedef struct qi_dims {
@@ -214,7 +228,7 @@ int qi_quantize_act(qi_ctx* ctx, const void* x, int x_dtype, int M, int K, int l
  *   val = (acc - zp_a[m] * w.rowsum[n]) * s_a[m] * w.s[n] + w.bias[n]   (fp32)
  * then the epilogue ep (NULL = QI_EPI_STORE) writes y [M, w.n] bf16 (ld ldy) or
  * updates ep->residual.  acc_debug, if not NULL, receives the raw int32
- * accumulators [M, w.n].  Requires w.k % 128 == 0, w.n % 16 == 0, ldy % 8 == 0. */
+ * accumulators [M, w.n] (not written by the QKV_NORM_ROPE epilogue).  Requires w.k % 128 == 0, w.n % 16 == 0, ldy % 8 == 0. */
 int qi_w8a8_linear(qi_ctx* ctx, const int8_t* qa, const float* s_a, const int32_t* zp_a, int M,
                    const qi_w8* w, const qi_epilogue* ep, uint16_t* y, int ldy,
                    int32_t* acc_debug, void* stream);

@@ -366,3 +366,42 @@ def test_attention_growing_scores_rescale_path(ctx):
     ctx.check()
     ref = _oracle_attn(q, k, v, ends, heads)
     assert rel_l2(bf16_np(o), ref) < 4e-3
+
+
+@pytest.mark.parametrize("M,heads", [(80, 2), (300, 4), (4608, 32)])
+def test_qkv_fused_epilogue_matches_two_step_path(ctx, M, heads):
+    # The fused QKV epilogue (W8A8 GEMM + Q/K RMSNorm + RoPE) against the
+    # two-step path (W8A8 GEMM storing bf16, then qi_qk_norm_rope).  v must be
+    # identical; q and k may differ only where the sum of squares, accumulated
+    # in another order, moves the normalisation by one ulp.
+    H = heads * 128
+    ws, keep, _, _ = _w8_pair(ctx, 3 * H, H, 17)
+    x, (qa, sa, zpa) = _acts(M, H, 23)
+    qa_g, sa_g, zp_g = (cuda(torch.from_numpy(a)) for a in (qa, sa, zpa))
+    wq = cuda(synth.norm_weight(2, "q", 128))
+    wk = cuda(synth.norm_weight(2, "k", 128))
+    groups = [("text", 16, None), ("image", M - 16, (1, M - 16))]
+    cos, sin = (cuda(t) for t in qi.qi_rope_tables(groups))
+    y = torch.empty((M, 3 * H), dtype=torch.bfloat16, device="cuda")
+    qi.qi_w8a8_linear(ctx, qa_g, sa_g, zp_g, ws, y=y)
+    q2, k2, v2 = (torch.empty((M, H), dtype=torch.bfloat16, device="cuda") for _ in range(3))
+    qi.qi_qk_norm_rope(ctx, y, heads, wq, wk, cos, sin, 1e-6, q2, k2, v2)
+    q1, k1, v1 = (torch.empty((M, H), dtype=torch.bfloat16, device="cuda") for _ in range(3))
+    ep = qi.qi_epilogue()
+    ep.kind = qi.QI_EPI_QKV_NORM_ROPE
+    ep.hidden, ep.eps, ep.ld_out = H, 1e-6, H
+    ep.norm_q, ep.norm_k = wq.data_ptr(), wk.data_ptr()
+    ep.rope_cos, ep.rope_sin = cos.data_ptr(), sin.data_ptr()
+    ep.q_out, ep.k_out, ep.v_out = q1.data_ptr(), k1.data_ptr(), v1.data_ptr()
+    qi.qi_w8a8_linear(ctx, qa_g, sa_g, zp_g, ws, epilogue=ep)
+    ctx.check()
+    assert torch.equal(v1, v2)
+    for a, b in ((q1, q2), (k1, k2)):
+        a, b = bf16_np(a), bf16_np(b)
+        # a rotated pair whose inputs differ by at most one bf16 step each can
+        # differ by up to ~2 steps of the pair's norm (which the rotation keeps),
+        # even where the rotated value itself is near zero
+        pair_norm = np.sqrt((b.reshape(M, -1, 2) ** 2).sum(-1, keepdims=True))
+        bound = 4 * BF16_ULP * np.broadcast_to(pair_norm, (M, H // 2, 2)).reshape(M, H) + 1e-6
+        assert np.all(np.abs(a - b) <= bound)
+        assert np.mean(a == b) > 0.99
