@@ -165,6 +165,8 @@ struct BlockBufs {
   uint16_t* q;      // [T, H]
   uint16_t* o;      // [T, H]
   uint16_t* g;      // [T, F]
+  uint32_t* o_range;   // [T][2] row ranges of the attention output
+  uint32_t* g_range;   // [T][2] row ranges of the GELU output
 };
 
 BlockBufs carve_block(Carve& c, const qi_dims& d, int T) {
@@ -177,6 +179,8 @@ BlockBufs carve_block(Carve& c, const qi_dims& d, int T) {
   b.q = c.take<uint16_t>(static_cast<size_t>(T) * H);
   b.o = c.take<uint16_t>(static_cast<size_t>(T) * H);
   b.g = c.take<uint16_t>(static_cast<size_t>(T) * F);
+  b.o_range = c.take<uint32_t>(static_cast<size_t>(T) * 2);
+  b.g_range = c.take<uint32_t>(static_cast<size_t>(T) * 2);
   return b;
 }
 
@@ -253,12 +257,24 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, ui
 
 namespace {
 
+struct QuantExtras {
+  const uint16_t* res_y = nullptr;     // LN: residual add x += gate * y first
+  const uint16_t* res_gate = nullptr;
+  uint32_t* zero_range = nullptr;      // LN: clear these row ranges
+  const uint32_t* range = nullptr;     // plain: producer-published row ranges
+};
+
 int run_quant(qi_ctx* ctx, const void* x, bool xbf16, int M, int K, int ldx,
               const uint16_t* shift, const uint16_t* scale, int mod_ld, const qi::GroupTable& gt,
               int row0, float eps, int8_t* q, float* s, int32_t* zp, uint16_t* u_bf16,
-              cudaStream_t st) {
+              cudaStream_t st, const QuantExtras& ex = QuantExtras()) {
   (void)ctx;
   qi::QuantParams p;
+  memset(&p, 0, sizeof(p));
+  p.res_y = ex.res_y;
+  p.res_gate = ex.res_gate;
+  p.zero_range = ex.zero_range;
+  p.range = ex.range;
   p.x = x;
   p.x_bf16 = xbf16 ? 1 : 0;
   p.M = M;
@@ -284,7 +300,7 @@ int run_quant(qi_ctx* ctx, const void* x, bool xbf16, int M, int K, int ldx,
 int run_w8a8(qi_ctx* ctx, const int8_t* qa, const float* sa, const int32_t* zp, int M,
              const qi_w8& w, int epi, uint16_t* y, int ldy, float* res, int ldr,
              const uint16_t* gate, int gate_ld, const qi::GroupTable& gt, int row0,
-             int32_t* acc_debug, cudaStream_t st) {
+             int32_t* acc_debug, cudaStream_t st, uint32_t* row_range = nullptr) {
   if (M == 0) return QI_OK;
   qi::GemmParams p;
   memset(&p, 0, sizeof(p));
@@ -306,6 +322,7 @@ int run_w8a8(qi_ctx* ctx, const int8_t* qa, const float* sa, const int32_t* zp, 
   p.groups = gt;
   p.row0 = row0;
   p.acc_debug = acc_debug;
+  p.row_range = row_range;
   p.status = ctx->status;
   Prof pr(ctx, QI_KCLASS_GEMM_I8, st);
   const int r = qi::launch_gemm(true, epi, qa, w.k, w.q, w.k, p, ctx->num_sms, st);
@@ -345,10 +362,15 @@ int run_block(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, float* x
   BlockBufs b = carve_block(c, d, T);
   const int mld = 6 * H;
   int r;
-  // attention half
-  if ((r = run_quant(ctx, x, false, T, H, H, mod + 0 * H, mod + 1 * H, mld, gt, row0, d.eps,
-                     b.uq, b.sa, b.zp, nullptr, st)))
-    return r;
+  // attention half.  LN1 + modulate + quantize; it also clears the row
+  // ranges that the attention epilogue will publish for the next quantizer.
+  {
+    QuantExtras ex;
+    ex.zero_range = b.o_range;
+    if ((r = run_quant(ctx, x, false, T, H, H, mod + 0 * H, mod + 1 * H, mld, gt, row0, d.eps,
+                       b.uq, b.sa, b.zp, nullptr, st, ex)))
+      return r;
+  }
   // QKV projection with Q/K RMSNorm + RoPE fused into its epilogue: q goes to
   // the block's q buffer, k and v straight into this layer's K/V rows.
   {
@@ -381,6 +403,7 @@ int run_block(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, float* x
     if (rr != 0) return cuda_fail("QKV GEMM launch");
   }
   qi::AttnParams ap;
+  memset(&ap, 0, sizeof(ap));
   ap.q = b.q;
   ap.k = kl;
   ap.v = vl;
@@ -394,6 +417,7 @@ int run_block(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, float* x
   ap.q_offset = row0;
   ap.sm_scale = 1.0f / sqrtf(static_cast<float>(d.head_dim));
   ap.groups = gt;
+  ap.row_range = b.o_range;
   ap.status = ctx->status;
   {
     Prof pr(ctx, QI_KCLASS_ATTN, st);
@@ -401,22 +425,39 @@ int run_block(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, float* x
     if (r2 == -2) return fail(QI_ERR_CUDA, "cuTensorMapEncodeTiled failed (attention operands)");
     if (r2 != 0) return cuda_fail("attention launch");
   }
-  if ((r = run_quant(ctx, b.o, true, T, H, H, nullptr, nullptr, 0, gt, row0, d.eps, b.uq, b.sa,
-                     b.zp, nullptr, st)))
-    return r;
-  if ((r = run_w8a8(ctx, b.uq, b.sa, b.zp, T, w.out, qi::EPI_GATED, nullptr, 0, x, H,
-                    mod + 2 * H, mld, gt, row0, nullptr, st)))
-    return r;
-  // MLP half
-  if ((r = run_quant(ctx, x, false, T, H, H, mod + 3 * H, mod + 4 * H, mld, gt, row0, d.eps,
-                     b.uq, b.sa, b.zp, nullptr, st)))
-    return r;
-  if ((r = run_w8a8(ctx, b.uq, b.sa, b.zp, T, w.up, qi::EPI_GELU, b.g, F, nullptr, 0, nullptr, 0,
+  {
+    QuantExtras ex;   // the attention epilogue published each row's range
+    ex.range = b.o_range;
+    if ((r = run_quant(ctx, b.o, true, T, H, H, nullptr, nullptr, 0, gt, row0, d.eps, b.uq, b.sa,
+                       b.zp, nullptr, st, ex)))
+      return r;
+  }
+  // output projection stored as bf16 (into the attention output's buffer,
+  // already consumed); its gated residual is applied by the LN2 kernel below,
+  // which reads the residual stream anyway
+  if ((r = run_w8a8(ctx, b.uq, b.sa, b.zp, T, w.out, qi::EPI_BF16, b.o, H, nullptr, 0, nullptr, 0,
                     gt, row0, nullptr, st)))
     return r;
-  if ((r = run_quant(ctx, b.g, true, T, F, F, nullptr, nullptr, 0, gt, row0, d.eps, b.uq, b.sa,
-                     b.zp, nullptr, st)))
+  // MLP half: x += gate1 * out, LN2 + modulate + quantize; clears the GELU ranges
+  {
+    QuantExtras ex;
+    ex.res_y = b.o;
+    ex.res_gate = mod + 2 * H;
+    ex.zero_range = b.g_range;
+    if ((r = run_quant(ctx, x, false, T, H, H, mod + 3 * H, mod + 4 * H, mld, gt, row0, d.eps,
+                       b.uq, b.sa, b.zp, nullptr, st, ex)))
+      return r;
+  }
+  if ((r = run_w8a8(ctx, b.uq, b.sa, b.zp, T, w.up, qi::EPI_GELU, b.g, F, nullptr, 0, nullptr, 0,
+                    gt, row0, nullptr, st, b.g_range)))
     return r;
+  {
+    QuantExtras ex;   // the GELU epilogue published each row's range
+    ex.range = b.g_range;
+    if ((r = run_quant(ctx, b.g, true, T, F, F, nullptr, nullptr, 0, gt, row0, d.eps, b.uq, b.sa,
+                       b.zp, nullptr, st, ex)))
+      return r;
+  }
   if ((r = run_w8a8(ctx, b.uq, b.sa, b.zp, T, w.down, qi::EPI_GATED, nullptr, 0, x, H,
                     mod + 5 * H, mld, gt, row0, nullptr, st)))
     return r;
@@ -770,6 +811,7 @@ int qi_attn_block_causal(qi_ctx* ctx, const uint16_t* q, int ldq, int Sq, int q_
   int r;
   if ((r = check_groups(groups, Sk, &gt))) return r;
   qi::AttnParams p;
+  memset(&p, 0, sizeof(p));
   p.q = q;
   p.k = k;
   p.v = v;

@@ -337,21 +337,32 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
     if (ok && n_kv > 0 && mbar_wait_warp(o_full, 0, status)) {
       tc_fence_after();
       const float inv = l > 0.f ? 1.0f / l : 0.f;
+      float rlo = 0.f, rhi = 0.f;   // range of the stored bf16 values of this row
       // every lane of the warp takes part in the (warp-wide) TMEM loads
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t r[32];
         tmem_ld32(tO + c * 32, r);
         if (qrow < p.Sq) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float a = bf16_round_f(__uint_as_float(r[2 * i]) * inv);
+            const float b = bf16_round_f(__uint_as_float(r[2 * i + 1]) * inv);
+            rlo = fminf(rlo, fminf(a, b));
+            rhi = fmaxf(rhi, fmaxf(a, b));
+            pk[i] = pack_bf16x2(a, b);
+          }
           uint4* dst = reinterpret_cast<uint4*>(p.o + static_cast<int64_t>(qrow) * p.ldo + hc + c * 32);
 #pragma unroll
-          for (int v = 0; v < 4; ++v)
-            dst[v] = make_uint4(
-                pack_bf16x2(__uint_as_float(r[8 * v + 0]) * inv, __uint_as_float(r[8 * v + 1]) * inv),
-                pack_bf16x2(__uint_as_float(r[8 * v + 2]) * inv, __uint_as_float(r[8 * v + 3]) * inv),
-                pack_bf16x2(__uint_as_float(r[8 * v + 4]) * inv, __uint_as_float(r[8 * v + 5]) * inv),
-                pack_bf16x2(__uint_as_float(r[8 * v + 6]) * inv, __uint_as_float(r[8 * v + 7]) * inv));
+          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
         }
+      }
+      if (p.row_range && qrow < p.Sq) {
+        // per-row range for the next quantizer (non-negative floats order like
+        // their bit patterns; negative zero is normalised to +0)
+        atomicMax(p.row_range + 2 * static_cast<size_t>(qrow), __float_as_uint(__fsub_rn(0.0f, rlo)));
+        atomicMax(p.row_range + 2 * static_cast<size_t>(qrow) + 1, __float_as_uint(__fadd_rn(rhi, 0.0f)));
       }
     }
   }

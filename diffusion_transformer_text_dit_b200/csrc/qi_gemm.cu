@@ -38,10 +38,17 @@ struct GemmCfg {
   static_assert(2 * STAGES + 5 <= 31, "barrier area");
 };
 
+// GELU, tanh form: 0.5 x (1 + tanh(z)), z = sqrt(2/pi) (x + 0.044715 x^3).
+// Evaluated as x / (1 + e^(-2z)) (the same function: 0.5 (1 + tanh z) is the
+// logistic of 2z), with the hardware base-2 exponential and a fast divide;
+// relative error ~1e-6, far below the bf16 rounding of the result.
 __device__ __forceinline__ float gelu_tanh_f(float x) {
   const float k0 = 0.7978845608028654f;   // sqrt(2/pi)
   const float k1 = 0.044715f;
-  return 0.5f * x * (1.0f + tanhf(k0 * (x + k1 * x * x * x)));
+  const float z = k0 * fmaf(k1 * x, x * x, x);
+  float e;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-2.8853900817779268f * z));   // e^(-2z)
+  return __fdividef(x, 1.0f + e);
 }
 
 // W8A8 dequantization of 32 accumulator columns starting at column nb,
@@ -293,6 +300,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         if (acc == 0) acc_phase ^= 1u;
         continue;
       }
+      float rlo = 0.f, rhi = 0.f;   // GELU: row range of this warp's half tile
 #pragma unroll 1
       for (int c = half * (BN / 64); c < (half + 1) * (BN / 64); ++c) {
         uint32_t r[32];
@@ -333,8 +341,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           for (int j = 0; j < 16; ++j) {
             float a0 = v[2 * j], a1 = v[2 * j + 1];
             if (EPI == EPI_GELU) {
-              a0 = gelu_tanh_f(bf16_round_f(a0));
-              a1 = gelu_tanh_f(bf16_round_f(a1));
+              a0 = bf16_round_f(gelu_tanh_f(bf16_round_f(a0)));
+              a1 = bf16_round_f(gelu_tanh_f(bf16_round_f(a1)));
+              if (8 * (j >> 2) < ncols) {   // the stored values' range for the quantizer
+                rlo = fminf(rlo, fminf(a0, a1));
+                rhi = fmaxf(rhi, fmaxf(a0, a1));
+              }
             }
             w[j] = pack_bf16x2(a0, a1);
           }
@@ -396,6 +408,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             lat[j] = x;
           }
         }
+      }
+      if (EPI == EPI_GELU && p.row_range && row_ok) {
+        // non-negative floats order like their bit patterns; 0 - lo and hi + 0
+        // turn a negative zero into +0 so it cannot win the unsigned max
+        atomicMax(p.row_range + 2 * static_cast<size_t>(m), __float_as_uint(__fsub_rn(0.0f, rlo)));
+        atomicMax(p.row_range + 2 * static_cast<size_t>(m) + 1, __float_as_uint(__fadd_rn(rhi, 0.0f)));
       }
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;

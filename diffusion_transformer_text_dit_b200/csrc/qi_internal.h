@@ -51,6 +51,7 @@ struct GemmParams {
   uint16_t* k_out;
   uint16_t* v_out_bf16;
   int ldo;
+  uint32_t* row_range;    // GELU: optional per-row [-min, max] bit patterns of the bf16 output
   int* status;            // device status word
 };
 
@@ -81,6 +82,13 @@ struct QuantParams {
   float* s;               // [M]
   int32_t* zp;            // [M]
   uint16_t* u_bf16;       // if non-null: write bf16(u) [M, ldq] instead of quantizing
+  // LN variant: residual add before the LayerNorm, x += gate[row set] * y
+  const uint16_t* res_y;  // bf16 [M, K] or null
+  const uint16_t* res_gate;   // gate row of set r at res_gate + r * mod_ld
+  uint32_t* zero_range;   // if non-null: rows' [2] range words set to 0 (for a later producer)
+  // plain variant: the row's range was published by the producer as
+  // [float bits of -min, float bits of max] (both >= 0); no reduction needed
+  const uint32_t* range;
 };
 int launch_quant(const QuantParams& p, cudaStream_t st);
 
@@ -114,6 +122,7 @@ struct AttnParams {
   int Sq, Sk, heads, q_offset;
   float sm_scale;
   GroupTable groups;
+  uint32_t* row_range;    // optional per-query-row [-min, max] bit patterns of the bf16 output
   int* status;            // device status word
 };
 int launch_attention(const AttnParams& p, cudaStream_t st);

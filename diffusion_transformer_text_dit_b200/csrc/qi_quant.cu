@@ -106,7 +106,7 @@ __device__ __forceinline__ void load8(const void* base, int64_t off, float* v) {
 // to QCH chunks of 8 consecutive elements: chunk c of thread t covers
 // [8 (t + c blockDim), +8), so each load instruction of a warp reads one
 // contiguous segment of the row.
-template <bool XBF16, bool LN>
+template <bool XBF16, bool LN, bool RANGE>
 __global__ void __launch_bounds__(1024) quant_kernel(const QuantParams p) {
   __shared__ float red[64];
   const int row = blockIdx.x;
@@ -121,7 +121,33 @@ __global__ void __launch_bounds__(1024) quant_kernel(const QuantParams p) {
     if (ch < nchunk) load8<XBF16>(p.x, static_cast<int64_t>(row) * p.ldx + ch * 8, v[c]);
   }
 
+  if (LN && p.zero_range && tid == 0) {
+    p.zero_range[2 * static_cast<int64_t>(row)] = 0u;
+    p.zero_range[2 * static_cast<int64_t>(row) + 1] = 0u;
+  }
+
   if (LN) {
+    if (p.res_y) {
+      // residual add of the previous Linear: x = x + gate[row set] * y (fp32),
+      // written back so the residual stream carries it
+      const int rs0 = p.groups.row_set[group_of(p.groups, p.row0 + row)];
+      const uint16_t* gt = p.res_gate + static_cast<int64_t>(rs0) * p.mod_ld;
+      float* xw = const_cast<float*>(static_cast<const float*>(p.x)) + static_cast<int64_t>(row) * p.ldx;
+#pragma unroll
+      for (int c = 0; c < QCH; ++c) {
+        const int ch = tid + c * nt;
+        if (ch < nchunk) {
+          float fy[8], fg[8];
+          load8<true>(p.res_y, static_cast<int64_t>(row) * p.K + ch * 8, fy);
+          load8<true>(gt, ch * 8, fg);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) v[c][i] = fmaf(fg[i], fy[i], v[c][i]);
+          float4* o4 = reinterpret_cast<float4*>(xw + ch * 8);
+          o4[0] = make_float4(v[c][0], v[c][1], v[c][2], v[c][3]);
+          o4[1] = make_float4(v[c][4], v[c][5], v[c][6], v[c][7]);
+        }
+      }
+    }
     float s = 0.f, ss = 0.f;
 #pragma unroll
     for (int c = 0; c < QCH; ++c)
@@ -169,17 +195,23 @@ __global__ void __launch_bounds__(1024) quant_kernel(const QuantParams p) {
   }
 
   float lo = 0.f, hi = 0.f;
+  if (RANGE) {
+    // range published by the producer: [-min, max] as float bit patterns
+    lo = -__uint_as_float(p.range[2 * static_cast<int64_t>(row)]);
+    hi = __uint_as_float(p.range[2 * static_cast<int64_t>(row) + 1]);
+  } else {
 #pragma unroll
-  for (int c = 0; c < QCH; ++c)
-    if (tid + c * nt < nchunk)
+    for (int c = 0; c < QCH; ++c)
+      if (tid + c * nt < nchunk)
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        lo = fminf(lo, v[c][i]);
-        hi = fmaxf(hi, v[c][i]);
-      }
-  const float2 mm = block_reduce2<true>(lo, hi, red);
-  lo = mm.x;
-  hi = mm.y;
+        for (int i = 0; i < 8; ++i) {
+          lo = fminf(lo, v[c][i]);
+          hi = fmaxf(hi, v[c][i]);
+        }
+    const float2 mm = block_reduce2<true>(lo, hi, red);
+    lo = mm.x;
+    hi = mm.y;
+  }
   float s = __fdiv_rn(__fsub_rn(hi, lo), 255.0f);
   int zp;
   if (s == 0.0f) {
@@ -189,6 +221,11 @@ __global__ void __launch_bounds__(1024) quant_kernel(const QuantParams p) {
     const float z = rintf(__fsub_rn(-128.0f, __fdiv_rn(lo, s)));
     zp = static_cast<int>(fminf(fmaxf(z, -128.0f), 127.0f));
   }
+  // rint(u / s) with the IEEE quotient, computed as u * (1/s): |u/s| <= 255, so
+  // the product is within ~3e-5 of the exact quotient and rounds the same way
+  // unless its fraction is within 1e-4 of one half; those rare elements take
+  // the exact division.
+  const float inv_s = __fdiv_rn(1.0f, s);
 #pragma unroll
   for (int c = 0; c < QCH; ++c) {
     const int ch = tid + c * nt;
@@ -196,7 +233,10 @@ __global__ void __launch_bounds__(1024) quant_kernel(const QuantParams p) {
       uint32_t packed[2] = {0u, 0u};
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        int qv = static_cast<int>(rintf(__fdiv_rn(v[c][i], s))) + zp;
+        const float t = v[c][i] * inv_s;
+        float rq = rintf(t);
+        if (fabsf(fabsf(t - rq) - 0.5f) < 1e-4f) rq = rintf(__fdiv_rn(v[c][i], s));
+        int qv = static_cast<int>(rq) + zp;
         qv = max(-128, min(127, qv));
         packed[i >> 2] |= (static_cast<uint32_t>(qv) & 0xFFu) << (8 * (i & 3));
       }
@@ -217,12 +257,15 @@ int launch_quant(const QuantParams& p, cudaStream_t st) {
   nt = ((nt + 31) / 32) * 32;
   if (nt < 32) nt = 32;
   dim3 grid(p.M), block(nt);
+  if (p.ln && p.range) return -1;                 // LN computes its own range
+  if (p.res_y && (!p.ln || p.x_bf16)) return -1;  // the residual add writes the fp32 stream
   if (p.x_bf16) {
-    if (p.ln) quant_kernel<true, true><<<grid, block, 0, st>>>(p);
-    else quant_kernel<true, false><<<grid, block, 0, st>>>(p);
+    if (p.ln) quant_kernel<true, true, false><<<grid, block, 0, st>>>(p);
+    else if (p.range) quant_kernel<true, false, true><<<grid, block, 0, st>>>(p);
+    else quant_kernel<true, false, false><<<grid, block, 0, st>>>(p);
   } else {
-    if (p.ln) quant_kernel<false, true><<<grid, block, 0, st>>>(p);
-    else quant_kernel<false, false><<<grid, block, 0, st>>>(p);
+    if (p.ln) quant_kernel<false, true, false><<<grid, block, 0, st>>>(p);
+    else quant_kernel<false, false, false><<<grid, block, 0, st>>>(p);
   }
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
