@@ -40,14 +40,19 @@ CFG = synth.STEP1024
 
 # ------------------------------------------------------------------ workload arithmetic
 
-def algorithmic_work(cfg: synth.DitConfig):
-    """Per-step algorithmic work: int8 ops of the W8A8 Linears, bf16 FLOPs of the
-    unmasked attention pairs, and the bytes of the bandwidth-bound parts."""
-    H, F, S, d, h = cfg.hidden, cfg.mlp, cfg.tokens, cfg.head_dim, cfg.heads
-    per_block_ops = 2 * S * (3 * H * H + H * H + F * H + H * F)
+def algorithmic_work(cfg: synth.DitConfig, cached: bool = False):
+    """Per-step algorithmic work: int8 ops of the W8A8 Linears and bf16 FLOPs of
+    the visible (unmasked) query-key pairs.  A cached step processes only the
+    target rows, which still attend over every key."""
+    H, F, d, h = cfg.hidden, cfg.mlp, cfg.head_dim, cfg.heads
+    rows = cfg.target_tokens if cached else cfg.tokens
+    per_block_ops = 2 * rows * (3 * H * H + H * H + F * H + H * F)
     ends = np.cumsum(cfg.group_sizes())
     starts = np.concatenate([[0], ends[:-1]])
-    pairs = int(sum((e - s) * e for s, e in zip(starts, ends)))   # query x visible keys
+    if cached:
+        pairs = int(cfg.target_tokens * ends[-1])
+    else:
+        pairs = int(sum((e - s) * e for s, e in zip(starts, ends)))   # query x visible keys
     attn_flops = 4 * d * h * pairs
     return {
         "gemm_i8_ops_per_step": cfg.blocks * per_block_ops,
@@ -215,32 +220,59 @@ def run_reference(args, rank):
     print(json.dumps(out), flush=True)
 
 
+# ------------------------------------------------------------------ ranks
+
+class Ranks:
+    """Barrier and max-over-ranks for the timing of independent replicas.  The
+    step has no cross-device exchange: these are the only collectives."""
+
+    def __init__(self, world: int, backend: str = "nccl", device=None):
+        self.world = world
+        self.dist = None
+        self.device = device
+        if world > 1:
+            import torch.distributed as dist
+            kw = {"device_id": device} if backend == "nccl" else {}
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
+            self.dist = dist
+
+    def barrier(self):
+        if self.dist is not None:
+            self.dist.barrier()
+
+    def max(self, v: float) -> float:
+        if self.dist is None:
+            return v
+        dev = self.device if self.device is not None else "cpu"
+        t = torch.tensor([v], device=dev, dtype=torch.float64)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.dist is not None:
+            self.dist.destroy_process_group()
+            self.dist = None
+
+
+def aggregate_throughput(world: int, steps: int, max_ms: float) -> float:
+    """Whole-job steps/s: every replica runs `steps` steps; the slowest sets the time."""
+    return world * steps / (max_ms / 1e3)
+
+
 # ------------------------------------------------------------------ GPU arm
+
+WORKLOADS = {c.name: c for c in (synth.STEP1024, synth.EDIT1024, synth.GEN2048)}
+
 
 def run_ours(args, rank, world, local_rank):
     from diffusion_transformer_text_dit_b200 import build_lib, qi
     build_lib.build()
     torch.cuda.set_device(local_rank)
-    dist = None
-    if world > 1:
-        import torch.distributed as dist_mod
-        dist = dist_mod
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local_rank))
-
-    def barrier():
-        if dist is not None:
-            dist.barrier()
-
-    def max_over_ranks(v: float) -> float:
-        if dist is None:
-            return v
-        t = torch.tensor([v], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    ranks = Ranks(world, "nccl", torch.device("cuda", local_rank))
 
     ctx = qi.Context(local_rank)
-    cfg = CFG
+    cfg = WORKLOADS[args.workload]
+    denoise = cfg.steps > 1            # the 40-step 2048^2 workload
     model, dims = build_model(ctx, qi, cfg, "cuda")
     S, H = cfg.tokens, cfg.hidden
     gd = [(g.kind, g.tokens, g.grid) for g in cfg.groups]
@@ -250,44 +282,73 @@ def run_ours(args, rank, world, local_rank):
     cos, sin = cos.cuda(), sin.cuda()
     sig = qi.qi_sigma_schedule(40, cfg.target_tokens).tolist()
     ws = torch.empty(qi.qi_step_workspace_bytes(dims, S), dtype=torch.uint8, device="cuda")
+    kv = torch.empty((cfg.blocks, 2, S, H), dtype=torch.bfloat16, device="cuda")
     txt = synth.text_features(cfg, device="cuda")
+    ref = synth.ref_latents(cfg, device="cuda")
     lat0 = synth.latents(cfg, device="cuda")
     lat = lat0.clone()
     stream = torch.cuda.current_stream()
 
-    def step(i, latents, text):
+    def step(i, latents, text, mode=qi.QI_KV_NONE):
         j = i % 40
-        qi.qi_denoise_step(ctx, model, latents, text, cfg.text_tokens, None, groups, cos, sin,
-                           sig[j], sig[j + 1], qi.QI_KV_NONE, None, None, ws)
+        cached = mode == qi.QI_KV_READ_PREFIX
+        qi.qi_denoise_step(ctx, model, latents, None if cached else text, cfg.text_tokens,
+                           None if cached else ref, groups, cos, sin, sig[j], sig[j + 1], mode,
+                           None if mode == qi.QI_KV_NONE else kv, None, ws)
+
+    def denoise_40(latents, text):
+        # FlowMatch Euler over the 40-step schedule; the prefix K/V of the
+        # first step are reused by the 39 later steps
+        step(0, latents, text, qi.QI_KV_WRITE_PREFIX)
+        for i in range(1, 40):
+            step(i, latents, text, qi.QI_KV_READ_PREFIX)
+
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+
+    def timed(fn):
+        ranks.barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ranks.barrier()
+        return ranks.max(e0.elapsed_time(e1))
 
     for i in range(args.warmup):
         step(i, lat, txt)
     ctx.check()
 
-    # ---------------- device-resident timed region
+    # ---------------- device-resident timed region (profiled per kernel class)
     clocks = ClockSampler([local_rank]) if rank == 0 else None
     if clocks:
         clocks.start()
         time.sleep(0.3)
     ctx.profile(True)
-    barrier()
-    torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(args.steps):
-        step(i, lat, txt)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    ms = e0.elapsed_time(e1)
+    if denoise:
+        n_steps = 40
+        ms_max = timed(lambda: denoise_40(lat, txt))
+    else:
+        n_steps = args.steps
+        ms_max = timed(lambda: [step(i, lat, txt) for i in range(n_steps)])
     prof = ctx.profile_read()
     ctx.profile(False)
     clk = clocks.stop() if clocks else None
     ctx.check()
-    ms_max = max_over_ranks(ms)
-    ms_per_step = ms_max / args.steps
-    value = world * args.steps / (ms_max / 1e3)
+    ms_per_step = ms_max / n_steps
+    value = aggregate_throughput(world, n_steps, ms_max)
+
+    # ---------------- cached-prefix steps (the pages' later denoising steps)
+    extra = {}
+    if not denoise:
+        step(0, lat, txt, qi.QI_KV_WRITE_PREFIX)
+        cms = timed(lambda: [step(i + 1, lat, txt, qi.QI_KV_READ_PREFIX) for i in range(args.steps)])
+        extra["cached_step"] = {"value": aggregate_throughput(world, args.steps, cms),
+                                "unit": "steps/s", "ms_per_step": cms / args.steps,
+                                "note": "target rows only; prefix K/V read from the cache"}
+    else:
+        extra["seconds_per_40_steps"] = ms_max / 1e3
 
     # ---------------- end to end through the public call with host buffers
     h_lat = lat0.cpu().pin_memory()
@@ -295,71 +356,75 @@ def run_ours(args, rank, world, local_rank):
     h_out = torch.empty_like(h_lat).pin_memory()
     d_lat = torch.empty_like(lat0)
     d_txt = torch.empty_like(txt)
-    h2d = h_lat.numel() * 4 + h_txt.numel() * 2
-    d2h = h_out.numel() * 4
-    for i in range(2):
-        d_lat.copy_(h_lat, non_blocking=True)
-        d_txt.copy_(h_txt, non_blocking=True)
-        step(i, d_lat, d_txt)
-        h_out.copy_(d_lat, non_blocking=True)
-    barrier()
-    torch.cuda.synchronize()
-    e0.record(stream)
-    for i in range(args.steps):
-        d_lat.copy_(h_lat, non_blocking=True)
-        d_txt.copy_(h_txt, non_blocking=True)
-        step(i, d_lat, d_txt)
-        h_out.copy_(d_lat, non_blocking=True)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
-    e2e = world * args.steps / (e2e_ms / 1e3)
+    if denoise:
+        # inputs copied in before the first step, the result copied out after the last
+        def e2e_run():
+            d_lat.copy_(h_lat, non_blocking=True)
+            d_txt.copy_(h_txt, non_blocking=True)
+            denoise_40(d_lat, d_txt)
+            h_out.copy_(d_lat, non_blocking=True)
+        h2d = (h_lat.numel() * 4 + h_txt.numel() * 2) / 40
+        d2h = h_out.numel() * 4 / 40
+        e2e_ms = timed(e2e_run)
+        e2e = aggregate_throughput(world, 40, e2e_ms)
+    else:
+        def e2e_run():
+            for i in range(args.steps):
+                d_lat.copy_(h_lat, non_blocking=True)
+                d_txt.copy_(h_txt, non_blocking=True)
+                step(i, d_lat, d_txt)
+                h_out.copy_(d_lat, non_blocking=True)
+        h2d = h_lat.numel() * 4 + h_txt.numel() * 2
+        d2h = h_out.numel() * 4
+        e2e_run()
+        e2e_ms = timed(e2e_run)
+        e2e = aggregate_throughput(world, args.steps, e2e_ms)
     ctx.check()
 
     if rank != 0:
-        if dist is not None:
-            dist.destroy_process_group()
+        ranks.close()
         return
 
     # ---------------- roofline of the dominant kernel class
-    work = algorithmic_work(cfg)
+    if denoise:
+        w_full, w_cached = algorithmic_work(cfg, False), algorithmic_work(cfg, True)
+        work = {k: (w_full[k] + 39 * w_cached[k]) / 40 for k in ("gemm_i8_ops_per_step", "attn_flops_per_step")}
+    else:
+        work = algorithmic_work(cfg)
     pk = peaks()
     tot = {k: v[2] for k, v in prof.items()}
     dom = max(tot, key=tot.get)
-    kernels = {k: {"launches_per_step": prof[k][0] / args.steps,
-                   "ms_per_step": tot[k] / args.steps,
+    kernels = {k: {"launches_per_step": prof[k][0] / n_steps,
+                   "ms_per_step": tot[k] / n_steps,
                    "share": tot[k] / max(sum(tot.values()), 1e-9)} for k in tot if prof[k][0]}
     if dom == "attention":
-        achieved = work["attn_flops_per_step"] * args.steps / (tot[dom] / 1e3) / 1e12
+        achieved = work["attn_flops_per_step"] * n_steps / (tot[dom] / 1e3) / 1e12
         roof = {"bound": "tensor", "unit": "TFLOP/s", "peak": pk["bf16_sust"],
                 "peak_note": f"bf16 dense, sustained, {pk['src']}"}
     elif dom == "gemm_i8":
-        achieved = work["gemm_i8_ops_per_step"] * args.steps / (tot[dom] / 1e3) / 1e12
+        achieved = work["gemm_i8_ops_per_step"] * n_steps / (tot[dom] / 1e3) / 1e12
         roof = {"bound": "tensor", "unit": "TOP/s", "peak": 2 * pk["bf16_sust"],
                 "peak_note": f"int8 dense = bf16 sustained {pk['src']} x nominal int8/bf16 ratio 2"}
     else:
         achieved = None
         roof = {"bound": "hbm", "unit": "GB/s", "peak": pk["hbm"], "peak_note": pk["src"]}
-    launches_per_kernel = prof[dom][0] / args.steps
-    tr = kernel_traffic(dom)
+    tr = kernel_traffic(dom) if not denoise and cfg is synth.STEP1024 else None
     roof.update({"kernel": dom, "achieved": achieved,
                  "frac": (achieved / roof["peak"]) if achieved else None,
-                 "traffic": tr, "ms_per_step": tot[dom] / args.steps,
-                 "launches_per_step": launches_per_kernel})
-    # secondary: the other tensor-core class, for the metric's second half
+                 "traffic": tr, "ms_per_step": tot[dom] / n_steps,
+                 "launches_per_step": prof[dom][0] / n_steps})
     other = {}
     if prof["gemm_i8"][0]:
-        a = work["gemm_i8_ops_per_step"] * args.steps / (tot["gemm_i8"] / 1e3) / 1e12
+        a = work["gemm_i8_ops_per_step"] * n_steps / (tot["gemm_i8"] / 1e3) / 1e12
         other["gemm_i8"] = {"achieved_tops": a, "peak_tops": 2 * pk["bf16_sust"],
                             "frac": a / (2 * pk["bf16_sust"])}
     if prof["attention"][0]:
-        a = work["attn_flops_per_step"] * args.steps / (tot["attention"] / 1e3) / 1e12
+        a = work["attn_flops_per_step"] * n_steps / (tot["attention"] / 1e3) / 1e12
         other["attention"] = {"achieved_tflops": a, "peak_tflops": pk["bf16_sust"],
                               "frac": a / pk["bf16_sust"]}
 
     cpu = None
-    if world == 1 and not args.no_cpu_baseline:
+    if world == 1 and not args.no_cpu_baseline and cfg is synth.STEP1024:
         osamp = OracleSample()
         tb = osamp.time_block()
         v = 1.0 / (tb * cfg.blocks)
@@ -367,21 +432,23 @@ def run_ours(args, rank, world, local_rank):
                "sample": (f"1 of {cfg.blocks} blocks of the 1024^2 step (S={cfg.tokens}), "
                           f"float64 numpy oracle, {tb:.1f} s, extrapolated x{cfg.blocks}")}
 
+    desc = (f"{cfg.name}: {cfg.blocks} blocks, hidden {H}, {cfg.heads}x128 heads, MLP {cfg.mlp}, "
+            f"groups {'|'.join(str(n) for n in cfg.group_sizes())} tokens, "
+            + ("40-step FlowMatch Euler denoise, prefix K/V cached from step 2"
+               if denoise else "uncached step")
+            + ", all attn/MLP Linears W8A8 (int8 GEMMs, bf16 attention)")
     out = {
         "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "steps": n_steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
         "data": "synthetic",
-        "config": {"workload": (f"{cfg.name}: {cfg.blocks} blocks, hidden {H}, {cfg.heads}x128 "
-                                f"heads, MLP {cfg.mlp}, {cfg.text_tokens} text + "
-                                f"{cfg.target_tokens} image tokens, uncached step, all "
-                                f"attn/MLP Linears W8A8 (int8 GEMMs, bf16 attention)"),
-                   "tokens": S, "blocks": cfg.blocks, "global_batch": world,
+        "config": {"workload": desc, "tokens": S, "blocks": cfg.blocks, "global_batch": world,
                    "l2": "inputs larger than L2: ~12.8 GB of weights streamed per step",
                    "parallelism": f"replicas x{world}"},
         "roofline": roof,
         "tensor_core_fracs": other,
         "kernels": kernels,
+        "extra": extra,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e, "unit": "steps/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
@@ -389,12 +456,12 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clk,
     }
     print(json.dumps(out), flush=True)
-    if dist is not None:
-        dist.destroy_process_group()
+    ranks.close()
 
 
 def run_ncu_case(args):
     """A few launches of one kernel at the 1024^2 step's shapes, for ncu captures:
+    gemms:     the block's four W8A8 GEMMs (QKV, out, up, down) in block order;
     gemm_down: W8A8 down projection, M = 4608, N = 4096, K = 16384 (operands
                142 MB > L2);
     attention: block-causal attention over [512 | 4096] tokens, 32 heads."""
@@ -404,7 +471,47 @@ def run_ncu_case(args):
     cfg = CFG
     S, H, F = cfg.tokens, cfg.hidden, cfg.mlp
     g = torch.Generator(device="cuda").manual_seed(5)
-    if args.ncu_case == "gemm_down":
+    if args.ncu_case == "gemms":
+        # the four W8A8 GEMMs of a block at the 1024^2 shapes, in block order:
+        # QKV (fused norm/RoPE epilogue), out, up (+GELU), down (+gated residual)
+        def w8(n, k, seed):
+            w = torch.randn(n, k, device="cuda", generator=g) * 0.02
+            q, s_, rs = qi.qi_prepare_w8(ctx, w)
+            return q, s_, rs, torch.zeros(n, device="cuda", dtype=torch.bfloat16)
+        Wqkv, Wout, Wup, Wdown = w8(3 * H, H, 1), w8(H, H, 2), w8(F, H, 3), w8(H, F, 4)
+        qa = torch.randint(-128, 128, (S, F), device="cuda", generator=g, dtype=torch.int8)
+        sa = torch.rand(S, device="cuda", generator=g) * 0.01 + 1e-3
+        zp = torch.randint(-128, 128, (S,), device="cuda", generator=g, dtype=torch.int32)
+        qa_h = qa[:, :H].contiguous()
+        y = torch.empty((S, F), device="cuda", dtype=torch.bfloat16)
+        x = torch.zeros((S, H), device="cuda", dtype=torch.float32)
+        gate = torch.ones((2, H), device="cuda", dtype=torch.bfloat16)
+        qo, ko, vo = (torch.empty((S, H), device="cuda", dtype=torch.bfloat16) for _ in range(3))
+        nq = torch.ones(128, device="cuda", dtype=torch.bfloat16)
+        cos_t = torch.ones((S, 64), device="cuda")
+        sin_t = torch.zeros((S, 64), device="cuda")
+        groups = qi.groups_struct(list(np.cumsum(cfg.group_sizes())), cfg.group_row_sets())
+        import ctypes
+        ep_qkv = qi.qi_epilogue()
+        ep_qkv.kind = qi.QI_EPI_QKV_NORM_ROPE
+        ep_qkv.hidden, ep_qkv.eps, ep_qkv.ld_out = H, 1e-6, H
+        ep_qkv.norm_q = ep_qkv.norm_k = nq.data_ptr()
+        ep_qkv.rope_cos, ep_qkv.rope_sin = cos_t.data_ptr(), sin_t.data_ptr()
+        ep_qkv.q_out, ep_qkv.k_out, ep_qkv.v_out = qo.data_ptr(), ko.data_ptr(), vo.data_ptr()
+        ep_gelu = qi.qi_epilogue()
+        ep_gelu.kind = qi.QI_EPI_GELU_TANH
+        ep_res = qi.qi_epilogue()
+        ep_res.kind = qi.QI_EPI_GATED_RESIDUAL
+        ep_res.residual, ep_res.ld_residual = x.data_ptr(), H
+        ep_res.gate, ep_res.gate_ld = gate.data_ptr(), H
+        ep_res.groups = ctypes.pointer(groups)
+        yh = y[:, :H].contiguous()
+        for _ in range(args.warmup + args.steps):
+            qi.qi_w8a8_linear(ctx, qa_h, sa, zp, qi.w8_struct(*Wqkv), epilogue=ep_qkv)
+            qi.qi_w8a8_linear(ctx, qa_h, sa, zp, qi.w8_struct(*Wout), y=yh)
+            qi.qi_w8a8_linear(ctx, qa_h, sa, zp, qi.w8_struct(*Wup), epilogue=ep_gelu, y=y)
+            qi.qi_w8a8_linear(ctx, qa, sa, zp, qi.w8_struct(*Wdown), epilogue=ep_res)
+    elif args.ncu_case == "gemm_down":
         qa = torch.randint(-128, 128, (S, F), device="cuda", generator=g, dtype=torch.int8)
         sa = torch.rand(S, device="cuda", generator=g) * 0.01 + 1e-3
         zp = torch.randint(-128, 128, (S,), device="cuda", generator=g, dtype=torch.int32)
@@ -436,7 +543,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--ncu-case", choices=("gemm_down", "attention"), default=None,
+    ap.add_argument("--workload", choices=tuple(WORKLOADS), default=synth.STEP1024.name,
+                    help="step_1024px (default): one uncached 1024^2 step per iteration, plus "
+                         "a cached-prefix measurement; edit_1024px: the edit sequence; "
+                         "denoise40_2048px: the full 40-step 2048^2 denoise")
+    ap.add_argument("--ncu-case", choices=("gemms", "gemm_down", "attention"), default=None,
                     help="launch one kernel a few times (for ncu captures) and exit")
     args = ap.parse_args()
     if args.ncu_case:

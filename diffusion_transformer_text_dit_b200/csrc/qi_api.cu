@@ -161,7 +161,6 @@ struct BlockBufs {
   int8_t* uq;       // [T, max(H, F)]
   float* sa;        // [T]
   int32_t* zp;      // [T]
-  uint16_t* qkv;    // [T, 3H]
   uint16_t* q;      // [T, H]
   uint16_t* o;      // [T, H]
   uint16_t* g;      // [T, F]
@@ -175,7 +174,6 @@ BlockBufs carve_block(Carve& c, const qi_dims& d, int T) {
   b.uq = c.take<int8_t>(static_cast<size_t>(T) * W);
   b.sa = c.take<float>(T);
   b.zp = c.take<int32_t>(T);
-  b.qkv = c.take<uint16_t>(static_cast<size_t>(T) * 3 * H);
   b.q = c.take<uint16_t>(static_cast<size_t>(T) * H);
   b.o = c.take<uint16_t>(static_cast<size_t>(T) * H);
   b.g = c.take<uint16_t>(static_cast<size_t>(T) * F);

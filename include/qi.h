@@ -295,7 +295,7 @@ int qi_dit_block_forward(qi_ctx* ctx, const qi_dims* dims, const qi_block_weight
  * counterpart there.
  *   - Sizes whose scratch (qi_block_workspace_bytes) exceeds 16 MiB are rejected
  *     with QI_ERR_WORKSPACE before anything is launched (at hidden 256 / mlp
- *     1024 up to 2,974 rows fit; at hidden 4096 / mlp 16384 up to 186 rows).
+ *     1024 up to 4,071 rows fit; at hidden 4096 / mlp 16384 up to 255 rows).
  *   - The first call on a device looks up the array's device address (once,
  *     with that device current; the current device must be the context's).
  *     Make that first call before any stream capture.

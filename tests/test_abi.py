@@ -62,9 +62,9 @@ def test_sigma_schedule_matches_oracle(L):
 def test_workspace_sizes(L):
     d = qi.dims_struct(4096, 32, 16384, 64, 32)
     b = qi.qi_block_workspace_bytes(d, 4608)
-    # int8 [T,F] + qkv [T,3H] + q,o [T,H] + g [T,F] (bf16)
+    # int8 [T,F] + q,o [T,H] + g [T,F] (bf16)
     T, H, F = 4608, 4096, 16384
-    assert b >= T * F + 2 * T * (3 * H + 2 * H + F)
+    assert b >= T * F + 2 * T * (2 * H + F)
     s = qi.qi_step_workspace_bytes(d, 4608)
     assert s > b + 32 * 2 * T * H * 2
 

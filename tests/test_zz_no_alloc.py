@@ -59,10 +59,10 @@ def test_noalloc_block_matches_workspace_call_twice(ctx):
 
 
 def test_noalloc_rejects_rows_beyond_the_fixed_scratch(ctx):
-    cfg = synth.BLOCK512   # hidden 4096, mlp 16384: 186 rows fit in the 16 MiB scratch
+    cfg = synth.BLOCK512   # hidden 4096, mlp 16384: 255 rows fit in the 16 MiB scratch
     dims = qi.dims_struct(cfg.hidden, cfg.heads, cfg.mlp, cfg.patch, 1)
     bw = qi.qi_block_weights()   # never reached: the size check comes first
-    T = 187
+    T = 256
     g = qi.groups_struct([T], [1])
     dummy = torch.zeros(16, device="cuda")
     with pytest.raises(qi.QiError) as e:
