@@ -47,7 +47,11 @@ int fail(int code, const char* fmt, ...) {
 }
 
 int cuda_fail(const char* what) {
-  const cudaError_t e = cudaGetLastError();
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) {   // already read by the launcher
+    e = qi::last_launch_error();
+    qi::last_launch_error() = cudaSuccess;
+  }
   return fail(QI_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 

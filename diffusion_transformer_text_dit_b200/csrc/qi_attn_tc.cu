@@ -379,9 +379,10 @@ int launch_attention(const AttnParams& p, cudaStream_t st) {
   if (p.Sq == 0) return 0;
   static bool attr = false;
   if (!attr) {
-    if (cudaFuncSetAttribute(fa_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, FA_SMEM) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(fa_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, FA_SMEM) != cudaSuccess) {
+      launch_result();
       return -1;
+    }
     attr = true;
   }
   const int W = p.heads * 128;
@@ -395,7 +396,7 @@ int launch_attention(const AttnParams& p, cudaStream_t st) {
     return -2;
   dim3 grid((p.Sq + 2 * FA_ROWS - 1) / (2 * FA_ROWS), p.heads);
   fa_kernel<<<grid, FA_THREADS, FA_SMEM, st>>>(tq, tk, tv, p);
-  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+  return launch_result();
 }
 
 }  // namespace qi

@@ -437,15 +437,16 @@ static int launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const Gem
   auto kern = gemm_kernel<I8, BN, EPI>;
   static bool attr_set = false;   // per instantiation
   if (!attr_set) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess) {
+      launch_result();
       return -1;
+    }
     attr_set = true;
   }
   const int tiles = ((p.M + GEMM_BM - 1) / GEMM_BM) * ((p.N + BN - 1) / BN);
   const int grid = tiles < num_sms ? tiles : num_sms;
   kern<<<grid, GEMM_THREADS, C::SMEM_BYTES, st>>>(ta, tb, p);
-  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+  return launch_result();
 }
 
 template <bool I8, int EPI>

@@ -10,6 +10,19 @@
 
 namespace qi {
 
+// The CUDA error of the last failed launch on this thread (launchers return -1
+// after reading and clearing cudaGetLastError; the C ABI reports this one).
+inline cudaError_t& last_launch_error() {
+  static thread_local cudaError_t e = cudaSuccess;
+  return e;
+}
+inline int launch_result() {
+  const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) return 0;
+  last_launch_error() = e;
+  return -1;
+}
+
 enum GemmEpilogue {
   EPI_BF16 = 0,    // y (bf16) = value
   EPI_GELU = 1,    // y (bf16) = GELU_tanh(bf16(value))

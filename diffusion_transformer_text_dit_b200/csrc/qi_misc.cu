@@ -66,7 +66,7 @@ int launch_qk_norm_rope(const QkNormRopeParams& p, cudaStream_t st) {
   if (p.T == 0) return 0;
   if (p.d != 128) return -1;
   qk_norm_rope_kernel<<<p.T, 256, 0, st>>>(p);
-  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+  return launch_result();
 }
 
 // ---------------------------------------------------------------- GEMV
@@ -172,9 +172,10 @@ int launch_gemv(const GemvParams& p, cudaStream_t st) {
   const size_t smem = static_cast<size_t>(p.R) * p.k * sizeof(float);
   static bool attr = false;
   if (!attr) {
-    if (cudaFuncSetAttribute(gemv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(gemv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024) != cudaSuccess) {
+      launch_result();
       return -1;
+    }
     attr = true;
   }
   if (smem > 64 * 1024) return -1;
@@ -186,7 +187,7 @@ int launch_gemv(const GemvParams& p, cudaStream_t st) {
   const int max_grid = sms * 8;
   if (grid > max_grid) grid = max_grid;
   gemv_kernel<<<grid, GEMV_THREADS, smem, st>>>(p);
-  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+  return launch_result();
 }
 
 // ---------------------------------------------------------------- small kernels
@@ -204,7 +205,7 @@ __global__ void timestep_embedding_kernel(float t0, float t1, float* out) {
 
 int launch_timestep_embedding(float t0, float t1, float* out, cudaStream_t st) {
   timestep_embedding_kernel<<<2, 128, 0, st>>>(t0, t1, out);
-  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+  return launch_result();
 }
 
 __global__ void f32_to_bf16_kernel(const float* __restrict__ x, uint16_t* __restrict__ y, int64_t n) {
@@ -220,7 +221,7 @@ int launch_f32_to_bf16(const float* x, uint16_t* y, int64_t n, cudaStream_t st) 
   int64_t g = (n + 255) / 256;
   if (g > 148 * 16) g = 148 * 16;
   f32_to_bf16_kernel<<<static_cast<int>(g), 256, 0, st>>>(x, y, n);
-  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+  return launch_result();
 }
 
 // x += dt * v in fp32, one rounding per operation (no fused multiply-add).
@@ -235,7 +236,7 @@ int launch_euler(float* x, const float* v, int64_t n, float dt, cudaStream_t st)
   int64_t g = (n + 255) / 256;
   if (g > 148 * 16) g = 148 * 16;
   euler_kernel<<<static_cast<int>(g), 256, 0, st>>>(x, v, n, dt);
-  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+  return launch_result();
 }
 
 // Failure-detection probe: wait on an mbarrier that nothing ever arrives on,
@@ -260,7 +261,7 @@ __global__ void timeout_probe_kernel(uint64_t limit_ns, int* status) {
 
 int launch_timeout_probe(uint64_t limit_ns, int* status, cudaStream_t st) {
   timeout_probe_kernel<<<1, 32, 0, st>>>(limit_ns, status);
-  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+  return launch_result();
 }
 
 }  // namespace qi

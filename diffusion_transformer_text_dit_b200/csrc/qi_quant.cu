@@ -267,7 +267,7 @@ int launch_quant(const QuantParams& p, cudaStream_t st) {
     if (p.ln) quant_kernel<false, true, false><<<grid, block, 0, st>>>(p);
     else quant_kernel<false, false, false><<<grid, block, 0, st>>>(p);
   }
-  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+  return launch_result();
 }
 
 // ---------------------------------------------------------------- weights
@@ -307,7 +307,7 @@ int launch_prepare_w8(const float* w, int n, int k, int8_t* q, float* s, int32_t
                       cudaStream_t st) {
   if (n == 0) return 0;
   prepare_w8_kernel<<<n, QT, 0, st>>>(w, k, q, s, rowsum);
-  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+  return launch_result();
 }
 
 }  // namespace qi
