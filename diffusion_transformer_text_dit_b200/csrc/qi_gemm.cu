@@ -64,16 +64,26 @@ __device__ __forceinline__ void dequant32_bf16(const GemmParams& p, const uint32
   }
 }
 
+// "Accumulator buffer drained" signal of one epilogue warp.  In a CTA pair
+// the barrier lives in the even CTA, whose thread issues the MMAs for both.
+template <bool PAIR>
+__device__ __forceinline__ void tempty_signal(uint32_t addr) {
+  if (PAIR)
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
+  else
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(addr) : "memory");
+}
+
 // Fused epilogue of the QKV projection: the W columns handled by one epilogue
 // warp are W/128 whole heads of q, k or v.  For q and k each head row is read from TMEM
 // twice: once for the sum of squares of its bf16 values, once to apply
 //   r = 1/sqrt(mean + eps), n = bf16(y r), y' = bf16(n w)     (cast before scale)
 //   (a, b) -> (bf16(a c - b s), bf16(a s + b c))              (RoPE, pair = column/2)
 // with explicitly rounded fp32 operations; v is stored as bf16(y).
-template <int W>
+template <int W, bool PAIR>
 __device__ __forceinline__ void qkv_epilogue(const GemmParams& p, uint32_t t_row, int m,
                                              bool row_ok, float sa, int32_t zp, int n0, int lane,
-                                             uint64_t* tempty_bar) {
+                                             uint32_t tempty_addr) {
   const int which = n0 / p.H;
   const int col0 = n0 - which * p.H;
   uint16_t* out = which == 0 ? p.q_out : (which == 1 ? p.k_out : p.v_out_bf16);
@@ -103,7 +113,7 @@ __device__ __forceinline__ void qkv_epilogue(const GemmParams& p, uint32_t t_row
       if (hh == W / 128 - 1 && c == 3) {   // this warp's last TMEM read of the accumulator
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(tempty_bar);
+        if (lane == 0) tempty_signal<PAIR>(tempty_addr);
       }
       if (!row_ok) continue;
       float y[32];
@@ -139,6 +149,150 @@ __device__ __forceinline__ void qkv_epilogue(const GemmParams& p, uint32_t t_row
 #pragma unroll
       for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
     }
+  }
+}
+
+// Epilogue of one accumulator tile, run by the 8 epilogue warps: warp
+// (quarter, half) reads TMEM lanes 32*quarter .. +31 (rows m0 + 32*quarter + lane)
+// and half `half` of the BN columns, signals the accumulator buffer free after
+// its last TMEM read, and writes the fused result.
+template <bool I8, int BN, int EPI, bool PAIR>
+__device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tmem_acc, int m0,
+                                              int n0, int quarter, int half, int lane,
+                                              uint32_t tempty_addr) {
+  const int row_in_tile = quarter * 32 + lane;
+  const int m = m0 + row_in_tile;
+  const bool row_ok = m < p.M;
+  float sa = 0.f;
+  int32_t zp = 0;
+  int rs = 0;
+  if (row_ok) {
+    if (I8) {
+      sa = p.s_a[m];
+      zp = p.zp_a[m];
+    }
+    if (EPI == EPI_GATED) rs = p.groups.row_set[group_of(p.groups, p.row0 + m)];
+  }
+  const uint32_t t_row = tmem_acc + (static_cast<uint32_t>(quarter * 32) << 16);
+  if constexpr (EPI == EPI_QKV) {
+    qkv_epilogue<BN / 2, PAIR>(p, t_row + half * (BN / 2), m, row_ok, sa, zp,
+                               n0 + half * (BN / 2), lane, tempty_addr);
+    return;
+  }
+  float rlo = 0.f, rhi = 0.f;   // GELU: row range of this warp's half tile
+#pragma unroll 1
+  for (int c = half * (BN / 64); c < (half + 1) * (BN / 64); ++c) {
+    uint32_t r[32];
+    tmem_ld32(t_row + c * 32, r);
+    if (c == (half + 1) * (BN / 64) - 1) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tempty_signal<PAIR>(tempty_addr);
+    }
+    const int nb = n0 + c * 32;
+    if (!row_ok || nb >= p.N) continue;
+    const int ncols = min(32, p.N - nb);
+    if (p.acc_debug) {
+      int4* dst = reinterpret_cast<int4*>(p.acc_debug + static_cast<size_t>(m) * p.N + nb);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (4 * j < ncols)
+          dst[j] = make_int4(static_cast<int>(r[4 * j]), static_cast<int>(r[4 * j + 1]),
+                             static_cast<int>(r[4 * j + 2]), static_cast<int>(r[4 * j + 3]));
+    }
+    float v[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const int n = nb + j;
+      const int nn = n < p.N ? n : p.N - 1;
+      const float b = p.bias ? bf16_bits_to_float(__ldg(p.bias + nn)) : 0.f;
+      if (I8) {
+        const int32_t corr = static_cast<int32_t>(r[j]) - zp * __ldg(p.rowsum + nn);
+        v[j] = fmaf(static_cast<float>(corr) * sa, __ldg(p.s_w + nn), b);
+      } else {
+        v[j] = __uint_as_float(r[j]) + b;
+      }
+    }
+    if (EPI == EPI_BF16 || EPI == EPI_GELU) {
+      uint16_t* dst = p.y + static_cast<size_t>(m) * p.ldy + nb;
+      uint32_t w[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        float a0 = v[2 * j], a1 = v[2 * j + 1];
+        if (EPI == EPI_GELU) {
+          a0 = bf16_round_f(gelu_tanh_f(bf16_round_f(a0)));
+          a1 = bf16_round_f(gelu_tanh_f(bf16_round_f(a1)));
+          if (8 * (j >> 2) < ncols) {   // the stored values' range for the quantizer
+            rlo = fminf(rlo, fminf(a0, a1));
+            rhi = fmaxf(rhi, fmaxf(a0, a1));
+          }
+        }
+        w[j] = pack_bf16x2(a0, a1);
+      }
+      if (ncols == 32) {
+        uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          d4[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+      } else {
+        // ragged N tail: ncols is a multiple of 16 (n % 16 == 0)
+        uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (8 * j < ncols)
+            d4[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+      }
+    } else if (EPI == EPI_GATED) {
+      // x += gate * bf16(y)  (fp32 residual stream)
+      float4* dst = reinterpret_cast<float4*>(p.yf + static_cast<size_t>(m) * p.ldyf + nb);
+      const uint4* g4 =
+          reinterpret_cast<const uint4*>(p.gate + static_cast<size_t>(rs) * p.gate_ld + nb);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (8 * j >= ncols) break;
+        const uint4 gr = __ldg(g4 + j);
+        const uint32_t gw[4] = {gr.x, gr.y, gr.z, gr.w};
+        float4 a = dst[2 * j], b = dst[2 * j + 1];
+        a.x += __uint_as_float(gw[0] << 16) * bf16_round_f(v[8 * j + 0]);
+        a.y += __uint_as_float(gw[0] & 0xFFFF0000u) * bf16_round_f(v[8 * j + 1]);
+        a.z += __uint_as_float(gw[1] << 16) * bf16_round_f(v[8 * j + 2]);
+        a.w += __uint_as_float(gw[1] & 0xFFFF0000u) * bf16_round_f(v[8 * j + 3]);
+        b.x += __uint_as_float(gw[2] << 16) * bf16_round_f(v[8 * j + 4]);
+        b.y += __uint_as_float(gw[2] & 0xFFFF0000u) * bf16_round_f(v[8 * j + 5]);
+        b.z += __uint_as_float(gw[3] << 16) * bf16_round_f(v[8 * j + 6]);
+        b.w += __uint_as_float(gw[3] & 0xFFFF0000u) * bf16_round_f(v[8 * j + 7]);
+        dst[2 * j] = a;
+        dst[2 * j + 1] = b;
+      }
+    } else if (EPI == EPI_F32) {
+      float4* dst = reinterpret_cast<float4*>(p.yf + static_cast<size_t>(m) * p.ldyf + nb);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (4 * j < ncols) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+    } else if (EPI == EPI_EULER) {
+      // FlowMatch Euler: x += (sigma_next - sigma) * v, fp32, no FMA
+      float4* lat = reinterpret_cast<float4*>(p.yf + static_cast<size_t>(m) * p.ldyf + nb);
+      float4* vo = p.v_out ? reinterpret_cast<float4*>(p.v_out + static_cast<size_t>(m) * p.ldyf + nb)
+                           : nullptr;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (4 * j >= ncols) break;
+        const float4 vv = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        if (vo) vo[j] = vv;
+        float4 x = lat[j];
+        x.x = __fadd_rn(x.x, __fmul_rn(p.dt, vv.x));
+        x.y = __fadd_rn(x.y, __fmul_rn(p.dt, vv.y));
+        x.z = __fadd_rn(x.z, __fmul_rn(p.dt, vv.z));
+        x.w = __fadd_rn(x.w, __fmul_rn(p.dt, vv.w));
+        lat[j] = x;
+      }
+    }
+  }
+  if (EPI == EPI_GELU && p.row_range && row_ok) {
+    // non-negative floats order like their bit patterns; 0 - lo and hi + 0
+    // turn a negative zero into +0 so it cannot win the unsigned max
+    atomicMax(p.row_range + 2 * static_cast<size_t>(m), __float_as_uint(__fsub_rn(0.0f, rlo)));
+    atomicMax(p.row_range + 2 * static_cast<size_t>(m) + 1, __float_as_uint(__fadd_rn(rhi, 0.0f)));
   }
 }
 
@@ -271,7 +425,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;
     const int half = (warp - 2) >> 2;          // 0: warps 2-5, 1: warps 6-9
-    const int row_in_tile = quarter * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
@@ -279,142 +432,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       const int n0 = (tile / m_tiles) * BN;
       if (!mbar_wait_warp(&tfull[acc], acc_phase, p.status)) break;
       tc_fence_after();
-      const int m = m0 + row_in_tile;
-      const bool row_ok = m < p.M;
-      float sa = 0.f;
-      int32_t zp = 0;
-      int rs = 0;
-      if (row_ok) {
-        if (I8) {
-          sa = p.s_a[m];
-          zp = p.zp_a[m];
-        }
-        if (EPI == EPI_GATED) rs = p.groups.row_set[group_of(p.groups, p.row0 + m)];
-      }
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                             static_cast<uint32_t>(acc * BN);
-      if constexpr (EPI == EPI_QKV) {
-        qkv_epilogue<BN / 2>(p, t_row + half * (BN / 2), m, row_ok, sa, zp, n0 + half * (BN / 2),
-                             lane, &tempty[acc]);
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
-        continue;
-      }
-      float rlo = 0.f, rhi = 0.f;   // GELU: row range of this warp's half tile
-#pragma unroll 1
-      for (int c = half * (BN / 64); c < (half + 1) * (BN / 64); ++c) {
-        uint32_t r[32];
-        tmem_ld32(t_row + c * 32, r);
-        if (c == (half + 1) * (BN / 64) - 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty[acc]);
-        }
-        const int nb = n0 + c * 32;
-        if (!row_ok || nb >= p.N) continue;
-        const int ncols = min(32, p.N - nb);
-        if (p.acc_debug) {
-          int4* dst = reinterpret_cast<int4*>(p.acc_debug + static_cast<size_t>(m) * p.N + nb);
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            if (4 * j < ncols)
-              dst[j] = make_int4(static_cast<int>(r[4 * j]), static_cast<int>(r[4 * j + 1]),
-                                 static_cast<int>(r[4 * j + 2]), static_cast<int>(r[4 * j + 3]));
-        }
-        float v[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int n = nb + j;
-          const int nn = n < p.N ? n : p.N - 1;
-          const float b = p.bias ? bf16_bits_to_float(__ldg(p.bias + nn)) : 0.f;
-          if (I8) {
-            const int32_t corr = static_cast<int32_t>(r[j]) - zp * __ldg(p.rowsum + nn);
-            v[j] = fmaf(static_cast<float>(corr) * sa, __ldg(p.s_w + nn), b);
-          } else {
-            v[j] = __uint_as_float(r[j]) + b;
-          }
-        }
-        if (EPI == EPI_BF16 || EPI == EPI_GELU) {
-          uint16_t* dst = p.y + static_cast<size_t>(m) * p.ldy + nb;
-          uint32_t w[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            float a0 = v[2 * j], a1 = v[2 * j + 1];
-            if (EPI == EPI_GELU) {
-              a0 = bf16_round_f(gelu_tanh_f(bf16_round_f(a0)));
-              a1 = bf16_round_f(gelu_tanh_f(bf16_round_f(a1)));
-              if (8 * (j >> 2) < ncols) {   // the stored values' range for the quantizer
-                rlo = fminf(rlo, fminf(a0, a1));
-                rhi = fmaxf(rhi, fmaxf(a0, a1));
-              }
-            }
-            w[j] = pack_bf16x2(a0, a1);
-          }
-          if (ncols == 32) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              d4[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
-          } else {
-            // ragged N tail: ncols is a multiple of 16 (n % 16 == 0)
-            uint4* d4 = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              if (8 * j < ncols)
-                d4[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
-          }
-        } else if (EPI == EPI_GATED) {
-          // x += gate * bf16(y)  (fp32 residual stream)
-          float4* dst = reinterpret_cast<float4*>(p.yf + static_cast<size_t>(m) * p.ldyf + nb);
-          const uint4* g4 =
-              reinterpret_cast<const uint4*>(p.gate + static_cast<size_t>(rs) * p.gate_ld + nb);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            if (8 * j >= ncols) break;
-            const uint4 gr = __ldg(g4 + j);
-            const uint32_t gw[4] = {gr.x, gr.y, gr.z, gr.w};
-            float4 a = dst[2 * j], b = dst[2 * j + 1];
-            a.x += __uint_as_float(gw[0] << 16) * bf16_round_f(v[8 * j + 0]);
-            a.y += __uint_as_float(gw[0] & 0xFFFF0000u) * bf16_round_f(v[8 * j + 1]);
-            a.z += __uint_as_float(gw[1] << 16) * bf16_round_f(v[8 * j + 2]);
-            a.w += __uint_as_float(gw[1] & 0xFFFF0000u) * bf16_round_f(v[8 * j + 3]);
-            b.x += __uint_as_float(gw[2] << 16) * bf16_round_f(v[8 * j + 4]);
-            b.y += __uint_as_float(gw[2] & 0xFFFF0000u) * bf16_round_f(v[8 * j + 5]);
-            b.z += __uint_as_float(gw[3] << 16) * bf16_round_f(v[8 * j + 6]);
-            b.w += __uint_as_float(gw[3] & 0xFFFF0000u) * bf16_round_f(v[8 * j + 7]);
-            dst[2 * j] = a;
-            dst[2 * j + 1] = b;
-          }
-        } else if (EPI == EPI_F32) {
-          float4* dst = reinterpret_cast<float4*>(p.yf + static_cast<size_t>(m) * p.ldyf + nb);
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            if (4 * j < ncols) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-        } else if (EPI == EPI_EULER) {
-          // FlowMatch Euler: x += (sigma_next - sigma) * v, fp32, no FMA
-          float4* lat = reinterpret_cast<float4*>(p.yf + static_cast<size_t>(m) * p.ldyf + nb);
-          float4* vo = p.v_out ? reinterpret_cast<float4*>(p.v_out + static_cast<size_t>(m) * p.ldyf + nb)
-                               : nullptr;
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            if (4 * j >= ncols) break;
-            const float4 vv = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-            if (vo) vo[j] = vv;
-            float4 x = lat[j];
-            x.x = __fadd_rn(x.x, __fmul_rn(p.dt, vv.x));
-            x.y = __fadd_rn(x.y, __fmul_rn(p.dt, vv.y));
-            x.z = __fadd_rn(x.z, __fmul_rn(p.dt, vv.z));
-            x.w = __fadd_rn(x.w, __fmul_rn(p.dt, vv.w));
-            lat[j] = x;
-          }
-        }
-      }
-      if (EPI == EPI_GELU && p.row_range && row_ok) {
-        // non-negative floats order like their bit patterns; 0 - lo and hi + 0
-        // turn a negative zero into +0 so it cannot win the unsigned max
-        atomicMax(p.row_range + 2 * static_cast<size_t>(m), __float_as_uint(__fsub_rn(0.0f, rlo)));
-        atomicMax(p.row_range + 2 * static_cast<size_t>(m) + 1, __float_as_uint(__fadd_rn(rhi, 0.0f)));
-      }
+      epilogue_tile<I8, BN, EPI, false>(p, tmem_base + static_cast<uint32_t>(acc * BN), m0, n0,
+                                        quarter, half, lane, smem_u32(&tempty[acc]));
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
@@ -425,6 +444,279 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- CTA-pair int8 GEMM
+//
+// Two CTAs of a cluster (one per SM) share one 256 x 256 tile: CTA r loads rows
+// m0 + 128 r .. +127 of A and rows n0 + 128 r .. +127 of B into its own shared
+// memory, and the even CTA issues tcgen05.mma.cta_group::2 (M = 256, N = 256),
+// which reads both CTAs' operands and accumulates rows 128 r .. +127 of the
+// tile into CTA r's TMEM.  Each SM then streams 256 bytes of operands per 128
+// bytes of K instead of 384, the operand traffic that bounds the single-CTA
+// 128 x 256 tile.  Barriers:
+//   full[s]   even CTA: both CTAs' TMA loads of stage s complete on it (the even
+//             CTA's producer arms it with the bytes of both)
+//   empty[s]  in each CTA: stage s of that CTA may be refilled (multicast commit)
+//   tfull[a]  in each CTA: accumulator buffer a is complete (multicast commit)
+//   tempty[a] even CTA: all 16 epilogue warps of the pair have drained buffer a
+
+constexpr int PAIR_STAGES = 6;
+constexpr int PAIR_A_BYTES = 128 * GEMM_BK_BYTES;
+constexpr int PAIR_B_BYTES = 128 * GEMM_BK_BYTES;
+constexpr int PAIR_STAGE_BYTES = PAIR_A_BYTES + PAIR_B_BYTES;
+constexpr int PAIR_SMEM_BYTES = 1024 + PAIR_STAGES * PAIR_STAGE_BYTES + 256;
+static_assert(2 * PAIR_STAGES + 5 <= 31, "barrier area");
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Address of the same shared-memory object in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+// Every thread of both CTAs; orders shared-memory and barrier set-up (release /
+// acquire at cluster scope).  The non-.aligned form: lanes may arrive apart.
+__device__ __forceinline__ void cluster_sync_all() {
+  __syncwarp();
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+  __syncwarp();
+}
+
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for a phase completed by arrivals from both CTAs of the pair.
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, int* status) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (has_error(status)) return false;
+    if (globaltimer_ns() - t0 > QI_WAIT_NS) {
+      set_error(status, QI_DEV_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// TMA tile load into this CTA's shared memory whose completion is counted on
+// an mbarrier of either CTA of the pair (`bar_cluster` is a shared::cluster
+// address).  Plain load: no multicast.
+__device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap* map, uint32_t bar_cluster,
+                                                 void* smem, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(x), "r"(y)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_i8_pair(uint32_t d_tmem, uint64_t a, uint64_t b,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
+}
+
+// Arrive on the barrier at this offset in every CTA of `mask` once all MMAs
+// issued so far by this thread have completed.
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar, uint16_t mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(smem_u32(bar)),
+      "h"(mask)
+      : "memory");
+}
+
+// TMEM allocation / release for a CTA pair: one warp of each CTA executes it;
+// the same columns are allocated in both SMs.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(dst)),
+               "r"(ncols));
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols));
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const GemmParams p) {
+  constexpr int BN = 256;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + PAIR_STAGES * PAIR_A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + PAIR_STAGES * PAIR_STAGE_BYTES);
+  uint64_t* full = bars;                          // [STAGES] (even CTA)
+  uint64_t* empty = bars + PAIR_STAGES;           // [STAGES]
+  uint64_t* tfull = bars + 2 * PAIR_STAGES;       // [2]
+  uint64_t* tempty = bars + 2 * PAIR_STAGES + 2;  // [2] (even CTA)
+  uint64_t* drain = bars + 2 * PAIR_STAGES + 4;   // MMA drain on the error path
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * PAIR_STAGES + 5);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const int pair = blockIdx.x >> 1;
+  const int num_pairs = gridDim.x >> 1;
+  const int m_tiles = (p.M + 2 * GEMM_BM - 1) / (2 * GEMM_BM);
+  const int n_tiles = (p.N + BN - 1) / BN;
+  const int num_tiles = m_tiles * n_tiles;
+  const int num_kb = p.num_kb;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < PAIR_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 2 * GEMM_EPI_WARPS);
+    }
+    mbar_init(drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, 2 * BN);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();   // barriers of both CTAs initialised before any remote arrive
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+        const int m0 = (tile % m_tiles) * (2 * GEMM_BM) + static_cast<int>(rank) * GEMM_BM;
+        const int n0 = (tile / m_tiles) * BN + static_cast<int>(rank) * (BN / 2);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, p.status)) { ok = false; break; }
+          const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * PAIR_STAGE_BYTES);
+          tma_load_2d_pair(&tmA, fb, sA + stage * PAIR_A_BYTES, kb * GEMM_BK_BYTES, m0);
+          tma_load_2d_pair(&tmB, fb, sB + stage * PAIR_B_BYTES, kb * GEMM_BK_BYTES, n0);
+          if (++stage == PAIR_STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        // Error path: the loads in flight must land before the CTAs exit.  The
+        // even CTA waits (bounded) on the full barriers it armed, which also
+        // count the odd CTA's bytes; the odd CTA, which cannot wait on the even
+        // CTA's barriers, gives its last loads a fixed 200 us.
+        if (rank == 0) {
+          for (int s = 0; s < PAIR_STAGES; ++s) {
+            const uint32_t par = (s < stage) ? phase : (phase ^ 1u);
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(&full[s], par) && globaltimer_ns() - t0 < QI_WAIT_NS) {
+            }
+          }
+        } else {
+          const uint64_t t0 = globaltimer_ns();
+          while (globaltimer_ns() - t0 < 200000ull) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc = umma_idesc(true, 2 * GEMM_BM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+        if (!mbar_wait_cluster(&tempty[acc], acc_phase ^ 1u, p.status)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&full[stage], phase, p.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t adesc = umma_desc_kmajor_sw128(smem_u32(sA + stage * PAIR_A_BYTES));
+          const uint64_t bdesc = umma_desc_kmajor_sw128(smem_u32(sB + stage * PAIR_B_BYTES));
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {   // 4 x 32 bytes of K per stage
+            const uint64_t off = static_cast<uint64_t>(k * 32) >> 4;
+            umma_i8_pair(d_tmem, adesc + off, bdesc + off, idesc, (kb | k) != 0);
+          }
+          umma_commit_pair(&empty[stage], 0x3);
+          if (++stage == PAIR_STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit_pair(&tfull[acc], 0x3);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      if (!ok) {
+        // make sure no MMA is still writing TMEM before it is released
+        umma_commit_pair(drain, 0x1);
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < QI_WAIT_NS) {
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = pair; tile < num_tiles; tile += num_pairs) {
+      const int m0 = (tile % m_tiles) * (2 * GEMM_BM) + static_cast<int>(rank) * GEMM_BM;
+      const int n0 = (tile / m_tiles) * BN;
+      if (!mbar_wait_warp(&tfull[acc], acc_phase, p.status)) break;
+      tc_fence_after();
+      epilogue_tile<true, BN, EPI, true>(p, tmem_base + static_cast<uint32_t>(acc * BN), m0, n0,
+                                         quarter, half, lane, mapa_shared(smem_u32(&tempty[acc]), 0));
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  // Neither CTA leaves (or frees TMEM) while the other may still read its
+  // shared memory, arrive on its barriers, or have MMAs writing its TMEM.
+  tc_fence_before();
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, 2 * BN);
   }
 }
 
@@ -446,6 +738,59 @@ static int launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const Gem
   const int tiles = ((p.M + GEMM_BM - 1) / GEMM_BM) * ((p.N + BN - 1) / BN);
   const int grid = tiles < num_sms ? tiles : num_sms;
   kern<<<grid, GEMM_THREADS, C::SMEM_BYTES, st>>>(ta, tb, p);
+  return launch_result();
+}
+
+
+// Clusters of two that can be resident at once (0 if the pair kernel cannot run).
+template <int EPI>
+static int pair_capacity() {
+  static int cap = -1;   // per instantiation
+  if (cap < 0) {
+    auto kern = gemm_pair_kernel<EPI>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PAIR_SMEM_BYTES) != cudaSuccess) {
+      launch_result();
+      return cap = 0;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = PAIR_SMEM_BYTES;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+      launch_result();
+      n = 0;
+    }
+    cap = n;
+  }
+  return cap;
+}
+
+template <int EPI>
+static int launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
+                            int max_pairs, cudaStream_t st) {
+  const int tiles = ((p.M + 2 * GEMM_BM - 1) / (2 * GEMM_BM)) * ((p.N + 255) / 256);
+  const int pairs = tiles < max_pairs ? tiles : max_pairs;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = PAIR_SMEM_BYTES;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, gemm_pair_kernel<EPI>, ta, tb, p);
   return launch_result();
 }
 
@@ -473,13 +818,36 @@ int launch_gemm(bool int8, int epi, const void* A, int lda, const void* B, int l
       int8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const int esz = int8 ? 1 : 2;
   const uint32_t box_inner = GEMM_BK_BYTES / esz;
+  // int8 GEMMs with 256-wide tiles run on CTA pairs (each CTA loads 128 rows
+  // of A and 128 of B); the rest on single CTAs.
+  int max_pairs = 0;
+  if (int8 && bn == 256 && !(epi == EPI_QKV && p.H % 256 != 0)) {
+    switch (epi) {
+      case EPI_BF16: max_pairs = pair_capacity<EPI_BF16>(); break;
+      case EPI_GELU: max_pairs = pair_capacity<EPI_GELU>(); break;
+      case EPI_GATED: max_pairs = pair_capacity<EPI_GATED>(); break;
+      case EPI_QKV: max_pairs = pair_capacity<EPI_QKV>(); break;
+    }
+    max_pairs = max_pairs < num_sms / 2 ? max_pairs : num_sms / 2;
+  }
+  const bool use_pair = max_pairs > 0;
   CUtensorMap ta, tb;
   if (!make_tmap_2d(&ta, A, dt, static_cast<uint64_t>(p.K), static_cast<uint64_t>(p.M),
                     static_cast<uint64_t>(lda) * esz, box_inner, GEMM_BM))
     return -2;
   if (!make_tmap_2d(&tb, B, dt, static_cast<uint64_t>(p.K), static_cast<uint64_t>(p.N),
-                    static_cast<uint64_t>(ldb) * esz, box_inner, static_cast<uint32_t>(bn)))
+                    static_cast<uint64_t>(ldb) * esz, box_inner,
+                    static_cast<uint32_t>(use_pair ? bn / 2 : bn)))
     return -2;
+  if (use_pair) {
+    switch (epi) {
+      case EPI_BF16: return launch_gemm_pair<EPI_BF16>(ta, tb, p, max_pairs, st);
+      case EPI_GELU: return launch_gemm_pair<EPI_GELU>(ta, tb, p, max_pairs, st);
+      case EPI_GATED: return launch_gemm_pair<EPI_GATED>(ta, tb, p, max_pairs, st);
+      case EPI_QKV: return launch_gemm_pair<EPI_QKV>(ta, tb, p, max_pairs, st);
+    }
+    return -1;
+  }
   if (int8) {
     switch (epi) {
       case EPI_BF16: return launch_gemm_bn<true, EPI_BF16>(bn, ta, tb, p, num_sms, st);
