@@ -106,6 +106,33 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Two fp32 lanes in one 64-bit register: the paired fp32 instructions of
+// sm_100 (fma.rn.f32x2, add.f32x2) halve the issue slots of the softmax.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+  return d;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 __device__ __forceinline__ int fa_key_limit(const GroupTable& g, int t) {
   return g.end[group_of(g, t)];
 }
@@ -278,17 +305,23 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
       const bool masked = k0 + FA_ROWS > kv_min;
       uint32_t r[128];
       tmem_ld128(tS, r);                     // the whole S row, read once
-      float mx = -INFINITY;
       if (masked) {
 #pragma unroll
-        for (int i = 0; i < 128; ++i) {
+        for (int i = 0; i < 128; ++i)
           if (k0 + i >= lim) r[i] = __float_as_uint(-INFINITY);
-          mx = fmaxf(mx, __uint_as_float(r[i]));
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 128; ++i) mx = fmaxf(mx, __uint_as_float(r[i]));
       }
+      // row maximum: 8 independent chains of three-input maxima (a single
+      // chain over 128 values would put the max latency 128 times on the
+      // softmax's critical path)
+      float m8[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) m8[k] = fmaxf(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1]));
+#pragma unroll
+      for (int i = 16; i < 128; i += 16)
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          m8[k] = fmax3(m8[k], __uint_as_float(r[i + 2 * k]), __uint_as_float(r[i + 2 * k + 1]));
+      const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
       const float mx2 = mx * sl2;
       // New reference maximum for this row if it grew by more than 8 (base 2).
       const bool grow = (j == 0) || (mx2 > m_ref + 8.0f);
@@ -315,18 +348,34 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         }
         tmem_st_wait();
       }
-      float sum = 0.f;
+      // P = 2^(s sl2 - m_ref): the scale-subtract as paired fp32 FMAs, the row
+      // sum in 4 paired partial sums (8 independent chains)
+      const uint64_t sl2x2 = f2_pack(sl2, sl2);
+      const uint64_t negm2 = f2_pack(-m_ref, -m_ref);
+      uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(r[32 * c + 2 * i]), sl2, -m_ref));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(r[32 * c + 2 * i + 1]), sl2, -m_ref));
-          sum += p0 + p1;
+          const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(r[32 * c + 2 * i]),
+                                             __uint_as_float(r[32 * c + 2 * i + 1])),
+                                     sl2x2, negm2);
+          float x0, x1;
+          f2_unpack(x2, x0, x1);
+          const float p0 = ex2_approx(x0);
+          const float p1 = ex2_approx(x1);
+          acc2[i & 3] = f2_add(acc2[i & 3], f2_pack(p0, p1));
           pk[i] = pack_bf16x2(p0, p1);
         }
         tmem_st16(tS + c * 16, pk);   // P (bf16) over the first 64 columns of S
+      }
+      float sum;
+      {
+        float a0, a1, b0, b1;
+        f2_unpack(f2_add(acc2[0], acc2[1]), a0, a1);
+        f2_unpack(f2_add(acc2[2], acc2[3]), b0, b1);
+        sum = (a0 + b0) + (a1 + b1);
       }
       l += sum;
       tmem_st_wait();

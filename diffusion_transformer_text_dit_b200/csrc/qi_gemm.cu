@@ -34,8 +34,9 @@ struct GemmCfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = (BN == 256) ? 4 : (BN == 128 ? 6 : 8);
   static constexpr int TMEM_COLS = (2 * BN < 32) ? 32 : 2 * BN;
-  static constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + 256;
-  static_assert(2 * STAGES + 5 <= 31, "barrier area");
+  static constexpr int COL_BYTES = 2 * BN * 12;   // two tiles of (s_w, rowsum, bias)
+  static constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + 256 + COL_BYTES;
+  static_assert(2 * STAGES + 8 <= 32, "barrier area");
 };
 
 // GELU, tanh form: 0.5 x (1 + tanh(z)), z = sqrt(2/pi) (x + 0.044715 x^3).
@@ -51,17 +52,77 @@ __device__ __forceinline__ float gelu_tanh_f(float x) {
   return __fdividef(x, 1.0f + e);
 }
 
-// W8A8 dequantization of 32 accumulator columns starting at column nb,
-// rounded to bf16 (the Linear's output dtype).
-__device__ __forceinline__ void dequant32_bf16(const GemmParams& p, const uint32_t (&r)[32], int nb,
-                                               float sa, int32_t zp, float (&y)[32]) {
+// Per-column constants of one tile (s_w, rowsum, bias as fp32), staged in
+// shared memory by the epilogue warps so that each output element reads them
+// with broadcast 16-byte loads instead of three global loads.  Indexed by the
+// column's offset in the tile; columns past N hold zeros.
+struct ColTable {
+  const float* sw;
+  const int32_t* rs;
+  const float* b;
+};
+
+// Dequantise 32 accumulator columns (tile offset c0, a multiple of 32):
+//   v = (acc - zp rowsum) s_a s_w + bias      (kind::i8)
+//   v = acc + bias                            (kind::f16)
+template <bool I8>
+__device__ __forceinline__ void dequant32(const ColTable& t, const uint32_t (&r)[32], int c0,
+                                          float sa, int32_t zp, float (&v)[32]) {
+  const float4* sw4 = reinterpret_cast<const float4*>(t.sw + c0);
+  const int4* rs4 = reinterpret_cast<const int4*>(t.rs + c0);
+  const float4* b4 = reinterpret_cast<const float4*>(t.b + c0);
 #pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    const int n = nb + j;
-    const float b = p.bias ? bf16_bits_to_float(__ldg(p.bias + n)) : 0.f;
-    const int32_t corr = static_cast<int32_t>(r[j]) - zp * __ldg(p.rowsum + n);
-    y[j] = bf16_round_f(fmaf(static_cast<float>(corr) * sa, __ldg(p.s_w + n), b));
+  for (int q = 0; q < 8; ++q) {
+    const float4 bb = b4[q];
+    const float bv[4] = {bb.x, bb.y, bb.z, bb.w};
+    if (I8) {
+      const float4 ww = sw4[q];
+      const int4 rr = rs4[q];
+      const float wv[4] = {ww.x, ww.y, ww.z, ww.w};
+      const int32_t rv[4] = {rr.x, rr.y, rr.z, rr.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int32_t corr = static_cast<int32_t>(r[4 * q + e]) - zp * rv[e];
+        v[4 * q + e] = fmaf(static_cast<float>(corr) * sa, wv[e], bv[e]);
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) v[4 * q + e] = __uint_as_float(r[4 * q + e]) + bv[e];
+    }
   }
+}
+
+// W8A8 dequantization of 32 accumulator columns rounded to bf16 (the
+// Linear's output dtype).
+__device__ __forceinline__ void dequant32_bf16(const ColTable& t, const uint32_t (&r)[32], int c0,
+                                               float sa, int32_t zp, float (&y)[32]) {
+  dequant32<true>(t, r, c0, sa, zp, y);
+#pragma unroll
+  for (int j = 0; j < 32; ++j) y[j] = bf16_round_f(y[j]);
+}
+
+// Stage the constants of the tile's columns n0 .. n0 + BN - 1 (the 256
+// epilogue threads, numbered et = 0 .. 255) and arrive on `ready` (one arrival
+// per epilogue warp); the caller then waits on `ready` with a bounded wait.
+// Buffers alternate with the accumulator buffer: a warp writes the buffer of
+// tile i + 2 only after the wait of tile i + 1, which needs every warp's
+// arrival for tile i + 1, made after that warp finished tile i.
+template <bool I8, int BN>
+__device__ __forceinline__ void stage_columns(const GemmParams& p, float* sw, int32_t* rs, float* b,
+                                              int n0, int et, uint64_t* ready) {
+#pragma unroll 1
+  for (int c = et; c < BN; c += 32 * GEMM_EPI_WARPS) {
+    const int n = n0 + c;
+    const bool in = n < p.N;
+    if (I8) {
+      sw[c] = in ? __ldg(p.s_w + n) : 0.f;
+      rs[c] = in ? __ldg(p.rowsum + n) : 0;
+    }
+    b[c] = (in && p.bias) ? bf16_bits_to_float(__ldg(p.bias + n)) : 0.f;
+  }
+  __threadfence_block();
+  __syncwarp();
+  if ((et & 31) == 0) mbar_arrive(ready);
 }
 
 // "Accumulator buffer drained" signal of one epilogue warp.  In a CTA pair
@@ -81,9 +142,9 @@ __device__ __forceinline__ void tempty_signal(uint32_t addr) {
 //   (a, b) -> (bf16(a c - b s), bf16(a s + b c))              (RoPE, pair = column/2)
 // with explicitly rounded fp32 operations; v is stored as bf16(y).
 template <int W, bool PAIR>
-__device__ __forceinline__ void qkv_epilogue(const GemmParams& p, uint32_t t_row, int m,
-                                             bool row_ok, float sa, int32_t zp, int n0, int lane,
-                                             uint32_t tempty_addr) {
+__device__ __forceinline__ void qkv_epilogue(const GemmParams& p, const ColTable& ct, int cb,
+                                             uint32_t t_row, int m, bool row_ok, float sa,
+                                             int32_t zp, int n0, int lane, uint32_t tempty_addr) {
   const int which = n0 / p.H;
   const int col0 = n0 - which * p.H;
   uint16_t* out = which == 0 ? p.q_out : (which == 1 ? p.k_out : p.v_out_bf16);
@@ -99,7 +160,7 @@ __device__ __forceinline__ void qkv_epilogue(const GemmParams& p, uint32_t t_row
         tmem_ld32(t_row + hh * 128 + c * 32, r);
         if (row_ok) {
           float y[32];
-          dequant32_bf16(p, r, n0 + hh * 128 + c * 32, sa, zp, y);
+          dequant32_bf16(ct, r, cb + hh * 128 + c * 32, sa, zp, y);
 #pragma unroll
           for (int j = 0; j < 32; ++j) ss = __fadd_rn(ss, __fmul_rn(y[j], y[j]));
         }
@@ -117,7 +178,7 @@ __device__ __forceinline__ void qkv_epilogue(const GemmParams& p, uint32_t t_row
       }
       if (!row_ok) continue;
       float y[32];
-      dequant32_bf16(p, r, n0 + hh * 128 + c * 32, sa, zp, y);
+      dequant32_bf16(ct, r, cb + hh * 128 + c * 32, sa, zp, y);
       uint32_t pk[16];
       if (which < 2) {
         const float4* c4 = reinterpret_cast<const float4*>(p.rcos + static_cast<size_t>(m) * 64 + c * 16);
@@ -157,9 +218,9 @@ __device__ __forceinline__ void qkv_epilogue(const GemmParams& p, uint32_t t_row
 // and half `half` of the BN columns, signals the accumulator buffer free after
 // its last TMEM read, and writes the fused result.
 template <bool I8, int BN, int EPI, bool PAIR>
-__device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tmem_acc, int m0,
-                                              int n0, int quarter, int half, int lane,
-                                              uint32_t tempty_addr) {
+__device__ __forceinline__ void epilogue_tile(const GemmParams& p, const ColTable& ct,
+                                              uint32_t tmem_acc, int m0, int n0, int quarter,
+                                              int half, int lane, uint32_t tempty_addr) {
   const int row_in_tile = quarter * 32 + lane;
   const int m = m0 + row_in_tile;
   const bool row_ok = m < p.M;
@@ -175,8 +236,8 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tmem
   }
   const uint32_t t_row = tmem_acc + (static_cast<uint32_t>(quarter * 32) << 16);
   if constexpr (EPI == EPI_QKV) {
-    qkv_epilogue<BN / 2, PAIR>(p, t_row + half * (BN / 2), m, row_ok, sa, zp,
-                               n0 + half * (BN / 2), lane, tempty_addr);
+    qkv_epilogue<BN / 2, PAIR>(p, ct, half * (BN / 2), t_row + half * (BN / 2), m, row_ok, sa,
+                               zp, n0 + half * (BN / 2), lane, tempty_addr);
     return;
   }
   float rlo = 0.f, rhi = 0.f;   // GELU: row range of this warp's half tile
@@ -201,18 +262,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tmem
                              static_cast<int>(r[4 * j + 2]), static_cast<int>(r[4 * j + 3]));
     }
     float v[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const int n = nb + j;
-      const int nn = n < p.N ? n : p.N - 1;
-      const float b = p.bias ? bf16_bits_to_float(__ldg(p.bias + nn)) : 0.f;
-      if (I8) {
-        const int32_t corr = static_cast<int32_t>(r[j]) - zp * __ldg(p.rowsum + nn);
-        v[j] = fmaf(static_cast<float>(corr) * sa, __ldg(p.s_w + nn), b);
-      } else {
-        v[j] = __uint_as_float(r[j]) + b;
-      }
-    }
+    dequant32<I8>(ct, r, c * 32, sa, zp, v);
     if (EPI == EPI_BF16 || EPI == EPI_GELU) {
       uint16_t* dst = p.y + static_cast<size_t>(m) * p.ldy + nb;
       uint32_t w[16];
@@ -313,6 +363,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   uint64_t* tempty = bars + 2 * C::STAGES + 2; // [2]
   uint64_t* drain = bars + 2 * C::STAGES + 4;  // MMA drain on the error path
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 5);
+  uint64_t* cols_ready = bars + 2 * C::STAGES + 6;   // [2] column tables staged
+  float* col_sw = reinterpret_cast<float*>(smem + C::STAGES * C::STAGE_BYTES + 256);   // [2][BN]
+  int32_t* col_rs = reinterpret_cast<int32_t*>(col_sw + 2 * BN);                        // [2][BN]
+  float* col_b = reinterpret_cast<float*>(col_rs + 2 * BN);                             // [2][BN]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -331,6 +385,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       mbar_init(&tempty[a], GEMM_EPI_WARPS);
     }
     mbar_init(drain, 1);
+    for (int a = 0; a < 2; ++a) mbar_init(&cols_ready[a], GEMM_EPI_WARPS);
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -430,9 +485,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       const int m0 = (tile % m_tiles) * GEMM_BM;
       const int n0 = (tile / m_tiles) * BN;
+      const ColTable ct{col_sw + acc * BN, col_rs + acc * BN, col_b + acc * BN};
+      stage_columns<I8, BN>(p, col_sw + acc * BN, col_rs + acc * BN, col_b + acc * BN, n0,
+                            threadIdx.x - 64, &cols_ready[acc]);
+      if (!mbar_wait_warp(&cols_ready[acc], acc_phase, p.status)) break;
       if (!mbar_wait_warp(&tfull[acc], acc_phase, p.status)) break;
       tc_fence_after();
-      epilogue_tile<I8, BN, EPI, false>(p, tmem_base + static_cast<uint32_t>(acc * BN), m0, n0,
+      epilogue_tile<I8, BN, EPI, false>(p, ct, tmem_base + static_cast<uint32_t>(acc * BN), m0, n0,
                                         quarter, half, lane, smem_u32(&tempty[acc]));
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
@@ -466,8 +525,9 @@ constexpr int PAIR_STAGES = 6;
 constexpr int PAIR_A_BYTES = 128 * GEMM_BK_BYTES;
 constexpr int PAIR_B_BYTES = 128 * GEMM_BK_BYTES;
 constexpr int PAIR_STAGE_BYTES = PAIR_A_BYTES + PAIR_B_BYTES;
-constexpr int PAIR_SMEM_BYTES = 1024 + PAIR_STAGES * PAIR_STAGE_BYTES + 256;
-static_assert(2 * PAIR_STAGES + 5 <= 31, "barrier area");
+constexpr int PAIR_COL_BYTES = 2 * 256 * 12;
+constexpr int PAIR_SMEM_BYTES = 1024 + PAIR_STAGES * PAIR_STAGE_BYTES + 256 + PAIR_COL_BYTES;
+static_assert(2 * PAIR_STAGES + 8 <= 32, "barrier area");
 
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
@@ -580,6 +640,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   uint64_t* tempty = bars + 2 * PAIR_STAGES + 2;  // [2] (even CTA)
   uint64_t* drain = bars + 2 * PAIR_STAGES + 4;   // MMA drain on the error path
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * PAIR_STAGES + 5);
+  uint64_t* cols_ready = bars + 2 * PAIR_STAGES + 6;   // [2] column tables staged
+  float* col_sw = reinterpret_cast<float*>(smem + PAIR_STAGES * PAIR_STAGE_BYTES + 256);   // [2][BN]
+  int32_t* col_rs = reinterpret_cast<int32_t*>(col_sw + 2 * BN);                            // [2][BN]
+  float* col_b = reinterpret_cast<float*>(col_rs + 2 * BN);                                 // [2][BN]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -599,6 +663,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], 2 * GEMM_EPI_WARPS);
+      mbar_init(&cols_ready[a], GEMM_EPI_WARPS);
     }
     mbar_init(drain, 1);
     fence_mbar_init();
@@ -701,9 +766,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     for (int tile = pair; tile < num_tiles; tile += num_pairs) {
       const int m0 = (tile % m_tiles) * (2 * GEMM_BM) + static_cast<int>(rank) * GEMM_BM;
       const int n0 = (tile / m_tiles) * BN;
+      const ColTable ct{col_sw + acc * BN, col_rs + acc * BN, col_b + acc * BN};
+      stage_columns<true, BN>(p, col_sw + acc * BN, col_rs + acc * BN, col_b + acc * BN, n0,
+                              threadIdx.x - 64, &cols_ready[acc]);
+      if (!mbar_wait_warp(&cols_ready[acc], acc_phase, p.status)) break;
       if (!mbar_wait_warp(&tfull[acc], acc_phase, p.status)) break;
       tc_fence_after();
-      epilogue_tile<true, BN, EPI, true>(p, tmem_base + static_cast<uint32_t>(acc * BN), m0, n0,
+      epilogue_tile<true, BN, EPI, true>(p, ct, tmem_base + static_cast<uint32_t>(acc * BN), m0, n0,
                                          quarter, half, lane, mapa_shared(smem_u32(&tempty[acc]), 0));
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
