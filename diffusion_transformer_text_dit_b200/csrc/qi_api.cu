@@ -270,7 +270,6 @@ int run_quant(qi_ctx* ctx, const void* x, bool xbf16, int M, int K, int ldx,
               const uint16_t* shift, const uint16_t* scale, int mod_ld, const qi::GroupTable& gt,
               int row0, float eps, int8_t* q, float* s, int32_t* zp, uint16_t* u_bf16,
               cudaStream_t st, const QuantExtras& ex = QuantExtras()) {
-  (void)ctx;
   qi::QuantParams p;
   memset(&p, 0, sizeof(p));
   p.res_y = ex.res_y;

@@ -25,8 +25,9 @@
 // exact in value because the final normalisation divides by the same sum.
 //
 // Warps: 0-3 softmax of tile A (TMEM lanes 0-127), 4-7 softmax of tile B,
-// 8 TMA producer, 9 TMEM allocator + MMA issuer.  K/V stream through a 2-stage
-// ring; every barrier wait is bounded (qi_common.cuh).
+// 8 TMA producer, 9 TMEM allocator + MMA issuer.  K streams through a 3-stage
+// ring (a stage is released once both S MMAs have read it), V through a
+// 2-stage ring; every barrier wait is bounded (qi_common.cuh).
 #include "qi_common.cuh"
 #include "qi_internal.h"
 
@@ -36,7 +37,9 @@ constexpr int FA_ROWS = 128;                   // rows per Q tile, keys per K/V 
 constexpr int FA_THREADS = 320;
 constexpr int FA_TILE = 128 * 128 * 2;         // 32 KB: 128 rows x 128 bf16
 constexpr int FA_HALF = FA_TILE / 2;           // one 64-column (128-byte) swizzle region
-constexpr int FA_SMEM = 1024 + 6 * FA_TILE + 256;
+constexpr int FA_KST = 3;                      // K ring stages
+constexpr int FA_VST = 2;                      // V ring stages
+constexpr int FA_SMEM = 1024 + (2 + FA_KST + FA_VST) * FA_TILE + 256;
 
 // MN-major operand with the 128-byte swizzle: 64 elements (128 B) contiguous
 // along N, K rows 128 B apart inside an 8-row group, 8-row groups 1024 B
@@ -106,33 +109,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-  float d;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-  return d;
-}
-
-// Two fp32 lanes in one 64-bit register: the paired fp32 instructions of
-// sm_100 (fma.rn.f32x2, add.f32x2) halve the issue slots of the softmax.
-__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
-  uint64_t d;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
-  return d;
-}
-__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-
 __device__ __forceinline__ int fa_key_limit(const GroupTable& g, int t) {
   return g.end[group_of(g, t)];
 }
@@ -144,19 +120,20 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
   extern __shared__ uint8_t fa_smem_raw[];
   const uint32_t raw_addr = smem_u32(fa_smem_raw);
   uint8_t* smem = fa_smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
-  uint8_t* sQ = smem;                      // [2][FA_TILE]: tile A, tile B
-  uint8_t* sK = smem + 2 * FA_TILE;        // [2 stages][FA_TILE]
-  uint8_t* sV = smem + 4 * FA_TILE;        // [2 stages][FA_TILE]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 6 * FA_TILE);
+  uint8_t* sQ = smem;                              // [2][FA_TILE]: tile A, tile B
+  uint8_t* sK = smem + 2 * FA_TILE;                // [FA_KST][FA_TILE]
+  uint8_t* sV = smem + (2 + FA_KST) * FA_TILE;     // [FA_VST][FA_TILE]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (2 + FA_KST + FA_VST) * FA_TILE);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;      // [2]
-  uint64_t* v_full = bars + 3;      // [2]
-  uint64_t* kv_empty = bars + 5;    // [2]
-  uint64_t* s_full = bars + 7;      // [2] per Q tile
-  uint64_t* p_full = bars + 9;      // [2] per Q tile
-  uint64_t* o_full = bars + 11;
-  uint64_t* drain = bars + 12;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  uint64_t* k_full = bars + 1;                     // [FA_KST]
+  uint64_t* k_empty = k_full + FA_KST;             // [FA_KST]
+  uint64_t* v_full = k_empty + FA_KST;             // [FA_VST]
+  uint64_t* v_empty = v_full + FA_VST;             // [FA_VST]
+  uint64_t* s_full = v_empty + FA_VST;             // [2] per Q tile
+  uint64_t* p_full = s_full + 2;                   // [2] per Q tile
+  uint64_t* o_full = p_full + 2;
+  uint64_t* drain = o_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_ctiles = (p.Sq + 2 * FA_ROWS - 1) / (2 * FA_ROWS);
@@ -171,10 +148,15 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < FA_KST; ++s) {
       mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < FA_VST; ++s) {
       mbar_init(&v_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&v_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
       mbar_init(&p_full[s], 128);
     }
@@ -204,31 +186,41 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         for (int half = 0; half < 2; ++half)
           tma_load_2d(&tmQ, q_full, sQ + t * FA_TILE + half * FA_HALF, hc + 64 * half,
                       q0 + t * FA_ROWS);
+      // K(j) into stage j % FA_KST once S_B(j - FA_KST) has read it; V(j) into
+      // stage j % FA_VST once PV_B(j - FA_VST) has.  K runs further ahead:
+      // the next S MMA needs it well before the next PV needs V.
       bool ok = true;
-      int j = 0;
-      for (; j < n_kv; ++j) {
-        const int st = j & 1;
-        if (!mbar_wait(&kv_empty[st], ((j >> 1) & 1) ^ 1u, status)) { ok = false; break; }
-        mbar_arrive_expect_tx(&k_full[st], FA_TILE);
+      int jk = 0, jv = 0;   // tiles whose loads were issued
+      for (int j = 0; j < n_kv; ++j) {
+        const int ks = j % FA_KST, kr = j / FA_KST;
+        if (!mbar_wait(&k_empty[ks], (kr & 1) ^ 1u, status)) { ok = false; break; }
+        mbar_arrive_expect_tx(&k_full[ks], FA_TILE);
         for (int half = 0; half < 2; ++half)
-          tma_load_2d(&tmK, &k_full[st], sK + st * FA_TILE + half * FA_HALF, hc + 64 * half,
+          tma_load_2d(&tmK, &k_full[ks], sK + ks * FA_TILE + half * FA_HALF, hc + 64 * half,
                       j * FA_ROWS);
-        mbar_arrive_expect_tx(&v_full[st], FA_TILE);
+        jk = j + 1;
+        const int vs = j % FA_VST, vr = j / FA_VST;
+        if (!mbar_wait(&v_empty[vs], (vr & 1) ^ 1u, status)) { ok = false; break; }
+        mbar_arrive_expect_tx(&v_full[vs], FA_TILE);
         for (int half = 0; half < 2; ++half)
-          tma_load_2d(&tmV, &v_full[st], sV + st * FA_TILE + half * FA_HALF, hc + 64 * half,
+          tma_load_2d(&tmV, &v_full[vs], sV + vs * FA_TILE + half * FA_HALF, hc + 64 * half,
                       j * FA_ROWS);
+        jv = j + 1;
       }
       if (!ok) {
-        // bounded drain of the loads already armed (Q and the last two K/V tiles)
+        // bounded drain of the loads already armed (Q, the last K and V tiles)
         const uint64_t t0 = globaltimer_ns();
         while (!mbar_try_wait(q_full, 0) && globaltimer_ns() - t0 < QI_WAIT_NS) {
         }
-        for (int jj = j - 2; jj < j; ++jj) {
-          if (jj < 0) continue;
-          const int st = jj & 1;
-          const uint32_t par = (jj >> 1) & 1;
+        for (int jj = (jk > FA_KST ? jk - FA_KST : 0); jj < jk; ++jj) {
           const uint64_t t1 = globaltimer_ns();
-          while (!(mbar_try_wait(&k_full[st], par) && mbar_try_wait(&v_full[st], par)) &&
+          while (!mbar_try_wait(&k_full[jj % FA_KST], (jj / FA_KST) & 1) &&
+                 globaltimer_ns() - t1 < QI_WAIT_NS) {
+          }
+        }
+        for (int jj = (jv > FA_VST ? jv - FA_VST : 0); jj < jv; ++jj) {
+          const uint64_t t1 = globaltimer_ns();
+          while (!mbar_try_wait(&v_full[jj % FA_VST], (jj / FA_VST) & 1) &&
                  globaltimer_ns() - t1 < QI_WAIT_NS) {
           }
         }
@@ -241,8 +233,8 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
       constexpr uint32_t idesc_pv = umma_idesc(false, 128, 128) | (1u << 16);   // B MN-major
       bool ok = mbar_wait(q_full, 0, status);
       auto issue_s = [&](int X, int jj) -> bool {
-        const int st = jj & 1;
-        if (!mbar_wait(&k_full[st], (jj >> 1) & 1, status)) return false;
+        const int st = jj % FA_KST;
+        if (!mbar_wait(&k_full[st], (jj / FA_KST) & 1, status)) return false;
         tc_fence_after();
         const uint32_t qa = smem_u32(sQ + X * FA_TILE), kb = smem_u32(sK + st * FA_TILE);
 #pragma unroll
@@ -255,8 +247,8 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         return true;
       };
       auto issue_pv = [&](int X, int jj) -> bool {
-        const int st = jj & 1;
-        if (!mbar_wait(&v_full[st], (jj >> 1) & 1, status)) return false;
+        const int st = jj % FA_VST;
+        if (!mbar_wait(&v_full[st], (jj / FA_VST) & 1, status)) return false;
         if (!mbar_wait(&p_full[X], jj & 1, status)) return false;
         tc_fence_after();
         const uint32_t vb = smem_u32(sV + st * FA_TILE);
@@ -267,13 +259,19 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
                       (jj > 0 || kk > 0) ? 1u : 0u);
         return true;
       };
-      if (ok && n_kv > 0) ok = issue_s(0, 0) && issue_s(1, 0);
+      if (ok && n_kv > 0) {
+        ok = issue_s(0, 0) && issue_s(1, 0);
+        if (ok) umma_commit(&k_empty[0]);
+      }
       for (int j = 0; ok && j < n_kv; ++j) {
         ok = issue_pv(0, j);
         if (ok && j + 1 < n_kv) ok = issue_s(0, j + 1);
         if (ok) ok = issue_pv(1, j);
-        if (ok) umma_commit(&kv_empty[j & 1]);
-        if (ok && j + 1 < n_kv) ok = issue_s(1, j + 1);
+        if (ok) umma_commit(&v_empty[j % FA_VST]);
+        if (ok && j + 1 < n_kv) {
+          ok = issue_s(1, j + 1);
+          if (ok) umma_commit(&k_empty[(j + 1) % FA_KST]);
+        }
       }
       if (ok) {
         umma_commit(o_full);

@@ -84,41 +84,93 @@ __device__ __forceinline__ float2 block_reduce2(float a, float b, float* red) {
   return make_float2(ra, rb);
 }
 
-template <bool XBF16>
-__device__ __forceinline__ void load8(const void* base, int64_t off, float* v) {
-  if (XBF16) {
-    const uint4 raw = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(base) + off);
-    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+// rint(v / s) for |v / s| <= 255 + rounding, by the exact IEEE quotient
+// (the rare elements near a rounding tie; kept out of line).
+__device__ __noinline__ int exact_code(float v, float s) { return __float2int_rn(__fdiv_rn(v, s)); }
+
+// Codes q = rint(v / s) + zp of 8 values (4 fp32 pairs), not yet saturated.
+// v * (1/s) is within ~3e-5 of the IEEE quotient (|v / s| <= 255), so it
+// rounds the same way unless its fraction lies within 1e-4 of one half; a
+// chunk holding such an element recomputes its codes from the exact quotient.
+// Rounding uses the 1.5 * 2^23 shifter: t + 1.5 * 2^23 rounds t to an integer
+// (ties to even, as rint) and leaves it in the low mantissa bits, so
+// q = bits(t + shifter) - bits(shifter) + zp.
+__device__ __forceinline__ void quant_codes8(const uint64_t (&v)[4], float inv_s, float s, int zp,
+                                             int (&q)[8]) {
+  constexpr float kShift = 12582912.0f;
+  const uint64_t inv2 = f2_pack(inv_s, inv_s), sh2 = f2_pack(kShift, kShift);
+  const int bias = 0x4B400000 - zp;
+  float worst = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint64_t t = f2_mul(v[i], inv2);
+    const uint64_t y = f2_add(t, sh2);
+    float f0, f1, y0, y1;
+    f2_unpack(f2_sub(t, f2_sub(y, sh2)), f0, f1);   // t - rint(t), exact
+    f2_unpack(y, y0, y1);
+    worst = fmax3(worst, fabsf(f0), fabsf(f1));
+    q[2 * i] = __float_as_int(y0) - bias;
+    q[2 * i + 1] = __float_as_int(y1) - bias;
+  }
+  if (worst > 0.4999f) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      v[2 * i] = __uint_as_float(w[i] << 16);
-      v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+      float e0, e1;
+      f2_unpack(v[i], e0, e1);
+      q[2 * i] = exact_code(e0, s) + zp;
+      q[2 * i + 1] = exact_code(e1, s) + zp;
     }
-  } else {
-    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(base) + off);
-    const float4 a = p[0], b = p[1];
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
   }
 }
 
+// Four codes, each saturated to [-128, 127], packed little-endian (a0 first).
+__device__ __forceinline__ uint32_t pack4_sat_s8(int a0, int a1, int a2, int a3) {
+  uint32_t hi, r;
+  asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, 0;" : "=r"(hi) : "r"(a3), "r"(a2));
+  asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a1), "r"(a0), "r"(hi));
+  return r;
+}
+
+// 8 bf16 values (one 16-byte load) as 4 fp32 pairs.
+__device__ __forceinline__ void load8_bf16_pairs(const uint16_t* p, uint64_t (&d)[4]) {
+  const uint4 raw = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) d[i] = f2_pack(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+}
+
 // One CTA per row with blockDim.x = max(32, K / 32) threads, each holding up
-// to QCH chunks of 8 consecutive elements: chunk c of thread t covers
-// [8 (t + c blockDim), +8), so each load instruction of a warp reads one
-// contiguous segment of the row.
+// to QCH chunks of 8 consecutive elements (as fp32 pairs): chunk c of thread t
+// covers [8 (t + c blockDim), +8), so each load instruction of a warp reads
+// one contiguous segment of the row.  The element-wise work uses the paired
+// fp32 instructions (IEEE-rounded per lane, so every value is what the scalar
+// formula gives).  (Measured on B200: this beats persistent blocks that
+// prefetch the next row into registers or through a bulk-copy ring; those hold
+// fewer warps per SM and the per-row barriers then dominate.)
 template <bool XBF16, bool LN, bool RANGE>
-__global__ void __launch_bounds__(1024) quant_kernel(const QuantParams p) {
+__global__ void __launch_bounds__(512) quant_kernel(const QuantParams p) {
   __shared__ float red[64];
   const int row = blockIdx.x;
   const int tid = threadIdx.x;
   const int nt = blockDim.x;
   const int nchunk = p.K >> 3;
-  float v[QCH][8];
+  uint64_t v[QCH][4];   // chunk c: elements (2i, 2i+1) in v[c][i]
 
 #pragma unroll
   for (int c = 0; c < QCH; ++c) {
     const int ch = tid + c * nt;
-    if (ch < nchunk) load8<XBF16>(p.x, static_cast<int64_t>(row) * p.ldx + ch * 8, v[c]);
+    if (ch >= nchunk) continue;
+    if (XBF16) {
+      load8_bf16_pairs(static_cast<const uint16_t*>(p.x) + static_cast<int64_t>(row) * p.ldx + ch * 8, v[c]);
+    } else {
+      const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(p.x) +
+                                                          static_cast<int64_t>(row) * p.ldx + ch * 8);
+      const float4 a = src[0], b = src[1];
+      v[c][0] = f2_pack(a.x, a.y);
+      v[c][1] = f2_pack(a.z, a.w);
+      v[c][2] = f2_pack(b.x, b.y);
+      v[c][3] = f2_pack(b.z, b.w);
+    }
   }
 
   if (LN && p.zero_range && tid == 0) {
@@ -136,28 +188,33 @@ __global__ void __launch_bounds__(1024) quant_kernel(const QuantParams p) {
 #pragma unroll
       for (int c = 0; c < QCH; ++c) {
         const int ch = tid + c * nt;
-        if (ch < nchunk) {
-          float fy[8], fg[8];
-          load8<true>(p.res_y, static_cast<int64_t>(row) * p.K + ch * 8, fy);
-          load8<true>(gt, ch * 8, fg);
+        if (ch >= nchunk) continue;
+        uint64_t fy[4], fg[4];
+        load8_bf16_pairs(p.res_y + static_cast<int64_t>(row) * p.K + ch * 8, fy);
+        load8_bf16_pairs(gt + ch * 8, fg);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) v[c][i] = fmaf(fg[i], fy[i], v[c][i]);
-          float4* o4 = reinterpret_cast<float4*>(xw + ch * 8);
-          o4[0] = make_float4(v[c][0], v[c][1], v[c][2], v[c][3]);
-          o4[1] = make_float4(v[c][4], v[c][5], v[c][6], v[c][7]);
-        }
+        for (int i = 0; i < 4; ++i) v[c][i] = f2_fma(fg[i], fy[i], v[c][i]);
+        float e[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) f2_unpack(v[c][i], e[2 * i], e[2 * i + 1]);
+        float4* o4 = reinterpret_cast<float4*>(xw + ch * 8);
+        o4[0] = make_float4(e[0], e[1], e[2], e[3]);
+        o4[1] = make_float4(e[4], e[5], e[6], e[7]);
       }
     }
-    float s = 0.f, ss = 0.f;
+    uint64_t s2 = 0ull, ss2 = 0ull;
 #pragma unroll
     for (int c = 0; c < QCH; ++c)
       if (tid + c * nt < nchunk)
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          s += v[c][i];
-          ss = fmaf(v[c][i], v[c][i], ss);
+        for (int i = 0; i < 4; ++i) {
+          s2 = f2_add(s2, v[c][i]);
+          ss2 = f2_fma(v[c][i], v[c][i], ss2);
         }
-    const float2 t = block_reduce2<false>(s, ss, red);
+    float s0, s1, q0, q1;
+    f2_unpack(s2, s0, s1);
+    f2_unpack(ss2, q0, q1);
+    const float2 t = block_reduce2<false>(s0 + s1, q0 + q1, red);
     const float inv_k = 1.0f / static_cast<float>(p.K);
     const float mean = t.x * inv_k;
     const float var = fmaxf(t.y * inv_k - mean * mean, 0.0f);
@@ -165,30 +222,33 @@ __global__ void __launch_bounds__(1024) quant_kernel(const QuantParams p) {
     const int rs = p.groups.row_set[group_of(p.groups, p.row0 + row)];
     const uint16_t* sh = p.shift + static_cast<int64_t>(rs) * p.mod_ld;
     const uint16_t* sc = p.scale + static_cast<int64_t>(rs) * p.mod_ld;
+    const uint64_t mean2 = f2_pack(mean, mean), rstd2 = f2_pack(rstd, rstd), one2 = f2_pack(1.0f, 1.0f);
+    // u = ((x - mean) rstd) (1 + scale) + shift
 #pragma unroll
     for (int c = 0; c < QCH; ++c) {
       const int ch = tid + c * nt;
-      if (ch < nchunk) {
-        float fsh[8], fsc[8];
-        load8<true>(sh, ch * 8, fsh);
-        load8<true>(sc, ch * 8, fsc);
+      if (ch >= nchunk) continue;
+      uint64_t fsh[4], fsc[4];
+      load8_bf16_pairs(sh + ch * 8, fsh);
+      load8_bf16_pairs(sc + ch * 8, fsc);
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          v[c][i] = fmaf((v[c][i] - mean) * rstd, 1.0f + fsc[i], fsh[i]);
-      }
+      for (int i = 0; i < 4; ++i)
+        v[c][i] = f2_fma(f2_mul(f2_sub(v[c][i], mean2), rstd2), f2_add(one2, fsc[i]), fsh[i]);
     }
     if (p.u_bf16) {   // modulated activation for a BF16 Linear
 #pragma unroll
       for (int c = 0; c < QCH; ++c) {
         const int ch = tid + c * nt;
-        if (ch < nchunk) {
-          uint4 o;
-          o.x = pack_bf16x2(v[c][0], v[c][1]);
-          o.y = pack_bf16x2(v[c][2], v[c][3]);
-          o.z = pack_bf16x2(v[c][4], v[c][5]);
-          o.w = pack_bf16x2(v[c][6], v[c][7]);
-          *reinterpret_cast<uint4*>(p.u_bf16 + static_cast<int64_t>(row) * p.ldq + ch * 8) = o;
+        if (ch >= nchunk) continue;
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float e0, e1;
+          f2_unpack(v[c][i], e0, e1);
+          w[i] = pack_bf16x2(e0, e1);
         }
+        *reinterpret_cast<uint4*>(p.u_bf16 + static_cast<int64_t>(row) * p.ldq + ch * 8) =
+            make_uint4(w[0], w[1], w[2], w[3]);
       }
       return;
     }
@@ -204,9 +264,11 @@ __global__ void __launch_bounds__(1024) quant_kernel(const QuantParams p) {
     for (int c = 0; c < QCH; ++c)
       if (tid + c * nt < nchunk)
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          lo = fminf(lo, v[c][i]);
-          hi = fmaxf(hi, v[c][i]);
+        for (int i = 0; i < 4; ++i) {
+          float e0, e1;
+          f2_unpack(v[c][i], e0, e1);
+          lo = fmin3(lo, e0, e1);
+          hi = fmax3(hi, e0, e1);
         }
     const float2 mm = block_reduce2<true>(lo, hi, red);
     lo = mm.x;
@@ -221,28 +283,15 @@ __global__ void __launch_bounds__(1024) quant_kernel(const QuantParams p) {
     const float z = rintf(__fsub_rn(-128.0f, __fdiv_rn(lo, s)));
     zp = static_cast<int>(fminf(fmaxf(z, -128.0f), 127.0f));
   }
-  // rint(u / s) with the IEEE quotient, computed as u * (1/s): |u/s| <= 255, so
-  // the product is within ~3e-5 of the exact quotient and rounds the same way
-  // unless its fraction is within 1e-4 of one half; those rare elements take
-  // the exact division.
   const float inv_s = __fdiv_rn(1.0f, s);
 #pragma unroll
   for (int c = 0; c < QCH; ++c) {
     const int ch = tid + c * nt;
-    if (ch < nchunk) {
-      uint32_t packed[2] = {0u, 0u};
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float t = v[c][i] * inv_s;
-        float rq = rintf(t);
-        if (fabsf(fabsf(t - rq) - 0.5f) < 1e-4f) rq = rintf(__fdiv_rn(v[c][i], s));
-        int qv = static_cast<int>(rq) + zp;
-        qv = max(-128, min(127, qv));
-        packed[i >> 2] |= (static_cast<uint32_t>(qv) & 0xFFu) << (8 * (i & 3));
-      }
-      *reinterpret_cast<uint2*>(p.q + static_cast<int64_t>(row) * p.ldq + ch * 8) =
-          make_uint2(packed[0], packed[1]);
-    }
+    if (ch >= nchunk) continue;
+    int qv[8];
+    quant_codes8(v[c], inv_s, s, zp, qv);
+    *reinterpret_cast<uint2*>(p.q + static_cast<int64_t>(row) * p.ldq + ch * 8) =
+        make_uint2(pack4_sat_s8(qv[0], qv[1], qv[2], qv[3]), pack4_sat_s8(qv[4], qv[5], qv[6], qv[7]));
   }
   if (tid == 0) {
     p.s[row] = s;
@@ -250,24 +299,27 @@ __global__ void __launch_bounds__(1024) quant_kernel(const QuantParams p) {
   }
 }
 
+template <bool XBF16, bool LN, bool RANGE>
+static int launch_quant_t(const QuantParams& p, int nt, cudaStream_t st) {
+  quant_kernel<XBF16, LN, RANGE><<<p.M, nt, 0, st>>>(p);
+  return launch_result();
+}
+
 int launch_quant(const QuantParams& p, cudaStream_t st) {
   if (p.M == 0) return 0;
-  if (p.K % 8 != 0 || p.K > 1024 * 8 * QCH) return -1;
+  if (p.K % 8 != 0 || p.K > 512 * 8 * QCH) return -1;   // K <= 16384
   int nt = (p.K / 8 + QCH - 1) / QCH;   // threads so that each holds <= QCH chunks
   nt = ((nt + 31) / 32) * 32;
   if (nt < 32) nt = 32;
-  dim3 grid(p.M), block(nt);
   if (p.ln && p.range) return -1;                 // LN computes its own range
   if (p.res_y && (!p.ln || p.x_bf16)) return -1;  // the residual add writes the fp32 stream
   if (p.x_bf16) {
-    if (p.ln) quant_kernel<true, true, false><<<grid, block, 0, st>>>(p);
-    else if (p.range) quant_kernel<true, false, true><<<grid, block, 0, st>>>(p);
-    else quant_kernel<true, false, false><<<grid, block, 0, st>>>(p);
-  } else {
-    if (p.ln) quant_kernel<false, true, false><<<grid, block, 0, st>>>(p);
-    else quant_kernel<false, false, false><<<grid, block, 0, st>>>(p);
+    if (p.ln) return launch_quant_t<true, true, false>(p, nt, st);
+    if (p.range) return launch_quant_t<true, false, true>(p, nt, st);
+    return launch_quant_t<true, false, false>(p, nt, st);
   }
-  return launch_result();
+  if (p.ln) return launch_quant_t<false, true, false>(p, nt, st);
+  return launch_quant_t<false, false, false>(p, nt, st);
 }
 
 // ---------------------------------------------------------------- weights
