@@ -261,7 +261,7 @@ def aggregate_throughput(world: int, steps: int, max_ms: float) -> float:
 
 # ------------------------------------------------------------------ GPU arm
 
-WORKLOADS = {c.name: c for c in (synth.STEP1024, synth.EDIT1024, synth.GEN2048)}
+WORKLOADS = {c.name: c for c in (synth.STEP1024, synth.EDIT1024, synth.EDIT3REF1024, synth.GEN2048)}
 
 
 def run_ours(args, rank, world, local_rank):
@@ -546,6 +546,7 @@ def main():
     ap.add_argument("--workload", choices=tuple(WORKLOADS), default=synth.STEP1024.name,
                     help="step_1024px (default): one uncached 1024^2 step per iteration, plus "
                          "a cached-prefix measurement; edit_1024px: the edit sequence; "
+                         "edit_3ref_1024px: an edit with three reference images; "
                          "denoise40_2048px: the full 40-step 2048^2 denoise")
     ap.add_argument("--ncu-case", choices=("gemms", "gemm_down", "attention"), default=None,
                     help="launch one kernel a few times (for ncu captures) and exit")

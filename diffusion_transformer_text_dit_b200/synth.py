@@ -28,7 +28,7 @@ from typing import Optional, Sequence, Tuple
 import torch
 
 __all__ = [
-    "Group", "DitConfig", "TINY", "BLOCK512", "STEP1024", "EDIT1024", "GEN2048",
+    "Group", "DitConfig", "TINY", "BLOCK512", "STEP1024", "EDIT1024", "EDIT3REF1024", "GEN2048",
     "CONFIGS", "gen", "linear_weight", "bias", "norm_weight", "latents",
     "text_features", "ref_latents", "hidden_states", "mod_table", "block_weights", "model_weights",
 ]
@@ -103,12 +103,18 @@ STEP1024 = DitConfig("step_1024px", 4096, 32, 128, 16384, 32, 64,
 EDIT1024 = DitConfig("edit_1024px", 4096, 32, 128, 16384, 32, 64,
                      (Group(_TEXT, 256), Group(_IMAGE, 1024, (32, 32)),
                       Group(_IMAGE, 4096, (64, 64))))
+# Multi-reference edit step: 256 text + three references (32x32, 32x32, 24x24)
+# + 4096 target tokens; each reference is its own group of the block-causal mask.
+EDIT3REF1024 = DitConfig("edit_3ref_1024px", 4096, 32, 128, 16384, 32, 64,
+                         (Group(_TEXT, 256), Group(_IMAGE, 1024, (32, 32)),
+                          Group(_IMAGE, 1024, (32, 32)), Group(_IMAGE, 576, (24, 24)),
+                          Group(_IMAGE, 4096, (64, 64))))
 # 40-step denoise at 2048x2048: 512 text + 16384 image tokens.
 GEN2048 = DitConfig("denoise40_2048px", 4096, 32, 128, 16384, 32, 64,
                     (Group(_TEXT, 512), Group(_IMAGE, 16384, (128, 128))),
                     steps=40, latent_seed=42)
 
-CONFIGS = {c.name: c for c in (TINY, BLOCK512, STEP1024, EDIT1024, GEN2048)}
+CONFIGS = {c.name: c for c in (TINY, BLOCK512, STEP1024, EDIT1024, EDIT3REF1024, GEN2048)}
 
 
 def gen(seed: int, *tags) -> torch.Generator:

@@ -63,8 +63,12 @@ class Setup:
     synth.TINY.replace(name="tiny_step_32blk", blocks=32),
     synth.TINY.replace(name="tiny_edit", blocks=2, patch=64,
                        groups=(synth.Group("text", 12), synth.Group("image", 16, (4, 4)),
+                               synth.Group("image", 64, (8, 8)))),
+    synth.TINY.replace(name="tiny_edit_3ref", blocks=2, patch=64,
+                       groups=(synth.Group("text", 12), synth.Group("image", 16, (4, 4)),
+                               synth.Group("image", 36, (6, 6)), synth.Group("image", 9, (3, 3)),
                                synth.Group("image", 64, (8, 8))))],
-    ids=["2blk", "32blk", "edit"])
+    ids=["2blk", "32blk", "edit", "edit_3ref"])
 def test_step_vs_oracle(ctx, cfg):
     s = Setup(ctx, cfg)
     sig = O.sigma_schedule(40, cfg.target_tokens)
@@ -76,11 +80,12 @@ def test_step_vs_oracle(ctx, cfg):
     assert np.array_equal(lat1.numpy(), O.euler_update(s.lat.numpy(), v.numpy(), sig[3], sig[4]))
 
 
-@pytest.mark.parametrize("edit", [False, True], ids=["text_image", "text_ref_image"])
+@pytest.mark.parametrize("edit", [0, 1, 3], ids=["text_image", "text_ref_image", "text_3ref_image"])
 def test_step_cached_equals_uncached(ctx, edit):
-    groups = ((synth.Group("text", 128), synth.Group("image", 64, (8, 8)),
-               synth.Group("image", 256, (16, 16))) if edit else
-              (synth.Group("text", 100), synth.Group("image", 256, (16, 16))))
+    refs = [synth.Group("image", 64, (8, 8)), synth.Group("image", 100, (10, 10)),
+            synth.Group("image", 48, (6, 8))][:edit]
+    groups = ((synth.Group("text", 128 if edit else 100),) + tuple(refs) +
+              (synth.Group("image", 256, (16, 16)),))
     cfg = synth.TINY.replace(name="cache", blocks=3, patch=64, groups=groups)
     s = Setup(ctx, cfg)
     sig = O.sigma_schedule(40, cfg.target_tokens)

@@ -204,6 +204,18 @@ def test_rope_positions_edit_frames_and_range():
     assert p[512:, 1].min() == -64 and p[512:, 1].max() == 63
 
 
+def test_rope_positions_multi_reference_frames():
+    # k-th image group at frame L + k: three references, then the target
+    groups = [("text", 5, None), ("image", 4, (2, 2)), ("image", 9, (3, 3)),
+              ("image", 6, (2, 3)), ("image", 16, (4, 4))]
+    pos = O.rope_positions(groups)
+    ends = np.cumsum([n for _, n, _ in groups])
+    for k, (a, b) in enumerate(zip(ends[:-1], ends[1:])):
+        assert np.all(pos[a:b, 0] == 5 + k)
+    # each image group is centred on its own grid, whatever precedes it
+    assert np.array_equal(pos[9:18, 1:], O.rope_positions([("image", 9, (3, 3))])[:, 1:])
+
+
 def test_rope_tables_axis_layout():
     pos = np.array([[5, -3, 7]])
     c, s = O.rope_tables(pos)
@@ -293,6 +305,23 @@ def test_attention_text_image_and_mask_invariance():
     out2 = O.attention_block_causal(q, k2, v2, g, g, 0.3)
     assert np.array_equal(out2[:12], out[:12])
     assert not np.allclose(out2[12:], out[12:])
+
+
+def test_attention_many_groups_reduce_to_full_attention_on_prefixes():
+    # [text | ref1 | ref2 | ref3 | target]: the rows of group g attend exactly
+    # like full (one-group) attention over the sequence cut at the end of g
+    ends = [4, 9, 12, 18, 27]
+    g = O.group_ids(ends)
+    q, k, v = (rng.standard_normal((27, 2, 8)) for _ in range(3))
+    out = O.attention_block_causal(q, k, v, g, g, 0.25)
+    start = 0
+    for e in ends:
+        sub = O.attention_block_causal(q[:e], k[:e], v[:e], np.zeros(e, np.int64),
+                                       np.zeros(e, np.int64), 0.25)
+        assert np.allclose(out[start:e], sub[start:e], atol=1e-12)
+        start = e
+    sc = 0.25 * math.sqrt(8)
+    assert np.allclose(out[9:12], _sdpa(q[9:12] * sc, k[:12], v[:12]), atol=1e-12)
 
 
 # ------------------------------------------------------------ timestep
