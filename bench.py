@@ -16,6 +16,7 @@ on the host cores (rank 0 only), a bounded sample per step.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import hashlib
 import json
@@ -43,7 +44,12 @@ CFG = synth.STEP1024
 def algorithmic_work(cfg: synth.DitConfig, cached: bool = False):
     """Per-step algorithmic work: int8 ops of the W8A8 Linears and bf16 FLOPs of
     the visible (unmasked) query-key pairs.  A cached step processes only the
-    target rows, which still attend over every key."""
+    target rows, which still attend over every key.  A true-CFG step does the
+    work of both of its sequences."""
+    if cfg.uncond_text:
+        a = algorithmic_work(dataclasses.replace(cfg, uncond_text=0), cached)
+        b = algorithmic_work(cfg.uncond(), cached)
+        return {k: a[k] + b[k] for k in a}
     H, F, d, h = cfg.hidden, cfg.mlp, cfg.head_dim, cfg.heads
     rows = cfg.target_tokens if cached else cfg.tokens
     per_block_ops = 2 * rows * (3 * H * H + H * H + F * H + H * F)
@@ -261,7 +267,8 @@ def aggregate_throughput(world: int, steps: int, max_ms: float) -> float:
 
 # ------------------------------------------------------------------ GPU arm
 
-WORKLOADS = {c.name: c for c in (synth.STEP1024, synth.EDIT1024, synth.EDIT3REF1024, synth.GEN2048)}
+WORKLOADS = {c.name: c for c in (synth.STEP1024, synth.EDIT1024, synth.EDIT3REF1024, synth.CFG1024,
+                                  synth.GEN2048)}
 
 
 def run_ours(args, rank, world, local_rank):
@@ -288,10 +295,29 @@ def run_ours(args, rank, world, local_rank):
     lat0 = synth.latents(cfg, device="cuda")
     lat = lat0.clone()
     stream = torch.cuda.current_stream()
+    if cfg.uncond_text:
+        # true CFG: the negative prompt's sequence, run in one batch with the prompt's
+        ucfg = cfg.uncond()
+        S_u = ucfg.tokens
+        gd_u = [(g.kind, g.tokens, g.grid) for g in ucfg.groups]
+        groups_u = qi.groups_struct(list(np.cumsum(ucfg.group_sizes())), ucfg.group_row_sets())
+        cos_u, sin_u = (t.cuda() for t in qi.qi_rope_tables(gd_u))
+        kv_u = torch.empty((cfg.blocks, 2, S_u, H), dtype=torch.bfloat16, device="cuda")
+        txt_u = synth.text_features(ucfg, device="cuda")
+        ws = torch.empty(qi.qi_step_cfg_workspace_bytes(dims, S, S_u, cfg.target_tokens),
+                         dtype=torch.uint8, device="cuda")
 
     def step(i, latents, text, mode=qi.QI_KV_NONE):
         j = i % 40
         cached = mode == qi.QI_KV_READ_PREFIX
+        if cfg.uncond_text:
+            sc = qi.seq_struct(None if cached else text, cfg.text_tokens, None if cached else ref,
+                               groups, cos, sin, None if mode == qi.QI_KV_NONE else kv)
+            su = qi.seq_struct(None if cached else txt_u, ucfg.text_tokens, None if cached else ref,
+                               groups_u, cos_u, sin_u, None if mode == qi.QI_KV_NONE else kv_u)
+            qi.qi_denoise_step_cfg(ctx, model, latents, sc, su, cfg.guidance, sig[j], sig[j + 1],
+                                   mode, None, ws)
+            return
         qi.qi_denoise_step(ctx, model, latents, None if cached else text, cfg.text_tokens,
                            None if cached else ref, groups, cos, sin, sig[j], sig[j + 1], mode,
                            None if mode == qi.QI_KV_NONE else kv, None, ws)
@@ -434,6 +460,8 @@ def run_ours(args, rank, world, local_rank):
 
     desc = (f"{cfg.name}: {cfg.blocks} blocks, hidden {H}, {cfg.heads}x128 heads, MLP {cfg.mlp}, "
             f"groups {'|'.join(str(n) for n in cfg.group_sizes())} tokens, "
+            + (f"true CFG with a {cfg.uncond_text}-token negative prompt in the same batch "
+               f"(scale {cfg.guidance}), " if cfg.uncond_text else "")
             + ("40-step FlowMatch Euler denoise, prefix K/V cached from step 2"
                if denoise else "uncached step")
             + ", all attn/MLP Linears W8A8 (int8 GEMMs, bf16 attention)")
@@ -547,6 +575,8 @@ def main():
                     help="step_1024px (default): one uncached 1024^2 step per iteration, plus "
                          "a cached-prefix measurement; edit_1024px: the edit sequence; "
                          "edit_3ref_1024px: an edit with three reference images; "
+                         "cfg_1024px: true classifier-free guidance (prompt + negative prompt "
+                         "as one batch); "
                          "denoise40_2048px: the full 40-step 2048^2 denoise")
     ap.add_argument("--ncu-case", choices=("gemms", "gemm_down", "attention"), default=None,
                     help="launch one kernel a few times (for ncu captures) and exit")

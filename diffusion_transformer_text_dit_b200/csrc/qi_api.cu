@@ -354,11 +354,27 @@ int run_bf16_linear(qi_ctx* ctx, const uint16_t* a, int M, int lda, const qi_lin
   return QI_OK;
 }
 
-int run_block(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, float* x, int T, int row0,
-              const uint16_t* mod, const qi::GroupTable& gt, int S, const float* cs,
-              const float* sn, uint16_t* kl, uint16_t* vl, uint8_t* ws, size_t ws_bytes,
-              cudaStream_t st) {
+// One sequence of a block batch: its processed rows are rows off .. off+T-1 of
+// the batch; they are rows row0 .. row0+T-1 of the sequence, whose S keys and
+// values live in kl / vl ([S, H] bf16 each) and whose groups define the mask.
+struct SeqAttn {
+  int off, T, row0, S;
+  qi::GroupTable gt;
+  uint16_t* kl;
+  uint16_t* vl;
+};
+
+// One block over the processed rows of up to two sequences (a true-CFG batch):
+// every Linear, quantizer and norm runs once over all T rows (rows_gt maps a
+// row, offset by rows_row0, to its modulation row set; cs/sn hold the RoPE
+// tables of the T rows); attention runs per sequence.
+int run_block_multi(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, float* x, int T,
+                    const qi::GroupTable& rows_gt, int rows_row0, const uint16_t* mod,
+                    const float* cs, const float* sn, const SeqAttn* seqs, int nseq, uint8_t* ws,
+                    size_t ws_bytes, cudaStream_t st) {
   const int H = d.hidden, F = d.mlp;
+  const qi::GroupTable& gt = rows_gt;
+  const int row0 = rows_row0;
   Carve c{ws, ws_bytes, 0};
   BlockBufs b = carve_block(c, d, T);
   const int mld = 6 * H;
@@ -393,8 +409,13 @@ int run_block(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, float* x
     p.rcos = cs;
     p.rsin = sn;
     p.q_out = b.q;
-    p.k_out = kl + static_cast<size_t>(row0) * H;
-    p.v_out_bf16 = vl + static_cast<size_t>(row0) * H;
+    p.k_out = seqs[0].kl + static_cast<size_t>(seqs[0].row0) * H;
+    p.v_out_bf16 = seqs[0].vl + static_cast<size_t>(seqs[0].row0) * H;
+    if (nseq > 1) {
+      p.kv_split = seqs[1].off;
+      p.k_out2 = seqs[1].kl + static_cast<size_t>(seqs[1].row0) * H;
+      p.v_out2 = seqs[1].vl + static_cast<size_t>(seqs[1].row0) * H;
+    }
     p.ldo = H;
     p.status = ctx->status;
     Prof pr(ctx, QI_KCLASS_GEMM_I8, st);
@@ -403,24 +424,25 @@ int run_block(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, float* x
     if (rr == -2) return fail(QI_ERR_CUDA, "cuTensorMapEncodeTiled failed (QKV operands)");
     if (rr != 0) return cuda_fail("QKV GEMM launch");
   }
-  qi::AttnParams ap;
-  memset(&ap, 0, sizeof(ap));
-  ap.q = b.q;
-  ap.k = kl;
-  ap.v = vl;
-  ap.o = b.o;
-  ap.ldq = H;
-  ap.ldkv = H;
-  ap.ldo = H;
-  ap.Sq = T;
-  ap.Sk = S;
-  ap.heads = d.heads;
-  ap.q_offset = row0;
-  ap.sm_scale = 1.0f / sqrtf(static_cast<float>(d.head_dim));
-  ap.groups = gt;
-  ap.row_range = b.o_range;
-  ap.status = ctx->status;
-  {
+  for (int sq = 0; sq < nseq; ++sq) {
+    const SeqAttn& q = seqs[sq];
+    qi::AttnParams ap;
+    memset(&ap, 0, sizeof(ap));
+    ap.q = b.q + static_cast<size_t>(q.off) * H;
+    ap.k = q.kl;
+    ap.v = q.vl;
+    ap.o = b.o + static_cast<size_t>(q.off) * H;
+    ap.ldq = H;
+    ap.ldkv = H;
+    ap.ldo = H;
+    ap.Sq = q.T;
+    ap.Sk = q.S;
+    ap.heads = d.heads;
+    ap.q_offset = q.row0;
+    ap.sm_scale = 1.0f / sqrtf(static_cast<float>(d.head_dim));
+    ap.groups = q.gt;
+    ap.row_range = b.o_range + 2 * static_cast<size_t>(q.off);
+    ap.status = ctx->status;
     Prof pr(ctx, QI_KCLASS_ATTN, st);
     const int r2 = qi::launch_attention(ap, st);
     if (r2 == -2) return fail(QI_ERR_CUDA, "cuTensorMapEncodeTiled failed (attention operands)");
@@ -463,6 +485,21 @@ int run_block(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, float* x
                     mod + 5 * H, mld, gt, row0, nullptr, st)))
     return r;
   return QI_OK;
+}
+
+int run_block(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, float* x, int T, int row0,
+              const uint16_t* mod, const qi::GroupTable& gt, int S, const float* cs,
+              const float* sn, uint16_t* kl, uint16_t* vl, uint8_t* ws, size_t ws_bytes,
+              cudaStream_t st) {
+  SeqAttn one;
+  one.off = 0;
+  one.T = T;
+  one.row0 = row0;
+  one.S = S;
+  one.gt = gt;
+  one.kl = kl;
+  one.vl = vl;
+  return run_block_multi(ctx, d, w, x, T, gt, row0, mod, cs, sn, &one, 1, ws, ws_bytes, st);
 }
 
 int check_block_weights(const qi_dims& d, const qi_block_weights* w) {
@@ -652,7 +689,7 @@ int qi_last_error(char* buf, size_t n) {
 int qi_prepare_w8(qi_ctx* ctx, const float* w, int n, int k, int8_t* q, float* s,
                   int32_t* rowsum, void* stream) {
   if (!ctx || !w || !q || !s || !rowsum) return fail(QI_ERR_INVALID_ARG, "NULL argument");
-  if (n < 0 || k < 8 || k % 8 != 0) return fail(QI_ERR_UNSUPPORTED_SHAPE, "need k % 8 == 0");
+  if (n < 0 || k < 8 || k % 8 != 0) return fail(QI_ERR_UNSUPPORTED_SHAPE, "need k %% 8 == 0");
   if (qi::launch_prepare_w8(w, n, k, q, s, rowsum, S(stream)) != 0)
     return cuda_fail("prepare_w8 launch");
   return QI_OK;
@@ -1036,6 +1073,230 @@ int qi_euler_update(qi_ctx* ctx, float* x, const float* v, int64_t n, float sigm
   if (!ctx || !x || !v || n < 0) return fail(QI_ERR_INVALID_ARG, "bad arguments");
   const float dt = sigma_next - sigma;
   if (qi::launch_euler(x, v, n, dt, S(stream)) != 0) return cuda_fail("euler launch");
+  return QI_OK;
+}
+
+
+// ---------------------------------------------------------------- true CFG step
+
+namespace {
+
+// A validated sequence of a CFG step.
+struct SeqPlan {
+  qi::GroupTable gt;
+  int S, P, N, L, R, row0, T;
+};
+
+int plan_seq(const qi_seq* q, int kv_mode, const char* which, SeqPlan* sp) {
+  int r;
+  if (!q || !q->rope_cos || !q->rope_sin)
+    return fail(QI_ERR_INVALID_ARG, "%s sequence: NULL argument", which);
+  if ((r = check_groups(q->groups, -1, &sp->gt))) return r;
+  const qi::GroupTable& gt = sp->gt;
+  if (gt.n < 2) return fail(QI_ERR_INVALID_ARG, "%s sequence needs a prefix and a target group", which);
+  for (int g = 0; g < gt.n; ++g)
+    if (gt.row_set[g] != (g == gt.n - 1 ? 1 : 0))
+      return fail(QI_ERR_INVALID_ARG, "%s sequence: row sets must be 0 for prefix groups and 1 for the target", which);
+  sp->S = gt.end[gt.n - 1];
+  sp->P = gt.end[gt.n - 2];
+  sp->N = sp->S - sp->P;
+  sp->L = q->text_tokens;
+  sp->R = sp->P - sp->L;
+  if (sp->L < 1 || sp->R < 0) return fail(QI_ERR_INVALID_ARG, "%s sequence: text_tokens outside the prefix", which);
+  if (kv_mode != QI_KV_READ_PREFIX && !q->txt) return fail(QI_ERR_INVALID_ARG, "%s sequence: txt is NULL", which);
+  if (sp->R > 0 && !q->ref_latents && kv_mode != QI_KV_READ_PREFIX)
+    return fail(QI_ERR_INVALID_ARG, "%s sequence holds reference tokens but ref_latents is NULL", which);
+  if (kv_mode != QI_KV_NONE && !q->kv_cache)
+    return fail(QI_ERR_INVALID_ARG, "%s sequence: kv_cache is required with prefix caching", which);
+  if ((q->txt && !aligned16(q->txt)) || (q->ref_latents && !aligned16(q->ref_latents)) ||
+      (q->kv_cache && !aligned16(q->kv_cache)) || !aligned16(q->rope_cos) || !aligned16(q->rope_sin))
+    return fail(QI_ERR_ALIGNMENT, "%s sequence: pointers must be 16-byte aligned", which);
+  sp->row0 = kv_mode == QI_KV_READ_PREFIX ? sp->P : 0;
+  sp->T = sp->S - sp->row0;
+  return QI_OK;
+}
+
+struct CfgBufs {
+  StepBufs sb;        // x [T, H], time-conditioning buffers, lat_bf16, u_final [2N, H], own K/V
+  float* cos;         // [T, 64] RoPE tables of the processed rows of both sequences
+  float* sin;
+  float* v;           // [2N, P] conditional then unconditional velocity
+};
+
+CfgBufs carve_cfg(Carve& c, const qi_dims& d, int T, int S_c, int S_u, int N, bool own_kv) {
+  CfgBufs b;
+  const size_t H = d.hidden, P = d.patch;
+  b.sb.x = c.take<float>(static_cast<size_t>(T) * H);
+  b.sb.emb = c.take<float>(2 * 256);
+  b.sb.h1 = c.take<float>(2 * H);
+  b.sb.temb = c.take<float>(2 * H);
+  b.sb.block_mod = c.take<uint16_t>(static_cast<size_t>(d.blocks) * 2 * 6 * H);
+  b.sb.final_mod = c.take<uint16_t>(2 * 2 * H);
+  b.sb.lat_bf16 = c.take<uint16_t>(static_cast<size_t>(S_c + S_u) * P);
+  b.sb.u_final = c.take<uint16_t>(static_cast<size_t>(2 * N) * H);
+  b.sb.kv = own_kv ? c.take<uint16_t>(static_cast<size_t>(d.blocks) * 2 * (S_c + S_u) * H) : nullptr;
+  b.cos = c.take<float>(static_cast<size_t>(T) * 64);
+  b.sin = c.take<float>(static_cast<size_t>(T) * 64);
+  b.v = c.take<float>(static_cast<size_t>(2 * N) * P);
+  b.sb.block_ws_bytes = block_bytes(d, T);
+  b.sb.block_ws = c.take<uint8_t>(b.sb.block_ws_bytes);
+  return b;
+}
+
+}  // namespace
+
+int qi_step_cfg_workspace_bytes(const qi_dims* dims, int S_cond, int S_uncond, int target_tokens,
+                                size_t* bytes) {
+  int r;
+  if ((r = check_dims(dims))) return r;
+  if (!bytes || S_cond < 1 || S_uncond < 1 || target_tokens < 1 || target_tokens > S_cond ||
+      target_tokens > S_uncond)
+    return fail(QI_ERR_INVALID_ARG, "bad arguments");
+  Carve c{nullptr, 0, 0};
+  carve_cfg(c, *dims, S_cond + S_uncond, S_cond, S_uncond, target_tokens, true);
+  *bytes = c.off + 256;
+  return QI_OK;
+}
+
+int qi_denoise_step_cfg(qi_ctx* ctx, const qi_model* model, float* latents, const qi_seq* cond,
+                        const qi_seq* uncond, float guidance, float sigma, float sigma_next,
+                        int kv_mode, float* v_out, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+  int r;
+  if (!ctx || !latents || !cond || !uncond || !workspace) return fail(QI_ERR_INVALID_ARG, "NULL argument");
+  if ((r = check_model(model))) return r;
+  if (kv_mode != QI_KV_NONE && kv_mode != QI_KV_WRITE_PREFIX && kv_mode != QI_KV_READ_PREFIX)
+    return fail(QI_ERR_INVALID_ARG, "bad kv_mode");
+  const qi_dims& d = model->dims;
+  SeqPlan sp[2];
+  if ((r = plan_seq(cond, kv_mode, "conditional", &sp[0]))) return r;
+  if ((r = plan_seq(uncond, kv_mode, "unconditional", &sp[1]))) return r;
+  if (sp[0].N != sp[1].N)
+    return fail(QI_ERR_INVALID_ARG, "both sequences must end in target groups of the same size");
+  if (!aligned16(latents) || !aligned16(workspace) || (v_out && !aligned16(v_out)))
+    return fail(QI_ERR_ALIGNMENT, "pointers must be 16-byte aligned");
+  const int N = sp[0].N, T = sp[0].T + sp[1].T;
+  // row -> modulation row set over the processed rows of both sequences
+  qi::GroupTable rows;
+  memset(&rows, 0, sizeof(rows));
+  if (kv_mode == QI_KV_READ_PREFIX) {
+    rows.n = 2;
+    rows.end[0] = sp[0].T;
+    rows.end[1] = T;
+    rows.row_set[0] = rows.row_set[1] = 1;
+  } else {
+    if (sp[0].gt.n + sp[1].gt.n > QI_MAX_GROUPS)
+      return fail(QI_ERR_UNSUPPORTED_SHAPE, "the two sequences hold more than %d groups together", QI_MAX_GROUPS);
+    for (int b = 0; b < 2; ++b)
+      for (int g = 0; g < sp[b].gt.n; ++g) {
+        rows.end[rows.n] = (b ? sp[0].S : 0) + sp[b].gt.end[g];
+        rows.row_set[rows.n] = sp[b].gt.row_set[g];
+        ++rows.n;
+      }
+  }
+  const bool own_kv = cond->kv_cache == nullptr || uncond->kv_cache == nullptr;
+  size_t need = 0;
+  {
+    Carve c{nullptr, 0, 0};
+    carve_cfg(c, d, T, sp[0].S, sp[1].S, N, own_kv);
+    need = c.off + 256;
+  }
+  if (workspace_bytes < need)
+    return fail(QI_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", workspace_bytes, need);
+
+  cudaStream_t st = S(stream);
+  const int H = d.hidden, P = d.patch;
+  Carve c{static_cast<uint8_t*>(workspace), workspace_bytes, 0};
+  CfgBufs b = carve_cfg(c, d, T, sp[0].S, sp[1].S, N, own_kv);
+  const qi_seq* seq[2] = {cond, uncond};
+  uint16_t* kv[2];
+  kv[0] = cond->kv_cache ? cond->kv_cache : b.sb.kv;
+  kv[1] = uncond->kv_cache ? uncond->kv_cache
+                           : b.sb.kv + static_cast<size_t>(d.blocks) * 2 * sp[0].S * H;
+  const int off[2] = {0, sp[0].T};
+
+  // RoPE rows of the processed rows, both sequences back to back
+  for (int q = 0; q < 2; ++q) {
+    const size_t n = static_cast<size_t>(sp[q].T) * 64 * sizeof(float);
+    const size_t so = static_cast<size_t>(sp[q].row0) * 64, dof = static_cast<size_t>(off[q]) * 64;
+    if (cudaMemcpyAsync(b.cos + dof, seq[q]->rope_cos + so, n, cudaMemcpyDeviceToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(b.sin + dof, seq[q]->rope_sin + so, n, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+      return cuda_fail("RoPE row copy");
+  }
+  if ((r = run_time_conditioning(ctx, *model, sigma, b.sb.block_mod, b.sb.final_mod, b.sb, st)))
+    return r;
+
+  // residual streams: text, references (uncached steps) and the shared target
+  uint16_t* lat_t = b.sb.lat_bf16 + static_cast<size_t>(sp[0].S + sp[1].S - N) * P;
+  {
+    Prof pr(ctx, QI_KCLASS_OTHER, st);
+    if (qi::launch_f32_to_bf16(latents, lat_t, static_cast<int64_t>(N) * P, st))
+      return cuda_fail("cast launch");
+  }
+  size_t lat_off = 0;
+  for (int q = 0; q < 2; ++q) {
+    float* xs = b.sb.x + static_cast<size_t>(off[q]) * H;
+    if (sp[q].row0 == 0) {
+      if ((r = run_bf16_linear(ctx, seq[q]->txt, sp[q].L, H, model->txt_in, qi::EPI_F32, xs, H,
+                               0.f, nullptr, st)))
+        return r;
+      if (sp[q].R > 0) {
+        uint16_t* lr = b.sb.lat_bf16 + lat_off;
+        lat_off += static_cast<size_t>(sp[q].R) * P;
+        {
+          Prof pr(ctx, QI_KCLASS_OTHER, st);
+          if (qi::launch_f32_to_bf16(seq[q]->ref_latents, lr, static_cast<int64_t>(sp[q].R) * P, st))
+            return cuda_fail("cast launch");
+        }
+        if ((r = run_bf16_linear(ctx, lr, sp[q].R, P, model->img_in, qi::EPI_F32,
+                                 xs + static_cast<size_t>(sp[q].L) * H, H, 0.f, nullptr, st)))
+          return r;
+      }
+    }
+    if ((r = run_bf16_linear(ctx, lat_t, N, P, model->img_in, qi::EPI_F32,
+                             xs + static_cast<size_t>(sp[q].P - sp[q].row0) * H, H, 0.f, nullptr, st)))
+      return r;
+  }
+
+  for (int l = 0; l < d.blocks; ++l) {
+    SeqAttn sa[2];
+    for (int q = 0; q < 2; ++q) {
+      sa[q].off = off[q];
+      sa[q].T = sp[q].T;
+      sa[q].row0 = sp[q].row0;
+      sa[q].S = sp[q].S;
+      sa[q].gt = sp[q].gt;
+      sa[q].kl = kv[q] + static_cast<size_t>(l) * 2 * sp[q].S * H;
+      sa[q].vl = sa[q].kl + static_cast<size_t>(sp[q].S) * H;
+    }
+    if ((r = run_block_multi(ctx, d, model->blocks[l], b.sb.x, T, rows, 0,
+                             b.sb.block_mod + static_cast<size_t>(l) * 2 * 6 * H, b.cos, b.sin, sa,
+                             2, b.sb.block_ws, b.sb.block_ws_bytes, st)))
+      return r;
+  }
+
+  // final adaLN of both targets, one proj_out over their 2N rows, then the
+  // guided velocity and the Euler update
+  qi::GroupTable one;
+  memset(&one, 0, sizeof(one));
+  one.n = 1;
+  one.end[0] = N;
+  const uint16_t* fm = b.sb.final_mod + 2 * H;   // row 1 (the step's sigma)
+  for (int q = 0; q < 2; ++q) {
+    const float* xt = b.sb.x + static_cast<size_t>(off[q] + sp[q].P - sp[q].row0) * H;
+    if ((r = run_quant(ctx, xt, false, N, H, H, fm, fm + H, 0, one, 0, d.eps, nullptr, nullptr,
+                       nullptr, b.sb.u_final + static_cast<size_t>(q) * N * H, st)))
+      return r;
+  }
+  if ((r = run_bf16_linear(ctx, b.sb.u_final, 2 * N, H, model->proj_out, qi::EPI_F32, b.v, P, 0.f,
+                           nullptr, st)))
+    return r;
+  {
+    Prof pr(ctx, QI_KCLASS_OTHER, st);
+    if (qi::launch_cfg_euler(latents, b.v, b.v + static_cast<size_t>(N) * P,
+                             static_cast<int64_t>(N) * P, guidance, sigma_next - sigma, v_out, st))
+      return cuda_fail("guidance launch");
+  }
   return QI_OK;
 }
 

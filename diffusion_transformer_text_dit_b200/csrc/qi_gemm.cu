@@ -147,7 +147,12 @@ __device__ __forceinline__ void qkv_epilogue(const GemmParams& p, const ColTable
                                              int32_t zp, int n0, int lane, uint32_t tempty_addr) {
   const int which = n0 / p.H;
   const int col0 = n0 - which * p.H;
-  uint16_t* out = which == 0 ? p.q_out : (which == 1 ? p.k_out : p.v_out_bf16);
+  // q rows are contiguous; K/V rows of a second sequence go to its own buffer
+  const bool second = which > 0 && p.k_out2 != nullptr && m >= p.kv_split;
+  const int mo = second ? m - p.kv_split : m;
+  uint16_t* out = which == 0 ? p.q_out
+                             : (which == 1 ? (second ? p.k_out2 : p.k_out)
+                                           : (second ? p.v_out2 : p.v_out_bf16));
   const uint16_t* w = which == 0 ? p.wq : p.wk;
 #pragma unroll 1
   for (int hh = 0; hh < W / 128; ++hh) {
@@ -205,7 +210,7 @@ __device__ __forceinline__ void qkv_epilogue(const GemmParams& p, const ColTable
 #pragma unroll
         for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(y[2 * i], y[2 * i + 1]);
       }
-      uint4* dst = reinterpret_cast<uint4*>(out + static_cast<size_t>(m) * p.ldo + col0 +
+      uint4* dst = reinterpret_cast<uint4*>(out + static_cast<size_t>(mo) * p.ldo + col0 +
                                             hh * 128 + c * 32);
 #pragma unroll
       for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);

@@ -61,8 +61,11 @@ struct GemmParams {
   const float* rcos;      // [M, 64] tables of the rows of this GEMM
   const float* rsin;
   uint16_t* q_out;        // [M, H] rows of this GEMM
-  uint16_t* k_out;
+  uint16_t* k_out;        // K/V rows m < kv_split (all rows if k_out2 is null)
   uint16_t* v_out_bf16;
+  uint16_t* k_out2;       // K/V rows m >= kv_split go to k_out2/v_out2 row m - kv_split
+  uint16_t* v_out2;       // (a batch of two sequences with separate K/V buffers)
+  int kv_split;
   int ldo;
   uint32_t* row_range;    // GELU: optional per-row [-min, max] bit patterns of the bf16 output
   int* status;            // device status word
@@ -163,5 +166,9 @@ int launch_timestep_embedding(float t0, float t1, float* out, cudaStream_t st);
 int launch_timeout_probe(uint64_t limit_ns, int* status, cudaStream_t st);
 int launch_f32_to_bf16(const float* x, uint16_t* y, int64_t n, cudaStream_t st);
 int launch_euler(float* x, const float* v, int64_t n, float dt, cudaStream_t st);
+// Classifier-free guidance + Euler: v = v_u + g (v_c - v_u), x += dt v, fp32,
+// one rounding per operation; v_out (optional) receives v.
+int launch_cfg_euler(float* x, const float* v_c, const float* v_u, int64_t n, float g, float dt,
+                     float* v_out, cudaStream_t st);
 
 }  // namespace qi

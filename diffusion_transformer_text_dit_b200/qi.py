@@ -81,6 +81,12 @@ class qi_model(C.Structure):
                 ("proj_out", qi_linear_bf16)]
 
 
+class qi_seq(C.Structure):
+    _fields_ = [("txt", C.c_void_p), ("text_tokens", C.c_int32), ("ref_latents", C.c_void_p),
+                ("groups", C.POINTER(qi_groups)), ("rope_cos", C.c_void_p),
+                ("rope_sin", C.c_void_p), ("kv_cache", C.c_void_p)]
+
+
 # ------------------------------------------------------------------ loading
 
 _lib = None
@@ -122,6 +128,11 @@ _SIGS = {
                         C.c_void_p, C.POINTER(qi_groups), C.c_void_p, C.c_void_p, C.c_float,
                         C.c_float, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p, C.c_size_t,
                         C.c_void_p],
+    "qi_step_cfg_workspace_bytes": [C.POINTER(qi_dims), C.c_int, C.c_int, C.c_int,
+                                    C.POINTER(C.c_size_t)],
+    "qi_denoise_step_cfg": [C.c_void_p, C.POINTER(qi_model), C.c_void_p, C.POINTER(qi_seq),
+                            C.POINTER(qi_seq), C.c_float, C.c_float, C.c_float, C.c_int,
+                            C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p],
     "qi_euler_update": [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int64, C.c_float, C.c_float,
                         C.c_void_p],
     "qi_rope_tables": [C.c_int, C.POINTER(C.c_int32), C.POINTER(C.c_int32),
@@ -372,6 +383,34 @@ def qi_denoise_step(ctx: Context, model: "Model", latents, txt, text_tokens, ref
                                 text_tokens, ptr(ref_latents), C.byref(groups), ptr(cos),
                                 ptr(sin), sigma, sigma_next, kv_mode, ptr(kv_cache), ptr(v_out),
                                 ptr(workspace), workspace.numel(), stream_ptr(stream)))
+
+
+def seq_struct(txt, text_tokens, ref_latents, groups: qi_groups, cos, sin, kv_cache=None):
+    """A qi_seq for qi_denoise_step_cfg.  The struct holds raw device pointers,
+    so it keeps references to every tensor (and the groups) it points to: a
+    tensor freed while the struct lives would let the caching allocator hand
+    its memory to a later tensor before the step reads it."""
+    s = qi_seq()
+    s.txt, s.text_tokens, s.ref_latents = ptr(txt), text_tokens, ptr(ref_latents)
+    s.groups = C.pointer(groups)
+    s.rope_cos, s.rope_sin, s.kv_cache = ptr(cos), ptr(sin), ptr(kv_cache)
+    s._keep = (txt, ref_latents, groups, cos, sin, kv_cache)
+    return s
+
+
+def qi_step_cfg_workspace_bytes(dims: qi_dims, S_cond: int, S_uncond: int, target_tokens: int) -> int:
+    n = C.c_size_t()
+    check(lib().qi_step_cfg_workspace_bytes(C.byref(dims), S_cond, S_uncond, target_tokens,
+                                            C.byref(n)))
+    return n.value
+
+
+def qi_denoise_step_cfg(ctx: Context, model: "Model", latents, cond: qi_seq, uncond: qi_seq,
+                        guidance, sigma, sigma_next, kv_mode, v_out, workspace, stream=None):
+    check(lib().qi_denoise_step_cfg(ctx.handle, C.byref(model.struct), ptr(latents),
+                                    C.byref(cond), C.byref(uncond), guidance, sigma, sigma_next,
+                                    kv_mode, ptr(v_out), ptr(workspace), workspace.numel(),
+                                    stream_ptr(stream)))
 
 
 def qi_euler_update(ctx: Context, x, v, sigma, sigma_next, stream=None):

@@ -28,7 +28,8 @@ from typing import Optional, Sequence, Tuple
 import torch
 
 __all__ = [
-    "Group", "DitConfig", "TINY", "BLOCK512", "STEP1024", "EDIT1024", "EDIT3REF1024", "GEN2048",
+    "Group", "DitConfig", "TINY", "BLOCK512", "STEP1024", "EDIT1024", "EDIT3REF1024", "CFG1024",
+    "GEN2048",
     "CONFIGS", "gen", "linear_weight", "bias", "norm_weight", "latents",
     "text_features", "ref_latents", "hidden_states", "mod_table", "block_weights", "model_weights",
 ]
@@ -58,6 +59,8 @@ class DitConfig:
     latent_seed: int = 1
     steps: int = 1
     t: Optional[float] = None                  # fixed timestep for block-only workloads
+    uncond_text: int = 0                       # true CFG: negative-prompt tokens (0 = no guidance)
+    guidance: float = 4.0                      # true CFG scale
 
     @property
     def tokens(self) -> int:
@@ -82,6 +85,14 @@ class DitConfig:
         """Modulation row set per group: 0 for conditioning prefix groups, 1 for the target."""
         return tuple(0 if i < len(self.groups) - 1 else 1 for i in range(len(self.groups)))
 
+    def uncond(self) -> "DitConfig":
+        """The unconditional (negative prompt) sequence of a true-CFG workload:
+        the text group holds uncond_text tokens, the rest is unchanged."""
+        assert self.uncond_text > 0 and self.groups[0].kind == "text"
+        return dataclasses.replace(self, name=self.name + "_uncond", input_seed=self.input_seed + 1000,
+                                   groups=(Group("text", self.uncond_text),) + self.groups[1:],
+                                   uncond_text=0)
+
     def replace(self, **kw) -> "DitConfig":
         return dataclasses.replace(self, **kw)
 
@@ -103,6 +114,10 @@ STEP1024 = DitConfig("step_1024px", 4096, 32, 128, 16384, 32, 64,
 EDIT1024 = DitConfig("edit_1024px", 4096, 32, 128, 16384, 32, 64,
                      (Group(_TEXT, 256), Group(_IMAGE, 1024, (32, 32)),
                       Group(_IMAGE, 4096, (64, 64))))
+# True-CFG step at 1024x1024: the 512-token prompt and a 256-token negative
+# prompt over the same 4096 target tokens, run as one batch.
+CFG1024 = DitConfig("cfg_1024px", 4096, 32, 128, 16384, 32, 64,
+                    (Group(_TEXT, 512), Group(_IMAGE, 4096, (64, 64))), uncond_text=256)
 # Multi-reference edit step: 256 text + three references (32x32, 32x32, 24x24)
 # + 4096 target tokens; each reference is its own group of the block-causal mask.
 EDIT3REF1024 = DitConfig("edit_3ref_1024px", 4096, 32, 128, 16384, 32, 64,
@@ -114,7 +129,7 @@ GEN2048 = DitConfig("denoise40_2048px", 4096, 32, 128, 16384, 32, 64,
                     (Group(_TEXT, 512), Group(_IMAGE, 16384, (128, 128))),
                     steps=40, latent_seed=42)
 
-CONFIGS = {c.name: c for c in (TINY, BLOCK512, STEP1024, EDIT1024, EDIT3REF1024, GEN2048)}
+CONFIGS = {c.name: c for c in (TINY, BLOCK512, STEP1024, EDIT1024, EDIT3REF1024, CFG1024, GEN2048)}
 
 
 def gen(seed: int, *tags) -> torch.Generator:

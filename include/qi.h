@@ -17,7 +17,11 @@
  *          16x16 px tile; 3-axis RoPE positions; 64 rotation pairs per head;
  *          shifted sigmas and the Euler update x += (sigma_next - sigma) * v.
  *   [MNN]  qwen-image-mnn, "What runs where": 3-axis RoPE, block-causal mask
- *          and modulation rows as the joint-sequence bookkeeping.
+ *          and modulation rows as the joint-sequence bookkeeping; "Install /
+ *          run": a true CFG scale > 1 with a negative prompt enables
+ *          classifier-free guidance.
+ *   [QC]   "Qwen Image 2.1 native qualification", "Native CLI cases": CFG,
+ *          single- and multi-reference edit (up to ten references) cases.
  *   [PX]   EliovpAI "Qwen_Image-2.1-MXFP4-Paiton-RDNA4", "Runtime precision and
  *          quality" / "Tested operating limits": cached text-prefix pass
  *          (prefix KV reuse); unsupported settings rejected before GPU work.
@@ -339,6 +343,43 @@ int qi_denoise_step(qi_ctx* ctx, const qi_model* model, float* latents, const ui
                     const float* rope_cos, const float* rope_sin, float sigma, float sigma_next,
                     int kv_mode, uint16_t* kv_cache, float* v_out, void* workspace,
                     size_t workspace_bytes, void* stream);
+
+/* One sequence of a classifier-free-guidance step (qi_denoise_step_cfg);
+ * the fields mean what the arguments of the same names of qi_denoise_step do. */
+typedef struct qi_seq {
+  const uint16_t* txt;        /* [text_tokens, H] bf16; may be NULL in READ_PREFIX mode */
+  int text_tokens;
+  const float* ref_latents;   /* [R, P] fp32 reference latents, NULL if none */
+  const qi_groups* groups;    /* the joint sequence, target last */
+  const float* rope_cos;      /* [S, 64] fp32 */
+  const float* rope_sin;
+  uint16_t* kv_cache;         /* [blocks][2][S][H] bf16; may be NULL in QI_KV_NONE mode */
+} qi_seq;
+
+/* Workspace bytes needed by qi_denoise_step_cfg for a conditional sequence of
+ * S_cond tokens and an unconditional one of S_uncond, both ending in a target
+ * group of target_tokens. */
+int qi_step_cfg_workspace_bytes(const qi_dims* dims, int S_cond, int S_uncond, int target_tokens,
+                                size_t* bytes);
+
+/* One denoising step with true classifier-free guidance ([MNN] Install / run;
+ * [QC] Native CLI cases).  The conditional sequence and the unconditional one
+ * (a negative prompt of any text length, the same target and usually the same
+ * references) run as one batch: every Linear, quantizer and norm runs once over
+ * the rows of both (shared weights, twice the GEMM rows), attention runs per
+ * sequence with its own mask and K/V.  Each sequence's velocity is
+ * bit-identical to what qi_denoise_step computes for it alone.  Then
+ *   v = v_u + guidance (v_c - v_u),   latents += (sigma_next - sigma) v
+ * in fp32 with one rounding per operation and no fused multiply-add (the pages
+ * give the guidance scale but no formula; this is the plain reading, with no
+ * renormalization).  latents [N, P] fp32 (in/out); v_out [N, P] fp32 gets the
+ * guided v if not NULL.  Both target groups must hold N tokens; in uncached
+ * modes the two sequences together may have at most QI_MAX_GROUPS groups.
+ * kv_mode applies to both sequences (each with its own kv_cache). */
+int qi_denoise_step_cfg(qi_ctx* ctx, const qi_model* model, float* latents, const qi_seq* cond,
+                        const qi_seq* uncond, float guidance, float sigma, float sigma_next,
+                        int kv_mode, float* v_out, void* workspace, size_t workspace_bytes,
+                        void* stream);
 
 /* x += (sigma_next - sigma) * v over n fp32 values, one rounding per operation
  * (no fused multiply-add); sigma_next - sigma is rounded to fp32 first ([GC] Sampler). */

@@ -430,6 +430,17 @@ def euler_update(x, v, sigma, sigma_next) -> np.ndarray:
     return (x + (dt * v).astype(F32)).astype(F32)
 
 
+def cfg_combine(v_cond, v_uncond, guidance) -> np.ndarray:
+    """True classifier-free guidance of one step (qwen-image-mnn, "Install /
+    run": a true CFG scale with a negative prompt): v_u + g (v_c - v_u) in
+    fp32, one rounding per operation, no FMA.  The pages give the scale, not
+    the formula; this is the plain reading, with no renormalization."""
+    vc = np.asarray(v_cond, F32)
+    vu = np.asarray(v_uncond, F32)
+    d = (vc - vu).astype(F32)
+    return (vu + (F32(guidance) * d).astype(F32)).astype(F32)
+
+
 # ----------------------------------------------------------------------------
 # Whole denoising step
 # ----------------------------------------------------------------------------

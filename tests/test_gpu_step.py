@@ -106,3 +106,92 @@ def test_step_1024px_deterministic_aba(ctx):
     assert torch.equal(a, a2) and torch.equal(va, va2)
     assert not torch.equal(va, vb)
     assert torch.isfinite(va).all()
+
+
+# ------------------------------------------------------------------ true CFG
+
+class CfgSetup:
+    """A conditional and an unconditional (negative prompt) sequence over the
+    same target; the negative prompt is shorter."""
+
+    def __init__(self, ctx, blocks=2, refs=0, text_c=12, text_u=7):
+        ref_groups = tuple(synth.Group("image", n, g) for n, g in
+                           ((16, (4, 4)), (36, (6, 6)))[:refs])
+        tgt = synth.Group("image", 64, (8, 8))
+        self.cfg_c = synth.TINY.replace(name="cfg_c", blocks=blocks, patch=64,
+                                        groups=(synth.Group("text", text_c),) + ref_groups + (tgt,))
+        self.cfg_u = self.cfg_c.replace(name="cfg_u", groups=(synth.Group("text", text_u),) + ref_groups + (tgt,))
+        self.c = Setup(ctx, self.cfg_c)
+        self.u = Setup(ctx, self.cfg_u)
+        self.u.model = self.c.model   # one model: same weights for both passes
+        # the negative prompt's text rows: another draw of the same distribution
+        self.u.txt = synth.text_features(self.cfg_u.replace(input_seed=9))
+        self.u.ref = self.c.ref
+        S_c, S_u, N = self.cfg_c.tokens, self.cfg_u.tokens, self.cfg_c.target_tokens
+        self.ws = torch.empty(qi.qi_step_cfg_workspace_bytes(self.c.dims, S_c, S_u, N),
+                              dtype=torch.uint8, device="cuda")
+
+    def seq(self, s, mode):
+        return qi.seq_struct(cuda(s.txt) if mode != qi.QI_KV_READ_PREFIX else None,
+                             s.cfg.text_tokens,
+                             cuda(s.ref) if (s.ref is not None and mode != qi.QI_KV_READ_PREFIX) else None,
+                             s.groups, s.cos, s.sin, s.kv if mode != qi.QI_KV_NONE else None)
+
+    def step(self, ctx, lat, g, sigma, sigma_next, mode=qi.QI_KV_NONE):
+        sc, su = self.seq(self.c, mode), self.seq(self.u, mode)
+        latg = cuda(lat)
+        v = torch.empty_like(latg)
+        qi.qi_denoise_step_cfg(ctx, self.c.model, latg, sc, su, g, sigma, sigma_next, mode, v,
+                               self.ws)
+        ctx.check()
+        return latg.cpu(), v.cpu()
+
+
+@pytest.mark.parametrize("refs", [0, 2], ids=["text_image", "text_2ref_image"])
+def test_cfg_batch_equals_two_single_steps(ctx, refs):
+    s = CfgSetup(ctx, refs=refs)
+    sig = O.sigma_schedule(40, s.cfg_c.target_tokens)
+    a, b = float(sig[5]), float(sig[6])
+    lat, v = s.step(ctx, s.c.lat, 4.0, a, b)
+    _, vc = s.c.gpu_step(ctx, s.c.lat, a, b)
+    _, vu = s.u.gpu_step(ctx, s.c.lat, a, b)
+    # each sequence of the batch computes exactly its single-sequence velocity
+    assert np.array_equal(v.numpy(), O.cfg_combine(vc.numpy(), vu.numpy(), 4.0))
+    assert np.array_equal(lat.numpy(), O.euler_update(s.c.lat.numpy(), v.numpy(), a, b))
+    assert not np.array_equal(vc.numpy(), vu.numpy())
+
+
+def test_cfg_step_vs_oracle(ctx):
+    s = CfgSetup(ctx, refs=1)
+    sig = O.sigma_schedule(40, s.cfg_c.target_tokens)
+    a, b = float(sig[2]), float(sig[3])
+    _, v = s.step(ctx, s.c.lat, 3.0, a, b)
+    _, ovc = s.c.oracle_step(s.c.lat, a, b)
+    _, ovu = s.u.oracle_step(s.c.lat, a, b)
+    ov = O.cfg_combine(ovc, ovu, 3.0)
+    assert np.all(np.isfinite(v.numpy()))
+    assert rel_l2(v.numpy(), ov) < 2e-2
+
+
+def test_cfg_cached_equals_uncached(ctx):
+    s = CfgSetup(ctx, blocks=3, refs=1)
+    sig = O.sigma_schedule(40, s.cfg_c.target_tokens)
+    a1, _ = s.step(ctx, s.c.lat, 2.5, float(sig[0]), float(sig[1]), qi.QI_KV_WRITE_PREFIX)
+    u2, _ = s.step(ctx, a1, 2.5, float(sig[1]), float(sig[2]), qi.QI_KV_NONE)
+    c2, _ = s.step(ctx, a1, 2.5, float(sig[1]), float(sig[2]), qi.QI_KV_READ_PREFIX)
+    assert torch.equal(u2, c2)
+
+
+def test_cfg_rejects_mismatched_targets(ctx):
+    s = CfgSetup(ctx)
+    other = synth.TINY.replace(name="cfg_bad", blocks=2, patch=64,
+                               groups=(synth.Group("text", 7), synth.Group("image", 16, (4, 4))))
+    bad = Setup(ctx, other)
+    latg = cuda(s.c.lat)
+    before = latg.clone()
+    with pytest.raises(qi.QiError) as e:
+        qi.qi_denoise_step_cfg(ctx, s.c.model, latg, s.seq(s.c, qi.QI_KV_NONE),
+                               s.seq(bad, qi.QI_KV_NONE), 2.0, 1.0, 0.9, qi.QI_KV_NONE, None, s.ws)
+    assert e.value.code == qi.QI_ERR_INVALID_ARG
+    torch.cuda.synchronize()
+    assert torch.equal(latg, before)

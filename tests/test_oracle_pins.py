@@ -388,6 +388,24 @@ def test_euler_fp32_rounding():
     assert np.allclose(z, x - v, atol=1e-5)
 
 
+def test_cfg_combine_special_cases():
+    vc = rng.standard_normal(257).astype(np.float32)
+    vu = rng.standard_normal(257).astype(np.float32)
+    # scale 0 is the unconditional velocity, equal velocities are unchanged
+    assert np.array_equal(O.cfg_combine(vc, vu, 0.0), vu)
+    assert np.array_equal(O.cfg_combine(vu, vu, 7.5), vu)
+    # scale 1 gives v_c exactly where v_c - v_u is exact (Sterbenz: v_u/2 <= v_c <= 2 v_u)
+    a = np.float32(1.0) + rng.random(100).astype(np.float32)
+    b = a * np.float32(1.5)
+    assert np.array_equal(O.cfg_combine(b, a, 1.0), b)
+    # hand values: 0.5 + 3 (1 - 0.5) = 2
+    assert O.cfg_combine(np.float32([1.0]), np.float32([0.5]), 3.0)[0] == np.float32(2.0)
+    # within a few fp32 ulps of the exact value
+    g = 4.0
+    exact = vu.astype(np.float64) + g * (vc.astype(np.float64) - vu.astype(np.float64))
+    assert np.allclose(O.cfg_combine(vc, vu, g), exact, rtol=0, atol=4e-6 * (1 + np.abs(exact)).max())
+
+
 def test_w8_call_count_golden():
     g = json.load(open(os.path.join(GOLDEN, "w8_call_count.json")))
     blocks = range(g["first_block"], g["last_block"] + 1)
