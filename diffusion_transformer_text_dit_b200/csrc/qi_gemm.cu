@@ -136,10 +136,10 @@ __device__ __forceinline__ void tempty_signal(uint32_t addr) {
 }
 
 // Fused epilogue of the QKV projection: the W columns handled by one epilogue
-// warp are W/128 whole heads of q, k or v.  For q and k each head row is read from TMEM
-// twice: once for the sum of squares of its bf16 values, once to apply
-//   r = 1/sqrt(mean + eps), n = bf16(y r), y' = bf16(n w)     (cast before scale)
-//   (a, b) -> (bf16(a c - b s), bf16(a s + b c))              (RoPE, pair = column/2)
+// warp are W/128 whole heads of q, k or v.  A q or k head row is read from
+// TMEM once and held (dequantized, bf16-rounded) in registers for
+//   r = 1/sqrt(mean(y^2) + eps), n = bf16(y r), y' = bf16(n w)   (cast before scale)
+//   (a, b) -> (bf16(a c - b s), bf16(a s + b c))                 (RoPE, pair = column/2)
 // with explicitly rounded fp32 operations; v is stored as bf16(y).
 template <int W, bool PAIR>
 __device__ __forceinline__ void qkv_epilogue(const GemmParams& p, const ColTable& ct, int cb,
@@ -156,64 +156,80 @@ __device__ __forceinline__ void qkv_epilogue(const GemmParams& p, const ColTable
   const uint16_t* w = which == 0 ? p.wq : p.wk;
 #pragma unroll 1
   for (int hh = 0; hh < W / 128; ++hh) {
-    float rs = 1.0f;
-    if (which < 2) {
-      float ss = 0.f;
+    const bool last = hh == W / 128 - 1;   // this warp's last TMEM reads of the accumulator
+    uint4* dst_row = reinterpret_cast<uint4*>(out + static_cast<size_t>(mo) * p.ldo + col0 + hh * 128);
+    if (which == 2) {
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         uint32_t r[32];
         tmem_ld32(t_row + hh * 128 + c * 32, r);
-        if (row_ok) {
-          float y[32];
-          dequant32_bf16(ct, r, cb + hh * 128 + c * 32, sa, zp, y);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) ss = __fadd_rn(ss, __fmul_rn(y[j], y[j]));
+        if (last && c == 3) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) tempty_signal<PAIR>(tempty_addr);
         }
+        if (!row_ok) continue;
+        float y[32];
+        dequant32_bf16(ct, r, cb + hh * 128 + c * 32, sa, zp, y);
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(y[2 * i], y[2 * i + 1]);
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+          dst_row[c * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
       }
-      rs = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(ss, 128.0f), p.eps)));
+      continue;
     }
-#pragma unroll 1
+    // the head row as bf16 pairs (the dequantized values are bf16 already)
+    uint32_t yp[4][16];
+    float ss = 0.f;
+#pragma unroll
     for (int c = 0; c < 4; ++c) {
       uint32_t r[32];
       tmem_ld32(t_row + hh * 128 + c * 32, r);
-      if (hh == W / 128 - 1 && c == 3) {   // this warp's last TMEM read of the accumulator
+      if (last && c == 3) {
         tc_fence_before();
         __syncwarp();
         if (lane == 0) tempty_signal<PAIR>(tempty_addr);
       }
-      if (!row_ok) continue;
-      float y[32];
-      dequant32_bf16(ct, r, cb + hh * 128 + c * 32, sa, zp, y);
-      uint32_t pk[16];
-      if (which < 2) {
-        const float4* c4 = reinterpret_cast<const float4*>(p.rcos + static_cast<size_t>(m) * 64 + c * 16);
-        const float4* s4 = reinterpret_cast<const float4*>(p.rsin + static_cast<size_t>(m) * 64 + c * 16);
-        const uint4* w4 = reinterpret_cast<const uint4*>(w + c * 32);
+      if (row_ok) {
+        float y[32];
+        dequant32_bf16(ct, r, cb + hh * 128 + c * 32, sa, zp, y);
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const float4 cc = __ldg(c4 + g), sn = __ldg(s4 + g);
-          const uint4 wv = __ldg(w4 + g);
-          const float cs[4] = {cc.x, cc.y, cc.z, cc.w}, si[4] = {sn.x, sn.y, sn.z, sn.w};
-          const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+        for (int j = 0; j < 32; ++j) ss = __fadd_rn(ss, __fmul_rn(y[j], y[j]));
 #pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            const int i = 4 * g + t;   // pair index in the chunk
-            const float a = bf16_round_f(__fmul_rn(bf16_round_f(__fmul_rn(y[2 * i], rs)),
-                                                   __uint_as_float(ww[t] << 16)));
-            const float b = bf16_round_f(__fmul_rn(bf16_round_f(__fmul_rn(y[2 * i + 1], rs)),
-                                                   __uint_as_float(ww[t] & 0xFFFF0000u)));
-            pk[i] = pack_bf16x2(__fsub_rn(__fmul_rn(a, cs[t]), __fmul_rn(b, si[t])),
-                                __fadd_rn(__fmul_rn(a, si[t]), __fmul_rn(b, cs[t])));
-          }
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(y[2 * i], y[2 * i + 1]);
+        for (int i = 0; i < 16; ++i) yp[c][i] = pack_bf16x2(y[2 * i], y[2 * i + 1]);
       }
-      uint4* dst = reinterpret_cast<uint4*>(out + static_cast<size_t>(mo) * p.ldo + col0 +
-                                            hh * 128 + c * 32);
+    }
+    if (!row_ok) continue;
+    const float rs = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(ss, 128.0f), p.eps)));
 #pragma unroll
-      for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+    for (int c = 0; c < 4; ++c) {
+      uint32_t pk[16];
+      const float4* c4 = reinterpret_cast<const float4*>(p.rcos + static_cast<size_t>(m) * 64 + c * 16);
+      const float4* s4 = reinterpret_cast<const float4*>(p.rsin + static_cast<size_t>(m) * 64 + c * 16);
+      const uint4* w4 = reinterpret_cast<const uint4*>(w + c * 32);
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const float4 cc = __ldg(c4 + g), sn = __ldg(s4 + g);
+        const uint4 wv = __ldg(w4 + g);
+        const float cs[4] = {cc.x, cc.y, cc.z, cc.w}, si[4] = {sn.x, sn.y, sn.z, sn.w};
+        const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int i = 4 * g + t;   // pair index in the chunk
+          const float y0 = __uint_as_float(yp[c][i] << 16), y1 = __uint_as_float(yp[c][i] & 0xFFFF0000u);
+          const float a = bf16_round_f(__fmul_rn(bf16_round_f(__fmul_rn(y0, rs)),
+                                                 __uint_as_float(ww[t] << 16)));
+          const float b = bf16_round_f(__fmul_rn(bf16_round_f(__fmul_rn(y1, rs)),
+                                                 __uint_as_float(ww[t] & 0xFFFF0000u)));
+          pk[i] = pack_bf16x2(__fsub_rn(__fmul_rn(a, cs[t]), __fmul_rn(b, si[t])),
+                              __fadd_rn(__fmul_rn(a, si[t]), __fmul_rn(b, cs[t])));
+        }
+      }
+#pragma unroll
+      for (int v = 0; v < 4; ++v)
+        dst_row[c * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
     }
   }
 }
