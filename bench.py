@@ -268,7 +268,7 @@ def aggregate_throughput(world: int, steps: int, max_ms: float) -> float:
 # ------------------------------------------------------------------ GPU arm
 
 WORKLOADS = {c.name: c for c in (synth.STEP1024, synth.EDIT1024, synth.EDIT3REF1024, synth.CFG1024,
-                                  synth.GEN2048)}
+                                  synth.GEN2048, synth.GEN2048_SCHED)}
 
 
 def run_ours(args, rank, world, local_rank):
@@ -324,10 +324,15 @@ def run_ours(args, rank, world, local_rank):
 
     def denoise_40(latents, text):
         # FlowMatch Euler over the 40-step schedule; the prefix K/V of the
-        # first step are reused by the 39 later steps
+        # first step are reused by the 39 later steps.  With a precision
+        # schedule, attention switches to fp8 from step fp8_from_step on (the
+        # prefix pass stays at full precision).
         step(0, latents, text, qi.QI_KV_WRITE_PREFIX)
         for i in range(1, 40):
+            if cfg.fp8_from_step and i + 1 == cfg.fp8_from_step:
+                ctx.set_attention_fp8(True)
             step(i, latents, text, qi.QI_KV_READ_PREFIX)
+        ctx.set_attention_fp8(False)
 
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
@@ -464,7 +469,9 @@ def run_ours(args, rank, world, local_rank):
                f"(scale {cfg.guidance}), " if cfg.uncond_text else "")
             + ("40-step FlowMatch Euler denoise, prefix K/V cached from step 2"
                if denoise else "uncached step")
-            + ", all attn/MLP Linears W8A8 (int8 GEMMs, bf16 attention)")
+            + ", all attn/MLP Linears W8A8 (int8 GEMMs), "
+            + (f"bf16 attention in steps 1-{cfg.fp8_from_step - 1} and fp8 (e4m3) attention from "
+               f"step {cfg.fp8_from_step}" if cfg.fp8_from_step else "bf16 attention"))
     out = {
         "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world,
         "steps": n_steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
@@ -577,7 +584,9 @@ def main():
                          "edit_3ref_1024px: an edit with three reference images; "
                          "cfg_1024px: true classifier-free guidance (prompt + negative prompt "
                          "as one batch); "
-                         "denoise40_2048px: the full 40-step 2048^2 denoise")
+                         "denoise40_2048px: the full 40-step 2048^2 denoise; "
+                         "denoise40_2048px_sched: the same with the pages' precision schedule "
+                         "(fp8 attention from step 8)")
     ap.add_argument("--ncu-case", choices=("gemms", "gemm_down", "attention"), default=None,
                     help="launch one kernel a few times (for ncu captures) and exit")
     args = ap.parse_args()

@@ -29,6 +29,7 @@ struct qi_ctx {
   cudaEvent_t* prof_ev;          // [2 * QI_PROF_MAX_PAIRS]
   int* prof_cls;                 // [QI_PROF_MAX_PAIRS]
   long long launches[QI_PROF_CLASSES];
+  int attn_fp8;                  // steps run e4m3 attention (qi_ctx_set_attention_fp8)
 };
 
 namespace {
@@ -192,6 +193,13 @@ size_t block_bytes(const qi_dims& d, int T) {
   return c.off + 256;
 }
 
+// e4m3 copies of the attention operands of one block (fp8 attention): q for
+// the batch's processed rows, then per sequence its K rows and its V rows.
+struct Fp8Bufs {
+  uint8_t* q;
+  uint8_t* kv;
+};
+
 struct StepBufs {
   float* x;             // [S, H] fp32 residual stream
   float* emb;           // [2, 256]
@@ -202,6 +210,7 @@ struct StepBufs {
   uint16_t* lat_bf16;   // [S, P] bf16 copies of the latents fed to img_in
   uint16_t* u_final;    // [S, H]
   uint16_t* kv;         // [blocks][2][S][H] when the caller passes no cache
+  Fp8Bufs f8;           // e4m3 attention operands (fp8 attention)
   uint8_t* block_ws;
   size_t block_ws_bytes;
 };
@@ -218,6 +227,8 @@ StepBufs carve_step(Carve& c, const qi_dims& d, int Sq, int S, bool own_kv) {
   b.lat_bf16 = c.take<uint16_t>(static_cast<size_t>(S) * P);
   b.u_final = c.take<uint16_t>(static_cast<size_t>(S) * H);
   b.kv = own_kv ? c.take<uint16_t>(static_cast<size_t>(d.blocks) * 2 * S * H) : nullptr;
+  b.f8.q = c.take<uint8_t>(static_cast<size_t>(Sq) * H);
+  b.f8.kv = c.take<uint8_t>(static_cast<size_t>(2) * S * H);
   b.block_ws_bytes = block_bytes(d, Sq);
   b.block_ws = c.take<uint8_t>(b.block_ws_bytes);
   return b;
@@ -371,7 +382,7 @@ struct SeqAttn {
 int run_block_multi(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, float* x, int T,
                     const qi::GroupTable& rows_gt, int rows_row0, const uint16_t* mod,
                     const float* cs, const float* sn, const SeqAttn* seqs, int nseq, uint8_t* ws,
-                    size_t ws_bytes, cudaStream_t st) {
+                    size_t ws_bytes, cudaStream_t st, const Fp8Bufs* f8 = nullptr) {
   const int H = d.hidden, F = d.mlp;
   const qi::GroupTable& gt = rows_gt;
   const int row0 = rows_row0;
@@ -424,13 +435,37 @@ int run_block_multi(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, fl
     if (rr == -2) return fail(QI_ERR_CUDA, "cuTensorMapEncodeTiled failed (QKV operands)");
     if (rr != 0) return cuda_fail("QKV GEMM launch");
   }
+  if (f8) {
+    // fp8 attention: e4m3 copies of q and of every sequence's K and V rows
+    Prof pr(ctx, QI_KCLASS_OTHER, st);
+    if (qi::launch_bf16_to_e4m3(b.q, f8->q, static_cast<int64_t>(T) * H, st))
+      return cuda_fail("e4m3 cast launch");
+    size_t o = 0;
+    for (int sq = 0; sq < nseq; ++sq) {
+      const size_t n = static_cast<size_t>(seqs[sq].S) * H;
+      if (qi::launch_bf16_to_e4m3(seqs[sq].kl, f8->kv + o, static_cast<int64_t>(n), st) ||
+          qi::launch_bf16_to_e4m3(seqs[sq].vl, f8->kv + o + n, static_cast<int64_t>(n), st))
+        return cuda_fail("e4m3 cast launch");
+      o += 2 * n;
+    }
+  }
+  size_t kv8 = 0;
   for (int sq = 0; sq < nseq; ++sq) {
     const SeqAttn& q = seqs[sq];
     qi::AttnParams ap;
     memset(&ap, 0, sizeof(ap));
-    ap.q = b.q + static_cast<size_t>(q.off) * H;
-    ap.k = q.kl;
-    ap.v = q.vl;
+    if (f8) {
+      const size_t n = static_cast<size_t>(q.S) * H;
+      ap.q = f8->q + static_cast<size_t>(q.off) * H;
+      ap.k = f8->kv + kv8;
+      ap.v = f8->kv + kv8 + n;
+      ap.fp8 = 1;
+      kv8 += 2 * n;
+    } else {
+      ap.q = b.q + static_cast<size_t>(q.off) * H;
+      ap.k = q.kl;
+      ap.v = q.vl;
+    }
     ap.o = b.o + static_cast<size_t>(q.off) * H;
     ap.ldq = H;
     ap.ldkv = H;
@@ -490,7 +525,7 @@ int run_block_multi(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, fl
 int run_block(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, float* x, int T, int row0,
               const uint16_t* mod, const qi::GroupTable& gt, int S, const float* cs,
               const float* sn, uint16_t* kl, uint16_t* vl, uint8_t* ws, size_t ws_bytes,
-              cudaStream_t st) {
+              cudaStream_t st, const Fp8Bufs* f8 = nullptr) {
   SeqAttn one;
   one.off = 0;
   one.T = T;
@@ -499,7 +534,7 @@ int run_block(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, float* x
   one.gt = gt;
   one.kl = kl;
   one.vl = vl;
-  return run_block_multi(ctx, d, w, x, T, gt, row0, mod, cs, sn, &one, 1, ws, ws_bytes, st);
+  return run_block_multi(ctx, d, w, x, T, gt, row0, mod, cs, sn, &one, 1, ws, ws_bytes, st, f8);
 }
 
 int check_block_weights(const qi_dims& d, const qi_block_weights* w) {
@@ -641,6 +676,7 @@ int qi_ctx_create(int device, qi_ctx** out) {
   c->prof_used = 0;
   c->prof_ev = nullptr;
   c->prof_cls = nullptr;
+  c->attn_fp8 = 0;
   for (int i = 0; i < QI_PROF_CLASSES; ++i) c->launches[i] = 0;
   if (cudaMalloc(&c->status, 256) != cudaSuccess) {
     delete c;
@@ -832,17 +868,19 @@ int qi_qk_norm_rope(qi_ctx* ctx, const uint16_t* qkv, int T, int heads, int head
   return QI_OK;
 }
 
-int qi_attn_block_causal(qi_ctx* ctx, const uint16_t* q, int ldq, int Sq, int q_offset,
-                         const uint16_t* k, const uint16_t* v, int ldkv, int Sk, int heads,
-                         int head_dim, const qi_groups* groups, float sm_scale, uint16_t* o,
-                         int ldo, void* stream) {
+namespace {
+
+int attn_call(qi_ctx* ctx, const void* q, int ldq, int Sq, int q_offset, const void* k,
+              const void* v, int ldkv, int Sk, int heads, int head_dim, const qi_groups* groups,
+              float sm_scale, uint16_t* o, int ldo, void* stream, bool fp8) {
   if (!ctx || !q || !k || !v || !o) return fail(QI_ERR_INVALID_ARG, "NULL argument");
   if (head_dim != 128) return fail(QI_ERR_UNSUPPORTED_SHAPE, "head_dim must be 128");
   if (Sq < 0 || Sk < 1 || q_offset < 0 || q_offset + Sq > Sk || heads < 1)
     return fail(QI_ERR_INVALID_ARG, "need 0 <= q_offset, q_offset + Sq <= Sk");
   const int W = heads * head_dim;
-  if (ldq < W || ldkv < W || ldo < W || ldq % 8 || ldkv % 8 || ldo % 8)
-    return fail(QI_ERR_ALIGNMENT, "leading dimensions must be >= heads*128 and multiples of 8");
+  const int qa = fp8 ? 16 : 8;   // elements per 16 bytes
+  if (ldq < W || ldkv < W || ldo < W || ldq % qa || ldkv % qa || ldo % 8)
+    return fail(QI_ERR_ALIGNMENT, "leading dimensions must be >= heads*128 and 16-byte multiples");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
     return fail(QI_ERR_ALIGNMENT, "q/k/v/o must be 16-byte aligned");
   qi::GroupTable gt;
@@ -853,6 +891,7 @@ int qi_attn_block_causal(qi_ctx* ctx, const uint16_t* q, int ldq, int Sq, int q_
   p.q = q;
   p.k = k;
   p.v = v;
+  p.fp8 = fp8 ? 1 : 0;
   p.o = o;
   p.ldq = ldq;
   p.ldkv = ldkv;
@@ -870,6 +909,39 @@ int qi_attn_block_causal(qi_ctx* ctx, const uint16_t* q, int ldq, int Sq, int q_
     if (r2 == -2) return fail(QI_ERR_CUDA, "cuTensorMapEncodeTiled failed (attention operands)");
     if (r2 != 0) return cuda_fail("attention launch");
   }
+  return QI_OK;
+}
+
+}  // namespace
+
+int qi_attn_block_causal(qi_ctx* ctx, const uint16_t* q, int ldq, int Sq, int q_offset,
+                         const uint16_t* k, const uint16_t* v, int ldkv, int Sk, int heads,
+                         int head_dim, const qi_groups* groups, float sm_scale, uint16_t* o,
+                         int ldo, void* stream) {
+  return attn_call(ctx, q, ldq, Sq, q_offset, k, v, ldkv, Sk, heads, head_dim, groups, sm_scale,
+                   o, ldo, stream, false);
+}
+
+int qi_attn_block_causal_fp8(qi_ctx* ctx, const uint8_t* q, int ldq, int Sq, int q_offset,
+                             const uint8_t* k, const uint8_t* v, int ldkv, int Sk, int heads,
+                             int head_dim, const qi_groups* groups, float sm_scale, uint16_t* o,
+                             int ldo, void* stream) {
+  return attn_call(ctx, q, ldq, Sq, q_offset, k, v, ldkv, Sk, heads, head_dim, groups, sm_scale,
+                   o, ldo, stream, true);
+}
+
+int qi_to_e4m3(qi_ctx* ctx, const uint16_t* x, int64_t n, uint8_t* y, void* stream) {
+  if (!ctx || !x || !y) return fail(QI_ERR_INVALID_ARG, "NULL argument");
+  if (n < 0 || n % 16) return fail(QI_ERR_INVALID_ARG, "n must be a multiple of 16");
+  if (!aligned16(x) || !aligned16(y)) return fail(QI_ERR_ALIGNMENT, "pointers must be 16-byte aligned");
+  Prof pr(ctx, QI_KCLASS_OTHER, S(stream));
+  if (qi::launch_bf16_to_e4m3(x, y, n, S(stream))) return cuda_fail("e4m3 cast launch");
+  return QI_OK;
+}
+
+int qi_ctx_set_attention_fp8(qi_ctx* ctx, int enable) {
+  if (!ctx) return fail(QI_ERR_INVALID_ARG, "NULL context");
+  ctx->attn_fp8 = enable ? 1 : 0;
   return QI_OK;
 }
 
@@ -1048,7 +1120,7 @@ int qi_denoise_step(qi_ctx* ctx, const qi_model* model, float* latents, const ui
                        b.block_mod + static_cast<size_t>(l) * 2 * 6 * H, gt, S_tok,
                        rope_cos + static_cast<size_t>(row0) * 64,
                        rope_sin + static_cast<size_t>(row0) * 64, kl, vl, b.block_ws,
-                       b.block_ws_bytes, st)))
+                       b.block_ws_bytes, st, ctx->attn_fp8 ? &b.f8 : nullptr)))
       return r;
   }
 
@@ -1135,6 +1207,8 @@ CfgBufs carve_cfg(Carve& c, const qi_dims& d, int T, int S_c, int S_u, int N, bo
   b.sb.lat_bf16 = c.take<uint16_t>(static_cast<size_t>(S_c + S_u) * P);
   b.sb.u_final = c.take<uint16_t>(static_cast<size_t>(2 * N) * H);
   b.sb.kv = own_kv ? c.take<uint16_t>(static_cast<size_t>(d.blocks) * 2 * (S_c + S_u) * H) : nullptr;
+  b.sb.f8.q = c.take<uint8_t>(static_cast<size_t>(T) * H);
+  b.sb.f8.kv = c.take<uint8_t>(static_cast<size_t>(2) * (S_c + S_u) * H);
   b.cos = c.take<float>(static_cast<size_t>(T) * 64);
   b.sin = c.take<float>(static_cast<size_t>(T) * 64);
   b.v = c.take<float>(static_cast<size_t>(2 * N) * P);
@@ -1271,7 +1345,8 @@ int qi_denoise_step_cfg(qi_ctx* ctx, const qi_model* model, float* latents, cons
     }
     if ((r = run_block_multi(ctx, d, model->blocks[l], b.sb.x, T, rows, 0,
                              b.sb.block_mod + static_cast<size_t>(l) * 2 * 6 * H, b.cos, b.sin, sa,
-                             2, b.sb.block_ws, b.sb.block_ws_bytes, st)))
+                             2, b.sb.block_ws, b.sb.block_ws_bytes, st,
+                             ctx->attn_fp8 ? &b.sb.f8 : nullptr)))
       return r;
   }
 

@@ -35,11 +35,51 @@ namespace qi {
 
 constexpr int FA_ROWS = 128;                   // rows per Q tile, keys per K/V tile
 constexpr int FA_THREADS = 320;
-constexpr int FA_TILE = 128 * 128 * 2;         // 32 KB: 128 rows x 128 bf16
-constexpr int FA_HALF = FA_TILE / 2;           // one 64-column (128-byte) swizzle region
 constexpr int FA_KST = 3;                      // K ring stages
 constexpr int FA_VST = 2;                      // V ring stages
-constexpr int FA_SMEM = 1024 + (2 + FA_KST + FA_VST) * FA_TILE + 256;
+
+// Tile geometry of the two element types.  A tile is 128 rows x 128 head
+// columns: bf16 -> two 64-column (128-byte) swizzle regions of 16 KB; e4m3 ->
+// one 128-column (128-byte) region of 16 KB.
+template <bool FP8>
+struct FaCfg {
+  static constexpr int TILE = FP8 ? 128 * 128 : 128 * 128 * 2;
+  static constexpr int REGION = 128 * 128;       // bytes of one 128-byte-wide swizzle region
+  static constexpr int REGIONS = TILE / REGION;  // 1 (e4m3) or 2 (bf16)
+  static constexpr int SMEM = 1024 + (2 + FA_KST + FA_VST) * TILE + 256;
+};
+
+// tcgen05.mma kind::f8f6f4 with A = B = e4m3 (format 0) and an fp32
+// accumulator: D format 1 (bits 4-5), B major bit 16, N >> 3 (17-22), M >> 4 (24-28).
+__host__ __device__ constexpr uint32_t umma_idesc_e4m3(int M, int N, bool b_mn_major) {
+  return (1u << 4) | (b_mn_major ? (1u << 16) : 0u) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+__device__ __forceinline__ void umma_e4m3(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
+}
+// D (TMEM) += A (TMEM, e4m3, 4 keys per 32-bit column) x B (smem descriptor).
+__device__ __forceinline__ void umma_e4m3_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate));
+}
+// Four values rounded to e4m3 (nearest, ties to even, saturating at +-448),
+// packed little-endian (a first).
+__device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
+  uint16_t lo, hi;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(b), "f"(a));
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(d), "f"(c));
+  return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+}
 
 // MN-major operand with the 128-byte swizzle: 64 elements (128 B) contiguous
 // along N, K rows 128 B apart inside an 8-row group, 8-row groups 1024 B
@@ -63,6 +103,12 @@ __device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]));
 }
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
@@ -113,9 +159,13 @@ __device__ __forceinline__ int fa_key_limit(const GroupTable& g, int t) {
   return g.end[group_of(g, t)];
 }
 
+template <bool FP8>
 __global__ void __launch_bounds__(FA_THREADS, 1)
     fa_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+  using Cfg = FaCfg<FP8>;
+  constexpr int FA_TILE = Cfg::TILE;
+  constexpr int FA_HALF = Cfg::REGION;
   int* status = p.status;
   extern __shared__ uint8_t fa_smem_raw[];
   const uint32_t raw_addr = smem_u32(fa_smem_raw);
@@ -183,7 +233,7 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
     if (lane == 0) {
       mbar_arrive_expect_tx(q_full, 2 * FA_TILE);
       for (int t = 0; t < 2; ++t)
-        for (int half = 0; half < 2; ++half)
+        for (int half = 0; half < Cfg::REGIONS; ++half)
           tma_load_2d(&tmQ, q_full, sQ + t * FA_TILE + half * FA_HALF, hc + 64 * half,
                       q0 + t * FA_ROWS);
       // K(j) into stage j % FA_KST once S_B(j - FA_KST) has read it; V(j) into
@@ -195,14 +245,14 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         const int ks = j % FA_KST, kr = j / FA_KST;
         if (!mbar_wait(&k_empty[ks], (kr & 1) ^ 1u, status)) { ok = false; break; }
         mbar_arrive_expect_tx(&k_full[ks], FA_TILE);
-        for (int half = 0; half < 2; ++half)
+        for (int half = 0; half < Cfg::REGIONS; ++half)
           tma_load_2d(&tmK, &k_full[ks], sK + ks * FA_TILE + half * FA_HALF, hc + 64 * half,
                       j * FA_ROWS);
         jk = j + 1;
         const int vs = j % FA_VST, vr = j / FA_VST;
         if (!mbar_wait(&v_empty[vs], (vr & 1) ^ 1u, status)) { ok = false; break; }
         mbar_arrive_expect_tx(&v_full[vs], FA_TILE);
-        for (int half = 0; half < 2; ++half)
+        for (int half = 0; half < Cfg::REGIONS; ++half)
           tma_load_2d(&tmV, &v_full[vs], sV + vs * FA_TILE + half * FA_HALF, hc + 64 * half,
                       j * FA_ROWS);
         jv = j + 1;
@@ -229,19 +279,27 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_s = umma_idesc(false, 128, 128);
-      constexpr uint32_t idesc_pv = umma_idesc(false, 128, 128) | (1u << 16);   // B MN-major
+      constexpr uint32_t idesc_s = FP8 ? umma_idesc_e4m3(128, 128, false) : umma_idesc(false, 128, 128);
+      constexpr uint32_t idesc_pv = FP8 ? umma_idesc_e4m3(128, 128, true)
+                                        : (umma_idesc(false, 128, 128) | (1u << 16));   // B MN-major
       bool ok = mbar_wait(q_full, 0, status);
       auto issue_s = [&](int X, int jj) -> bool {
         const int st = jj % FA_KST;
         if (!mbar_wait(&k_full[st], (jj / FA_KST) & 1, status)) return false;
         tc_fence_after();
         const uint32_t qa = smem_u32(sQ + X * FA_TILE), kb = smem_u32(sK + st * FA_TILE);
+        if (FP8) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * FA_HALF + (kk & 3) * 32;
-          umma_f16(tmem_base + X * 128, umma_desc_kmajor_sw128(qa + off),
-                   umma_desc_kmajor_sw128(kb + off), idesc_s, kk > 0);
+          for (int kk = 0; kk < 4; ++kk)   // 32 e4m3 values (32 bytes) of the head per instruction
+            umma_e4m3(tmem_base + X * 128, umma_desc_kmajor_sw128(qa + kk * 32),
+                      umma_desc_kmajor_sw128(kb + kk * 32), idesc_s, kk > 0);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * FA_HALF + (kk & 3) * 32;
+            umma_f16(tmem_base + X * 128, umma_desc_kmajor_sw128(qa + off),
+                     umma_desc_kmajor_sw128(kb + off), idesc_s, kk > 0);
+          }
         }
         umma_commit(&s_full[X]);
         return true;
@@ -252,11 +310,19 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         if (!mbar_wait(&p_full[X], jj & 1, status)) return false;
         tc_fence_after();
         const uint32_t vb = smem_u32(sV + st * FA_TILE);
+        if (FP8) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)   // 16 keys per instruction: two 8-row groups
-          umma_f16_ts(tmem_base + 256 + X * 128, tmem_base + X * 128 + kk * 8,
-                      umma_desc_mnmajor_sw128(vb + kk * 2048, FA_HALF), idesc_pv,
-                      (jj > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk)   // 32 keys per instruction (8 columns of e4m3 P)
+            umma_e4m3_ts(tmem_base + 256 + X * 128, tmem_base + X * 128 + kk * 8,
+                         umma_desc_mnmajor_sw128(vb + kk * 32 * 128, FA_HALF), idesc_pv,
+                         (jj > 0 || kk > 0) ? 1u : 0u);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)   // 16 keys per instruction: two 8-row groups
+            umma_f16_ts(tmem_base + 256 + X * 128, tmem_base + X * 128 + kk * 8,
+                        umma_desc_mnmajor_sw128(vb + kk * 2048, FA_HALF), idesc_pv,
+                        (jj > 0 || kk > 0) ? 1u : 0u);
+        }
         return true;
       };
       if (ok && n_kv > 0) {
@@ -353,7 +419,8 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
       uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
+        uint32_t pk[16];   // bf16: 16 words of 2 keys; e4m3: 8 words of 4 keys
+        float e0 = 0.f, e1 = 0.f;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(r[32 * c + 2 * i]),
@@ -364,9 +431,25 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
           const float p0 = ex2_approx(x0);
           const float p1 = ex2_approx(x1);
           acc2[i & 3] = f2_add(acc2[i & 3], f2_pack(p0, p1));
-          pk[i] = pack_bf16x2(p0, p1);
+          if (FP8) {
+            if (i & 1) {
+              pk[i >> 1] = pack_e4m3x4(e0, e1, p0, p1);   // keys 2i-2 .. 2i+1 of the chunk
+            } else {
+              e0 = p0;
+              e1 = p1;
+            }
+          } else {
+            pk[i] = pack_bf16x2(p0, p1);
+          }
         }
-        tmem_st16(tS + c * 16, pk);   // P (bf16) over the first 64 columns of S
+        if (FP8) {
+          uint32_t q8[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) q8[u] = pk[u];
+          tmem_st8(tS + c * 8, q8);     // P (e4m3) over the first 32 columns of S
+        } else {
+          tmem_st16(tS + c * 16, pk);   // P (bf16) over the first 64 columns of S
+        }
       }
       float sum;
       {
@@ -422,28 +505,34 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
   }
 }
 
-int launch_attention(const AttnParams& p, cudaStream_t st) {
-  if (p.Sq == 0) return 0;
-  static bool attr = false;
+template <bool FP8>
+static int launch_attention_t(const AttnParams& p, cudaStream_t st) {
+  using Cfg = FaCfg<FP8>;
+  static bool attr = false;   // per instantiation
   if (!attr) {
-    if (cudaFuncSetAttribute(fa_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, FA_SMEM) != cudaSuccess) {
+    if (cudaFuncSetAttribute(fa_kernel<FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM) != cudaSuccess) {
       launch_result();
       return -1;
     }
     attr = true;
   }
   const int W = p.heads * 128;
+  const CUtensorMapDataType dt = FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const uint64_t esz = FP8 ? 1 : 2;
+  const uint32_t box = FP8 ? 128 : 64;   // one 128-byte swizzle row per box
   CUtensorMap tq, tk, tv;
-  if (!make_tmap_2d(&tq, p.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, p.Sq,
-                    static_cast<uint64_t>(p.ldq) * 2, 64, FA_ROWS) ||
-      !make_tmap_2d(&tk, p.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, p.Sk,
-                    static_cast<uint64_t>(p.ldkv) * 2, 64, FA_ROWS) ||
-      !make_tmap_2d(&tv, p.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, p.Sk,
-                    static_cast<uint64_t>(p.ldkv) * 2, 64, FA_ROWS))
+  if (!make_tmap_2d(&tq, p.q, dt, W, p.Sq, static_cast<uint64_t>(p.ldq) * esz, box, FA_ROWS) ||
+      !make_tmap_2d(&tk, p.k, dt, W, p.Sk, static_cast<uint64_t>(p.ldkv) * esz, box, FA_ROWS) ||
+      !make_tmap_2d(&tv, p.v, dt, W, p.Sk, static_cast<uint64_t>(p.ldkv) * esz, box, FA_ROWS))
     return -2;
   dim3 grid((p.Sq + 2 * FA_ROWS - 1) / (2 * FA_ROWS), p.heads);
-  fa_kernel<<<grid, FA_THREADS, FA_SMEM, st>>>(tq, tk, tv, p);
+  fa_kernel<FP8><<<grid, FA_THREADS, Cfg::SMEM, st>>>(tq, tk, tv, p);
   return launch_result();
+}
+
+int launch_attention(const AttnParams& p, cudaStream_t st) {
+  if (p.Sq == 0) return 0;
+  return p.fp8 ? launch_attention_t<true>(p, st) : launch_attention_t<false>(p, st);
 }
 
 }  // namespace qi

@@ -130,10 +130,11 @@ int launch_qk_norm_rope(const QkNormRopeParams& p, cudaStream_t st);
 
 // Block-causal attention.
 struct AttnParams {
-  const uint16_t* q;      // [Sq, ldq]
-  const uint16_t* k;      // [Sk, ldkv]
-  const uint16_t* v;
-  uint16_t* o;            // [Sq, ldo]
+  const void* q;          // [Sq, ldq] bf16, or e4m3 bytes when fp8
+  const void* k;          // [Sk, ldkv]
+  const void* v;
+  int fp8;                // 1: q, k, v are e4m3 (tcgen05 kind::f8f6f4, P as e4m3)
+  uint16_t* o;            // [Sq, ldo] bf16
   int ldq, ldkv, ldo;
   int Sq, Sk, heads, q_offset;
   float sm_scale;
@@ -166,6 +167,8 @@ int launch_timestep_embedding(float t0, float t1, float* out, cudaStream_t st);
 int launch_timeout_probe(uint64_t limit_ns, int* status, cudaStream_t st);
 int launch_f32_to_bf16(const float* x, uint16_t* y, int64_t n, cudaStream_t st);
 int launch_euler(float* x, const float* v, int64_t n, float dt, cudaStream_t st);
+// bf16 -> e4m3 (round to nearest, ties to even, saturating), n % 8 == 0.
+int launch_bf16_to_e4m3(const uint16_t* x, uint8_t* y, int64_t n, cudaStream_t st);
 // Classifier-free guidance + Euler: v = v_u + g (v_c - v_u), x += dt v, fp32,
 // one rounding per operation; v_out (optional) receives v.
 int launch_cfg_euler(float* x, const float* v_c, const float* v_u, int64_t n, float g, float dt,

@@ -112,6 +112,11 @@ _SIGS = {
     "qi_attn_block_causal": [C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_int, C.c_void_p,
                              C.c_void_p, C.c_int, C.c_int, C.c_int, C.c_int,
                              C.POINTER(qi_groups), C.c_float, C.c_void_p, C.c_int, C.c_void_p],
+    "qi_attn_block_causal_fp8": [C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_int, C.c_void_p,
+                                 C.c_void_p, C.c_int, C.c_int, C.c_int, C.c_int,
+                                 C.POINTER(qi_groups), C.c_float, C.c_void_p, C.c_int, C.c_void_p],
+    "qi_to_e4m3": [C.c_void_p, C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p],
+    "qi_ctx_set_attention_fp8": [C.c_void_p, C.c_int],
     "qi_block_workspace_bytes": [C.POINTER(qi_dims), C.c_int, C.POINTER(C.c_size_t)],
     "qi_dit_block_forward": [C.c_void_p, C.POINTER(qi_dims), C.POINTER(qi_block_weights),
                              C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.POINTER(qi_groups),
@@ -218,6 +223,10 @@ class Context:
 
     def check(self, stream=None):
         check(lib().qi_ctx_check(self.handle, stream_ptr(stream)))
+
+    def set_attention_fp8(self, enable: bool):
+        """e4m3 attention in the steps run on this context (qi_ctx_set_attention_fp8)."""
+        check(lib().qi_ctx_set_attention_fp8(self.handle, 1 if enable else 0))
 
     def profile(self, enable: bool):
         """Reset launch counters; time every launch with CUDA events if enable."""
@@ -327,6 +336,30 @@ def qi_attn_block_causal(ctx: Context, q, k, v, groups: qi_groups, q_offset: int
                                      k.shape[1], Sk, heads, 128, C.byref(groups), sm_scale,
                                      ptr(o), o.shape[1], stream_ptr(stream)))
     return o
+
+
+def qi_attn_block_causal_fp8(ctx: Context, q8, k8, v8, groups: qi_groups, q_offset: int = 0,
+                             heads: Optional[int] = None, sm_scale: Optional[float] = None,
+                             o: Optional[torch.Tensor] = None, stream=None):
+    """Block-causal attention on e4m3 operands (uint8 tensors of e4m3 bytes)."""
+    Sq, W = q8.shape
+    Sk = k8.shape[0]
+    heads = heads if heads is not None else W // 128
+    sm_scale = sm_scale if sm_scale is not None else 128 ** -0.5
+    if o is None:
+        o = torch.empty((Sq, W), dtype=torch.bfloat16, device=q8.device)
+    check(lib().qi_attn_block_causal_fp8(ctx.handle, ptr(q8), q8.shape[1], Sq, q_offset, ptr(k8),
+                                         ptr(v8), k8.shape[1], Sk, heads, 128, C.byref(groups),
+                                         sm_scale, ptr(o), o.shape[1], stream_ptr(stream)))
+    return o
+
+
+def qi_to_e4m3(ctx: Context, x: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None):
+    """e4m3 bytes (uint8) of a bf16 tensor."""
+    if out is None:
+        out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    check(lib().qi_to_e4m3(ctx.handle, ptr(x), x.numel(), ptr(out), stream_ptr(stream)))
+    return out
 
 
 def dims_struct(hidden, heads, mlp, patch, blocks, eps=1e-6) -> qi_dims:

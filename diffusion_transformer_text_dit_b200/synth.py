@@ -29,7 +29,7 @@ import torch
 
 __all__ = [
     "Group", "DitConfig", "TINY", "BLOCK512", "STEP1024", "EDIT1024", "EDIT3REF1024", "CFG1024",
-    "GEN2048",
+    "GEN2048", "GEN2048_SCHED",
     "CONFIGS", "gen", "linear_weight", "bias", "norm_weight", "latents",
     "text_features", "ref_latents", "hidden_states", "mod_table", "block_weights", "model_weights",
 ]
@@ -60,6 +60,7 @@ class DitConfig:
     steps: int = 1
     t: Optional[float] = None                  # fixed timestep for block-only workloads
     uncond_text: int = 0                       # true CFG: negative-prompt tokens (0 = no guidance)
+    fp8_from_step: int = 0                     # precision schedule: fp8 attention from this step (1-based; 0 = never)
     guidance: float = 4.0                      # true CFG scale
 
     @property
@@ -129,7 +130,12 @@ GEN2048 = DitConfig("denoise40_2048px", 4096, 32, 128, 16384, 32, 64,
                     (Group(_TEXT, 512), Group(_IMAGE, 16384, (128, 128))),
                     steps=40, latent_seed=42)
 
-CONFIGS = {c.name: c for c in (TINY, BLOCK512, STEP1024, EDIT1024, EDIT3REF1024, CFG1024, GEN2048)}
+# The same denoise with the pages' precision schedule: the prefix pass and
+# steps 1-7 with bf16 attention, steps 8-40 with fp8 (e4m3) attention.
+GEN2048_SCHED = GEN2048.replace(name="denoise40_2048px_sched", fp8_from_step=8)
+
+CONFIGS = {c.name: c for c in (TINY, BLOCK512, STEP1024, EDIT1024, EDIT3REF1024, CFG1024, GEN2048,
+                               GEN2048_SCHED)}
 
 
 def gen(seed: int, *tags) -> torch.Generator:

@@ -267,6 +267,34 @@ int qi_attn_block_causal(qi_ctx* ctx, const uint16_t* q, int ldq, int Sq, int q_
 
 /* ------------------------------------------------------------------ block */
 
+/* Block-causal attention with e4m3 operands (the pages' reduced-precision
+ * attention for later denoising steps: [PX] Runtime precision and quality,
+ * "int8/fp8 attention for steps 8-40").  q, k, v are e4m3 bytes (ld in
+ * elements = bytes; see qi_to_e4m3); S = Q K^T accumulates in fp32 on
+ * tcgen05.mma kind::f8f6f4, the softmax runs in fp32 as in
+ * qi_attn_block_causal, P is rounded to e4m3 (nearest, ties to even,
+ * saturating) before P.V, the row sum uses the unrounded fp32 P values, and O
+ * is written as bf16.  No scale factors: e4m3 covers +-448, which the
+ * RMS-normalised q and k and the attention weights P <= 256 stay within.
+ * Other arguments and checks as qi_attn_block_causal; ldq and ldkv must be
+ * multiples of 16. */
+int qi_attn_block_causal_fp8(qi_ctx* ctx, const uint8_t* q, int ldq, int Sq, int q_offset,
+                             const uint8_t* k, const uint8_t* v, int ldkv, int Sk, int heads,
+                             int head_dim, const qi_groups* groups, float sm_scale, uint16_t* o,
+                             int ldo, void* stream);
+
+/* y = e4m3(x) for n bf16 values (round to nearest, ties to even, saturating at
+ * +-448); n % 16 == 0. */
+int qi_to_e4m3(qi_ctx* ctx, const uint16_t* x, int64_t n, uint8_t* y, void* stream);
+
+/* Attention precision of the steps run on this context (qi_denoise_step,
+ * qi_denoise_step_cfg): enable != 0 -> every block converts q and the
+ * layer's K/V rows to e4m3 and runs qi_attn_block_causal_fp8's kernel
+ * (the pages' schedule: the prefix pass and the first seven steps at full
+ * precision, later steps with fp8 attention - the caller switches between
+ * steps).  Block-level calls are not affected.  Default 0. */
+int qi_ctx_set_attention_fp8(qi_ctx* ctx, int enable);
+
 /* Workspace bytes needed by qi_dit_block_forward for T processed rows. */
 int qi_block_workspace_bytes(const qi_dims* dims, int T, size_t* bytes);
 

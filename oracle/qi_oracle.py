@@ -284,6 +284,85 @@ def attention_block_causal(q, k, v, q_group, k_group, sm_scale) -> np.ndarray:
     return out
 
 
+def e4m3_round(x) -> np.ndarray:
+    """Round to the nearest FP8 E4M3 value (ties to even), saturating at +-448.
+
+    E4M3: 1 sign, 4 exponent (bias 7), 3 mantissa bits; normal values
+    (1 + m/8) 2^(e-7) for e = 1..15 (all mantissas except e = 15, m = 7, the
+    NaN code), subnormals (m/8) 2^-6.  So the spacing of the values in
+    [2^e, 2^(e+1)) is 2^(e-3) for e >= -6, and 2^-9 below 2^-6.  (The
+    reduced-precision attention of "Qwen_Image-2.1-MXFP4-Paiton-RDNA4",
+    "Runtime precision and quality": int8/fp8 attention for later steps.)
+    """
+    x = np.asarray(x, F64)
+    a = np.abs(x)
+    _, ex = np.frexp(np.where(a > 0, a, 1.0))          # a = m 2^ex, m in [0.5, 1)
+    e = np.maximum(ex - 1, -6)                          # binade exponent, subnormals share -6
+    quantum = np.ldexp(1.0, e - 3)
+    r = np.rint(a / quantum) * quantum                  # a / quantum is exact: quantum is 2^k
+    r = np.minimum(r, 448.0)
+    return np.where(x < 0, -r, r)
+
+
+def attention_block_causal_fp8(q, k, v, q_group, k_group, sm_scale, tile=128,
+                               quantize=True, fp32_scores=True) -> np.ndarray:
+    """Block-causal attention with e4m3 operands, following the method of the
+    reduced-precision attention step by step (the reading of "int8/fp8
+    attention" this build takes; the pages give no further detail):
+
+      * q, k, v are rounded to e4m3;
+      * keys are processed in tiles of ``tile`` keys from key 0; each row keeps
+        a reference maximum m (base 2) set by the first tile and moved only
+        when a tile's row maximum exceeds it by more than 8, rescaling the
+        running sums by 2^(m_old - m_new);
+      * per tile P = 2^(s log2(e) sm_scale - m), rounded to e4m3 before it
+        multiplies V; the row sum takes the unrounded P;
+      * O = (sum_tiles P_e4m3 V) / (sum_tiles P).
+
+    With ``quantize=False, fp32_scores=False`` (no rounding anywhere) this is
+    exactly the masked softmax attention above, which pins the tile
+    bookkeeping.  By default S and the reference-maximum decisions are taken
+    in fp32, like the tensor-core accumulation and the softmax they restate;
+    everything else is float64.
+    """
+    rnd = e4m3_round if quantize else (lambda a: np.asarray(a, F64))
+    q = rnd(q)
+    k = rnd(k)
+    v = rnd(v)
+    qg = np.asarray(q_group)
+    kg = np.asarray(k_group)
+    Sq, heads, _ = q.shape
+    Sk = k.shape[0]
+    R = F32 if fp32_scores else F64
+    sl2 = R(R(sm_scale) * R(1.4426950408889634))
+    out = np.empty(q.shape, dtype=F64)
+    for h in range(heads):
+        for i in range(Sq):
+            vis = kg <= qg[i]
+            m = -np.inf
+            l = 0.0
+            o = np.zeros(q.shape[2], F64)
+            for t0 in range(0, Sk, tile):
+                t1 = min(t0 + tile, Sk)
+                sv = vis[t0:t1]
+                if not sv.any():
+                    continue
+                s = (k[t0:t1, h, :] @ q[i, h, :]).astype(R)        # scores of the tile
+                mx2 = R(R(s[sv].max()) * sl2)
+                if t0 == 0 or mx2 > R(m + R(8.0)):
+                    m_new = max(m, float(mx2)) if t0 else float(mx2)
+                    f = 2.0 ** (m - m_new) if t0 else 1.0
+                    l *= f
+                    o *= f
+                    m = R(m_new)
+                x = s.astype(F64) * float(sl2) - float(m)
+                p = np.where(sv, np.exp2(x), 0.0)
+                l += p.sum()
+                o += rnd(p) @ v[t0:t1, h, :]
+            out[i, h, :] = o / l
+    return out
+
+
 # ----------------------------------------------------------------------------
 # One transformer block
 # ----------------------------------------------------------------------------
@@ -302,7 +381,7 @@ def prepare_block(wts: dict) -> dict:
 
 def dit_block(x, pw: dict, mod, row_set, q_group, k_group, cos, sin, heads, head_dim, eps,
               kv_prefix: Optional[Tuple[np.ndarray, np.ndarray]] = None,
-              return_kv: bool = False):
+              return_kv: bool = False, attn: str = "bf16"):
     """One single-stream block on the rows in ``x``.
 
     x: [T, H] residual stream of the rows processed (float64);
@@ -340,7 +419,10 @@ def dit_block(x, pw: dict, mod, row_set, q_group, k_group, cos, sin, heads, head
         v_all = np.concatenate([kv_prefix[1], v], axis=0)
     else:
         k_all, v_all = k, v
-    o = attention_block_causal(q, k_all, v_all, q_group, k_group, 1.0 / math.sqrt(head_dim))
+    if attn == "fp8":
+        o = attention_block_causal_fp8(q, k_all, v_all, q_group, k_group, 1.0 / math.sqrt(head_dim))
+    else:
+        o = attention_block_causal(q, k_all, v_all, q_group, k_group, 1.0 / math.sqrt(head_dim))
     # The attention output and the GELU output are activation tensors of the
     # BF16 transformer (FlagOS card: the Linears outside the W8A8 set and the
     # activations stay BF16), so the per-token quantizer sees them as bf16
@@ -449,7 +531,7 @@ def cfg_combine(v_cond, v_uncond, guidance) -> np.ndarray:
 def step_forward(latents, txt, ref_latents, mw: dict, blocks_pw: Sequence[dict],
                  blocks_mod_w: Sequence[Tuple], groups, heads, head_dim, eps, sigma, sigma_next,
                  kv_cache: Optional[Dict[int, Tuple[np.ndarray, np.ndarray]]] = None,
-                 mode: str = "none", return_v: bool = False):
+                 mode: str = "none", return_v: bool = False, attn: str = "bf16"):
     """One FlowMatch Euler step of the DiT.
 
     latents [N, P] fp32 (target tokens); txt [L, H] text features (bf16 values);
@@ -495,7 +577,8 @@ def step_forward(latents, txt, ref_latents, mw: dict, blocks_pw: Sequence[dict],
         mod = np.stack([adaln_rows(temb_0, wm, bm), adaln_rows(temb_t, wm, bm)])
         kvp = kv_cache[l] if mode == "read" else None
         x, kv = dit_block(x, pw, mod, row_set_all[rows], gid[rows], gid, cos_all[rows],
-                          sin_all[rows], heads, head_dim, eps, kv_prefix=kvp, return_kv=True)
+                          sin_all[rows], heads, head_dim, eps, kv_prefix=kvp, return_kv=True,
+                          attn=attn)
         if mode == "write":
             kv_cache[l] = (kv[0][:P_tok], kv[1][:P_tok])
 

@@ -324,6 +324,58 @@ def test_attention_many_groups_reduce_to_full_attention_on_prefixes():
     assert np.allclose(out[9:12], _sdpa(q[9:12] * sc, k[:12], v[:12]), atol=1e-12)
 
 
+def _e4m3_decode(b):
+    # straight from the format: 1 sign, 4 exponent (bias 7), 3 mantissa bits
+    sgn = -1.0 if b & 0x80 else 1.0
+    e, m = (b >> 3) & 15, b & 7
+    if e == 15 and m == 7:
+        return None                                   # NaN code
+    return sgn * (m / 8.0 * 2.0 ** -6 if e == 0 else (1 + m / 8.0) * 2.0 ** (e - 7))
+
+
+def test_e4m3_round_codes_ties_and_saturation():
+    vals = sorted({v for v in (_e4m3_decode(b) for b in range(256)) if v is not None})
+    assert len(vals) == 253 and max(vals) == 448.0 and min(vals) == -448.0
+    a = np.array(vals)
+    assert np.array_equal(O.e4m3_round(a), a)         # every value is its own rounding
+    pos = np.array([v for v in vals if v >= 0])
+    codes = {(_e4m3_decode(b)): b for b in range(128) if _e4m3_decode(b) is not None}
+    mid = (pos[:-1] + pos[1:]) / 2                    # ties go to the even mantissa
+    want = np.where([codes[lo] % 2 == 0 for lo in pos[:-1]], pos[:-1], pos[1:])
+    assert np.array_equal(O.e4m3_round(mid), want)
+    assert O.e4m3_round(np.array([0.3]))[0] == 0.3125  # quantum 2^-5 in [0.25, 0.5)
+    assert np.array_equal(O.e4m3_round(np.array([460.0, 1e6, -500.0])), [448.0, 448.0, -448.0])
+    assert np.array_equal(O.e4m3_round(np.array([2.0 ** -10, 1.5 * 2.0 ** -10, -2.0 ** -12])),
+                          [0.0, 2.0 ** -9, 0.0])
+
+
+def test_attention_fp8_unquantized_reduces_to_exact_attention():
+    ends = [6, 13, 30]
+    g = O.group_ids(ends)
+    q, k, v = (rng.standard_normal((30, 2, 8)) for _ in range(3))
+    # scores that grow along the keys force the reference-maximum rescales
+    k[:, :, 0] += np.linspace(0, 60, 30)[:, None]
+    q[:, :, 0] = np.abs(q[:, :, 0]) + 1.0
+    ref = O.attention_block_causal(q, k, v, g, g, 0.4)
+    for tile in (4, 7, 128):
+        out = O.attention_block_causal_fp8(q, k, v, g, g, 0.4, tile=tile, quantize=False,
+                                           fp32_scores=False)
+        assert np.allclose(out, ref, rtol=1e-10, atol=1e-12)
+        # fp32 scores: within fp32 rounding of the scores
+        out32 = O.attention_block_causal_fp8(q, k, v, g, g, 0.4, tile=tile, quantize=False)
+        assert np.linalg.norm(out32 - ref) / np.linalg.norm(ref) < 1e-5
+
+
+def test_attention_fp8_error_is_e4m3_sized():
+    ends = [16, 80]
+    g = O.group_ids(ends)
+    q, k, v = (rng.standard_normal((80, 2, 32)) for _ in range(3))
+    ref = O.attention_block_causal(q, k, v, g, g, 1 / math.sqrt(32))
+    out = O.attention_block_causal_fp8(q, k, v, g, g, 1 / math.sqrt(32), tile=16)
+    err = np.linalg.norm(out - ref) / np.linalg.norm(ref)
+    assert 1e-3 < err < 8e-2
+
+
 # ------------------------------------------------------------ timestep
 
 
