@@ -939,6 +939,17 @@ int qi_to_e4m3(qi_ctx* ctx, const uint16_t* x, int64_t n, uint8_t* y, void* stre
   return QI_OK;
 }
 
+int qi_mxfp4_decode(qi_ctx* ctx, const uint8_t* packed, const uint8_t* scales, int n,
+                    int k_stored, int k, float* w, void* stream) {
+  if (!ctx || !packed || !scales || !w) return fail(QI_ERR_INVALID_ARG, "NULL argument");
+  if (n < 0 || k_stored < 32 || k_stored % 32 || k < 1 || k > k_stored)
+    return fail(QI_ERR_INVALID_ARG, "need k_stored a positive multiple of 32 and 1 <= k <= k_stored");
+  Prof pr(ctx, QI_KCLASS_OTHER, S(stream));
+  if (qi::launch_mxfp4_decode(packed, scales, n, k_stored, k, w, S(stream)))
+    return cuda_fail("MXFP4 decode launch");
+  return QI_OK;
+}
+
 int qi_ctx_set_attention_fp8(qi_ctx* ctx, int enable) {
   if (!ctx) return fail(QI_ERR_INVALID_ARG, "NULL context");
   ctx->attn_fp8 = enable ? 1 : 0;

@@ -167,6 +167,9 @@ int launch_timestep_embedding(float t0, float t1, float* out, cudaStream_t st);
 int launch_timeout_probe(uint64_t limit_ns, int* status, cudaStream_t st);
 int launch_f32_to_bf16(const float* x, uint16_t* y, int64_t n, cudaStream_t st);
 int launch_euler(float* x, const float* v, int64_t n, float dt, cudaStream_t st);
+// MXFP4 (E2M1 codes, low nibble first; E8M0 scale per 32 columns) -> fp32 [n, k].
+int launch_mxfp4_decode(const uint8_t* packed, const uint8_t* scales, int n, int k_stored, int k,
+                        float* w, cudaStream_t st);
 // bf16 -> e4m3 (round to nearest, ties to even, saturating), n % 8 == 0.
 int launch_bf16_to_e4m3(const uint16_t* x, uint8_t* y, int64_t n, cudaStream_t st);
 // Classifier-free guidance + Euler: v = v_u + g (v_c - v_u), x += dt v, fp32,

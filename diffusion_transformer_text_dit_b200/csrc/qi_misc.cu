@@ -239,6 +239,50 @@ int launch_euler(float* x, const float* v, int64_t n, float dt, cudaStream_t st)
   return launch_result();
 }
 
+// MXFP4 weights -> fp32: w[n, k] = e2m1(code) * 2^(scale[n, k / 32] - 127).
+// E2M1 codes (1 sign, 2 exponent, 1 mantissa bit): magnitudes 0, 0.5, 1, 1.5,
+// 2, 3, 4, 6; two codes per byte, the lower column in the low nibble; one
+// E8M0 scale byte per 32 columns (255 = NaN).  One thread per packed byte.
+__global__ void mxfp4_decode_kernel(const uint8_t* __restrict__ packed,
+                                    const uint8_t* __restrict__ scales, int n, int k_stored, int k,
+                                    float* __restrict__ w) {
+  const int bytes_per_row = k_stored / 2;
+  const int64_t total = static_cast<int64_t>(n) * bytes_per_row;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int row = static_cast<int>(i / bytes_per_row);
+    const int col = static_cast<int>(i % bytes_per_row) * 2;
+    if (col >= k) continue;
+    const uint8_t b = packed[i];
+    const uint8_t e8 = scales[static_cast<int64_t>(row) * (k_stored / 32) + col / 32];
+    // 2^(e8 - 127) built from its bits: exponent field e8 for e8 >= 1, the
+    // denormal 2^-127 for e8 = 0; 255 encodes NaN
+    const float scale = e8 == 255 ? __int_as_float(0x7FC00000)
+                                  : __int_as_float(e8 == 0 ? 0x00400000 : static_cast<int>(e8) << 23);
+    float out[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int c = (b >> (4 * h)) & 15;
+      const int e = (c >> 1) & 3, m = c & 1;
+      float mag = e == 0 ? 0.5f * m : (1.0f + 0.5f * m) * static_cast<float>(1 << (e - 1));
+      out[h] = (c & 8) ? -mag * scale : mag * scale;
+    }
+    float* dst = w + static_cast<int64_t>(row) * k + col;
+    dst[0] = out[0];
+    if (col + 1 < k) dst[1] = out[1];
+  }
+}
+
+int launch_mxfp4_decode(const uint8_t* packed, const uint8_t* scales, int n, int k_stored, int k,
+                        float* w, cudaStream_t st) {
+  const int64_t total = static_cast<int64_t>(n) * (k_stored / 2);
+  if (total == 0) return 0;
+  int64_t g = (total + 255) / 256;
+  if (g > 148 * 32) g = 148 * 32;
+  mxfp4_decode_kernel<<<static_cast<int>(g), 256, 0, st>>>(packed, scales, n, k_stored, k, w);
+  return launch_result();
+}
+
 // bf16 -> e4m3 (nearest, ties to even, saturating at +-448), 8 values per
 // thread step: the operands of the fp8 attention.
 __global__ void bf16_to_e4m3_kernel(const uint4* __restrict__ x, uint2* __restrict__ y, int64_t n8) {

@@ -117,6 +117,8 @@ _SIGS = {
                                  C.POINTER(qi_groups), C.c_float, C.c_void_p, C.c_int, C.c_void_p],
     "qi_to_e4m3": [C.c_void_p, C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p],
     "qi_ctx_set_attention_fp8": [C.c_void_p, C.c_int],
+    "qi_mxfp4_decode": [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_int,
+                        C.c_void_p, C.c_void_p],
     "qi_block_workspace_bytes": [C.POINTER(qi_dims), C.c_int, C.POINTER(C.c_size_t)],
     "qi_dit_block_forward": [C.c_void_p, C.POINTER(qi_dims), C.POINTER(qi_block_weights),
                              C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.POINTER(qi_groups),
@@ -359,6 +361,18 @@ def qi_to_e4m3(ctx: Context, x: torch.Tensor, out: Optional[torch.Tensor] = None
     if out is None:
         out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
     check(lib().qi_to_e4m3(ctx.handle, ptr(x), x.numel(), ptr(out), stream_ptr(stream)))
+    return out
+
+
+def qi_mxfp4_decode(ctx: Context, packed, scales, k: Optional[int] = None, out=None, stream=None):
+    """fp32 weights [n, k] from MXFP4 codes (packed [n, k_stored/2] uint8) and E8M0 scales."""
+    n, half = packed.shape
+    k_stored = 2 * half
+    k = k_stored if k is None else k
+    if out is None:
+        out = torch.empty((n, k), dtype=torch.float32, device=packed.device)
+    check(lib().qi_mxfp4_decode(ctx.handle, ptr(packed), ptr(scales), n, k_stored, k, ptr(out),
+                                stream_ptr(stream)))
     return out
 
 

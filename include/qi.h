@@ -287,6 +287,19 @@ int qi_attn_block_causal_fp8(qi_ctx* ctx, const uint8_t* q, int ldq, int Sq, int
  * +-448); n % 16 == 0. */
 int qi_to_e4m3(qi_ctx* ctx, const uint16_t* x, int64_t n, uint8_t* y, void* stream);
 
+/* MXFP4 checkpoint weights -> fp32 ([PX] Runtime precision and quality /
+ * What was quantized: E2M1 values packed low nibble first, an E8M0 scale per
+ * group of 32 input columns; rows zero-padded to a multiple of 32 columns,
+ * the padding removed on load).  packed [n, k_stored/2] bytes, scales
+ * [n, k_stored/32] bytes, w [n, k] fp32 with k <= k_stored:
+ *   w[r, c] = e2m1(code) * 2^(scale[r, c/32] - 127)   (E8M0 255 -> NaN)
+ * E2M1 magnitudes (exponent bias 1, one mantissa bit): 0, 0.5, 1, 1.5, 2, 3,
+ * 4, 6.  The result feeds qi_prepare_w8 like any fp32 weight.  The runtime
+ * keeps the W8A8 int8 codes: the pages' MXFP4 is a storage format that a
+ * loader reconstructs for computation. */
+int qi_mxfp4_decode(qi_ctx* ctx, const uint8_t* packed, const uint8_t* scales, int n,
+                    int k_stored, int k, float* w, void* stream);
+
 /* Attention precision of the steps run on this context (qi_denoise_step,
  * qi_denoise_step_cfg): enable != 0 -> every block converts q and the
  * layer's K/V rows to e4m3 and runs qi_attn_block_causal_fp8's kernel

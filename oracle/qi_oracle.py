@@ -284,6 +284,35 @@ def attention_block_causal(q, k, v, q_group, k_group, sm_scale) -> np.ndarray:
     return out
 
 
+def mxfp4_decode(packed, scales, k=None) -> np.ndarray:
+    """MXFP4 checkpoint weights to fp32 ("Qwen_Image-2.1-MXFP4-Paiton-RDNA4",
+    "What was quantized": E2M1 values packed low nibble first, one E8M0 scale
+    per group of 32 input columns, rows zero-padded to a multiple of 32 columns
+    and the padding removed on load).
+
+    E2M1: code = sign << 3 | exponent << 1 | mantissa, exponent bias 1:
+    exponent 0 -> mantissa * 0.5 (subnormal), else (1 + mantissa / 2) 2^(e-1).
+    E8M0: 2^(e - 127), 255 = NaN.  w[r, c] = e2m1 * scale, in fp32.
+    """
+    packed = np.asarray(packed, np.uint8)
+    scales = np.asarray(scales, np.uint8)
+    n, half = packed.shape
+    k_stored = 2 * half
+    k = k_stored if k is None else k
+    codes = np.empty((n, k_stored), np.int64)
+    codes[:, 0::2] = packed & 15
+    codes[:, 1::2] = packed >> 4
+    e = (codes >> 1) & 3
+    m = codes & 1
+    mag = np.where(e == 0, 0.5 * m, (1.0 + 0.5 * m) * np.exp2(np.maximum(e - 1, 0)))
+    val = np.where(codes & 8, -mag, mag).astype(F32)
+    sc = np.ldexp(np.float32(1.0), np.minimum(scales.astype(np.int64), 254) - 127).astype(F32)
+    sc = np.where(scales == 255, np.float32(np.nan), sc).astype(F32)
+    with np.errstate(over="ignore"):   # 6 x 2^127 overflows to inf in fp32, as it must
+        w = (val * np.repeat(sc, 32, axis=1)).astype(F32)
+    return w[:, :k]
+
+
 def e4m3_round(x) -> np.ndarray:
     """Round to the nearest FP8 E4M3 value (ties to even), saturating at +-448.
 

@@ -150,3 +150,21 @@ def test_schedule_bf16_prefix_then_fp8_steps_vs_oracle(ctx):
                            cfg.eps, float(sig[7]), float(sig[8]), kv_cache=cache, mode="read",
                            return_v=True, attn="fp8")
     assert rel_l2(v.numpy(), ov) < 3e-2
+
+
+# ------------------------------------------------------------------ MXFP4 checkpoint weights
+
+def test_mxfp4_decode_bit_exact_and_w8_prepare(ctx):
+    g = _gen(11)
+    n, k_stored, k = 96, 4096 + 32, 4096 + 16          # padded rows, padding removed on decode
+    packed = torch.randint(0, 256, (n, k_stored // 2), generator=g, dtype=torch.uint8)
+    scales = torch.randint(110, 135, (n, k_stored // 32), generator=g, dtype=torch.uint8)
+    scales[0, :4] = torch.tensor([0, 1, 254, 255], dtype=torch.uint8)   # denormal, extremes, NaN
+    w = qi.qi_mxfp4_decode(ctx, cuda(packed), cuda(scales), k=k).cpu().numpy()
+    ref = O.mxfp4_decode(packed.numpy(), scales.numpy(), k=k)
+    assert np.array_equal(w, ref, equal_nan=True)
+    # the decoded (finite) weights go through the W8A8 weight preparation unchanged
+    wd = torch.from_numpy(ref[1:]).contiguous()
+    q, s, rs = qi.qi_prepare_w8(ctx, cuda(wd))
+    oq, os_, ors = O.prepare_w8(ref[1:])
+    assert np.array_equal(q.cpu().numpy(), oq) and np.array_equal(s.cpu().numpy(), os_)

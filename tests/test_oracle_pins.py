@@ -324,6 +324,22 @@ def test_attention_many_groups_reduce_to_full_attention_on_prefixes():
     assert np.allclose(out[9:12], _sdpa(q[9:12] * sc, k[:12], v[:12]), atol=1e-12)
 
 
+def test_mxfp4_decode_format():
+    # one row of 64 codes: the 16 E2M1 codes twice per 32-column group, scales 2^0 and 2^3
+    codes = np.array(list(range(16)) * 4, np.uint8)
+    packed = (codes[0::2] | (codes[1::2] << 4)).astype(np.uint8)[None, :]   # low nibble first
+    scales = np.array([[127, 130]], np.uint8)
+    w = O.mxfp4_decode(packed, scales)
+    e2m1 = [0, 0.5, 1, 1.5, 2, 3, 4, 6, -0.0, -0.5, -1, -1.5, -2, -3, -4, -6]
+    assert np.array_equal(w[0, :16], e2m1) and np.array_equal(w[0, 16:32], e2m1)
+    assert np.array_equal(w[0, 32:48], np.array(e2m1) * 8)
+    # padding columns are dropped; E8M0 extremes: 2^-127 (denormal) and NaN
+    assert O.mxfp4_decode(packed, scales, k=40).shape == (1, 40)
+    ext = O.mxfp4_decode(np.full((1, 16), 0x22, np.uint8), np.array([[0]], np.uint8))
+    assert ext[0, 0] == np.float32(2.0 ** -127)          # code 2 = 1.0, E8M0 0 = 2^-127 (an fp32 denormal)
+    assert np.all(np.isnan(O.mxfp4_decode(packed[:, :16], np.array([[255]], np.uint8))))
+
+
 def _e4m3_decode(b):
     # straight from the format: 1 sign, 4 exponent (bias 7), 3 mantissa bits
     sgn = -1.0 if b & 0x80 else 1.0
