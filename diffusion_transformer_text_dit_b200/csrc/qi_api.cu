@@ -304,6 +304,7 @@ int run_quant(qi_ctx* ctx, const void* x, bool xbf16, int M, int K, int ldx,
   p.s = s;
   p.zp = zp;
   p.u_bf16 = u_bf16;
+  p.status = ctx->status;
   Prof pr(ctx, QI_KCLASS_QUANT, st);
   if (qi::launch_quant(p, st) != 0) return cuda_fail("quantize launch");
   return QI_OK;

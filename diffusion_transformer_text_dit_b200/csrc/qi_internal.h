@@ -105,6 +105,7 @@ struct QuantParams {
   // plain variant: the row's range was published by the producer as
   // [float bits of -min, float bits of max] (both >= 0); no reduction needed
   const uint32_t* range;
+  int* status;            // device status word (bounded wait for the row copy)
 };
 int launch_quant(const QuantParams& p, cudaStream_t st);
 

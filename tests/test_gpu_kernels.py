@@ -42,7 +42,7 @@ def test_prepare_w8_bit_exact(ctx, n, k):
 
 # ------------------------------------------------------------------ activation quant
 
-@pytest.mark.parametrize("M,K", [(1, 256), (80, 256), (77, 4096), (1280, 4096), (33, 16384)])
+@pytest.mark.parametrize("M,K", [(1, 256), (80, 256), (5, 1032), (77, 4096), (1280, 4096), (33, 16384)])
 def test_quantize_plain_bit_exact(ctx, M, K):
     x = _bf16((M, K), M * 7 + K, 1.0) * torch.logspace(-3, 2, M).reshape(M, 1).to(torch.bfloat16)
     x = x.to(torch.bfloat16)
@@ -58,8 +58,9 @@ def test_quantize_plain_bit_exact(ctx, M, K):
     assert np.array_equal(q.cpu().numpy(), oq)
 
 
-def test_quantize_fp32_input_bit_exact(ctx):
-    x = torch.randn(300, 4096, generator=_gen(5)) * 3 + 0.7
+@pytest.mark.parametrize("K", [4096, 1000])
+def test_quantize_fp32_input_bit_exact(ctx, K):
+    x = torch.randn(300, K, generator=_gen(5)) * 3 + 0.7
     q, s, zp = qi.qi_quantize_act(ctx, cuda(x))
     oq, os_, ozp = O.quantize_act(x.numpy())
     assert np.array_equal(s.cpu().numpy(), os_) and np.array_equal(zp.cpu().numpy(), ozp)
