@@ -227,6 +227,8 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();      // the previous kernel's outputs are complete from here on
+  pdl_trigger();
 
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
@@ -526,7 +528,7 @@ static int launch_attention_t(const AttnParams& p, cudaStream_t st) {
       !make_tmap_2d(&tv, p.v, dt, W, p.Sk, static_cast<uint64_t>(p.ldkv) * esz, box, FA_ROWS))
     return -2;
   dim3 grid((p.Sq + 2 * FA_ROWS - 1) / (2 * FA_ROWS), p.heads);
-  fa_kernel<FP8><<<grid, FA_THREADS, Cfg::SMEM, st>>>(tq, tk, tv, p);
+  launch_pdl(fa_kernel<FP8>, grid, dim3(FA_THREADS), Cfg::SMEM, st, 1, tq, tk, tv, p);
   return launch_result();
 }
 

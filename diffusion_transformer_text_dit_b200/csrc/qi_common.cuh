@@ -115,6 +115,18 @@ __device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, uint64_t* ba
       : "memory");
 }
 
+// ---------------------------------------------------------------- dependent launch
+
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may be scheduled while the previous kernel of the stream is
+// still running.  pdl_wait() blocks until that kernel has completed and its
+// memory operations are visible (a no-op for an ordinary launch), so it comes
+// before the first access to memory that the previous kernel writes or reads;
+// pdl_trigger() lets the next kernel of the stream be scheduled (it still
+// waits in its own pdl_wait() for this one to complete).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // 1-D bulk copy of `bytes` from global to this CTA's shared memory, completing
 // on `bar`.  Both addresses 16-byte aligned, bytes a multiple of 16.
 __device__ __forceinline__ void bulk_load_1d(void* smem, const void* gmem, uint32_t bytes,

@@ -421,6 +421,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();      // the previous kernel's outputs are complete from here on
+  pdl_trigger();
 
   constexpr int ELEMS_PER_KB = I8 ? 128 : 64;
 
@@ -701,6 +703,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   cluster_sync_all();   // barriers of both CTAs initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();      // the previous kernel's outputs are complete from here on
+  pdl_trigger();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (both CTAs)
@@ -827,7 +831,7 @@ static int launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const Gem
   }
   const int tiles = ((p.M + GEMM_BM - 1) / GEMM_BM) * ((p.N + BN - 1) / BN);
   const int grid = tiles < num_sms ? tiles : num_sms;
-  kern<<<grid, GEMM_THREADS, C::SMEM_BYTES, st>>>(ta, tb, p);
+  launch_pdl(kern, dim3(grid), dim3(GEMM_THREADS), C::SMEM_BYTES, st, 1, ta, tb, p);
   return launch_result();
 }
 
@@ -868,19 +872,7 @@ static int launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const 
                             int max_pairs, cudaStream_t st) {
   const int tiles = ((p.M + 2 * GEMM_BM - 1) / (2 * GEMM_BM)) * ((p.N + 255) / 256);
   const int pairs = tiles < max_pairs ? tiles : max_pairs;
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.gridDim = dim3(2 * pairs, 1, 1);
-  cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
-  cfg.dynamicSmemBytes = PAIR_SMEM_BYTES;
-  cfg.stream = st;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaLaunchKernelEx(&cfg, gemm_pair_kernel<EPI>, ta, tb, p);
+  launch_pdl(gemm_pair_kernel<EPI>, dim3(2 * pairs), dim3(GEMM_THREADS), PAIR_SMEM_BYTES, st, 2, ta, tb, p);
   return launch_result();
 }
 

@@ -23,6 +23,35 @@ inline int launch_result() {
   return -1;
 }
 
+// Launch `kern` with programmatic stream serialization (and, for
+// cluster_x > 1, clusters of cluster_x CTAs): the kernel may be scheduled
+// while the previous kernel of the stream drains; it calls pdl_wait() before
+// its first access to memory that kernel touches.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, unsigned cluster_x, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  unsigned na = 0;
+  attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[na].val.programmaticStreamSerializationAllowed = 1;
+  ++na;
+  if (cluster_x > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = cluster_x;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 enum GemmEpilogue {
   EPI_BF16 = 0,    // y (bf16) = value
   EPI_GELU = 1,    // y (bf16) = GELU_tanh(bf16(value))

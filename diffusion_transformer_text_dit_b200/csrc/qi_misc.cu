@@ -95,6 +95,8 @@ __device__ __forceinline__ float dot8(const uint4 w, const float4 a, const float
 
 __global__ void __launch_bounds__(GEMV_THREADS) gemv_kernel(const GemvParams p) {
   extern __shared__ float4 xs4[];
+  pdl_wait();
+  pdl_trigger();
   float* xs = reinterpret_cast<float*>(xs4);
   const int total_in = p.R * p.k;
   for (int i = threadIdx.x; i < total_in; i += GEMV_THREADS) {
@@ -186,7 +188,7 @@ int launch_gemv(const GemvParams& p, cudaStream_t st) {
   int grid = (total + per_cta - 1) / per_cta;
   const int max_grid = sms * 8;
   if (grid > max_grid) grid = max_grid;
-  gemv_kernel<<<grid, GEMV_THREADS, smem, st>>>(p);
+  launch_pdl(gemv_kernel, dim3(grid), dim3(GEMV_THREADS), smem, st, 1, p);
   return launch_result();
 }
 
@@ -195,6 +197,8 @@ int launch_gemv(const GemvParams& p, cudaStream_t st) {
 // out[r] = [cos(1000 t_r f_i), sin(1000 t_r f_i)], f_i = exp(-ln(1e4) i / 128), i < 128,
 // for the two timesteps t_0 (row 0) and t_1 (row 1).  Evaluated in double.
 __global__ void timestep_embedding_kernel(float t0, float t1, float* out) {
+  pdl_wait();
+  pdl_trigger();
   const int r = blockIdx.x;
   const int i = threadIdx.x;   // 0..127
   const double f = exp(-log(10000.0) * static_cast<double>(i) / 128.0);
@@ -204,11 +208,13 @@ __global__ void timestep_embedding_kernel(float t0, float t1, float* out) {
 }
 
 int launch_timestep_embedding(float t0, float t1, float* out, cudaStream_t st) {
-  timestep_embedding_kernel<<<2, 128, 0, st>>>(t0, t1, out);
+  launch_pdl(timestep_embedding_kernel, dim3(2), dim3(128), 0, st, 1, t0, t1, out);
   return launch_result();
 }
 
 __global__ void f32_to_bf16_kernel(const float* __restrict__ x, uint16_t* __restrict__ y, int64_t n) {
+  pdl_wait();
+  pdl_trigger();
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     __nv_bfloat16 h = __float2bfloat16_rn(x[i]);
@@ -220,12 +226,14 @@ int launch_f32_to_bf16(const float* x, uint16_t* y, int64_t n, cudaStream_t st) 
   if (n == 0) return 0;
   int64_t g = (n + 255) / 256;
   if (g > 148 * 16) g = 148 * 16;
-  f32_to_bf16_kernel<<<static_cast<int>(g), 256, 0, st>>>(x, y, n);
+  launch_pdl(f32_to_bf16_kernel, dim3(static_cast<unsigned>(g)), dim3(256), 0, st, 1, x, y, n);
   return launch_result();
 }
 
 // x += dt * v in fp32, one rounding per operation (no fused multiply-add).
 __global__ void euler_kernel(float* __restrict__ x, const float* __restrict__ v, int64_t n, float dt) {
+  pdl_wait();
+  pdl_trigger();
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x)
     x[i] = __fadd_rn(x[i], __fmul_rn(dt, v[i]));
@@ -235,7 +243,7 @@ int launch_euler(float* x, const float* v, int64_t n, float dt, cudaStream_t st)
   if (n == 0) return 0;
   int64_t g = (n + 255) / 256;
   if (g > 148 * 16) g = 148 * 16;
-  euler_kernel<<<static_cast<int>(g), 256, 0, st>>>(x, v, n, dt);
+  launch_pdl(euler_kernel, dim3(static_cast<unsigned>(g)), dim3(256), 0, st, 1, x, v, n, dt);
   return launch_result();
 }
 
@@ -286,6 +294,8 @@ int launch_mxfp4_decode(const uint8_t* packed, const uint8_t* scales, int n, int
 // bf16 -> e4m3 (nearest, ties to even, saturating at +-448), 8 values per
 // thread step: the operands of the fp8 attention.
 __global__ void bf16_to_e4m3_kernel(const uint4* __restrict__ x, uint2* __restrict__ y, int64_t n8) {
+  pdl_wait();
+  pdl_trigger();
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n8;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const uint4 v = x[i];
@@ -307,8 +317,8 @@ int launch_bf16_to_e4m3(const uint16_t* x, uint8_t* y, int64_t n, cudaStream_t s
   const int64_t n8 = n / 8;
   int64_t g = (n8 + 255) / 256;
   if (g > 148 * 16) g = 148 * 16;
-  bf16_to_e4m3_kernel<<<static_cast<int>(g), 256, 0, st>>>(reinterpret_cast<const uint4*>(x),
-                                                          reinterpret_cast<uint2*>(y), n8);
+  launch_pdl(bf16_to_e4m3_kernel, dim3(static_cast<unsigned>(g)), dim3(256), 0, st, 1,
+             reinterpret_cast<const uint4*>(x), reinterpret_cast<uint2*>(y), n8);
   return launch_result();
 }
 
@@ -319,6 +329,8 @@ int launch_bf16_to_e4m3(const uint16_t* x, uint8_t* y, int64_t n, cudaStream_t s
 __global__ void cfg_euler_kernel(float* __restrict__ x, const float* __restrict__ vc,
                                  const float* __restrict__ vu, int64_t n, float g, float dt,
                                  float* __restrict__ vout) {
+  pdl_wait();
+  pdl_trigger();
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const float u = vu[i];
@@ -333,7 +345,7 @@ int launch_cfg_euler(float* x, const float* v_c, const float* v_u, int64_t n, fl
   if (n == 0) return 0;
   int64_t gr = (n + 255) / 256;
   if (gr > 148 * 16) gr = 148 * 16;
-  cfg_euler_kernel<<<static_cast<int>(gr), 256, 0, st>>>(x, v_c, v_u, n, g, dt, v_out);
+  launch_pdl(cfg_euler_kernel, dim3(static_cast<unsigned>(gr)), dim3(256), 0, st, 1, x, v_c, v_u, n, g, dt, v_out);
   return launch_result();
 }
 

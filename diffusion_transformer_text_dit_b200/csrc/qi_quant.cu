@@ -183,6 +183,8 @@ constexpr int LN_CH = 4;
 template <bool XBF16>
 __global__ void __launch_bounds__(512) quant_ln_kernel(const QuantParams p) {
   __shared__ float red[64];
+  pdl_wait();
+  pdl_trigger();
   const int row = blockIdx.x;
   const int tid = threadIdx.x;
   const int nt = blockDim.x;
@@ -343,6 +345,8 @@ __global__ void __launch_bounds__(QS_MAX_THREADS, 6) quant_kernel(const QuantPar
   const int nunit = p.K / VPU;
   const uint32_t xbytes = static_cast<uint32_t>(p.K) * (XBF16 ? 2u : 4u);
   const uint4* xs = reinterpret_cast<const uint4*>(qs_row);
+  pdl_wait();
+  pdl_trigger();
 
   if (tid == 0) {
     mbar_init(&bar, 1);
@@ -417,7 +421,7 @@ static int launch_quant_ln_t(const QuantParams& p, cudaStream_t st) {
   int nt = (p.K / 8 + LN_CH - 1) / LN_CH;   // threads so that each holds <= LN_CH chunks
   nt = ((nt + 31) / 32) * 32;
   if (nt < 32) nt = 32;
-  quant_ln_kernel<XBF16><<<p.M, nt, 0, st>>>(p);
+  launch_pdl(quant_ln_kernel<XBF16>, dim3(p.M), dim3(nt), 0, st, 1, p);
   return launch_result();
 }
 
@@ -437,7 +441,7 @@ static int launch_quant_t(const QuantParams& p, cudaStream_t st) {
   nt = ((nt + 31) / 32) * 32;
   nt = nt < 32 ? 32 : (nt > QS_MAX_THREADS ? QS_MAX_THREADS : nt);
   const size_t smem = static_cast<size_t>(p.K) * (XBF16 ? 2 : 4);
-  quant_kernel<XBF16, RANGE><<<p.M, nt, smem, st>>>(p);
+  launch_pdl(quant_kernel<XBF16, RANGE>, dim3(p.M), dim3(nt), smem, st, 1, p);
   return launch_result();
 }
 
