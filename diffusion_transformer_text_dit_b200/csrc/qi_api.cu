@@ -428,6 +428,19 @@ int run_block_multi(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, fl
       p.k_out2 = seqs[1].kl + static_cast<size_t>(seqs[1].row0) * H;
       p.v_out2 = seqs[1].vl + static_cast<size_t>(seqs[1].row0) * H;
     }
+    if (f8) {
+      // e4m3 copies for fp8 attention, written by the same epilogue: q rows,
+      // and each sequence's K/V rows at their place in its e4m3 K | V block
+      p.q8_out = f8->q;
+      const size_t n0 = static_cast<size_t>(seqs[0].S) * H;
+      p.k8_out = f8->kv + static_cast<size_t>(seqs[0].row0) * H;
+      p.v8_out = f8->kv + n0 + static_cast<size_t>(seqs[0].row0) * H;
+      if (nseq > 1) {
+        const size_t n1 = static_cast<size_t>(seqs[1].S) * H;
+        p.k8_out2 = f8->kv + 2 * n0 + static_cast<size_t>(seqs[1].row0) * H;
+        p.v8_out2 = f8->kv + 2 * n0 + n1 + static_cast<size_t>(seqs[1].row0) * H;
+      }
+    }
     p.ldo = H;
     p.status = ctx->status;
     Prof pr(ctx, QI_KCLASS_GEMM_I8, st);
@@ -437,16 +450,23 @@ int run_block_multi(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, fl
     if (rr != 0) return cuda_fail("QKV GEMM launch");
   }
   if (f8) {
-    // fp8 attention: e4m3 copies of q and of every sequence's K and V rows
-    Prof pr(ctx, QI_KCLASS_OTHER, st);
-    if (qi::launch_bf16_to_e4m3(b.q, f8->q, static_cast<int64_t>(T) * H, st))
-      return cuda_fail("e4m3 cast launch");
+    // fp8 attention: the QKV epilogue wrote e4m3 q and the e4m3 K/V rows it
+    // produced; the K/V rows this call did not produce (a cached prefix) are
+    // cast from their bf16 rows
     size_t o = 0;
     for (int sq = 0; sq < nseq; ++sq) {
       const size_t n = static_cast<size_t>(seqs[sq].S) * H;
-      if (qi::launch_bf16_to_e4m3(seqs[sq].kl, f8->kv + o, static_cast<int64_t>(n), st) ||
-          qi::launch_bf16_to_e4m3(seqs[sq].vl, f8->kv + o + n, static_cast<int64_t>(n), st))
-        return cuda_fail("e4m3 cast launch");
+      const int lo = seqs[sq].row0, hi = seqs[sq].row0 + seqs[sq].T;   // rows written above
+      const int spans[2][2] = {{0, lo}, {hi, seqs[sq].S}};
+      for (const auto& sp : spans) {
+        if (sp[1] <= sp[0]) continue;
+        Prof pr(ctx, QI_KCLASS_OTHER, st);
+        const size_t r0 = static_cast<size_t>(sp[0]) * H;
+        const int64_t cnt = static_cast<int64_t>(sp[1] - sp[0]) * H;
+        if (qi::launch_bf16_to_e4m3(seqs[sq].kl + r0, f8->kv + o + r0, cnt, st) ||
+            qi::launch_bf16_to_e4m3(seqs[sq].vl + r0, f8->kv + o + n + r0, cnt, st))
+          return cuda_fail("e4m3 cast launch");
+      }
       o += 2 * n;
     }
   }

@@ -135,12 +135,34 @@ __device__ __forceinline__ void tempty_signal(uint32_t addr) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(addr) : "memory");
 }
 
+// e4m3 codes (round to nearest even, saturating at +-448) of the two bf16
+// values of a packed word, first value in the low byte.
+__device__ __forceinline__ uint32_t e4m3x2_of_bf16x2(uint32_t w) {
+  uint16_t h;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
+      : "=h"(h)
+      : "f"(__uint_as_float(w & 0xFFFF0000u)), "f"(__uint_as_float(w << 16)));
+  return h;
+}
+
+// 32 stored bf16 values (16 packed words) as 32 e4m3 bytes at dst.
+__device__ __forceinline__ void store_e4m3_32(uint8_t* dst, const uint32_t (&pk)[16]) {
+  uint32_t e[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) e[i] = e4m3x2_of_bf16x2(pk[2 * i]) | (e4m3x2_of_bf16x2(pk[2 * i + 1]) << 16);
+  uint4* d = reinterpret_cast<uint4*>(dst);
+  d[0] = make_uint4(e[0], e[1], e[2], e[3]);
+  d[1] = make_uint4(e[4], e[5], e[6], e[7]);
+}
+
 // Fused epilogue of the QKV projection: the W columns handled by one epilogue
 // warp are W/128 whole heads of q, k or v.  A q or k head row is read from
 // TMEM once and held (dequantized, bf16-rounded) in registers for
 //   r = 1/sqrt(mean(y^2) + eps), n = bf16(y r), y' = bf16(n w)   (cast before scale)
 //   (a, b) -> (bf16(a c - b s), bf16(a s + b c))                 (RoPE, pair = column/2)
-// with explicitly rounded fp32 operations; v is stored as bf16(y).
+// with explicitly rounded fp32 operations; v is stored as bf16(y).  For fp8
+// attention each stored bf16 row is also written as e4m3 (the value a
+// separate cast of the bf16 tensor gives).
 template <int W, bool PAIR>
 __device__ __forceinline__ void qkv_epilogue(const GemmParams& p, const ColTable& ct, int cb,
                                              uint32_t t_row, int m, bool row_ok, float sa,
@@ -153,6 +175,13 @@ __device__ __forceinline__ void qkv_epilogue(const GemmParams& p, const ColTable
   uint16_t* out = which == 0 ? p.q_out
                              : (which == 1 ? (second ? p.k_out2 : p.k_out)
                                            : (second ? p.v_out2 : p.v_out_bf16));
+  // e4m3 row of this head (read from the kernel parameters where it is used)
+  auto row8 = [&](int hh) -> uint8_t* {
+    uint8_t* o8 = which == 0 ? p.q8_out
+                             : (which == 1 ? (second ? p.k8_out2 : p.k8_out) : (second ? p.v8_out2 : p.v8_out));
+    return o8 + static_cast<size_t>(mo) * p.ldo + col0 + hh * 128;
+  };
+  const bool has8 = p.q8_out != nullptr;   // fp8 attention: all five are set
   const uint16_t* w = which == 0 ? p.wq : p.wk;
 #pragma unroll 1
   for (int hh = 0; hh < W / 128; ++hh) {
@@ -177,6 +206,7 @@ __device__ __forceinline__ void qkv_epilogue(const GemmParams& p, const ColTable
 #pragma unroll
         for (int v = 0; v < 4; ++v)
           dst_row[c * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        if (has8) store_e4m3_32(row8(hh) + c * 32, pk);
       }
       continue;
     }
@@ -230,6 +260,7 @@ __device__ __forceinline__ void qkv_epilogue(const GemmParams& p, const ColTable
 #pragma unroll
       for (int v = 0; v < 4; ++v)
         dst_row[c * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+      if (has8) store_e4m3_32(row8(hh) + c * 32, pk);
     }
   }
 }

@@ -95,6 +95,13 @@ struct GemmParams {
   uint16_t* k_out2;       // K/V rows m >= kv_split go to k_out2/v_out2 row m - kv_split
   uint16_t* v_out2;       // (a batch of two sequences with separate K/V buffers)
   int kv_split;
+  // optional e4m3 copies of the q / k / v rows above (same rows and ldo, one
+  // byte per element: round to nearest even, saturating), for fp8 attention
+  uint8_t* q8_out;
+  uint8_t* k8_out;
+  uint8_t* v8_out;
+  uint8_t* k8_out2;
+  uint8_t* v8_out2;
   int ldo;
   uint32_t* row_range;    // GELU: optional per-row [-min, max] bit patterns of the bf16 output
   int* status;            // device status word

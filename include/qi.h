@@ -301,8 +301,10 @@ int qi_mxfp4_decode(qi_ctx* ctx, const uint8_t* packed, const uint8_t* scales, i
                     int k_stored, int k, float* w, void* stream);
 
 /* Attention precision of the steps run on this context (qi_denoise_step,
- * qi_denoise_step_cfg): enable != 0 -> every block converts q and the
- * layer's K/V rows to e4m3 and runs qi_attn_block_causal_fp8's kernel
+ * qi_denoise_step_cfg): enable != 0 -> in every block the QKV projection
+ * also writes e4m3 (round to nearest even, saturating) copies of the q, k, v
+ * rows it produces, cached prefix K/V rows are converted the same way, and
+ * qi_attn_block_causal_fp8's kernel runs on them
  * (the pages' schedule: the prefix pass and the first seven steps at full
  * precision, later steps with fp8 attention - the caller switches between
  * steps).  Block-level calls are not affected.  Default 0. */

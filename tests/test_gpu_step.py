@@ -182,6 +182,40 @@ def test_cfg_cached_equals_uncached(ctx):
     assert torch.equal(u2, c2)
 
 
+@pytest.mark.parametrize("refs", [0, 2], ids=["text_image", "text_2ref_image"])
+def test_cfg_fp8_batch_equals_two_single_fp8_steps(ctx, refs):
+    """fp8 attention in a true-CFG batch: the QKV epilogue writes each
+    sequence's e4m3 K/V rows at that sequence's own place, so each velocity of
+    the batch is exactly its single-sequence fp8 velocity."""
+    s = CfgSetup(ctx, refs=refs)
+    sig = O.sigma_schedule(40, s.cfg_c.target_tokens)
+    a, b = float(sig[5]), float(sig[6])
+    ctx.set_attention_fp8(True)
+    try:
+        _, v = s.step(ctx, s.c.lat, 4.0, a, b)
+        _, vc = s.c.gpu_step(ctx, s.c.lat, a, b)
+        _, vu = s.u.gpu_step(ctx, s.c.lat, a, b)
+    finally:
+        ctx.set_attention_fp8(False)
+    assert np.array_equal(v.numpy(), O.cfg_combine(vc.numpy(), vu.numpy(), 4.0))
+    assert not np.array_equal(vc.numpy(), vu.numpy())
+
+
+def test_cfg_fp8_cached_equals_uncached(ctx):
+    """Cached fp8 steps cast only the cached prefix K/V rows of each sequence
+    to e4m3; the uncached step gets all of them from the QKV epilogue."""
+    s = CfgSetup(ctx, blocks=3, refs=1)
+    sig = O.sigma_schedule(40, s.cfg_c.target_tokens)
+    ctx.set_attention_fp8(True)
+    try:
+        a1, _ = s.step(ctx, s.c.lat, 2.5, float(sig[0]), float(sig[1]), qi.QI_KV_WRITE_PREFIX)
+        u2, _ = s.step(ctx, a1, 2.5, float(sig[1]), float(sig[2]), qi.QI_KV_NONE)
+        c2, _ = s.step(ctx, a1, 2.5, float(sig[1]), float(sig[2]), qi.QI_KV_READ_PREFIX)
+    finally:
+        ctx.set_attention_fp8(False)
+    assert torch.equal(u2, c2)
+
+
 def test_cfg_rejects_mismatched_targets(ctx):
     s = CfgSetup(ctx)
     other = synth.TINY.replace(name="cfg_bad", blocks=2, patch=64,
