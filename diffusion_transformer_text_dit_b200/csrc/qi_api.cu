@@ -756,7 +756,9 @@ int qi_quantize_act(qi_ctx* ctx, const void* x, int x_dtype, int M, int K, int l
                     const uint16_t* shift, const uint16_t* scale, int mod_ld,
                     const qi_groups* groups, int row0, float eps, int8_t* q, float* s_a,
                     int32_t* zp_a, void* stream) {
-  if (!ctx || !x || !q || !s_a || !zp_a) return fail(QI_ERR_INVALID_ARG, "NULL argument");
+  if (!ctx) return fail(QI_ERR_INVALID_ARG, "NULL argument");
+  if (M == 0) return QI_OK;   // no rows: nothing to do (the row pointers may be NULL)
+  if (!x || !q || !s_a || !zp_a) return fail(QI_ERR_INVALID_ARG, "NULL argument");
   if (x_dtype != QI_F32 && x_dtype != QI_BF16) return fail(QI_ERR_INVALID_ARG, "bad x_dtype");
   if (M < 0 || K < 8 || K % 8 != 0 || K > 16384 || ldx < K || ldx % 8 != 0)
     return fail(QI_ERR_UNSUPPORTED_SHAPE, "quantize: need 8 <= K <= 16384, K %% 8 == 0, ldx %% 8 == 0");
@@ -781,7 +783,9 @@ int qi_quantize_act(qi_ctx* ctx, const void* x, int x_dtype, int M, int K, int l
 int qi_w8a8_linear(qi_ctx* ctx, const int8_t* qa, const float* s_a, const int32_t* zp_a, int M,
                    const qi_w8* w, const qi_epilogue* ep, uint16_t* y, int ldy,
                    int32_t* acc_debug, void* stream) {
-  if (!ctx || !qa || !s_a || !zp_a) return fail(QI_ERR_INVALID_ARG, "NULL argument");
+  if (!ctx) return fail(QI_ERR_INVALID_ARG, "NULL argument");
+  if (M == 0) return QI_OK;   // no rows: nothing to do (the row pointers may be NULL)
+  if (!qa || !s_a || !zp_a) return fail(QI_ERR_INVALID_ARG, "NULL argument");
   if (M < 0) return fail(QI_ERR_INVALID_ARG, "M < 0");
   int r;
   if ((r = check_w8(w, "w", -1, -1))) return r;
@@ -851,7 +855,9 @@ int qi_w8a8_linear(qi_ctx* ctx, const int8_t* qa, const float* s_a, const int32_
 
 int qi_bf16_linear(qi_ctx* ctx, const uint16_t* a, int M, int lda, const qi_linear_bf16* w,
                    float* y, int ldy, void* stream) {
-  if (!ctx || !a || !y) return fail(QI_ERR_INVALID_ARG, "NULL argument");
+  if (!ctx) return fail(QI_ERR_INVALID_ARG, "NULL argument");
+  if (M == 0) return QI_OK;   // no rows: nothing to do (the row pointers may be NULL)
+  if (!a || !y) return fail(QI_ERR_INVALID_ARG, "NULL argument");
   int r;
   if ((r = check_bf16_linear(w, "w", -1, -1))) return r;
   if (M < 0 || w->k % 64 != 0 || w->k < 64 || w->n % 16 != 0 || lda < w->k || lda % 8 != 0 ||
@@ -894,7 +900,9 @@ namespace {
 int attn_call(qi_ctx* ctx, const void* q, int ldq, int Sq, int q_offset, const void* k,
               const void* v, int ldkv, int Sk, int heads, int head_dim, const qi_groups* groups,
               float sm_scale, uint16_t* o, int ldo, void* stream, bool fp8) {
-  if (!ctx || !q || !k || !v || !o) return fail(QI_ERR_INVALID_ARG, "NULL argument");
+  if (!ctx) return fail(QI_ERR_INVALID_ARG, "NULL argument");
+  if (Sq == 0) return QI_OK;   // no query rows: nothing to do (the pointers may be NULL)
+  if (!q || !k || !v || !o) return fail(QI_ERR_INVALID_ARG, "NULL argument");
   if (head_dim != 128) return fail(QI_ERR_UNSUPPORTED_SHAPE, "head_dim must be 128");
   if (Sq < 0 || Sk < 1 || q_offset < 0 || q_offset + Sq > Sk || heads < 1)
     return fail(QI_ERR_INVALID_ARG, "need 0 <= q_offset, q_offset + Sq <= Sk");

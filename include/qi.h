@@ -32,7 +32,10 @@
  *     qi_last_error() returns a text description of the last failure on the
  *     calling thread.
  *   - Tensor pointers are device pointers owned by the caller unless stated
- *     otherwise; all must be 16-byte aligned.  Matrices are row-major
+ *     otherwise; all must be 16-byte aligned.  A call on zero rows
+ *     (qi_quantize_act, qi_w8a8_linear, qi_bf16_linear with M = 0; the
+ *     attention calls with Sq = 0) returns QI_OK and touches nothing; its row
+ *     pointers may then be NULL.  Matrices are row-major
  *     [rows, ld] with ld in elements.  bf16 values are passed as uint16_t bit
  *     patterns.  Weights are [out, in] (K-major).
  *   - Every device call is asynchronous on the given CUDA stream

@@ -58,13 +58,35 @@ def test_quantize_plain_bit_exact(ctx, M, K):
     assert np.array_equal(q.cpu().numpy(), oq)
 
 
-@pytest.mark.parametrize("K", [4096, 1000])
+@pytest.mark.parametrize("K", [4096, 1000, 16384])   # 16384 fp32: the largest staged row (64 KB)
 def test_quantize_fp32_input_bit_exact(ctx, K):
     x = torch.randn(300, K, generator=_gen(5)) * 3 + 0.7
     q, s, zp = qi.qi_quantize_act(ctx, cuda(x))
     oq, os_, ozp = O.quantize_act(x.numpy())
     assert np.array_equal(s.cpu().numpy(), os_) and np.array_equal(zp.cpu().numpy(), ozp)
     assert np.array_equal(q.cpu().numpy(), oq)
+
+
+def test_empty_inputs_are_noops(ctx):
+    """Zero rows: quantization and attention return OK and write nothing (a
+    zero-element tensor hands the library a NULL pointer, which is allowed
+    for a call on zero rows)."""
+    x = cuda(_bf16((4, 256), 3, 1.0))
+    q = torch.full((4, 256), 7, dtype=torch.int8, device="cuda")
+    s = torch.full((4,), 2.0, device="cuda")
+    zp = torch.full((4,), 5, dtype=torch.int32, device="cuda")
+    qi.qi_quantize_act(ctx, x[:0], out=(q[:0], s[:0], zp[:0]))
+    y = torch.full((4, 64), 3.0, dtype=torch.bfloat16, device="cuda")
+    qi.qi_w8a8_linear(ctx, q[:0], s[:0], zp[:0], qi.qi_w8(), y=y[:0])
+    H, S = 256, 40
+    qkv = cuda(_bf16((3, S, H), 4, 1.0))
+    o = torch.full((S, H), 1.5, dtype=torch.bfloat16, device="cuda")
+    g = qi.groups_struct([8, S], [0, 1])
+    qi.qi_attn_block_causal(ctx, qkv[0][:0], qkv[1], qkv[2], g, q_offset=S, o=o[:0])
+    torch.cuda.synchronize()
+    ctx.check()
+    assert bool((q == 7).all()) and bool((s == 2.0).all()) and bool((zp == 5).all())
+    assert bool((o == 1.5).all()) and bool((y == 3.0).all())
 
 
 @pytest.mark.parametrize("H,L,N", [(256, 16, 64), (4096, 256, 1024)])
