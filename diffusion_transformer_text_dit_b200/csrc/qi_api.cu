@@ -653,20 +653,42 @@ namespace {
 constexpr int QI_NOALLOC_MAX_DEVICES = 64;
 std::mutex g_noalloc_mu;
 void* g_noalloc_addr[QI_NOALLOC_MAX_DEVICES] = {};
+CUcontext g_noalloc_cuctx[QI_NOALLOC_MAX_DEVICES] = {};
+
+// The CUDA context current on this thread (driver entry point looked up once).
+int current_cu_context(CUcontext* out) {
+  static PFN_cuCtxGetCurrent_v4000 get = nullptr;
+  if (!get) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+      return fail(QI_ERR_CUDA, "cuCtxGetCurrent is not available");
+    get = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(fn);
+  }
+  if (get(out) != CUDA_SUCCESS || !*out) return fail(QI_ERR_CUDA, "no current CUDA context");
+  return QI_OK;
+}
 
 // Device address of the scratch array on the current device.  The array's
-// name is only a host-side stand-in, so the address is looked up once per
-// device (with that device current) and cached.
+// name is only a host-side stand-in, so the address is looked up with the
+// device current and cached per device together with the CUDA context it was
+// found in: after a device reset the module is loaded again into a new
+// context, and the address is looked up again instead of reusing a stale one.
 int noalloc_scratch(int device, void** out) {
   if (device < 0 || device >= QI_NOALLOC_MAX_DEVICES)
     return fail(QI_ERR_INVALID_ARG, "device %d outside 0..%d", device, QI_NOALLOC_MAX_DEVICES - 1);
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_addr[device]) {
+  CUcontext cur = nullptr;
+  int r;
+  if ((r = current_cu_context(&cur))) return r;
+  if (!g_noalloc_addr[device] || g_noalloc_cuctx[device] != cur) {
     void* p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, qi_noalloc_scratch);
     if (e != cudaSuccess || !p)
       return fail(QI_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
     g_noalloc_addr[device] = p;
+    g_noalloc_cuctx[device] = cur;
   }
   *out = g_noalloc_addr[device];
   return QI_OK;
@@ -757,11 +779,10 @@ int qi_quantize_act(qi_ctx* ctx, const void* x, int x_dtype, int M, int K, int l
                     const qi_groups* groups, int row0, float eps, int8_t* q, float* s_a,
                     int32_t* zp_a, void* stream) {
   if (!ctx) return fail(QI_ERR_INVALID_ARG, "NULL argument");
-  if (M == 0) return QI_OK;   // no rows: nothing to do (the row pointers may be NULL)
-  if (!x || !q || !s_a || !zp_a) return fail(QI_ERR_INVALID_ARG, "NULL argument");
   if (x_dtype != QI_F32 && x_dtype != QI_BF16) return fail(QI_ERR_INVALID_ARG, "bad x_dtype");
   if (M < 0 || K < 8 || K % 8 != 0 || K > 16384 || ldx < K || ldx % 8 != 0)
     return fail(QI_ERR_UNSUPPORTED_SHAPE, "quantize: need 8 <= K <= 16384, K %% 8 == 0, ldx %% 8 == 0");
+  if (M > 0 && (!x || !q || !s_a || !zp_a)) return fail(QI_ERR_INVALID_ARG, "NULL argument");
   if (!aligned16(x) || !aligned16(q)) return fail(QI_ERR_ALIGNMENT, "x / q must be 16-byte aligned");
   qi::GroupTable gt;
   memset(&gt, 0, sizeof(gt));
@@ -776,6 +797,7 @@ int qi_quantize_act(qi_ctx* ctx, const void* x, int x_dtype, int M, int K, int l
     if (row0 < 0 || row0 + M > gt.end[gt.n - 1])
       return fail(QI_ERR_INVALID_ARG, "rows row0..row0+M-1 fall outside the groups");
   }
+  if (M == 0) return QI_OK;   // no rows: nothing to do (the row pointers may be NULL)
   return run_quant(ctx, x, x_dtype == QI_BF16, M, K, ldx, shift, scale, mod_ld, gt, row0, eps, q,
                    s_a, zp_a, nullptr, S(stream));
 }
@@ -784,9 +806,11 @@ int qi_w8a8_linear(qi_ctx* ctx, const int8_t* qa, const float* s_a, const int32_
                    const qi_w8* w, const qi_epilogue* ep, uint16_t* y, int ldy,
                    int32_t* acc_debug, void* stream) {
   if (!ctx) return fail(QI_ERR_INVALID_ARG, "NULL argument");
-  if (M == 0) return QI_OK;   // no rows: nothing to do (the row pointers may be NULL)
-  if (!qa || !s_a || !zp_a) return fail(QI_ERR_INVALID_ARG, "NULL argument");
   if (M < 0) return fail(QI_ERR_INVALID_ARG, "M < 0");
+  // Weight, epilogue and layout checks come first, so that a zero-row call
+  // with bad arguments is rejected like any other; only the row pointers
+  // (qa, s_a, zp_a, y, residual, q/k/v outputs) may be NULL when M == 0.
+  if (M > 0 && (!qa || !s_a || !zp_a)) return fail(QI_ERR_INVALID_ARG, "NULL argument");
   int r;
   if ((r = check_w8(w, "w", -1, -1))) return r;
   if (!aligned16(qa)) return fail(QI_ERR_ALIGNMENT, "qa must be 16-byte aligned");
@@ -796,9 +820,10 @@ int qi_w8a8_linear(qi_ctx* ctx, const int8_t* qa, const float* s_a, const int32_
   gt.n = 1;
   gt.end[0] = 1 << 30;
   if (kind == QI_EPI_STORE || kind == QI_EPI_GELU_TANH) {
-    if (!y) return fail(QI_ERR_INVALID_ARG, "y is NULL");
+    if (!y && M > 0) return fail(QI_ERR_INVALID_ARG, "y is NULL");
     if (!aligned16(y) || ldy < w->n || ldy % 8 != 0)
       return fail(QI_ERR_ALIGNMENT, "y must be 16-byte aligned with ldy %% 8 == 0, ldy >= n");
+    if (M == 0) return QI_OK;
     return run_w8a8(ctx, qa, s_a, zp_a, M, *w, kind == QI_EPI_STORE ? qi::EPI_BF16 : qi::EPI_GELU,
                     y, ldy, nullptr, 0, nullptr, 0, gt, 0, acc_debug, S(stream));
   }
@@ -806,8 +831,8 @@ int qi_w8a8_linear(qi_ctx* ctx, const int8_t* qa, const float* s_a, const int32_
     const int H = ep->hidden;
     if (H < 128 || H % 128 != 0 || w->n != 3 * H)
       return fail(QI_ERR_UNSUPPORTED_SHAPE, "QKV epilogue: need hidden %% 128 == 0 and n == 3 * hidden");
-    if (!ep->norm_q || !ep->norm_k || !ep->rope_cos || !ep->rope_sin || !ep->q_out ||
-        !ep->k_out || !ep->v_out)
+    if (!ep->norm_q || !ep->norm_k ||
+        (M > 0 && (!ep->rope_cos || !ep->rope_sin || !ep->q_out || !ep->k_out || !ep->v_out)))
       return fail(QI_ERR_INVALID_ARG, "QKV epilogue: NULL pointer");
     if (ep->ld_out < H || ep->ld_out % 8 != 0 || !aligned16(ep->q_out) || !aligned16(ep->k_out) ||
         !aligned16(ep->v_out) || !aligned16(ep->rope_cos) || !aligned16(ep->rope_sin) ||
@@ -844,11 +869,12 @@ int qi_w8a8_linear(qi_ctx* ctx, const int8_t* qa, const float* s_a, const int32_
     return QI_OK;
   }
   if (kind != QI_EPI_GATED_RESIDUAL) return fail(QI_ERR_INVALID_ARG, "bad epilogue kind");
-  if (!ep->residual || !ep->gate) return fail(QI_ERR_INVALID_ARG, "residual / gate is NULL");
+  if ((M > 0 && !ep->residual) || !ep->gate) return fail(QI_ERR_INVALID_ARG, "residual / gate is NULL");
   if (ep->ld_residual < w->n) return fail(QI_ERR_INVALID_ARG, "ld_residual < n");
   if ((r = check_groups(ep->groups, -1, &gt))) return r;
   if (ep->row0 < 0 || ep->row0 + M > gt.end[gt.n - 1])
     return fail(QI_ERR_INVALID_ARG, "rows row0..row0+M-1 fall outside the groups");
+  if (M == 0) return QI_OK;
   return run_w8a8(ctx, qa, s_a, zp_a, M, *w, qi::EPI_GATED, nullptr, 0, ep->residual,
                   ep->ld_residual, ep->gate, ep->gate_ld, gt, ep->row0, acc_debug, S(stream));
 }
@@ -856,14 +882,14 @@ int qi_w8a8_linear(qi_ctx* ctx, const int8_t* qa, const float* s_a, const int32_
 int qi_bf16_linear(qi_ctx* ctx, const uint16_t* a, int M, int lda, const qi_linear_bf16* w,
                    float* y, int ldy, void* stream) {
   if (!ctx) return fail(QI_ERR_INVALID_ARG, "NULL argument");
-  if (M == 0) return QI_OK;   // no rows: nothing to do (the row pointers may be NULL)
-  if (!a || !y) return fail(QI_ERR_INVALID_ARG, "NULL argument");
+  if (M > 0 && (!a || !y)) return fail(QI_ERR_INVALID_ARG, "NULL argument");
   int r;
   if ((r = check_bf16_linear(w, "w", -1, -1))) return r;
   if (M < 0 || w->k % 64 != 0 || w->k < 64 || w->n % 16 != 0 || lda < w->k || lda % 8 != 0 ||
       ldy < w->n)
     return fail(QI_ERR_UNSUPPORTED_SHAPE, "bf16 linear: need k %% 64 == 0, n %% 16 == 0, lda %% 8 == 0");
   if (!aligned16(a)) return fail(QI_ERR_ALIGNMENT, "a must be 16-byte aligned");
+  if (M == 0) return QI_OK;   // no rows: nothing to do (the row pointers may be NULL)
   return run_bf16_linear(ctx, a, M, lda, *w, qi::EPI_F32, y, ldy, 0.f, nullptr, S(stream));
 }
 
@@ -901,8 +927,7 @@ int attn_call(qi_ctx* ctx, const void* q, int ldq, int Sq, int q_offset, const v
               const void* v, int ldkv, int Sk, int heads, int head_dim, const qi_groups* groups,
               float sm_scale, uint16_t* o, int ldo, void* stream, bool fp8) {
   if (!ctx) return fail(QI_ERR_INVALID_ARG, "NULL argument");
-  if (Sq == 0) return QI_OK;   // no query rows: nothing to do (the pointers may be NULL)
-  if (!q || !k || !v || !o) return fail(QI_ERR_INVALID_ARG, "NULL argument");
+  if (Sq > 0 && (!q || !k || !v || !o)) return fail(QI_ERR_INVALID_ARG, "NULL argument");
   if (head_dim != 128) return fail(QI_ERR_UNSUPPORTED_SHAPE, "head_dim must be 128");
   if (Sq < 0 || Sk < 1 || q_offset < 0 || q_offset + Sq > Sk || heads < 1)
     return fail(QI_ERR_INVALID_ARG, "need 0 <= q_offset, q_offset + Sq <= Sk");
@@ -915,6 +940,7 @@ int attn_call(qi_ctx* ctx, const void* q, int ldq, int Sq, int q_offset, const v
   qi::GroupTable gt;
   int r;
   if ((r = check_groups(groups, Sk, &gt))) return r;
+  if (Sq == 0) return QI_OK;   // no query rows: nothing to do (the pointers may be NULL)
   qi::AttnParams p;
   memset(&p, 0, sizeof(p));
   p.q = q;
@@ -1050,8 +1076,11 @@ int qi_dit_block_forward_noalloc(qi_ctx* ctx, const qi_dims* dims, const qi_bloc
                 cur, ctx->device);
   void* scratch = nullptr;
   if ((r = noalloc_scratch(cur, &scratch))) return r;
-  // Every region of the block's scratch is written before it is read, so
-  // nothing has to be cleared between calls.
+  // The block writes every region of its scratch before reading it, with one
+  // ordering to keep: the two row-range tables that the attention and GELU
+  // epilogues publish with atomicMax are cleared by the LayerNorm quantizers
+  // that run before those producers in the same call.  So nothing left by an
+  // earlier call is read, and nothing has to be cleared here.
   return qi_dit_block_forward(ctx, dims, w, x, T, row0, mod, groups, rope_cos, rope_sin, k_layer,
                               v_layer, kv_mode, scratch, QI_NOALLOC_SCRATCH_BYTES, stream);
 }

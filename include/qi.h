@@ -34,8 +34,9 @@
  *   - Tensor pointers are device pointers owned by the caller unless stated
  *     otherwise; all must be 16-byte aligned.  A call on zero rows
  *     (qi_quantize_act, qi_w8a8_linear, qi_bf16_linear with M = 0; the
- *     attention calls with Sq = 0) returns QI_OK and touches nothing; its row
- *     pointers may then be NULL.  Matrices are row-major
+ *     attention calls with Sq = 0) checks its other arguments (weights,
+ *     shapes, epilogue, groups) like any call, then returns QI_OK and touches
+ *     nothing; its row pointers may be NULL.  Matrices are row-major
  *     [rows, ld] with ld in elements.  bf16 values are passed as uint16_t bit
  *     patterns.  Weights are [out, in] (K-major).
  *   - Every device call is asynchronous on the given CUDA stream
@@ -346,11 +347,16 @@ int qi_dit_block_forward(qi_ctx* ctx, const qi_dims* dims, const qi_block_weight
  *   - Sizes whose scratch (qi_block_workspace_bytes) exceeds 16 MiB are rejected
  *     with QI_ERR_WORKSPACE before anything is launched (at hidden 256 / mlp
  *     1024 up to 4,071 rows fit; at hidden 4096 / mlp 16384 up to 255 rows).
- *   - The first call on a device looks up the array's device address (once,
- *     with that device current; the current device must be the context's).
- *     Make that first call before any stream capture.
- *   - All calls share the one array and it keeps the last call's contents;
- *     every region is written before it is read, so nothing needs clearing.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current; the current device must be the context's) and
+ *     caches it with the CUDA context it belongs to; a call in a new context
+ *     (after a device reset) looks it up again.  Make the first call on a
+ *     device, and the first after a reset, before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents.
+ *     The block writes each region before reading it; the per-row range
+ *     tables that the attention and GELU epilogues fill with atomic maxima
+ *     are cleared by the LayerNorm quantizers that run before them in the
+ *     same call, so nothing needs clearing between calls.
  *     Calls whose kernels overlap on the GPU (different streams, or several
  *     host threads) race on it: serialize them.
  * Arguments and results are those of qi_dit_block_forward. */

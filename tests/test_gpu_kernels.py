@@ -89,6 +89,51 @@ def test_empty_inputs_are_noops(ctx):
     assert bool((o == 1.5).all()) and bool((y == 3.0).all())
 
 
+def test_empty_inputs_still_validate_their_other_arguments(ctx):
+    """A zero-row call is rejected for the same bad weight, dtype, shape,
+    epilogue or group table as a call with rows: only its row pointers may be
+    NULL."""
+    L = qi.lib()
+    h = ctx.handle
+    st = qi.stream_ptr()
+    # quantizer: bad dtype, bad K
+    assert L.qi_quantize_act(h, None, 7, 0, 256, 256, None, None, 0, None, 0, 1e-6, None, None,
+                             None, st) == qi.QI_ERR_INVALID_ARG
+    assert L.qi_quantize_act(h, None, qi.QI_BF16, 0, 100, 100, None, None, 0, None, 0, 1e-6,
+                             None, None, None, st) == qi.QI_ERR_UNSUPPORTED_SHAPE
+    # W8A8 Linear: NULL weight codes, bad K, bad epilogue kind
+    bad_w = qi.qi_w8()
+    assert L.qi_w8a8_linear(h, None, None, None, 0, qi.C.byref(bad_w), None, None, 0, None,
+                            st) == qi.QI_ERR_INVALID_ARG
+    q = torch.zeros((64, 100), dtype=torch.int8, device="cuda")
+    s = torch.ones(64, device="cuda")
+    rs = torch.zeros(64, dtype=torch.int32, device="cuda")
+    w = qi.w8_struct(q, s, rs)
+    assert L.qi_w8a8_linear(h, None, None, None, 0, qi.C.byref(w), None, None, 64, None,
+                            st) == qi.QI_ERR_UNSUPPORTED_SHAPE
+    q2 = torch.zeros((64, 128), dtype=torch.int8, device="cuda")
+    w2 = qi.w8_struct(q2, s, rs)
+    ep = qi.qi_epilogue()
+    ep.kind = 9
+    assert L.qi_w8a8_linear(h, None, None, None, 0, qi.C.byref(w2), qi.C.byref(ep), None, 64,
+                            None, st) == qi.QI_ERR_INVALID_ARG
+    # ... while the same zero-row call with good arguments is a no-op
+    assert L.qi_w8a8_linear(h, None, None, None, 0, qi.C.byref(w2), None, None, 64, None,
+                            st) == qi.QI_OK
+    # BF16 Linear: k not a multiple of 64
+    wb = torch.zeros((64, 96), dtype=torch.bfloat16, device="cuda")
+    assert L.qi_bf16_linear(h, None, 0, 96, qi.C.byref(qi.bf16_struct(wb)), None, 64,
+                            st) == qi.QI_ERR_UNSUPPORTED_SHAPE
+    # attention: head_dim 64, and a group table that does not end at Sk
+    g = qi.groups_struct([8, 40], [0, 1])
+    assert L.qi_attn_block_causal(h, None, 256, 0, 40, None, None, 256, 40, 2, 64,
+                                  qi.C.byref(g), 0.1, None, 256, st) == qi.QI_ERR_UNSUPPORTED_SHAPE
+    g_bad = qi.groups_struct([8, 30], [0, 1])
+    assert L.qi_attn_block_causal(h, None, 256, 0, 40, None, None, 256, 40, 2, 128,
+                                  qi.C.byref(g_bad), 0.1, None, 256, st) == qi.QI_ERR_INVALID_ARG
+    ctx.check()
+
+
 @pytest.mark.parametrize("H,L,N", [(256, 16, 64), (4096, 256, 1024)])
 def test_quantize_ln_modulate(ctx, H, L, N):
     cfg = synth.TINY.replace(hidden=H)
