@@ -392,6 +392,34 @@ def attention_block_causal_fp8(q, k, v, q_group, k_group, sm_scale, tile=128,
     return out
 
 
+def attention_block_causal_fp8_plain(q, k, v, q_group, k_group, sm_scale) -> np.ndarray:
+    """Block-causal attention with e4m3 operands, in the plainest reading of
+    the pages' "int8/fp8 attention" ("Qwen_Image-2.1-MXFP4-Paiton-RDNA4",
+    "Runtime precision and quality"), with no tiling:
+
+      * q, k, v are rounded to e4m3;
+      * per query row, s = (q . k) sm_scale over the visible keys, m = max s;
+      * P = exp(s - m) (float64), rounded to e4m3 before it multiplies V;
+      * O = (sum_j e4m3(P_j) v_j) / (sum_j P_j), the row sum over unrounded P.
+
+    It differs from a tiled kernel only where the kernel takes scheduling
+    decisions (which maximum each tile subtracts): those shift P by a power
+    of two, which e4m3 rounds identically except below its smallest normal
+    value 2^-6.
+    """
+    q = e4m3_round(q)
+    k = e4m3_round(k)
+    v = e4m3_round(v)
+    visible = np.asarray(k_group)[None, :] <= np.asarray(q_group)[:, None]
+    out = np.empty(q.shape, dtype=F64)
+    for h in range(q.shape[1]):
+        s = (q[:, h, :] @ k[:, h, :].T) * sm_scale
+        s = np.where(visible, s, -np.inf)
+        p = np.exp(s - s.max(axis=1, keepdims=True))
+        out[:, h, :] = (e4m3_round(p) @ v[:, h, :]) / p.sum(axis=1, keepdims=True)
+    return out
+
+
 # ----------------------------------------------------------------------------
 # One transformer block
 # ----------------------------------------------------------------------------
@@ -557,6 +585,33 @@ def cfg_combine(v_cond, v_uncond, guidance) -> np.ndarray:
 # ----------------------------------------------------------------------------
 
 
+def joint_inputs(latents, txt, ref_latents, mw: dict, groups, mode: str = "none"):
+    """Rows of the joint sequence that enter the first block, and their indices.
+
+    Core AI port, "Graph contracts": the DiT takes the text features and the
+    latent tokens as separate inputs and runs one single-stream sequence
+    [text | image].  Reading (see the design notes): text rows enter through
+    the text in-projection (a BF16 Linear H -> H), reference-image rows of an
+    edit sequence through the same image in-projection as the target latents
+    (P -> H), in the order of the groups.  In "read" mode (cached prefix) only
+    the target rows are formed.
+    Returns (x [rows, H] float64, row indices into the sequence).
+    """
+    sizes = [n for _, n, _ in groups]
+    S = sum(sizes)
+    P_tok = S - sizes[-1]
+    x_img = linear(np.asarray(latents, F64), mw["img_in"], mw["img_in_b"])
+    if mode == "read":
+        return x_img, np.arange(P_tok, S)
+    parts = [linear(np.asarray(txt, F64), mw["txt_in"], mw["txt_in_b"])]
+    if ref_latents is not None:
+        parts.append(linear(np.asarray(ref_latents, F64), mw["img_in"], mw["img_in_b"]))
+    parts.append(x_img)
+    x = np.concatenate(parts, axis=0)
+    assert x.shape[0] == S
+    return x, np.arange(S)
+
+
 def step_forward(latents, txt, ref_latents, mw: dict, blocks_pw: Sequence[dict],
                  blocks_mod_w: Sequence[Tuple], groups, heads, head_dim, eps, sigma, sigma_next,
                  kv_cache: Optional[Dict[int, Tuple[np.ndarray, np.ndarray]]] = None,
@@ -586,21 +641,7 @@ def step_forward(latents, txt, ref_latents, mw: dict, blocks_pw: Sequence[dict],
     temb_t = time_embed(sigma, mw)
     temb_0 = time_embed(0.0, mw)
 
-    x_img = linear(np.asarray(latents, F64), mw["img_in"], mw["img_in_b"])
-    if mode == "read":
-        rows = np.arange(P_tok, S)
-        x = x_img
-    else:
-        rows = np.arange(S)
-        # text rows enter through the text in-projection, reference-image
-        # rows (edit sequences) through the same image in-projection as the
-        # target latents
-        parts = [linear(np.asarray(txt, F64), mw["txt_in"], mw["txt_in_b"])]
-        if ref_latents is not None:
-            parts.append(linear(np.asarray(ref_latents, F64), mw["img_in"], mw["img_in_b"]))
-        parts.append(x_img)
-        x = np.concatenate(parts, axis=0)
-    assert x.shape[0] == len(rows)
+    x, rows = joint_inputs(latents, txt, ref_latents, mw, groups, mode)
 
     for l, (pw, (wm, bm)) in enumerate(zip(blocks_pw, blocks_mod_w)):
         mod = np.stack([adaln_rows(temb_0, wm, bm), adaln_rows(temb_t, wm, bm)])

@@ -392,6 +392,52 @@ def test_attention_fp8_error_is_e4m3_sized():
     assert 1e-3 < err < 8e-2
 
 
+def test_attention_fp8_plain_uniform_scores_closed_form():
+    """q = 0: every visible score is 0, so P = exp(0) = 1 exactly (an e4m3
+    value) and the output is the plain mean of the e4m3-rounded values of the
+    visible keys; a numerator or denominator over the wrong key set, or P
+    rounded in the row sum, would move it."""
+    ends = [5, 12, 20]
+    g = O.group_ids(ends)
+    k = rng.standard_normal((20, 2, 16))
+    v = rng.standard_normal((20, 2, 16)) * 3
+    q = np.zeros((20, 2, 16))
+    out = O.attention_block_causal_fp8_plain(q, k, v, g, g, 0.3)
+    v8 = O.e4m3_round(v)
+    for i in range(20):
+        n_vis = ends[g[i]]
+        assert np.allclose(out[i], v8[:n_vis].mean(axis=0), rtol=0, atol=1e-12)
+
+
+def test_attention_fp8_plain_row_sum_uses_unrounded_p():
+    """Constant V rows (an e4m3 value c): O = c * sum(e4m3(P)) / sum(P), which
+    differs from c by at most one e4m3 half-step (2^-4 relative) and, with
+    varied scores, is not exactly c -- the row sum takes the unrounded P."""
+    g = O.group_ids([40])
+    q = rng.standard_normal((40, 1, 16))
+    k = rng.standard_normal((40, 1, 16))
+    v = np.full((40, 1, 16), 0.75)          # e4m3-exact
+    out = O.attention_block_causal_fp8_plain(q, k, v, g, g, 0.7)
+    q8, k8 = O.e4m3_round(q), O.e4m3_round(k)
+    for i in range(40):
+        s = (k8[:, 0] @ q8[i, 0]) * 0.7
+        p = np.exp(s - s.max())
+        want = 0.75 * O.e4m3_round(p).sum() / p.sum()
+        assert np.allclose(out[i, 0], want, rtol=1e-12)
+    ratio = out[:, 0, 0] / 0.75
+    assert np.all(np.abs(ratio - 1) <= 2.0 ** -4) and np.any(ratio != 1)
+
+
+def test_attention_fp8_plain_error_is_e4m3_sized():
+    ends = [16, 80]
+    g = O.group_ids(ends)
+    q, k, v = (rng.standard_normal((80, 2, 32)) for _ in range(3))
+    ref = O.attention_block_causal(q, k, v, g, g, 1 / math.sqrt(32))
+    out = O.attention_block_causal_fp8_plain(q, k, v, g, g, 1 / math.sqrt(32))
+    err = np.linalg.norm(out - ref) / np.linalg.norm(ref)
+    assert 1e-3 < err < 8e-2
+
+
 # ------------------------------------------------------------ timestep
 
 
@@ -574,6 +620,75 @@ def _tiny_model(H, P, seed):
             "img_in": wt(H, P), "img_in_b": b(H), "txt_in": wt(H, H), "txt_in_b": b(H),
             "final_mod": wt(2 * H, H), "final_mod_b": b(2 * H),
             "proj_out": wt(P, H), "proj_out_b": b(P)}
+
+
+def test_adaln_rows_chunk_order():
+    """Zero weights and a bias equal to the chunk index: the six rows come out
+    as (shift1, scale1, gate1, shift2, scale2, gate2) = 0, 1, ..., 5 in that
+    order; an interleaved reshape would mix them."""
+    H = 8
+    b = np.repeat(np.arange(6.0), H)
+    rows = O.adaln_rows(rng.standard_normal(H), np.zeros((6 * H, H)), b)
+    assert rows.shape == (6, H)
+    for i in range(6):
+        assert np.array_equal(rows[i], np.full(H, float(i)))
+
+
+def test_adaln_rows_linear_part_closed_form():
+    """Chunk i of W_mod = (i + 1) I: row i = (i + 1) SiLU(temb), SiLU written
+    out with math.exp element by element."""
+    H = 6
+    t = rng.standard_normal(H) * 2
+    w = np.concatenate([(i + 1) * np.eye(H) for i in range(6)])
+    rows = O.adaln_rows(t, w, np.zeros(6 * H))
+    silu = np.array([x / (1.0 + math.exp(-x)) for x in t])
+    for i in range(6):
+        assert np.allclose(rows[i], (i + 1) * silu, rtol=1e-14, atol=0)
+
+
+def test_joint_inputs_routing():
+    """Text rows go through the text in-projection, reference and target
+    latent rows through the image in-projection, in the groups' order; in
+    the cached mode only the target rows are formed (torch float64 Linears)."""
+    H, P = 256, 64
+    mw = _tiny_model(H, P, 12)
+    groups = [("text", 3, None), ("image", 4, (2, 2)), ("image", 6, (2, 3))]
+    r = np.random.default_rng(13)
+    lat = r.standard_normal((6, P)).astype(F32)
+    ref = r.standard_normal((4, P)).astype(F32)
+    txt = O.bf16_round(r.standard_normal((3, H)))
+    T = lambda a: torch.from_numpy(np.asarray(a, np.float64))
+    want_t = F.linear(T(txt), T(mw["txt_in"]), T(mw["txt_in_b"])).numpy()
+    want_r = F.linear(T(ref), T(mw["img_in"]), T(mw["img_in_b"])).numpy()
+    want_l = F.linear(T(lat), T(mw["img_in"]), T(mw["img_in_b"])).numpy()
+    x, rows = O.joint_inputs(lat, txt, ref, mw, groups, "none")
+    assert np.array_equal(rows, np.arange(13))
+    assert np.allclose(x[:3], want_t, rtol=1e-12, atol=1e-12)
+    assert np.allclose(x[3:7], want_r, rtol=1e-12, atol=1e-12)
+    assert np.allclose(x[7:], want_l, rtol=1e-12, atol=1e-12)
+    # the two in-projections differ, so a swapped route fails the checks above
+    assert not np.allclose(F.linear(T(ref), T(mw["txt_in"][:, :P]), T(mw["txt_in_b"])).numpy(), want_r)
+    xr, rows_r = O.joint_inputs(lat, None, None, mw, groups, "read")
+    assert np.array_equal(rows_r, np.arange(7, 13)) and np.allclose(xr, want_l, rtol=1e-12, atol=1e-12)
+
+
+def test_step_text_reaches_v_only_through_blocks():
+    """With identity blocks (zero gates) v does not depend on the text rows;
+    with one real block it does (the target attends to the text group)."""
+    H, P, heads, d, eps = 256, 64, 2, 128, 1e-6
+    mw = _tiny_model(H, P, 14)
+    groups = [("text", 4, None), ("image", 6, (2, 3))]
+    r = np.random.default_rng(15)
+    lat = r.standard_normal((6, P)).astype(F32)
+    txt_a = O.bf16_round(r.standard_normal((4, H)))
+    txt_b = O.bf16_round(r.standard_normal((4, H)))
+    pw = [O.prepare_block(_tiny_weights(H, 512, d, 3))]
+    zero_mod = (np.zeros((6 * H, H)), np.zeros(6 * H))
+    live_mod = (O.bf16_round(r.standard_normal((6 * H, H)) * 0.02), O.bf16_round(r.standard_normal(6 * H) * 0.3))
+    run = lambda txt, mod: O.step_forward(lat, txt, None, mw, pw, [mod], groups, heads, d, eps,
+                                          0.8, 0.75, return_v=True)[1]
+    assert np.array_equal(run(txt_a, zero_mod), run(txt_b, zero_mod))
+    assert not np.allclose(run(txt_a, live_mod), run(txt_b, live_mod))
 
 
 def test_step_with_identity_blocks_closed_form():
