@@ -49,7 +49,9 @@ def algorithmic_work(cfg: synth.DitConfig, cached: bool = False):
     if cfg.uncond_text:
         a = algorithmic_work(dataclasses.replace(cfg, uncond_text=0), cached)
         b = algorithmic_work(cfg.uncond(), cached)
-        return {k: a[k] + b[k] for k in a}
+        out = {k: a[k] + b[k] for k in a}
+        out["gemv_bytes_per_step"] = a["gemv_bytes_per_step"]   # one time conditioning
+        return out
     H, F, d, h = cfg.hidden, cfg.mlp, cfg.head_dim, cfg.heads
     rows = cfg.target_tokens if cached else cfg.tokens
     per_block_ops = 2 * rows * (3 * H * H + H * H + F * H + H * F)
@@ -60,10 +62,30 @@ def algorithmic_work(cfg: synth.DitConfig, cached: bool = False):
     else:
         pairs = int(sum((e - s) * e for s, e in zip(starts, ends)))   # query x visible keys
     attn_flops = 4 * d * h * pairs
+    # HBM bytes of the four activation quantizers per row: LN1 reads the fp32
+    # residual (4H) and writes int8 codes (H); the attention-output quantizer
+    # reads bf16 (2H) and writes H; LN2 reads the residual and the output
+    # projection (4H + 2H), writes the residual back (4H) and the codes (H);
+    # the GELU-output quantizer reads 2F and writes F.  Plus 8 bytes (scale,
+    # zero point) per row and quantizer, and the final LayerNorm (4H in, 2H out
+    # per target row).
+    quant = cfg.blocks * rows * (19 * H + 3 * F + 32) + cfg.target_tokens * 6 * H
+    # GEMV weight bytes: the adaLN rows of every block (6H x H bf16), the final
+    # adaLN (2H x H) and the timestep MLP (H x 256 + H x H)
+    gemv = 2 * (cfg.blocks * 6 * H * H + 2 * H * H + H * 256 + H * H)
+    # bf16 Linears: text and reference in-projections (uncached), image
+    # in-projection and proj_out of the target rows
+    P, N = cfg.patch, cfg.target_tokens
+    bf16 = 2 * N * P * H * 2
+    if not cached:
+        bf16 += 2 * cfg.text_tokens * H * H + 2 * (cfg.prefix_tokens - cfg.text_tokens) * P * H
     return {
         "gemm_i8_ops_per_step": cfg.blocks * per_block_ops,
         "attn_flops_per_step": cfg.blocks * attn_flops,
         "attn_pairs_per_head": pairs,
+        "quant_bytes_per_step": quant,
+        "gemv_bytes_per_step": gemv,
+        "bf16_linear_flops_per_step": bf16,
     }
 
 
@@ -139,13 +161,30 @@ def build_model(ctx, qi, cfg, device):
     return qi.Model(ctx, dims, blocks, glob, device=device), dims
 
 
+PEAKS_INT8 = os.path.join(ROOT, "profiles", "peaks_int8.json")
+
+
 def peaks():
+    """Roofline denominators.  HBM and dense bf16: the machine's measured copy and
+    cuBLAS figures (MEASURED_PEAKS.json), else the recorded fallback.  Dense
+    int8: cuBLASLt's int8 GEMM (torch._int_mm at 8192^3) measured by
+    `bench.py --measure-peaks` into profiles/peaks_int8.json, burst and
+    sustained (4 s), else 2 x bf16 (the nominal ratio)."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
-        return {"hbm": d["hbm_gbs"], "bf16": d["bf16_tflops"],
-                "bf16_sust": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "src": "measured"}
-    return {"hbm": 6650.0, "bf16": 1590.0, "bf16_sust": 1400.0, "src": "fallback"}
+        pk = {"hbm": d["hbm_gbs"], "bf16": d["bf16_tflops"],
+              "bf16_sust": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "src": "measured"}
+    else:
+        pk = {"hbm": 6650.0, "bf16": 1590.0, "bf16_sust": 1400.0, "src": "fallback"}
+    if os.path.exists(PEAKS_INT8):
+        d = json.load(open(PEAKS_INT8))["int8_cublaslt"]
+        pk.update({"int8": d["burst_tops"], "int8_sust": d["sustained_tops"],
+                   "int8_src": "measured cuBLASLt int8 GEMM 8192^3 (profiles/peaks_int8.json)"})
+    else:
+        pk.update({"int8": 2 * pk["bf16"], "int8_sust": 2 * pk["bf16_sust"],
+                   "int8_src": f"2 x bf16 {pk['src']} (nominal int8/bf16 ratio)"})
+    return pk
 
 
 def kernel_traffic(cls: str):
@@ -168,9 +207,16 @@ def kernel_traffic(cls: str):
 # ------------------------------------------------------------------ CPU oracle sample
 
 class OracleSample:
-    """The CPU oracle on whole blocks of the 1024^2 step (S = 4608), prepared once."""
+    """The CPU oracle as it stands, on a bounded sample of the 1024^2 step
+    (S = 4608): one block on its last `rows` rows (target tokens), which
+    attend over all S keys; the K/V of the earlier rows are computed once at
+    set-up by the same oracle block (untimed).  The block's cost is linear in
+    its rows (the Linears per row, the attention per query row), so a sample
+    extrapolates to the step by (S / rows) x blocks.  Target rows attend over
+    all 4608 keys against 4153 on average over the sequence, so the
+    extrapolation overstates the step's attention part by about 10%."""
 
-    def __init__(self):
+    def __init__(self, rows: int = CFG.tokens // 4):
         from oracle import qi_oracle as O
         self.O = O
         try:
@@ -179,6 +225,7 @@ class OracleSample:
         except Exception:
             self.cores = os.cpu_count()
         cfg = CFG
+        self.rows = rows
         wts = synth.block_weights(cfg, 0)
         self.pw = O.prepare_block({k: v.float().numpy() for k, v in wts.items()})
         del wts
@@ -189,28 +236,46 @@ class OracleSample:
         self.gid = O.group_ids(ends)
         self.rs = np.where(self.gid < len(ends) - 1, 0, 1)
         self.cos, self.sin = O.rope_tables(O.rope_positions(gd))
+        self.split = cfg.tokens - rows
+        sp = self.split
+        _, self.kv = O.dit_block(self.x[:sp], self.pw, self.mod, self.rs[:sp], self.gid[:sp],
+                                 self.gid[:sp], self.cos[:sp], self.sin[:sp], cfg.heads,
+                                 cfg.head_dim, cfg.eps, return_kv=True)
 
-    def time_block(self) -> float:
-        cfg = CFG
+    def time_sample(self) -> float:
+        cfg, sp = CFG, self.split
         t0 = time.perf_counter()
-        self.O.dit_block(self.x, self.pw, self.mod, self.rs, self.gid, self.gid, self.cos,
-                         self.sin, cfg.heads, cfg.head_dim, cfg.eps)
+        self.O.dit_block(self.x[sp:], self.pw, self.mod, self.rs[sp:], self.gid[sp:], self.gid,
+                         self.cos[sp:], self.sin[sp:], cfg.heads, cfg.head_dim, cfg.eps,
+                         kv_prefix=self.kv)
         return time.perf_counter() - t0
+
+    def step_seconds(self, sample_s: float) -> float:
+        return sample_s * (CFG.tokens / self.rows) * CFG.blocks
+
+    def describe(self, sample_s: float) -> str:
+        return (f"oracle block (float64 numpy) on the last {self.rows} of {CFG.tokens} rows of the "
+                f"1024^2 step (target rows, attending over all keys; the earlier rows' K/V from an "
+                f"untimed set-up run of the same block), {sample_s:.1f} s, extrapolated "
+                f"x{CFG.tokens / self.rows:g} rows x{CFG.blocks} blocks; step-level ops "
+                f"(<1% of the work) omitted")
 
 
 def run_reference(args, rank):
     if rank != 0:
         return
-    sample = OracleSample()
+    # each step times one sample (~5 s on 16 cores), so W + K steps end
+    # within a few minutes
+    sample = OracleSample(rows=CFG.tokens // 8)
     per = []
     for i in range(args.warmup + args.steps):
-        t = sample.time_block()
+        t = sample.time_sample()
         if i >= args.warmup:
             per.append(t)
-    step_s = float(np.mean(per)) * CFG.blocks
+    mean_s = float(np.mean(per))
+    step_s = sample.step_seconds(mean_s)
     value = 1.0 / step_s
-    desc = (f"1 of {CFG.blocks} blocks of the 1024^2 step (S={CFG.tokens}) per step, float64 "
-            f"numpy oracle, extrapolated x{CFG.blocks}; step-level ops (<1% of the work) omitted")
+    desc = sample.describe(mean_s) + " (mean of the timed steps)"
     out = {
         "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
@@ -351,24 +416,32 @@ def run_ours(args, rank, world, local_rank):
         step(i, lat, txt)
     ctx.check()
 
-    # ---------------- device-resident timed region (profiled per kernel class)
+    def run_timed():
+        if denoise:
+            return 40, timed(lambda: denoise_40(lat, txt))
+        return args.steps, timed(lambda: [step(i, lat, txt) for i in range(args.steps)])
+
+    # ---------------- device-resident timed region: the headline, with no
+    # per-launch instrumentation (launches are only counted)
     clocks = ClockSampler([local_rank]) if rank == 0 else None
     if clocks:
         clocks.start()
         time.sleep(0.3)
-    ctx.profile(True)
-    if denoise:
-        n_steps = 40
-        ms_max = timed(lambda: denoise_40(lat, txt))
-    else:
-        n_steps = args.steps
-        ms_max = timed(lambda: [step(i, lat, txt) for i in range(n_steps)])
-    prof = ctx.profile_read()
     ctx.profile(False)
+    n_steps, ms_max = run_timed()
+    counts = ctx.profile_read()
     clk = clocks.stop() if clocks else None
     ctx.check()
     ms_per_step = ms_max / n_steps
     value = aggregate_throughput(world, n_steps, ms_max)
+
+    # ---------------- the same steps again with every launch bracketed by CUDA
+    # events on its stream: per-kernel-class device time for the rooflines
+    ctx.profile(True)
+    _, ms_prof = run_timed()
+    prof = ctx.profile_read()
+    ctx.profile(False)
+    ctx.check()
 
     # ---------------- cached-prefix steps (the pages' later denoising steps)
     extra = {}
@@ -416,10 +489,11 @@ def run_ours(args, rank, world, local_rank):
         ranks.close()
         return
 
-    # ---------------- roofline of the dominant kernel class
+    # ---------------- rooflines: the dominant kernel class, the tensor-core
+    # classes, and the whole step (sum of every class's roofline time)
     if denoise:
         w_full, w_cached = algorithmic_work(cfg, False), algorithmic_work(cfg, True)
-        work = {k: (w_full[k] + 39 * w_cached[k]) / 40 for k in ("gemm_i8_ops_per_step", "attn_flops_per_step")}
+        work = {k: (w_full[k] + 39 * w_cached[k]) / 40 for k in w_full}
     else:
         work = algorithmic_work(cfg)
     pk = peaks()
@@ -434,8 +508,8 @@ def run_ours(args, rank, world, local_rank):
                 "peak_note": f"bf16 dense, sustained, {pk['src']}"}
     elif dom == "gemm_i8":
         achieved = work["gemm_i8_ops_per_step"] * n_steps / (tot[dom] / 1e3) / 1e12
-        roof = {"bound": "tensor", "unit": "TOP/s", "peak": 2 * pk["bf16_sust"],
-                "peak_note": f"int8 dense = bf16 sustained {pk['src']} x nominal int8/bf16 ratio 2"}
+        roof = {"bound": "tensor", "unit": "TOP/s", "peak": pk["int8_sust"],
+                "peak_note": f"int8 dense, sustained: {pk['int8_src']}"}
     else:
         achieved = None
         roof = {"bound": "hbm", "unit": "GB/s", "peak": pk["hbm"], "peak_note": pk["src"]}
@@ -443,25 +517,42 @@ def run_ours(args, rank, world, local_rank):
     roof.update({"kernel": dom, "achieved": achieved,
                  "frac": (achieved / roof["peak"]) if achieved else None,
                  "traffic": tr, "ms_per_step": tot[dom] / n_steps,
-                 "launches_per_step": prof[dom][0] / n_steps})
+                 "launches_per_step": prof[dom][0] / n_steps,
+                 "timing": "CUDA events around each launch on its stream, in a second run of "
+                           "the same steps (the headline run is not instrumented)"})
     other = {}
     if prof["gemm_i8"][0]:
         a = work["gemm_i8_ops_per_step"] * n_steps / (tot["gemm_i8"] / 1e3) / 1e12
-        other["gemm_i8"] = {"achieved_tops": a, "peak_tops": 2 * pk["bf16_sust"],
-                            "frac": a / (2 * pk["bf16_sust"])}
+        other["gemm_i8"] = {"achieved_tops": a, "peak_tops": pk["int8_sust"],
+                            "frac": a / pk["int8_sust"], "frac_of_burst": a / pk["int8"],
+                            "peak_note": pk["int8_src"]}
     if prof["attention"][0]:
         a = work["attn_flops_per_step"] * n_steps / (tot["attention"] / 1e3) / 1e12
         other["attention"] = {"achieved_tflops": a, "peak_tflops": pk["bf16_sust"],
-                              "frac": a / pk["bf16_sust"]}
+                              "frac": a / pk["bf16_sust"], "frac_of_burst": a / pk["bf16"],
+                              "peak_note": f"bf16 dense {pk['src']}"}
+    # whole step: each class's algorithmic work at its own roofline, summed,
+    # against the measured (uninstrumented) step time
+    ideal = {
+        "gemm_i8": work["gemm_i8_ops_per_step"] / (pk["int8_sust"] * 1e12) * 1e3,
+        "attention": work["attn_flops_per_step"] / (pk["bf16_sust"] * 1e12) * 1e3,
+        "quant": work["quant_bytes_per_step"] / (pk["hbm"] * 1e9) * 1e3,
+        "gemv": work["gemv_bytes_per_step"] / (pk["hbm"] * 1e9) * 1e3,
+        "gemm_bf16": work["bf16_linear_flops_per_step"] / (pk["bf16_sust"] * 1e12) * 1e3,
+    }
+    step_roof = {"ideal_ms": sum(ideal.values()), "measured_ms": ms_per_step,
+                 "frac": sum(ideal.values()) / ms_per_step,
+                 "ideal_ms_by_class": ideal,
+                 "note": "sum over kernel classes of algorithmic work / peak (int8 and bf16 "
+                         "sustained tensor peaks, HBM copy bandwidth) over the measured step"}
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline and cfg is synth.STEP1024:
-        osamp = OracleSample()
-        tb = osamp.time_block()
-        v = 1.0 / (tb * cfg.blocks)
+        osamp = OracleSample(rows=CFG.tokens // 4)
+        ts = float(np.mean([osamp.time_sample() for _ in range(3)]))
+        v = 1.0 / osamp.step_seconds(ts)
         cpu = {"value": v, "unit": "steps/s", "cores": osamp.cores, "kind": "oracle",
-               "sample": (f"1 of {cfg.blocks} blocks of the 1024^2 step (S={cfg.tokens}), "
-                          f"float64 numpy oracle, {tb:.1f} s, extrapolated x{cfg.blocks}")}
+               "sample": osamp.describe(ts) + " (mean of 3 samples)"}
 
     desc = (f"{cfg.name}: {cfg.blocks} blocks, hidden {H}, {cfg.heads}x128 heads, MLP {cfg.mlp}, "
             f"groups {'|'.join(str(n) for n in cfg.group_sizes())} tokens, "
@@ -482,12 +573,13 @@ def run_ours(args, rank, world, local_rank):
                    "parallelism": f"replicas x{world}"},
         "roofline": roof,
         "tensor_core_fracs": other,
+        "step_roofline": step_roof,
         "kernels": kernels,
         "extra": extra,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e, "unit": "steps/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": int(sum(v[0] for v in prof.values())),
+        "gpu_launches": int(sum(v[0] for v in counts.values())),
         "clocks": clk,
     }
     print(json.dumps(out), flush=True)
@@ -499,7 +591,10 @@ def run_ncu_case(args):
     gemms:     the block's four W8A8 GEMMs (QKV, out, up, down) in block order;
     gemm_down: W8A8 down projection, M = 4608, N = 4096, K = 16384 (operands
                142 MB > L2);
-    attention: block-causal attention over [512 | 4096] tokens, 32 heads."""
+    attention: block-causal attention over [512 | 4096] tokens, 32 heads;
+    block:     one whole block at S = 4608 (4 quantizer launches, 4 GEMMs, attention);
+    gemv:      the time conditioning of an 8-block model (3 GEMV launches)."""
+    import ctypes as C
     from diffusion_transformer_text_dit_b200 import build_lib, qi
     build_lib.build()
     ctx = qi.Context(0)
@@ -558,6 +653,58 @@ def run_ncu_case(args):
         y = torch.empty((S, H), device="cuda", dtype=torch.bfloat16)
         for _ in range(args.warmup + args.steps):
             qi.qi_w8a8_linear(ctx, qa, sa, zp, ws, y=y)
+    elif args.ncu_case == "block":
+        # one whole block at the 1024^2 shapes (S = 4608): every quantizer form
+        # (LayerNorm with and without the residual add, range-fed on the
+        # attention and GELU outputs), the four GEMMs and the attention
+        wts = synth.block_weights(cfg, 0, device="cuda")
+        bw = qi.BlockWeights(ctx, wts)
+        del wts
+        dims = qi.dims_struct(H, cfg.heads, F, cfg.patch, 1)
+        groups = qi.groups_struct(list(np.cumsum(cfg.group_sizes())), cfg.group_row_sets())
+        cos, sin = (t.cuda() for t in qi.qi_rope_tables([(gr.kind, gr.tokens, gr.grid) for gr in cfg.groups]))
+        x0 = synth.hidden_states(cfg, S, device="cuda")
+        mod = synth.mod_table(cfg, device="cuda")
+        kl = torch.empty((S, H), dtype=torch.bfloat16, device="cuda")
+        vl = torch.empty_like(kl)
+        ws = torch.empty(qi.qi_block_workspace_bytes(dims, S), dtype=torch.uint8, device="cuda")
+        x = x0.clone()
+        for _ in range(args.warmup + args.steps):
+            x.copy_(x0)
+            qi.qi_dit_block_forward(ctx, dims, bw.struct, x, 0, mod, groups, cos, sin, kl, vl,
+                                    qi.QI_KV_NONE, ws)
+    elif args.ncu_case == "gemv":
+        # the time conditioning of an 8-block model (1.6 GB of adaLN weights;
+        # a 32-block step reads 4x as many): one GEMV launch covers every
+        # block's adaLN rows and the final adaLN
+        nb = 8
+        wts = synth.block_weights(cfg, 0, device="cuda")
+        bw = qi.BlockWeights(ctx, wts)
+        del wts
+        mods = [synth.linear_weight(cfg.weight_seed, ("ncu_mod", l), 6 * H, H, "cuda").to(torch.bfloat16)
+                for l in range(nb)]
+        structs = []
+        for l in range(nb):
+            st_ = qi.qi_block_weights.from_buffer_copy(bw.struct)
+            st_.mod = qi.bf16_struct(mods[l])
+            structs.append(st_)
+        dims = qi.dims_struct(H, cfg.heads, F, cfg.patch, nb)
+        model = qi.Model.__new__(qi.Model)
+        model.dims = dims
+        model.g = {k: v.to(torch.bfloat16).contiguous() for k, v in synth.model_weights(cfg, device="cuda").items()}
+        arr = (qi.qi_block_weights * nb)(*structs)
+        m = qi.qi_model()
+        m.dims = dims
+        m.blocks = C.cast(arr, C.POINTER(qi.qi_block_weights))
+        for name in ("t1", "t2", "img_in", "txt_in", "final_mod", "proj_out"):
+            setattr(m, name, qi.bf16_struct(model.g[name], model.g[name + "_b"]))
+        model.struct = m
+        model._arr = arr
+        ws = torch.empty(qi.qi_step_workspace_bytes(dims, 8), dtype=torch.uint8, device="cuda")
+        bm = torch.empty((nb, 2, 6 * H), dtype=torch.bfloat16, device="cuda")
+        fm = torch.empty((2, 2 * H), dtype=torch.bfloat16, device="cuda")
+        for i in range(args.warmup + args.steps):
+            qi.qi_time_conditioning(ctx, model, 0.5 + 0.01 * i, bm, fm, ws)
     elif args.ncu_case == "attention":
         q = (torch.randn(S, H, device="cuda", generator=g)).to(torch.bfloat16)
         k = (torch.randn(S, H, device="cuda", generator=g)).to(torch.bfloat16)
@@ -569,6 +716,73 @@ def run_ncu_case(args):
     torch.cuda.synchronize()
     ctx.check()
     print(json.dumps({"ncu_case": args.ncu_case, "launches": args.warmup + args.steps}))
+
+
+def measure_peaks(args):
+    """Dense tensor peaks on this GPU, each as a burst (20 launches after 3
+    warm-up) and sustained (back-to-back launches for 4 s, SM clock sampled):
+      int8_cublaslt  cuBLASLt int8 GEMM, torch._int_mm [8192 x 8192] x [8192 x 8192]
+      bf16_cublas    cuBLAS bf16 GEMM, torch.matmul at 8192^3
+      int8_probe / bf16_probe  libqi's tensor-pipe probe: back-to-back
+                     tcgen05.mma on shared-memory operands on every SM (the
+                     pipe's own rate at the clock it runs at)
+    Writes profiles/peaks_int8.json (read by the roofline) and prints it."""
+    from diffusion_transformer_text_dit_b200 import build_lib, qi
+    build_lib.build()
+    torch.cuda.set_device(0)
+    ctx = qi.Context(0)
+    st = torch.cuda.current_stream()
+    n = 8192
+    g = torch.Generator(device="cuda").manual_seed(0)
+    a8 = torch.randint(-128, 128, (n, n), dtype=torch.int8, device="cuda", generator=g)
+    b8 = torch.randint(-128, 128, (n, n), dtype=torch.int8, device="cuda", generator=g).t()
+    ab = torch.randn(n, n, device="cuda", generator=g).to(torch.bfloat16)
+    bb = torch.randn(n, n, device="cuda", generator=g).to(torch.bfloat16).t()
+    probe_ops = {True: None, False: None}
+
+    def probe(i8):
+        probe_ops[i8] = qi.qi_debug_mma_probe(ctx, i8, 20000)
+
+    cases = {"int8_cublaslt": (lambda: torch._int_mm(a8, b8), 2 * n ** 3),
+             "bf16_cublas": (lambda: torch.matmul(ab, bb), 2 * n ** 3),
+             "int8_probe": (lambda: probe(True), None),
+             "bf16_probe": (lambda: probe(False), None)}
+    out = {"gpu": torch.cuda.get_device_name(0),
+           "date": datetime.datetime.now(datetime.timezone.utc).isoformat(timespec="seconds"),
+           "command": "python bench.py --measure-peaks"}
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for name, (fn, ops) in cases.items():
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0.record(st)
+        for _ in range(20):
+            fn()
+        e1.record(st)
+        torch.cuda.synchronize()
+        ops = ops if ops is not None else probe_ops[name.startswith("int8")]
+        burst = ops * 20 / (e0.elapsed_time(e1) / 1e3) / 1e12
+        clocks = ClockSampler([0])
+        clocks.start()
+        time.sleep(0.3)
+        e0.record(st)
+        t_end = time.time() + 4.0
+        launches = 0
+        while time.time() < t_end:
+            for _ in range(8):
+                fn()
+            launches += 8
+            torch.cuda.synchronize()
+        e1.record(st)
+        torch.cuda.synchronize()
+        clk = clocks.stop()
+        sust = ops * launches / (e0.elapsed_time(e1) / 1e3) / 1e12
+        out[name] = {"burst_tops": burst, "sustained_tops": sust, "sustained_seconds":
+                     e0.elapsed_time(e1) / 1e3, "ops_per_launch": ops, "clocks": clk}
+    ctx.check()
+    with open(PEAKS_INT8, "w") as f:
+        json.dump(out, f, indent=1)
+    print(json.dumps(out), flush=True)
 
 
 def main():
@@ -587,9 +801,16 @@ def main():
                          "denoise40_2048px: the full 40-step 2048^2 denoise; "
                          "denoise40_2048px_sched: the same with the pages' precision schedule "
                          "(fp8 attention from step 8)")
-    ap.add_argument("--ncu-case", choices=("gemms", "gemm_down", "attention"), default=None,
+    ap.add_argument("--ncu-case", choices=("gemms", "gemm_down", "attention", "block", "gemv"),
+                    default=None,
                     help="launch one kernel a few times (for ncu captures) and exit")
+    ap.add_argument("--measure-peaks", action="store_true",
+                    help="measure dense int8 / bf16 tensor peaks (cuBLASLt, cuBLAS and libqi's "
+                         "tcgen05 probe) into profiles/peaks_int8.json and exit")
     args = ap.parse_args()
+    if args.measure_peaks:
+        measure_peaks(args)
+        return
     if args.ncu_case:
         run_ncu_case(args)
         return

@@ -30,6 +30,8 @@ struct qi_ctx {
   int* prof_cls;                 // [QI_PROF_MAX_PAIRS]
   long long launches[QI_PROF_CLASSES];
   int attn_fp8;                  // steps run e4m3 attention (qi_ctx_set_attention_fp8)
+  bool taps_on;                  // copy the quantizers' inputs and outputs (qi_ctx_set_block_taps)
+  qi_block_taps taps;
 };
 
 namespace {
@@ -275,7 +277,25 @@ struct QuantExtras {
   const uint16_t* res_gate = nullptr;
   uint32_t* zero_range = nullptr;      // LN: clear these row ranges
   const uint32_t* range = nullptr;     // plain: producer-published row ranges
+  float* u_f32 = nullptr;              // LN: also write the quantized value u (fp32 tap)
 };
+
+// Stream-ordered device copy of a tap (skipped when the tap is NULL).
+int tap_copy(void* dst, const void* src, size_t bytes, cudaStream_t st) {
+  if (!dst || bytes == 0) return QI_OK;
+  if (cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return cuda_fail("tap copy");
+  return QI_OK;
+}
+
+// Copy one quantizer's codes, scales and zero points into the taps.
+int tap_codes(int8_t* q_dst, float* s_dst, int32_t* zp_dst, const int8_t* q, const float* s,
+              const int32_t* zp, int T, int K, cudaStream_t st) {
+  int r;
+  if ((r = tap_copy(q_dst, q, static_cast<size_t>(T) * K, st))) return r;
+  if ((r = tap_copy(s_dst, s, static_cast<size_t>(T) * sizeof(float), st))) return r;
+  return tap_copy(zp_dst, zp, static_cast<size_t>(T) * sizeof(int32_t), st);
+}
 
 int run_quant(qi_ctx* ctx, const void* x, bool xbf16, int M, int K, int ldx,
               const uint16_t* shift, const uint16_t* scale, int mod_ld, const qi::GroupTable& gt,
@@ -287,6 +307,7 @@ int run_quant(qi_ctx* ctx, const void* x, bool xbf16, int M, int K, int ldx,
   p.res_gate = ex.res_gate;
   p.zero_range = ex.zero_range;
   p.range = ex.range;
+  p.u_f32 = ex.u_f32;
   p.x = x;
   p.x_bf16 = xbf16 ? 1 : 0;
   p.M = M;
@@ -393,12 +414,15 @@ int run_block_multi(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, fl
   int r;
   // attention half.  LN1 + modulate + quantize; it also clears the row
   // ranges that the attention epilogue will publish for the next quantizer.
+  const qi_block_taps* tp = ctx->taps_on ? &ctx->taps : nullptr;
   {
     QuantExtras ex;
     ex.zero_range = b.o_range;
+    ex.u_f32 = tp ? tp->u1 : nullptr;
     if ((r = run_quant(ctx, x, false, T, H, H, mod + 0 * H, mod + 1 * H, mld, gt, row0, d.eps,
                        b.uq, b.sa, b.zp, nullptr, st, ex)))
       return r;
+    if (tp && (r = tap_codes(tp->q1, tp->s1, tp->zp1, b.uq, b.sa, b.zp, T, H, st))) return r;
   }
   // QKV projection with Q/K RMSNorm + RoPE fused into its epilogue: q goes to
   // the block's q buffer, k and v straight into this layer's K/V rows.
@@ -504,12 +528,16 @@ int run_block_multi(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, fl
     if (r2 == -2) return fail(QI_ERR_CUDA, "cuTensorMapEncodeTiled failed (attention operands)");
     if (r2 != 0) return cuda_fail("attention launch");
   }
+  if (tp && ((r = tap_copy(tp->o, b.o, static_cast<size_t>(T) * H * 2, st)) ||
+             (r = tap_copy(tp->o_range, b.o_range, static_cast<size_t>(T) * 8, st))))
+    return r;
   {
     QuantExtras ex;   // the attention epilogue published each row's range
     ex.range = b.o_range;
     if ((r = run_quant(ctx, b.o, true, T, H, H, nullptr, nullptr, 0, gt, row0, d.eps, b.uq, b.sa,
                        b.zp, nullptr, st, ex)))
       return r;
+    if (tp && (r = tap_codes(tp->qo, tp->so, tp->zpo, b.uq, b.sa, b.zp, T, H, st))) return r;
   }
   // output projection stored as bf16 (into the attention output's buffer,
   // already consumed); its gated residual is applied by the LN2 kernel below,
@@ -523,12 +551,19 @@ int run_block_multi(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, fl
     ex.res_y = b.o;
     ex.res_gate = mod + 2 * H;
     ex.zero_range = b.g_range;
+    ex.u_f32 = tp ? tp->u2 : nullptr;
     if ((r = run_quant(ctx, x, false, T, H, H, mod + 3 * H, mod + 4 * H, mld, gt, row0, d.eps,
                        b.uq, b.sa, b.zp, nullptr, st, ex)))
+      return r;
+    if (tp && ((r = tap_copy(tp->x_mid, x, static_cast<size_t>(T) * H * 4, st)) ||
+               (r = tap_codes(tp->q2, tp->s2, tp->zp2, b.uq, b.sa, b.zp, T, H, st))))
       return r;
   }
   if ((r = run_w8a8(ctx, b.uq, b.sa, b.zp, T, w.up, qi::EPI_GELU, b.g, F, nullptr, 0, nullptr, 0,
                     gt, row0, nullptr, st, b.g_range)))
+    return r;
+  if (tp && ((r = tap_copy(tp->g, b.g, static_cast<size_t>(T) * F * 2, st)) ||
+             (r = tap_copy(tp->g_range, b.g_range, static_cast<size_t>(T) * 8, st))))
     return r;
   {
     QuantExtras ex;   // the GELU epilogue published each row's range
@@ -536,6 +571,7 @@ int run_block_multi(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, fl
     if ((r = run_quant(ctx, b.g, true, T, F, F, nullptr, nullptr, 0, gt, row0, d.eps, b.uq, b.sa,
                        b.zp, nullptr, st, ex)))
       return r;
+    if (tp && (r = tap_codes(tp->qg, tp->sg, tp->zpg, b.uq, b.sa, b.zp, T, F, st))) return r;
   }
   if ((r = run_w8a8(ctx, b.uq, b.sa, b.zp, T, w.down, qi::EPI_GATED, nullptr, 0, x, H,
                     mod + 5 * H, mld, gt, row0, nullptr, st)))
@@ -720,6 +756,8 @@ int qi_ctx_create(int device, qi_ctx** out) {
   c->prof_ev = nullptr;
   c->prof_cls = nullptr;
   c->attn_fp8 = 0;
+  c->taps_on = false;
+  memset(&c->taps, 0, sizeof(c->taps));
   for (int i = 0; i < QI_PROF_CLASSES; ++i) c->launches[i] = 0;
   if (cudaMalloc(&c->status, 256) != cudaSuccess) {
     delete c;
@@ -1002,6 +1040,24 @@ int qi_mxfp4_decode(qi_ctx* ctx, const uint8_t* packed, const uint8_t* scales, i
   Prof pr(ctx, QI_KCLASS_OTHER, S(stream));
   if (qi::launch_mxfp4_decode(packed, scales, n, k_stored, k, w, S(stream)))
     return cuda_fail("MXFP4 decode launch");
+  return QI_OK;
+}
+
+int qi_ctx_set_block_taps(qi_ctx* ctx, const qi_block_taps* taps) {
+  if (!ctx) return fail(QI_ERR_INVALID_ARG, "NULL context");
+  if (!taps) {
+    ctx->taps_on = false;
+    memset(&ctx->taps, 0, sizeof(ctx->taps));
+    return QI_OK;
+  }
+  const void* ptrs[] = {taps->u1, taps->q1, taps->s1, taps->zp1, taps->o, taps->o_range,
+                        taps->qo, taps->so, taps->zpo, taps->x_mid, taps->u2, taps->q2,
+                        taps->s2, taps->zp2, taps->g, taps->g_range, taps->qg, taps->sg,
+                        taps->zpg};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return fail(QI_ERR_ALIGNMENT, "tap buffers must be 16-byte aligned");
+  ctx->taps = *taps;
+  ctx->taps_on = true;
   return QI_OK;
 }
 
@@ -1533,6 +1589,15 @@ int qi_ctx_profile_read(qi_ctx* ctx, int kernel_class, long long* launches, int*
     *total_ms += ms;
     *timed += 1;
   }
+  return QI_OK;
+}
+
+int qi_debug_mma_probe(qi_ctx* ctx, int int8, int iters, void* stream) {
+  if (!ctx) return fail(QI_ERR_INVALID_ARG, "ctx is NULL");
+  if (iters < 1 || iters > 100000) return fail(QI_ERR_INVALID_ARG, "iters outside 1 .. 100000");
+  Prof pr(ctx, QI_KCLASS_OTHER, S(stream));
+  if (qi::launch_mma_probe(int8 != 0, iters, ctx->num_sms, ctx->status, S(stream)) != 0)
+    return cuda_fail("mma probe launch");
   return QI_OK;
 }
 

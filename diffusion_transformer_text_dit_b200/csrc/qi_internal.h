@@ -138,6 +138,7 @@ struct QuantParams {
   const uint16_t* res_y;  // bf16 [M, K] or null
   const uint16_t* res_gate;   // gate row of set r at res_gate + r * mod_ld
   uint32_t* zero_range;   // if non-null: rows' [2] range words set to 0 (for a later producer)
+  float* u_f32;           // LN variant, if non-null: also write u (the quantized value) [M, ldq] fp32
   // plain variant: the row's range was published by the producer as
   // [float bits of -min, float bits of max] (both >= 0); no reduction needed
   const uint32_t* range;
@@ -202,6 +203,9 @@ int launch_gemv(const GemvParams& p, cudaStream_t st);
 
 int launch_timestep_embedding(float t0, float t1, float* out, cudaStream_t st);
 int launch_timeout_probe(uint64_t limit_ns, int* status, cudaStream_t st);
+// Back-to-back tcgen05.mma (kind::i8 or kind::f16, M = 128, N = 256) on
+// shared-memory operands, `iters` x 4 MMAs per CTA, one CTA per SM.
+int launch_mma_probe(bool i8, int iters, int num_sms, int* status, cudaStream_t st);
 int launch_f32_to_bf16(const float* x, uint16_t* y, int64_t n, cudaStream_t st);
 int launch_euler(float* x, const float* v, int64_t n, float dt, cudaStream_t st);
 // MXFP4 (E2M1 codes, low nibble first; E8M0 scale per 32 columns) -> fp32 [n, k].

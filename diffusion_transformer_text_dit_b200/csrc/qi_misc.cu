@@ -374,4 +374,88 @@ int launch_timeout_probe(uint64_t limit_ns, int* status, cudaStream_t st) {
   return launch_result();
 }
 
+// ---------------------------------------------------------------- tensor-pipe probe
+//
+// Back-to-back tcgen05.mma (M = 128, N = 256, one 128-byte K row = 4 MMAs per
+// iteration) on operands resident in shared memory: no loads, no epilogue, so
+// the launch measures the tensor pipe's own rate at the clock the GPU holds
+// while it runs.  The operands are pseudo-random (int8 bytes, or bf16 values
+// of magnitude [1, 2) with random signs), so the switching activity, and with
+// it the power drawn, is that of real data.  One CTA per SM.
+constexpr int PROBE_A_BYTES = 128 * 128;
+constexpr int PROBE_B_BYTES = 256 * 128;
+constexpr int PROBE_SMEM = 1024 + PROBE_A_BYTES + PROBE_B_BYTES;
+
+template <bool I8>
+__global__ void __launch_bounds__(128, 1) mma_probe_kernel(int iters, int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint64_t done;
+  __shared__ uint32_t tslot;
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint32_t* w = reinterpret_cast<uint32_t*>(sm);
+  for (int i = threadIdx.x; i < (PROBE_A_BYTES + PROBE_B_BYTES) / 4; i += blockDim.x) {
+    uint32_t h = static_cast<uint32_t>(i) * 2654435761u + blockIdx.x * 40503u;
+    h ^= h >> 15;
+    h *= 2246822519u;
+    h ^= h >> 13;
+    // bf16: exponent of 1.0 with a random mantissa and sign in each half
+    w[i] = I8 ? h : ((h & 0x807F807Fu) | 0x3F803F80u);
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  if (threadIdx.x < 32) {
+    tmem_alloc(&tslot, 256);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 0) {
+    mbar_init(&done, 1);
+    fence_mbar_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tslot;
+  if (threadIdx.x == 0) {
+    constexpr uint32_t idesc = umma_idesc(I8, 128, 256);
+    const uint64_t a = umma_desc_kmajor_sw128(smem_u32(sm));
+    const uint64_t b = umma_desc_kmajor_sw128(smem_u32(sm + PROBE_A_BYTES));
+    for (int it = 0; it < iters; ++it) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint64_t off = static_cast<uint64_t>(k * 32) >> 4;
+        if (I8)
+          umma_i8(tmem, a + off, b + off, idesc, (it | k) != 0);
+        else
+          umma_f16(tmem, a + off, b + off, idesc, (it | k) != 0);
+      }
+    }
+    umma_commit(&done);
+    if (!mbar_wait(&done, 0, status)) {
+      // the MMAs must be finished before their TMEM is released
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(&done, 0) && globaltimer_ns() - t0 < QI_WAIT_NS) {
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (threadIdx.x < 32) tmem_dealloc(tmem, 256);
+}
+
+int launch_mma_probe(bool i8, int iters, int num_sms, int* status, cudaStream_t st) {
+  static bool attr[2] = {false, false};
+  auto kern = i8 ? mma_probe_kernel<true> : mma_probe_kernel<false>;
+  if (!attr[i8]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PROBE_SMEM) !=
+        cudaSuccess) {
+      launch_result();
+      return -1;
+    }
+    attr[i8] = true;
+  }
+  kern<<<num_sms, 128, PROBE_SMEM, st>>>(iters, status);
+  return launch_result();
+}
+
 }  // namespace qi

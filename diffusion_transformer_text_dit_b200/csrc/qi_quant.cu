@@ -280,6 +280,19 @@ __global__ void __launch_bounds__(512) quant_ln_kernel(const QuantParams p) {
     }
     return;
   }
+  if (p.u_f32) {   // tap: the exact fp32 values quantized below
+#pragma unroll
+    for (int c = 0; c < LN_CH; ++c) {
+      const int ch = tid + c * nt;
+      if (ch >= nchunk) continue;
+      float e[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) f2_unpack(v[c][i], e[2 * i], e[2 * i + 1]);
+      float4* o4 = reinterpret_cast<float4*>(p.u_f32 + static_cast<int64_t>(row) * p.ldq + ch * 8);
+      o4[0] = make_float4(e[0], e[1], e[2], e[3]);
+      o4[1] = make_float4(e[4], e[5], e[6], e[7]);
+    }
+  }
   float lo = 0.f, hi = 0.f;
 #pragma unroll
   for (int c = 0; c < LN_CH; ++c)

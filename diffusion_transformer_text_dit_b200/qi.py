@@ -87,6 +87,14 @@ class qi_seq(C.Structure):
                 ("rope_sin", C.c_void_p), ("kv_cache", C.c_void_p)]
 
 
+TAP_FIELDS = ("u1", "q1", "s1", "zp1", "o", "o_range", "qo", "so", "zpo", "x_mid", "u2", "q2",
+              "s2", "zp2", "g", "g_range", "qg", "sg", "zpg")
+
+
+class qi_block_taps(C.Structure):
+    _fields_ = [(name, C.c_void_p) for name in TAP_FIELDS]
+
+
 # ------------------------------------------------------------------ loading
 
 _lib = None
@@ -117,6 +125,7 @@ _SIGS = {
                                  C.POINTER(qi_groups), C.c_float, C.c_void_p, C.c_int, C.c_void_p],
     "qi_to_e4m3": [C.c_void_p, C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p],
     "qi_ctx_set_attention_fp8": [C.c_void_p, C.c_int],
+    "qi_ctx_set_block_taps": [C.c_void_p, C.POINTER(qi_block_taps)],
     "qi_mxfp4_decode": [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_int,
                         C.c_void_p, C.c_void_p],
     "qi_block_workspace_bytes": [C.POINTER(qi_dims), C.c_int, C.POINTER(C.c_size_t)],
@@ -146,6 +155,7 @@ _SIGS = {
                        C.POINTER(C.c_int32), C.POINTER(C.c_int32), C.c_void_p, C.c_void_p],
     "qi_sigma_schedule": [C.c_int, C.c_int, C.c_void_p],
     "qi_debug_timeout_probe": [C.c_void_p, C.c_uint64, C.c_void_p],
+    "qi_debug_mma_probe": [C.c_void_p, C.c_int, C.c_int, C.c_void_p],
     "qi_ctx_profile": [C.c_void_p, C.c_int],
     "qi_ctx_profile_read": [C.c_void_p, C.c_int, C.POINTER(C.c_longlong), C.POINTER(C.c_int),
                             C.POINTER(C.c_double)],
@@ -229,6 +239,19 @@ class Context:
     def set_attention_fp8(self, enable: bool):
         """e4m3 attention in the steps run on this context (qi_ctx_set_attention_fp8)."""
         check(lib().qi_ctx_set_attention_fp8(self.handle, 1 if enable else 0))
+
+    def set_block_taps(self, taps: Optional[dict]):
+        """Copy each block quantizer's input and output into the given device
+        tensors (qi_ctx_set_block_taps; keys from TAP_FIELDS), or stop (None)."""
+        if taps is None:
+            check(lib().qi_ctx_set_block_taps(self.handle, None))
+            self._taps = None
+            return
+        st = qi_block_taps()
+        for name in TAP_FIELDS:
+            setattr(st, name, ptr(taps.get(name)))
+        check(lib().qi_ctx_set_block_taps(self.handle, C.byref(st)))
+        self._taps = taps   # keep the buffers alive while the library holds their pointers
 
     def profile(self, enable: bool):
         """Reset launch counters; time every launch with CUDA events if enable."""
@@ -483,6 +506,13 @@ def qi_sigma_schedule(steps: int, image_tokens: int):
     out = torch.empty(steps + 1, dtype=torch.float32)
     check(lib().qi_sigma_schedule(steps, image_tokens, out.data_ptr()))
     return out
+
+
+def qi_debug_mma_probe(ctx: Context, int8: bool, iters: int, stream=None):
+    """Back-to-back tcgen05.mma on every SM; returns the ops of the launch."""
+    check(lib().qi_debug_mma_probe(ctx.handle, 1 if int8 else 0, iters, stream_ptr(stream)))
+    sms = torch.cuda.get_device_properties(ctx.device).multi_processor_count
+    return sms * iters * 4 * 2 * 128 * 256 * (32 if int8 else 16)
 
 
 def qi_debug_timeout_probe(ctx: Context, limit_ns: int, stream=None):

@@ -314,6 +314,49 @@ int qi_mxfp4_decode(qi_ctx* ctx, const uint8_t* packed, const uint8_t* scales, i
  * steps).  Block-level calls are not affected.  Default 0. */
 int qi_ctx_set_attention_fp8(qi_ctx* ctx, int enable);
 
+/* Copies of what each activation quantizer of a block reads and writes, for
+ * checking those quantizers bit for bit at their own inputs ([W8]: dynamic
+ * asymmetric INT8 per token with FP32 scales).  Every pointer is a caller-owned
+ * device buffer for the block's T processed rows, or NULL to skip that tap.
+ *   u1, u2     [T, H] fp32: LN(x)(1 + scale) + shift as the two LayerNorm
+ *              quantizers computed and quantized it (written by those kernels)
+ *   x_mid      [T, H] fp32: the residual stream after the attention half
+ *              (x + gate1 * out), the input of the second LayerNorm
+ *   o          [T, H] bf16: attention output, the input of the third quantizer
+ *   g          [T, F] bf16: GELU output, the input of the fourth quantizer
+ *   o_range, g_range [T, 2] uint32: the range the attention / GELU epilogue
+ *              published for each row, as float bits of (-min(min, 0), max(max, 0))
+ *   q*, s*, zp* codes [T, H or F] int8, scales [T] fp32, zero points [T] int32
+ *              of quantizer 1 (u1), o (o), 2 (u2) and g (g).
+ * The taps are copied with stream-ordered device copies after the kernels that
+ * produce them; they cost time and are meant for tests. */
+typedef struct qi_block_taps {
+  float* u1;
+  int8_t* q1;
+  float* s1;
+  int32_t* zp1;
+  uint16_t* o;
+  uint32_t* o_range;
+  int8_t* qo;
+  float* so;
+  int32_t* zpo;
+  float* x_mid;
+  float* u2;
+  int8_t* q2;
+  float* s2;
+  int32_t* zp2;
+  uint16_t* g;
+  uint32_t* g_range;
+  int8_t* qg;
+  float* sg;
+  int32_t* zpg;
+} qi_block_taps;
+
+/* Take the taps above in every block this context runs from now on (each block
+ * overwrites them), or stop with taps = NULL.  The struct is copied; the
+ * buffers must hold the T rows of the blocks run.  Host-side, no launch. */
+int qi_ctx_set_block_taps(qi_ctx* ctx, const qi_block_taps* taps);
+
 /* Workspace bytes needed by qi_dit_block_forward for T processed rows. */
 int qi_block_workspace_bytes(const qi_dims* dims, int T, size_t* bytes);
 
@@ -453,6 +496,15 @@ int qi_rope_tables(int n_groups, const int32_t* kinds, const int32_t* tokens,
  * e^mu / (e^mu + 1/sigma - 1), mu linear in image_tokens (0.5 at 256 tokens,
  * 0.9 at 8192), tail stretched to 0.02, then 0 appended.  Writes HOST sigmas[steps+1]. */
 int qi_sigma_schedule(int steps, int image_tokens, float* sigmas);
+
+/* Tensor-pipe probe (measurement support): one CTA per SM issues iters x 4
+ * back-to-back tcgen05.mma (M = 128, N = 256, K = 32 int8 bytes for
+ * int8 != 0, else K = 16 bf16 values) on pseudo-random operands held in shared
+ * memory, with no memory traffic and no epilogue.  Work per launch:
+ * num_SMs * iters * 4 * 2 * 128 * 256 * K operations.  Time it with CUDA events
+ * on `stream`; the result is the tensor pipe's dense rate at the clock the GPU
+ * holds meanwhile.  iters in 1 .. 100000. */
+int qi_debug_mma_probe(qi_ctx* ctx, int int8, int iters, void* stream);
 
 /* Failure-detection probe: launch one CTA that waits on an mbarrier nothing
  * arrives on, bounded by limit_ns (1e3 .. 5e9).  The wait expires, the kernel

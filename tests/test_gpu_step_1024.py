@@ -1,0 +1,120 @@
+"""Full-width parity of the two 1024x1024 workloads against the oracle.
+
+The full 32-block step (hidden 4096, 32 heads, MLP 16384, [512 text | 4096
+image] tokens, uncached) and the image-conditioned edit ([256 text | 1024
+reference | 4096 target]: a first step that writes the text + reference K/V,
+then a second step that reads them and processes the target rows only) are
+compared with velocities the float64 oracle computed on the same seeded
+inputs (tests/golden/make_step_goldens.py; the oracle needs 10-30 minutes per
+step, so its outputs are stored).  Tolerance: rel-L2 <= 2e-2 on v after the
+32-block stack.  The Euler update must be bit-exact given the GPU's own v
+(RGBA-Image-2.1 Core AI port, "Graph contracts", Sampler), and the cached
+second step must equal the uncached one bit for bit ("Qwen Image 2.1 native
+qualification", "Numerical checks": cached vs uncached second steps).
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from diffusion_transformer_text_dit_b200 import qi, synth
+from oracle import qi_oracle as O
+from tests._util import cuda, rel_l2
+from tests.golden.make_step_goldens import input_hashes
+
+pytestmark = pytest.mark.gpu
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, f"{name}.json")) as f:
+        meta = json.load(f)
+    return meta, [np.load(os.path.join(GOLDEN, st["v"])) for st in meta["steps"]]
+
+
+@pytest.fixture(scope="module")
+def model(ctx):
+    """The 32-block model of both workloads (same weight seed and shapes),
+    drawn on the host one block at a time exactly as the oracle run drew it."""
+    cfg = synth.STEP1024
+    assert synth.EDIT1024.weight_seed == cfg.weight_seed and synth.EDIT1024.hidden == cfg.hidden
+    blocks = []
+    for l in range(cfg.blocks):
+        wts = synth.block_weights(cfg, l)
+        blocks.append(qi.BlockWeights(ctx, wts))
+        del wts
+    dims = qi.dims_struct(cfg.hidden, cfg.heads, cfg.mlp, cfg.patch, cfg.blocks)
+    m = qi.Model(ctx, dims, blocks, synth.model_weights(cfg))
+    yield m
+    del m, blocks
+    torch.cuda.empty_cache()
+
+
+class Run:
+    def __init__(self, ctx, model, cfg):
+        self.ctx, self.model, self.cfg = ctx, model, cfg
+        S, H = cfg.tokens, cfg.hidden
+        gd = [(g.kind, g.tokens, g.grid) for g in cfg.groups]
+        self.groups = qi.groups_struct(list(np.cumsum(cfg.group_sizes())), cfg.group_row_sets())
+        cos, sin = qi.qi_rope_tables(gd)
+        self.cos, self.sin = cuda(cos), cuda(sin)
+        self.ws = torch.empty(qi.qi_step_workspace_bytes(model.dims, S), dtype=torch.uint8,
+                              device="cuda")
+        self.kv = torch.zeros((cfg.blocks, 2, S, H), dtype=torch.bfloat16, device="cuda")
+        self.txt = cuda(synth.text_features(cfg))
+        ref = synth.ref_latents(cfg)
+        self.ref = cuda(ref) if ref is not None else None
+
+    def step(self, lat, sigma, sigma_next, mode):
+        latg = cuda(torch.from_numpy(np.ascontiguousarray(lat)))
+        v = torch.empty_like(latg)
+        cached = mode == qi.QI_KV_READ_PREFIX
+        qi.qi_denoise_step(self.ctx, self.model, latg, None if cached else self.txt,
+                           self.cfg.text_tokens, None if cached else self.ref, self.groups,
+                           self.cos, self.sin, sigma, sigma_next, mode,
+                           None if mode == qi.QI_KV_NONE else self.kv, v, self.ws)
+        self.ctx.check()
+        return latg.cpu().numpy(), v.cpu().numpy()
+
+
+def _check_inputs(cfg, meta):
+    assert meta["inputs"] == input_hashes(cfg), "the seeded inputs changed since the oracle ran"
+
+
+def test_step_1024px_vs_oracle(ctx, model):
+    cfg = synth.STEP1024
+    meta, (ov,) = _golden("step_1024px")
+    _check_inputs(cfg, meta)
+    st = meta["steps"][0]
+    lat0 = synth.latents(cfg).numpy()
+    lat1, v = Run(ctx, model, cfg).step(lat0, st["sigma"], st["sigma_next"], qi.QI_KV_NONE)
+    assert np.all(np.isfinite(v))
+    err = rel_l2(v, ov)
+    assert err <= 2e-2, f"v rel-L2 {err:.3e} after 32 blocks"
+    assert np.array_equal(lat1, O.euler_update(lat0, v, st["sigma"], st["sigma_next"]))
+
+
+def test_edit_1024px_write_then_cached_step_vs_oracle(ctx, model):
+    cfg = synth.EDIT1024
+    meta, (ov1, ov2) = _golden("edit_1024px")
+    _check_inputs(cfg, meta)
+    s1, s2 = meta["steps"]
+    r = Run(ctx, model, cfg)
+    lat0 = synth.latents(cfg).numpy()
+    # first step: every token processed, the text + reference K/V kept
+    lat1, v1 = r.step(lat0, s1["sigma"], s1["sigma_next"], qi.QI_KV_WRITE_PREFIX)
+    err1 = rel_l2(v1, ov1)
+    assert np.all(np.isfinite(v1)) and err1 <= 2e-2, f"step 1 v rel-L2 {err1:.3e}"
+    assert np.array_equal(lat1, O.euler_update(lat0, v1, s1["sigma"], s1["sigma_next"]))
+    # second step from the oracle's step-1 latents: the target rows only,
+    # attending over the cached prefix K/V of the first step
+    olat1 = O.euler_update(lat0, ov1, s1["sigma"], s1["sigma_next"])
+    c2, v2 = r.step(olat1, s2["sigma"], s2["sigma_next"], qi.QI_KV_READ_PREFIX)
+    err2 = rel_l2(v2, ov2)
+    assert np.all(np.isfinite(v2)) and err2 <= 2e-2, f"cached step 2 v rel-L2 {err2:.3e}"
+    assert np.array_equal(c2, O.euler_update(olat1, v2, s2["sigma"], s2["sigma_next"]))
+    # and the uncached second step gives the same latents bit for bit
+    u2, _ = r.step(olat1, s2["sigma"], s2["sigma_next"], qi.QI_KV_NONE)
+    assert np.array_equal(u2, c2)
