@@ -178,9 +178,16 @@ def peaks():
     else:
         pk = {"hbm": 6650.0, "bf16": 1590.0, "bf16_sust": 1400.0, "src": "fallback"}
     if os.path.exists(PEAKS_INT8):
-        d = json.load(open(PEAKS_INT8))["int8_cublaslt"]
+        dd = json.load(open(PEAKS_INT8))
+        d = dd["int8_cublaslt"]
         pk.update({"int8": d["burst_tops"], "int8_sust": d["sustained_tops"],
                    "int8_src": "measured cuBLASLt int8 GEMM 8192^3 (profiles/peaks_int8.json)"})
+        # the tensor pipe's own rate per MHz (back-to-back tcgen05.mma probe),
+        # to put a kernel against the pipe at the clock its run actually held
+        for kind in ("int8", "bf16"):
+            pr = dd.get(f"{kind}_probe")
+            if pr and pr["clocks"].get("sm_mhz"):
+                pk[f"{kind}_pipe_per_mhz"] = pr["sustained_tops"] / pr["clocks"]["sm_mhz"]
     else:
         pk.update({"int8": 2 * pk["bf16"], "int8_sust": 2 * pk["bf16_sust"],
                    "int8_src": f"2 x bf16 {pk['src']} (nominal int8/bf16 ratio)"})
@@ -531,6 +538,12 @@ def run_ours(args, rank, world, local_rank):
         other["attention"] = {"achieved_tflops": a, "peak_tflops": pk["bf16_sust"],
                               "frac": a / pk["bf16_sust"], "frac_of_burst": a / pk["bf16"],
                               "peak_note": f"bf16 dense {pk['src']}"}
+    mhz = (clk or {}).get("sm_mhz")
+    for cls, kind, key in (("gemm_i8", "int8", "achieved_tops"), ("attention", "bf16", "achieved_tflops")):
+        if cls in other and mhz and pk.get(f"{kind}_pipe_per_mhz"):
+            pipe = pk[f"{kind}_pipe_per_mhz"] * mhz
+            other[cls]["tensor_pipe_at_bench_clock"] = pipe
+            other[cls]["frac_of_tensor_pipe_at_bench_clock"] = other[cls][key] / pipe
     # whole step: each class's algorithmic work at its own roofline, summed,
     # against the measured (uninstrumented) step time
     ideal = {

@@ -398,6 +398,24 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const ColTabl
   }
 }
 
+// Tile order of the persistent loops.  Tiles are walked in groups of
+// group_m consecutive M tiles: inside a group M varies fastest, then N; the
+// groups follow each other along M.  The tiles in flight at one time then
+// share a band of A rows and a band of B columns.  group_m = m_tiles is the
+// plain M-fastest order, in which every wave of tiles re-reads all of A: right
+// when A is small enough to stay in L2, wasteful when it is not (the MLP down
+// projection's A is 75 MB at 4608 x 16384).
+__device__ __forceinline__ void tile_coords(int tile, int m_tiles, int group_m, int n_tiles,
+                                            int& mt, int& nt) {
+  const int per_group = group_m * n_tiles;
+  const int g = tile / per_group;
+  const int first = g * group_m;
+  const int gm = min(group_m, m_tiles - first);
+  const int local = tile - g * per_group;
+  mt = first + local % gm;
+  nt = local / gm;
+}
+
 template <bool I8, int BN, int EPI>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -464,8 +482,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       uint32_t phase = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int m0 = (tile % m_tiles) * GEMM_BM;
-        const int n0 = (tile / m_tiles) * BN;
+        int mt, nt;
+        tile_coords(tile, m_tiles, p.group_m, n_tiles, mt, nt);
+        const int m0 = mt * GEMM_BM;
+        const int n0 = nt * BN;
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, p.status)) { ok = false; break; }
           mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
@@ -537,8 +557,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-      const int m0 = (tile % m_tiles) * GEMM_BM;
-      const int n0 = (tile / m_tiles) * BN;
+      int mt, nt;
+      tile_coords(tile, m_tiles, p.group_m, n_tiles, mt, nt);
+      const int m0 = mt * GEMM_BM;
+      const int n0 = nt * BN;
       const ColTable ct{col_sw + acc * BN, col_rs + acc * BN, col_b + acc * BN};
       stage_columns<I8, BN>(p, col_sw + acc * BN, col_rs + acc * BN, col_b + acc * BN, n0,
                             threadIdx.x - 64, &cols_ready[acc]);
@@ -744,8 +766,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       uint32_t phase = 0;
       bool ok = true;
       for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
-        const int m0 = (tile % m_tiles) * (2 * GEMM_BM) + static_cast<int>(rank) * GEMM_BM;
-        const int n0 = (tile / m_tiles) * BN + static_cast<int>(rank) * (BN / 2);
+        int mt, nt;
+        tile_coords(tile, m_tiles, p.group_m, n_tiles, mt, nt);
+        const int m0 = mt * (2 * GEMM_BM) + static_cast<int>(rank) * GEMM_BM;
+        const int n0 = nt * BN + static_cast<int>(rank) * (BN / 2);
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, p.status)) { ok = false; break; }
           const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
@@ -820,8 +844,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = pair; tile < num_tiles; tile += num_pairs) {
-      const int m0 = (tile % m_tiles) * (2 * GEMM_BM) + static_cast<int>(rank) * GEMM_BM;
-      const int n0 = (tile / m_tiles) * BN;
+      int mt, nt;
+      tile_coords(tile, m_tiles, p.group_m, n_tiles, mt, nt);
+      const int m0 = mt * (2 * GEMM_BM) + static_cast<int>(rank) * GEMM_BM;
+      const int n0 = nt * BN;
       const ColTable ct{col_sw + acc * BN, col_rs + acc * BN, col_b + acc * BN};
       stage_columns<true, BN>(p, col_sw + acc * BN, col_rs + acc * BN, col_b + acc * BN, n0,
                               threadIdx.x - 64, &cols_ready[acc]);
@@ -944,6 +970,16 @@ int launch_gemm(bool int8, int epi, const void* A, int lda, const void* B, int l
     max_pairs = max_pairs < num_sms / 2 ? max_pairs : num_sms / 2;
   }
   const bool use_pair = max_pairs > 0;
+  // Tile order: when A (M x K) is too large to stay in L2 next to the B
+  // panels in flight, walk the tiles in two bands of M tiles so that each
+  // wave of tiles reads half of A instead of all of it.
+  GemmParams q = p;
+  {
+    const int bm = use_pair ? 2 * GEMM_BM : GEMM_BM;
+    const int m_tiles = (p.M + bm - 1) / bm;
+    const double a_bytes = static_cast<double>(p.M) * p.K * esz;
+    q.group_m = (a_bytes > 48.0 * (1 << 20) && m_tiles >= 4) ? (m_tiles + 1) / 2 : m_tiles;
+  }
   CUtensorMap ta, tb;
   if (!make_tmap_2d(&ta, A, dt, static_cast<uint64_t>(p.K), static_cast<uint64_t>(p.M),
                     static_cast<uint64_t>(lda) * esz, box_inner, GEMM_BM))
@@ -954,27 +990,27 @@ int launch_gemm(bool int8, int epi, const void* A, int lda, const void* B, int l
     return -2;
   if (use_pair) {
     switch (epi) {
-      case EPI_BF16: return launch_gemm_pair<EPI_BF16>(ta, tb, p, max_pairs, st);
-      case EPI_GELU: return launch_gemm_pair<EPI_GELU>(ta, tb, p, max_pairs, st);
-      case EPI_GATED: return launch_gemm_pair<EPI_GATED>(ta, tb, p, max_pairs, st);
-      case EPI_QKV: return launch_gemm_pair<EPI_QKV>(ta, tb, p, max_pairs, st);
+      case EPI_BF16: return launch_gemm_pair<EPI_BF16>(ta, tb, q, max_pairs, st);
+      case EPI_GELU: return launch_gemm_pair<EPI_GELU>(ta, tb, q, max_pairs, st);
+      case EPI_GATED: return launch_gemm_pair<EPI_GATED>(ta, tb, q, max_pairs, st);
+      case EPI_QKV: return launch_gemm_pair<EPI_QKV>(ta, tb, q, max_pairs, st);
     }
     return -1;
   }
   if (int8) {
     switch (epi) {
-      case EPI_BF16: return launch_gemm_bn<true, EPI_BF16>(bn, ta, tb, p, num_sms, st);
-      case EPI_GELU: return launch_gemm_bn<true, EPI_GELU>(bn, ta, tb, p, num_sms, st);
-      case EPI_GATED: return launch_gemm_bn<true, EPI_GATED>(bn, ta, tb, p, num_sms, st);
+      case EPI_BF16: return launch_gemm_bn<true, EPI_BF16>(bn, ta, tb, q, num_sms, st);
+      case EPI_GELU: return launch_gemm_bn<true, EPI_GELU>(bn, ta, tb, q, num_sms, st);
+      case EPI_GATED: return launch_gemm_bn<true, EPI_GATED>(bn, ta, tb, q, num_sms, st);
       case EPI_QKV:   // each epilogue half-tile must hold a whole head of one of q, k, v
-        if (bn == 256 && p.H % 256 == 0) return launch_gemm_t<true, 256, EPI_QKV>(ta, tb, p, num_sms, st);
+        if (bn == 256 && p.H % 256 == 0) return launch_gemm_t<true, 256, EPI_QKV>(ta, tb, q, num_sms, st);
         return -1;
     }
   } else {
     switch (epi) {
-      case EPI_BF16: return launch_gemm_bn<false, EPI_BF16>(bn, ta, tb, p, num_sms, st);
-      case EPI_F32: return launch_gemm_bn<false, EPI_F32>(bn, ta, tb, p, num_sms, st);
-      case EPI_EULER: return launch_gemm_bn<false, EPI_EULER>(bn, ta, tb, p, num_sms, st);
+      case EPI_BF16: return launch_gemm_bn<false, EPI_BF16>(bn, ta, tb, q, num_sms, st);
+      case EPI_F32: return launch_gemm_bn<false, EPI_F32>(bn, ta, tb, q, num_sms, st);
+      case EPI_EULER: return launch_gemm_bn<false, EPI_EULER>(bn, ta, tb, q, num_sms, st);
     }
   }
   return -1;

@@ -104,6 +104,7 @@ struct GemmParams {
   uint8_t* v8_out2;
   int ldo;
   uint32_t* row_range;    // GELU: optional per-row [-min, max] bit patterns of the bf16 output
+  int group_m;            // tile order: bands of group_m M tiles (set by launch_gemm)
   int* status;            // device status word
 };
 

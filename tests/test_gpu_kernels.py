@@ -77,7 +77,9 @@ def test_empty_inputs_are_noops(ctx):
     zp = torch.full((4,), 5, dtype=torch.int32, device="cuda")
     qi.qi_quantize_act(ctx, x[:0], out=(q[:0], s[:0], zp[:0]))
     y = torch.full((4, 64), 3.0, dtype=torch.bfloat16, device="cuda")
-    qi.qi_w8a8_linear(ctx, q[:0], s[:0], zp[:0], qi.qi_w8(), y=y[:0])
+    wq = torch.zeros((64, 256), dtype=torch.int8, device="cuda")
+    w = qi.w8_struct(wq, torch.ones(64, device="cuda"), torch.zeros(64, dtype=torch.int32, device="cuda"))
+    qi.qi_w8a8_linear(ctx, q[:0], s[:0], zp[:0], w, y=y[:0])
     H, S = 256, 40
     qkv = cuda(_bf16((3, S, H), 4, 1.0))
     o = torch.full((S, H), 1.5, dtype=torch.bfloat16, device="cuda")

@@ -113,7 +113,8 @@ def _tie_rows(dtype):
     u / s, or within a few ulps of one."""
     rows = []
     # power-of-two scale: lo = -8, hi = 127/16 -> s = 1/16, zp = 0; u = (k + 1/2)/16
-    k = np.arange(-128, 127)
+    # for |k + 1/2| < 127 (both signs stay inside [lo, hi])
+    k = np.arange(-127, 127)
     ties = ((k + 0.5) / 16).astype(F32)
     rows.append(np.concatenate([[-8.0, 127 / 16], ties, -ties[::-1]]).astype(F32))
     if dtype == "f32":
@@ -151,5 +152,5 @@ def test_quantizer_rounding_ties(ctx, dtype):
     assert np.array_equal(q.cpu().numpy(), oq)
     # the power-of-two row: ties go to the even code
     assert s.cpu().numpy()[0] == F32(1 / 16) and zp.cpu().numpy()[0] == 0
-    codes = q.cpu().numpy()[0, 2:2 + 255].astype(np.int64)
+    codes = q.cpu().numpy()[0, 2:2 + 2 * 254].astype(np.int64)
     assert np.all(codes % 2 == 0)
