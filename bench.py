@@ -54,7 +54,15 @@ def algorithmic_work(cfg: synth.DitConfig, cached: bool = False):
         return out
     H, F, d, h = cfg.hidden, cfg.mlp, cfg.head_dim, cfg.heads
     rows = cfg.target_tokens if cached else cfg.tokens
-    per_block_ops = 2 * rows * (3 * H * H + H * H + F * H + H * F)
+    # 2 x rows x (weights) of each block Linear, split by its precision
+    sizes = {"qk": 2 * H * H, "v": H * H, "out": H * H, "up": F * H, "down": H * F}
+    i8_ops = bf16_block = 0
+    for l in range(cfg.blocks):
+        for name, kind in synth.linear_precision(cfg, l).items():
+            if kind == "w8":
+                i8_ops += 2 * rows * sizes[name]
+            else:
+                bf16_block += 2 * rows * sizes[name]
     ends = np.cumsum(cfg.group_sizes())
     starts = np.concatenate([[0], ends[:-1]])
     if cached:
@@ -69,7 +77,17 @@ def algorithmic_work(cfg: synth.DitConfig, cached: bool = False):
     # the GELU-output quantizer reads 2F and writes F.  Plus 8 bytes (scale,
     # zero point) per row and quantizer, and the final LayerNorm (4H in, 2H out
     # per target row).
-    quant = cfg.blocks * rows * (19 * H + 3 * F + 32) + cfg.target_tokens * 6 * H
+    quant = cfg.target_tokens * 6 * H
+    for l in range(cfg.blocks):
+        pr = synth.linear_precision(cfg, l)
+        w8 = {k: v == "w8" for k, v in pr.items()}
+        b = 4 * H                                             # LN1 reads the fp32 residual
+        b += (H + 8) if w8["qk"] else 0                       # ... writes codes for W8A8 q, k
+        b += 2 * H if not (w8["qk"] and w8["v"]) else 0       # ... and bf16 u for a BF16 part
+        b += (3 * H + 8) if w8["out"] else 0                  # attention-output quantizer
+        b += 10 * H + ((H + 8) if w8["up"] else 2 * H)        # LN2 with the residual add
+        b += (3 * F + 8) if w8["down"] else 0                 # GELU-output quantizer
+        quant += rows * b
     # GEMV weight bytes: the adaLN rows of every block (6H x H bf16), the final
     # adaLN (2H x H) and the timestep MLP (H x 256 + H x H)
     gemv = 2 * (cfg.blocks * 6 * H * H + 2 * H * H + H * 256 + H * H)
@@ -79,8 +97,9 @@ def algorithmic_work(cfg: synth.DitConfig, cached: bool = False):
     bf16 = 2 * N * P * H * 2
     if not cached:
         bf16 += 2 * cfg.text_tokens * H * H + 2 * (cfg.prefix_tokens - cfg.text_tokens) * P * H
+    bf16 += bf16_block
     return {
-        "gemm_i8_ops_per_step": cfg.blocks * per_block_ops,
+        "gemm_i8_ops_per_step": i8_ops,
         "attn_flops_per_step": cfg.blocks * attn_flops,
         "attn_pairs_per_head": pairs,
         "quant_bytes_per_step": quant,
@@ -154,7 +173,8 @@ def build_model(ctx, qi, cfg, device):
     blocks = []
     for l in range(cfg.blocks):
         wts = synth.block_weights(cfg, l, device=device)
-        blocks.append(qi.BlockWeights(ctx, wts, device=device))
+        blocks.append(qi.BlockWeights(ctx, wts, device=device,
+                                      precision=synth.linear_precision(cfg, l)))
         del wts
     glob = synth.model_weights(cfg, device=device)
     dims = qi.dims_struct(cfg.hidden, cfg.heads, cfg.mlp, cfg.patch, cfg.blocks)
@@ -340,7 +360,7 @@ def aggregate_throughput(world: int, steps: int, max_ms: float) -> float:
 # ------------------------------------------------------------------ GPU arm
 
 WORKLOADS = {c.name: c for c in (synth.STEP1024, synth.EDIT1024, synth.EDIT3REF1024, synth.CFG1024,
-                                  synth.GEN2048, synth.GEN2048_SCHED)}
+                                  synth.GEN2048, synth.GEN2048_SCHED, synth.STEP1024_PAGES)}
 
 
 def run_ours(args, rank, world, local_rank):
@@ -573,7 +593,10 @@ def run_ours(args, rank, world, local_rank):
                f"(scale {cfg.guidance}), " if cfg.uncond_text else "")
             + ("40-step FlowMatch Euler denoise, prefix K/V cached from step 2"
                if denoise else "uncached step")
-            + ", all attn/MLP Linears W8A8 (int8 GEMMs), "
+            + (", all attn/MLP Linears W8A8 (int8 GEMMs), " if cfg.precision == "w8a8" else
+               ", the pages' precision layout (W8A8 q, k, MLP up/down in blocks 2-29 on int8 "
+               "GEMMs; v, out projection and all Linears of blocks 0, 1, 30, 31 in BF16 on "
+               "bf16 GEMMs), ")
             + (f"bf16 attention in steps 1-{cfg.fp8_from_step - 1} and fp8 (e4m3) attention from "
                f"step {cfg.fp8_from_step}" if cfg.fp8_from_step else "bf16 attention"))
     out = {
@@ -807,7 +830,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", choices=tuple(WORKLOADS), default=synth.STEP1024.name,
                     help="step_1024px (default): one uncached 1024^2 step per iteration, plus "
-                         "a cached-prefix measurement; edit_1024px: the edit sequence; "
+                         "a cached-prefix measurement; step_1024px_pagesmask: the same step with "
+                         "the pages' W8A8/BF16 layout; edit_1024px: the edit sequence; "
                          "edit_3ref_1024px: an edit with three reference images; "
                          "cfg_1024px: true classifier-free guidance (prompt + negative prompt "
                          "as one batch); "

@@ -278,6 +278,7 @@ struct QuantExtras {
   uint32_t* zero_range = nullptr;      // LN: clear these row ranges
   const uint32_t* range = nullptr;     // plain: producer-published row ranges
   float* u_f32 = nullptr;              // LN: also write the quantized value u (fp32 tap)
+  bool quant_too = false;              // LN with u_bf16: quantize as well as write bf16(u)
 };
 
 // Stream-ordered device copy of a tap (skipped when the tap is NULL).
@@ -308,6 +309,7 @@ int run_quant(qi_ctx* ctx, const void* x, bool xbf16, int M, int K, int ldx,
   p.zero_range = ex.zero_range;
   p.range = ex.range;
   p.u_f32 = ex.u_f32;
+  p.quant_too = ex.quant_too ? 1 : 0;
   p.x = x;
   p.x_bf16 = xbf16 ? 1 : 0;
   p.M = M;
@@ -397,10 +399,51 @@ struct SeqAttn {
   uint16_t* vl;
 };
 
+// Which Linears of a block are W8A8 and which BF16 (qi_block_weights).
+struct BlockPrecision {
+  int qkv_w8_cols;   // columns of q | k | v computed by the W8A8 GEMM: 3H, 2H (v BF16) or 0
+  bool out_w8, up_w8, down_w8;
+};
+
+BlockPrecision block_precision(const qi_dims& d, const qi_block_weights& w) {
+  BlockPrecision bp;
+  bp.qkv_w8_cols = w.qkv.q ? w.qkv.n : 0;
+  bp.out_w8 = w.out.q != nullptr;
+  bp.up_w8 = w.up.q != nullptr;
+  bp.down_w8 = w.down.q != nullptr;
+  (void)d;
+  return bp;
+}
+
+// A BF16 block Linear on tcgen05 kind::f16 (CTA pairs for 256-wide tiles)
+// with one of the block epilogues; `p` carries the epilogue fields.
+int run_bf16_block_linear(qi_ctx* ctx, const uint16_t* a, int M, int lda, const qi_linear_bf16& w,
+                          int epi, qi::GemmParams p, cudaStream_t st) {
+  if (M == 0) return QI_OK;
+  p.M = M;
+  p.N = w.n;
+  p.K = w.k;
+  p.num_kb = w.k / 64;
+  p.s_a = nullptr;
+  p.zp_a = nullptr;
+  p.s_w = nullptr;
+  p.rowsum = nullptr;
+  p.bias = w.bias;
+  p.status = ctx->status;
+  Prof pr(ctx, QI_KCLASS_GEMM_BF16, st);
+  const int r = qi::launch_gemm(false, epi, a, lda, w.w, w.k, p, ctx->num_sms, st);
+  if (r == -2) return fail(QI_ERR_CUDA, "cuTensorMapEncodeTiled failed (BF16 block Linear)");
+  if (r != 0) return cuda_fail("BF16 block Linear launch");
+  return QI_OK;
+}
+
 // One block over the processed rows of up to two sequences (a true-CFG batch):
 // every Linear, quantizer and norm runs once over all T rows (rows_gt maps a
 // row, offset by rows_row0, to its modulation row set; cs/sn hold the RoPE
-// tables of the T rows); attention runs per sequence.
+// tables of the T rows); attention runs per sequence.  Each Linear is W8A8 or
+// BF16 as the weights say; a BF16 Linear reads the bf16 activation (for the
+// LayerNorm values, the LN kernel writes it into the attention-output buffer,
+// which is free at that point).
 int run_block_multi(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, float* x, int T,
                     const qi::GroupTable& rows_gt, int rows_row0, const uint16_t* mod,
                     const float* cs, const float* sn, const SeqAttn* seqs, int nseq, uint8_t* ws,
@@ -410,34 +453,31 @@ int run_block_multi(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, fl
   const int row0 = rows_row0;
   Carve c{ws, ws_bytes, 0};
   BlockBufs b = carve_block(c, d, T);
+  const BlockPrecision bp = block_precision(d, w);
   const int mld = 6 * H;
   int r;
-  // attention half.  LN1 + modulate + quantize; it also clears the row
-  // ranges that the attention epilogue will publish for the next quantizer.
+  // attention half.  LN1 + modulate + quantize (and/or the bf16 value for a
+  // BF16 q | k | v part); it also clears the row ranges that the attention
+  // epilogue will publish for the next quantizer.
   const qi_block_taps* tp = ctx->taps_on ? &ctx->taps : nullptr;
+  const bool qkv_bf16 = bp.qkv_w8_cols < 3 * H;
   {
     QuantExtras ex;
     ex.zero_range = b.o_range;
     ex.u_f32 = tp ? tp->u1 : nullptr;
+    ex.quant_too = bp.qkv_w8_cols > 0;
     if ((r = run_quant(ctx, x, false, T, H, H, mod + 0 * H, mod + 1 * H, mld, gt, row0, d.eps,
-                       b.uq, b.sa, b.zp, nullptr, st, ex)))
+                       b.uq, b.sa, b.zp, qkv_bf16 ? b.o : nullptr, st, ex)))
       return r;
-    if (tp && (r = tap_codes(tp->q1, tp->s1, tp->zp1, b.uq, b.sa, b.zp, T, H, st))) return r;
+    if (tp && bp.qkv_w8_cols > 0 &&
+        (r = tap_codes(tp->q1, tp->s1, tp->zp1, b.uq, b.sa, b.zp, T, H, st)))
+      return r;
   }
   // QKV projection with Q/K RMSNorm + RoPE fused into its epilogue: q goes to
   // the block's q buffer, k and v straight into this layer's K/V rows.
   {
     qi::GemmParams p;
     memset(&p, 0, sizeof(p));
-    p.M = T;
-    p.N = w.qkv.n;
-    p.K = w.qkv.k;
-    p.num_kb = w.qkv.k / 128;
-    p.s_a = b.sa;
-    p.zp_a = b.zp;
-    p.s_w = w.qkv.s;
-    p.rowsum = w.qkv.rowsum;
-    p.bias = w.qkv.bias;
     p.H = H;
     p.eps = d.eps;
     p.wq = w.norm_q;
@@ -467,11 +507,28 @@ int run_block_multi(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, fl
     }
     p.ldo = H;
     p.status = ctx->status;
-    Prof pr(ctx, QI_KCLASS_GEMM_I8, st);
-    const int rr = qi::launch_gemm(true, qi::EPI_QKV, b.uq, w.qkv.k, w.qkv.q, w.qkv.k, p,
-                                   ctx->num_sms, st);
-    if (rr == -2) return fail(QI_ERR_CUDA, "cuTensorMapEncodeTiled failed (QKV operands)");
-    if (rr != 0) return cuda_fail("QKV GEMM launch");
+    if (bp.qkv_w8_cols > 0) {
+      qi::GemmParams pw = p;
+      pw.M = T;
+      pw.N = w.qkv.n;
+      pw.K = w.qkv.k;
+      pw.num_kb = w.qkv.k / 128;
+      pw.s_a = b.sa;
+      pw.zp_a = b.zp;
+      pw.s_w = w.qkv.s;
+      pw.rowsum = w.qkv.rowsum;
+      pw.bias = w.qkv.bias;
+      pw.n_base = 0;
+      Prof pr(ctx, QI_KCLASS_GEMM_I8, st);
+      const int rr = qi::launch_gemm(true, qi::EPI_QKV, b.uq, w.qkv.k, w.qkv.q, w.qkv.k, pw,
+                                     ctx->num_sms, st);
+      if (rr == -2) return fail(QI_ERR_CUDA, "cuTensorMapEncodeTiled failed (QKV operands)");
+      if (rr != 0) return cuda_fail("QKV GEMM launch");
+    }
+    if (qkv_bf16) {
+      p.n_base = bp.qkv_w8_cols;   // the v rows (2H) or all of q | k | v (0)
+      if ((r = run_bf16_block_linear(ctx, b.o, T, H, w.qkv_bf16, qi::EPI_QKV, p, st))) return r;
+    }
   }
   if (f8) {
     // fp8 attention: the QKV epilogue wrote e4m3 q and the e4m3 K/V rows it
@@ -521,7 +578,7 @@ int run_block_multi(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, fl
     ap.q_offset = q.row0;
     ap.sm_scale = 1.0f / sqrtf(static_cast<float>(d.head_dim));
     ap.groups = q.gt;
-    ap.row_range = b.o_range + 2 * static_cast<size_t>(q.off);
+    ap.row_range = bp.out_w8 ? b.o_range + 2 * static_cast<size_t>(q.off) : nullptr;
     ap.status = ctx->status;
     Prof pr(ctx, QI_KCLASS_ATTN, st);
     const int r2 = qi::launch_attention(ap, st);
@@ -529,53 +586,87 @@ int run_block_multi(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, fl
     if (r2 != 0) return cuda_fail("attention launch");
   }
   if (tp && ((r = tap_copy(tp->o, b.o, static_cast<size_t>(T) * H * 2, st)) ||
-             (r = tap_copy(tp->o_range, b.o_range, static_cast<size_t>(T) * 8, st))))
+             (bp.out_w8 && (r = tap_copy(tp->o_range, b.o_range, static_cast<size_t>(T) * 8, st)))))
     return r;
-  {
-    QuantExtras ex;   // the attention epilogue published each row's range
-    ex.range = b.o_range;
-    if ((r = run_quant(ctx, b.o, true, T, H, H, nullptr, nullptr, 0, gt, row0, d.eps, b.uq, b.sa,
-                       b.zp, nullptr, st, ex)))
+  // output projection stored as bf16 into the q buffer (consumed by the
+  // attention); its gated residual is applied by the LN2 kernel below, which
+  // reads the residual stream anyway
+  uint16_t* y_out = b.q;
+  if (bp.out_w8) {
+    {
+      QuantExtras ex;   // the attention epilogue published each row's range
+      ex.range = b.o_range;
+      if ((r = run_quant(ctx, b.o, true, T, H, H, nullptr, nullptr, 0, gt, row0, d.eps, b.uq,
+                         b.sa, b.zp, nullptr, st, ex)))
+        return r;
+      if (tp && (r = tap_codes(tp->qo, tp->so, tp->zpo, b.uq, b.sa, b.zp, T, H, st))) return r;
+    }
+    if ((r = run_w8a8(ctx, b.uq, b.sa, b.zp, T, w.out, qi::EPI_BF16, y_out, H, nullptr, 0, nullptr,
+                      0, gt, row0, nullptr, st)))
       return r;
-    if (tp && (r = tap_codes(tp->qo, tp->so, tp->zpo, b.uq, b.sa, b.zp, T, H, st))) return r;
+  } else {
+    qi::GemmParams p;
+    memset(&p, 0, sizeof(p));
+    p.y = y_out;
+    p.ldy = H;
+    if ((r = run_bf16_block_linear(ctx, b.o, T, H, w.out_bf16, qi::EPI_BF16, p, st))) return r;
   }
-  // output projection stored as bf16 (into the attention output's buffer,
-  // already consumed); its gated residual is applied by the LN2 kernel below,
-  // which reads the residual stream anyway
-  if ((r = run_w8a8(ctx, b.uq, b.sa, b.zp, T, w.out, qi::EPI_BF16, b.o, H, nullptr, 0, nullptr, 0,
-                    gt, row0, nullptr, st)))
-    return r;
-  // MLP half: x += gate1 * out, LN2 + modulate + quantize; clears the GELU ranges
+  // MLP half: x += gate1 * out, LN2 + modulate + quantize (and/or the bf16
+  // value for a BF16 up projection, into the attention-output buffer, now
+  // consumed); clears the GELU ranges
   {
     QuantExtras ex;
-    ex.res_y = b.o;
+    ex.res_y = y_out;
     ex.res_gate = mod + 2 * H;
     ex.zero_range = b.g_range;
     ex.u_f32 = tp ? tp->u2 : nullptr;
+    ex.quant_too = bp.up_w8;
     if ((r = run_quant(ctx, x, false, T, H, H, mod + 3 * H, mod + 4 * H, mld, gt, row0, d.eps,
-                       b.uq, b.sa, b.zp, nullptr, st, ex)))
+                       b.uq, b.sa, b.zp, bp.up_w8 ? nullptr : b.o, st, ex)))
       return r;
     if (tp && ((r = tap_copy(tp->x_mid, x, static_cast<size_t>(T) * H * 4, st)) ||
-               (r = tap_codes(tp->q2, tp->s2, tp->zp2, b.uq, b.sa, b.zp, T, H, st))))
+               (bp.up_w8 && (r = tap_codes(tp->q2, tp->s2, tp->zp2, b.uq, b.sa, b.zp, T, H, st)))))
       return r;
   }
-  if ((r = run_w8a8(ctx, b.uq, b.sa, b.zp, T, w.up, qi::EPI_GELU, b.g, F, nullptr, 0, nullptr, 0,
-                    gt, row0, nullptr, st, b.g_range)))
-    return r;
+  uint32_t* g_range = bp.down_w8 ? b.g_range : nullptr;
+  if (bp.up_w8) {
+    if ((r = run_w8a8(ctx, b.uq, b.sa, b.zp, T, w.up, qi::EPI_GELU, b.g, F, nullptr, 0, nullptr, 0,
+                      gt, row0, nullptr, st, g_range)))
+      return r;
+  } else {
+    qi::GemmParams p;
+    memset(&p, 0, sizeof(p));
+    p.y = b.g;
+    p.ldy = F;
+    p.row_range = g_range;
+    if ((r = run_bf16_block_linear(ctx, b.o, T, H, w.up_bf16, qi::EPI_GELU, p, st))) return r;
+  }
   if (tp && ((r = tap_copy(tp->g, b.g, static_cast<size_t>(T) * F * 2, st)) ||
-             (r = tap_copy(tp->g_range, b.g_range, static_cast<size_t>(T) * 8, st))))
+             (bp.down_w8 && (r = tap_copy(tp->g_range, b.g_range, static_cast<size_t>(T) * 8, st)))))
     return r;
-  {
-    QuantExtras ex;   // the GELU epilogue published each row's range
-    ex.range = b.g_range;
-    if ((r = run_quant(ctx, b.g, true, T, F, F, nullptr, nullptr, 0, gt, row0, d.eps, b.uq, b.sa,
-                       b.zp, nullptr, st, ex)))
+  if (bp.down_w8) {
+    {
+      QuantExtras ex;   // the GELU epilogue published each row's range
+      ex.range = b.g_range;
+      if ((r = run_quant(ctx, b.g, true, T, F, F, nullptr, nullptr, 0, gt, row0, d.eps, b.uq,
+                         b.sa, b.zp, nullptr, st, ex)))
+        return r;
+      if (tp && (r = tap_codes(tp->qg, tp->sg, tp->zpg, b.uq, b.sa, b.zp, T, F, st))) return r;
+    }
+    if ((r = run_w8a8(ctx, b.uq, b.sa, b.zp, T, w.down, qi::EPI_GATED, nullptr, 0, x, H,
+                      mod + 5 * H, mld, gt, row0, nullptr, st)))
       return r;
-    if (tp && (r = tap_codes(tp->qg, tp->sg, tp->zpg, b.uq, b.sa, b.zp, T, F, st))) return r;
+  } else {
+    qi::GemmParams p;
+    memset(&p, 0, sizeof(p));
+    p.yf = x;
+    p.ldyf = H;
+    p.gate = mod + 5 * H;
+    p.gate_ld = mld;
+    p.groups = gt;
+    p.row0 = row0;
+    if ((r = run_bf16_block_linear(ctx, b.g, T, F, w.down_bf16, qi::EPI_GATED, p, st))) return r;
   }
-  if ((r = run_w8a8(ctx, b.uq, b.sa, b.zp, T, w.down, qi::EPI_GATED, nullptr, 0, x, H,
-                    mod + 5 * H, mld, gt, row0, nullptr, st)))
-    return r;
   return QI_OK;
 }
 
@@ -594,14 +685,30 @@ int run_block(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, float* x
   return run_block_multi(ctx, d, w, x, T, gt, row0, mod, cs, sn, &one, 1, ws, ws_bytes, st, f8);
 }
 
+// A block Linear given either as W8A8 codes or as a BF16 weight.
+int check_linear(const qi_w8* w8, const qi_linear_bf16* bf, const char* name, int n, int k) {
+  if (w8->q) return check_w8(w8, name, n, k);
+  int r;
+  if ((r = check_bf16_linear(bf, name, n, k))) return r;
+  if (k % 64 != 0) return fail(QI_ERR_UNSUPPORTED_SHAPE, "BF16 weight %s: k %% 64 != 0", name);
+  return QI_OK;
+}
+
 int check_block_weights(const qi_dims& d, const qi_block_weights* w) {
   if (!w) return fail(QI_ERR_INVALID_ARG, "block weights are NULL");
   const int H = d.hidden, F = d.mlp;
   int r;
-  if ((r = check_w8(&w->qkv, "qkv", 3 * H, H))) return r;
-  if ((r = check_w8(&w->out, "out", H, H))) return r;
-  if ((r = check_w8(&w->up, "up", F, H))) return r;
-  if ((r = check_w8(&w->down, "down", H, F))) return r;
+  if (!w->qkv.q) {
+    if ((r = check_linear(&w->qkv, &w->qkv_bf16, "qkv", 3 * H, H))) return r;
+  } else if (w->qkv.n == 2 * H) {   // q, k W8A8; v BF16
+    if ((r = check_w8(&w->qkv, "qkv (q, k rows)", 2 * H, H))) return r;
+    if ((r = check_bf16_linear(&w->qkv_bf16, "qkv_bf16 (v rows)", H, H))) return r;
+  } else if ((r = check_w8(&w->qkv, "qkv", 3 * H, H))) {
+    return r;
+  }
+  if ((r = check_linear(&w->out, &w->out_bf16, "out", H, H))) return r;
+  if ((r = check_linear(&w->up, &w->up_bf16, "up", F, H))) return r;
+  if ((r = check_linear(&w->down, &w->down_bf16, "down", H, F))) return r;
   if (!w->norm_q || !w->norm_k) return fail(QI_ERR_INVALID_ARG, "norm_q / norm_k is NULL");
   if (!aligned16(w->norm_q) || !aligned16(w->norm_k))
     return fail(QI_ERR_ALIGNMENT, "norm_q / norm_k must be 16-byte aligned");

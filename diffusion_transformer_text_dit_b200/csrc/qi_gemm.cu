@@ -92,11 +92,12 @@ __device__ __forceinline__ void dequant32(const ColTable& t, const uint32_t (&r)
   }
 }
 
-// W8A8 dequantization of 32 accumulator columns rounded to bf16 (the
-// Linear's output dtype).
+// 32 accumulator columns dequantized (W8A8) or biased (BF16) and rounded to
+// bf16 (the Linear's output dtype).
+template <bool I8>
 __device__ __forceinline__ void dequant32_bf16(const ColTable& t, const uint32_t (&r)[32], int c0,
                                                float sa, int32_t zp, float (&y)[32]) {
-  dequant32<true>(t, r, c0, sa, zp, y);
+  dequant32<I8>(t, r, c0, sa, zp, y);
 #pragma unroll
   for (int j = 0; j < 32; ++j) y[j] = bf16_round_f(y[j]);
 }
@@ -163,12 +164,15 @@ __device__ __forceinline__ void store_e4m3_32(uint8_t* dst, const uint32_t (&pk)
 // with explicitly rounded fp32 operations; v is stored as bf16(y).  For fp8
 // attention each stored bf16 row is also written as e4m3 (the value a
 // separate cast of the bf16 tensor gives).
-template <int W, bool PAIR>
+template <bool I8, int W, bool PAIR>
 __device__ __forceinline__ void qkv_epilogue(const GemmParams& p, const ColTable& ct, int cb,
                                              uint32_t t_row, int m, bool row_ok, float sa,
                                              int32_t zp, int n0, int lane, uint32_t tempty_addr) {
-  const int which = n0 / p.H;
-  const int col0 = n0 - which * p.H;
+  // column n of this GEMM is column n_base + n of the q | k | v projection
+  // (a GEMM may cover only part of it: the W8A8 q, k rows and a BF16 v)
+  const int gn = n0 + p.n_base;
+  const int which = gn / p.H;
+  const int col0 = gn - which * p.H;
   // q rows are contiguous; K/V rows of a second sequence go to its own buffer
   const bool second = which > 0 && p.k_out2 != nullptr && m >= p.kv_split;
   const int mo = second ? m - p.kv_split : m;
@@ -199,7 +203,7 @@ __device__ __forceinline__ void qkv_epilogue(const GemmParams& p, const ColTable
         }
         if (!row_ok) continue;
         float y[32];
-        dequant32_bf16(ct, r, cb + hh * 128 + c * 32, sa, zp, y);
+        dequant32_bf16<I8>(ct, r, cb + hh * 128 + c * 32, sa, zp, y);
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(y[2 * i], y[2 * i + 1]);
@@ -224,7 +228,7 @@ __device__ __forceinline__ void qkv_epilogue(const GemmParams& p, const ColTable
       }
       if (row_ok) {
         float y[32];
-        dequant32_bf16(ct, r, cb + hh * 128 + c * 32, sa, zp, y);
+        dequant32_bf16<I8>(ct, r, cb + hh * 128 + c * 32, sa, zp, y);
 #pragma unroll
         for (int j = 0; j < 32; ++j) ss = __fadd_rn(ss, __fmul_rn(y[j], y[j]));
 #pragma unroll
@@ -288,7 +292,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const ColTabl
   }
   const uint32_t t_row = tmem_acc + (static_cast<uint32_t>(quarter * 32) << 16);
   if constexpr (EPI == EPI_QKV) {
-    qkv_epilogue<BN / 2, PAIR>(p, ct, half * (BN / 2), t_row + half * (BN / 2), m, row_ok, sa,
+    qkv_epilogue<I8, BN / 2, PAIR>(p, ct, half * (BN / 2), t_row + half * (BN / 2), m, row_ok, sa,
                                zp, n0 + half * (BN / 2), lane, tempty_addr);
     return;
   }
@@ -675,6 +679,15 @@ __device__ __forceinline__ void umma_i8_pair(uint32_t d_tmem, uint64_t a, uint64
       "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
 }
 
+__device__ __forceinline__ void umma_f16_pair(uint32_t d_tmem, uint64_t a, uint64_t b,
+                                              uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
+}
+
 // Arrive on the barrier at this offset in every CTA of `mask` once all MMAs
 // issued so far by this thread have completed.
 __device__ __forceinline__ void umma_commit_pair(uint64_t* bar, uint16_t mask) {
@@ -699,7 +712,7 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols
   asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols));
 }
 
-template <int EPI>
+template <bool I8, int EPI>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const GemmParams p) {
@@ -774,8 +787,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           if (!mbar_wait(&empty[stage], phase ^ 1u, p.status)) { ok = false; break; }
           const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
           if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * PAIR_STAGE_BYTES);
-          tma_load_2d_pair(&tmA, fb, sA + stage * PAIR_A_BYTES, kb * GEMM_BK_BYTES, m0);
-          tma_load_2d_pair(&tmB, fb, sB + stage * PAIR_B_BYTES, kb * GEMM_BK_BYTES, n0);
+          // one 128-byte K row per stage: 128 int8 or 64 bf16 elements
+          tma_load_2d_pair(&tmA, fb, sA + stage * PAIR_A_BYTES, kb * (I8 ? 128 : 64), m0);
+          tma_load_2d_pair(&tmB, fb, sB + stage * PAIR_B_BYTES, kb * (I8 ? 128 : 64), n0);
           if (++stage == PAIR_STAGES) { stage = 0; phase ^= 1u; }
         }
       }
@@ -801,7 +815,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (even CTA)
     if (lane == 0 && rank == 0) {
-      constexpr uint32_t idesc = umma_idesc(true, 2 * GEMM_BM, BN);
+      constexpr uint32_t idesc = umma_idesc(I8, 2 * GEMM_BM, BN);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -819,7 +833,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 #pragma unroll
           for (int k = 0; k < 4; ++k) {   // 4 x 32 bytes of K per stage
             const uint64_t off = static_cast<uint64_t>(k * 32) >> 4;
-            umma_i8_pair(d_tmem, adesc + off, bdesc + off, idesc, (kb | k) != 0);
+            if (I8)
+              umma_i8_pair(d_tmem, adesc + off, bdesc + off, idesc, (kb | k) != 0);
+            else
+              umma_f16_pair(d_tmem, adesc + off, bdesc + off, idesc, (kb | k) != 0);
           }
           umma_commit_pair(&empty[stage], 0x3);
           if (++stage == PAIR_STAGES) { stage = 0; phase ^= 1u; }
@@ -849,12 +866,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       const int m0 = mt * (2 * GEMM_BM) + static_cast<int>(rank) * GEMM_BM;
       const int n0 = nt * BN;
       const ColTable ct{col_sw + acc * BN, col_rs + acc * BN, col_b + acc * BN};
-      stage_columns<true, BN>(p, col_sw + acc * BN, col_rs + acc * BN, col_b + acc * BN, n0,
-                              threadIdx.x - 64, &cols_ready[acc]);
+      stage_columns<I8, BN>(p, col_sw + acc * BN, col_rs + acc * BN, col_b + acc * BN, n0,
+                            threadIdx.x - 64, &cols_ready[acc]);
       if (!mbar_wait_warp(&cols_ready[acc], acc_phase, p.status)) break;
       if (!mbar_wait_warp(&tfull[acc], acc_phase, p.status)) break;
       tc_fence_after();
-      epilogue_tile<true, BN, EPI, true>(p, ct, tmem_base + static_cast<uint32_t>(acc * BN), m0, n0,
+      epilogue_tile<I8, BN, EPI, true>(p, ct, tmem_base + static_cast<uint32_t>(acc * BN), m0, n0,
                                          quarter, half, lane, mapa_shared(smem_u32(&tempty[acc]), 0));
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
@@ -894,11 +911,11 @@ static int launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const Gem
 
 
 // Clusters of two that can be resident at once (0 if the pair kernel cannot run).
-template <int EPI>
+template <bool I8, int EPI>
 static int pair_capacity() {
   static int cap = -1;   // per instantiation
   if (cap < 0) {
-    auto kern = gemm_pair_kernel<EPI>;
+    auto kern = gemm_pair_kernel<I8, EPI>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PAIR_SMEM_BYTES) != cudaSuccess) {
       launch_result();
       return cap = 0;
@@ -924,12 +941,12 @@ static int pair_capacity() {
   return cap;
 }
 
-template <int EPI>
+template <bool I8, int EPI>
 static int launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
                             int max_pairs, cudaStream_t st) {
   const int tiles = ((p.M + 2 * GEMM_BM - 1) / (2 * GEMM_BM)) * ((p.N + 255) / 256);
   const int pairs = tiles < max_pairs ? tiles : max_pairs;
-  launch_pdl(gemm_pair_kernel<EPI>, dim3(2 * pairs), dim3(GEMM_THREADS), PAIR_SMEM_BYTES, st, 2, ta, tb, p);
+  launch_pdl(gemm_pair_kernel<I8, EPI>, dim3(2 * pairs), dim3(GEMM_THREADS), PAIR_SMEM_BYTES, st, 2, ta, tb, p);
   return launch_result();
 }
 
@@ -957,15 +974,24 @@ int launch_gemm(bool int8, int epi, const void* A, int lda, const void* B, int l
       int8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const int esz = int8 ? 1 : 2;
   const uint32_t box_inner = GEMM_BK_BYTES / esz;
-  // int8 GEMMs with 256-wide tiles run on CTA pairs (each CTA loads 128 rows
-  // of A and 128 of B); the rest on single CTAs.
+  // GEMMs with 256-wide tiles and a block-Linear epilogue run on CTA pairs
+  // (each CTA loads 128 rows of A and 128 of B); the rest on single CTAs.
   int max_pairs = 0;
-  if (int8 && bn == 256 && !(epi == EPI_QKV && p.H % 256 != 0)) {
-    switch (epi) {
-      case EPI_BF16: max_pairs = pair_capacity<EPI_BF16>(); break;
-      case EPI_GELU: max_pairs = pair_capacity<EPI_GELU>(); break;
-      case EPI_GATED: max_pairs = pair_capacity<EPI_GATED>(); break;
-      case EPI_QKV: max_pairs = pair_capacity<EPI_QKV>(); break;
+  if (bn == 256 && !(epi == EPI_QKV && p.H % 256 != 0)) {
+    if (int8) {
+      switch (epi) {
+        case EPI_BF16: max_pairs = pair_capacity<true, EPI_BF16>(); break;
+        case EPI_GELU: max_pairs = pair_capacity<true, EPI_GELU>(); break;
+        case EPI_GATED: max_pairs = pair_capacity<true, EPI_GATED>(); break;
+        case EPI_QKV: max_pairs = pair_capacity<true, EPI_QKV>(); break;
+      }
+    } else {
+      switch (epi) {
+        case EPI_BF16: max_pairs = pair_capacity<false, EPI_BF16>(); break;
+        case EPI_GELU: max_pairs = pair_capacity<false, EPI_GELU>(); break;
+        case EPI_GATED: max_pairs = pair_capacity<false, EPI_GATED>(); break;
+        case EPI_QKV: max_pairs = pair_capacity<false, EPI_QKV>(); break;
+      }
     }
     max_pairs = max_pairs < num_sms / 2 ? max_pairs : num_sms / 2;
   }
@@ -989,11 +1015,20 @@ int launch_gemm(bool int8, int epi, const void* A, int lda, const void* B, int l
                     static_cast<uint32_t>(use_pair ? bn / 2 : bn)))
     return -2;
   if (use_pair) {
-    switch (epi) {
-      case EPI_BF16: return launch_gemm_pair<EPI_BF16>(ta, tb, q, max_pairs, st);
-      case EPI_GELU: return launch_gemm_pair<EPI_GELU>(ta, tb, q, max_pairs, st);
-      case EPI_GATED: return launch_gemm_pair<EPI_GATED>(ta, tb, q, max_pairs, st);
-      case EPI_QKV: return launch_gemm_pair<EPI_QKV>(ta, tb, q, max_pairs, st);
+    if (int8) {
+      switch (epi) {
+        case EPI_BF16: return launch_gemm_pair<true, EPI_BF16>(ta, tb, q, max_pairs, st);
+        case EPI_GELU: return launch_gemm_pair<true, EPI_GELU>(ta, tb, q, max_pairs, st);
+        case EPI_GATED: return launch_gemm_pair<true, EPI_GATED>(ta, tb, q, max_pairs, st);
+        case EPI_QKV: return launch_gemm_pair<true, EPI_QKV>(ta, tb, q, max_pairs, st);
+      }
+    } else {
+      switch (epi) {
+        case EPI_BF16: return launch_gemm_pair<false, EPI_BF16>(ta, tb, q, max_pairs, st);
+        case EPI_GELU: return launch_gemm_pair<false, EPI_GELU>(ta, tb, q, max_pairs, st);
+        case EPI_GATED: return launch_gemm_pair<false, EPI_GATED>(ta, tb, q, max_pairs, st);
+        case EPI_QKV: return launch_gemm_pair<false, EPI_QKV>(ta, tb, q, max_pairs, st);
+      }
     }
     return -1;
   }
@@ -1009,8 +1044,13 @@ int launch_gemm(bool int8, int epi, const void* A, int lda, const void* B, int l
   } else {
     switch (epi) {
       case EPI_BF16: return launch_gemm_bn<false, EPI_BF16>(bn, ta, tb, q, num_sms, st);
+      case EPI_GELU: return launch_gemm_bn<false, EPI_GELU>(bn, ta, tb, q, num_sms, st);
+      case EPI_GATED: return launch_gemm_bn<false, EPI_GATED>(bn, ta, tb, q, num_sms, st);
       case EPI_F32: return launch_gemm_bn<false, EPI_F32>(bn, ta, tb, q, num_sms, st);
       case EPI_EULER: return launch_gemm_bn<false, EPI_EULER>(bn, ta, tb, q, num_sms, st);
+      case EPI_QKV:
+        if (bn == 256 && p.H % 256 == 0) return launch_gemm_t<false, 256, EPI_QKV>(ta, tb, q, num_sms, st);
+        return -1;
     }
   }
   return -1;

@@ -82,8 +82,11 @@ struct GemmParams {
   int32_t* acc_debug;     // optional raw int32 accumulators [M, N]
   float dt;               // Euler: sigma_next - sigma
   float* v_out;           // Euler: optional velocity [M, ldyf]
-  // fused QKV epilogue (N = 3H; a tile holds whole heads of one of q, k, v)
+  // fused QKV epilogue (a tile holds whole heads of one of q, k, v): column
+  // n of this GEMM is column n_base + n of the [q | k | v] projection (N = 3H
+  // with n_base 0, or a part: the q, k columns, or the v columns at n_base 2H)
   int H;
+  int n_base;
   float eps;
   const uint16_t* wq;     // [128] bf16 RMSNorm scales
   const uint16_t* wk;
@@ -134,7 +137,8 @@ struct QuantParams {
   int ldq;
   float* s;               // [M]
   int32_t* zp;            // [M]
-  uint16_t* u_bf16;       // if non-null: write bf16(u) [M, ldq] instead of quantizing
+  uint16_t* u_bf16;       // if non-null: write bf16(u) [M, ldq] instead of quantizing ...
+  int quant_too;          // ... or as well as quantizing (LN variant)
   // LN variant: residual add before the LayerNorm, x += gate[row set] * y
   const uint16_t* res_y;  // bf16 [M, K] or null
   const uint16_t* res_gate;   // gate row of set r at res_gate + r * mod_ld

@@ -278,7 +278,7 @@ __global__ void __launch_bounds__(512) quant_ln_kernel(const QuantParams p) {
       *reinterpret_cast<uint4*>(p.u_bf16 + static_cast<int64_t>(row) * p.ldq + ch * 8) =
           make_uint4(w[0], w[1], w[2], w[3]);
     }
-    return;
+    if (!p.quant_too) return;
   }
   if (p.u_f32) {   // tap: the exact fp32 values quantized below
 #pragma unroll

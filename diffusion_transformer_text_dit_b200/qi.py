@@ -71,7 +71,9 @@ class qi_dims(C.Structure):
 
 class qi_block_weights(C.Structure):
     _fields_ = [("qkv", qi_w8), ("out", qi_w8), ("up", qi_w8), ("down", qi_w8),
-                ("norm_q", C.c_void_p), ("norm_k", C.c_void_p), ("mod", qi_linear_bf16)]
+                ("norm_q", C.c_void_p), ("norm_k", C.c_void_p), ("mod", qi_linear_bf16),
+                ("qkv_bf16", qi_linear_bf16), ("out_bf16", qi_linear_bf16),
+                ("up_bf16", qi_linear_bf16), ("down_bf16", qi_linear_bf16)]
 
 
 class qi_model(C.Structure):
@@ -522,18 +524,47 @@ def qi_debug_timeout_probe(ctx: Context, limit_ns: int, stream=None):
 # ------------------------------------------------------------------ model holders
 
 class BlockWeights:
-    """Device copies of one block's weights, quantized on the GPU by qi_prepare_w8."""
+    """Device copies of one block's weights.  W8A8 Linears are quantized on the
+    GPU by qi_prepare_w8; BF16 ones are cast to bf16.  ``precision`` maps "qk",
+    "v", "out", "up", "down" to "w8" or "bf16" (default: all W8A8); q and k
+    share one setting (they are one GEMM)."""
 
-    def __init__(self, ctx: Context, wts: dict, device="cuda"):
+    def __init__(self, ctx: Context, wts: dict, device="cuda", precision: Optional[dict] = None):
         self.t = {}
+        prec = {"qk": "w8", "v": "w8", "out": "w8", "up": "w8", "down": "w8"}
+        prec.update(precision or {})
         st = qi_block_weights()
-        for name in ("qkv", "out", "up", "down"):
-            w32 = wts[name].to(device=device, dtype=torch.float32).contiguous()
+
+        def w8(w, b):
+            w32 = w.to(device=device, dtype=torch.float32).contiguous()
             q, s, rs = qi_prepare_w8(ctx, w32)
             del w32
-            b = wts[name + "_b"].to(device=device, dtype=torch.bfloat16).contiguous()
-            self.t[name] = (q, s, rs, b)
-            setattr(st, name, w8_struct(q, s, rs, b))
+            b = b.to(device=device, dtype=torch.bfloat16).contiguous()
+            return (q, s, rs, b), w8_struct(q, s, rs, b)
+
+        def bf(w, b):
+            wb = w.to(device=device, dtype=torch.bfloat16).contiguous()
+            b = b.to(device=device, dtype=torch.bfloat16).contiguous()
+            return (wb, b), bf16_struct(wb, b)
+
+        W, B = wts["qkv"], wts["qkv_b"]
+        H = W.shape[0] // 3
+        if prec["qk"] == "w8" and prec["v"] == "w8":
+            self.t["qkv"], st.qkv = w8(W, B)
+        elif prec["qk"] == "w8":
+            self.t["qkv"], st.qkv = w8(W[:2 * H], B[:2 * H])
+            self.t["qkv_bf16"], st.qkv_bf16 = bf(W[2 * H:], B[2 * H:])
+        elif prec["v"] == "bf16":
+            self.t["qkv_bf16"], st.qkv_bf16 = bf(W, B)
+        else:
+            raise ValueError("q, k in BF16 with v in W8A8 is not a supported layout")
+        for name in ("out", "up", "down"):
+            if prec[name] == "w8":
+                self.t[name], s8 = w8(wts[name], wts[name + "_b"])
+                setattr(st, name, s8)
+            else:
+                self.t[name + "_bf16"], sb = bf(wts[name], wts[name + "_b"])
+                setattr(st, name + "_bf16", sb)
         self.t["norm_q"] = wts["norm_q"].to(device=device, dtype=torch.bfloat16).contiguous()
         self.t["norm_k"] = wts["norm_k"].to(device=device, dtype=torch.bfloat16).contiguous()
         st.norm_q = ptr(self.t["norm_q"])

@@ -29,7 +29,7 @@ import torch
 
 __all__ = [
     "Group", "DitConfig", "TINY", "BLOCK512", "STEP1024", "EDIT1024", "EDIT3REF1024", "CFG1024",
-    "GEN2048", "GEN2048_SCHED",
+    "GEN2048", "GEN2048_SCHED", "STEP1024_PAGES", "linear_precision",
     "CONFIGS", "gen", "linear_weight", "bias", "norm_weight", "latents",
     "text_features", "ref_latents", "hidden_states", "mod_table", "block_weights", "model_weights",
 ]
@@ -62,6 +62,7 @@ class DitConfig:
     uncond_text: int = 0                       # true CFG: negative-prompt tokens (0 = no guidance)
     fp8_from_step: int = 0                     # precision schedule: fp8 attention from this step (1-based; 0 = never)
     guidance: float = 4.0                      # true CFG scale
+    precision: str = "w8a8"                    # "w8a8": every attn/MLP Linear W8A8; "pages": the pages' layout
 
     @property
     def tokens(self) -> int:
@@ -134,8 +135,27 @@ GEN2048 = DitConfig("denoise40_2048px", 4096, 32, 128, 16384, 32, 64,
 # steps 1-7 with bf16 attention, steps 8-40 with fp8 (e4m3) attention.
 GEN2048_SCHED = GEN2048.replace(name="denoise40_2048px_sched", fp8_from_step=8)
 
+# The same step with the pages' mixed-precision layout (FlagRelease W8A8 card,
+# "Quantization and validation", Scope): W8A8 for the attention q, k and the
+# two MLP Linears of blocks 2-29 (112 modules), BF16 for v, the output
+# projection and every Linear of blocks 0, 1, 30 and 31.
+STEP1024_PAGES = STEP1024.replace(name="step_1024px_pagesmask", precision="pages")
+
 CONFIGS = {c.name: c for c in (TINY, BLOCK512, STEP1024, EDIT1024, EDIT3REF1024, CFG1024, GEN2048,
-                               GEN2048_SCHED)}
+                               GEN2048_SCHED, STEP1024_PAGES)}
+
+
+def linear_precision(cfg: DitConfig, layer: int) -> dict:
+    """Which Linears of block ``layer`` are W8A8 ("w8") and which BF16
+    ("bf16"): keys "qk" (the q and k rows of the fused projection), "v",
+    "out", "up", "down".  The pages' layout keeps the first two and the last
+    two blocks entirely in BF16 (blocks 2-29 of 32 carry the W8A8 Linears)."""
+    if cfg.precision == "w8a8":
+        return {"qk": "w8", "v": "w8", "out": "w8", "up": "w8", "down": "w8"}
+    assert cfg.precision == "pages"
+    if 2 <= layer < cfg.blocks - 2:
+        return {"qk": "w8", "v": "bf16", "out": "bf16", "up": "w8", "down": "w8"}
+    return {"qk": "bf16", "v": "bf16", "out": "bf16", "up": "bf16", "down": "bf16"}
 
 
 def gen(seed: int, *tags) -> torch.Generator:

@@ -142,14 +142,28 @@ typedef struct qi_dims {
   float eps;          /* LayerNorm / RMSNorm epsilon (1e-6) */
 } qi_dims;
 
+/* One block's weights.  Each of the four Linears is W8A8 ([W8]) or BF16: the
+ * pages' deployed layout keeps some Linears in BF16 ([W8] "Scope": only the
+ * attention q/k and the MLP Linears of blocks 2-29 are W8A8, everything else
+ * stays BF16).  A Linear whose W8A8 codes are NULL (q == NULL) uses the BF16
+ * weight of the same name.  The fused q | k | v projection comes in three
+ * forms: qkv.n == 3H (all W8A8); qkv.n == 2H (q, k W8A8) with qkv_bf16 holding
+ * the v rows (n = H); or qkv.q == NULL with qkv_bf16.n == 3H (all BF16).  A
+ * BF16 Linear takes the bf16-rounded activation (the LayerNorm + modulate
+ * value, the attention output or the GELU output) and accumulates in fp32 on
+ * tcgen05 kind::f16; its output is rounded to bf16 like a W8A8 Linear's. */
 typedef struct qi_block_weights {
-  qi_w8 qkv;               /* n = 3H: rows [0,H) = q, [H,2H) = k, [2H,3H) = v */
+  qi_w8 qkv;               /* n = 3H: rows [0,H) = q, [H,2H) = k, [2H,3H) = v (or n = 2H, see above) */
   qi_w8 out;               /* n = H, k = H */
   qi_w8 up;                /* n = F, k = H */
   qi_w8 down;              /* n = H, k = F */
   const uint16_t* norm_q;  /* [head_dim] bf16 RMSNorm scale */
   const uint16_t* norm_k;
   qi_linear_bf16 mod;      /* adaLN: n = 6H, k = H (used by the step-level calls) */
+  qi_linear_bf16 qkv_bf16; /* BF16 forms, used where the W8A8 codes are NULL (qkv: see above) */
+  qi_linear_bf16 out_bf16;
+  qi_linear_bf16 up_bf16;
+  qi_linear_bf16 down_bf16;
 } qi_block_weights;
 
 typedef struct qi_model {

@@ -138,6 +138,27 @@ def w8a8_apply(u, wq) -> np.ndarray:
     return w8a8_linear(qa, sa, zpa, *wq)[1]
 
 
+def bf16_linear(x, w, b=None) -> np.ndarray:
+    """A Linear kept in BF16 (FlagOS card, "Quantization and validation": the
+    Linears outside the W8A8 set and the activations stay BF16): the input is
+    the bf16 activation, the weight is bf16, the products are summed exactly
+    (float64 is exact for the short sums of bf16 x bf16 products used here to
+    far below bf16 resolution) and the output is rounded to bf16 once.
+    Returns bf16 values as float32."""
+    y = np.asarray(bf16_round(x), F64) @ np.asarray(bf16_round(w), F64).T
+    if b is not None:
+        y = y + np.asarray(b, F64)[None, :]
+    return bf16_round(y)
+
+
+def linear_apply(u, lin) -> np.ndarray:
+    """Apply one block Linear as prepared by ``prepare_block``: a W8A8 tuple
+    (q, s, rowsum, bias) or a BF16 one ("bf16", w, bias)."""
+    if isinstance(lin[0], str):
+        return bf16_linear(u, lin[1], lin[2])
+    return w8a8_apply(u, lin)
+
+
 # ----------------------------------------------------------------------------
 # Norms, modulation, activation
 # ----------------------------------------------------------------------------
@@ -425,12 +446,41 @@ def attention_block_causal_fp8_plain(q, k, v, q_group, k_group, sm_scale) -> np.
 # ----------------------------------------------------------------------------
 
 
-def prepare_block(wts: dict) -> dict:
-    """Quantize the four W8A8 Linears of a block (fp32 weights -> codes, scales, rowsums)."""
+PRECISION_W8A8 = {"qk": "w8", "v": "w8", "out": "w8", "up": "w8", "down": "w8"}
+
+
+def prepare_block(wts: dict, precision: Optional[dict] = None) -> dict:
+    """Prepare the Linears of a block from fp32 weights: W8A8 ones quantized
+    (codes, scales, rowsums), BF16 ones rounded to bf16.
+
+    precision maps "qk" (the q and k rows of the fused projection), "v", "out",
+    "up", "down" to "w8" or "bf16"; default all W8A8.  The pages' deployed
+    layout (FlagOS card, "Quantization and validation", Scope) keeps only q, k
+    and the MLP Linears of blocks 2-29 in W8A8.  W8A8 weights are quantized per
+    output row, so splitting the q | k | v projection by rows leaves every
+    code and scale unchanged.  "qkv" holds the projection's parts in column
+    order: a list of (Linear, first column)."""
+    prec = dict(PRECISION_W8A8)
+    prec.update(precision or {})
     out = {}
-    for name in ("qkv", "out", "up", "down"):
-        q, s, rs = prepare_w8(wts[name])
-        out[name] = (q, s, rs, np.asarray(wts[name + "_b"], F32))
+
+    def prep(w, b, kind):
+        w = np.asarray(w, F32)
+        b = np.asarray(b, F32)
+        if kind == "bf16":
+            return ("bf16", bf16_round(w), b)
+        q, s, rs = prepare_w8(w)
+        return (q, s, rs, b)
+
+    w3, b3 = np.asarray(wts["qkv"], F32), np.asarray(wts["qkv_b"], F32)
+    H = w3.shape[0] // 3
+    if prec["qk"] == prec["v"]:
+        out["qkv"] = [(prep(w3, b3, prec["qk"]), 0)]
+    else:
+        out["qkv"] = [(prep(w3[:2 * H], b3[:2 * H], prec["qk"]), 0),
+                      (prep(w3[2 * H:], b3[2 * H:], prec["v"]), 2 * H)]
+    for name in ("out", "up", "down"):
+        out[name] = prep(wts[name], wts[name + "_b"], prec[name])
     out["norm_q"] = np.asarray(wts["norm_q"], F32)
     out["norm_k"] = np.asarray(wts["norm_k"], F32)
     return out
@@ -464,7 +514,8 @@ def dit_block(x, pw: dict, mod, row_set, q_group, k_group, cos, sin, heads, head
     shift1, scale1, gate1, shift2, scale2, gate2 = (m[:, i, :] for i in range(6))
 
     u1 = modulate(layer_norm(x, eps), shift1, scale1)
-    qkv = w8a8_apply(u1, pw["qkv"])                         # bf16 values [T, 3H]
+    parts = pw["qkv"] if isinstance(pw["qkv"], list) else [(pw["qkv"], 0)]
+    qkv = np.concatenate([linear_apply(u1, lin) for lin, _ in parts], axis=1)   # bf16 [T, 3H]
     q = qkv[:, 0:H].reshape(T, heads, head_dim)
     k = qkv[:, H:2 * H].reshape(T, heads, head_dim)
     v = qkv[:, 2 * H:3 * H].reshape(T, heads, head_dim)
@@ -487,10 +538,10 @@ def dit_block(x, pw: dict, mod, row_set, q_group, k_group, cos, sin, heads, head
     # the CUDA path.
     o = bf16_round(o.reshape(T, H))
 
-    x = x + gate1 * w8a8_apply(o, pw["out"])
+    x = x + gate1 * linear_apply(o, pw["out"])
     u2 = modulate(layer_norm(x, eps), shift2, scale2)
-    g = bf16_round(gelu_tanh(w8a8_apply(u2, pw["up"])))
-    x = x + gate2 * w8a8_apply(g, pw["down"])
+    g = bf16_round(gelu_tanh(linear_apply(u2, pw["up"])))
+    x = x + gate2 * linear_apply(g, pw["down"])
     if return_kv:
         return x, (k, v)
     return x

@@ -12,8 +12,8 @@ from tests._util import bf16_np, cuda, rel_l2
 pytestmark = pytest.mark.gpu
 
 
-def oracle_block_weights(wts):
-    return O.prepare_block({k: v.float().numpy() for k, v in wts.items()})
+def oracle_block_weights(wts, precision=None):
+    return O.prepare_block({k: v.float().numpy() for k, v in wts.items()}, precision)
 
 
 def run_block(ctx, cfg, wts, x, mod, sizes, kv=None, row0=0, mode=qi.QI_KV_NONE, bw=None):
@@ -40,13 +40,58 @@ def run_block(ctx, cfg, wts, x, mod, sizes, kv=None, row0=0, mode=qi.QI_KV_NONE,
     return xg, kv, bw, gd
 
 
-def oracle_block(cfg, wts, x, mod, sizes, gd):
+def oracle_block(cfg, wts, x, mod, sizes, gd, precision=None):
     ends = list(np.cumsum(sizes))
     gid = O.group_ids(ends)
     rs = np.where(gid < len(sizes) - 1, 0, 1)
     cos, sin = O.rope_tables(O.rope_positions(gd))
-    return O.dit_block(x.numpy(), oracle_block_weights(wts), bf16_np(mod), rs, gid, gid, cos, sin,
-                       cfg.heads, cfg.head_dim, cfg.eps)
+    return O.dit_block(x.numpy(), oracle_block_weights(wts, precision), bf16_np(mod), rs, gid, gid,
+                       cos, sin, cfg.heads, cfg.head_dim, cfg.eps)
+
+
+# Per-Linear precision layouts (FlagRelease W8A8 card, "Quantization and
+# validation", Scope: only q, k and the MLP Linears of blocks 2-29 are W8A8;
+# the rest stays BF16).  Together they take every branch of the block: the
+# q | k | v projection all W8A8, W8A8 q, k with BF16 v, all BF16; the output
+# projection and each MLP Linear in either precision.
+PRECISIONS = {
+    "pages_mid": {"v": "bf16", "out": "bf16"},
+    "all_bf16": {"qk": "bf16", "v": "bf16", "out": "bf16", "up": "bf16", "down": "bf16"},
+    "bf16_mlp": {"up": "bf16", "down": "bf16"},
+    "bf16_down": {"down": "bf16"},
+}
+
+
+@pytest.mark.parametrize("cfg", [synth.TINY, synth.BLOCK512], ids=["tiny", "block_512px"])
+@pytest.mark.parametrize("prec", list(PRECISIONS), ids=list(PRECISIONS))
+def test_block_mixed_precision_vs_oracle(ctx, cfg, prec):
+    precision = PRECISIONS[prec]
+    wts = synth.block_weights(cfg, 0)
+    sizes = cfg.group_sizes()
+    x = synth.hidden_states(cfg, cfg.tokens)
+    mod = synth.mod_table(cfg)
+    bw = qi.BlockWeights(ctx, wts, precision=precision)
+    xg, _, _, gd = run_block(ctx, cfg, wts, x, mod, sizes, bw=bw)
+    ref = oracle_block(cfg, wts, x, mod, sizes, gd, precision)
+    out = xg.cpu().numpy()
+    assert np.all(np.isfinite(out))
+    assert rel_l2(out, ref) < 1e-2
+    assert rel_l2(out - x.numpy(), ref - x.numpy()) < 1e-2
+
+
+def test_block_mixed_precision_cached_prefix_bit_identical(ctx):
+    cfg = synth.TINY
+    sizes = [128, 64, 192]
+    wts = synth.block_weights(cfg, 1)
+    S = sum(sizes)
+    x = synth.hidden_states(cfg, S, tag="xc")
+    mod = synth.mod_table(cfg, tag="modc")
+    bw = qi.BlockWeights(ctx, wts, precision=PRECISIONS["pages_mid"])
+    full, kv, bw, _ = run_block(ctx, cfg, wts, x, mod, sizes, mode=qi.QI_KV_WRITE_PREFIX, bw=bw)
+    P = S - sizes[-1]
+    part, _, _, _ = run_block(ctx, cfg, wts, x[P:].contiguous(), mod, sizes, kv=kv, row0=P,
+                              mode=qi.QI_KV_READ_PREFIX, bw=bw)
+    assert torch.equal(full[P:], part)
 
 
 @pytest.mark.parametrize("cfg", [synth.TINY, synth.TINY.replace(

@@ -19,8 +19,9 @@ class Setup:
         self.glob = synth.model_weights(cfg)
         self.blocks = [synth.block_weights(cfg, l) for l in range(cfg.blocks)]
         self.dims = qi.dims_struct(H, cfg.heads, cfg.mlp, cfg.patch, cfg.blocks)
-        self.model = qi.Model(ctx, self.dims, [qi.BlockWeights(ctx, b) for b in self.blocks],
-                              self.glob)
+        self.model = qi.Model(ctx, self.dims,
+                              [qi.BlockWeights(ctx, b, precision=synth.linear_precision(cfg, l))
+                               for l, b in enumerate(self.blocks)], self.glob)
         self.gd = [(g.kind, g.tokens, g.grid) for g in cfg.groups]
         self.ends = list(np.cumsum(cfg.group_sizes()))
         self.groups = qi.groups_struct(self.ends, cfg.group_row_sets())
@@ -50,7 +51,8 @@ class Setup:
     def oracle_step(self, lat, sigma, sigma_next):
         cfg = self.cfg
         mw = {k: bf16_np(t) for k, t in self.glob.items()}
-        pws = [O.prepare_block({k: v.float().numpy() for k, v in b.items()}) for b in self.blocks]
+        pws = [O.prepare_block({k: v.float().numpy() for k, v in b.items()},
+                               synth.linear_precision(cfg, l)) for l, b in enumerate(self.blocks)]
         mods = [(bf16_np(b["mod"]), bf16_np(b["mod_b"])) for b in self.blocks]
         return O.step_forward(lat.numpy(), bf16_np(self.txt),
                               None if self.ref is None else self.ref.numpy(), mw, pws, mods,
@@ -67,8 +69,9 @@ class Setup:
     synth.TINY.replace(name="tiny_edit_3ref", blocks=2, patch=64,
                        groups=(synth.Group("text", 12), synth.Group("image", 16, (4, 4)),
                                synth.Group("image", 36, (6, 6)), synth.Group("image", 9, (3, 3)),
-                               synth.Group("image", 64, (8, 8))))],
-    ids=["2blk", "32blk", "edit", "edit_3ref"])
+                               synth.Group("image", 64, (8, 8)))),
+    synth.TINY.replace(name="tiny_pages", blocks=6, precision="pages")],
+    ids=["2blk", "32blk", "edit", "edit_3ref", "pages_mask_6blk"])
 def test_step_vs_oracle(ctx, cfg):
     s = Setup(ctx, cfg)
     sig = O.sigma_schedule(40, cfg.target_tokens)
@@ -80,13 +83,15 @@ def test_step_vs_oracle(ctx, cfg):
     assert np.array_equal(lat1.numpy(), O.euler_update(s.lat.numpy(), v.numpy(), sig[3], sig[4]))
 
 
-@pytest.mark.parametrize("edit", [0, 1, 3], ids=["text_image", "text_ref_image", "text_3ref_image"])
-def test_step_cached_equals_uncached(ctx, edit):
+@pytest.mark.parametrize("edit,precision", [(0, "w8a8"), (1, "w8a8"), (3, "w8a8"), (1, "pages")],
+                         ids=["text_image", "text_ref_image", "text_3ref_image", "pages_mask"])
+def test_step_cached_equals_uncached(ctx, edit, precision):
     refs = [synth.Group("image", 64, (8, 8)), synth.Group("image", 100, (10, 10)),
             synth.Group("image", 48, (6, 8))][:edit]
     groups = ((synth.Group("text", 128 if edit else 100),) + tuple(refs) +
               (synth.Group("image", 256, (16, 16)),))
-    cfg = synth.TINY.replace(name="cache", blocks=3, patch=64, groups=groups)
+    cfg = synth.TINY.replace(name="cache", blocks=3 if precision == "w8a8" else 5, patch=64,
+                             groups=groups, precision=precision)
     s = Setup(ctx, cfg)
     sig = O.sigma_schedule(40, cfg.target_tokens)
     a1, _ = s.gpu_step(ctx, s.lat, float(sig[0]), float(sig[1]), qi.QI_KV_WRITE_PREFIX)

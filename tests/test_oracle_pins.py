@@ -596,6 +596,60 @@ def test_block_vs_unquantized_torch_formulation(sizes):
     assert np.linalg.norm((bad - x) - (ref - x)) / np.linalg.norm(ref - x) > 0.1
 
 
+def test_bf16_linear_exact_sum_brute_force():
+    """BF16 Linear: bf16 input and weight, the exact sum of the products (here
+    with Python fractions), the bias, one rounding to bf16."""
+    from fractions import Fraction
+    r = np.random.default_rng(21)
+    x = r.standard_normal((3, 24)) * 3
+    w = r.standard_normal((5, 24)) * 0.1
+    b = O.bf16_round(r.standard_normal(5) * 0.1)
+    y = O.bf16_linear(x, w, b)
+    xb, wb = O.bf16_round(x), O.bf16_round(w)
+    for i in range(3):
+        for j in range(5):
+            exact = sum(Fraction(float(xb[i, k])) * Fraction(float(wb[j, k])) for k in range(24))
+            exact += Fraction(float(b[j]))
+            assert y[i, j] == O.bf16_round(np.array([float(exact)]))[0]
+    # identity weight, no bias: the bf16-rounded input itself
+    assert np.array_equal(O.bf16_linear(x[:, :5], np.eye(5)), O.bf16_round(x[:, :5]))
+
+
+def test_prepare_block_precision_split_and_bf16_block():
+    """Mixed precision (the pages' layout): the q, k rows keep exactly the
+    codes of the all-W8A8 projection (per-row quantization), the v rows and
+    the BF16 Linears are bf16 weights; a block with every Linear in BF16 is
+    much closer to the unquantized formulation than the W8A8 block, and the
+    W8A8 q, k / BF16 v block sits in between."""
+    H, F_, heads, d, eps = 256, 512, 2, 128, 1e-6
+    w = _tiny_weights(H, F_, d, 7)
+    full = O.prepare_block(w)
+    mixed = O.prepare_block(w, {"v": "bf16", "out": "bf16"})
+    (q8, s8, rs8, b8), c0 = full["qkv"][0]
+    (qk, sk, rsk, bk), c1 = mixed["qkv"][0]
+    assert c0 == c1 == 0 and np.array_equal(qk, q8[:2 * H]) and np.array_equal(sk, s8[:2 * H])
+    (tag, wv, bv), cv = mixed["qkv"][1]
+    assert tag == "bf16" and cv == 2 * H and np.array_equal(wv, O.bf16_round(w["qkv"][2 * H:]))
+    assert mixed["out"][0] == "bf16" and not isinstance(mixed["up"][0], str)
+    allbf = O.prepare_block(w, {k: "bf16" for k in O.PRECISION_W8A8})
+    sizes = [4, 8]
+    S = sum(sizes)
+    gid = O.group_ids(list(np.cumsum(sizes)))
+    row_set = np.where(gid < 1, 0, 1)
+    groups = [("text", 4, None), ("image", 8, (1, 8))]
+    pos = O.rope_positions(groups)
+    c, sn = O.rope_tables(pos)
+    r = np.random.default_rng(3)
+    x = r.standard_normal((S, H))
+    mod = O.bf16_round(r.standard_normal((2, 6, H)) * 0.5)
+    ref = _torch_block(x, w, mod, row_set, gid, pos, heads, d, eps)
+    err = {}
+    for name, pw in (("w8", full), ("mixed", mixed), ("bf16", allbf)):
+        out = O.dit_block(x, pw, mod, row_set, gid, gid, c, sn, heads, d, eps)
+        err[name] = np.linalg.norm((out - x) - (ref - x)) / np.linalg.norm(ref - x)
+    assert err["bf16"] < 0.01 and err["bf16"] < err["mixed"] < err["w8"] < 0.03, err
+
+
 def test_block_zero_gates_is_identity():
     H, F_, heads, d = 256, 512, 2, 128
     pw = O.prepare_block(_tiny_weights(H, F_, d, 9))
