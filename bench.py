@@ -61,7 +61,7 @@ def algorithmic_work(cfg: synth.DitConfig, cached: bool = False):
         for name, kind in synth.linear_precision(cfg, l).items():
             if kind == "w8":
                 i8_ops += 2 * rows * sizes[name]
-            else:
+            else:   # BF16 weights, or MXFP4 weights decoded to bf16 in the GEMM
                 bf16_block += 2 * rows * sizes[name]
     ends = np.cumsum(cfg.group_sizes())
     starts = np.concatenate([[0], ends[:-1]])
@@ -360,7 +360,19 @@ def aggregate_throughput(world: int, steps: int, max_ms: float) -> float:
 # ------------------------------------------------------------------ GPU arm
 
 WORKLOADS = {c.name: c for c in (synth.STEP1024, synth.EDIT1024, synth.EDIT3REF1024, synth.CFG1024,
-                                  synth.GEN2048, synth.GEN2048_SCHED, synth.STEP1024_PAGES)}
+                                  synth.GEN2048, synth.GEN2048_SCHED, synth.STEP1024_PAGES,
+                                  synth.STEP1024_MXFP4)}
+
+
+def weight_bytes_per_step(cfg) -> float:
+    """HBM bytes of weights one step streams: the block Linears at their
+    storage width (int8 1 B, bf16 2 B, MXFP4 4.25 bits) and the bf16 adaLN rows."""
+    H, F = cfg.hidden, cfg.mlp
+    sizes = {"qk": 2 * H * H, "v": H * H, "out": H * H, "up": F * H, "down": H * F}
+    width = {"w8": 1.0, "bf16": 2.0, "mx": 4.25 / 8}
+    lin = sum(sizes[n] * width[k] for l in range(cfg.blocks)
+              for n, k in synth.linear_precision(cfg, l).items())
+    return lin + cfg.blocks * 6 * H * H * 2
 
 
 def run_ours(args, rank, world, local_rank):
@@ -593,10 +605,12 @@ def run_ours(args, rank, world, local_rank):
                f"(scale {cfg.guidance}), " if cfg.uncond_text else "")
             + ("40-step FlowMatch Euler denoise, prefix K/V cached from step 2"
                if denoise else "uncached step")
-            + (", all attn/MLP Linears W8A8 (int8 GEMMs), " if cfg.precision == "w8a8" else
-               ", the pages' precision layout (W8A8 q, k, MLP up/down in blocks 2-29 on int8 "
-               "GEMMs; v, out projection and all Linears of blocks 0, 1, 30, 31 in BF16 on "
-               "bf16 GEMMs), ")
+            + {"w8a8": ", all attn/MLP Linears W8A8 (int8 GEMMs), ",
+               "pages": ", the pages' precision layout (W8A8 q, k, MLP up/down in blocks 2-29 on "
+                        "int8 GEMMs; v, out projection and all Linears of blocks 0, 1, 30, 31 in "
+                        "BF16 on bf16 GEMMs), ",
+               "mxfp4": ", all attn/MLP Linears with MXFP4 weights (synthetic checkpoint) decoded "
+                        "to bf16 inside bf16 GEMMs, bf16 activations, "}[cfg.precision]
             + (f"bf16 attention in steps 1-{cfg.fp8_from_step - 1} and fp8 (e4m3) attention from "
                f"step {cfg.fp8_from_step}" if cfg.fp8_from_step else "bf16 attention"))
     out = {
@@ -605,7 +619,8 @@ def run_ours(args, rank, world, local_rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
         "data": "synthetic",
         "config": {"workload": desc, "tokens": S, "blocks": cfg.blocks, "global_batch": world,
-                   "l2": "inputs larger than L2: ~12.8 GB of weights streamed per step",
+                   "l2": f"inputs larger than L2: ~{weight_bytes_per_step(cfg) / 1e9:.1f} GB of "
+                         f"weights streamed per step",
                    "parallelism": f"replicas x{world}"},
         "roofline": roof,
         "tensor_core_fracs": other,

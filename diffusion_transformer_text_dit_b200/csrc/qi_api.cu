@@ -418,20 +418,23 @@ BlockPrecision block_precision(const qi_dims& d, const qi_block_weights& w) {
 // A BF16 block Linear on tcgen05 kind::f16 (CTA pairs for 256-wide tiles)
 // with one of the block epilogues; `p` carries the epilogue fields.
 int run_bf16_block_linear(qi_ctx* ctx, const uint16_t* a, int M, int lda, const qi_linear_bf16& w,
-                          int epi, qi::GemmParams p, cudaStream_t st) {
+                          const qi_mxfp4& mx, int epi, qi::GemmParams p, cudaStream_t st) {
   if (M == 0) return QI_OK;
+  const bool is_mx = mx.packed != nullptr;
   p.M = M;
-  p.N = w.n;
-  p.K = w.k;
-  p.num_kb = w.k / 64;
+  p.N = is_mx ? mx.n : w.n;
+  p.K = is_mx ? mx.k : w.k;
+  p.num_kb = p.K / 64;
   p.s_a = nullptr;
   p.zp_a = nullptr;
   p.s_w = nullptr;
   p.rowsum = nullptr;
-  p.bias = w.bias;
+  p.bias = is_mx ? mx.bias : w.bias;
+  p.b_packed = is_mx ? mx.packed : nullptr;
+  p.b_scales = is_mx ? mx.scales : nullptr;
   p.status = ctx->status;
   Prof pr(ctx, QI_KCLASS_GEMM_BF16, st);
-  const int r = qi::launch_gemm(false, epi, a, lda, w.w, w.k, p, ctx->num_sms, st);
+  const int r = qi::launch_gemm(false, epi, a, lda, is_mx ? nullptr : w.w, p.K, p, ctx->num_sms, st);
   if (r == -2) return fail(QI_ERR_CUDA, "cuTensorMapEncodeTiled failed (BF16 block Linear)");
   if (r != 0) return cuda_fail("BF16 block Linear launch");
   return QI_OK;
@@ -527,7 +530,8 @@ int run_block_multi(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, fl
     }
     if (qkv_bf16) {
       p.n_base = bp.qkv_w8_cols;   // the v rows (2H) or all of q | k | v (0)
-      if ((r = run_bf16_block_linear(ctx, b.o, T, H, w.qkv_bf16, qi::EPI_QKV, p, st))) return r;
+      if ((r = run_bf16_block_linear(ctx, b.o, T, H, w.qkv_bf16, w.qkv_mx, qi::EPI_QKV, p, st)))
+        return r;
     }
   }
   if (f8) {
@@ -609,7 +613,8 @@ int run_block_multi(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, fl
     memset(&p, 0, sizeof(p));
     p.y = y_out;
     p.ldy = H;
-    if ((r = run_bf16_block_linear(ctx, b.o, T, H, w.out_bf16, qi::EPI_BF16, p, st))) return r;
+    if ((r = run_bf16_block_linear(ctx, b.o, T, H, w.out_bf16, w.out_mx, qi::EPI_BF16, p, st)))
+      return r;
   }
   // MLP half: x += gate1 * out, LN2 + modulate + quantize (and/or the bf16
   // value for a BF16 up projection, into the attention-output buffer, now
@@ -639,7 +644,8 @@ int run_block_multi(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, fl
     p.y = b.g;
     p.ldy = F;
     p.row_range = g_range;
-    if ((r = run_bf16_block_linear(ctx, b.o, T, H, w.up_bf16, qi::EPI_GELU, p, st))) return r;
+    if ((r = run_bf16_block_linear(ctx, b.o, T, H, w.up_bf16, w.up_mx, qi::EPI_GELU, p, st)))
+      return r;
   }
   if (tp && ((r = tap_copy(tp->g, b.g, static_cast<size_t>(T) * F * 2, st)) ||
              (bp.down_w8 && (r = tap_copy(tp->g_range, b.g_range, static_cast<size_t>(T) * 8, st)))))
@@ -665,7 +671,9 @@ int run_block_multi(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, fl
     p.gate_ld = mld;
     p.groups = gt;
     p.row0 = row0;
-    if ((r = run_bf16_block_linear(ctx, b.g, T, F, w.down_bf16, qi::EPI_GATED, p, st))) return r;
+    if ((r = run_bf16_block_linear(ctx, b.g, T, F, w.down_bf16, w.down_mx, qi::EPI_GATED, p,
+                                   st)))
+      return r;
   }
   return QI_OK;
 }
@@ -685,9 +693,25 @@ int run_block(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, float* x
   return run_block_multi(ctx, d, w, x, T, gt, row0, mod, cs, sn, &one, 1, ws, ws_bytes, st, f8);
 }
 
-// A block Linear given either as W8A8 codes or as a BF16 weight.
-int check_linear(const qi_w8* w8, const qi_linear_bf16* bf, const char* name, int n, int k) {
+int check_mx(const qi_mxfp4* w, const char* name, int n, int k) {
+  if (!w || !w->packed || !w->scales)
+    return fail(QI_ERR_INVALID_ARG, "MXFP4 weight %s has a NULL pointer", name);
+  if ((n >= 0 && w->n != n) || (k >= 0 && w->k != k))
+    return fail(QI_ERR_UNSUPPORTED_SHAPE, "MXFP4 weight %s is [%d, %d], expected [%d, %d]", name,
+                w->n, w->k, n, k);
+  if (w->k < 64 || w->k % 64 != 0 || w->n < 256 || w->n % 256 != 0)
+    return fail(QI_ERR_UNSUPPORTED_SHAPE, "MXFP4 weight %s: need k %% 64 == 0 and n %% 256 == 0",
+                name);
+  if (!aligned16(w->packed) || !aligned16(w->scales) || (w->bias && !aligned16(w->bias)))
+    return fail(QI_ERR_ALIGNMENT, "MXFP4 weight %s: pointers must be 16-byte aligned", name);
+  return QI_OK;
+}
+
+// A block Linear given as W8A8 codes, MXFP4 codes or a BF16 weight.
+int check_linear(const qi_w8* w8, const qi_linear_bf16* bf, const qi_mxfp4* mx, const char* name,
+                 int n, int k) {
   if (w8->q) return check_w8(w8, name, n, k);
+  if (mx->packed) return check_mx(mx, name, n, k);
   int r;
   if ((r = check_bf16_linear(bf, name, n, k))) return r;
   if (k % 64 != 0) return fail(QI_ERR_UNSUPPORTED_SHAPE, "BF16 weight %s: k %% 64 != 0", name);
@@ -699,16 +723,16 @@ int check_block_weights(const qi_dims& d, const qi_block_weights* w) {
   const int H = d.hidden, F = d.mlp;
   int r;
   if (!w->qkv.q) {
-    if ((r = check_linear(&w->qkv, &w->qkv_bf16, "qkv", 3 * H, H))) return r;
+    if ((r = check_linear(&w->qkv, &w->qkv_bf16, &w->qkv_mx, "qkv", 3 * H, H))) return r;
   } else if (w->qkv.n == 2 * H) {   // q, k W8A8; v BF16
     if ((r = check_w8(&w->qkv, "qkv (q, k rows)", 2 * H, H))) return r;
     if ((r = check_bf16_linear(&w->qkv_bf16, "qkv_bf16 (v rows)", H, H))) return r;
   } else if ((r = check_w8(&w->qkv, "qkv", 3 * H, H))) {
     return r;
   }
-  if ((r = check_linear(&w->out, &w->out_bf16, "out", H, H))) return r;
-  if ((r = check_linear(&w->up, &w->up_bf16, "up", F, H))) return r;
-  if ((r = check_linear(&w->down, &w->down_bf16, "down", H, F))) return r;
+  if ((r = check_linear(&w->out, &w->out_bf16, &w->out_mx, "out", H, H))) return r;
+  if ((r = check_linear(&w->up, &w->up_bf16, &w->up_mx, "up", F, H))) return r;
+  if ((r = check_linear(&w->down, &w->down_bf16, &w->down_mx, "down", H, F))) return r;
   if (!w->norm_q || !w->norm_k) return fail(QI_ERR_INVALID_ARG, "norm_q / norm_k is NULL");
   if (!aligned16(w->norm_q) || !aligned16(w->norm_k))
     return fail(QI_ERR_ALIGNMENT, "norm_q / norm_k must be 16-byte aligned");
@@ -1022,6 +1046,26 @@ int qi_w8a8_linear(qi_ctx* ctx, const int8_t* qa, const float* s_a, const int32_
   if (M == 0) return QI_OK;
   return run_w8a8(ctx, qa, s_a, zp_a, M, *w, qi::EPI_GATED, nullptr, 0, ep->residual,
                   ep->ld_residual, ep->gate, ep->gate_ld, gt, ep->row0, acc_debug, S(stream));
+}
+
+int qi_mxfp4_linear(qi_ctx* ctx, const uint16_t* a, int M, int lda, const qi_mxfp4* w,
+                    uint16_t* y, int ldy, void* stream) {
+  if (!ctx) return fail(QI_ERR_INVALID_ARG, "NULL argument");
+  if (M < 0) return fail(QI_ERR_INVALID_ARG, "M < 0");
+  if (M > 0 && (!a || !y)) return fail(QI_ERR_INVALID_ARG, "NULL argument");
+  int r;
+  if ((r = check_mx(w, "w", -1, -1))) return r;
+  if (lda < w->k || lda % 8 != 0 || ldy < w->n || ldy % 8 != 0)
+    return fail(QI_ERR_UNSUPPORTED_SHAPE, "mxfp4 linear: need lda >= k, ldy >= n, both %% 8 == 0");
+  if (!aligned16(a) || !aligned16(y)) return fail(QI_ERR_ALIGNMENT, "a / y must be 16-byte aligned");
+  if (M == 0) return QI_OK;
+  qi::GemmParams p;
+  memset(&p, 0, sizeof(p));
+  p.y = y;
+  p.ldy = ldy;
+  qi_linear_bf16 none;
+  memset(&none, 0, sizeof(none));
+  return run_bf16_block_linear(ctx, a, M, lda, none, *w, qi::EPI_BF16, p, S(stream));
 }
 
 int qi_bf16_linear(qi_ctx* ctx, const uint16_t* a, int M, int lda, const qi_linear_bf16* w,

@@ -712,8 +712,105 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols
   asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols));
 }
 
-template <bool I8, int EPI>
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
+// ---------------------------------------------------------------- MXFP4 B operand
+//
+// MXFP4 weights (EliovpAI "Qwen_Image-2.1-MXFP4-Paiton-RDNA4", "What was
+// quantized": E2M1 values packed two per byte, low nibble first, one E8M0
+// scale per 32 input columns) are decoded to bf16 inside the GEMM's load
+// path, so HBM holds 4.25 bits per weight.  E2M1 magnitudes are 0, 0.5, 1,
+// 1.5, 2, 3, 4, 6 (exponent bias 1, one mantissa bit), E8M0 is 2^(e - 127)
+// (255 = NaN); every product e2m1 x 2^(e - 127) has at most two significant
+// bits, so its bf16 value is exact.
+constexpr int MX_WARPS = 4;   // converter warps per CTA (one B row per thread)
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// Byte tables of the bf16 values of the 8 E2M1 magnitudes at scale 2^(e-127),
+// for 2 <= e <= 252 (every value then a normal bf16): magnitude c has the
+// exponent field e + E[c] (E = -1, 0, 0, 1, 1, 2, 2 for c = 1..7) and the
+// mantissa bit 0x40 for c = 3, 5, 7; c = 0 is +0.  lo0/lo1 hold the low bytes
+// of c = 0..3 / 4..7, hi0/hi1 the high bytes.
+struct MxTable {
+  uint32_t lo0, lo1, hi0, hi1;
+};
+__device__ __forceinline__ MxTable mx_table(uint32_t e) {
+  const uint32_t p0 = (e & 1u) << 7, p1 = ((e + 1u) & 1u) << 7;   // exponent LSB in bit 7
+  MxTable t;
+  t.lo0 = (p1 << 8) | (p0 << 16) | ((p0 | 0x40u) << 24);             // c = 0 .. 3 (c1: e - 1 ~ e + 1)
+  t.lo1 = p1 | ((p1 | 0x40u) << 8) | (p0 << 16) | ((p0 | 0x40u) << 24);
+  t.hi0 = (((e - 1u) >> 1) << 8) | ((e >> 1) << 16) | ((e >> 1) << 24);
+  t.hi1 = ((e + 1u) >> 1) | (((e + 1u) >> 1) << 8) | (((e + 2u) >> 1) << 16) | (((e + 2u) >> 1) << 24);
+  return t;
+}
+
+// 8 E2M1 codes (one 32-bit word, low nibble first) -> 8 bf16 values (4 words).
+__device__ __forceinline__ void mx_decode8(const MxTable& t, uint32_t w, uint32_t (&o)[4]) {
+  const uint32_t sel = w & 0x77777777u;                 // magnitudes as byte selectors
+  const uint32_t sg = (w << 4);                         // sign bit of every even nibble -> bit 7 of its byte
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t s = h ? (sel >> 16) : sel;
+    const uint32_t lo = prmt(t.lo0, t.lo1, s);
+    uint32_t hi = prmt(t.hi0, t.hi1, s);
+    // bit 7 of each value's byte: nibble 4h+0 from (w << 4), 4h+1 from w, ...
+    const uint32_t sbits = prmt(w, sg, h ? 0x3726u : 0x1504u);
+    hi |= sbits & 0x80808080u;
+    o[2 * h] = prmt(lo, hi, 0x5140u);
+    o[2 * h + 1] = prmt(lo, hi, 0x7362u);
+  }
+}
+
+// The general decode of 8 codes (any E8M0 byte, including the extremes and
+// the NaN marker 255): the fp32 value e2m1 x 2^(e-127), rounded to bf16.
+__device__ __noinline__ void mx_decode8_general(uint32_t e, uint32_t w, uint32_t (&o)[4]) {
+  const float scale = e == 255u ? __int_as_float(0x7FC00000) :
+                      (e == 0u ? __int_as_float(0x00400000) : __int_as_float(static_cast<int>(e << 23)));
+  float v[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t c = (w >> (4 * i)) & 15u;
+    const uint32_t ex = (c >> 1) & 3u, m = c & 1u;
+    const float mag = ex == 0u ? 0.5f * static_cast<float>(m)
+                               : (1.0f + 0.5f * static_cast<float>(m)) * static_cast<float>(1u << (ex - 1u));
+    v[i] = ((c & 8u) ? -mag : mag) * scale;
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) o[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+}
+
+// 32 codes (16 bytes) of one scale group -> 32 bf16 values (four 16-byte chunks).
+__device__ __forceinline__ void mx_decode32(uint32_t e, const uint4& w, uint32_t (&o)[16]) {
+  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+  if (e >= 2u && e <= 252u) {
+    const MxTable t = mx_table(e);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t q[4];
+      mx_decode8(t, ws[i], q);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) o[4 * i + j] = q[j];
+    }
+  } else {
+#pragma unroll 1
+    for (int i = 0; i < 4; ++i) {
+      uint32_t q[4];
+      mx_decode8_general(e, ws[i], q);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) o[4 * i + j] = q[j];
+    }
+  }
+}
+
+// With MXB the B operand is MXFP4 (bf16 A, kind::f16): MX_WARPS extra warps
+// per CTA decode this CTA's 128 B rows of each stage into the 128-byte
+// swizzled bf16 layout that TMA would have written, fence the writes for the
+// tensor core and arrive on the even CTA's full barrier.
+template <bool I8, int EPI, bool MXB = false>
+__global__ void __launch_bounds__(MXB ? GEMM_THREADS + 32 * MX_WARPS : GEMM_THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const GemmParams p) {
   constexpr int BN = 256;
@@ -746,7 +843,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < PAIR_STAGES; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], MXB ? 1 + 2 * MX_WARPS : 1);   // + the converter warps of both CTAs
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -759,7 +856,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmA);
-    prefetch_tmap(&tmB);
+    if (!MXB) prefetch_tmap(&tmB);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, 2 * BN);
@@ -786,10 +883,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, p.status)) { ok = false; break; }
           const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
-          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * PAIR_STAGE_BYTES);
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], MXB ? 2 * PAIR_A_BYTES : 2 * PAIR_STAGE_BYTES);
           // one 128-byte K row per stage: 128 int8 or 64 bf16 elements
           tma_load_2d_pair(&tmA, fb, sA + stage * PAIR_A_BYTES, kb * (I8 ? 128 : 64), m0);
-          tma_load_2d_pair(&tmB, fb, sB + stage * PAIR_B_BYTES, kb * (I8 ? 128 : 64), n0);
+          if (!MXB)
+            tma_load_2d_pair(&tmB, fb, sB + stage * PAIR_B_BYTES, kb * (I8 ? 128 : 64), n0);
           if (++stage == PAIR_STAGES) { stage = 0; phase ^= 1u; }
         }
       }
@@ -826,7 +924,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
         for (int kb = 0; kb < num_kb; ++kb) {
-          if (!mbar_wait(&full[stage], phase, p.status)) { ok = false; break; }
+          // (with MXB the stage also holds the converters' shared-memory
+          // writes of both CTAs, released at cluster scope)
+          if (!(MXB ? mbar_wait_cluster(&full[stage], phase, p.status)
+                    : mbar_wait(&full[stage], phase, p.status))) { ok = false; break; }
           tc_fence_after();
           const uint64_t adesc = umma_desc_kmajor_sw128(smem_u32(sA + stage * PAIR_A_BYTES));
           const uint64_t bdesc = umma_desc_kmajor_sw128(smem_u32(sB + stage * PAIR_B_BYTES));
@@ -854,7 +955,65 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         }
       }
     }
-  } else {
+  } else if (MXB && warp >= 2 + GEMM_EPI_WARPS) {
+    // ------------------------------------------------------------ MXFP4 converters (both CTAs)
+    // thread t decodes row n0 + t of this CTA's B half: per stage its 64
+    // codes (32 bytes) and their two E8M0 scales, loaded one stage ahead
+    const int t = threadIdx.x - 32 * (2 + GEMM_EPI_WARPS);
+    const size_t kh = static_cast<size_t>(p.K) / 2, kscl = static_cast<size_t>(p.K) / 32;
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int tile = pair; tile < num_tiles && ok; tile += num_pairs) {
+      int mt, nt;
+      tile_coords(tile, m_tiles, p.group_m, n_tiles, mt, nt);
+      const int n = nt * BN + static_cast<int>(rank) * (BN / 2) + t;
+      const bool n_ok = n < p.N;
+      const uint4* prow = reinterpret_cast<const uint4*>(p.b_packed + (n_ok ? n : 0) * kh);
+      const uint16_t* srow = reinterpret_cast<const uint16_t*>(p.b_scales + (n_ok ? n : 0) * kscl);
+      uint4 c0 = make_uint4(0, 0, 0, 0), c1 = c0;
+      uint32_t sc = 0;
+      if (n_ok) {
+        c0 = __ldg(prow);
+        c1 = __ldg(prow + 1);
+        sc = __ldg(srow);
+      }
+      for (int kb = 0; kb < num_kb; ++kb) {
+        const uint4 d0 = c0, d1 = c1;
+        const uint32_t dsc = sc;
+        if (n_ok && kb + 1 < num_kb) {   // next stage's codes, in flight while this one decodes
+          c0 = __ldg(prow + 2 * (kb + 1));
+          c1 = __ldg(prow + 2 * (kb + 1) + 1);
+          sc = __ldg(srow + kb + 1);
+        }
+        uint32_t o[32];
+        {
+          uint32_t a[16], b[16];
+          mx_decode32(dsc & 0xFFu, d0, a);
+          mx_decode32(dsc >> 8, d1, b);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            o[i] = n_ok ? a[i] : 0u;
+            o[16 + i] = n_ok ? b[i] : 0u;
+          }
+        }
+        if (!mbar_wait_warp(&empty[stage], phase ^ 1u, p.status)) { ok = false; break; }
+        // 128-byte swizzle: 16-byte chunk c of row t goes to chunk c ^ (t & 7)
+        uint8_t* row = sB + stage * PAIR_B_BYTES + t * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(row + ((c ^ (t & 7)) << 4)) =
+              make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) {
+          const uint32_t fr = mapa_shared(smem_u32(&full[stage]), 0);
+          asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(fr) : "memory");
+        }
+        if (++stage == PAIR_STAGES) { stage = 0; phase ^= 1u; }
+      }
+    }
+  } else if (warp >= 2 && warp < 2 + GEMM_EPI_WARPS) {
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int quarter = warp & 3;
     const int half = (warp - 2) >> 2;
@@ -911,11 +1070,11 @@ static int launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const Gem
 
 
 // Clusters of two that can be resident at once (0 if the pair kernel cannot run).
-template <bool I8, int EPI>
+template <bool I8, int EPI, bool MXB = false>
 static int pair_capacity() {
   static int cap = -1;   // per instantiation
   if (cap < 0) {
-    auto kern = gemm_pair_kernel<I8, EPI>;
+    auto kern = gemm_pair_kernel<I8, EPI, MXB>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PAIR_SMEM_BYTES) != cudaSuccess) {
       launch_result();
       return cap = 0;
@@ -927,7 +1086,7 @@ static int pair_capacity() {
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.gridDim = dim3(2, 1, 1);
-    cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
+    cfg.blockDim = dim3(MXB ? GEMM_THREADS + 32 * MX_WARPS : GEMM_THREADS, 1, 1);
     cfg.dynamicSmemBytes = PAIR_SMEM_BYTES;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
@@ -941,13 +1100,45 @@ static int pair_capacity() {
   return cap;
 }
 
-template <bool I8, int EPI>
+template <bool I8, int EPI, bool MXB = false>
 static int launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
                             int max_pairs, cudaStream_t st) {
   const int tiles = ((p.M + 2 * GEMM_BM - 1) / (2 * GEMM_BM)) * ((p.N + 255) / 256);
   const int pairs = tiles < max_pairs ? tiles : max_pairs;
-  launch_pdl(gemm_pair_kernel<I8, EPI>, dim3(2 * pairs), dim3(GEMM_THREADS), PAIR_SMEM_BYTES, st, 2, ta, tb, p);
+  launch_pdl(gemm_pair_kernel<I8, EPI, MXB>, dim3(2 * pairs),
+             dim3(MXB ? GEMM_THREADS + 32 * MX_WARPS : GEMM_THREADS), PAIR_SMEM_BYTES, st, 2, ta, tb, p);
   return launch_result();
+}
+
+// BF16 GEMM whose B operand is MXFP4 (p.b_packed [N, K/2] codes, p.b_scales
+// [N, K/32] E8M0), decoded in the load path; CTA pairs, N % 256 == 0.
+static int launch_gemm_mx(int epi, const void* A, int lda, const GemmParams& p, int num_sms,
+                          cudaStream_t st) {
+  int max_pairs = 0;
+  switch (epi) {
+    case EPI_BF16: max_pairs = pair_capacity<false, EPI_BF16, true>(); break;
+    case EPI_GELU: max_pairs = pair_capacity<false, EPI_GELU, true>(); break;
+    case EPI_GATED: max_pairs = pair_capacity<false, EPI_GATED, true>(); break;
+    case EPI_QKV: max_pairs = pair_capacity<false, EPI_QKV, true>(); break;
+    default: return -1;
+  }
+  max_pairs = max_pairs < num_sms / 2 ? max_pairs : num_sms / 2;
+  if (max_pairs < 1 || p.N % 256 != 0 || p.K % 64 != 0 || (epi == EPI_QKV && p.H % 256 != 0))
+    return -1;
+  GemmParams q = p;
+  const int m_tiles = (p.M + 2 * GEMM_BM - 1) / (2 * GEMM_BM);
+  q.group_m = m_tiles;   // B is small (4.25 bits per weight); A stays in L2
+  CUtensorMap ta;
+  if (!make_tmap_2d(&ta, A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<uint64_t>(p.K),
+                    static_cast<uint64_t>(p.M), static_cast<uint64_t>(lda) * 2, 64, GEMM_BM))
+    return -2;
+  switch (epi) {
+    case EPI_BF16: return launch_gemm_pair<false, EPI_BF16, true>(ta, ta, q, max_pairs, st);
+    case EPI_GELU: return launch_gemm_pair<false, EPI_GELU, true>(ta, ta, q, max_pairs, st);
+    case EPI_GATED: return launch_gemm_pair<false, EPI_GATED, true>(ta, ta, q, max_pairs, st);
+    case EPI_QKV: return launch_gemm_pair<false, EPI_QKV, true>(ta, ta, q, max_pairs, st);
+  }
+  return -1;
 }
 
 template <bool I8, int EPI>
@@ -969,6 +1160,7 @@ int pick_block_n(int N) {
 
 int launch_gemm(bool int8, int epi, const void* A, int lda, const void* B, int ldb,
                 const GemmParams& p, int num_sms, cudaStream_t st) {
+  if (p.b_packed) return int8 ? -1 : launch_gemm_mx(epi, A, lda, p, num_sms, st);
   const int bn = pick_block_n(p.N);
   const CUtensorMapDataType dt =
       int8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;

@@ -108,6 +108,10 @@ struct GemmParams {
   int ldo;
   uint32_t* row_range;    // GELU: optional per-row [-min, max] bit patterns of the bf16 output
   int group_m;            // tile order: bands of group_m M tiles (set by launch_gemm)
+  // MXFP4 B operand (BF16 GEMM only): E2M1 codes [N, K/2] (low nibble first)
+  // and E8M0 scales [N, K/32], decoded to bf16 in the load path; B is unused
+  const uint8_t* b_packed;
+  const uint8_t* b_scales;
   int* status;            // device status word
 };
 

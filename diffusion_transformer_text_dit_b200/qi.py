@@ -69,11 +69,18 @@ class qi_dims(C.Structure):
                 ("eps", C.c_float)]
 
 
+class qi_mxfp4(C.Structure):
+    _fields_ = [("packed", C.c_void_p), ("scales", C.c_void_p), ("bias", C.c_void_p),
+                ("n", C.c_int32), ("k", C.c_int32)]
+
+
 class qi_block_weights(C.Structure):
     _fields_ = [("qkv", qi_w8), ("out", qi_w8), ("up", qi_w8), ("down", qi_w8),
                 ("norm_q", C.c_void_p), ("norm_k", C.c_void_p), ("mod", qi_linear_bf16),
                 ("qkv_bf16", qi_linear_bf16), ("out_bf16", qi_linear_bf16),
-                ("up_bf16", qi_linear_bf16), ("down_bf16", qi_linear_bf16)]
+                ("up_bf16", qi_linear_bf16), ("down_bf16", qi_linear_bf16),
+                ("qkv_mx", qi_mxfp4), ("out_mx", qi_mxfp4), ("up_mx", qi_mxfp4),
+                ("down_mx", qi_mxfp4)]
 
 
 class qi_model(C.Structure):
@@ -116,6 +123,8 @@ _SIGS = {
                        C.c_void_p, C.c_void_p],
     "qi_bf16_linear": [C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.POINTER(qi_linear_bf16),
                        C.c_void_p, C.c_int, C.c_void_p],
+    "qi_mxfp4_linear": [C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.POINTER(qi_mxfp4),
+                        C.c_void_p, C.c_int, C.c_void_p],
     "qi_qk_norm_rope": [C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_int, C.c_void_p,
                         C.c_void_p, C.c_void_p, C.c_void_p, C.c_float, C.c_void_p, C.c_void_p,
                         C.c_void_p, C.c_int, C.c_void_p],
@@ -342,6 +351,26 @@ def qi_bf16_linear(ctx: Context, a: torch.Tensor, w: qi_linear_bf16, y: torch.Te
     return y
 
 
+def mx_struct(packed, scales, bias=None) -> qi_mxfp4:
+    """An MXFP4 Linear: packed [n, k/2] uint8 codes, scales [n, k/32] uint8 E8M0."""
+    m = qi_mxfp4()
+    m.packed, m.scales, m.bias = ptr(packed), ptr(scales), ptr(bias)
+    m.n = packed.shape[0]
+    m.k = 2 * packed.shape[1]
+    return m
+
+
+def qi_mxfp4_linear(ctx: Context, a: torch.Tensor, w: qi_mxfp4, y: Optional[torch.Tensor] = None,
+                    stream=None):
+    """bf16 y [M, n] = a [M, k] (bf16) x decode(w)^T + bias, MXFP4 decoded inside the GEMM."""
+    M = a.shape[0]
+    if y is None:
+        y = torch.empty((M, w.n), dtype=torch.bfloat16, device=a.device)
+    check(lib().qi_mxfp4_linear(ctx.handle, ptr(a), M, a.shape[1], C.byref(w), ptr(y), y.shape[1],
+                                stream_ptr(stream)))
+    return y
+
+
 def qi_qk_norm_rope(ctx: Context, qkv, heads, wq, wk, cos, sin, eps, q_out, k_out, v_out,
                     stream=None):
     T = qkv.shape[0]
@@ -547,9 +576,19 @@ class BlockWeights:
             b = b.to(device=device, dtype=torch.bfloat16).contiguous()
             return (wb, b), bf16_struct(wb, b)
 
-        W, B = wts["qkv"], wts["qkv_b"]
-        H = W.shape[0] // 3
-        if prec["qk"] == "w8" and prec["v"] == "w8":
+        def mx(codes, b):
+            pk = codes[0].to(device=device, dtype=torch.uint8).contiguous()
+            sc = codes[1].to(device=device, dtype=torch.uint8).contiguous()
+            b = b.to(device=device, dtype=torch.bfloat16).contiguous()
+            return (pk, sc, b), mx_struct(pk, sc, b)
+
+        W, B = wts["qkv"] if "qkv" in wts else None, wts["qkv_b"]
+        H = B.shape[0] // 3
+        if prec["qk"] == "mx" or prec["v"] == "mx":
+            if not (prec["qk"] == prec["v"] == "mx"):
+                raise ValueError("an MXFP4 q | k | v projection is MXFP4 throughout")
+            self.t["qkv_mx"], st.qkv_mx = mx(wts["qkv_mx"], B)
+        elif prec["qk"] == "w8" and prec["v"] == "w8":
             self.t["qkv"], st.qkv = w8(W, B)
         elif prec["qk"] == "w8":
             self.t["qkv"], st.qkv = w8(W[:2 * H], B[:2 * H])
@@ -562,6 +601,9 @@ class BlockWeights:
             if prec[name] == "w8":
                 self.t[name], s8 = w8(wts[name], wts[name + "_b"])
                 setattr(st, name, s8)
+            elif prec[name] == "mx":
+                self.t[name + "_mx"], sm = mx(wts[name + "_mx"], wts[name + "_b"])
+                setattr(st, name + "_mx", sm)
             else:
                 self.t[name + "_bf16"], sb = bf(wts[name], wts[name + "_b"])
                 setattr(st, name + "_bf16", sb)

@@ -29,7 +29,8 @@ import torch
 
 __all__ = [
     "Group", "DitConfig", "TINY", "BLOCK512", "STEP1024", "EDIT1024", "EDIT3REF1024", "CFG1024",
-    "GEN2048", "GEN2048_SCHED", "STEP1024_PAGES", "linear_precision",
+    "GEN2048", "GEN2048_SCHED", "STEP1024_PAGES", "STEP1024_MXFP4", "linear_precision",
+    "mxfp4_weight",
     "CONFIGS", "gen", "linear_weight", "bias", "norm_weight", "latents",
     "text_features", "ref_latents", "hidden_states", "mod_table", "block_weights", "model_weights",
 ]
@@ -62,7 +63,7 @@ class DitConfig:
     uncond_text: int = 0                       # true CFG: negative-prompt tokens (0 = no guidance)
     fp8_from_step: int = 0                     # precision schedule: fp8 attention from this step (1-based; 0 = never)
     guidance: float = 4.0                      # true CFG scale
-    precision: str = "w8a8"                    # "w8a8": every attn/MLP Linear W8A8; "pages": the pages' layout
+    precision: str = "w8a8"                    # "w8a8" | "pages" (W8A8/BF16 layout) | "mxfp4" (MXFP4 weights)
 
     @property
     def tokens(self) -> int:
@@ -145,6 +146,14 @@ CONFIGS = {c.name: c for c in (TINY, BLOCK512, STEP1024, EDIT1024, EDIT3REF1024,
                                GEN2048_SCHED, STEP1024_PAGES)}
 
 
+# The same step with every block Linear stored as MXFP4 and run on bf16
+# activations (EliovpAI "Qwen_Image-2.1-MXFP4-Paiton-RDNA4": MXFP4 weights;
+# the exact profile keeps BF16 activation arithmetic).  The block Linears are
+# a synthetic MXFP4 checkpoint (random codes and scales), see mxfp4_weight.
+STEP1024_MXFP4 = STEP1024.replace(name="step_1024px_mxfp4", precision="mxfp4")
+CONFIGS[STEP1024_MXFP4.name] = STEP1024_MXFP4
+
+
 def linear_precision(cfg: DitConfig, layer: int) -> dict:
     """Which Linears of block ``layer`` are W8A8 ("w8") and which BF16
     ("bf16"): keys "qk" (the q and k rows of the fused projection), "v",
@@ -152,6 +161,8 @@ def linear_precision(cfg: DitConfig, layer: int) -> dict:
     two blocks entirely in BF16 (blocks 2-29 of 32 carry the W8A8 Linears)."""
     if cfg.precision == "w8a8":
         return {"qk": "w8", "v": "w8", "out": "w8", "up": "w8", "down": "w8"}
+    if cfg.precision == "mxfp4":
+        return {"qk": "mx", "v": "mx", "out": "mx", "up": "mx", "down": "mx"}
     assert cfg.precision == "pages"
     if 2 <= layer < cfg.blocks - 2:
         return {"qk": "w8", "v": "bf16", "out": "bf16", "up": "w8", "down": "w8"}
@@ -226,6 +237,17 @@ def mod_table(cfg: DitConfig, rows: int = 2, device="cpu", tag="mod") -> torch.T
     return _normal((rows, 6, cfg.hidden), 0.5, gen(cfg.input_seed, tag), device).to(torch.bfloat16)
 
 
+def mxfp4_weight(seed, tag, n, k, device="cpu"):
+    """A synthetic MXFP4 checkpoint tensor [n, k]: E2M1 codes, two per byte
+    (low nibble first), uniform over the 16 codes -> packed uint8 [n, k/2];
+    one E8M0 scale byte per 32 columns, uniform in 118..121 (2^-9 .. 2^-6)
+    -> uint8 [n, k/32].  Random bytes only: no value is computed."""
+    g = gen(seed, "mx", tag)
+    packed = torch.randint(0, 256, (n, k // 2), generator=g, dtype=torch.uint8)
+    scales = torch.randint(118, 122, (n, k // 32), generator=g, dtype=torch.uint8)
+    return packed.to(device), scales.to(device)
+
+
 def block_weights(cfg: DitConfig, layer: int, device="cpu") -> dict:
     """Random-init weights of one block.
 
@@ -235,6 +257,19 @@ def block_weights(cfg: DitConfig, layer: int, device="cpu") -> dict:
     """
     s, H, F, d = cfg.weight_seed, cfg.hidden, cfg.mlp, cfg.head_dim
     L = ("blk", layer)
+    if cfg.precision == "mxfp4":
+        # the four Linears as MXFP4 codes (``<name>_mx`` = (packed, scales))
+        out = {name + "_mx": mxfp4_weight(s, L + (name,), n, k, device)
+               for name, n, k in (("qkv", 3 * H, H), ("out", H, H), ("up", F, H), ("down", H, F))}
+        out.update({
+            "qkv_b": bias(s, L + ("qkv",), 3 * H, device), "out_b": bias(s, L + ("out",), H, device),
+            "up_b": bias(s, L + ("up",), F, device), "down_b": bias(s, L + ("down",), H, device),
+            "norm_q": norm_weight(s, L + ("nq",), d, device),
+            "norm_k": norm_weight(s, L + ("nk",), d, device),
+            "mod": linear_weight(s, L + ("mod",), 6 * H, H, device).to(torch.bfloat16),
+            "mod_b": bias(s, L + ("mod",), 6 * H, device),
+        })
+        return out
     return {
         "qkv": linear_weight(s, L + ("qkv",), 3 * H, H, device),
         "qkv_b": bias(s, L + ("qkv",), 3 * H, device),

@@ -142,6 +142,22 @@ typedef struct qi_dims {
   float eps;          /* LayerNorm / RMSNorm epsilon (1e-6) */
 } qi_dims;
 
+/* One Linear stored as MXFP4 ([PX] What was quantized: E2M1 values packed two
+ * per byte, low nibble first; one E8M0 scale per 32 input columns), used with
+ * bf16 activations ([PX] Runtime precision and quality: the exact profile runs
+ * MXFP4 weights with BF16 activation arithmetic).  The GEMM decodes the codes
+ * to bf16 tile by tile in shared memory (every E2M1 x 2^(e-127) value is
+ * exact in bf16; E8M0 255 decodes to NaN) and accumulates in fp32 on tcgen05
+ * kind::f16, so HBM holds 4.25 bits per weight and no decoded copy exists.
+ *   packed [n, k/2] bytes, scales [n, k/32] bytes, bias [n] bf16 or NULL;
+ *   k % 64 == 0, n % 256 == 0; packed and scales 16-byte aligned. */
+typedef struct qi_mxfp4 {
+  const uint8_t* packed;
+  const uint8_t* scales;
+  const uint16_t* bias;
+  int32_t n, k;
+} qi_mxfp4;
+
 /* One block's weights.  Each of the four Linears is W8A8 ([W8]) or BF16: the
  * pages' deployed layout keeps some Linears in BF16 ([W8] "Scope": only the
  * attention q/k and the MLP Linears of blocks 2-29 are W8A8, everything else
@@ -164,6 +180,10 @@ typedef struct qi_block_weights {
   qi_linear_bf16 out_bf16;
   qi_linear_bf16 up_bf16;
   qi_linear_bf16 down_bf16;
+  qi_mxfp4 qkv_mx;         /* MXFP4 forms, used where the W8A8 codes are NULL and packed != NULL */
+  qi_mxfp4 out_mx;         /*   (qkv_mx: all of q | k | v, n = 3H); bf16 activations as for BF16 */
+  qi_mxfp4 up_mx;
+  qi_mxfp4 down_mx;
 } qi_block_weights;
 
 typedef struct qi_model {
@@ -254,6 +274,13 @@ int qi_quantize_act(qi_ctx* ctx, const void* x, int x_dtype, int M, int K, int l
 int qi_w8a8_linear(qi_ctx* ctx, const int8_t* qa, const float* s_a, const int32_t* zp_a, int M,
                    const qi_w8* w, const qi_epilogue* ep, uint16_t* y, int ldy,
                    int32_t* acc_debug, void* stream);
+
+/* Linear with MXFP4 weights (qi_mxfp4) on bf16 activations:
+ *   y [M, w.n] bf16 (ld ldy) = bf16(a [M, w.k] decode(w)^T + bias)
+ * the weights decoded to bf16 in shared memory inside the GEMM (fp32
+ * accumulation on tcgen05 kind::f16, CTA pairs).  lda % 8 == 0, ldy % 8 == 0. */
+int qi_mxfp4_linear(qi_ctx* ctx, const uint16_t* a, int M, int lda, const qi_mxfp4* w,
+                    uint16_t* y, int ldy, void* stream);
 
 /* BF16 Linear on tcgen05 tensor cores: y [M, w.n] fp32 (ld ldy) = a [M, w.k] W^T + b.
  * Requires w.k % 64 == 0, w.n % 16 == 0, lda % 8 == 0. */

@@ -454,7 +454,10 @@ def prepare_block(wts: dict, precision: Optional[dict] = None) -> dict:
     (codes, scales, rowsums), BF16 ones rounded to bf16.
 
     precision maps "qk" (the q and k rows of the fused projection), "v", "out",
-    "up", "down" to "w8" or "bf16"; default all W8A8.  The pages' deployed
+    "up", "down" to "w8", "bf16" or "mx"; default all W8A8.  "mx" Linears come
+    as MXFP4 codes ``wts[name + "_mx"] = (packed, scales)`` and run as BF16
+    Linears on their decoded weights ("Qwen_Image-2.1-MXFP4-Paiton-RDNA4":
+    MXFP4 weights, the exact profile with BF16 activation arithmetic).  The pages' deployed
     layout (FlagOS card, "Quantization and validation", Scope) keeps only q, k
     and the MLP Linears of blocks 2-29 in W8A8.  W8A8 weights are quantized per
     output row, so splitting the q | k | v projection by rows leaves every
@@ -465,22 +468,35 @@ def prepare_block(wts: dict, precision: Optional[dict] = None) -> dict:
     out = {}
 
     def prep(w, b, kind):
-        w = np.asarray(w, F32)
         b = np.asarray(b, F32)
+        if kind == "mx":        # MXFP4 codes (packed, scales), decoded; exact in bf16
+            return ("bf16", mxfp4_decode(*w), b)
+        w = np.asarray(w, F32)
         if kind == "bf16":
             return ("bf16", bf16_round(w), b)
         q, s, rs = prepare_w8(w)
         return (q, s, rs, b)
 
-    w3, b3 = np.asarray(wts["qkv"], F32), np.asarray(wts["qkv_b"], F32)
-    H = w3.shape[0] // 3
-    if prec["qk"] == prec["v"]:
+    def weight(name, kind):
+        return wts[name + "_mx"] if kind == "mx" else wts[name]
+
+    b3 = np.asarray(wts["qkv_b"], F32)
+    H = b3.shape[0] // 3
+    if prec["qk"] == "mx" or prec["v"] == "mx":
+        assert prec["qk"] == prec["v"] == "mx", "an MXFP4 q | k | v projection is MXFP4 throughout"
+        out["qkv"] = [(prep(wts["qkv_mx"], b3, "mx"), 0)]
+        w3 = None
+    else:
+        w3 = np.asarray(wts["qkv"], F32)
+    if w3 is None:
+        pass
+    elif prec["qk"] == prec["v"]:
         out["qkv"] = [(prep(w3, b3, prec["qk"]), 0)]
     else:
         out["qkv"] = [(prep(w3[:2 * H], b3[:2 * H], prec["qk"]), 0),
                       (prep(w3[2 * H:], b3[2 * H:], prec["v"]), 2 * H)]
     for name in ("out", "up", "down"):
-        out[name] = prep(wts[name], wts[name + "_b"], prec[name])
+        out[name] = prep(weight(name, prec[name]), wts[name + "_b"], prec[name])
     out["norm_q"] = np.asarray(wts["norm_q"], F32)
     out["norm_k"] = np.asarray(wts["norm_k"], F32)
     return out

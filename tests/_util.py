@@ -16,3 +16,15 @@ def rel_l2(a, b) -> float:
 
 def cuda(t: torch.Tensor, dtype=None) -> torch.Tensor:
     return t.to(device="cuda", dtype=dtype or t.dtype).contiguous()
+
+
+def oracle_weights(wts: dict) -> dict:
+    """A block's drawn weights as the oracle takes them: float tensors as fp32
+    numpy arrays, MXFP4 code pairs (packed, scales) as uint8 numpy arrays."""
+    out = {}
+    for k, v in wts.items():
+        if isinstance(v, tuple):
+            out[k] = tuple(t.detach().cpu().numpy() for t in v)
+        else:
+            out[k] = v.detach().to("cpu", torch.float32).numpy()
+    return out

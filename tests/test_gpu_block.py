@@ -7,13 +7,13 @@ import torch
 
 from diffusion_transformer_text_dit_b200 import qi, synth
 from oracle import qi_oracle as O
-from tests._util import bf16_np, cuda, rel_l2
+from tests._util import bf16_np, cuda, oracle_weights, rel_l2
 
 pytestmark = pytest.mark.gpu
 
 
 def oracle_block_weights(wts, precision=None):
-    return O.prepare_block({k: v.float().numpy() for k, v in wts.items()}, precision)
+    return O.prepare_block(oracle_weights(wts), precision)
 
 
 def run_block(ctx, cfg, wts, x, mod, sizes, kv=None, row0=0, mode=qi.QI_KV_NONE, bw=None):

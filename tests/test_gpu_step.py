@@ -7,7 +7,7 @@ import torch
 
 from diffusion_transformer_text_dit_b200 import qi, synth
 from oracle import qi_oracle as O
-from tests._util import bf16_np, cuda, rel_l2
+from tests._util import bf16_np, cuda, oracle_weights, rel_l2
 
 pytestmark = pytest.mark.gpu
 
@@ -51,8 +51,8 @@ class Setup:
     def oracle_step(self, lat, sigma, sigma_next):
         cfg = self.cfg
         mw = {k: bf16_np(t) for k, t in self.glob.items()}
-        pws = [O.prepare_block({k: v.float().numpy() for k, v in b.items()},
-                               synth.linear_precision(cfg, l)) for l, b in enumerate(self.blocks)]
+        pws = [O.prepare_block(oracle_weights(b), synth.linear_precision(cfg, l))
+               for l, b in enumerate(self.blocks)]
         mods = [(bf16_np(b["mod"]), bf16_np(b["mod_b"])) for b in self.blocks]
         return O.step_forward(lat.numpy(), bf16_np(self.txt),
                               None if self.ref is None else self.ref.numpy(), mw, pws, mods,
@@ -70,8 +70,9 @@ class Setup:
                        groups=(synth.Group("text", 12), synth.Group("image", 16, (4, 4)),
                                synth.Group("image", 36, (6, 6)), synth.Group("image", 9, (3, 3)),
                                synth.Group("image", 64, (8, 8)))),
-    synth.TINY.replace(name="tiny_pages", blocks=6, precision="pages")],
-    ids=["2blk", "32blk", "edit", "edit_3ref", "pages_mask_6blk"])
+    synth.TINY.replace(name="tiny_pages", blocks=6, precision="pages"),
+    synth.TINY.replace(name="tiny_mxfp4", blocks=3, patch=64, precision="mxfp4")],
+    ids=["2blk", "32blk", "edit", "edit_3ref", "pages_mask_6blk", "mxfp4_3blk"])
 def test_step_vs_oracle(ctx, cfg):
     s = Setup(ctx, cfg)
     sig = O.sigma_schedule(40, cfg.target_tokens)
@@ -83,8 +84,10 @@ def test_step_vs_oracle(ctx, cfg):
     assert np.array_equal(lat1.numpy(), O.euler_update(s.lat.numpy(), v.numpy(), sig[3], sig[4]))
 
 
-@pytest.mark.parametrize("edit,precision", [(0, "w8a8"), (1, "w8a8"), (3, "w8a8"), (1, "pages")],
-                         ids=["text_image", "text_ref_image", "text_3ref_image", "pages_mask"])
+@pytest.mark.parametrize("edit,precision", [(0, "w8a8"), (1, "w8a8"), (3, "w8a8"), (1, "pages"),
+                                            (1, "mxfp4")],
+                         ids=["text_image", "text_ref_image", "text_3ref_image", "pages_mask",
+                              "mxfp4"])
 def test_step_cached_equals_uncached(ctx, edit, precision):
     refs = [synth.Group("image", 64, (8, 8)), synth.Group("image", 100, (10, 10)),
             synth.Group("image", 48, (6, 8))][:edit]
