@@ -1204,7 +1204,7 @@ int qi_ctx_set_block_taps(qi_ctx* ctx, const qi_block_taps* taps) {
   const void* ptrs[] = {taps->u1, taps->q1, taps->s1, taps->zp1, taps->o, taps->o_range,
                         taps->qo, taps->so, taps->zpo, taps->x_mid, taps->u2, taps->q2,
                         taps->s2, taps->zp2, taps->g, taps->g_range, taps->qg, taps->sg,
-                        taps->zpg};
+                        taps->zpg, taps->x_layers};
   for (const void* q : ptrs)
     if (!aligned16(q)) return fail(QI_ERR_ALIGNMENT, "tap buffers must be 16-byte aligned");
   ctx->taps = *taps;
@@ -1389,6 +1389,9 @@ int qi_denoise_step(qi_ctx* ctx, const qi_model* model, float* latents, const ui
                            st)))
     return r;
 
+  float* x_layers = ctx->taps_on ? ctx->taps.x_layers : nullptr;
+  const size_t x_bytes = static_cast<size_t>(T) * H * sizeof(float);
+  if (x_layers && (r = tap_copy(x_layers, x, x_bytes, st))) return r;
   for (int l = 0; l < d.blocks; ++l) {
     uint16_t* kl = kv + static_cast<size_t>(l) * 2 * S_tok * H;
     uint16_t* vl = kl + static_cast<size_t>(S_tok) * H;
@@ -1397,6 +1400,9 @@ int qi_denoise_step(qi_ctx* ctx, const qi_model* model, float* latents, const ui
                        rope_cos + static_cast<size_t>(row0) * 64,
                        rope_sin + static_cast<size_t>(row0) * 64, kl, vl, b.block_ws,
                        b.block_ws_bytes, st, ctx->attn_fp8 ? &b.f8 : nullptr)))
+      return r;
+    if (x_layers &&
+        (r = tap_copy(reinterpret_cast<uint8_t*>(x_layers) + (l + 1) * x_bytes, x, x_bytes, st)))
       return r;
   }
 

@@ -958,7 +958,10 @@ __global__ void __launch_bounds__(MXB ? GEMM_THREADS + 32 * MX_WARPS : GEMM_THRE
   } else if (MXB && warp >= 2 + GEMM_EPI_WARPS) {
     // ------------------------------------------------------------ MXFP4 converters (both CTAs)
     // thread t decodes row n0 + t of this CTA's B half: per stage its 64
-    // codes (32 bytes) and their two E8M0 scales, loaded one stage ahead
+    // codes (32 bytes) and their two E8M0 scales.  The loads run MX_DEPTH
+    // stages ahead in a register ring, so the L2 latency of one stage's codes
+    // is hidden behind the decoding of the stages before it.
+    constexpr int MX_DEPTH = 4;
     const int t = threadIdx.x - 32 * (2 + GEMM_EPI_WARPS);
     const size_t kh = static_cast<size_t>(p.K) / 2, kscl = static_cast<size_t>(p.K) / 32;
     int stage = 0;
@@ -971,46 +974,58 @@ __global__ void __launch_bounds__(MXB ? GEMM_THREADS + 32 * MX_WARPS : GEMM_THRE
       const bool n_ok = n < p.N;
       const uint4* prow = reinterpret_cast<const uint4*>(p.b_packed + (n_ok ? n : 0) * kh);
       const uint16_t* srow = reinterpret_cast<const uint16_t*>(p.b_scales + (n_ok ? n : 0) * kscl);
-      uint4 c0 = make_uint4(0, 0, 0, 0), c1 = c0;
-      uint32_t sc = 0;
-      if (n_ok) {
-        c0 = __ldg(prow);
-        c1 = __ldg(prow + 1);
-        sc = __ldg(srow);
+      uint4 ca[MX_DEPTH], cb[MX_DEPTH];
+      uint32_t sc[MX_DEPTH];
+#pragma unroll
+      for (int u = 0; u < MX_DEPTH; ++u) {
+        ca[u] = cb[u] = make_uint4(0, 0, 0, 0);
+        sc[u] = 0;
+        if (n_ok && u < num_kb) {
+          ca[u] = __ldg(prow + 2 * u);
+          cb[u] = __ldg(prow + 2 * u + 1);
+          sc[u] = __ldg(srow + u);
+        }
       }
-      for (int kb = 0; kb < num_kb; ++kb) {
-        const uint4 d0 = c0, d1 = c1;
-        const uint32_t dsc = sc;
-        if (n_ok && kb + 1 < num_kb) {   // next stage's codes, in flight while this one decodes
-          c0 = __ldg(prow + 2 * (kb + 1));
-          c1 = __ldg(prow + 2 * (kb + 1) + 1);
-          sc = __ldg(srow + kb + 1);
-        }
-        uint32_t o[32];
-        {
-          uint32_t a[16], b[16];
-          mx_decode32(dsc & 0xFFu, d0, a);
-          mx_decode32(dsc >> 8, d1, b);
+#pragma unroll 1
+      for (int kb0 = 0; kb0 < num_kb && ok; kb0 += MX_DEPTH) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            o[i] = n_ok ? a[i] : 0u;
-            o[16 + i] = n_ok ? b[i] : 0u;
+        for (int u = 0; u < MX_DEPTH; ++u) {
+          const int kb = kb0 + u;
+          if (kb >= num_kb) break;
+          const uint4 d0 = ca[u], d1 = cb[u];
+          const uint32_t dsc = sc[u];
+          if (n_ok && kb + MX_DEPTH < num_kb) {
+            ca[u] = __ldg(prow + 2 * (kb + MX_DEPTH));
+            cb[u] = __ldg(prow + 2 * (kb + MX_DEPTH) + 1);
+            sc[u] = __ldg(srow + kb + MX_DEPTH);
           }
-        }
-        if (!mbar_wait_warp(&empty[stage], phase ^ 1u, p.status)) { ok = false; break; }
-        // 128-byte swizzle: 16-byte chunk c of row t goes to chunk c ^ (t & 7)
-        uint8_t* row = sB + stage * PAIR_B_BYTES + t * 128;
+          uint32_t o[32];
+          {
+            uint32_t a[16], b[16];
+            mx_decode32(dsc & 0xFFu, d0, a);
+            mx_decode32(dsc >> 8, d1, b);
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<uint4*>(row + ((c ^ (t & 7)) << 4)) =
-              make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        __syncwarp();
-        if (lane == 0) {
-          const uint32_t fr = mapa_shared(smem_u32(&full[stage]), 0);
-          asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(fr) : "memory");
+            for (int i = 0; i < 16; ++i) {
+              o[i] = n_ok ? a[i] : 0u;
+              o[16 + i] = n_ok ? b[i] : 0u;
+            }
+          }
+          if (!mbar_wait_warp(&empty[stage], phase ^ 1u, p.status)) { ok = false; break; }
+          // 128-byte swizzle: 16-byte chunk c of row t goes to chunk c ^ (t & 7)
+          uint8_t* row = sB + stage * PAIR_B_BYTES + t * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(row + ((c ^ (t & 7)) << 4)) =
+                make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+          if (lane == 0) {
+            const uint32_t fr = mapa_shared(smem_u32(&full[stage]), 0);
+            asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(fr)
+                         : "memory");
+          }
+          if (++stage == PAIR_STAGES) { stage = 0; phase ^= 1u; }
         }
-        if (++stage == PAIR_STAGES) { stage = 0; phase ^= 1u; }
       }
     }
   } else if (warp >= 2 && warp < 2 + GEMM_EPI_WARPS) {

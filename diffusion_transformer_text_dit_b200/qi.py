@@ -97,7 +97,7 @@ class qi_seq(C.Structure):
 
 
 TAP_FIELDS = ("u1", "q1", "s1", "zp1", "o", "o_range", "qo", "so", "zpo", "x_mid", "u2", "q2",
-              "s2", "zp2", "g", "g_range", "qg", "sg", "zpg")
+              "s2", "zp2", "g", "g_range", "qg", "sg", "zpg", "x_layers")
 
 
 class qi_block_taps(C.Structure):
@@ -319,10 +319,15 @@ def qi_quantize_act(ctx: Context, x: torch.Tensor, shift=None, scale=None, mod_l
     return q, s, zp
 
 
+# The weight structs hold raw device pointers, so each keeps references to the
+# tensors it points to: a tensor freed while the struct lives would let the
+# caching allocator hand its memory to a later tensor before a call reads it.
+
 def w8_struct(q, s, rowsum, bias=None) -> qi_w8:
     w = qi_w8()
     w.q, w.s, w.rowsum, w.bias = ptr(q), ptr(s), ptr(rowsum), ptr(bias)
     w.n, w.k = q.shape
+    w._keep = (q, s, rowsum, bias)
     return w
 
 
@@ -330,6 +335,7 @@ def bf16_struct(w, bias=None) -> qi_linear_bf16:
     s = qi_linear_bf16()
     s.w, s.bias = ptr(w), ptr(bias)
     s.n, s.k = w.shape
+    s._keep = (w, bias)
     return s
 
 
@@ -357,6 +363,7 @@ def mx_struct(packed, scales, bias=None) -> qi_mxfp4:
     m.packed, m.scales, m.bias = ptr(packed), ptr(scales), ptr(bias)
     m.n = packed.shape[0]
     m.k = 2 * packed.shape[1]
+    m._keep = (packed, scales, bias)
     return m
 
 

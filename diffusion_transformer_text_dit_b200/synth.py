@@ -29,7 +29,7 @@ import torch
 
 __all__ = [
     "Group", "DitConfig", "TINY", "BLOCK512", "STEP1024", "EDIT1024", "EDIT3REF1024", "CFG1024",
-    "GEN2048", "GEN2048_SCHED", "STEP1024_PAGES", "STEP1024_MXFP4", "linear_precision",
+    "GEN2048", "GEN2048_SCHED", "STEP1024_PAGES", "STEP1024_MXFP4", "STEP1024_BF16", "linear_precision",
     "mxfp4_weight",
     "CONFIGS", "gen", "linear_weight", "bias", "norm_weight", "latents",
     "text_features", "ref_latents", "hidden_states", "mod_table", "block_weights", "model_weights",
@@ -63,7 +63,7 @@ class DitConfig:
     uncond_text: int = 0                       # true CFG: negative-prompt tokens (0 = no guidance)
     fp8_from_step: int = 0                     # precision schedule: fp8 attention from this step (1-based; 0 = never)
     guidance: float = 4.0                      # true CFG scale
-    precision: str = "w8a8"                    # "w8a8" | "pages" (W8A8/BF16 layout) | "mxfp4" (MXFP4 weights)
+    precision: str = "w8a8"                    # "w8a8" | "pages" (W8A8/BF16 layout) | "mxfp4" | "bf16"
 
     @property
     def tokens(self) -> int:
@@ -152,6 +152,9 @@ CONFIGS = {c.name: c for c in (TINY, BLOCK512, STEP1024, EDIT1024, EDIT3REF1024,
 # a synthetic MXFP4 checkpoint (random codes and scales), see mxfp4_weight.
 STEP1024_MXFP4 = STEP1024.replace(name="step_1024px_mxfp4", precision="mxfp4")
 CONFIGS[STEP1024_MXFP4.name] = STEP1024_MXFP4
+# The same step on the BF16 path: every block Linear in BF16 (same weight draws).
+STEP1024_BF16 = STEP1024.replace(name="step_1024px_bf16", precision="bf16")
+CONFIGS[STEP1024_BF16.name] = STEP1024_BF16
 
 
 def linear_precision(cfg: DitConfig, layer: int) -> dict:
@@ -163,6 +166,8 @@ def linear_precision(cfg: DitConfig, layer: int) -> dict:
         return {"qk": "w8", "v": "w8", "out": "w8", "up": "w8", "down": "w8"}
     if cfg.precision == "mxfp4":
         return {"qk": "mx", "v": "mx", "out": "mx", "up": "mx", "down": "mx"}
+    if cfg.precision == "bf16":
+        return {"qk": "bf16", "v": "bf16", "out": "bf16", "up": "bf16", "down": "bf16"}
     assert cfg.precision == "pages"
     if 2 <= layer < cfg.blocks - 2:
         return {"qk": "w8", "v": "bf16", "out": "bf16", "up": "w8", "down": "w8"}

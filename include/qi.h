@@ -391,6 +391,8 @@ typedef struct qi_block_taps {
   int8_t* qg;
   float* sg;
   int32_t* zpg;
+  float* x_layers;   /* qi_denoise_step only: [blocks + 1][T][H] fp32, the residual stream
+                        before the first block and after each block */
 } qi_block_taps;
 
 /* Take the taps above in every block this context runs from now on (each block

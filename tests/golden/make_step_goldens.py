@@ -10,6 +10,14 @@ bounded), and runs ``oracle.qi_oracle.step_forward``.
 
     python tests/golden/make_step_goldens.py step_1024px
     python tests/golden/make_step_goldens.py edit_1024px
+    python tests/golden/make_step_goldens.py step_1024px_bf16
+    python tests/golden/make_step_goldens.py step_1024px_sensitivity
+
+``step_1024px_bf16`` is the same step with every block Linear in BF16 (the
+BF16 path); ``step_1024px_sensitivity`` runs the W8A8 step once more on the
+latents moved by one fp32 ulp each and records how far that moves v: the
+spread that two correct implementations of the same quantized stack, which
+round differently, can show after 32 blocks.
 
 Writes ``<workload>_v*.npy`` (fp32 [4096, 64] velocities) and
 ``<workload>.json`` (seeds, sigmas, input hashes, output hashes, oracle
@@ -76,7 +84,8 @@ class LazyBlocks:
         for l in range(self.cfg.blocks):
             wts = synth.block_weights(self.cfg, l)
             self.slot = (wts["mod"].float().numpy(), wts["mod_b"].float().numpy())
-            pw = O.prepare_block({k: v.float().numpy() for k, v in wts.items()})
+            pw = O.prepare_block({k: v.float().numpy() for k, v in wts.items()},
+                                 synth.linear_precision(self.cfg, l))
             del wts
             t = time.time() - self.t0
             print(f"  block {l + 1}/{self.cfg.blocks} drawn at {t:.0f} s", flush=True)
@@ -102,7 +111,7 @@ def run_step(cfg, lat, sigma, sigma_next, mode, kv_cache):
 
 
 def main(name: str):
-    cfg = synth.CONFIGS[name]
+    cfg = synth.CONFIGS["step_1024px" if name == "step_1024px_sensitivity" else name]
     sig = O.sigma_schedule(40, cfg.target_tokens)
     lat0 = synth.latents(cfg).numpy()
     meta = {"workload": name, "tokens": cfg.tokens, "groups": list(cfg.group_sizes()),
@@ -110,12 +119,23 @@ def main(name: str):
             "latent_seed": cfg.latent_seed, "sigmas": [float(sig[0]), float(sig[1]), float(sig[2])],
             "inputs": input_hashes(cfg), "oracle": "oracle.qi_oracle.step_forward (float64 numpy)",
             "cores": os.cpu_count()}
-    if name == "step_1024px":
+    if name in ("step_1024px", "step_1024px_bf16"):
         # one uncached step sigma_0 -> sigma_1
         _, v, secs = run_step(cfg, lat0, float(sig[0]), float(sig[1]), "none", None)
         np.save(os.path.join(HERE, f"{name}_v.npy"), v)
+        meta["precision"] = cfg.precision
         meta["steps"] = [{"mode": "none", "sigma": float(sig[0]), "sigma_next": float(sig[1]),
                           "v": f"{name}_v.npy", "v_sha": sha(v), "oracle_seconds": secs}]
+    elif name == "step_1024px_sensitivity":
+        # the W8A8 step on latents moved by one ulp (toward +inf), against the
+        # stored velocity of the unmoved latents
+        base = np.load(os.path.join(HERE, "step_1024px_v.npy"))
+        lat_up = np.nextafter(lat0, np.float32(np.inf)).astype(np.float32)
+        _, v, secs = run_step(cfg, lat_up, float(sig[0]), float(sig[1]), "none", None)
+        d = float(np.linalg.norm(v.astype(np.float64) - base) / np.linalg.norm(base))
+        meta["steps"] = [{"mode": "none", "sigma": float(sig[0]), "sigma_next": float(sig[1]),
+                          "latents": "nextafter(latents, +inf): every latent moved by one fp32 ulp",
+                          "v_rel_l2_vs_step_1024px": d, "v_sha": sha(v), "oracle_seconds": secs}]
     elif name == "edit_1024px":
         # step 1 writes the text + reference K/V; step 2 reads them and
         # processes the target rows only, from the oracle's step-1 latents

@@ -21,7 +21,7 @@ import torch
 
 from diffusion_transformer_text_dit_b200 import qi, synth
 from oracle import qi_oracle as O
-from tests._util import cuda, rel_l2
+from tests._util import cuda, oracle_weights, rel_l2
 from tests.golden.make_step_goldens import input_hashes
 
 pytestmark = pytest.mark.gpu
@@ -94,6 +94,42 @@ def test_step_1024px_vs_oracle(ctx, model):
     err = rel_l2(v, ov)
     assert err <= 2e-2, f"v rel-L2 {err:.3e} after 32 blocks"
     assert np.array_equal(lat1, O.euler_update(lat0, v, st["sigma"], st["sigma_next"]))
+
+
+def test_step_1024px_blocks_teacher_forced(ctx, model):
+    """Blocks of the full-width step against the oracle's block on the GPU's
+    own input to that block (the residual stream tapped before and after
+    every block): the first, a middle and the last block each within rel-L2
+    1e-2 of the oracle, on the whole block output and on the block's own
+    contribution (the delta), as for the single 512px block."""
+    cfg = synth.STEP1024
+    S, H = cfg.tokens, cfg.hidden
+    meta, _ = _golden("step_1024px")
+    st = meta["steps"][0]
+    r = Run(ctx, model, cfg)
+    x_layers = torch.empty((cfg.blocks + 1, S, H), dtype=torch.float32, device="cuda")
+    ctx.set_block_taps({"x_layers": x_layers})
+    try:
+        r.step(synth.latents(cfg).numpy(), st["sigma"], st["sigma_next"], qi.QI_KV_NONE)
+    finally:
+        ctx.set_block_taps(None)
+    mw = oracle_weights(synth.model_weights(cfg))
+    temb_0, temb_t = O.time_embed(0.0, mw), O.time_embed(st["sigma"], mw)
+    gd = [(g.kind, g.tokens, g.grid) for g in cfg.groups]
+    ends = list(np.cumsum(cfg.group_sizes()))
+    gid = O.group_ids(ends)
+    rs = np.where(gid < len(ends) - 1, 0, 1)
+    cos, sin = O.rope_tables(O.rope_positions(gd))
+    for l in (0, cfg.blocks // 2, cfg.blocks - 1):
+        wts = oracle_weights(synth.block_weights(cfg, l))
+        mod = np.stack([O.adaln_rows(temb_0, wts["mod"], wts["mod_b"]),
+                        O.adaln_rows(temb_t, wts["mod"], wts["mod_b"])])
+        x_in = x_layers[l].cpu().numpy()
+        got = x_layers[l + 1].cpu().numpy()
+        ref = O.dit_block(x_in, O.prepare_block(wts), mod, rs, gid, gid, cos, sin, cfg.heads,
+                          cfg.head_dim, cfg.eps)
+        e_out, e_delta = rel_l2(got, ref), rel_l2(got - x_in, ref - x_in)
+        assert e_out <= 1e-2 and e_delta <= 1e-2, (l, e_out, e_delta)
 
 
 def test_edit_1024px_write_then_cached_step_vs_oracle(ctx, model):
