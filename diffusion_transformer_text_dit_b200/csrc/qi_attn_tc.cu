@@ -217,17 +217,23 @@ __global__ void __maxnreg__(200)
           tma_load_2d(&tmQ, q_full, sQ + t * FA_TILE + half * FA_HALF, hc + 64 * half,
                       q0 + t * FA_ROWS);
       // K(j) into stage j % KST once S_B(j - KST) has read it; V(j) into
-      // stage j % VST once PV_B(j - VST) has.
+      // stage j % VST once PV_B(j - VST) has.  K runs one tile ahead of V:
+      // S(j+1) is issued early in the softmax of tile j, PV(j) only at its end.
       bool ok = true;
       int jk = 0, jv = 0;   // tiles whose loads were issued
-      for (int j = 0; j < n_kv; ++j) {
-        const int ks = j % KST, kr = j / KST;
-        if (!mbar_wait(&k_empty[ks], (kr & 1) ^ 1u, status)) { ok = false; break; }
+      auto load_k = [&](int jj) -> bool {
+        const int ks = jj % KST, kr = jj / KST;
+        if (!mbar_wait(&k_empty[ks], (kr & 1) ^ 1u, status)) return false;
         mbar_arrive_expect_tx(&k_full[ks], FA_TILE);
         for (int half = 0; half < Cfg::REGIONS; ++half)
           tma_load_2d(&tmK, &k_full[ks], sK + ks * FA_TILE + half * FA_HALF, hc + 64 * half,
-                      j * FA_ROWS);
-        jk = j + 1;
+                      jj * FA_ROWS);
+        jk = jj + 1;
+        return true;
+      };
+      if (n_kv > 0) ok = load_k(0);
+      for (int j = 0; ok && j < n_kv; ++j) {
+        if (j + 1 < n_kv && !load_k(j + 1)) { ok = false; break; }
         const int vs = j % VST, vr = j / VST;
         if (!mbar_wait(&v_empty[vs], (vr & 1) ^ 1u, status)) { ok = false; break; }
         mbar_arrive_expect_tx(&v_full[vs], FA_TILE);
