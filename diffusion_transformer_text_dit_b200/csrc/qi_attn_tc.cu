@@ -132,7 +132,7 @@ __device__ __forceinline__ int fa_key_limit(const GroupTable& g, int t) {
 }
 
 template <bool FP8>
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(FA_THREADS, 1)
     fa_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
   using Cfg = FaCfg<FP8>;
@@ -408,7 +408,10 @@ __global__ void __maxnreg__(200)
         float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          uint32_t pk[16];   // bf16: 16 words of 2 keys; e4m3: 8 words of 4 keys
+          // P goes to shared memory one 16-byte chunk at a time (8 bf16 or
+          // 16 e4m3 keys), as soon as its words are packed: chunk g of the
+          // row sits at chunk (g & 7) ^ (row & 7) of region g / 8
+          uint32_t pk[4];
           float e0 = 0.f, e1 = 0.f;
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
@@ -422,28 +425,23 @@ __global__ void __maxnreg__(200)
             acc2[i & 3] = f2_add(acc2[i & 3], f2_pack(p0, p1));
             if (FP8) {
               if (i & 1) {
-                pk[i >> 1] = pack_e4m3x4(e0, e1, p0, p1);   // keys 2i-2 .. 2i+1 of the chunk
+                pk[(i >> 1) & 3] = pack_e4m3x4(e0, e1, p0, p1);   // keys 2i-2 .. 2i+1 of the chunk
+                if ((i & 7) == 7) {
+                  const int g = 2 * c + (i >> 3);
+                  *reinterpret_cast<uint4*>(p_row + ((g ^ (row & 7)) << 4)) =
+                      make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                }
               } else {
                 e0 = p0;
                 e1 = p1;
               }
             } else {
-              pk[i] = pack_bf16x2(p0, p1);
-            }
-          }
-          if (FP8) {
-            // keys 32c .. 32c+31: 32 bytes = chunks 2c, 2c+1 of the one region
-#pragma unroll
-            for (int u = 0; u < 2; ++u)
-              *reinterpret_cast<uint4*>(p_row + (((2 * c + u) ^ (row & 7)) << 4)) =
-                  make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-          } else {
-            // keys 32c .. 32c+31: 64 bytes = chunks 4c .. 4c+3 (region c / 2)
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int g = 4 * c + u;
-              *reinterpret_cast<uint4*>(p_row + (g >> 3) * FA_HALF + (((g & 7) ^ (row & 7)) << 4)) =
-                  make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+              pk[i & 3] = pack_bf16x2(p0, p1);
+              if ((i & 3) == 3) {
+                const int g = 4 * c + (i >> 2);
+                *reinterpret_cast<uint4*>(p_row + (g >> 3) * FA_HALF + (((g & 7) ^ (row & 7)) << 4)) =
+                    make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              }
             }
           }
         }
