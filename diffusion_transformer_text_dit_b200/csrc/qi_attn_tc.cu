@@ -13,24 +13,21 @@
 //
 // One CTA = one head x 256 queries, as two 128-row tiles A and B that share
 // the key/value stream.  TMEM (512 columns): S_A | S_B | O_A | O_B, 128 fp32
-// columns each; P lives in shared memory.  Per key tile j of 128 keys:
+// columns each.  Per key tile j of 128 keys:
 //   S_X = Q_X K_j^T         tcgen05.mma kind::f16, A = Q (smem), B = K (smem), both K-major
-//   softmax warps of X load their S_X row into registers and release S_X at
-//   once, so S_X(j+1) is computed while they exponentiate; they write P_X as
-//   bf16 into shared memory (128-byte swizzle, K-major)
-//   O_X += P_X V_j          tcgen05.mma with A = P (smem), B = V (smem, MN-major)
-// The chain of a tile is thus its softmax alone: the next scores are ready
-// when the exponentials of this tile are done, and the two tiles' softmaxes
-// run side by side on their own warps.  The softmax keeps a per-row reference
-// maximum and rescales O (TMEM load / store) only when the running maximum
-// exceeds it by more than 8 (base 2): P <= 256 in between, exact in value
-// because the final normalisation divides by the same sum.  Before writing
-// P_X(j) (and before any rescale) a tile waits for PV_X(j-1).
+//   softmax warps of X read S_X (one query row per thread), write P_X as bf16
+//   into the first 64 columns of S_X
+//   O_X += P_X V_j          tcgen05.mma with A = P from TMEM, B = V (smem, MN-major)
+// Issue order (one thread): S_A0 S_B0 | PV_A(j) S_A(j+1) PV_B(j) S_B(j+1) ...
+// so each tile's softmax overlaps the other tile's MMAs.  The softmax keeps a
+// per-row reference maximum and rescales O (TMEM load / store) only when the
+// running maximum exceeds it by more than 8 (base 2): P <= 256 in between,
+// exact in value because the final normalisation divides by the same sum.
 //
 // Warps: 0-3 softmax of tile A (TMEM lanes 0-127), 4-7 softmax of tile B,
-// 8 TMA producer, 9 TMEM allocator + MMA issuer.  K streams through a 2-stage
-// ring (a stage is released once both S MMAs have read it), V through one
-// stage (3 and 2 for e4m3 tiles); every barrier wait is bounded (qi_common.cuh).
+// 8 TMA producer, 9 TMEM allocator + MMA issuer.  K streams through a 3-stage
+// ring (a stage is released once both S MMAs have read it), V through a
+// 2-stage ring; every barrier wait is bounded (qi_common.cuh).
 #include "qi_common.cuh"
 #include "qi_internal.h"
 
@@ -38,21 +35,18 @@ namespace qi {
 
 constexpr int FA_ROWS = 128;                   // rows per Q tile, keys per K/V tile
 constexpr int FA_THREADS = 320;
+constexpr int FA_KST = 3;                      // K ring stages
+constexpr int FA_VST = 2;                      // V ring stages
 
 // Tile geometry of the two element types.  A tile is 128 rows x 128 head
 // columns: bf16 -> two 64-column (128-byte) swizzle regions of 16 KB; e4m3 ->
 // one 128-column (128-byte) region of 16 KB.
-// Shared memory: Q (two tiles), a K ring, a V ring and P (two tiles); with
-// bf16 tiles (32 KB) the rings hold 2 K and 1 V tiles to fit 227 KB.
 template <bool FP8>
 struct FaCfg {
   static constexpr int TILE = FP8 ? 128 * 128 : 128 * 128 * 2;
   static constexpr int REGION = 128 * 128;       // bytes of one 128-byte-wide swizzle region
   static constexpr int REGIONS = TILE / REGION;  // 1 (e4m3) or 2 (bf16)
-  static constexpr int KST = FP8 ? 3 : 2;        // K ring stages
-  static constexpr int VST = FP8 ? 2 : 1;        // V ring stages
-  static constexpr int SMEM = 1024 + (2 + KST + VST + 2) * TILE + 256;
-  static_assert(SMEM <= 232448, "shared memory per CTA");
+  static constexpr int SMEM = 1024 + (2 + FA_KST + FA_VST) * TILE + 256;
 };
 
 // tcgen05.mma kind::f8f6f4 with A = B = e4m3 (format 0) and an fp32
@@ -68,6 +62,15 @@ __device__ __forceinline__ void umma_e4m3(uint32_t d_tmem, uint64_t a, uint64_t 
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
+}
+// D (TMEM) += A (TMEM, e4m3, 4 keys per 32-bit column) x B (smem descriptor).
+__device__ __forceinline__ void umma_e4m3_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate));
 }
 // Four values rounded to e4m3 (nearest, ties to even, saturating at +-448),
 // packed little-endian (a first).
@@ -92,6 +95,31 @@ __device__ __forceinline__ uint64_t umma_desc_mnmajor_sw128(uint32_t saddr, uint
   return d;
 }
 
+// D (TMEM) += A (TMEM, K-major) x B (smem descriptor), kind::f16.
+__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]));
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
@@ -138,26 +166,22 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
   using Cfg = FaCfg<FP8>;
   constexpr int FA_TILE = Cfg::TILE;
   constexpr int FA_HALF = Cfg::REGION;
-  constexpr int KST = Cfg::KST, VST = Cfg::VST;
   int* status = p.status;
   extern __shared__ uint8_t fa_smem_raw[];
   const uint32_t raw_addr = smem_u32(fa_smem_raw);
   uint8_t* smem = fa_smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   uint8_t* sQ = smem;                              // [2][FA_TILE]: tile A, tile B
-  uint8_t* sK = smem + 2 * FA_TILE;                // [KST][FA_TILE]
-  uint8_t* sV = sK + KST * FA_TILE;                // [VST][FA_TILE]
-  uint8_t* sP = sV + VST * FA_TILE;                // [2][FA_TILE]: P of tile A, tile B
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * FA_TILE);
+  uint8_t* sK = smem + 2 * FA_TILE;                // [FA_KST][FA_TILE]
+  uint8_t* sV = smem + (2 + FA_KST) * FA_TILE;     // [FA_VST][FA_TILE]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (2 + FA_KST + FA_VST) * FA_TILE);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;                     // [KST]
-  uint64_t* k_empty = k_full + KST;                // [KST]
-  uint64_t* v_full = k_empty + KST;                // [VST]
-  uint64_t* v_empty = v_full + VST;                // [VST]
-  uint64_t* s_full = v_empty + VST;                // [2] S_X(j) in TMEM
-  uint64_t* s_free = s_full + 2;                   // [2] S_X(j) loaded by the softmax warps
-  uint64_t* p_full = s_free + 2;                   // [2] P_X(j) in shared memory
-  uint64_t* pv_done = p_full + 2;                  // [2] O_X += P_X(j) V(j) complete
-  uint64_t* o_full = pv_done + 2;
+  uint64_t* k_full = bars + 1;                     // [FA_KST]
+  uint64_t* k_empty = k_full + FA_KST;             // [FA_KST]
+  uint64_t* v_full = k_empty + FA_KST;             // [FA_VST]
+  uint64_t* v_empty = v_full + FA_VST;             // [FA_VST]
+  uint64_t* s_full = v_empty + FA_VST;             // [2] per Q tile
+  uint64_t* p_full = s_full + 2;                   // [2] per Q tile
+  uint64_t* o_full = p_full + 2;
   uint64_t* drain = o_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
@@ -174,19 +198,17 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < KST; ++s) {
+    for (int s = 0; s < FA_KST; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&k_empty[s], 1);
     }
-    for (int s = 0; s < VST; ++s) {
+    for (int s = 0; s < FA_VST; ++s) {
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
-      mbar_init(&s_free[s], 4);    // one arrival per softmax warp of the tile
-      mbar_init(&p_full[s], 4);
-      mbar_init(&pv_done[s], 1);
+      mbar_init(&p_full[s], 128);
     }
     mbar_init(o_full, 1);
     mbar_init(drain, 1);
@@ -216,25 +238,20 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         for (int half = 0; half < Cfg::REGIONS; ++half)
           tma_load_2d(&tmQ, q_full, sQ + t * FA_TILE + half * FA_HALF, hc + 64 * half,
                       q0 + t * FA_ROWS);
-      // K(j) into stage j % KST once S_B(j - KST) has read it; V(j) into
-      // stage j % VST once PV_B(j - VST) has.  K runs one tile ahead of V:
-      // S(j+1) is issued early in the softmax of tile j, PV(j) only at its end.
+      // K(j) into stage j % FA_KST once S_B(j - FA_KST) has read it; V(j) into
+      // stage j % FA_VST once PV_B(j - FA_VST) has.  K runs further ahead:
+      // the next S MMA needs it well before the next PV needs V.
       bool ok = true;
       int jk = 0, jv = 0;   // tiles whose loads were issued
-      auto load_k = [&](int jj) -> bool {
-        const int ks = jj % KST, kr = jj / KST;
-        if (!mbar_wait(&k_empty[ks], (kr & 1) ^ 1u, status)) return false;
+      for (int j = 0; j < n_kv; ++j) {
+        const int ks = j % FA_KST, kr = j / FA_KST;
+        if (!mbar_wait(&k_empty[ks], (kr & 1) ^ 1u, status)) { ok = false; break; }
         mbar_arrive_expect_tx(&k_full[ks], FA_TILE);
         for (int half = 0; half < Cfg::REGIONS; ++half)
           tma_load_2d(&tmK, &k_full[ks], sK + ks * FA_TILE + half * FA_HALF, hc + 64 * half,
-                      jj * FA_ROWS);
-        jk = jj + 1;
-        return true;
-      };
-      if (n_kv > 0) ok = load_k(0);
-      for (int j = 0; ok && j < n_kv; ++j) {
-        if (j + 1 < n_kv && !load_k(j + 1)) { ok = false; break; }
-        const int vs = j % VST, vr = j / VST;
+                      j * FA_ROWS);
+        jk = j + 1;
+        const int vs = j % FA_VST, vr = j / FA_VST;
         if (!mbar_wait(&v_empty[vs], (vr & 1) ^ 1u, status)) { ok = false; break; }
         mbar_arrive_expect_tx(&v_full[vs], FA_TILE);
         for (int half = 0; half < Cfg::REGIONS; ++half)
@@ -247,15 +264,15 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         const uint64_t t0 = globaltimer_ns();
         while (!mbar_try_wait(q_full, 0) && globaltimer_ns() - t0 < QI_WAIT_NS) {
         }
-        for (int jj = (jk > KST ? jk - KST : 0); jj < jk; ++jj) {
+        for (int jj = (jk > FA_KST ? jk - FA_KST : 0); jj < jk; ++jj) {
           const uint64_t t1 = globaltimer_ns();
-          while (!mbar_try_wait(&k_full[jj % KST], (jj / KST) & 1) &&
+          while (!mbar_try_wait(&k_full[jj % FA_KST], (jj / FA_KST) & 1) &&
                  globaltimer_ns() - t1 < QI_WAIT_NS) {
           }
         }
-        for (int jj = (jv > VST ? jv - VST : 0); jj < jv; ++jj) {
+        for (int jj = (jv > FA_VST ? jv - FA_VST : 0); jj < jv; ++jj) {
           const uint64_t t1 = globaltimer_ns();
-          while (!mbar_try_wait(&v_full[jj % VST], (jj / VST) & 1) &&
+          while (!mbar_try_wait(&v_full[jj % FA_VST], (jj / FA_VST) & 1) &&
                  globaltimer_ns() - t1 < QI_WAIT_NS) {
           }
         }
@@ -263,18 +280,14 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
-    // Per key tile j: S_A(j+1) and S_B(j+1) go out as soon as the softmax
-    // warps of that tile hold S(j) in registers (so the next scores are
-    // computed while this tile's exponentials run), then PV_A(j) and PV_B(j)
-    // as soon as P(j) is in shared memory.
     if (lane == 0) {
       constexpr uint32_t idesc_s = FP8 ? umma_idesc_e4m3(128, 128, false) : umma_idesc(false, 128, 128);
       constexpr uint32_t idesc_pv = FP8 ? umma_idesc_e4m3(128, 128, true)
                                         : (umma_idesc(false, 128, 128) | (1u << 16));   // B MN-major
       bool ok = mbar_wait(q_full, 0, status);
       auto issue_s = [&](int X, int jj) -> bool {
-        const int st = jj % KST;
-        if (!mbar_wait(&k_full[st], (jj / KST) & 1, status)) return false;
+        const int st = jj % FA_KST;
+        if (!mbar_wait(&k_full[st], (jj / FA_KST) & 1, status)) return false;
         tc_fence_after();
         const uint32_t qa = smem_u32(sQ + X * FA_TILE), kb = smem_u32(sK + st * FA_TILE);
         if (FP8) {
@@ -294,28 +307,24 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         return true;
       };
       auto issue_pv = [&](int X, int jj) -> bool {
-        const int st = jj % VST;
-        if (!mbar_wait(&v_full[st], (jj / VST) & 1, status)) return false;
+        const int st = jj % FA_VST;
+        if (!mbar_wait(&v_full[st], (jj / FA_VST) & 1, status)) return false;
         if (!mbar_wait(&p_full[X], jj & 1, status)) return false;
         tc_fence_after();
         const uint32_t vb = smem_u32(sV + st * FA_TILE);
-        const uint32_t pa = smem_u32(sP + X * FA_TILE);
         if (FP8) {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)   // 32 keys per instruction
-            umma_e4m3(tmem_base + 256 + X * 128, umma_desc_kmajor_sw128(pa + kk * 32),
-                      umma_desc_mnmajor_sw128(vb + kk * 32 * 128, FA_HALF), idesc_pv,
-                      (jj > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk)   // 32 keys per instruction (8 columns of e4m3 P)
+            umma_e4m3_ts(tmem_base + 256 + X * 128, tmem_base + X * 128 + kk * 8,
+                         umma_desc_mnmajor_sw128(vb + kk * 32 * 128, FA_HALF), idesc_pv,
+                         (jj > 0 || kk > 0) ? 1u : 0u);
         } else {
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {   // 16 keys per instruction: two 8-row groups of V
-            const uint32_t off = (kk >> 2) * FA_HALF + (kk & 3) * 32;
-            umma_f16(tmem_base + 256 + X * 128, umma_desc_kmajor_sw128(pa + off),
-                     umma_desc_mnmajor_sw128(vb + kk * 2048, FA_HALF), idesc_pv,
-                     (jj > 0 || kk > 0) ? 1u : 0u);
-          }
+          for (int kk = 0; kk < 8; ++kk)   // 16 keys per instruction: two 8-row groups
+            umma_f16_ts(tmem_base + 256 + X * 128, tmem_base + X * 128 + kk * 8,
+                        umma_desc_mnmajor_sw128(vb + kk * 2048, FA_HALF), idesc_pv,
+                        (jj > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&pv_done[X]);
         return true;
       };
       if (ok && n_kv > 0) {
@@ -323,13 +332,14 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         if (ok) umma_commit(&k_empty[0]);
       }
       for (int j = 0; ok && j < n_kv; ++j) {
-        if (j + 1 < n_kv) {
-          ok = mbar_wait(&s_free[0], j & 1, status) && issue_s(0, j + 1) &&
-               mbar_wait(&s_free[1], j & 1, status) && issue_s(1, j + 1);
-          if (ok) umma_commit(&k_empty[(j + 1) % KST]);
+        ok = issue_pv(0, j);
+        if (ok && j + 1 < n_kv) ok = issue_s(0, j + 1);
+        if (ok) ok = issue_pv(1, j);
+        if (ok) umma_commit(&v_empty[j % FA_VST]);
+        if (ok && j + 1 < n_kv) {
+          ok = issue_s(1, j + 1);
+          if (ok) umma_commit(&k_empty[(j + 1) % FA_KST]);
         }
-        if (ok) ok = issue_pv(0, j) && issue_pv(1, j);
-        if (ok) umma_commit(&v_empty[j % VST]);
       }
       if (ok) {
         umma_commit(o_full);
@@ -351,9 +361,6 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
     const int qrow = q0 + X * FA_ROWS + row;
     const int lim = qrow < p.Sq ? min(fa_key_limit(p.groups, p.q_offset + qrow), p.Sk) : p.Sk;
     const float sl2 = p.sm_scale * 1.4426950408889634f;
-    // this row of P in shared memory: 128-byte swizzle rows, 16-byte chunk g of
-    // the row at chunk (g ^ (row & 7)) of its 128-byte region
-    uint8_t* p_row = sP + X * FA_TILE + row * 128;
     float m_ref = -INFINITY;   // reference maximum, base-2 scaled
     float l = 0.f;
     bool ok = true;
@@ -364,10 +371,6 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
       const bool masked = k0 + FA_ROWS > kv_min;
       uint32_t r[128];
       tmem_ld128(tS, r);                     // the whole S row, read once
-      // S(j) is in registers: the next S of this tile may overwrite TMEM
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[X]);
       if (masked) {
 #pragma unroll
         for (int i = 0; i < 128; ++i)
@@ -386,11 +389,6 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
           for (int k = 0; k < 8; ++k)
             m8[k] = fmax3(m8[k], __uint_as_float(r[i + 2 * k]), __uint_as_float(r[i + 2 * k + 1]));
         m_ref = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7])) * sl2;
-      } else {
-        // P(j-1) has been consumed and O holds every tile before j: this
-        // tile's P buffer may be rewritten and O rescaled
-        if (!mbar_wait_warp(&pv_done[X], (j - 1) & 1, status)) { ok = false; break; }
-        tc_fence_after();
       }
       // P = 2^(s sl2 - m_ref) with the current reference maximum (the
       // scale-subtract as paired fp32 FMAs, the row sum in 4 paired partial
@@ -408,10 +406,7 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          // P goes to shared memory one 16-byte chunk at a time (8 bf16 or
-          // 16 e4m3 keys), as soon as its words are packed: chunk g of the
-          // row sits at chunk (g & 7) ^ (row & 7) of region g / 8
-          uint32_t pk[4];
+          uint32_t pk[16];   // bf16: 16 words of 2 keys; e4m3: 8 words of 4 keys
           float e0 = 0.f, e1 = 0.f;
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
@@ -425,24 +420,22 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
             acc2[i & 3] = f2_add(acc2[i & 3], f2_pack(p0, p1));
             if (FP8) {
               if (i & 1) {
-                pk[(i >> 1) & 3] = pack_e4m3x4(e0, e1, p0, p1);   // keys 2i-2 .. 2i+1 of the chunk
-                if ((i & 7) == 7) {
-                  const int g = 2 * c + (i >> 3);
-                  *reinterpret_cast<uint4*>(p_row + ((g ^ (row & 7)) << 4)) =
-                      make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                }
+                pk[i >> 1] = pack_e4m3x4(e0, e1, p0, p1);   // keys 2i-2 .. 2i+1 of the chunk
               } else {
                 e0 = p0;
                 e1 = p1;
               }
             } else {
-              pk[i & 3] = pack_bf16x2(p0, p1);
-              if ((i & 3) == 3) {
-                const int g = 4 * c + (i >> 2);
-                *reinterpret_cast<uint4*>(p_row + (g >> 3) * FA_HALF + (((g & 7) ^ (row & 7)) << 4)) =
-                    make_uint4(pk[0], pk[1], pk[2], pk[3]);
-              }
+              pk[i] = pack_bf16x2(p0, p1);
             }
+          }
+          if (FP8) {
+            uint32_t q8[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) q8[u] = pk[u];
+            tmem_st8(tS + c * 8, q8);     // P (e4m3) over the first 32 columns of S
+          } else {
+            tmem_st16(tS + c * 16, pk);   // P (bf16) over the first 64 columns of S
           }
         }
         {
@@ -454,11 +447,12 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         if (j == 0 || attempt == 1) break;
         const float mx2 = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
         const bool grow = mx2 > m_ref + 8.0f;
-        // The O rescale is a warp-collective TMEM access, so the decision is
-        // taken per warp: if any row of the warp moved its reference, the
-        // whole warp rescales (factor 1 for the other rows) and recomputes P
-        // (the same values for the other rows).  O is complete up to tile
-        // j-1 (pv_done above) and PV(j) waits for this tile's P.
+        // The O rescale and the P stores are warp-collective TMEM accesses,
+        // so the decision is taken per warp: if any row of the warp moved its
+        // reference, the whole warp rescales (factor 1 for the other rows)
+        // and recomputes P (the same values for the other rows).  O is
+        // complete up to tile j-1: the commit that released S_X(j) covers
+        // every earlier MMA.
         if (!__any_sync(0xffffffffu, grow)) break;
         float f = 1.0f;
         if (grow) {
@@ -467,6 +461,7 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
           l *= f;
           m_ref = m_new;
         }
+        tmem_st_wait();   // this attempt's P stores land before the next ones
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t o[32];
@@ -478,12 +473,9 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         tmem_st_wait();
       }
       l += sum;
-      // P(j) in shared memory (generic writes made visible to the tensor
-      // core's async proxy) and any O rescale landed: PV(j) may run
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      tmem_st_wait();
       tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[X]);
+      mbar_arrive(&p_full[X]);
     }
     ok = __all_sync(0xffffffffu, ok);
     if (ok && n_kv > 0 && mbar_wait_warp(o_full, 0, status)) {
