@@ -244,7 +244,7 @@ namespace qi {
 
 bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, uint64_t inner,
                   uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner,
-                  uint32_t box_outer) {
+                  uint32_t box_outer, bool swizzle128) {
   static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
   if (!encode) {
     void* fn = nullptr;
@@ -260,7 +260,8 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, ui
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
   const CUresult r = encode(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
-                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -699,8 +700,8 @@ int check_mx(const qi_mxfp4* w, const char* name, int n, int k) {
   if ((n >= 0 && w->n != n) || (k >= 0 && w->k != k))
     return fail(QI_ERR_UNSUPPORTED_SHAPE, "MXFP4 weight %s is [%d, %d], expected [%d, %d]", name,
                 w->n, w->k, n, k);
-  if (w->k < 64 || w->k % 64 != 0 || w->n < 256 || w->n % 256 != 0)
-    return fail(QI_ERR_UNSUPPORTED_SHAPE, "MXFP4 weight %s: need k %% 64 == 0 and n %% 256 == 0",
+  if (w->k < 256 || w->k % 256 != 0 || w->n < 256 || w->n % 256 != 0)
+    return fail(QI_ERR_UNSUPPORTED_SHAPE, "MXFP4 weight %s: need k %% 256 == 0 and n %% 256 == 0",
                 name);
   if (!aligned16(w->packed) || !aligned16(w->scales) || (w->bias && !aligned16(w->bias)))
     return fail(QI_ERR_ALIGNMENT, "MXFP4 weight %s: pointers must be 16-byte aligned", name);

@@ -607,7 +607,12 @@ constexpr int PAIR_B_BYTES = 128 * GEMM_BK_BYTES;
 constexpr int PAIR_STAGE_BYTES = PAIR_A_BYTES + PAIR_B_BYTES;
 constexpr int PAIR_COL_BYTES = 2 * 256 * 12;
 constexpr int PAIR_SMEM_BYTES = 1024 + PAIR_STAGES * PAIR_STAGE_BYTES + 256 + PAIR_COL_BYTES;
-static_assert(2 * PAIR_STAGES + 8 <= 32, "barrier area");
+static_assert(3 * PAIR_STAGES + 8 <= 32, "barrier area");
+// MXFP4 B operand: each stage's E2M1 codes of this CTA's 128 B rows (32 bytes a
+// row) are brought in by TMA before the converter warps decode them
+constexpr int MX_CODE_BYTES = 128 * 32;
+constexpr int PAIR_SMEM_BYTES_MX = PAIR_SMEM_BYTES + PAIR_STAGES * MX_CODE_BYTES;
+static_assert(PAIR_SMEM_BYTES_MX <= 232448, "shared memory per CTA");
 
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
@@ -830,6 +835,8 @@ __global__ void __launch_bounds__(MXB ? GEMM_THREADS + 32 * MX_WARPS : GEMM_THRE
   float* col_sw = reinterpret_cast<float*>(smem + PAIR_STAGES * PAIR_STAGE_BYTES + 256);   // [2][BN]
   int32_t* col_rs = reinterpret_cast<int32_t*>(col_sw + 2 * BN);                            // [2][BN]
   float* col_b = reinterpret_cast<float*>(col_rs + 2 * BN);                                 // [2][BN]
+  uint8_t* sC = reinterpret_cast<uint8_t*>(col_b + 2 * BN);    // MXB: [STAGES][128 rows][32 B] codes
+  uint64_t* c_full = bars + 2 * PAIR_STAGES + 8;               // MXB: [STAGES] codes landed (own CTA)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -845,6 +852,7 @@ __global__ void __launch_bounds__(MXB ? GEMM_THREADS + 32 * MX_WARPS : GEMM_THRE
     for (int s = 0; s < PAIR_STAGES; ++s) {
       mbar_init(&full[s], MXB ? 1 + 2 * MX_WARPS : 1);   // + the converter warps of both CTAs
       mbar_init(&empty[s], 1);
+      if (MXB) mbar_init(&c_full[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
@@ -856,7 +864,7 @@ __global__ void __launch_bounds__(MXB ? GEMM_THREADS + 32 * MX_WARPS : GEMM_THRE
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmA);
-    if (!MXB) prefetch_tmap(&tmB);
+    prefetch_tmap(&tmB);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, 2 * BN);
@@ -886,8 +894,13 @@ __global__ void __launch_bounds__(MXB ? GEMM_THREADS + 32 * MX_WARPS : GEMM_THRE
           if (rank == 0) mbar_arrive_expect_tx(&full[stage], MXB ? 2 * PAIR_A_BYTES : 2 * PAIR_STAGE_BYTES);
           // one 128-byte K row per stage: 128 int8 or 64 bf16 elements
           tma_load_2d_pair(&tmA, fb, sA + stage * PAIR_A_BYTES, kb * (I8 ? 128 : 64), m0);
-          if (!MXB)
+          if (!MXB) {
             tma_load_2d_pair(&tmB, fb, sB + stage * PAIR_B_BYTES, kb * (I8 ? 128 : 64), n0);
+          } else {
+            // this CTA's rows of the stage's MXFP4 codes, for its converter warps
+            mbar_arrive_expect_tx(&c_full[stage], MX_CODE_BYTES);
+            tma_load_2d(&tmB, &c_full[stage], sC + stage * MX_CODE_BYTES, kb * 32, n0);
+          }
           if (++stage == PAIR_STAGES) { stage = 0; phase ^= 1u; }
         }
       }
@@ -896,6 +909,14 @@ __global__ void __launch_bounds__(MXB ? GEMM_THREADS + 32 * MX_WARPS : GEMM_THRE
         // even CTA waits (bounded) on the full barriers it armed, which also
         // count the odd CTA's bytes; the odd CTA, which cannot wait on the even
         // CTA's barriers, gives its last loads a fixed 200 us.
+        if (MXB) {   // this CTA's own code loads
+          for (int s = 0; s < PAIR_STAGES; ++s) {
+            const uint32_t par = (s < stage) ? phase : (phase ^ 1u);
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(&c_full[s], par) && globaltimer_ns() - t0 < QI_WAIT_NS) {
+            }
+          }
+        }
         if (rank == 0) {
           for (int s = 0; s < PAIR_STAGES; ++s) {
             const uint32_t par = (s < stage) ? phase : (phase ^ 1u);
@@ -957,13 +978,11 @@ __global__ void __launch_bounds__(MXB ? GEMM_THREADS + 32 * MX_WARPS : GEMM_THRE
     }
   } else if (MXB && warp >= 2 + GEMM_EPI_WARPS) {
     // ------------------------------------------------------------ MXFP4 converters (both CTAs)
-    // thread t decodes row n0 + t of this CTA's B half: per stage its 64
-    // codes (32 bytes) and their two E8M0 scales.  The loads run MX_DEPTH
-    // stages ahead in a register ring, so the L2 latency of one stage's codes
-    // is hidden behind the decoding of the stages before it.
-    constexpr int MX_DEPTH = 4;
+    // thread t decodes row n0 + t of this CTA's B half: per stage the row's 64
+    // codes (32 bytes, brought to shared memory by the producer's TMA) and its
+    // two E8M0 scales (read 8 bytes = 4 stages at a time, one batch ahead)
     const int t = threadIdx.x - 32 * (2 + GEMM_EPI_WARPS);
-    const size_t kh = static_cast<size_t>(p.K) / 2, kscl = static_cast<size_t>(p.K) / 32;
+    const size_t kscl = static_cast<size_t>(p.K) / 32;
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
@@ -972,60 +991,46 @@ __global__ void __launch_bounds__(MXB ? GEMM_THREADS + 32 * MX_WARPS : GEMM_THRE
       tile_coords(tile, m_tiles, p.group_m, n_tiles, mt, nt);
       const int n = nt * BN + static_cast<int>(rank) * (BN / 2) + t;
       const bool n_ok = n < p.N;
-      const uint4* prow = reinterpret_cast<const uint4*>(p.b_packed + (n_ok ? n : 0) * kh);
-      const uint16_t* srow = reinterpret_cast<const uint16_t*>(p.b_scales + (n_ok ? n : 0) * kscl);
-      uint4 ca[MX_DEPTH], cb[MX_DEPTH];
-      uint32_t sc[MX_DEPTH];
-#pragma unroll
-      for (int u = 0; u < MX_DEPTH; ++u) {
-        ca[u] = cb[u] = make_uint4(0, 0, 0, 0);
-        sc[u] = 0;
-        if (n_ok && u < num_kb) {
-          ca[u] = __ldg(prow + 2 * u);
-          cb[u] = __ldg(prow + 2 * u + 1);
-          sc[u] = __ldg(srow + u);
-        }
-      }
+      const uint2* srow = reinterpret_cast<const uint2*>(p.b_scales + (n_ok ? n : 0) * kscl);
+      uint2 sc_next = n_ok ? __ldg(srow) : make_uint2(0, 0);
+      uint2 sc_cur = sc_next;
 #pragma unroll 1
-      for (int kb0 = 0; kb0 < num_kb && ok; kb0 += MX_DEPTH) {
-#pragma unroll
-        for (int u = 0; u < MX_DEPTH; ++u) {
-          const int kb = kb0 + u;
-          if (kb >= num_kb) break;
-          const uint4 d0 = ca[u], d1 = cb[u];
-          const uint32_t dsc = sc[u];
-          if (n_ok && kb + MX_DEPTH < num_kb) {
-            ca[u] = __ldg(prow + 2 * (kb + MX_DEPTH));
-            cb[u] = __ldg(prow + 2 * (kb + MX_DEPTH) + 1);
-            sc[u] = __ldg(srow + kb + MX_DEPTH);
-          }
-          uint32_t o[32];
-          {
-            uint32_t a[16], b[16];
-            mx_decode32(dsc & 0xFFu, d0, a);
-            mx_decode32(dsc >> 8, d1, b);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              o[i] = n_ok ? a[i] : 0u;
-              o[16 + i] = n_ok ? b[i] : 0u;
-            }
-          }
-          if (!mbar_wait_warp(&empty[stage], phase ^ 1u, p.status)) { ok = false; break; }
-          // 128-byte swizzle: 16-byte chunk c of row t goes to chunk c ^ (t & 7)
-          uint8_t* row = sB + stage * PAIR_B_BYTES + t * 128;
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4*>(row + ((c ^ (t & 7)) << 4)) =
-                make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          __syncwarp();
-          if (lane == 0) {
-            const uint32_t fr = mapa_shared(smem_u32(&full[stage]), 0);
-            asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(fr)
-                         : "memory");
-          }
-          if (++stage == PAIR_STAGES) { stage = 0; phase ^= 1u; }
+      for (int kb = 0; kb < num_kb; ++kb) {
+        if ((kb & 3) == 0) {   // scales of stages kb .. kb+3; prefetch the next four
+          sc_cur = sc_next;
+          if (n_ok && kb + 4 < num_kb) sc_next = __ldg(srow + (kb >> 2) + 1);
         }
+        const uint32_t sw = (kb & 2) ? sc_cur.y : sc_cur.x;
+        const uint32_t dsc = (kb & 1) ? (sw >> 16) : (sw & 0xFFFFu);
+        if (!mbar_wait_warp(&c_full[stage], phase, p.status)) { ok = false; break; }
+        const uint4* code = reinterpret_cast<const uint4*>(sC + stage * MX_CODE_BYTES + t * 32);
+        const uint4 d0 = code[0], d1 = code[1];
+        uint32_t o[32];
+        {
+          uint32_t a[16], b[16];
+          mx_decode32(dsc & 0xFFu, d0, a);
+          mx_decode32(dsc >> 8, d1, b);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            o[i] = n_ok ? a[i] : 0u;
+            o[16 + i] = n_ok ? b[i] : 0u;
+          }
+        }
+        if (!mbar_wait_warp(&empty[stage], phase ^ 1u, p.status)) { ok = false; break; }
+        // 128-byte swizzle: 16-byte chunk c of row t goes to chunk c ^ (t & 7)
+        uint8_t* row = sB + stage * PAIR_B_BYTES + t * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(row + ((c ^ (t & 7)) << 4)) =
+              make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) {
+          const uint32_t fr = mapa_shared(smem_u32(&full[stage]), 0);
+          asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(fr)
+                       : "memory");
+        }
+        if (++stage == PAIR_STAGES) { stage = 0; phase ^= 1u; }
       }
     }
   } else if (warp >= 2 && warp < 2 + GEMM_EPI_WARPS) {
@@ -1090,7 +1095,8 @@ static int pair_capacity() {
   static int cap = -1;   // per instantiation
   if (cap < 0) {
     auto kern = gemm_pair_kernel<I8, EPI, MXB>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PAIR_SMEM_BYTES) != cudaSuccess) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             MXB ? PAIR_SMEM_BYTES_MX : PAIR_SMEM_BYTES) != cudaSuccess) {
       launch_result();
       return cap = 0;
     }
@@ -1102,7 +1108,7 @@ static int pair_capacity() {
     attr[0].val.clusterDim.z = 1;
     cfg.gridDim = dim3(2, 1, 1);
     cfg.blockDim = dim3(MXB ? GEMM_THREADS + 32 * MX_WARPS : GEMM_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = PAIR_SMEM_BYTES;
+    cfg.dynamicSmemBytes = MXB ? PAIR_SMEM_BYTES_MX : PAIR_SMEM_BYTES;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
@@ -1121,7 +1127,8 @@ static int launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const 
   const int tiles = ((p.M + 2 * GEMM_BM - 1) / (2 * GEMM_BM)) * ((p.N + 255) / 256);
   const int pairs = tiles < max_pairs ? tiles : max_pairs;
   launch_pdl(gemm_pair_kernel<I8, EPI, MXB>, dim3(2 * pairs),
-             dim3(MXB ? GEMM_THREADS + 32 * MX_WARPS : GEMM_THREADS), PAIR_SMEM_BYTES, st, 2, ta, tb, p);
+             dim3(MXB ? GEMM_THREADS + 32 * MX_WARPS : GEMM_THREADS),
+             MXB ? PAIR_SMEM_BYTES_MX : PAIR_SMEM_BYTES, st, 2, ta, tb, p);
   return launch_result();
 }
 
@@ -1138,20 +1145,24 @@ static int launch_gemm_mx(int epi, const void* A, int lda, const GemmParams& p, 
     default: return -1;
   }
   max_pairs = max_pairs < num_sms / 2 ? max_pairs : num_sms / 2;
-  if (max_pairs < 1 || p.N % 256 != 0 || p.K % 64 != 0 || (epi == EPI_QKV && p.H % 256 != 0))
+  if (max_pairs < 1 || p.N % 256 != 0 || p.K % 256 != 0 || (epi == EPI_QKV && p.H % 256 != 0))
     return -1;
   GemmParams q = p;
   const int m_tiles = (p.M + 2 * GEMM_BM - 1) / (2 * GEMM_BM);
   q.group_m = m_tiles;   // B is small (4.25 bits per weight); A stays in L2
-  CUtensorMap ta;
+  CUtensorMap ta, tc;
   if (!make_tmap_2d(&ta, A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<uint64_t>(p.K),
                     static_cast<uint64_t>(p.M), static_cast<uint64_t>(lda) * 2, 64, GEMM_BM))
     return -2;
+  // the packed codes [N, K/2] bytes: a box of 32 bytes (one stage) x 128 rows, unswizzled
+  if (!make_tmap_2d(&tc, p.b_packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, static_cast<uint64_t>(p.K) / 2,
+                    static_cast<uint64_t>(p.N), static_cast<uint64_t>(p.K) / 2, 32, 128, false))
+    return -2;
   switch (epi) {
-    case EPI_BF16: return launch_gemm_pair<false, EPI_BF16, true>(ta, ta, q, max_pairs, st);
-    case EPI_GELU: return launch_gemm_pair<false, EPI_GELU, true>(ta, ta, q, max_pairs, st);
-    case EPI_GATED: return launch_gemm_pair<false, EPI_GATED, true>(ta, ta, q, max_pairs, st);
-    case EPI_QKV: return launch_gemm_pair<false, EPI_QKV, true>(ta, ta, q, max_pairs, st);
+    case EPI_BF16: return launch_gemm_pair<false, EPI_BF16, true>(ta, tc, q, max_pairs, st);
+    case EPI_GELU: return launch_gemm_pair<false, EPI_GELU, true>(ta, tc, q, max_pairs, st);
+    case EPI_GATED: return launch_gemm_pair<false, EPI_GATED, true>(ta, tc, q, max_pairs, st);
+    case EPI_QKV: return launch_gemm_pair<false, EPI_QKV, true>(ta, tc, q, max_pairs, st);
   }
   return -1;
 }

@@ -115,11 +115,11 @@ struct GemmParams {
   int* status;            // device status word
 };
 
-// TMA descriptor for a row-major 2-D tensor [outer, inner] with a 128-byte
-// swizzled box of box_inner x box_outer elements.
+// TMA descriptor for a row-major 2-D tensor [outer, inner] with a box of
+// box_inner x box_outer elements, 128-byte swizzled unless swizzle128 is false.
 bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, uint64_t inner,
                   uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner,
-                  uint32_t box_outer);
+                  uint32_t box_outer, bool swizzle128 = true);
 
 int pick_block_n(int N);
 int launch_gemm(bool int8, int epi, const void* A, int lda, const void* B, int ldb,

@@ -150,7 +150,7 @@ typedef struct qi_dims {
  * exact in bf16; E8M0 255 decodes to NaN) and accumulates in fp32 on tcgen05
  * kind::f16, so HBM holds 4.25 bits per weight and no decoded copy exists.
  *   packed [n, k/2] bytes, scales [n, k/32] bytes, bias [n] bf16 or NULL;
- *   k % 64 == 0, n % 256 == 0; packed and scales 16-byte aligned. */
+ *   k % 256 == 0, n % 256 == 0; packed and scales 16-byte aligned. */
 typedef struct qi_mxfp4 {
   const uint8_t* packed;
   const uint8_t* scales;

@@ -34,7 +34,7 @@ def _oracle(a, packed, scales, b):
     return O.bf16_linear(bf16_np(a), w, bf16_np(b))
 
 
-@pytest.mark.parametrize("M,N,K", [(1, 256, 64), (77, 512, 128), (300, 768, 4096),
+@pytest.mark.parametrize("M,N,K", [(1, 256, 256), (77, 512, 512), (300, 768, 4096),
                                    (1280, 4096, 16384), (1000, 16384, 4096)])
 def test_mxfp4_linear_vs_oracle(ctx, M, N, K):
     a, packed, scales, b = _case(M, N, K, M + N + K)
@@ -70,13 +70,14 @@ def test_mxfp4_linear_extreme_scales(ctx):
 
 
 def test_mxfp4_linear_rejects_bad_shapes(ctx):
-    a, packed, scales, b = _case(8, 256, 64, 1)
-    w = qi.mx_struct(cuda(packed), cuda(scales), cuda(b))
-    w.n = 128   # n % 256 != 0
-    with pytest.raises(qi.QiError) as e:
-        qi.qi_mxfp4_linear(ctx, cuda(a), w, y=torch.empty((8, 256), dtype=torch.bfloat16,
-                                                           device="cuda"))
-    assert e.value.code == qi.QI_ERR_UNSUPPORTED_SHAPE
+    a, packed, scales, b = _case(8, 256, 256, 1)
+    y = torch.empty((8, 256), dtype=torch.bfloat16, device="cuda")
+    for field, bad in (("n", 128), ("k", 128)):   # n % 256 != 0, k % 256 != 0
+        w = qi.mx_struct(cuda(packed), cuda(scales), cuda(b))
+        setattr(w, field, bad)
+        with pytest.raises(qi.QiError) as e:
+            qi.qi_mxfp4_linear(ctx, cuda(a)[:, :w.k].contiguous(), w, y=y)
+        assert e.value.code == qi.QI_ERR_UNSUPPORTED_SHAPE
 
 
 def _block(ctx, cfg):
