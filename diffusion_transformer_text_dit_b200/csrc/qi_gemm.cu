@@ -980,7 +980,11 @@ __global__ void __launch_bounds__(MXB ? GEMM_THREADS + 32 * MX_WARPS : GEMM_THRE
     // ------------------------------------------------------------ MXFP4 converters (both CTAs)
     // thread t decodes row n0 + t of this CTA's B half: per stage the row's 64
     // codes (32 bytes, brought to shared memory by the producer's TMA) and its
-    // two E8M0 scales (read 8 bytes = 4 stages at a time, one batch ahead)
+    // two E8M0 scales (read 8 bytes = 4 stages at a time, one batch ahead).
+    // Stages are filled two at a time: one proxy fence and one arrival per
+    // stage pair, so the hand-over to the tensor core is paid half as often.
+    constexpr int MX_BATCH = 2;
+    static_assert(PAIR_STAGES % MX_BATCH == 0, "stage pairs must not straddle the ring");
     const int t = threadIdx.x - 32 * (2 + GEMM_EPI_WARPS);
     const size_t kscl = static_cast<size_t>(p.K) / 32;
     int stage = 0;
@@ -995,42 +999,53 @@ __global__ void __launch_bounds__(MXB ? GEMM_THREADS + 32 * MX_WARPS : GEMM_THRE
       uint2 sc_next = n_ok ? __ldg(srow) : make_uint2(0, 0);
       uint2 sc_cur = sc_next;
 #pragma unroll 1
-      for (int kb = 0; kb < num_kb; ++kb) {
-        if ((kb & 3) == 0) {   // scales of stages kb .. kb+3; prefetch the next four
+      for (int kb0 = 0; kb0 < num_kb; kb0 += MX_BATCH) {   // num_kb % 4 == 0 (k % 256 == 0)
+        if ((kb0 & 3) == 0) {   // scales of stages kb0 .. kb0+3; prefetch the next four
           sc_cur = sc_next;
-          if (n_ok && kb + 4 < num_kb) sc_next = __ldg(srow + (kb >> 2) + 1);
+          if (n_ok && kb0 + 4 < num_kb) sc_next = __ldg(srow + (kb0 >> 2) + 1);
         }
-        const uint32_t sw = (kb & 2) ? sc_cur.y : sc_cur.x;
-        const uint32_t dsc = (kb & 1) ? (sw >> 16) : (sw & 0xFFFFu);
-        if (!mbar_wait_warp(&c_full[stage], phase, p.status)) { ok = false; break; }
-        const uint4* code = reinterpret_cast<const uint4*>(sC + stage * MX_CODE_BYTES + t * 32);
-        const uint4 d0 = code[0], d1 = code[1];
-        uint32_t o[32];
-        {
+        uint32_t o[MX_BATCH][32];
+#pragma unroll
+        for (int u = 0; u < MX_BATCH; ++u) {
+          const int kb = kb0 + u;
+          const uint32_t sw = (kb & 2) ? sc_cur.y : sc_cur.x;
+          const uint32_t dsc = (kb & 1) ? (sw >> 16) : (sw & 0xFFFFu);
+          if (!mbar_wait_warp(&c_full[stage + u], phase, p.status)) { ok = false; break; }
+          const uint4* code = reinterpret_cast<const uint4*>(sC + (stage + u) * MX_CODE_BYTES + t * 32);
+          const uint4 d0 = code[0], d1 = code[1];
           uint32_t a[16], b[16];
           mx_decode32(dsc & 0xFFu, d0, a);
           mx_decode32(dsc >> 8, d1, b);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            o[i] = n_ok ? a[i] : 0u;
-            o[16 + i] = n_ok ? b[i] : 0u;
+            o[u][i] = n_ok ? a[i] : 0u;
+            o[u][16 + i] = n_ok ? b[i] : 0u;
           }
         }
-        if (!mbar_wait_warp(&empty[stage], phase ^ 1u, p.status)) { ok = false; break; }
-        // 128-byte swizzle: 16-byte chunk c of row t goes to chunk c ^ (t & 7)
-        uint8_t* row = sB + stage * PAIR_B_BYTES + t * 128;
+        if (!ok) break;
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<uint4*>(row + ((c ^ (t & 7)) << 4)) =
-              make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+        for (int u = 0; u < MX_BATCH; ++u) {
+          if (!mbar_wait_warp(&empty[stage + u], phase ^ 1u, p.status)) { ok = false; break; }
+          // 128-byte swizzle: 16-byte chunk c of row t goes to chunk c ^ (t & 7)
+          uint8_t* row = sB + (stage + u) * PAIR_B_BYTES + t * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(row + ((c ^ (t & 7)) << 4)) =
+                make_uint4(o[u][4 * c], o[u][4 * c + 1], o[u][4 * c + 2], o[u][4 * c + 3]);
+        }
+        if (!ok) break;
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
         if (lane == 0) {
-          const uint32_t fr = mapa_shared(smem_u32(&full[stage]), 0);
-          asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(fr)
-                       : "memory");
+#pragma unroll
+          for (int u = 0; u < MX_BATCH; ++u) {
+            const uint32_t fr = mapa_shared(smem_u32(&full[stage + u]), 0);
+            asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(fr)
+                         : "memory");
+          }
         }
-        if (++stage == PAIR_STAGES) { stage = 0; phase ^= 1u; }
+        stage += MX_BATCH;
+        if (stage == PAIR_STAGES) { stage = 0; phase ^= 1u; }
       }
     }
   } else if (warp >= 2 && warp < 2 + GEMM_EPI_WARPS) {
