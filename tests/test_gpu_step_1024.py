@@ -6,11 +6,22 @@ reference | 4096 target]: a first step that writes the text + reference K/V,
 then a second step that reads them and processes the target rows only) are
 compared with velocities the float64 oracle computed on the same seeded
 inputs (tests/golden/make_step_goldens.py; the oracle needs 10-30 minutes per
-step, so its outputs are stored).  Tolerance: rel-L2 <= 2e-2 on v after the
-32-block stack.  The Euler update must be bit-exact given the GPU's own v
-(RGBA-Image-2.1 Core AI port, "Graph contracts", Sampler), and the cached
-second step must equal the uncached one bit for bit ("Qwen Image 2.1 native
-qualification", "Numerical checks": cached vs uncached second steps).
+step, so its outputs are stored).  The Euler update must be bit-exact given
+the GPU's own v (RGBA-Image-2.1 Core AI port, "Graph contracts", Sampler),
+and the cached second step must equal the uncached one bit for bit ("Qwen
+Image 2.1 native qualification", "Numerical checks": cached vs uncached
+second steps).
+
+Tolerances.  The BF16 path (every block Linear in BF16) must be within rel-L2
+2e-2 of the oracle after the 32-block stack.  The W8A8 stack re-quantizes
+every activation per token in every block, so a rounding-sized difference
+anywhere flips int8 codes and the flips compound over 32 blocks: the oracle
+itself moves v by ``s`` (tests/golden/step_1024px_sensitivity.json, the oracle
+run again on latents moved by one fp32 ulp each) when its input changes by
+one ulp.  Two correct implementations that round differently are each such a
+perturbation of the exact quantized step, so they may differ by about
+sqrt(2) s; the W8A8 stack is held to max(2e-2, 2 s).  Every block on its own
+is held to 1e-2 at full width (the teacher-forced test below).
 """
 import json
 import os
@@ -83,6 +94,13 @@ def _check_inputs(cfg, meta):
     assert meta["inputs"] == input_hashes(cfg), "the seeded inputs changed since the oracle ran"
 
 
+def w8a8_stack_tolerance() -> float:
+    """max(2e-2, 2 x the oracle's one-ulp sensitivity of v after 32 W8A8 blocks)."""
+    with open(os.path.join(GOLDEN, "step_1024px_sensitivity.json")) as f:
+        s = json.load(f)["steps"][0]["v_rel_l2_vs_step_1024px"]
+    return max(2e-2, 2.0 * s)
+
+
 def test_step_1024px_vs_oracle(ctx, model):
     cfg = synth.STEP1024
     meta, (ov,) = _golden("step_1024px")
@@ -91,8 +109,29 @@ def test_step_1024px_vs_oracle(ctx, model):
     lat0 = synth.latents(cfg).numpy()
     lat1, v = Run(ctx, model, cfg).step(lat0, st["sigma"], st["sigma_next"], qi.QI_KV_NONE)
     assert np.all(np.isfinite(v))
+    err, tol = rel_l2(v, ov), w8a8_stack_tolerance()
+    assert err <= tol, f"v rel-L2 {err:.3e} after 32 W8A8 blocks (tolerance {tol:.3e})"
+    assert np.array_equal(lat1, O.euler_update(lat0, v, st["sigma"], st["sigma_next"]))
+
+
+def test_step_1024px_bf16_path_vs_oracle(ctx):
+    """The same step with every block Linear in BF16: within rel-L2 2e-2 of
+    the oracle's BF16 step after the 32-block stack."""
+    cfg = synth.STEP1024_BF16
+    meta, (ov,) = _golden("step_1024px_bf16")
+    _check_inputs(cfg, meta)
+    st = meta["steps"][0]
+    blocks = [qi.BlockWeights(ctx, synth.block_weights(cfg, l),
+                              precision=synth.linear_precision(cfg, l)) for l in range(cfg.blocks)]
+    dims = qi.dims_struct(cfg.hidden, cfg.heads, cfg.mlp, cfg.patch, cfg.blocks)
+    m = qi.Model(ctx, dims, blocks, synth.model_weights(cfg))
+    lat0 = synth.latents(cfg).numpy()
+    lat1, v = Run(ctx, m, cfg).step(lat0, st["sigma"], st["sigma_next"], qi.QI_KV_NONE)
+    del m, blocks
+    torch.cuda.empty_cache()
+    assert np.all(np.isfinite(v))
     err = rel_l2(v, ov)
-    assert err <= 2e-2, f"v rel-L2 {err:.3e} after 32 blocks"
+    assert err <= 2e-2, f"v rel-L2 {err:.3e} after 32 BF16 blocks"
     assert np.array_equal(lat1, O.euler_update(lat0, v, st["sigma"], st["sigma_next"]))
 
 
@@ -141,15 +180,16 @@ def test_edit_1024px_write_then_cached_step_vs_oracle(ctx, model):
     lat0 = synth.latents(cfg).numpy()
     # first step: every token processed, the text + reference K/V kept
     lat1, v1 = r.step(lat0, s1["sigma"], s1["sigma_next"], qi.QI_KV_WRITE_PREFIX)
+    tol = w8a8_stack_tolerance()
     err1 = rel_l2(v1, ov1)
-    assert np.all(np.isfinite(v1)) and err1 <= 2e-2, f"step 1 v rel-L2 {err1:.3e}"
+    assert np.all(np.isfinite(v1)) and err1 <= tol, f"step 1 v rel-L2 {err1:.3e} (tol {tol:.3e})"
     assert np.array_equal(lat1, O.euler_update(lat0, v1, s1["sigma"], s1["sigma_next"]))
     # second step from the oracle's step-1 latents: the target rows only,
     # attending over the cached prefix K/V of the first step
     olat1 = O.euler_update(lat0, ov1, s1["sigma"], s1["sigma_next"])
     c2, v2 = r.step(olat1, s2["sigma"], s2["sigma_next"], qi.QI_KV_READ_PREFIX)
     err2 = rel_l2(v2, ov2)
-    assert np.all(np.isfinite(v2)) and err2 <= 2e-2, f"cached step 2 v rel-L2 {err2:.3e}"
+    assert np.all(np.isfinite(v2)) and err2 <= tol, f"cached step 2 v rel-L2 {err2:.3e} (tol {tol:.3e})"
     assert np.array_equal(c2, O.euler_update(olat1, v2, s2["sigma"], s2["sigma_next"]))
     # and the uncached second step gives the same latents bit for bit
     u2, _ = r.step(olat1, s2["sigma"], s2["sigma_next"], qi.QI_KV_NONE)
