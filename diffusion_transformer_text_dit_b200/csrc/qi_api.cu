@@ -4,6 +4,7 @@
 #include <cudaTypedefs.h>
 #include <math.h>
 #include <stdarg.h>
+#include <stdint.h>
 #include <stdio.h>
 #include <string.h>
 
@@ -32,6 +33,8 @@ struct qi_ctx {
   int attn_fp8;                  // steps run e4m3 attention (qi_ctx_set_attention_fp8)
   bool taps_on;                  // copy the quantizers' inputs and outputs (qi_ctx_set_block_taps)
   qi_block_taps taps;
+  void* attn_scratch;            // key-range split scratch of qi_attn_block_causal(_fp8)
+  size_t attn_scratch_bytes;
 };
 
 namespace {
@@ -277,6 +280,8 @@ struct QuantExtras {
   const uint16_t* res_y = nullptr;     // LN: residual add x += gate * y first
   const uint16_t* res_gate = nullptr;
   uint32_t* zero_range = nullptr;      // LN: clear these row ranges
+  uint32_t* zero_words = nullptr;      // LN: clear these words (n_zero_words of them)
+  int n_zero_words = 0;
   const uint32_t* range = nullptr;     // plain: producer-published row ranges
   float* u_f32 = nullptr;              // LN: also write the quantized value u (fp32 tap)
   bool quant_too = false;              // LN with u_bf16: quantize as well as write bf16(u)
@@ -308,6 +313,8 @@ int run_quant(qi_ctx* ctx, const void* x, bool xbf16, int M, int K, int ldx,
   p.res_y = ex.res_y;
   p.res_gate = ex.res_gate;
   p.zero_range = ex.zero_range;
+  p.zero_words = ex.n_zero_words > 0 ? ex.zero_words : nullptr;
+  p.n_zero_words = ex.n_zero_words;
   p.range = ex.range;
   p.u_f32 = ex.u_f32;
   p.quant_too = ex.quant_too ? 1 : 0;
@@ -465,8 +472,33 @@ int run_block_multi(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, fl
   // epilogue will publish for the next quantizer.
   const qi_block_taps* tp = ctx->taps_on ? &ctx->taps : nullptr;
   const bool qkv_bf16 = bp.qkv_w8_cols < 3 * H;
+  // The attention's key-range split uses the GELU buffer b.g as scratch (free
+  // until the up projection).  The bytes it may take are those of the
+  // sequence's last group (T_last x F bf16), a bound that does not depend on
+  // which rows this call processes; LN1 clears the split counters.
+  auto split_setup = [&](const SeqAttn& q, qi::AttnParams& ap) {
+    const int start_last = q.gt.n >= 2 ? q.gt.end[q.gt.n - 2] : 0;
+    ap.Sk = q.S;
+    ap.heads = d.heads;
+    ap.groups = q.gt;
+    ap.num_sms = ctx->num_sms;
+    ap.split_scratch = b.g;
+    ap.split_bytes = static_cast<size_t>(q.S - start_last) * F * sizeof(uint16_t);
+  };
+  size_t split_counters = 0;
+  for (int sq = 0; sq < nseq; ++sq) {
+    qi::AttnParams ap;
+    memset(&ap, 0, sizeof(ap));
+    split_setup(seqs[sq], ap);
+    int kh = 0;
+    size_t need = 0, counters = 0;
+    qi::attention_split_plan(ap, &kh, &need, &counters);
+    if (counters > split_counters) split_counters = counters;
+  }
   {
     QuantExtras ex;
+    ex.zero_words = reinterpret_cast<uint32_t*>(b.g);
+    ex.n_zero_words = static_cast<int>(split_counters / 4);
     ex.zero_range = b.o_range;
     ex.u_f32 = tp ? tp->u1 : nullptr;
     ex.quant_too = bp.qkv_w8_cols > 0;
@@ -584,6 +616,7 @@ int run_block_multi(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, fl
     ap.sm_scale = 1.0f / sqrtf(static_cast<float>(d.head_dim));
     ap.groups = q.gt;
     ap.row_range = bp.out_w8 ? b.o_range + 2 * static_cast<size_t>(q.off) : nullptr;
+    split_setup(q, ap);
     ap.status = ctx->status;
     Prof pr(ctx, QI_KCLASS_ATTN, st);
     const int r2 = qi::launch_attention(ap, st);
@@ -890,6 +923,8 @@ int qi_ctx_create(int device, qi_ctx** out) {
   c->attn_fp8 = 0;
   c->taps_on = false;
   memset(&c->taps, 0, sizeof(c->taps));
+  c->attn_scratch = nullptr;
+  c->attn_scratch_bytes = 0;
   for (int i = 0; i < QI_PROF_CLASSES; ++i) c->launches[i] = 0;
   if (cudaMalloc(&c->status, 256) != cudaSuccess) {
     delete c;
@@ -912,6 +947,7 @@ int qi_ctx_destroy(qi_ctx* ctx) {
     delete[] ctx->prof_cls;
   }
   cudaFree(ctx->status);
+  if (ctx->attn_scratch) cudaFree(ctx->attn_scratch);
   delete ctx;
   return QI_OK;
 }
@@ -1148,6 +1184,32 @@ int attn_call(qi_ctx* ctx, const void* q, int ldq, int Sq, int q_offset, const v
   p.sm_scale = sm_scale;
   p.groups = gt;
   p.status = ctx->status;
+  p.num_sms = ctx->num_sms;
+  {
+    // key-range split scratch: owned by the context, grown on first need;
+    // its counters are cleared before every launch
+    int kh = 0;
+    size_t need = 0, counters = 0;
+    p.split_bytes = SIZE_MAX;
+    qi::attention_split_plan(p, &kh, &need, &counters);
+    if (kh > 0 && need > ctx->attn_scratch_bytes) {
+      if (ctx->attn_scratch) cudaFree(ctx->attn_scratch);
+      ctx->attn_scratch = nullptr;
+      ctx->attn_scratch_bytes = 0;
+      if (cudaMalloc(&ctx->attn_scratch, need) != cudaSuccess)
+        return cuda_fail("cudaMalloc(attention split scratch)");
+      ctx->attn_scratch_bytes = need;
+    }
+    if (kh > 0) {
+      if (cudaMemsetAsync(ctx->attn_scratch, 0, counters, S(stream)) != cudaSuccess)
+        return cuda_fail("attention split counters");
+      p.split_scratch = ctx->attn_scratch;
+      p.split_bytes = ctx->attn_scratch_bytes;
+    } else {
+      p.split_scratch = nullptr;
+      p.split_bytes = 0;
+    }
+  }
   {
     Prof pr(ctx, QI_KCLASS_ATTN, S(stream));
     const int r2 = qi::launch_attention(p, S(stream));
@@ -1158,6 +1220,25 @@ int attn_call(qi_ctx* ctx, const void* q, int ldq, int Sq, int q_offset, const v
 }
 
 }  // namespace
+
+int qi_attn_split_plan(int Sk, int heads, const qi_groups* groups, int num_sms,
+                       size_t scratch_bytes, int* split_heads, size_t* bytes) {
+  if (!split_heads || !bytes) return fail(QI_ERR_INVALID_ARG, "NULL output");
+  if (Sk < 1 || heads < 1 || num_sms < 1) return fail(QI_ERR_INVALID_ARG, "need Sk, heads, num_sms >= 1");
+  qi::GroupTable gt;
+  int r;
+  if ((r = check_groups(groups, Sk, &gt))) return r;
+  qi::AttnParams p;
+  memset(&p, 0, sizeof(p));
+  p.Sk = Sk;
+  p.heads = heads;
+  p.groups = gt;
+  p.num_sms = num_sms;
+  p.split_bytes = scratch_bytes;
+  size_t counters = 0;
+  qi::attention_split_plan(p, split_heads, bytes, &counters);
+  return QI_OK;
+}
 
 int qi_attn_block_causal(qi_ctx* ctx, const uint16_t* q, int ldq, int Sq, int q_offset,
                          const uint16_t* k, const uint16_t* v, int ldkv, int Sk, int heads,

@@ -28,6 +28,22 @@
 // 8 TMA producer, 9 TMEM allocator + MMA issuer.  K streams through a 3-stage
 // ring (a stage is released once both S MMAs have read it), V through a
 // 2-stage ring; every barrier wait is bounded (qi_common.cuh).
+//
+// Work units are (query tile pair, head); the grid is one CTA per unit,
+// heaviest first.  A grid of U units on P SMs (one CTA per SM) leaves its
+// last round partly idle when U mod P is small; the heaviest units of a few
+// whole heads are then split over the key range: two CTAs take key tiles
+// [0, n/2) and [n/2, n), each keeps its own reference maximum and row sum,
+// writes its unnormalised O, maximum and sum to scratch, and the CTA that
+// finishes second (an atomic counter per unit, no waiting) combines them:
+// m = max(m0, m1), O = (O0 2^(m0-m) + O1 2^(m1-m)) / (l0 2^(m0-m) + l1 2^(m1-m)).
+// The split is chosen from the shapes of the sequence, not of the launch, so
+// a row is split the same way in every launch that computes it.
+#include <algorithm>
+#include <functional>
+#include <mutex>
+#include <vector>
+
 #include "qi_common.cuh"
 #include "qi_internal.h"
 
@@ -37,6 +53,7 @@ constexpr int FA_ROWS = 128;                   // rows per Q tile, keys per K/V 
 constexpr int FA_THREADS = 320;
 constexpr int FA_KST = 3;                      // K ring stages
 constexpr int FA_VST = 2;                      // V ring stages
+constexpr int FA_OUT_BOX = FA_ROWS * 128;      // bytes of one staged 64-column bf16 output box
 
 // Tile geometry of the two element types.  A tile is 128 rows x 128 head
 // columns: bf16 -> two 64-column (128-byte) swizzle regions of 16 KB; e4m3 ->
@@ -47,6 +64,7 @@ struct FaCfg {
   static constexpr int REGION = 128 * 128;       // bytes of one 128-byte-wide swizzle region
   static constexpr int REGIONS = TILE / REGION;  // 1 (e4m3) or 2 (bf16)
   static constexpr int SMEM = 1024 + (2 + FA_KST + FA_VST) * TILE + 256;
+  static_assert(4 * FA_OUT_BOX <= (2 + FA_KST) * TILE, "output staging overlaps the V ring");
 };
 
 // tcgen05.mma kind::f8f6f4 with A = B = e4m3 (format 0) and an fp32
@@ -159,10 +177,69 @@ __device__ __forceinline__ int fa_key_limit(const GroupTable& g, int t) {
   return g.end[group_of(g, t)];
 }
 
+// Per-unit scratch of the key-range split (floats per half).
+constexpr int FA_PART_O = 2 * FA_ROWS * 128;   // 256 rows x 128 fp32
+constexpr int FA_PART_ML = 2 * FA_ROWS * 2;    // 256 rows x (maximum, sum)
+
+// Grid index -> (query tile pair, head, half, split unit).  Segments, in
+// launch order: the longest-range tiles of the unsplit heads (tile-major,
+// last tile first), the halves of the split heads' longest-range tiles, the
+// remaining tiles of every head (last tile first).  half = -1: not split.
+struct FaUnit {
+  int ct, h, half, su;
+};
+__device__ __forceinline__ FaUnit fa_unit(const AttnParams& p, int b) {
+  FaUnit u;
+  const int k = p.split_heads, nh = p.n_ctiles - p.ct_heavy;
+  const int seg_a = nh * (p.heads - k), seg_b = 2 * nh * k;
+  u.half = -1;
+  u.su = -1;
+  if (b < seg_a) {
+    u.ct = p.n_ctiles - 1 - b / (p.heads - k);
+    u.h = b % (p.heads - k);
+  } else if (b < seg_a + seg_b) {
+    const int v = b - seg_a;
+    u.half = v & 1;
+    u.su = v >> 1;
+    u.ct = p.n_ctiles - 1 - u.su / k;
+    u.h = p.heads - k + u.su % k;
+  } else {
+    const int v = b - seg_a - seg_b;
+    u.ct = p.ct_heavy - 1 - v / p.heads;
+    u.h = v % p.heads;
+  }
+  return u;
+}
+
+// o f + b g with both products rounded before the sum: symmetric in the two
+// halves of a split unit.
+__device__ __forceinline__ float fa_combine(uint32_t o, float f, float b, float g) {
+  return __fadd_rn(__fmul_rn(__uint_as_float(o), f), __fmul_rn(b, g));
+}
+
+// Named barrier 1 over the 8 softmax warps (threads 0-255): plain, and with
+// an AND of a predicate across them.
+__device__ __forceinline__ void fa_softmax_bar() {
+  asm volatile("bar.sync 1, 256;" ::: "memory");
+}
+__device__ __forceinline__ bool fa_softmax_all(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.b32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, 256, p;\n\t"
+      "selp.b32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred))
+      : "memory");
+  return r != 0;
+}
+
 template <bool FP8>
 __global__ void __launch_bounds__(FA_THREADS, 1)
     fa_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-              const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+              const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+              const AttnParams p) {
   using Cfg = FaCfg<FP8>;
   constexpr int FA_TILE = Cfg::TILE;
   constexpr int FA_HALF = Cfg::REGION;
@@ -184,16 +261,23 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
   uint64_t* o_full = p_full + 2;
   uint64_t* drain = o_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint32_t* order_slot = tmem_slot + 1;   // split: the counter value this CTA saw
+  // output staging for the TMA store, over Q and the first K stages (free
+  // once every MMA has completed): [tile][64-column box][128 rows][128 B]
+  uint8_t* fa_stage = smem;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_ctiles = (p.Sq + 2 * FA_ROWS - 1) / (2 * FA_ROWS);
-  const int ct = n_ctiles - 1 - static_cast<int>(blockIdx.x);   // heavy tiles first
-  const int h = blockIdx.y;
-  const int q0 = ct * 2 * FA_ROWS;
+  const FaUnit unit = fa_unit(p, static_cast<int>(blockIdx.x));
+  const int h = unit.h;
+  const int q0 = unit.ct * 2 * FA_ROWS;
   const int q_last = min(q0 + 2 * FA_ROWS, p.Sq) - 1;
   const int kv_end = min(fa_key_limit(p.groups, p.q_offset + q_last), p.Sk);
   const int kv_min = min(fa_key_limit(p.groups, p.q_offset + q0), p.Sk);
-  const int n_kv = (kv_end + FA_ROWS - 1) / FA_ROWS;
+  const int n_kv_all = (kv_end + FA_ROWS - 1) / FA_ROWS;
+  // key tiles [kv_lo, kv_lo + n_kv) of this CTA; local tile index i drives
+  // every ring stage and barrier phase, kv_lo + i the key coordinates
+  const int kv_lo = unit.half == 1 ? n_kv_all / 2 : 0;
+  const int n_kv = unit.half == 0 ? n_kv_all / 2 : n_kv_all - kv_lo;
   const int hc = h * 128;
 
   if (threadIdx.x == 0) {
@@ -218,6 +302,7 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
     prefetch_tmap(&tmQ);
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
+    prefetch_tmap(&tmO);
   }
   if (warp == 9) {
     tmem_alloc(tmem_slot, 512);
@@ -249,14 +334,14 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         mbar_arrive_expect_tx(&k_full[ks], FA_TILE);
         for (int half = 0; half < Cfg::REGIONS; ++half)
           tma_load_2d(&tmK, &k_full[ks], sK + ks * FA_TILE + half * FA_HALF, hc + 64 * half,
-                      j * FA_ROWS);
+                      (kv_lo + j) * FA_ROWS);
         jk = j + 1;
         const int vs = j % FA_VST, vr = j / FA_VST;
         if (!mbar_wait(&v_empty[vs], (vr & 1) ^ 1u, status)) { ok = false; break; }
         mbar_arrive_expect_tx(&v_full[vs], FA_TILE);
         for (int half = 0; half < Cfg::REGIONS; ++half)
           tma_load_2d(&tmV, &v_full[vs], sV + vs * FA_TILE + half * FA_HALF, hc + 64 * half,
-                      j * FA_ROWS);
+                      (kv_lo + j) * FA_ROWS);
         jv = j + 1;
       }
       if (!ok) {
@@ -367,7 +452,7 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
     for (int j = 0; j < n_kv; ++j) {
       if (!mbar_wait_warp(&s_full[X], j & 1, status)) { ok = false; break; }
       tc_fence_after();
-      const int k0 = j * FA_ROWS;
+      const int k0 = (kv_lo + j) * FA_ROWS;
       const bool masked = k0 + FA_ROWS > kv_min;
       uint32_t r[128];
       tmem_ld128(tS, r);                     // the whole S row, read once
@@ -389,6 +474,10 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
           for (int k = 0; k < 8; ++k)
             m8[k] = fmax3(m8[k], __uint_as_float(r[i + 2 * k]), __uint_as_float(r[i + 2 * k + 1]));
         m_ref = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7])) * sl2;
+        // a row with no key in this CTA's first tile (only the upper half of
+        // a split unit has one: its keys all lie below this key range) gets
+        // P = 2^-inf = 0 throughout and a zero sum
+        if (m_ref == -INFINITY) m_ref = 0.f;
       }
       // P = 2^(s sl2 - m_ref) with the current reference maximum (the
       // scale-subtract as paired fp32 FMAs, the row sum in 4 paired partial
@@ -478,36 +567,136 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
       mbar_arrive(&p_full[X]);
     }
     ok = __all_sync(0xffffffffu, ok);
-    if (ok && n_kv > 0 && mbar_wait_warp(o_full, 0, status)) {
+    // split unit: publish this half's partial, then count; the half that
+    // counts second combines (every softmax warp reaches both barriers: the
+    // o_full wait result is made uniform across them first)
+    bool store = ok && n_kv > 0 && mbar_wait_warp(o_full, 0, status);
+    float* other_o = nullptr;
+    float m_oth = 0.f, l_oth = 0.f;
+    if (unit.half >= 0) {
+      uint32_t* counter = static_cast<uint32_t*>(p.split_scratch) + unit.su;
+      const size_t n_units = static_cast<size_t>(p.n_ctiles - p.ct_heavy) * p.split_heads;
+      float* ml = reinterpret_cast<float*>(static_cast<uint8_t*>(p.split_scratch) +
+                                           ((n_units * 4 + 255) & ~static_cast<size_t>(255)));
+      float* po = ml + n_units * 2 * FA_PART_ML;
+      // partial O layout [32 column quads][256 rows] of float4: the 32 lanes
+      // of a warp (32 consecutive rows) store and load 512 contiguous bytes
+      const int prow = X * FA_ROWS + row;
+      if (store) {
+        tc_fence_after();
+        float4* mine = reinterpret_cast<float4*>(
+            po + (static_cast<size_t>(unit.su) * 2 + unit.half) * FA_PART_O) + prow;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tO + c * 32, r);
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            mine[(c * 8 + v) * 2 * FA_ROWS] =
+                make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                            __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+        }
+        float* mml = ml + (static_cast<size_t>(unit.su) * 2 + unit.half) * FA_PART_ML + prow * 2;
+        mml[0] = m_ref;
+        mml[1] = l;
+      }
+      __threadfence();
+      const bool all = fa_softmax_all(store);
+      if (threadIdx.x == 0) *order_slot = all ? atomicAdd(counter, 1u) : 0u;
+      fa_softmax_bar();
+      store = all && *order_slot == 1u;
+      if (store) {
+        __threadfence();
+        const size_t oth = static_cast<size_t>(unit.su) * 2 + (unit.half ^ 1);
+        other_o = po + oth * FA_PART_O + prow * 4;
+        m_oth = __ldcg(ml + oth * FA_PART_ML + prow * 2);
+        l_oth = __ldcg(ml + oth * FA_PART_ML + prow * 2 + 1);
+        if (threadIdx.x == 0) *counter = 0u;   // ready for the next launch
+      }
+    }
+    if (store) {
       tc_fence_after();
-      const float inv = l > 0.f ? 1.0f / l : 0.f;
+      // this CTA's O is scaled by f_me, the other half's by f_oth, and the
+      // sum of both normalises (an empty half, l = 0, has weight 0).  Products
+      // and sums are rounded separately (no FMA contraction), so the result
+      // does not depend on which half finished second.
+      float f_me = 1.f, f_oth = 0.f, lsum = l;
+      if (other_o) {
+        const float m = fmaxf(l > 0.f ? m_ref : -INFINITY, l_oth > 0.f ? m_oth : -INFINITY);
+        f_me = l > 0.f ? exp2f(m_ref - m) : 0.f;
+        f_oth = l_oth > 0.f ? exp2f(m_oth - m) : 0.f;
+        lsum = __fadd_rn(__fmul_rn(l, f_me), __fmul_rn(l_oth, f_oth));
+      }
+      const float inv = lsum > 0.f ? 1.0f / lsum : 0.f;
       float rlo = 0.f, rhi = 0.f;   // range of the stored bf16 values of this row
+      // the other half's partial is loaded one 32-column chunk ahead
+      const float4* src = reinterpret_cast<const float4*>(other_o);
+      float4 ahead[8];
+      if (other_o) {
+#pragma unroll
+        for (int v = 0; v < 8; ++v) ahead[v] = __ldcg(src + v * 2 * FA_ROWS);
+      }
       // every lane of the warp takes part in the (warp-wide) TMEM loads
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t r[32];
         tmem_ld32(tO + c * 32, r);
-        if (qrow < p.Sq) {
-          uint32_t pk[16];
+        if (other_o) {
+          float4 cur[8];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float a = bf16_round_f(__uint_as_float(r[2 * i]) * inv);
-            const float b = bf16_round_f(__uint_as_float(r[2 * i + 1]) * inv);
-            rlo = fminf(rlo, fminf(a, b));
-            rhi = fmaxf(rhi, fmaxf(a, b));
-            pk[i] = pack_bf16x2(a, b);
+          for (int v = 0; v < 8; ++v) cur[v] = ahead[v];
+          if (c + 1 < 4) {
+#pragma unroll
+            for (int v = 0; v < 8; ++v) ahead[v] = __ldcg(src + ((c + 1) * 8 + v) * 2 * FA_ROWS);
           }
-          uint4* dst = reinterpret_cast<uint4*>(p.o + static_cast<int64_t>(qrow) * p.ldo + hc + c * 32);
 #pragma unroll
-          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          for (int v = 0; v < 8; ++v) {
+            const float4 b = cur[v];
+            r[4 * v] = __float_as_uint(fa_combine(r[4 * v], f_me, b.x, f_oth));
+            r[4 * v + 1] = __float_as_uint(fa_combine(r[4 * v + 1], f_me, b.y, f_oth));
+            r[4 * v + 2] = __float_as_uint(fa_combine(r[4 * v + 2], f_me, b.z, f_oth));
+            r[4 * v + 3] = __float_as_uint(fa_combine(r[4 * v + 3], f_me, b.w, f_oth));
+          }
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float a = bf16_round_f(__uint_as_float(r[2 * i]) * inv);
+          const float b = bf16_round_f(__uint_as_float(r[2 * i + 1]) * inv);
+          rlo = fminf(rlo, fminf(a, b));
+          rhi = fmaxf(rhi, fmaxf(a, b));
+          pk[i] = pack_bf16x2(a, b);
+        }
+        // staged in the TMA store's layout: per tile and 64-column box, 128
+        // rows of 128 bytes, 16-byte chunk j of row r at chunk j ^ (r mod 8)
+        uint8_t* rowp = fa_stage + X * 2 * FA_OUT_BOX + (c >> 1) * FA_OUT_BOX + row * 128;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const int j = (c & 1) * 4 + v;
+          *reinterpret_cast<uint4*>(rowp + ((j ^ (row & 7)) << 4)) =
+              make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
         }
       }
+      fence_proxy_async_smem();
       if (p.row_range && qrow < p.Sq) {
         // per-row range for the next quantizer (non-negative floats order like
         // their bit patterns; negative zero is normalised to +0)
         atomicMax(p.row_range + 2 * static_cast<size_t>(qrow), __float_as_uint(__fsub_rn(0.0f, rlo)));
         atomicMax(p.row_range + 2 * static_cast<size_t>(qrow) + 1, __float_as_uint(__fadd_rn(rhi, 0.0f)));
       }
+    }
+    // every softmax thread arrives here; the staged tiles go out by TMA only
+    // if all of them were staged (rows past Sq are clipped by the store)
+    if (fa_softmax_all(store) && threadIdx.x == 0) {
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        if (q0 + t * FA_ROWS >= p.Sq) break;
+#pragma unroll
+        for (int box = 0; box < 2; ++box)
+          tma_store_2d(&tmO, fa_stage + (2 * t + box) * FA_OUT_BOX, hc + 64 * box, q0 + t * FA_ROWS);
+      }
+      bulk_commit_group();
+      bulk_wait_group_read0();
     }
   }
 
@@ -519,8 +708,134 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
   }
 }
 
+// ---------------------------------------------------------------- split plan
+
+static int host_key_limit(const GroupTable& g, int t) {
+  int k = 0;
+  while (k < g.n - 1 && t >= g.end[k]) ++k;
+  return g.end[k];
+}
+
+// Key tiles of query tile pair ct of a launch.
+static int host_n_kv(const AttnParams& p, int ct) {
+  const int q_last = std::min((ct + 1) * 2 * FA_ROWS, p.Sq) - 1;
+  const int kv_end = std::min(host_key_limit(p.groups, p.q_offset + q_last), p.Sk);
+  return (kv_end + FA_ROWS - 1) / FA_ROWS;
+}
+
+// Finish time of greedy dispatch, in grid order, of `n_full` units of cost
+// c_full and then `n_half` of cost c_half onto `sms` SMs (one CTA each).
+static long fa_makespan(int sms, int n_full, long c_full, int n_half, long c_half) {
+  std::vector<long> t(static_cast<size_t>(sms), 0);   // a min-heap of SM free times
+  auto push = [&](long cost) {
+    std::pop_heap(t.begin(), t.end(), std::greater<long>());
+    t.back() += cost;
+    std::push_heap(t.begin(), t.end(), std::greater<long>());
+  };
+  std::make_heap(t.begin(), t.end(), std::greater<long>());
+  for (int i = 0; i < n_full; ++i) push(c_full);
+  for (int i = 0; i < n_half; ++i) push(c_half);
+  return *std::max_element(t.begin(), t.end());
+}
+
+static size_t fa_split_scratch_bytes(size_t units) {
+  return ((units * 4 + 255) & ~static_cast<size_t>(255)) +
+         units * 2 * (FA_PART_ML + FA_PART_O) * sizeof(float);
+}
+
+// The split depends on the sequence (Sk, the group table), heads, the SM
+// count and the scratch the caller guarantees, never on the launch's query
+// rows.  It models the launch as the last group's query tiles of every head
+// (the rows a cached-prefix launch computes; in an uncached launch they are
+// the longest-range tiles too) and picks the number of whole heads whose
+// tiles are split in two that minimises the modelled finish time: costs in
+// key tiles plus two tiles of fixed work per CTA and one more per split half
+// (the partial write and the combine).  The shorter tiles of earlier groups
+// run after these and are left out of the model.
+static void attention_split_plan_compute(const AttnParams& p, int* split_heads, size_t* bytes,
+                                         size_t* counter_bytes) {
+  *split_heads = 0;
+  *bytes = 0;
+  *counter_bytes = 0;
+  const int n_kv = (p.Sk + FA_ROWS - 1) / FA_ROWS;
+  if (p.num_sms < 2 || n_kv < 8 || p.heads < 1) return;
+  const int start_last = p.groups.n >= 2 ? p.groups.end[p.groups.n - 2] : 0;
+  const int tiles = (p.Sk - start_last + 2 * FA_ROWS - 1) / (2 * FA_ROWS);
+  // capacity for tiles + 1 per head: an uncached launch whose last group does
+  // not start on a tile boundary has one more longest-range tile
+  int k_max = p.heads;
+  while (k_max > 0 && fa_split_scratch_bytes(static_cast<size_t>(tiles + 1) * k_max) > p.split_bytes)
+    --k_max;
+  const long c_full = n_kv + 2, c_half = (n_kv + 1) / 2 + 3;
+  const long base = fa_makespan(p.num_sms, tiles * p.heads, c_full, 0, c_half);
+  long best = base;
+  for (int k = 1; k <= k_max; ++k) {
+    const long t = fa_makespan(p.num_sms, tiles * (p.heads - k), c_full, 2 * tiles * k, c_half);
+    if (t < best) {
+      best = t;
+      *split_heads = k;
+    }
+  }
+  if (best * 100 > base * 97) *split_heads = 0;   // less than 3% modelled gain: no split
+  if (*split_heads > 0) {
+    const size_t units = static_cast<size_t>(tiles + 1) * *split_heads;
+    *bytes = fa_split_scratch_bytes(units);
+    *counter_bytes = units * 4;
+  }
+}
+
+// The plan is a pure function of a few integers; a step asks for the same
+// one in every block, so recent plans are kept (the model simulation costs
+// about a tenth of a millisecond of host time).
+void attention_split_plan(const AttnParams& p, int* split_heads, size_t* bytes,
+                          size_t* counter_bytes) {
+  struct Entry {
+    bool used;
+    int sk, heads, sms, n;
+    int end[16];
+    size_t cap;
+    int k;
+    size_t bytes, counters;
+  };
+  static Entry memo[16];
+  static int next = 0;
+  static std::mutex mu;
+  auto same = [&](const Entry& e) {
+    if (!e.used || e.sk != p.Sk || e.heads != p.heads || e.sms != p.num_sms ||
+        e.cap != p.split_bytes || e.n != p.groups.n)
+      return false;
+    for (int i = 0; i < p.groups.n; ++i)
+      if (e.end[i] != p.groups.end[i]) return false;
+    return true;
+  };
+  {
+    std::lock_guard<std::mutex> g(mu);
+    for (const Entry& e : memo)
+      if (same(e)) {
+        *split_heads = e.k;
+        *bytes = e.bytes;
+        *counter_bytes = e.counters;
+        return;
+      }
+  }
+  attention_split_plan_compute(p, split_heads, bytes, counter_bytes);
+  std::lock_guard<std::mutex> g(mu);
+  Entry& e = memo[next];
+  next = (next + 1) % 16;
+  e.used = true;
+  e.sk = p.Sk;
+  e.heads = p.heads;
+  e.sms = p.num_sms;
+  e.n = p.groups.n;
+  for (int i = 0; i < 16; ++i) e.end[i] = i < p.groups.n ? p.groups.end[i] : 0;
+  e.cap = p.split_bytes;
+  e.k = *split_heads;
+  e.bytes = *bytes;
+  e.counters = *counter_bytes;
+}
+
 template <bool FP8>
-static int launch_attention_t(const AttnParams& p, cudaStream_t st) {
+static int launch_attention_t(const AttnParams& p_in, cudaStream_t st) {
   using Cfg = FaCfg<FP8>;
   static bool attr = false;   // per instantiation
   if (!attr) {
@@ -530,17 +845,34 @@ static int launch_attention_t(const AttnParams& p, cudaStream_t st) {
     }
     attr = true;
   }
+  AttnParams p = p_in;
+  p.n_ctiles = (p.Sq + 2 * FA_ROWS - 1) / (2 * FA_ROWS);
+  // tiles [ct_heavy, n_ctiles) reach the last key tile (the key range grows
+  // with the query position)
+  const int n_kv_max = (p.Sk + FA_ROWS - 1) / FA_ROWS;
+  p.ct_heavy = p.n_ctiles;
+  while (p.ct_heavy > 0 && host_n_kv(p, p.ct_heavy - 1) == n_kv_max) --p.ct_heavy;
+  size_t need = 0, counters = 0;
+  p.split_heads = 0;
+  if (p.split_scratch) attention_split_plan(p, &p.split_heads, &need, &counters);
+  if (p.split_heads > 0 &&
+      fa_split_scratch_bytes(static_cast<size_t>(p.n_ctiles - p.ct_heavy) * p.split_heads) >
+          p.split_bytes)
+    p.split_heads = 0;   // not reached: the plan reserves a tile more than a launch can have
   const int W = p.heads * 128;
   const CUtensorMapDataType dt = FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const uint64_t esz = FP8 ? 1 : 2;
   const uint32_t box = FP8 ? 128 : 64;   // one 128-byte swizzle row per box
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (!make_tmap_2d(&tq, p.q, dt, W, p.Sq, static_cast<uint64_t>(p.ldq) * esz, box, FA_ROWS) ||
       !make_tmap_2d(&tk, p.k, dt, W, p.Sk, static_cast<uint64_t>(p.ldkv) * esz, box, FA_ROWS) ||
-      !make_tmap_2d(&tv, p.v, dt, W, p.Sk, static_cast<uint64_t>(p.ldkv) * esz, box, FA_ROWS))
+      !make_tmap_2d(&tv, p.v, dt, W, p.Sk, static_cast<uint64_t>(p.ldkv) * esz, box, FA_ROWS) ||
+      !make_tmap_2d(&to, p.o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, p.Sq,
+                    static_cast<uint64_t>(p.ldo) * 2, 64, FA_ROWS))
     return -2;
-  dim3 grid((p.Sq + 2 * FA_ROWS - 1) / (2 * FA_ROWS), p.heads);
-  launch_pdl(fa_kernel<FP8>, grid, dim3(FA_THREADS), Cfg::SMEM, st, 1, tq, tk, tv, p);
+  dim3 grid(static_cast<unsigned>(p.n_ctiles * p.heads +
+                                  (p.n_ctiles - p.ct_heavy) * p.split_heads));
+  launch_pdl(fa_kernel<FP8>, grid, dim3(FA_THREADS), Cfg::SMEM, st, 1, tq, tk, tv, to, p);
   return launch_result();
 }
 

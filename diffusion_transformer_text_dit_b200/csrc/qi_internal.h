@@ -147,6 +147,8 @@ struct QuantParams {
   const uint16_t* res_y;  // bf16 [M, K] or null
   const uint16_t* res_gate;   // gate row of set r at res_gate + r * mod_ld
   uint32_t* zero_range;   // if non-null: rows' [2] range words set to 0 (for a later producer)
+  uint32_t* zero_words;   // LN variant, if non-null: n_zero_words words set to 0 (by the first row)
+  int n_zero_words;
   float* u_f32;           // LN variant, if non-null: also write u (the quantized value) [M, ldq] fp32
   // plain variant: the row's range was published by the producer as
   // [float bits of -min, float bits of max] (both >= 0); no reduction needed
@@ -187,8 +189,30 @@ struct AttnParams {
   float sm_scale;
   GroupTable groups;
   uint32_t* row_range;    // optional per-query-row [-min, max] bit patterns of the bf16 output
+  // Key-range split of whole heads.  The query tiles with the longest key
+  // range (ceil(Sk / 128) key tiles) of the last `split_heads` heads run as
+  // two CTAs each, over key tiles [0, n/2) and [n/2, n); each half writes its
+  // unnormalised O, reference maximum and row sum to the scratch, and the
+  // half that finishes second combines the two.  launch_attention chooses
+  // split_heads from Sk, the group table, heads, the SM count and
+  // split_bytes alone, so two launches over the same sequence split the same
+  // rows whatever their query rows (a cached-prefix launch and the uncached
+  // one give identical target rows).  Scratch layout: counters [units]
+  // (must be zero at launch; the combining CTA sets its counter back to 0),
+  // then part_ml [units][2][256 rows][2] and part_o [units][2][32 column
+  // quads][256 rows][4] fp32.
+  void* split_scratch;    // 256-byte aligned device scratch, or null (no split)
+  size_t split_bytes;     // bytes the caller guarantees for it
+  int num_sms;
+  // filled in by launch_attention
+  int n_ctiles, ct_heavy, split_heads;
   int* status;            // device status word
 };
+// Split plan of a launch (reads Sk, groups, heads, num_sms, split_bytes):
+// heads split (0: none), the scratch bytes it may use and, at their start,
+// the bytes of counters that must be zero when the kernel starts.
+void attention_split_plan(const AttnParams& p, int* split_heads, size_t* bytes,
+                          size_t* counter_bytes);
 int launch_attention(const AttnParams& p, cudaStream_t st);
 
 // Thin GEMV for M <= 2 rows (timestep MLP, adaLN rows).

@@ -211,6 +211,8 @@ __global__ void __launch_bounds__(512) quant_ln_kernel(const QuantParams p) {
     p.zero_range[2 * static_cast<int64_t>(row)] = 0u;
     p.zero_range[2 * static_cast<int64_t>(row) + 1] = 0u;
   }
+  if (p.zero_words && row == 0)
+    for (int i = tid; i < p.n_zero_words; i += nt) p.zero_words[i] = 0u;
   const int rs = p.groups.row_set[group_of(p.groups, p.row0 + row)];
   if (!XBF16 && p.res_y) {
     const uint16_t* gt = p.res_gate + static_cast<int64_t>(rs) * p.mod_ld;

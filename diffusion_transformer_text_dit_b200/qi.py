@@ -135,6 +135,8 @@ _SIGS = {
                                  C.c_void_p, C.c_int, C.c_int, C.c_int, C.c_int,
                                  C.POINTER(qi_groups), C.c_float, C.c_void_p, C.c_int, C.c_void_p],
     "qi_to_e4m3": [C.c_void_p, C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p],
+    "qi_attn_split_plan": [C.c_int, C.c_int, C.POINTER(qi_groups), C.c_int, C.c_size_t,
+                           C.POINTER(C.c_int), C.POINTER(C.c_size_t)],
     "qi_ctx_set_attention_fp8": [C.c_void_p, C.c_int],
     "qi_ctx_set_block_taps": [C.c_void_p, C.POINTER(qi_block_taps)],
     "qi_mxfp4_decode": [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_int,
@@ -415,6 +417,16 @@ def qi_attn_block_causal_fp8(ctx: Context, q8, k8, v8, groups: qi_groups, q_offs
                                          ptr(v8), k8.shape[1], Sk, heads, 128, C.byref(groups),
                                          sm_scale, ptr(o), o.shape[1], stream_ptr(stream)))
     return o
+
+
+def qi_attn_split_plan(Sk: int, heads: int, groups: qi_groups, num_sms: int,
+                       scratch_bytes: Optional[int] = None):
+    """(split_heads, scratch bytes) of the attention's key-range split (host only)."""
+    k, nb = C.c_int(0), C.c_size_t(0)
+    sb = (1 << 64) - 1 if scratch_bytes is None else scratch_bytes
+    check(lib().qi_attn_split_plan(Sk, heads, C.byref(groups), num_sms, sb, C.byref(k),
+                                   C.byref(nb)))
+    return k.value, nb.value
 
 
 def qi_to_e4m3(ctx: Context, x: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None):

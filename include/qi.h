@@ -310,6 +310,29 @@ int qi_attn_block_causal(qi_ctx* ctx, const uint16_t* q, int ldq, int Sq, int q_
                          int head_dim, const qi_groups* groups, float sm_scale, uint16_t* o,
                          int ldo, void* stream);
 
+/* The attention calls above and the block and step calls below schedule one
+ * CTA per (256 query rows, head), longest key range first.  When that leaves
+ * the SMs' last round of CTAs mostly idle, the longest-range query tiles of
+ * the last `split_heads` heads are split over the key range: two CTAs take
+ * key tiles [0, n/2) and [n/2, n), each writes its unnormalised O, running
+ * maximum and row sum to device scratch, and the one that finishes second
+ * combines them (same softmax, rounding of those rows changes by about one
+ * bf16 step).  The choice depends on Sk, the groups, heads, the SM count and
+ * the scratch available only -- not on Sq or q_offset -- so a cached-prefix
+ * call computes the target rows bit for bit as the uncached call does.
+ * Scratch: qi_attn_block_causal(_fp8) allocate it in the context on first
+ * need (device memory freed by qi_ctx_destroy; calls sharing a context must
+ * not run concurrently on different streams); the block and step calls use
+ * the block workspace's MLP activation buffer, up to T_last x mlp x 2 bytes
+ * (T_last = tokens of the last group).
+ *
+ * qi_attn_split_plan reports that choice (host only, no device work):
+ * split_heads (0: no split) and the scratch bytes it uses, for a sequence of
+ * Sk tokens in `groups`, `heads` heads, num_sms SMs and scratch_bytes of
+ * scratch (SIZE_MAX: unbounded). */
+int qi_attn_split_plan(int Sk, int heads, const qi_groups* groups, int num_sms,
+                       size_t scratch_bytes, int* split_heads, size_t* bytes);
+
 /* ------------------------------------------------------------------ block */
 
 /* Block-causal attention with e4m3 operands (the pages' reduced-precision

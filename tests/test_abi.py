@@ -77,3 +77,26 @@ def test_invalid_arguments_rejected_without_a_device(L):
     assert L.qi_block_workspace_bytes(C.byref(bad), 10, C.byref(n)) == qi.QI_ERR_UNSUPPORTED_SHAPE
     assert "head_dim" in qi.last_error()
     assert L.qi_rope_tables(0, None, None, None, None, None, None) == qi.QI_ERR_INVALID_ARG
+
+
+def test_attention_split_plan(L):
+    """The attention's key-range split (host-side plan): taken where the last
+    round of CTAs would be mostly idle, bounded by the scratch, absent for
+    short key ranges and for grids whose last round is nearly full."""
+    g = lambda ends: qi.groups_struct(ends, [0] * len(ends))
+    k, nbytes = qi.qi_attn_split_plan(4608, 32, g([512, 4608]), 148)   # 1024x1024 step
+    assert 0 < k < 32 and nbytes > 0
+    # the scratch holds 17 tiles per split head: partial O, max and sum of two halves
+    assert nbytes >= 17 * k * 2 * 256 * (128 + 2) * 4
+    assert qi.qi_attn_split_plan(4608, 32, g([512, 4608]), 148, scratch_bytes=0) == (0, 0)
+    # one byte short: at most k - 1 heads fit, and then the last round still
+    # holds unsplit tiles, so no split is taken at all
+    assert qi.qi_attn_split_plan(4608, 32, g([512, 4608]), 148, scratch_bytes=nbytes - 1)[0] < k
+    assert qi.qi_attn_split_plan(16896, 32, g([512, 16896]), 148)[0] == 0   # 13.8 rounds
+    assert qi.qi_attn_split_plan(896, 32, g([128, 896]), 148)[0] == 0       # 7 key tiles
+    assert qi.qi_attn_split_plan(4130, 4, g([100, 130, 4130]), 148)[0] == 4
+    # the plan depends on the last group only through its length: the edit
+    # ([256 | 1024 | 4096]) splits as the step does
+    assert qi.qi_attn_split_plan(5376, 32, g([256, 1280, 5376]), 148)[0] == k
+    with pytest.raises(qi.QiError):
+        qi.qi_attn_split_plan(4608, 32, g([512, 4000]), 148)   # groups do not end at Sk

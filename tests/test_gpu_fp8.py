@@ -92,6 +92,28 @@ def test_attention_fp8_cached_rows_bit_identical(ctx):
     assert torch.equal(full[P:], part)
 
 
+def test_attention_fp8_key_split(ctx):
+    """The key-range split on e4m3 operands (every head split, as in the bf16
+    case): target rows of the cached call equal the uncached call's; the
+    split halves keep their own reference maxima, so sampled rows are held to
+    the plain reading's e4m3 bound, and closer to it than to exact attention."""
+    sizes, heads = [100, 30, 4000], 4
+    q, k, v, ends = _case(sizes, heads, 17)
+    g = qi.groups_struct(ends, [0] * len(ends))
+    n_sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert qi.qi_attn_split_plan(ends[-1], heads, g, n_sms)[0] == heads
+    full = _run_fp8(ctx, q, k, v, ends)
+    P = ends[-2]
+    part = _run_fp8(ctx, q[P:].contiguous(), k, v, ends, q_offset=P)
+    ctx.check()
+    assert torch.equal(full[P:], part)
+    rows = np.concatenate([np.arange(256), np.arange(256, ends[-1], 31)])
+    got = bf16_np(full)[rows]
+    e_plain = rel_l2(got, _oracle(q, k, v, ends, heads, fp8="plain", rows=rows))
+    e_exact = rel_l2(got, _oracle(q, k, v, ends, heads, fp8=False, rows=rows))
+    assert e_plain < E4M3_RMS and e_plain < e_exact and e_exact < 8e-2
+
+
 class _StepFp8:
     def __init__(self, ctx, blocks=2):
         from tests.test_gpu_step import Setup

@@ -374,6 +374,54 @@ def test_attention_cached_rows_bit_identical_and_mask_invariance(ctx):
     assert rel_l2(bf16_np(full)[P::7], ref) < 4e-3
 
 
+def _num_sms():
+    return torch.cuda.get_device_properties(0).multi_processor_count
+
+
+def test_attention_key_split_vs_oracle_and_cached_rows(ctx):
+    """Every head's longest-range query tiles split over the key range and
+    combined (4 heads x 17 tiles leave most SMs idle).  The first tile holds
+    rows of all three groups; those of the first two see no key of the upper
+    half (a zero-weight half in the combine).  Sampled rows against the
+    oracle; the cached-prefix call (the prefix not a multiple of the tile)
+    computes the target rows bit for bit as the uncached call does."""
+    sizes, heads = [100, 30, 4000], 4
+    q, k, v, ends = _attn_case(sizes, heads, 123)
+    S = ends[-1]
+    g = qi.groups_struct(ends, [0, 0, 1])
+    assert qi.qi_attn_split_plan(S, heads, g, _num_sms())[0] == heads
+    full = qi.qi_attn_block_causal(ctx, cuda(q), cuda(k), cuda(v), g)
+    ctx.check()
+    P = ends[-2]
+    part = qi.qi_attn_block_causal(ctx, cuda(q[P:].contiguous()), cuda(k), cuda(v), g, q_offset=P)
+    ctx.check()
+    assert torch.equal(full[P:], part)
+    rows = np.concatenate([np.arange(256), np.arange(256, S, 13)])
+    ref = _oracle_attn(q, k, v, ends, heads, q_rows=rows)
+    got = bf16_np(full)[rows]
+    assert rel_l2(got, ref) < 4e-3
+    assert np.abs(got - ref).max() < 2e-2
+
+
+def test_attention_key_split_full_size_1024px(ctx):
+    """The 1024x1024 step's attention ([512 | 4096] tokens, 32 heads): the
+    split takes some heads; sampled rows of every head against the oracle,
+    and rows of split and unsplit heads alike within the same tolerance."""
+    sizes, heads = [512, 4096], 32
+    q, k, v, ends = _attn_case(sizes, heads, 5)
+    g = qi.groups_struct(ends, [0, 1])
+    ks = qi.qi_attn_split_plan(ends[-1], heads, g, _num_sms())[0]
+    assert 0 < ks < heads
+    o = qi.qi_attn_block_causal(ctx, cuda(q), cuda(k), cuda(v), g)
+    ctx.check()
+    rows = np.arange(3, ends[-1], 29)
+    ref = _oracle_attn(q, k, v, ends, heads, q_rows=rows).reshape(len(rows), heads, 128)
+    got = bf16_np(o)[rows].reshape(len(rows), heads, 128)
+    for hs in (slice(0, heads - ks), slice(heads - ks, heads)):
+        assert rel_l2(got[:, hs], ref[:, hs]) < 4e-3
+        assert np.abs(got[:, hs] - ref[:, hs]).max() < 2e-2
+
+
 # ------------------------------------------------------------------ Euler, conditioning, probe
 
 def test_euler_bit_exact(ctx):
