@@ -182,9 +182,10 @@ constexpr int FA_PART_O = 2 * FA_ROWS * 128;   // 256 rows x 128 fp32
 constexpr int FA_PART_ML = 2 * FA_ROWS * 2;    // 256 rows x (maximum, sum)
 
 // Grid index -> (query tile pair, head, half, split unit).  Segments, in
-// launch order: the longest-range tiles of the unsplit heads (tile-major,
-// last tile first), the halves of the split heads' longest-range tiles, the
-// remaining tiles of every head (last tile first).  half = -1: not split.
+// launch order: the longest-range tiles of the unsplit heads, the halves of
+// the split heads' longest-range tiles, the remaining tiles of every head.
+// Within a segment, head-major with the last tile first, so that CTAs
+// dispatched together share a head's K/V in L2.  half = -1: not split.
 struct FaUnit {
   int ct, h, half, su;
 };
@@ -195,18 +196,18 @@ __device__ __forceinline__ FaUnit fa_unit(const AttnParams& p, int b) {
   u.half = -1;
   u.su = -1;
   if (b < seg_a) {
-    u.ct = p.n_ctiles - 1 - b / (p.heads - k);
-    u.h = b % (p.heads - k);
+    u.h = b / nh;
+    u.ct = p.n_ctiles - 1 - b % nh;
   } else if (b < seg_a + seg_b) {
     const int v = b - seg_a;
     u.half = v & 1;
     u.su = v >> 1;
-    u.ct = p.n_ctiles - 1 - u.su / k;
-    u.h = p.heads - k + u.su % k;
+    u.h = p.heads - k + u.su / nh;
+    u.ct = p.n_ctiles - 1 - u.su % nh;
   } else {
     const int v = b - seg_a - seg_b;
-    u.ct = p.ct_heavy - 1 - v / p.heads;
-    u.h = v % p.heads;
+    u.h = v / p.ct_heavy;
+    u.ct = p.ct_heavy - 1 - v % p.ct_heavy;
   }
   return u;
 }
