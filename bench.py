@@ -549,6 +549,11 @@ def run_ours(args, rank, world, local_rank):
         achieved = work["gemm_i8_ops_per_step"] * n_steps / (tot[dom] / 1e3) / 1e12
         roof = {"bound": "tensor", "unit": "TOP/s", "peak": pk["int8_sust"],
                 "peak_note": f"int8 dense, sustained: {pk['int8_src']}"}
+    elif dom == "gemm_bf16":
+        # BF16 Linears (and MXFP4 weights decoded to bf16 inside the GEMM)
+        achieved = work["bf16_linear_flops_per_step"] * n_steps / (tot[dom] / 1e3) / 1e12
+        roof = {"bound": "tensor", "unit": "TFLOP/s", "peak": pk["bf16_sust"],
+                "peak_note": f"bf16 dense, sustained, {pk['src']}"}
     else:
         achieved = None
         roof = {"bound": "hbm", "unit": "GB/s", "peak": pk["hbm"], "peak_note": pk["src"]}
@@ -570,8 +575,14 @@ def run_ours(args, rank, world, local_rank):
         other["attention"] = {"achieved_tflops": a, "peak_tflops": pk["bf16_sust"],
                               "frac": a / pk["bf16_sust"], "frac_of_burst": a / pk["bf16"],
                               "peak_note": f"bf16 dense {pk['src']}"}
+    if prof["gemm_bf16"][0] and work["bf16_linear_flops_per_step"]:
+        a = work["bf16_linear_flops_per_step"] * n_steps / (tot["gemm_bf16"] / 1e3) / 1e12
+        other["gemm_bf16"] = {"achieved_tflops": a, "peak_tflops": pk["bf16_sust"],
+                              "frac": a / pk["bf16_sust"], "frac_of_burst": a / pk["bf16"],
+                              "peak_note": f"bf16 dense {pk['src']}"}
     mhz = (clk or {}).get("sm_mhz")
-    for cls, kind, key in (("gemm_i8", "int8", "achieved_tops"), ("attention", "bf16", "achieved_tflops")):
+    for cls, kind, key in (("gemm_i8", "int8", "achieved_tops"), ("attention", "bf16", "achieved_tflops"),
+                           ("gemm_bf16", "bf16", "achieved_tflops")):
         if cls in other and mhz and pk.get(f"{kind}_pipe_per_mhz"):
             pipe = pk[f"{kind}_pipe_per_mhz"] * mhz
             other[cls]["tensor_pipe_at_bench_clock"] = pipe
