@@ -56,13 +56,15 @@ def algorithmic_work(cfg: synth.DitConfig, cached: bool = False):
     rows = cfg.target_tokens if cached else cfg.tokens
     # 2 x rows x (weights) of each block Linear, split by its precision
     sizes = {"qk": 2 * H * H, "v": H * H, "out": H * H, "up": F * H, "down": H * F}
-    i8_ops = bf16_block = 0
+    i8_ops = bf16_block = mx_weights = 0
     for l in range(cfg.blocks):
         for name, kind in synth.linear_precision(cfg, l).items():
             if kind == "w8":
                 i8_ops += 2 * rows * sizes[name]
             else:   # BF16 weights, or MXFP4 weights decoded to bf16 in the GEMM
                 bf16_block += 2 * rows * sizes[name]
+            if kind == "mx":
+                mx_weights += sizes[name]
     ends = np.cumsum(cfg.group_sizes())
     starts = np.concatenate([[0], ends[:-1]])
     if cached:
@@ -105,6 +107,9 @@ def algorithmic_work(cfg: synth.DitConfig, cached: bool = False):
         "quant_bytes_per_step": quant,
         "gemv_bytes_per_step": gemv,
         "bf16_linear_flops_per_step": bf16,
+        # expanding MXFP4 Linears to bf16: codes (0.5 B) + scales (1/32 B) in,
+        # bf16 (2 B) out per weight
+        "mx_expand_bytes_per_step": mx_weights * (0.5 + 1 / 32 + 2),
     }
 
 
@@ -169,15 +174,19 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ model setup
 
-def build_model(ctx, qi, cfg, device):
+def build_model(ctx, qi, cfg, device, mx_expand=True):
+    """The model on the device.  MXFP4 Linears expand into one shared bf16
+    scratch before their GEMMs unless mx_expand is False (then the GEMM
+    decodes the codes tile by tile in shared memory)."""
+    dims = qi.dims_struct(cfg.hidden, cfg.heads, cfg.mlp, cfg.patch, cfg.blocks)
+    scratch = qi.mx_expand_scratch(dims, device) if cfg.precision == "mxfp4" and mx_expand else None
     blocks = []
     for l in range(cfg.blocks):
         wts = synth.block_weights(cfg, l, device=device)
         blocks.append(qi.BlockWeights(ctx, wts, device=device,
-                                      precision=synth.linear_precision(cfg, l)))
+                                      precision=synth.linear_precision(cfg, l), mx_expand=scratch))
         del wts
     glob = synth.model_weights(cfg, device=device)
-    dims = qi.dims_struct(cfg.hidden, cfg.heads, cfg.mlp, cfg.patch, cfg.blocks)
     return qi.Model(ctx, dims, blocks, glob, device=device), dims
 
 
@@ -384,7 +393,7 @@ def run_ours(args, rank, world, local_rank):
     ctx = qi.Context(local_rank)
     cfg = WORKLOADS[args.workload]
     denoise = cfg.steps > 1            # the 40-step 2048^2 workload
-    model, dims = build_model(ctx, qi, cfg, "cuda")
+    model, dims = build_model(ctx, qi, cfg, "cuda", mx_expand=not args.mx_tile_decode)
     S, H = cfg.tokens, cfg.hidden
     gd = [(g.kind, g.tokens, g.grid) for g in cfg.groups]
     ends = list(np.cumsum(cfg.group_sizes()))
@@ -596,6 +605,8 @@ def run_ours(args, rank, world, local_rank):
         "gemv": work["gemv_bytes_per_step"] / (pk["hbm"] * 1e9) * 1e3,
         "gemm_bf16": work["bf16_linear_flops_per_step"] / (pk["bf16_sust"] * 1e12) * 1e3,
     }
+    if cfg.precision == "mxfp4" and not args.mx_tile_decode:
+        ideal["other"] = work["mx_expand_bytes_per_step"] / (pk["hbm"] * 1e9) * 1e3
     step_roof = {"ideal_ms": sum(ideal.values()), "measured_ms": ms_per_step,
                  "frac": sum(ideal.values()) / ms_per_step,
                  "ideal_ms_by_class": ideal,
@@ -620,14 +631,18 @@ def run_ours(args, rank, world, local_rank):
                "pages": ", the pages' precision layout (W8A8 q, k, MLP up/down in blocks 2-29 on "
                         "int8 GEMMs; v, out projection and all Linears of blocks 0, 1, 30, 31 in "
                         "BF16 on bf16 GEMMs), ",
-               "mxfp4": ", all attn/MLP Linears with MXFP4 weights (synthetic checkpoint) decoded "
-                        "to bf16 inside bf16 GEMMs, bf16 activations, "}[cfg.precision]
+               "mxfp4": (", all attn/MLP Linears with MXFP4 weights (synthetic checkpoint) "
+                         + ("decoded to bf16 inside bf16 GEMMs" if args.mx_tile_decode else
+                            "expanded to bf16 (one Linear at a time, into a shared scratch) "
+                            "before bf16 GEMMs")
+                         + ", bf16 activations, ")}[cfg.precision]
             + (f"bf16 attention in steps 1-{cfg.fp8_from_step - 1} and fp8 (e4m3) attention from "
                f"step {cfg.fp8_from_step}" if cfg.fp8_from_step else "bf16 attention"))
     out = {
         "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world,
         "steps": n_steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if cfg.precision in ("mxfp4", "bf16") else "int8",
         "data": "synthetic",
         "config": {"workload": desc, "tokens": S, "blocks": cfg.blocks, "global_batch": world,
                    "l2": f"inputs larger than L2: ~{weight_bytes_per_step(cfg) / 1e9:.1f} GB of "
@@ -863,7 +878,11 @@ def main():
                          "as one batch); "
                          "denoise40_2048px: the full 40-step 2048^2 denoise; "
                          "denoise40_2048px_sched: the same with the pages' precision schedule "
-                         "(fp8 attention from step 8)")
+                         "(fp8 attention from step 8); step_1024px_mxfp4: the 1024^2 step with "
+                         "MXFP4 weights and bf16 activations")
+    ap.add_argument("--mx-tile-decode", action="store_true",
+                    help="step_1024px_mxfp4: decode the MXFP4 codes inside the GEMM (tile by "
+                         "tile in shared memory) instead of expanding each Linear to bf16 first")
     ap.add_argument("--ncu-case", choices=("gemms", "gemm_down", "attention", "block", "gemv"),
                     default=None,
                     help="launch one kernel a few times (for ncu captures) and exit")

@@ -8,6 +8,7 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <algorithm>
 #include <mutex>
 #include <string>
 
@@ -425,9 +426,39 @@ BlockPrecision block_precision(const qi_dims& d, const qi_block_weights& w) {
 
 // A BF16 block Linear on tcgen05 kind::f16 (CTA pairs for 256-wide tiles)
 // with one of the block epilogues; `p` carries the epilogue fields.
+// Where an MXFP4 Linear is expanded to bf16 before its GEMM (MxExpand::buf
+// null: decoded inside the GEMM).  early: the expansion may overlap the
+// kernel before it (the buffer's previous reader is at least two kernels
+// back).
+struct MxExpand {
+  uint16_t* buf = nullptr;
+  size_t bytes = 0;
+  bool early = false;
+};
+
 int run_bf16_block_linear(qi_ctx* ctx, const uint16_t* a, int M, int lda, const qi_linear_bf16& w,
-                          const qi_mxfp4& mx, int epi, qi::GemmParams p, cudaStream_t st) {
+                          const qi_mxfp4& mx, int epi, qi::GemmParams p, cudaStream_t st,
+                          const MxExpand& ex = MxExpand()) {
   if (M == 0) return QI_OK;
+  if (mx.packed && ex.buf &&
+      ex.bytes >= static_cast<size_t>(mx.n) * static_cast<size_t>(mx.k) * sizeof(uint16_t)) {
+    // expand the MXFP4 weights into the scratch, then run them as BF16
+    uint16_t* expand = ex.buf;
+    {
+      Prof pr(ctx, QI_KCLASS_OTHER, st);
+      if (qi::launch_mxfp4_expand_bf16(mx.packed, mx.scales, mx.n, mx.k, expand, st, ex.early))
+        return cuda_fail("MXFP4 expansion launch");
+    }
+    qi_linear_bf16 wb;
+    memset(&wb, 0, sizeof(wb));
+    wb.w = expand;
+    wb.bias = mx.bias;
+    wb.n = mx.n;
+    wb.k = mx.k;
+    qi_mxfp4 none;
+    memset(&none, 0, sizeof(none));
+    return run_bf16_block_linear(ctx, a, M, lda, wb, none, epi, p, st);
+  }
   const bool is_mx = mx.packed != nullptr;
   p.M = M;
   p.N = is_mx ? mx.n : w.n;
@@ -472,6 +503,22 @@ int run_block_multi(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, fl
   // epilogue will publish for the next quantizer.
   const qi_block_taps* tp = ctx->taps_on ? &ctx->taps : nullptr;
   const bool qkv_bf16 = bp.qkv_w8_cols < 3 * H;
+  // MXFP4 expansion scratch.  With room for two of the largest Linears the
+  // Linears alternate between two halves (q | k | v and up in the first, out
+  // and down in the second): a half's previous reader is then at least two
+  // kernels before its next expansion, which may start early.  Otherwise all
+  // share the one buffer and each expansion waits for the kernel before it.
+  MxExpand mxa, mxb;
+  if (w.mx_expand) {
+    const size_t lin = static_cast<size_t>(std::max(3 * H, F)) * H * sizeof(uint16_t);
+    mxa.buf = mxb.buf = w.mx_expand;
+    mxa.bytes = mxb.bytes = w.mx_expand_bytes;
+    if (w.mx_expand_bytes >= 2 * lin) {
+      mxb.buf = w.mx_expand + lin / sizeof(uint16_t);
+      mxa.bytes = mxb.bytes = lin;
+      mxa.early = mxb.early = true;
+    }
+  }
   // The attention's key-range split uses the GELU buffer b.g as scratch (free
   // until the up projection).  The bytes it may take are those of the
   // sequence's last group (T_last x F bf16), a bound that does not depend on
@@ -563,7 +610,7 @@ int run_block_multi(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, fl
     }
     if (qkv_bf16) {
       p.n_base = bp.qkv_w8_cols;   // the v rows (2H) or all of q | k | v (0)
-      if ((r = run_bf16_block_linear(ctx, b.o, T, H, w.qkv_bf16, w.qkv_mx, qi::EPI_QKV, p, st)))
+      if ((r = run_bf16_block_linear(ctx, b.o, T, H, w.qkv_bf16, w.qkv_mx, qi::EPI_QKV, p, st, mxa)))
         return r;
     }
   }
@@ -647,7 +694,7 @@ int run_block_multi(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, fl
     memset(&p, 0, sizeof(p));
     p.y = y_out;
     p.ldy = H;
-    if ((r = run_bf16_block_linear(ctx, b.o, T, H, w.out_bf16, w.out_mx, qi::EPI_BF16, p, st)))
+    if ((r = run_bf16_block_linear(ctx, b.o, T, H, w.out_bf16, w.out_mx, qi::EPI_BF16, p, st, mxb)))
       return r;
   }
   // MLP half: x += gate1 * out, LN2 + modulate + quantize (and/or the bf16
@@ -678,7 +725,7 @@ int run_block_multi(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, fl
     p.y = b.g;
     p.ldy = F;
     p.row_range = g_range;
-    if ((r = run_bf16_block_linear(ctx, b.o, T, H, w.up_bf16, w.up_mx, qi::EPI_GELU, p, st)))
+    if ((r = run_bf16_block_linear(ctx, b.o, T, H, w.up_bf16, w.up_mx, qi::EPI_GELU, p, st, mxa)))
       return r;
   }
   if (tp && ((r = tap_copy(tp->g, b.g, static_cast<size_t>(T) * F * 2, st)) ||
@@ -706,7 +753,7 @@ int run_block_multi(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, fl
     p.groups = gt;
     p.row0 = row0;
     if ((r = run_bf16_block_linear(ctx, b.g, T, F, w.down_bf16, w.down_mx, qi::EPI_GATED, p,
-                                   st)))
+                                   st, mxb)))
       return r;
   }
   return QI_OK;
@@ -767,6 +814,8 @@ int check_block_weights(const qi_dims& d, const qi_block_weights* w) {
   if ((r = check_linear(&w->out, &w->out_bf16, &w->out_mx, "out", H, H))) return r;
   if ((r = check_linear(&w->up, &w->up_bf16, &w->up_mx, "up", F, H))) return r;
   if ((r = check_linear(&w->down, &w->down_bf16, &w->down_mx, "down", H, F))) return r;
+  if (w->mx_expand && !aligned16(w->mx_expand))
+    return fail(QI_ERR_ALIGNMENT, "mx_expand must be 16-byte aligned");
   if (!w->norm_q || !w->norm_k) return fail(QI_ERR_INVALID_ARG, "norm_q / norm_k is NULL");
   if (!aligned16(w->norm_q) || !aligned16(w->norm_k))
     return fail(QI_ERR_ALIGNMENT, "norm_q / norm_k must be 16-byte aligned");
@@ -1262,6 +1311,20 @@ int qi_to_e4m3(qi_ctx* ctx, const uint16_t* x, int64_t n, uint8_t* y, void* stre
   if (!aligned16(x) || !aligned16(y)) return fail(QI_ERR_ALIGNMENT, "pointers must be 16-byte aligned");
   Prof pr(ctx, QI_KCLASS_OTHER, S(stream));
   if (qi::launch_bf16_to_e4m3(x, y, n, S(stream))) return cuda_fail("e4m3 cast launch");
+  return QI_OK;
+}
+
+int qi_mxfp4_expand_bf16(qi_ctx* ctx, const uint8_t* packed, const uint8_t* scales, int n, int k,
+                         uint16_t* w, void* stream) {
+  if (!ctx) return fail(QI_ERR_INVALID_ARG, "NULL argument");
+  if (n < 0 || k < 32 || k % 32) return fail(QI_ERR_INVALID_ARG, "need n >= 0 and k a positive multiple of 32");
+  if (n == 0) return QI_OK;
+  if (!packed || !scales || !w) return fail(QI_ERR_INVALID_ARG, "NULL argument");
+  if (!aligned16(packed) || !aligned16(w))
+    return fail(QI_ERR_ALIGNMENT, "packed / w must be 16-byte aligned");
+  Prof pr(ctx, QI_KCLASS_OTHER, S(stream));
+  if (qi::launch_mxfp4_expand_bf16(packed, scales, n, k, w, S(stream)))
+    return cuda_fail("MXFP4 expansion launch");
   return QI_OK;
 }
 

@@ -242,6 +242,10 @@ int launch_mma_probe(bool i8, int iters, int num_sms, int* status, cudaStream_t 
 int launch_f32_to_bf16(const float* x, uint16_t* y, int64_t n, cudaStream_t st);
 int launch_euler(float* x, const float* v, int64_t n, float dt, cudaStream_t st);
 // MXFP4 (E2M1 codes, low nibble first; E8M0 scale per 32 columns) -> fp32 [n, k].
+// MXFP4 -> bf16 [n, k] (k % 32 == 0; packed and w 16-byte aligned).  early:
+// overlap the previous kernel of the stream (w must be free of readers).
+int launch_mxfp4_expand_bf16(const uint8_t* packed, const uint8_t* scales, int n, int k,
+                             uint16_t* w, cudaStream_t st, bool early = false);
 int launch_mxfp4_decode(const uint8_t* packed, const uint8_t* scales, int n, int k_stored, int k,
                         float* w, cudaStream_t st);
 // bf16 -> e4m3 (round to nearest, ties to even, saturating), n % 8 == 0.

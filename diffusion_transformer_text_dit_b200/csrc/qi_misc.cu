@@ -11,6 +11,7 @@
 #include <math.h>
 
 #include "qi_common.cuh"
+#include "qi_mx.cuh"
 #include "qi_internal.h"
 
 namespace qi {
@@ -290,6 +291,62 @@ int launch_mxfp4_decode(const uint8_t* packed, const uint8_t* scales, int n, int
   mxfp4_decode_kernel<<<static_cast<int>(g), 256, 0, st>>>(packed, scales, n, k_stored, k, w);
   return launch_result();
 }
+
+// MXFP4 weights -> bf16, for k % 32 == 0 (no padding): the same values as the
+// fp32 decode, each exact in bf16, by the GEMM's byte-table decoder
+// (qi_mx.cuh).  One thread per 32-bit word of codes (8 columns): a warp reads
+// 128 contiguous bytes of codes and writes 512 contiguous bytes of bf16 per
+// instruction; four words per thread are in flight at once.
+//
+// early: the kernel reads only the weights, which no kernel writes, and
+// writes a scratch buffer that the caller guarantees no earlier kernel still
+// reads; it then expands while the previous kernel of the stream is still
+// running (programmatic dependent launch) and waits for that kernel only at
+// its end, so that a kernel waiting on this one still finds every earlier
+// kernel complete.
+__global__ void mxfp4_expand_bf16_kernel(const uint32_t* __restrict__ packed,
+                                         const uint8_t* __restrict__ scales, int64_t words,
+                                         uint4* __restrict__ w, int early) {
+  constexpr int U = 4;
+  if (!early) pdl_wait();
+  pdl_trigger();
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i0 = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i0 < words;
+       i0 += U * stride) {
+    uint32_t c[U], e[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t i = i0 + u * stride;
+      c[u] = i < words ? packed[i] : 0u;
+      e[u] = i < words ? scales[i >> 2] : 127u;   // four words per scale group
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t i = i0 + u * stride;
+      if (i >= words) break;
+      uint32_t o[4];
+      if (e[u] >= 2u && e[u] <= 252u)
+        mx_decode8(mx_table(e[u]), c[u], o);
+      else
+        mx_decode8_general(e[u], c[u], o);
+      w[i] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+  if (early) pdl_wait();
+}
+
+int launch_mxfp4_expand_bf16(const uint8_t* packed, const uint8_t* scales, int n, int k,
+                             uint16_t* w, cudaStream_t st, bool early) {
+  const int64_t words = static_cast<int64_t>(n) * (k / 8);
+  if (words == 0) return 0;
+  int64_t g = (words + 255) / 256;
+  if (g > 148 * 8) g = 148 * 8;
+  launch_pdl(mxfp4_expand_bf16_kernel, dim3(static_cast<unsigned>(g)), dim3(256), 0, st, 1,
+             reinterpret_cast<const uint32_t*>(packed), scales, words, reinterpret_cast<uint4*>(w),
+             early ? 1 : 0);
+  return launch_result();
+}
+
 
 // bf16 -> e4m3 (nearest, ties to even, saturating at +-448), 8 values per
 // thread step: the operands of the fp8 attention.

@@ -80,7 +80,7 @@ class qi_block_weights(C.Structure):
                 ("qkv_bf16", qi_linear_bf16), ("out_bf16", qi_linear_bf16),
                 ("up_bf16", qi_linear_bf16), ("down_bf16", qi_linear_bf16),
                 ("qkv_mx", qi_mxfp4), ("out_mx", qi_mxfp4), ("up_mx", qi_mxfp4),
-                ("down_mx", qi_mxfp4)]
+                ("down_mx", qi_mxfp4), ("mx_expand", C.c_void_p), ("mx_expand_bytes", C.c_size_t)]
 
 
 class qi_model(C.Structure):
@@ -139,6 +139,8 @@ _SIGS = {
                            C.POINTER(C.c_int), C.POINTER(C.c_size_t)],
     "qi_ctx_set_attention_fp8": [C.c_void_p, C.c_int],
     "qi_ctx_set_block_taps": [C.c_void_p, C.POINTER(qi_block_taps)],
+    "qi_mxfp4_expand_bf16": [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_void_p,
+                             C.c_void_p],
     "qi_mxfp4_decode": [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_int,
                         C.c_void_p, C.c_void_p],
     "qi_block_workspace_bytes": [C.POINTER(qi_dims), C.c_int, C.POINTER(C.c_size_t)],
@@ -437,6 +439,25 @@ def qi_to_e4m3(ctx: Context, x: torch.Tensor, out: Optional[torch.Tensor] = None
     return out
 
 
+def qi_mxfp4_expand_bf16(ctx: Context, packed, scales, out=None, stream=None):
+    """bf16 weights [n, k] from MXFP4 codes (packed [n, k/2] uint8, scales [n, k/32])."""
+    n, half = packed.shape
+    k = 2 * half
+    if out is None:
+        out = torch.empty((n, k), dtype=torch.bfloat16, device=packed.device)
+    check(lib().qi_mxfp4_expand_bf16(ctx.handle, ptr(packed), ptr(scales), n, k, ptr(out),
+                                     stream_ptr(stream)))
+    return out
+
+
+def mx_expand_scratch(dims: "qi_dims", device="cuda", buffers: int = 2) -> torch.Tensor:
+    """Scratch for expanding MXFP4 block Linears to bf16: room for `buffers`
+    of the largest (max(3 hidden, mlp) x hidden); two let each expansion
+    overlap the kernel before it.  One tensor may serve every block."""
+    H, F = dims.hidden, dims.mlp
+    return torch.empty(buffers * max(3 * H, F) * H, dtype=torch.bfloat16, device=device)
+
+
 def qi_mxfp4_decode(ctx: Context, packed, scales, k: Optional[int] = None, out=None, stream=None):
     """fp32 weights [n, k] from MXFP4 codes (packed [n, k_stored/2] uint8) and E8M0 scales."""
     n, half = packed.shape
@@ -573,11 +594,15 @@ def qi_debug_timeout_probe(ctx: Context, limit_ns: int, stream=None):
 
 class BlockWeights:
     """Device copies of one block's weights.  W8A8 Linears are quantized on the
-    GPU by qi_prepare_w8; BF16 ones are cast to bf16.  ``precision`` maps "qk",
-    "v", "out", "up", "down" to "w8" or "bf16" (default: all W8A8); q and k
-    share one setting (they are one GEMM)."""
+    GPU by qi_prepare_w8; BF16 ones are cast to bf16; MXFP4 ones keep their
+    codes and scales.  ``precision`` maps "qk", "v", "out", "up", "down" to
+    "w8", "bf16" or "mx" (default: all W8A8); q and k share one setting (they
+    are one GEMM).  ``mx_expand`` (mx_expand_scratch) lets the block expand
+    each MXFP4 Linear to bf16 right before its GEMM instead of decoding tile
+    by tile inside it."""
 
-    def __init__(self, ctx: Context, wts: dict, device="cuda", precision: Optional[dict] = None):
+    def __init__(self, ctx: Context, wts: dict, device="cuda", precision: Optional[dict] = None,
+                 mx_expand: Optional[torch.Tensor] = None):
         self.t = {}
         prec = {"qk": "w8", "v": "w8", "out": "w8", "up": "w8", "down": "w8"}
         prec.update(precision or {})
@@ -634,6 +659,10 @@ class BlockWeights:
             self.t["mod"] = wts["mod"].to(device=device, dtype=torch.bfloat16).contiguous()
             self.t["mod_b"] = wts["mod_b"].to(device=device, dtype=torch.bfloat16).contiguous()
             st.mod = bf16_struct(self.t["mod"], self.t["mod_b"])
+        if mx_expand is not None:   # shared scratch: the caller keeps it alive
+            st.mx_expand = ptr(mx_expand)
+            st.mx_expand_bytes = mx_expand.numel() * mx_expand.element_size()
+            self.t["mx_expand"] = mx_expand
         self.struct = st
 
 

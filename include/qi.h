@@ -184,6 +184,18 @@ typedef struct qi_block_weights {
   qi_mxfp4 out_mx;         /*   (qkv_mx: all of q | k | v, n = 3H); bf16 activations as for BF16 */
   qi_mxfp4 up_mx;
   qi_mxfp4 down_mx;
+  /* Optional device scratch for the MXFP4 Linears (16-byte aligned).  Where it
+   * holds n x k bf16 values, an MXFP4 Linear is expanded into it (the exact
+   * bf16 weights, qi_mxfp4_expand_bf16) right before its GEMM, which then
+   * reads them as a BF16 Linear; otherwise the GEMM decodes the codes tile by
+   * tile in shared memory.  Both give the same outputs bit for bit.  HBM
+   * keeps the 4.25-bit weights either way.  With room for two of the largest
+   * Linears (2 x max(3H, F) x H bf16) the Linears alternate between two
+   * halves and each expansion overlaps the kernel before it; with room for
+   * one, they take turns in it.  Blocks may share one scratch (their calls
+   * are ordered on the stream).  NULL / 0: no expansion. */
+  uint16_t* mx_expand;
+  size_t mx_expand_bytes;
 } qi_block_weights;
 
 typedef struct qi_model {
@@ -354,6 +366,13 @@ int qi_attn_block_causal_fp8(qi_ctx* ctx, const uint8_t* q, int ldq, int Sq, int
 /* y = e4m3(x) for n bf16 values (round to nearest, ties to even, saturating at
  * +-448); n % 16 == 0. */
 int qi_to_e4m3(qi_ctx* ctx, const uint16_t* x, int64_t n, uint8_t* y, void* stream);
+
+/* MXFP4 weights -> bf16 w [n, k] (k % 32 == 0, no padding; packed, scales
+ * and w 16-byte aligned), the same values as qi_mxfp4_decode, each exact in
+ * bf16.  One thread per 32-column scale group.  The block calls use it to
+ * expand an MXFP4 Linear into qi_block_weights.mx_expand. */
+int qi_mxfp4_expand_bf16(qi_ctx* ctx, const uint8_t* packed, const uint8_t* scales, int n, int k,
+                         uint16_t* w, void* stream);
 
 /* MXFP4 checkpoint weights -> fp32 ([PX] Runtime precision and quality /
  * What was quantized: E2M1 values packed low nibble first, an E8M0 scale per

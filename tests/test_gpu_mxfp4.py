@@ -80,11 +80,26 @@ def test_mxfp4_linear_rejects_bad_shapes(ctx):
         assert e.value.code == qi.QI_ERR_UNSUPPORTED_SHAPE
 
 
-def _block(ctx, cfg):
+def test_mxfp4_expand_bf16_bit_exact(ctx):
+    """The bf16 expansion equals the oracle's decode value for value, at the
+    extreme scales too (E8M0 0 and 1: subnormal-sized weights; 255: NaN)."""
+    N, K = 512, 1024
+    packed, scales = synth.mxfp4_weight(3, ("expand", N, K), N, K)
+    scales = scales.clone()
+    scales[0, :4] = torch.tensor([0, 1, 254, 255], dtype=torch.uint8)
+    scales[9, :] = 0
+    got = bf16_np(qi.qi_mxfp4_expand_bf16(ctx, cuda(packed), cuda(scales)))
+    ctx.check()
+    ref = O.mxfp4_decode(packed.numpy(), scales.numpy())
+    assert np.array_equal(got, ref.astype(np.float32), equal_nan=True)
+    assert np.isnan(got[0, 96:128]).all() and not np.isnan(got[1:]).any()
+
+
+def _block(ctx, cfg, mx_expand=None):
     H, S = cfg.hidden, cfg.tokens
     wts = synth.block_weights(cfg, 0)
     prec = synth.linear_precision(cfg, 0)
-    bw = qi.BlockWeights(ctx, wts, precision=prec)
+    bw = qi.BlockWeights(ctx, wts, precision=prec, mx_expand=mx_expand)
     ends = list(np.cumsum(cfg.group_sizes()))
     gd = [(gr.kind, gr.tokens, gr.grid) for gr in cfg.groups]
     g = qi.groups_struct(ends, cfg.group_row_sets())
@@ -115,3 +130,20 @@ def test_block_mxfp4_vs_oracle(ctx, cfg):
     assert np.all(np.isfinite(out))
     assert rel_l2(out, ref) < 1e-2
     assert rel_l2(out - x, ref - x) < 1e-2
+
+
+@pytest.mark.parametrize("cfg", [synth.TINY.replace(precision="mxfp4"),
+                                 synth.BLOCK512.replace(precision="mxfp4")],
+                         ids=["tiny", "block_512px"])
+def test_block_mxfp4_expanded_equals_tile_decode(ctx, cfg):
+    """Expanding each MXFP4 Linear to bf16 before a BF16 GEMM gives the block
+    output of the GEMM that decodes in shared memory, bit for bit (the same
+    exact bf16 weights meet the same MMA sequence), with the scratch split in
+    two alternating halves or used whole."""
+    dims = qi.dims_struct(cfg.hidden, cfg.heads, cfg.mlp, cfg.patch, 1)
+    _, tile, _ = _block(ctx, cfg)
+    # two halves (each expansion overlapping the kernel before it), and one
+    for buffers in (2, 1):
+        _, expd, ref = _block(ctx, cfg, mx_expand=qi.mx_expand_scratch(dims, buffers=buffers))
+        assert np.array_equal(tile, expd), buffers
+        assert rel_l2(expd, ref) < 1e-2

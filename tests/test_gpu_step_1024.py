@@ -194,3 +194,28 @@ def test_edit_1024px_write_then_cached_step_vs_oracle(ctx, model):
     # and the uncached second step gives the same latents bit for bit
     u2, _ = r.step(olat1, s2["sigma"], s2["sigma_next"], qi.QI_KV_NONE)
     assert np.array_equal(u2, c2)
+
+
+def test_step_1024px_mxfp4_expanded_equals_tile_decode(ctx):
+    """The full-width 32-block step with MXFP4 weights: expanding each Linear
+    to bf16 in two alternating scratch halves (every expansion overlapping the
+    kernel before it) gives the velocity of decoding inside the GEMMs, bit
+    for bit; so no expansion overwrites weights a GEMM is still reading."""
+    cfg = synth.STEP1024_MXFP4
+    dims = qi.dims_struct(cfg.hidden, cfg.heads, cfg.mlp, cfg.patch, cfg.blocks)
+    scratch = qi.mx_expand_scratch(dims)
+    blocks = [qi.BlockWeights(ctx, synth.block_weights(cfg, l), precision=synth.linear_precision(cfg, l),
+                              mx_expand=scratch) for l in range(cfg.blocks)]
+    glob = synth.model_weights(cfg)
+    expanded = qi.Model(ctx, dims, blocks, glob)
+    for b in blocks:
+        b.struct.mx_expand, b.struct.mx_expand_bytes = None, 0
+    tiled = qi.Model(ctx, dims, blocks, glob)
+    st = _golden("step_1024px")[0]["steps"][0]
+    lat0 = synth.latents(cfg).numpy()
+    vs = [Run(ctx, m, cfg).step(lat0, st["sigma"], st["sigma_next"], qi.QI_KV_NONE)[1]
+          for m in (expanded, tiled, expanded)]
+    del expanded, tiled, blocks, scratch
+    torch.cuda.empty_cache()
+    assert np.all(np.isfinite(vs[0]))
+    assert np.array_equal(vs[0], vs[1]) and np.array_equal(vs[0], vs[2])
