@@ -296,7 +296,10 @@ int launch_mxfp4_decode(const uint8_t* packed, const uint8_t* scales, int n, int
 // fp32 decode, each exact in bf16, by the GEMM's byte-table decoder
 // (qi_mx.cuh).  One thread per 32-bit word of codes (8 columns): a warp reads
 // 128 contiguous bytes of codes and writes 512 contiguous bytes of bf16 per
-// instruction; four words per thread are in flight at once.
+// instruction; two words per thread are in flight at once.  (The writes are
+// 80% of the traffic; on B200 the kernel moves ~3.2 TB/s, about where a
+// write-dominated stream levels off; 4 or 8 words per thread, fewer CTAs or
+// streaming stores measured 3-15% slower.)
 //
 // early: the kernel reads only the weights, which no kernel writes, and
 // writes a scratch buffer that the caller guarantees no earlier kernel still
@@ -307,7 +310,7 @@ int launch_mxfp4_decode(const uint8_t* packed, const uint8_t* scales, int n, int
 __global__ void mxfp4_expand_bf16_kernel(const uint32_t* __restrict__ packed,
                                          const uint8_t* __restrict__ scales, int64_t words,
                                          uint4* __restrict__ w, int early) {
-  constexpr int U = 4;
+  constexpr int U = 2;
   if (!early) pdl_wait();
   pdl_trigger();
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
@@ -340,7 +343,7 @@ int launch_mxfp4_expand_bf16(const uint8_t* packed, const uint8_t* scales, int n
   const int64_t words = static_cast<int64_t>(n) * (k / 8);
   if (words == 0) return 0;
   int64_t g = (words + 255) / 256;
-  if (g > 148 * 8) g = 148 * 8;
+  if (g > 148 * 32) g = 148 * 32;
   launch_pdl(mxfp4_expand_bf16_kernel, dim3(static_cast<unsigned>(g)), dim3(256), 0, st, 1,
              reinterpret_cast<const uint32_t*>(packed), scales, words, reinterpret_cast<uint4*>(w),
              early ? 1 : 0);
