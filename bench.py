@@ -606,7 +606,8 @@ def run_ours(args, rank, world, local_rank):
         other["attention"] = {"achieved_tflops": a, "peak_tflops": pk["bf16_sust"],
                               "frac": a / pk["bf16_sust"], "frac_of_burst": a / pk["bf16"],
                               "peak_note": f"bf16 dense {pk['src']}"}
-    if prof["gemm_bf16"][0] and work["bf16_linear_flops_per_step"]:
+    if prof["gemm_bf16"][0] and work["bf16_linear_flops_per_step"] and \
+            tot["gemm_bf16"] > 0.05 * sum(tot.values()):   # block Linears in BF16 / MXFP4
         a = work["bf16_linear_flops_per_step"] * n_steps / (tot["gemm_bf16"] / 1e3) / 1e12
         other["gemm_bf16"] = {"achieved_tflops": a, "peak_tflops": pk["bf16_sust"],
                               "frac": a / pk["bf16_sust"], "frac_of_burst": a / pk["bf16"],
@@ -698,7 +699,8 @@ def run_ncu_case(args):
                142 MB > L2);
     attention: block-causal attention over [512 | 4096] tokens, 32 heads;
     block:     one whole block at S = 4608 (4 quantizer launches, 4 GEMMs, attention);
-    gemv:      the time conditioning of an 8-block model (3 GEMV launches)."""
+    gemv:      the time conditioning of an 8-block model (3 GEMV launches);
+    mx_expand: MXFP4 -> bf16 expansion of a 16384 x 4096 weight."""
     import ctypes as C
     from diffusion_transformer_text_dit_b200 import build_lib, qi
     build_lib.build()
@@ -810,6 +812,13 @@ def run_ncu_case(args):
         fm = torch.empty((2, 2 * H), dtype=torch.bfloat16, device="cuda")
         for i in range(args.warmup + args.steps):
             qi.qi_time_conditioning(ctx, model, 0.5 + 0.01 * i, bm, fm, ws)
+    elif args.ncu_case == "mx_expand":
+        # MXFP4 -> bf16 expansion of the MLP up projection's weights
+        pk = torch.randint(0, 256, (F, H // 2), dtype=torch.uint8, device="cuda", generator=g)
+        sc = torch.randint(118, 122, (F, H // 32), dtype=torch.uint8, device="cuda", generator=g)
+        w = torch.empty((F, H), dtype=torch.bfloat16, device="cuda")
+        for _ in range(args.warmup + args.steps):
+            qi.qi_mxfp4_expand_bf16(ctx, pk, sc, out=w)
     elif args.ncu_case == "attention":
         q = (torch.randn(S, H, device="cuda", generator=g)).to(torch.bfloat16)
         k = (torch.randn(S, H, device="cuda", generator=g)).to(torch.bfloat16)
@@ -911,7 +920,8 @@ def main():
     ap.add_argument("--mx-tile-decode", action="store_true",
                     help="step_1024px_mxfp4: decode the MXFP4 codes inside the GEMM (tile by "
                          "tile in shared memory) instead of expanding each Linear to bf16 first")
-    ap.add_argument("--ncu-case", choices=("gemms", "gemm_down", "attention", "block", "gemv"),
+    ap.add_argument("--ncu-case", choices=("gemms", "gemm_down", "attention", "block", "gemv",
+                                           "mx_expand"),
                     default=None,
                     help="launch one kernel a few times (for ncu captures) and exit")
     ap.add_argument("--measure-peaks", action="store_true",
