@@ -110,6 +110,7 @@ def test_step_1024px_vs_oracle(ctx, model):
     lat1, v = Run(ctx, model, cfg).step(lat0, st["sigma"], st["sigma_next"], qi.QI_KV_NONE)
     assert np.all(np.isfinite(v))
     err, tol = rel_l2(v, ov), w8a8_stack_tolerance()
+    print(f"step_1024px: v rel-L2 {err:.4e} (tolerance {tol:.4e})")
     assert err <= tol, f"v rel-L2 {err:.3e} after 32 W8A8 blocks (tolerance {tol:.3e})"
     assert np.array_equal(lat1, O.euler_update(lat0, v, st["sigma"], st["sigma_next"]))
 
@@ -131,6 +132,7 @@ def test_step_1024px_bf16_path_vs_oracle(ctx):
     torch.cuda.empty_cache()
     assert np.all(np.isfinite(v))
     err = rel_l2(v, ov)
+    print(f"step_1024px_bf16: v rel-L2 {err:.4e} (tolerance 2e-2)")
     assert err <= 2e-2, f"v rel-L2 {err:.3e} after 32 BF16 blocks"
     assert np.array_equal(lat1, O.euler_update(lat0, v, st["sigma"], st["sigma_next"]))
 
@@ -168,6 +170,7 @@ def test_step_1024px_blocks_teacher_forced(ctx, model):
         ref = O.dit_block(x_in, O.prepare_block(wts), mod, rs, gid, gid, cos, sin, cfg.heads,
                           cfg.head_dim, cfg.eps)
         e_out, e_delta = rel_l2(got, ref), rel_l2(got - x_in, ref - x_in)
+        print(f"block {l}: output rel-L2 {e_out:.4e}, delta rel-L2 {e_delta:.4e}")
         assert e_out <= 1e-2 and e_delta <= 1e-2, (l, e_out, e_delta)
 
 
@@ -182,6 +185,7 @@ def test_edit_1024px_write_then_cached_step_vs_oracle(ctx, model):
     lat1, v1 = r.step(lat0, s1["sigma"], s1["sigma_next"], qi.QI_KV_WRITE_PREFIX)
     tol = w8a8_stack_tolerance()
     err1 = rel_l2(v1, ov1)
+    print(f"edit_1024px step 1: v rel-L2 {err1:.4e} (tolerance {tol:.4e})")
     assert np.all(np.isfinite(v1)) and err1 <= tol, f"step 1 v rel-L2 {err1:.3e} (tol {tol:.3e})"
     assert np.array_equal(lat1, O.euler_update(lat0, v1, s1["sigma"], s1["sigma_next"]))
     # second step from the oracle's step-1 latents: the target rows only,
@@ -189,6 +193,7 @@ def test_edit_1024px_write_then_cached_step_vs_oracle(ctx, model):
     olat1 = O.euler_update(lat0, ov1, s1["sigma"], s1["sigma_next"])
     c2, v2 = r.step(olat1, s2["sigma"], s2["sigma_next"], qi.QI_KV_READ_PREFIX)
     err2 = rel_l2(v2, ov2)
+    print(f"edit_1024px cached step 2: v rel-L2 {err2:.4e} (tolerance {tol:.4e})")
     assert np.all(np.isfinite(v2)) and err2 <= tol, f"cached step 2 v rel-L2 {err2:.3e} (tol {tol:.3e})"
     assert np.array_equal(c2, O.euler_update(olat1, v2, s2["sigma"], s2["sigma_next"]))
     # and the uncached second step gives the same latents bit for bit
