@@ -520,9 +520,11 @@ int run_block_multi(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, fl
     }
   }
   // The attention's key-range split uses the GELU buffer b.g as scratch (free
-  // until the up projection).  The bytes it may take are those of the
-  // sequence's last group (T_last x F bf16), a bound that does not depend on
-  // which rows this call processes; LN1 clears the split counters.
+  // until the up projection).  The plan assumes the bytes of the sequence's
+  // last group (T_last x F bf16), a bound that does not depend on which rows
+  // this call processes; the launch checks its own need against the T x F
+  // bf16 the buffer holds.  LN1 clears the split counters.
+  const size_t g_bytes = static_cast<size_t>(T) * F * sizeof(uint16_t);
   auto split_setup = [&](const SeqAttn& q, qi::AttnParams& ap) {
     const int start_last = q.gt.n >= 2 ? q.gt.end[q.gt.n - 2] : 0;
     ap.Sk = q.S;
@@ -531,6 +533,7 @@ int run_block_multi(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, fl
     ap.num_sms = ctx->num_sms;
     ap.split_scratch = b.g;
     ap.split_bytes = static_cast<size_t>(q.S - start_last) * F * sizeof(uint16_t);
+    ap.split_have = g_bytes;
   };
   size_t split_counters = 0;
   for (int sq = 0; sq < nseq; ++sq) {
@@ -545,7 +548,7 @@ int run_block_multi(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, fl
   {
     QuantExtras ex;
     ex.zero_words = reinterpret_cast<uint32_t*>(b.g);
-    ex.n_zero_words = static_cast<int>(split_counters / 4);
+    ex.n_zero_words = static_cast<int>(std::min(split_counters, g_bytes) / 4);
     ex.zero_range = b.o_range;
     ex.u_f32 = tp ? tp->u1 : nullptr;
     ex.quant_too = bp.qkv_w8_cols > 0;
@@ -1254,6 +1257,7 @@ int attn_call(qi_ctx* ctx, const void* q, int ldq, int Sq, int q_offset, const v
         return cuda_fail("attention split counters");
       p.split_scratch = ctx->attn_scratch;
       p.split_bytes = ctx->attn_scratch_bytes;
+      p.split_have = ctx->attn_scratch_bytes;
     } else {
       p.split_scratch = nullptr;
       p.split_bytes = 0;

@@ -856,10 +856,14 @@ static int launch_attention_t(const AttnParams& p_in, cudaStream_t st) {
   size_t need = 0, counters = 0;
   p.split_heads = 0;
   if (p.split_scratch) attention_split_plan(p, &p.split_heads, &need, &counters);
+  // The plan bounds k by split_bytes with a tile more than any launch over
+  // all of the last group can have; a launch over fewer rows (a block call
+  // on part of the last group) may hold less scratch than that and then
+  // does not split.
   if (p.split_heads > 0 &&
       fa_split_scratch_bytes(static_cast<size_t>(p.n_ctiles - p.ct_heavy) * p.split_heads) >
-          p.split_bytes)
-    p.split_heads = 0;   // not reached: the plan reserves a tile more than a launch can have
+          std::min(p.split_bytes, p.split_have))
+    p.split_heads = 0;
   const int W = p.heads * 128;
   const CUtensorMapDataType dt = FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const uint64_t esz = FP8 ? 1 : 2;

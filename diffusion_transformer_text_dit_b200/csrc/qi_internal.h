@@ -202,7 +202,9 @@ struct AttnParams {
   // then part_ml [units][2][256 rows][2] and part_o [units][2][32 column
   // quads][256 rows][4] fp32.
   void* split_scratch;    // 256-byte aligned device scratch, or null (no split)
-  size_t split_bytes;     // bytes the caller guarantees for it
+  size_t split_bytes;     // bytes the plan may assume (the same for every launch of a sequence)
+  size_t split_have;      // bytes split_scratch holds in this launch (a launch needing more
+                          // than this does not split)
   int num_sms;
   // filled in by launch_attention
   int n_ctiles, ct_heavy, split_heads;

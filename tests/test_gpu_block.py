@@ -137,6 +137,36 @@ def test_block_cached_prefix_bit_identical(ctx, sizes):
     assert torch.equal(full[P:], part)
 
 
+def test_block_1024px_partial_cached_rows(ctx):
+    """Full-width block ([512 | 4096] tokens), cached calls on the last 64 and
+    the last 16 rows of the target group.  The attention splits the longest
+    query tiles of some heads over the key range; with 64 rows the block's
+    scratch holds the split's partials and the rows equal the uncached pass
+    bit for bit; with 16 rows it does not, so that call runs unsplit (no
+    write past its workspace) and differs only by rounding."""
+    cfg = synth.STEP1024.replace(blocks=1)
+    sizes = cfg.group_sizes()
+    S = sum(sizes)
+    ends = [int(e) for e in np.cumsum(sizes)]
+    assert qi.qi_attn_split_plan(S, cfg.heads, qi.groups_struct(ends, [0, 1]),
+                                 torch.cuda.get_device_properties(0).multi_processor_count)[0] > 0
+    wts = synth.block_weights(cfg, 0)
+    x = synth.hidden_states(cfg, S, tag="xp")
+    mod = synth.mod_table(cfg, tag="modp")
+    full, kv, bw, _ = run_block(ctx, cfg, wts, x, mod, sizes, mode=qi.QI_KV_WRITE_PREFIX)
+    for T, exact in ((64, True), (16, False)):
+        P = S - T
+        kv_copy = (kv[0].clone(), kv[1].clone())
+        part, _, _, _ = run_block(ctx, cfg, wts, x[P:].contiguous(), mod, sizes, kv=kv_copy, row0=P,
+                                  mode=qi.QI_KV_READ_PREFIX, bw=bw)
+        if exact:
+            assert torch.equal(full[P:], part)
+        else:
+            got, want, x0 = part.cpu().numpy(), full[P:].cpu().numpy(), x[P:].numpy()
+            assert np.all(np.isfinite(got))
+            assert rel_l2(got - x0, want - x0) < 2e-2
+
+
 def test_block_rejects_bad_arguments(ctx):
     cfg = synth.TINY
     wts = synth.block_weights(cfg, 0)
