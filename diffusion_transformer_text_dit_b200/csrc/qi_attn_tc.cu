@@ -218,6 +218,18 @@ __device__ __forceinline__ float fa_combine(uint32_t o, float f, float b, float 
   return __fadd_rn(__fmul_rn(__uint_as_float(o), f), __fmul_rn(b, g));
 }
 
+// Lane-wise minimum / maximum of two bf16 pairs.
+__device__ __forceinline__ uint32_t bf16x2_min(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("min.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
 // Named barrier 1 over the 8 softmax warps (threads 0-255): plain, and with
 // an AND of a predicate across them.
 __device__ __forceinline__ void fa_softmax_bar() {
@@ -629,7 +641,8 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         lsum = __fadd_rn(__fmul_rn(l, f_me), __fmul_rn(l_oth, f_oth));
       }
       const float inv = lsum > 0.f ? 1.0f / lsum : 0.f;
-      float rlo = 0.f, rhi = 0.f;   // range of the stored bf16 values of this row
+      const uint64_t inv2 = f2_pack(inv, inv);
+      uint32_t lo2 = 0u, hi2 = 0u;   // range of the stored bf16 values of this row, as bf16 pairs
       // the other half's partial is loaded one 32-column chunk ahead
       const float4* src = reinterpret_cast<const float4*>(other_o);
       float4 ahead[8];
@@ -659,14 +672,17 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
             r[4 * v + 3] = __float_as_uint(fa_combine(r[4 * v + 3], f_me, b.w, f_oth));
           }
         }
+        // O / l in paired fp32 multiplies, rounded to bf16 pairs; the row's
+        // range is taken over the stored bf16 pairs themselves
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float a = bf16_round_f(__uint_as_float(r[2 * i]) * inv);
-          const float b = bf16_round_f(__uint_as_float(r[2 * i + 1]) * inv);
-          rlo = fminf(rlo, fminf(a, b));
-          rhi = fmaxf(rhi, fmaxf(a, b));
+          float a, b;
+          f2_unpack(f2_mul(f2_pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), inv2),
+                    a, b);
           pk[i] = pack_bf16x2(a, b);
+          lo2 = bf16x2_min(lo2, pk[i]);
+          hi2 = bf16x2_max(hi2, pk[i]);
         }
         // staged in the TMA store's layout: per tile and 64-column box, 128
         // rows of 128 bytes, 16-byte chunk j of row r at chunk j ^ (r mod 8)
@@ -679,6 +695,10 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         }
       }
       fence_proxy_async_smem();
+      const float rlo = fminf(bf16_bits_to_float(static_cast<uint16_t>(lo2)),
+                              bf16_bits_to_float(static_cast<uint16_t>(lo2 >> 16)));
+      const float rhi = fmaxf(bf16_bits_to_float(static_cast<uint16_t>(hi2)),
+                              bf16_bits_to_float(static_cast<uint16_t>(hi2 >> 16)));
       if (p.row_range && qrow < p.Sq) {
         // per-row range for the next quantizer (non-negative floats order like
         // their bit patterns; negative zero is normalised to +0)
