@@ -336,7 +336,9 @@ int qi_attn_block_causal(qi_ctx* ctx, const uint16_t* q, int ldq, int Sq, int q_
  * need (device memory freed by qi_ctx_destroy; calls sharing a context must
  * not run concurrently on different streams); the block and step calls use
  * the block workspace's MLP activation buffer, up to T_last x mlp x 2 bytes
- * (T_last = tokens of the last group).
+ * (T_last = tokens of the last group).  A block call on fewer rows than the
+ * last group whose buffer cannot hold the split's partials runs unsplit
+ * (its rows then differ from the uncached call's by rounding only).
  *
  * qi_attn_split_plan reports that choice (host only, no device work):
  * split_heads (0: no split) and the scratch bytes it uses, for a sequence of
