@@ -825,6 +825,11 @@ def run_ncu_case(args):
         v = (torch.randn(S, H, device="cuda", generator=g)).to(torch.bfloat16)
         groups = qi.groups_struct(list(np.cumsum(cfg.group_sizes())), cfg.group_row_sets())
         o = torch.empty_like(q)
+        # the key-range split as in the step (whose blocks use their workspace)
+        _, need = qi.qi_attn_split_plan(S, cfg.heads, groups,
+                                        torch.cuda.get_device_properties(0).multi_processor_count)
+        if need:
+            qi.qi_ctx_reserve_attention(ctx, need)
         for _ in range(args.warmup + args.steps):
             qi.qi_attn_block_causal(ctx, q, k, v, groups, o=o)
     torch.cuda.synchronize()

@@ -1004,6 +1004,18 @@ int qi_ctx_destroy(qi_ctx* ctx) {
   return QI_OK;
 }
 
+int qi_ctx_reserve_attention(qi_ctx* ctx, size_t bytes) {
+  if (!ctx) return fail(QI_ERR_INVALID_ARG, "ctx is NULL");
+  if (bytes <= ctx->attn_scratch_bytes) return QI_OK;
+  if (ctx->attn_scratch) cudaFree(ctx->attn_scratch);   // synchronises the device
+  ctx->attn_scratch = nullptr;
+  ctx->attn_scratch_bytes = 0;
+  if (cudaMalloc(&ctx->attn_scratch, bytes) != cudaSuccess)
+    return cuda_fail("cudaMalloc(attention split scratch)");
+  ctx->attn_scratch_bytes = bytes;
+  return QI_OK;
+}
+
 int qi_ctx_check(qi_ctx* ctx, void* stream) {
   if (!ctx) return fail(QI_ERR_INVALID_ARG, "ctx is NULL");
   if (cudaStreamSynchronize(S(stream)) != cudaSuccess) return cuda_fail("stream synchronize");
@@ -1238,25 +1250,17 @@ int attn_call(qi_ctx* ctx, const void* q, int ldq, int Sq, int q_offset, const v
   p.status = ctx->status;
   p.num_sms = ctx->num_sms;
   {
-    // key-range split scratch: owned by the context, grown on first need;
-    // its counters are cleared before every launch
+    // key-range split: only into scratch the context already holds
+    // (qi_ctx_reserve_attention; this call allocates nothing); its counters
+    // are cleared before every launch
     int kh = 0;
     size_t need = 0, counters = 0;
-    p.split_bytes = SIZE_MAX;
-    qi::attention_split_plan(p, &kh, &need, &counters);
-    if (kh > 0 && need > ctx->attn_scratch_bytes) {
-      if (ctx->attn_scratch) cudaFree(ctx->attn_scratch);
-      ctx->attn_scratch = nullptr;
-      ctx->attn_scratch_bytes = 0;
-      if (cudaMalloc(&ctx->attn_scratch, need) != cudaSuccess)
-        return cuda_fail("cudaMalloc(attention split scratch)");
-      ctx->attn_scratch_bytes = need;
-    }
+    p.split_bytes = ctx->attn_scratch_bytes;
+    if (ctx->attn_scratch) qi::attention_split_plan(p, &kh, &need, &counters);
     if (kh > 0) {
       if (cudaMemsetAsync(ctx->attn_scratch, 0, counters, S(stream)) != cudaSuccess)
         return cuda_fail("attention split counters");
       p.split_scratch = ctx->attn_scratch;
-      p.split_bytes = ctx->attn_scratch_bytes;
       p.split_have = ctx->attn_scratch_bytes;
     } else {
       p.split_scratch = nullptr;

@@ -137,6 +137,7 @@ _SIGS = {
     "qi_to_e4m3": [C.c_void_p, C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p],
     "qi_attn_split_plan": [C.c_int, C.c_int, C.POINTER(qi_groups), C.c_int, C.c_size_t,
                            C.POINTER(C.c_int), C.POINTER(C.c_size_t)],
+    "qi_ctx_reserve_attention": [C.c_void_p, C.c_size_t],
     "qi_ctx_set_attention_fp8": [C.c_void_p, C.c_int],
     "qi_ctx_set_block_taps": [C.c_void_p, C.POINTER(qi_block_taps)],
     "qi_mxfp4_expand_bf16": [C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_void_p,
@@ -429,6 +430,11 @@ def qi_attn_split_plan(Sk: int, heads: int, groups: qi_groups, num_sms: int,
     check(lib().qi_attn_split_plan(Sk, heads, C.byref(groups), num_sms, sb, C.byref(k),
                                    C.byref(nb)))
     return k.value, nb.value
+
+
+def qi_ctx_reserve_attention(ctx: Context, bytes_: int) -> None:
+    """Reserve the context's scratch for the standalone attention calls' key-range split."""
+    check(lib().qi_ctx_reserve_attention(ctx.handle, bytes_))
 
 
 def qi_to_e4m3(ctx: Context, x: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None):

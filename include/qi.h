@@ -41,11 +41,13 @@
  *     patterns.  Weights are [out, in] (K-major).
  *   - Every device call is asynchronous on the given CUDA stream
  *     (cudaStream_t passed as void*; NULL = the legacy default stream).
- *     Nothing synchronizes except qi_ctx_check().
+ *     Nothing synchronizes except qi_ctx_check() (and
+ *     qi_ctx_reserve_attention() when it replaces a smaller scratch).
  *   - The library never allocates device memory in a compute call.  Scratch
  *     comes from a caller-owned workspace whose size the *_workspace_bytes
  *     functions return; qi_ctx_create() allocates only a 256-byte device
- *     status word.
+ *     status word, and qi_ctx_reserve_attention() the optional scratch of
+ *     the standalone attention calls.
  *   - Kernels never trap.  A pipeline wait that does not complete within 2 s
  *     records QI_ERR_TIMEOUT in the context's status word and the kernel
  *     returns; qi_ctx_check() reports it.
@@ -228,6 +230,13 @@ int qi_ctx_destroy(qi_ctx* ctx);
  * the stream reported an error, else QI_OK. */
 int qi_ctx_check(qi_ctx* ctx, void* stream);
 
+/* Reserve `bytes` of device scratch in the context for the attention's
+ * key-range split in qi_attn_block_causal(_fp8) (qi_attn_split_plan gives the
+ * bytes a sequence needs).  Grows the scratch if it is smaller (the device is
+ * synchronised when an old scratch is freed); freed by qi_ctx_destroy.
+ * Without it the standalone attention calls do not split. */
+int qi_ctx_reserve_attention(qi_ctx* ctx, size_t bytes);
+
 /* Copy the calling thread's last error text into buf (NUL-terminated). */
 int qi_last_error(char* buf, size_t n);
 
@@ -332,9 +341,10 @@ int qi_attn_block_causal(qi_ctx* ctx, const uint16_t* q, int ldq, int Sq, int q_
  * bf16 step).  The choice depends on Sk, the groups, heads, the SM count and
  * the scratch available only -- not on Sq or q_offset -- so a cached-prefix
  * call computes the target rows bit for bit as the uncached call does.
- * Scratch: qi_attn_block_causal(_fp8) allocate it in the context on first
- * need (device memory freed by qi_ctx_destroy; calls sharing a context must
- * not run concurrently on different streams); the block and step calls use
+ * Scratch: qi_attn_block_causal(_fp8) split only into scratch the context
+ * holds (qi_ctx_reserve_attention; they allocate nothing, and calls sharing a
+ * context must not run concurrently on different streams); the block and
+ * step calls use
  * the block workspace's MLP activation buffer, up to T_last x mlp x 2 bytes
  * (T_last = tokens of the last group).  A block call on fewer rows than the
  * last group whose buffer cannot hold the split's partials runs unsplit

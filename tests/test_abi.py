@@ -77,6 +77,7 @@ def test_invalid_arguments_rejected_without_a_device(L):
     assert L.qi_block_workspace_bytes(C.byref(bad), 10, C.byref(n)) == qi.QI_ERR_UNSUPPORTED_SHAPE
     assert "head_dim" in qi.last_error()
     assert L.qi_rope_tables(0, None, None, None, None, None, None) == qi.QI_ERR_INVALID_ARG
+    assert L.qi_ctx_reserve_attention(None, 1 << 20) == qi.QI_ERR_INVALID_ARG
 
 
 def test_attention_split_plan(L):

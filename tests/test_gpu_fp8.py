@@ -101,7 +101,9 @@ def test_attention_fp8_key_split(ctx):
     q, k, v, ends = _case(sizes, heads, 17)
     g = qi.groups_struct(ends, [0] * len(ends))
     n_sms = torch.cuda.get_device_properties(0).multi_processor_count
-    assert qi.qi_attn_split_plan(ends[-1], heads, g, n_sms)[0] == heads
+    ks, need = qi.qi_attn_split_plan(ends[-1], heads, g, n_sms)
+    assert ks == heads
+    qi.qi_ctx_reserve_attention(ctx, need)
     full = _run_fp8(ctx, q, k, v, ends)
     P = ends[-2]
     part = _run_fp8(ctx, q[P:].contiguous(), k, v, ends, q_offset=P)

@@ -389,7 +389,9 @@ def test_attention_key_split_vs_oracle_and_cached_rows(ctx):
     q, k, v, ends = _attn_case(sizes, heads, 123)
     S = ends[-1]
     g = qi.groups_struct(ends, [0, 0, 1])
-    assert qi.qi_attn_split_plan(S, heads, g, _num_sms())[0] == heads
+    ks, need = qi.qi_attn_split_plan(S, heads, g, _num_sms())
+    assert ks == heads
+    qi.qi_ctx_reserve_attention(ctx, need)
     full = qi.qi_attn_block_causal(ctx, cuda(q), cuda(k), cuda(v), g)
     ctx.check()
     P = ends[-2]
@@ -410,8 +412,9 @@ def test_attention_key_split_full_size_1024px(ctx):
     sizes, heads = [512, 4096], 32
     q, k, v, ends = _attn_case(sizes, heads, 5)
     g = qi.groups_struct(ends, [0, 1])
-    ks = qi.qi_attn_split_plan(ends[-1], heads, g, _num_sms())[0]
+    ks, need = qi.qi_attn_split_plan(ends[-1], heads, g, _num_sms())
     assert 0 < ks < heads
+    qi.qi_ctx_reserve_attention(ctx, need)
     o = qi.qi_attn_block_causal(ctx, cuda(q), cuda(k), cuda(v), g)
     ctx.check()
     rows = np.arange(3, ends[-1], 29)
