@@ -11,10 +11,12 @@ bounded), and runs ``oracle.qi_oracle.step_forward``.
     python tests/golden/make_step_goldens.py step_1024px
     python tests/golden/make_step_goldens.py edit_1024px
     python tests/golden/make_step_goldens.py step_1024px_bf16
+    python tests/golden/make_step_goldens.py step_1024px_mxfp4
     python tests/golden/make_step_goldens.py step_1024px_sensitivity
 
 ``step_1024px_bf16`` is the same step with every block Linear in BF16 (the
-BF16 path); ``step_1024px_sensitivity`` runs the W8A8 step once more on the
+BF16 path), ``step_1024px_mxfp4`` with every block Linear in MXFP4 (decoded
+weights, bf16 activations); ``step_1024px_sensitivity`` runs the W8A8 step once more on the
 latents moved by one fp32 ulp each and records how far that moves v: the
 spread that two correct implementations of the same quantized stack, which
 round differently, can show after 32 blocks.
@@ -64,7 +66,10 @@ def input_hashes(cfg) -> dict:
     out["model_weights"] = sha(*[g[k] for k in sorted(g)])
     for l in (0, cfg.blocks - 1):
         b = synth.block_weights(cfg, l)
-        out[f"block{l}"] = sha(*[b[k] for k in sorted(b)])
+        parts = []
+        for k in sorted(b):   # MXFP4 weights are (packed, scales) pairs
+            parts.extend(b[k] if isinstance(b[k], tuple) else [b[k]])
+        out[f"block{l}"] = sha(*parts)
     return out
 
 
@@ -84,7 +89,8 @@ class LazyBlocks:
         for l in range(self.cfg.blocks):
             wts = synth.block_weights(self.cfg, l)
             self.slot = (wts["mod"].float().numpy(), wts["mod_b"].float().numpy())
-            pw = O.prepare_block({k: v.float().numpy() for k, v in wts.items()},
+            pw = O.prepare_block({k: tuple(t.numpy() for t in v) if isinstance(v, tuple)
+                                  else v.float().numpy() for k, v in wts.items()},
                                  synth.linear_precision(self.cfg, l))
             del wts
             t = time.time() - self.t0
@@ -119,7 +125,7 @@ def main(name: str):
             "latent_seed": cfg.latent_seed, "sigmas": [float(sig[0]), float(sig[1]), float(sig[2])],
             "inputs": input_hashes(cfg), "oracle": "oracle.qi_oracle.step_forward (float64 numpy)",
             "cores": os.cpu_count()}
-    if name in ("step_1024px", "step_1024px_bf16"):
+    if name in ("step_1024px", "step_1024px_bf16", "step_1024px_mxfp4"):
         # one uncached step sigma_0 -> sigma_1
         _, v, secs = run_step(cfg, lat0, float(sig[0]), float(sig[1]), "none", None)
         np.save(os.path.join(HERE, f"{name}_v.npy"), v)
