@@ -12,11 +12,14 @@ bounded), and runs ``oracle.qi_oracle.step_forward``.
     python tests/golden/make_step_goldens.py edit_1024px
     python tests/golden/make_step_goldens.py step_1024px_bf16
     python tests/golden/make_step_goldens.py step_1024px_mxfp4
+    python tests/golden/make_step_goldens.py step_1024px_pagesmask
     python tests/golden/make_step_goldens.py step_1024px_sensitivity
+    python tests/golden/make_step_goldens.py step_1024px_pagesmask_sensitivity
 
 ``step_1024px_bf16`` is the same step with every block Linear in BF16 (the
 BF16 path), ``step_1024px_mxfp4`` with every block Linear in MXFP4 (decoded
-weights, bf16 activations); ``step_1024px_sensitivity`` runs the W8A8 step once more on the
+weights, bf16 activations), ``step_1024px_pagesmask`` with the pages' W8A8 /
+BF16 layout; ``<step>_sensitivity`` runs that step once more on the
 latents moved by one fp32 ulp each and records how far that moves v: the
 spread that two correct implementations of the same quantized stack, which
 round differently, can show after 32 blocks.
@@ -117,7 +120,8 @@ def run_step(cfg, lat, sigma, sigma_next, mode, kv_cache):
 
 
 def main(name: str):
-    cfg = synth.CONFIGS["step_1024px" if name == "step_1024px_sensitivity" else name]
+    base = name[:-len("_sensitivity")] if name.endswith("_sensitivity") else name
+    cfg = synth.CONFIGS[base]
     sig = O.sigma_schedule(40, cfg.target_tokens)
     lat0 = synth.latents(cfg).numpy()
     meta = {"workload": name, "tokens": cfg.tokens, "groups": list(cfg.group_sizes()),
@@ -125,23 +129,23 @@ def main(name: str):
             "latent_seed": cfg.latent_seed, "sigmas": [float(sig[0]), float(sig[1]), float(sig[2])],
             "inputs": input_hashes(cfg), "oracle": "oracle.qi_oracle.step_forward (float64 numpy)",
             "cores": os.cpu_count()}
-    if name in ("step_1024px", "step_1024px_bf16", "step_1024px_mxfp4"):
+    if name in ("step_1024px", "step_1024px_bf16", "step_1024px_mxfp4", "step_1024px_pagesmask"):
         # one uncached step sigma_0 -> sigma_1
         _, v, secs = run_step(cfg, lat0, float(sig[0]), float(sig[1]), "none", None)
         np.save(os.path.join(HERE, f"{name}_v.npy"), v)
         meta["precision"] = cfg.precision
         meta["steps"] = [{"mode": "none", "sigma": float(sig[0]), "sigma_next": float(sig[1]),
                           "v": f"{name}_v.npy", "v_sha": sha(v), "oracle_seconds": secs}]
-    elif name == "step_1024px_sensitivity":
-        # the W8A8 step on latents moved by one ulp (toward +inf), against the
+    elif name.endswith("_sensitivity"):
+        # the step on latents moved by one ulp (toward +inf), against the
         # stored velocity of the unmoved latents
-        base = np.load(os.path.join(HERE, "step_1024px_v.npy"))
+        v_base = np.load(os.path.join(HERE, f"{base}_v.npy"))
         lat_up = np.nextafter(lat0, np.float32(np.inf)).astype(np.float32)
         _, v, secs = run_step(cfg, lat_up, float(sig[0]), float(sig[1]), "none", None)
-        d = float(np.linalg.norm(v.astype(np.float64) - base) / np.linalg.norm(base))
+        d = float(np.linalg.norm(v.astype(np.float64) - v_base) / np.linalg.norm(v_base))
         meta["steps"] = [{"mode": "none", "sigma": float(sig[0]), "sigma_next": float(sig[1]),
                           "latents": "nextafter(latents, +inf): every latent moved by one fp32 ulp",
-                          "v_rel_l2_vs_step_1024px": d, "v_sha": sha(v), "oracle_seconds": secs}]
+                          f"v_rel_l2_vs_{base}": d, "v_sha": sha(v), "oracle_seconds": secs}]
     elif name == "edit_1024px":
         # step 1 writes the text + reference K/V; step 2 reads them and
         # processes the target rows only, from the oracle's step-1 latents
