@@ -12,8 +12,9 @@ and the cached second step must equal the uncached one bit for bit ("Qwen
 Image 2.1 native qualification", "Numerical checks": cached vs uncached
 second steps).
 
-Tolerances.  The BF16 path (every block Linear in BF16) must be within rel-L2
-2e-2 of the oracle after the 32-block stack.  The W8A8 stack re-quantizes
+Tolerances.  The BF16 path (every block Linear in BF16) and the MXFP4 path (every block
+Linear in MXFP4, bf16 activations) must be within rel-L2 2e-2 of the oracle
+after the 32-block stack.  The W8A8 stack re-quantizes
 every activation per token in every block, so a rounding-sized difference
 anywhere flips int8 codes and the flips compound over 32 blocks: the oracle
 itself moves v by ``s`` (tests/golden/step_1024px_sensitivity.json, the oracle
@@ -94,10 +95,11 @@ def _check_inputs(cfg, meta):
     assert meta["inputs"] == input_hashes(cfg), "the seeded inputs changed since the oracle ran"
 
 
-def w8a8_stack_tolerance() -> float:
-    """max(2e-2, 2 x the oracle's one-ulp sensitivity of v after 32 W8A8 blocks)."""
-    with open(os.path.join(GOLDEN, "step_1024px_sensitivity.json")) as f:
-        s = json.load(f)["steps"][0]["v_rel_l2_vs_step_1024px"]
+def w8a8_stack_tolerance(step: str = "step_1024px") -> float:
+    """max(2e-2, 2 x the oracle's one-ulp sensitivity of v after the 32 blocks
+    of `step`, a stack with W8A8 Linears)."""
+    with open(os.path.join(GOLDEN, f"{step}_sensitivity.json")) as f:
+        s = json.load(f)["steps"][0][f"v_rel_l2_vs_{step}"]
     return max(2e-2, 2.0 * s)
 
 
@@ -134,6 +136,31 @@ def test_step_1024px_bf16_path_vs_oracle(ctx):
     err = rel_l2(v, ov)
     print(f"step_1024px_bf16: v rel-L2 {err:.4e} (tolerance 2e-2)")
     assert err <= 2e-2, f"v rel-L2 {err:.3e} after 32 BF16 blocks"
+    assert np.array_equal(lat1, O.euler_update(lat0, v, st["sigma"], st["sigma_next"]))
+
+
+@pytest.mark.skipif(not os.path.exists(os.path.join(GOLDEN, "step_1024px_pagesmask_sensitivity.json")),
+                    reason="oracle golden not written yet")
+def test_step_1024px_pagesmask_vs_oracle(ctx):
+    """The step with the pages' layout (W8A8 q, k and MLP Linears in blocks
+    2-29, every other Linear BF16): within the W8A8-stack tolerance of its
+    own one-ulp sensitivity."""
+    cfg = synth.STEP1024_PAGES
+    meta, (ov,) = _golden("step_1024px_pagesmask")
+    _check_inputs(cfg, meta)
+    st = meta["steps"][0]
+    blocks = [qi.BlockWeights(ctx, synth.block_weights(cfg, l),
+                              precision=synth.linear_precision(cfg, l)) for l in range(cfg.blocks)]
+    dims = qi.dims_struct(cfg.hidden, cfg.heads, cfg.mlp, cfg.patch, cfg.blocks)
+    m = qi.Model(ctx, dims, blocks, synth.model_weights(cfg))
+    lat0 = synth.latents(cfg).numpy()
+    lat1, v = Run(ctx, m, cfg).step(lat0, st["sigma"], st["sigma_next"], qi.QI_KV_NONE)
+    del m, blocks
+    torch.cuda.empty_cache()
+    assert np.all(np.isfinite(v))
+    err, tol = rel_l2(v, ov), w8a8_stack_tolerance("step_1024px_pagesmask")
+    print(f"step_1024px_pagesmask: v rel-L2 {err:.4e} (tolerance {tol:.4e})")
+    assert err <= tol
     assert np.array_equal(lat1, O.euler_update(lat0, v, st["sigma"], st["sigma_next"]))
 
 
@@ -201,11 +228,14 @@ def test_edit_1024px_write_then_cached_step_vs_oracle(ctx, model):
     assert np.array_equal(u2, c2)
 
 
-def test_step_1024px_mxfp4_expanded_equals_tile_decode(ctx):
-    """The full-width 32-block step with MXFP4 weights: expanding each Linear
-    to bf16 in two alternating scratch halves (every expansion overlapping the
-    kernel before it) gives the velocity of decoding inside the GEMMs, bit
-    for bit; so no expansion overwrites weights a GEMM is still reading."""
+def test_step_1024px_mxfp4_vs_oracle_and_decode_paths(ctx):
+    """The full-width 32-block step with MXFP4 weights (every block Linear;
+    bf16 activations, no re-quantization): within rel-L2 2e-2 of the
+    oracle's step on the decoded weights, like the BF16 path.  Expanding each
+    Linear to bf16 in two alternating scratch halves (every expansion
+    overlapping the kernel before it) gives the velocity of decoding inside
+    the GEMMs bit for bit, so no expansion overwrites weights a GEMM is still
+    reading."""
     cfg = synth.STEP1024_MXFP4
     dims = qi.dims_struct(cfg.hidden, cfg.heads, cfg.mlp, cfg.patch, cfg.blocks)
     scratch = qi.mx_expand_scratch(dims)
@@ -216,11 +246,18 @@ def test_step_1024px_mxfp4_expanded_equals_tile_decode(ctx):
     for b in blocks:
         b.struct.mx_expand, b.struct.mx_expand_bytes = None, 0
     tiled = qi.Model(ctx, dims, blocks, glob)
-    st = _golden("step_1024px")[0]["steps"][0]
+    meta, (ov,) = _golden("step_1024px_mxfp4")
+    _check_inputs(cfg, meta)
+    st = meta["steps"][0]
     lat0 = synth.latents(cfg).numpy()
-    vs = [Run(ctx, m, cfg).step(lat0, st["sigma"], st["sigma_next"], qi.QI_KV_NONE)[1]
-          for m in (expanded, tiled, expanded)]
+    runs = [Run(ctx, m, cfg).step(lat0, st["sigma"], st["sigma_next"], qi.QI_KV_NONE)
+            for m in (expanded, tiled, expanded)]
     del expanded, tiled, blocks, scratch
     torch.cuda.empty_cache()
-    assert np.all(np.isfinite(vs[0]))
+    (lat1, v), vs = runs[0], [r[1] for r in runs]
+    assert np.all(np.isfinite(v))
     assert np.array_equal(vs[0], vs[1]) and np.array_equal(vs[0], vs[2])
+    err = rel_l2(v, ov)
+    print(f"step_1024px_mxfp4: v rel-L2 {err:.4e} (tolerance 2e-2)")
+    assert err <= 2e-2, f"v rel-L2 {err:.3e} after 32 MXFP4 blocks"
+    assert np.array_equal(lat1, O.euler_update(lat0, v, st["sigma"], st["sigma_next"]))
