@@ -139,8 +139,6 @@ def test_step_1024px_bf16_path_vs_oracle(ctx):
     assert np.array_equal(lat1, O.euler_update(lat0, v, st["sigma"], st["sigma_next"]))
 
 
-@pytest.mark.skipif(not os.path.exists(os.path.join(GOLDEN, "step_1024px_pagesmask_sensitivity.json")),
-                    reason="oracle golden not written yet")
 def test_step_1024px_pagesmask_vs_oracle(ctx):
     """The step with the pages' layout (W8A8 q, k and MLP Linears in blocks
     2-29, every other Linear BF16): within the W8A8-stack tolerance of its
