@@ -95,6 +95,16 @@ def test_mxfp4_expand_bf16_bit_exact(ctx):
     assert np.isnan(got[0, 96:128]).all() and not np.isnan(got[1:]).any()
 
 
+@pytest.mark.parametrize("N,K", [(1, 32), (100, 96), (257, 4096)])
+def test_mxfp4_expand_bf16_ragged_shapes(ctx, N, K):
+    """Any row count and any multiple of 32 columns (one scale group), the
+    grid's last partial block of words included."""
+    packed, scales = synth.mxfp4_weight(N + K, ("ragged", N, K), N, K)
+    got = bf16_np(qi.qi_mxfp4_expand_bf16(ctx, cuda(packed), cuda(scales)))
+    ctx.check()
+    assert np.array_equal(got, O.mxfp4_decode(packed.numpy(), scales.numpy()).astype(np.float32))
+
+
 def _block(ctx, cfg, mx_expand=None):
     H, S = cfg.hidden, cfg.tokens
     wts = synth.block_weights(cfg, 0)
