@@ -15,6 +15,14 @@ bounded), and runs ``oracle.qi_oracle.step_forward``.
     python tests/golden/make_step_goldens.py step_1024px_pagesmask
     python tests/golden/make_step_goldens.py step_1024px_sensitivity
     python tests/golden/make_step_goldens.py step_1024px_pagesmask_sensitivity
+    python tests/golden/make_step_goldens.py cfg_1024px_uncond
+    python tests/golden/make_step_goldens.py edit_3ref_1024px
+
+``cfg_1024px_uncond`` is the unconditional (negative prompt) sequence of the
+true-CFG workload, [256 text | 4096 image]: its conditional sequence is the
+1024x1024 step itself (same seeds), so the two stored velocities give the
+guided one.  ``edit_3ref_1024px`` is one uncached step of the multi-reference
+edit, [256 text | 1024 | 1024 | 576 references | 4096 target].
 
 ``step_1024px_bf16`` is the same step with every block Linear in BF16 (the
 BF16 path), ``step_1024px_mxfp4`` with every block Linear in MXFP4 (decoded
@@ -121,7 +129,7 @@ def run_step(cfg, lat, sigma, sigma_next, mode, kv_cache):
 
 def main(name: str):
     base = name[:-len("_sensitivity")] if name.endswith("_sensitivity") else name
-    cfg = synth.CONFIGS[base]
+    cfg = synth.CFG1024.uncond() if base == "cfg_1024px_uncond" else synth.CONFIGS[base]
     sig = O.sigma_schedule(40, cfg.target_tokens)
     lat0 = synth.latents(cfg).numpy()
     meta = {"workload": name, "tokens": cfg.tokens, "groups": list(cfg.group_sizes()),
@@ -129,7 +137,8 @@ def main(name: str):
             "latent_seed": cfg.latent_seed, "sigmas": [float(sig[0]), float(sig[1]), float(sig[2])],
             "inputs": input_hashes(cfg), "oracle": "oracle.qi_oracle.step_forward (float64 numpy)",
             "cores": os.cpu_count()}
-    if name in ("step_1024px", "step_1024px_bf16", "step_1024px_mxfp4", "step_1024px_pagesmask"):
+    if name in ("step_1024px", "step_1024px_bf16", "step_1024px_mxfp4", "step_1024px_pagesmask",
+                "cfg_1024px_uncond", "edit_3ref_1024px"):
         # one uncached step sigma_0 -> sigma_1
         _, v, secs = run_step(cfg, lat0, float(sig[0]), float(sig[1]), "none", None)
         np.save(os.path.join(HERE, f"{name}_v.npy"), v)

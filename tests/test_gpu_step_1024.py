@@ -259,3 +259,73 @@ def test_step_1024px_mxfp4_vs_oracle_and_decode_paths(ctx):
     print(f"step_1024px_mxfp4: v rel-L2 {err:.4e} (tolerance 2e-2)")
     assert err <= 2e-2, f"v rel-L2 {err:.3e} after 32 MXFP4 blocks"
     assert np.array_equal(lat1, O.euler_update(lat0, v, st["sigma"], st["sigma_next"]))
+
+
+def test_edit_3ref_1024px_vs_oracle_and_cache(ctx, model):
+    """The multi-reference edit at full width ([256 text | 1024 | 1024 | 576
+    references | 4096 target], each reference its own group of the
+    block-causal mask): one uncached step within the W8A8-stack tolerance of
+    the oracle; writing the four prefix groups' K/V gives the same velocity
+    bit for bit, and a second step that reads them equals the uncached second
+    step bit for bit."""
+    cfg = synth.EDIT3REF1024
+    assert cfg.weight_seed == synth.STEP1024.weight_seed and cfg.hidden == synth.STEP1024.hidden
+    meta, (ov,) = _golden("edit_3ref_1024px")
+    _check_inputs(cfg, meta)
+    st = meta["steps"][0]
+    r = Run(ctx, model, cfg)
+    lat0 = synth.latents(cfg).numpy()
+    lat1, v = r.step(lat0, st["sigma"], st["sigma_next"], qi.QI_KV_NONE)
+    assert np.all(np.isfinite(v))
+    err, tol = rel_l2(v, ov), w8a8_stack_tolerance()
+    print(f"edit_3ref_1024px: v rel-L2 {err:.4e} (tolerance {tol:.4e})")
+    assert err <= tol, f"v rel-L2 {err:.3e} (tolerance {tol:.3e})"
+    assert np.array_equal(lat1, O.euler_update(lat0, v, st["sigma"], st["sigma_next"]))
+    w1, vw = r.step(lat0, st["sigma"], st["sigma_next"], qi.QI_KV_WRITE_PREFIX)
+    assert np.array_equal(vw, v) and np.array_equal(w1, lat1)
+    sig = O.sigma_schedule(40, cfg.target_tokens)
+    c2, _ = r.step(lat1, float(sig[1]), float(sig[2]), qi.QI_KV_READ_PREFIX)
+    u2, _ = r.step(lat1, float(sig[1]), float(sig[2]), qi.QI_KV_NONE)
+    assert np.array_equal(c2, u2)
+
+
+def test_cfg_1024px_vs_oracle(ctx, model):
+    """True CFG at full width: the prompt's sequence is the 1024x1024 step
+    ([512 text | 4096]), the negative prompt's [256 text | 4096], guidance 4,
+    both in one batched step.  The batch's guided velocity equals the
+    guidance of the two single-sequence velocities bit for bit, and each of
+    those is within the W8A8-stack tolerance of the oracle's."""
+    cfg = synth.CFG1024
+    cond, ucfg = synth.STEP1024, cfg.uncond()
+    assert cfg.replace(name=cond.name, uncond_text=0) == cond
+    meta_c, (ovc,) = _golden("step_1024px")
+    meta_u, (ovu,) = _golden("cfg_1024px_uncond")
+    _check_inputs(cond, meta_c)
+    _check_inputs(ucfg, meta_u)
+    st = meta_u["steps"][0]
+    assert (st["sigma"], st["sigma_next"]) == (meta_c["steps"][0]["sigma"], meta_c["steps"][0]["sigma_next"])
+    a, b = st["sigma"], st["sigma_next"]
+    rc, ru = Run(ctx, model, cond), Run(ctx, model, ucfg)
+    lat0 = synth.latents(cfg).numpy()
+    _, vc = rc.step(lat0, a, b, qi.QI_KV_NONE)
+    _, vu = ru.step(lat0, a, b, qi.QI_KV_NONE)
+    ws = torch.empty(qi.qi_step_cfg_workspace_bytes(model.dims, cond.tokens, ucfg.tokens,
+                                                    cfg.target_tokens), dtype=torch.uint8, device="cuda")
+    sc = qi.seq_struct(rc.txt, cond.text_tokens, None, rc.groups, rc.cos, rc.sin)
+    su = qi.seq_struct(ru.txt, ucfg.text_tokens, None, ru.groups, ru.cos, ru.sin)
+    latg = cuda(torch.from_numpy(lat0.copy()))
+    vg = torch.empty_like(latg)
+    qi.qi_denoise_step_cfg(ctx, model, latg, sc, su, cfg.guidance, a, b, qi.QI_KV_NONE, vg, ws)
+    ctx.check()
+    v, lat1 = vg.cpu().numpy(), latg.cpu().numpy()
+    del ws, rc, ru
+    torch.cuda.empty_cache()
+    assert np.all(np.isfinite(v))
+    assert np.array_equal(v, O.cfg_combine(vc, vu, cfg.guidance))
+    assert np.array_equal(lat1, O.euler_update(lat0, v, a, b))
+    tol = w8a8_stack_tolerance()
+    ec, eu = rel_l2(vc, ovc), rel_l2(vu, ovu)
+    eg = rel_l2(v, O.cfg_combine(ovc, ovu, cfg.guidance))
+    print(f"cfg_1024px: prompt v rel-L2 {ec:.4e}, negative prompt v rel-L2 {eu:.4e} "
+          f"(tolerance {tol:.4e}); guided v rel-L2 {eg:.4e}")
+    assert ec <= tol and eu <= tol, (ec, eu, tol)
