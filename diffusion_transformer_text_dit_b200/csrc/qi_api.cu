@@ -1694,11 +1694,22 @@ int qi_denoise_step_cfg(qi_ctx* ctx, const qi_model* model, float* latents, cons
     rows.end[1] = T;
     rows.row_set[0] = rows.row_set[1] = 1;
   } else {
-    if (sp[0].gt.n + sp[1].gt.n > QI_MAX_GROUPS)
-      return fail(QI_ERR_UNSUPPORTED_SHAPE, "the two sequences hold more than %d groups together", QI_MAX_GROUPS);
+    // the table only maps rows to row sets, so neighbouring groups with the
+    // same row set become one run ([text | references] of each sequence use
+    // the prefix set): a prompt and a negative prompt with up to 10
+    // references each still fit
     for (int b = 0; b < 2; ++b)
       for (int g = 0; g < sp[b].gt.n; ++g) {
-        rows.end[rows.n] = (b ? sp[0].S : 0) + sp[b].gt.end[g];
+        const int end = (b ? sp[0].S : 0) + sp[b].gt.end[g];
+        if (rows.n > 0 && rows.row_set[rows.n - 1] == sp[b].gt.row_set[g]) {
+          rows.end[rows.n - 1] = end;
+          continue;
+        }
+        if (rows.n == QI_MAX_GROUPS)
+          return fail(QI_ERR_UNSUPPORTED_SHAPE,
+                      "the two sequences hold more than %d runs of equal row sets together",
+                      QI_MAX_GROUPS);
+        rows.end[rows.n] = end;
         rows.row_set[rows.n] = sp[b].gt.row_set[g];
         ++rows.n;
       }

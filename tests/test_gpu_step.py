@@ -11,6 +11,11 @@ from tests._util import bf16_np, cuda, oracle_weights, rel_l2
 
 pytestmark = pytest.mark.gpu
 
+# Ten reference images of mixed grids: the most the pages' edit flow takes
+# (each reference its own group of the block-causal mask).
+REF10 = tuple(synth.Group("image", h * w, (h, w))
+              for h, w in ((4, 4), (3, 3), (2, 2), (4, 4), (2, 3), (3, 3), (3, 4), (2, 2), (4, 4), (2, 4)))
+
 
 class Setup:
     def __init__(self, ctx, cfg):
@@ -70,9 +75,11 @@ class Setup:
                        groups=(synth.Group("text", 12), synth.Group("image", 16, (4, 4)),
                                synth.Group("image", 36, (6, 6)), synth.Group("image", 9, (3, 3)),
                                synth.Group("image", 64, (8, 8)))),
+    synth.TINY.replace(name="tiny_edit_10ref", blocks=2, patch=64,
+                       groups=(synth.Group("text", 12),) + REF10 + (synth.Group("image", 64, (8, 8)),)),
     synth.TINY.replace(name="tiny_pages", blocks=6, precision="pages"),
     synth.TINY.replace(name="tiny_mxfp4", blocks=3, patch=64, precision="mxfp4")],
-    ids=["2blk", "32blk", "edit", "edit_3ref", "pages_mask_6blk", "mxfp4_3blk"])
+    ids=["2blk", "32blk", "edit", "edit_3ref", "edit_10ref", "pages_mask_6blk", "mxfp4_3blk"])
 def test_step_vs_oracle(ctx, cfg):
     s = Setup(ctx, cfg)
     sig = O.sigma_schedule(40, cfg.target_tokens)
@@ -84,13 +91,13 @@ def test_step_vs_oracle(ctx, cfg):
     assert np.array_equal(lat1.numpy(), O.euler_update(s.lat.numpy(), v.numpy(), sig[3], sig[4]))
 
 
-@pytest.mark.parametrize("edit,precision", [(0, "w8a8"), (1, "w8a8"), (3, "w8a8"), (1, "pages"),
-                                            (1, "mxfp4")],
-                         ids=["text_image", "text_ref_image", "text_3ref_image", "pages_mask",
-                              "mxfp4"])
+@pytest.mark.parametrize("edit,precision", [(0, "w8a8"), (1, "w8a8"), (3, "w8a8"), (10, "w8a8"),
+                                            (1, "pages"), (1, "mxfp4")],
+                         ids=["text_image", "text_ref_image", "text_3ref_image", "text_10ref_image",
+                              "pages_mask", "mxfp4"])
 def test_step_cached_equals_uncached(ctx, edit, precision):
-    refs = [synth.Group("image", 64, (8, 8)), synth.Group("image", 100, (10, 10)),
-            synth.Group("image", 48, (6, 8))][:edit]
+    refs = ([synth.Group("image", 64, (8, 8)), synth.Group("image", 100, (10, 10)),
+             synth.Group("image", 48, (6, 8))][:edit] if edit <= 3 else list(REF10[:edit]))
     groups = ((synth.Group("text", 128 if edit else 100),) + tuple(refs) +
               (synth.Group("image", 256, (16, 16)),))
     cfg = synth.TINY.replace(name="cache", blocks=3 if precision == "w8a8" else 5, patch=64,
@@ -123,8 +130,8 @@ class CfgSetup:
     same target; the negative prompt is shorter."""
 
     def __init__(self, ctx, blocks=2, refs=0, text_c=12, text_u=7):
-        ref_groups = tuple(synth.Group("image", n, g) for n, g in
-                           ((16, (4, 4)), (36, (6, 6)))[:refs])
+        ref_groups = (tuple(synth.Group("image", n, g) for n, g in
+                            ((16, (4, 4)), (36, (6, 6)))[:refs]) if refs <= 2 else REF10[:refs])
         tgt = synth.Group("image", 64, (8, 8))
         self.cfg_c = synth.TINY.replace(name="cfg_c", blocks=blocks, patch=64,
                                         groups=(synth.Group("text", text_c),) + ref_groups + (tgt,))
@@ -155,7 +162,7 @@ class CfgSetup:
         return latg.cpu(), v.cpu()
 
 
-@pytest.mark.parametrize("refs", [0, 2], ids=["text_image", "text_2ref_image"])
+@pytest.mark.parametrize("refs", [0, 2, 10], ids=["text_image", "text_2ref_image", "text_10ref_image"])
 def test_cfg_batch_equals_two_single_steps(ctx, refs):
     s = CfgSetup(ctx, refs=refs)
     sig = O.sigma_schedule(40, s.cfg_c.target_tokens)
@@ -181,8 +188,24 @@ def test_cfg_step_vs_oracle(ctx):
     assert rel_l2(v.numpy(), ov) < 2e-2
 
 
-def test_cfg_cached_equals_uncached(ctx):
-    s = CfgSetup(ctx, blocks=3, refs=1)
+def test_cfg_10ref_step_vs_oracle(ctx):
+    """True CFG over ten references (24 groups in the two sequences): the
+    batch's row table merges neighbouring groups of the same row set, so it
+    runs, and its guided velocity matches the oracle's."""
+    s = CfgSetup(ctx, refs=10)
+    sig = O.sigma_schedule(40, s.cfg_c.target_tokens)
+    a, b = float(sig[2]), float(sig[3])
+    _, v = s.step(ctx, s.c.lat, 3.0, a, b)
+    _, ovc = s.c.oracle_step(s.c.lat, a, b)
+    _, ovu = s.u.oracle_step(s.c.lat, a, b)
+    ov = O.cfg_combine(ovc, ovu, 3.0)
+    assert np.all(np.isfinite(v.numpy()))
+    assert rel_l2(v.numpy(), ov) < 2e-2
+
+
+@pytest.mark.parametrize("refs", [1, 10], ids=["1ref", "10ref"])
+def test_cfg_cached_equals_uncached(ctx, refs):
+    s = CfgSetup(ctx, blocks=3, refs=refs)
     sig = O.sigma_schedule(40, s.cfg_c.target_tokens)
     a1, _ = s.step(ctx, s.c.lat, 2.5, float(sig[0]), float(sig[1]), qi.QI_KV_WRITE_PREFIX)
     u2, _ = s.step(ctx, a1, 2.5, float(sig[1]), float(sig[2]), qi.QI_KV_NONE)
