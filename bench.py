@@ -116,9 +116,10 @@ def algorithmic_work(cfg: synth.DitConfig, cached: bool = False):
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    """nvidia-smi sampling every 200 ms during the timed region."""
+    """nvidia-smi sampling every 100 ms; the summary keeps the samples whose
+    timestamps fall inside the timed region (window() marks it)."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -126,12 +127,17 @@ class ClockSampler:
         self.gpus = set(gpus)
         self.proc = None
         self.lines = []
+        self.t0 = self.t1 = None
+
+    def window(self, t0, t1):
+        """Wall-clock bounds (time.time()) of the timed region."""
+        self.t0, self.t1 = t0, t1
 
     def start(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
             return
@@ -151,25 +157,28 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.t.join(timeout=2)
-        sm, smax, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        rows = []
         for ln in self.lines:
             f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
+            if len(f) < 10:
                 continue
             try:
-                if int(f[0]) not in self.gpus:
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                if int(f[1]) not in self.gpus:
                     continue
-                sm.append(float(f[1]))
-                smax.append(float(f[2]))
+                rows.append((ts, float(f[2]), float(f[3]),
+                             {n for n, v in zip(names, f[6:10]) if v.lower().startswith("active")}))
             except ValueError:
                 continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
+        inside = [r for r in rows if self.t0 is not None and self.t0 - 0.05 <= r[0] <= self.t1 + 0.05]
+        use = inside if inside else rows
+        sm = [r[1] for r in use]
+        reasons = set().union(*[r[3] for r in use]) if use else set()
         return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "sm_max_mhz": max(r[2] for r in use) if use else None,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "in_timed_region": bool(inside)}
 
 
 # ------------------------------------------------------------------ model setup
@@ -476,7 +485,10 @@ def run_ours(args, rank, world, local_rank):
         clocks.start()
         time.sleep(0.3)
     ctx.profile(False)
+    t_start = time.time()
     n_steps, ms_max = run_timed()
+    if clocks:
+        clocks.window(t_start, time.time())
     counts = ctx.profile_read()
     clk = clocks.stop() if clocks else None
     ctx.check()

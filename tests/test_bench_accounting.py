@@ -63,3 +63,46 @@ def test_cfg_counts_both_sequences_and_one_time_conditioning():
     b = bench.algorithmic_work(cfg.uncond())
     assert w["gemm_i8_ops_per_step"] == a["gemm_i8_ops_per_step"] + b["gemm_i8_ops_per_step"]
     assert w["gemv_bytes_per_step"] == a["gemv_bytes_per_step"]
+
+
+class _Done:
+    """Stands in for the finished nvidia-smi process and its reader thread."""
+
+    def terminate(self):
+        pass
+
+    def wait(self, timeout=None):
+        return 0
+
+    def join(self, timeout=None):
+        pass
+
+
+def test_clock_summary_keeps_the_timed_region():
+    """Only samples stamped inside the timed region count: the idle clock
+    before it and a throttle reason after it are left out."""
+    import datetime
+    cs = bench.ClockSampler([0])
+    cs.proc, cs.t = _Done(), _Done()
+    t0 = datetime.datetime(2026, 1, 1, 12, 0, 0).timestamp()
+
+    def line(dt, mhz, gpu=0, power_cap="Not Active", thermal="Not Active"):
+        ts = datetime.datetime.fromtimestamp(t0 + dt).strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+        return f"{ts}, {gpu}, {mhz}, 1965, 900.0, 0x4, Not Active, Not Active, {thermal}, {power_cap}"
+
+    cs.lines = [line(-0.3, 1965), line(0.1, 1650, power_cap="Active"), line(0.2, 1640),
+                line(0.3, 1700, gpu=1, thermal="Active"), line(0.4, 1660), line(0.9, 1965, thermal="Active")]
+    cs.window(t0, t0 + 0.5)
+    out = cs.stop()
+    assert out["samples"] == 3 and out["in_timed_region"]
+    assert out["sm_mhz"] == 1650 and out["sm_max_mhz"] == 1965
+    assert out["reasons"] == ["sw_power_cap"]
+
+
+def test_clock_summary_without_a_window_uses_every_sample():
+    cs = bench.ClockSampler([0])
+    cs.proc, cs.t = _Done(), _Done()
+    cs.lines = ["2026/01/01 12:00:00.100, 0, 1800, 1965, 700.0, 0x0, Not Active, Not Active, "
+                "Not Active, Not Active", "garbage"]
+    out = cs.stop()
+    assert out["samples"] == 1 and not out["in_timed_region"] and out["reasons"] == []
