@@ -897,7 +897,8 @@ def measure_peaks(args):
         clocks.start()
         time.sleep(0.3)
         e0.record(st)
-        t_end = time.time() + 4.0
+        t_start = time.time()
+        t_end = t_start + 4.0
         launches = 0
         while time.time() < t_end:
             for _ in range(8):
@@ -906,6 +907,7 @@ def measure_peaks(args):
             torch.cuda.synchronize()
         e1.record(st)
         torch.cuda.synchronize()
+        clocks.window(t_start, time.time())
         clk = clocks.stop()
         sust = ops * launches / (e0.elapsed_time(e1) / 1e3) / 1e12
         out[name] = {"burst_tops": burst, "sustained_tops": sust, "sustained_seconds":
