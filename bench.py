@@ -495,26 +495,9 @@ def run_ours(args, rank, world, local_rank):
     ms_per_step = ms_max / n_steps
     value = aggregate_throughput(world, n_steps, ms_max)
 
-    # ---------------- the same steps again with every launch bracketed by CUDA
-    # events on its stream: per-kernel-class device time for the rooflines
-    ctx.profile(True)
-    _, ms_prof = run_timed()
-    prof = ctx.profile_read()
-    ctx.profile(False)
-    ctx.check()
-
-    # ---------------- cached-prefix steps (the pages' later denoising steps)
-    extra = {}
-    if not denoise:
-        step(0, lat, txt, qi.QI_KV_WRITE_PREFIX)
-        cms = timed(lambda: [step(i + 1, lat, txt, qi.QI_KV_READ_PREFIX) for i in range(args.steps)])
-        extra["cached_step"] = {"value": aggregate_throughput(world, args.steps, cms),
-                                "unit": "steps/s", "ms_per_step": cms / args.steps,
-                                "note": "target rows only; prefix K/V read from the cache"}
-    else:
-        extra["seconds_per_40_steps"] = ms_max / 1e3
-
-    # ---------------- end to end through the public call with host buffers
+    # ---------------- end to end through the public call with host buffers,
+    # right after the headline so that both meet the GPU in the same state
+    # (a 1 kW part settles to lower clocks under the power cap as a run goes on)
     h_lat = lat0.cpu().pin_memory()
     h_txt = txt.cpu().pin_memory()
     h_out = torch.empty_like(h_lat).pin_memory()
@@ -566,6 +549,25 @@ def run_ours(args, rank, world, local_rank):
         e2e_ms = timed(e2e_run)
         e2e = aggregate_throughput(world, args.steps, e2e_ms)
     ctx.check()
+
+    # ---------------- the same steps again with every launch bracketed by CUDA
+    # events on its stream: per-kernel-class device time for the rooflines
+    ctx.profile(True)
+    _, ms_prof = run_timed()
+    prof = ctx.profile_read()
+    ctx.profile(False)
+    ctx.check()
+
+    # ---------------- cached-prefix steps (the pages' later denoising steps)
+    extra = {}
+    if not denoise:
+        step(0, lat, txt, qi.QI_KV_WRITE_PREFIX)
+        cms = timed(lambda: [step(i + 1, lat, txt, qi.QI_KV_READ_PREFIX) for i in range(args.steps)])
+        extra["cached_step"] = {"value": aggregate_throughput(world, args.steps, cms),
+                                "unit": "steps/s", "ms_per_step": cms / args.steps,
+                                "note": "target rows only; prefix K/V read from the cache"}
+    else:
+        extra["seconds_per_40_steps"] = ms_max / 1e3
 
     if rank != 0:
         ranks.close()
