@@ -1695,9 +1695,9 @@ int qi_denoise_step_cfg(qi_ctx* ctx, const qi_model* model, float* latents, cons
     rows.row_set[0] = rows.row_set[1] = 1;
   } else {
     // the table only maps rows to row sets, so neighbouring groups with the
-    // same row set become one run ([text | references] of each sequence use
-    // the prefix set): a prompt and a negative prompt with up to 10
-    // references each still fit
+    // same row set become one run: [text | references] of each sequence use
+    // the prefix set, so a prompt and a negative prompt with any number of
+    // references make four runs
     for (int b = 0; b < 2; ++b)
       for (int g = 0; g < sp[b].gt.n; ++g) {
         const int end = (b ? sp[0].S : 0) + sp[b].gt.end[g];

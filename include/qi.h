@@ -565,11 +565,10 @@ int qi_step_cfg_workspace_bytes(const qi_dims* dims, int S_cond, int S_uncond, i
  * in fp32 with one rounding per operation and no fused multiply-add (the pages
  * give the guidance scale but no formula; this is the plain reading, with no
  * renormalization).  latents [N, P] fp32 (in/out); v_out [N, P] fp32 gets the
- * guided v if not NULL.  Both target groups must hold N tokens; in uncached
- * modes the two sequences together may have at most QI_MAX_GROUPS runs of
- * neighbouring groups with equal row sets (QI_ERR_UNSUPPORTED_SHAPE otherwise;
- * [text | references | target] with the usual prefix / target row sets is two
- * runs per sequence, whatever the number of references).
+ * guided v if not NULL.  Both target groups must hold N tokens; each sequence
+ * may have up to QI_MAX_GROUPS groups (its prefix groups use row set 0 and its
+ * target row set 1, as for qi_denoise_step, so the batch's table of row sets
+ * holds two runs per sequence whatever the number of references).
  * kv_mode applies to both sequences (each with its own kv_cache). */
 int qi_denoise_step_cfg(qi_ctx* ctx, const qi_model* model, float* latents, const qi_seq* cond,
                         const qi_seq* uncond, float guidance, float sigma, float sigma_next,

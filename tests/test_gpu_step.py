@@ -77,9 +77,12 @@ class Setup:
                                synth.Group("image", 64, (8, 8)))),
     synth.TINY.replace(name="tiny_edit_10ref", blocks=2, patch=64,
                        groups=(synth.Group("text", 12),) + REF10 + (synth.Group("image", 64, (8, 8)),)),
+    synth.TINY.replace(name="tiny_edit_14ref", blocks=2, patch=64,
+                       groups=(synth.Group("text", 12),) + REF10 + REF10[:4] + (synth.Group("image", 64, (8, 8)),)),
     synth.TINY.replace(name="tiny_pages", blocks=6, precision="pages"),
     synth.TINY.replace(name="tiny_mxfp4", blocks=3, patch=64, precision="mxfp4")],
-    ids=["2blk", "32blk", "edit", "edit_3ref", "edit_10ref", "pages_mask_6blk", "mxfp4_3blk"])
+    ids=["2blk", "32blk", "edit", "edit_3ref", "edit_10ref", "edit_14ref_max_groups", "pages_mask_6blk",
+         "mxfp4_3blk"])
 def test_step_vs_oracle(ctx, cfg):
     s = Setup(ctx, cfg)
     sig = O.sigma_schedule(40, cfg.target_tokens)
@@ -257,6 +260,25 @@ def test_cfg_rejects_mismatched_targets(ctx):
     with pytest.raises(qi.QiError) as e:
         qi.qi_denoise_step_cfg(ctx, s.c.model, latg, s.seq(s.c, qi.QI_KV_NONE),
                                s.seq(bad, qi.QI_KV_NONE), 2.0, 1.0, 0.9, qi.QI_KV_NONE, None, s.ws)
+    assert e.value.code == qi.QI_ERR_INVALID_ARG
+    torch.cuda.synchronize()
+    assert torch.equal(latg, before)
+
+
+def test_cfg_rejects_row_sets_other_than_prefix_and_target(ctx):
+    """The step fixes the row sets (0 for text and references, 1 for the
+    target), so each sequence is two runs of the batch's row table whatever
+    its number of references; other row sets are rejected before any launch,
+    latents untouched."""
+    s = CfgSetup(ctx, refs=10)
+    alt = lambda st: qi.groups_struct(st.ends, [g % 2 for g in range(len(st.ends))])
+    sc, su = s.seq(s.c, qi.QI_KV_NONE), s.seq(s.u, qi.QI_KV_NONE)
+    gc, gu = alt(s.c), alt(s.u)
+    sc.groups, su.groups = qi.C.pointer(gc), qi.C.pointer(gu)
+    latg = cuda(s.c.lat)
+    before = latg.clone()
+    with pytest.raises(qi.QiError) as e:
+        qi.qi_denoise_step_cfg(ctx, s.c.model, latg, sc, su, 2.0, 1.0, 0.9, qi.QI_KV_NONE, None, s.ws)
     assert e.value.code == qi.QI_ERR_INVALID_ARG
     torch.cuda.synchronize()
     assert torch.equal(latg, before)
