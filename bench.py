@@ -75,7 +75,8 @@ def algorithmic_work(cfg: synth.DitConfig, cached: bool = False):
     # HBM bytes of the four activation quantizers per row: LN1 reads the fp32
     # residual (4H) and writes int8 codes (H); the attention-output quantizer
     # reads bf16 (2H) and writes H; LN2 reads the residual and the output
-    # projection (4H + 2H), writes the residual back (4H) and the codes (H);
+    # projection (4H + 2H) and writes the codes (H) (the down projection's
+    # epilogue adds the output projection's gated term to the stream itself);
     # the GELU-output quantizer reads 2F and writes F.  Plus 8 bytes (scale,
     # zero point) per row and quantizer, and the final LayerNorm (4H in, 2H out
     # per target row).
@@ -87,7 +88,7 @@ def algorithmic_work(cfg: synth.DitConfig, cached: bool = False):
         b += (H + 8) if w8["qk"] else 0                       # ... writes codes for W8A8 q, k
         b += 2 * H if not (w8["qk"] and w8["v"]) else 0       # ... and bf16 u for a BF16 part
         b += (3 * H + 8) if w8["out"] else 0                  # attention-output quantizer
-        b += 10 * H + ((H + 8) if w8["up"] else 2 * H)        # LN2 with the residual add
+        b += 6 * H + ((H + 8) if w8["up"] else 2 * H)         # LN2 with the residual add
         b += (3 * F + 8) if w8["down"] else 0                 # GELU-output quantizer
         quant += rows * b
     # GEMV weight bytes: the adaLN rows of every block (6H x H bf16), the final

@@ -278,8 +278,9 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, ui
 namespace {
 
 struct QuantExtras {
-  const uint16_t* res_y = nullptr;     // LN: residual add x += gate * y first
+  const uint16_t* res_y = nullptr;     // LN: residual add x + gate * y first ...
   const uint16_t* res_gate = nullptr;
+  float* res_out = nullptr;            // ... written here if set
   uint32_t* zero_range = nullptr;      // LN: clear these row ranges
   uint32_t* zero_words = nullptr;      // LN: clear these words (n_zero_words of them)
   int n_zero_words = 0;
@@ -313,6 +314,7 @@ int run_quant(qi_ctx* ctx, const void* x, bool xbf16, int M, int K, int ldx,
   memset(&p, 0, sizeof(p));
   p.res_y = ex.res_y;
   p.res_gate = ex.res_gate;
+  p.res_out = ex.res_out;
   p.zero_range = ex.zero_range;
   p.zero_words = ex.n_zero_words > 0 ? ex.zero_words : nullptr;
   p.n_zero_words = ex.n_zero_words;
@@ -345,7 +347,8 @@ int run_quant(qi_ctx* ctx, const void* x, bool xbf16, int M, int K, int ldx,
 int run_w8a8(qi_ctx* ctx, const int8_t* qa, const float* sa, const int32_t* zp, int M,
              const qi_w8& w, int epi, uint16_t* y, int ldy, float* res, int ldr,
              const uint16_t* gate, int gate_ld, const qi::GroupTable& gt, int row0,
-             int32_t* acc_debug, cudaStream_t st, uint32_t* row_range = nullptr) {
+             int32_t* acc_debug, cudaStream_t st, uint32_t* row_range = nullptr,
+             const uint16_t* res_y = nullptr, int ld_res_y = 0, const uint16_t* gate1 = nullptr) {
   if (M == 0) return QI_OK;
   qi::GemmParams p;
   memset(&p, 0, sizeof(p));
@@ -364,6 +367,9 @@ int run_w8a8(qi_ctx* ctx, const int8_t* qa, const float* sa, const int32_t* zp, 
   p.ldyf = ldr;
   p.gate = gate;
   p.gate_ld = gate_ld;
+  p.res_y = res_y;
+  p.ld_res_y = ld_res_y;
+  p.gate1 = gate1;
   p.groups = gt;
   p.row0 = row0;
   p.acc_debug = acc_debug;
@@ -700,21 +706,23 @@ int run_block_multi(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, fl
     if ((r = run_bf16_block_linear(ctx, b.o, T, H, w.out_bf16, w.out_mx, qi::EPI_BF16, p, st, mxb)))
       return r;
   }
-  // MLP half: x += gate1 * out, LN2 + modulate + quantize (and/or the bf16
-  // value for a BF16 up projection, into the attention-output buffer, now
-  // consumed); clears the GELU ranges
+  // MLP half: LN2 + modulate + quantize of x + gate1 * out (and/or the
+  // bf16 value for a BF16 up projection, into the attention-output buffer,
+  // now consumed); clears the GELU ranges.  The stream itself is not written
+  // here: the down projection's epilogue adds gate1 * out (y_out, untouched
+  // until the next block's QKV projection) along with its own term.
   {
     QuantExtras ex;
     ex.res_y = y_out;
     ex.res_gate = mod + 2 * H;
+    ex.res_out = tp ? tp->x_mid : nullptr;
     ex.zero_range = b.g_range;
     ex.u_f32 = tp ? tp->u2 : nullptr;
     ex.quant_too = bp.up_w8;
     if ((r = run_quant(ctx, x, false, T, H, H, mod + 3 * H, mod + 4 * H, mld, gt, row0, d.eps,
                        b.uq, b.sa, b.zp, bp.up_w8 ? nullptr : b.o, st, ex)))
       return r;
-    if (tp && ((r = tap_copy(tp->x_mid, x, static_cast<size_t>(T) * H * 4, st)) ||
-               (bp.up_w8 && (r = tap_codes(tp->q2, tp->s2, tp->zp2, b.uq, b.sa, b.zp, T, H, st)))))
+    if (tp && bp.up_w8 && (r = tap_codes(tp->q2, tp->s2, tp->zp2, b.uq, b.sa, b.zp, T, H, st)))
       return r;
   }
   uint32_t* g_range = bp.down_w8 ? b.g_range : nullptr;
@@ -744,7 +752,7 @@ int run_block_multi(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, fl
       if (tp && (r = tap_codes(tp->qg, tp->sg, tp->zpg, b.uq, b.sa, b.zp, T, F, st))) return r;
     }
     if ((r = run_w8a8(ctx, b.uq, b.sa, b.zp, T, w.down, qi::EPI_GATED, nullptr, 0, x, H,
-                      mod + 5 * H, mld, gt, row0, nullptr, st)))
+                      mod + 5 * H, mld, gt, row0, nullptr, st, nullptr, y_out, H, mod + 2 * H)))
       return r;
   } else {
     qi::GemmParams p;
@@ -753,6 +761,9 @@ int run_block_multi(qi_ctx* ctx, const qi_dims& d, const qi_block_weights& w, fl
     p.ldyf = H;
     p.gate = mod + 5 * H;
     p.gate_ld = mld;
+    p.res_y = y_out;
+    p.ld_res_y = H;
+    p.gate1 = mod + 2 * H;
     p.groups = gt;
     p.row0 = row0;
     if ((r = run_bf16_block_linear(ctx, b.g, T, F, w.down_bf16, w.down_mx, qi::EPI_GATED, p,

@@ -350,7 +350,9 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const ColTabl
             d4[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
       }
     } else if (EPI == EPI_GATED) {
-      // x += gate * bf16(y)  (fp32 residual stream)
+      // x += gate * bf16(y)  (fp32 residual stream); with res_y, x first
+      // becomes x + gate1 * res_y, one rounding, as the LayerNorm before this
+      // Linear computed it
       float4* dst = reinterpret_cast<float4*>(p.yf + static_cast<size_t>(m) * p.ldyf + nb);
       const uint4* g4 =
           reinterpret_cast<const uint4*>(p.gate + static_cast<size_t>(rs) * p.gate_ld + nb);
@@ -360,6 +362,20 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, const ColTabl
         const uint4 gr = __ldg(g4 + j);
         const uint32_t gw[4] = {gr.x, gr.y, gr.z, gr.w};
         float4 a = dst[2 * j], b = dst[2 * j + 1];
+        if (p.res_y) {
+          const uint4 g1 = __ldg(reinterpret_cast<const uint4*>(
+                                     p.gate1 + static_cast<size_t>(rs) * p.gate_ld + nb) + j);
+          const uint4 y1 = __ldg(reinterpret_cast<const uint4*>(
+                                     p.res_y + static_cast<size_t>(m) * p.ld_res_y + nb) + j);
+          a.x = fmaf(__uint_as_float(g1.x << 16), __uint_as_float(y1.x << 16), a.x);
+          a.y = fmaf(__uint_as_float(g1.x & 0xFFFF0000u), __uint_as_float(y1.x & 0xFFFF0000u), a.y);
+          a.z = fmaf(__uint_as_float(g1.y << 16), __uint_as_float(y1.y << 16), a.z);
+          a.w = fmaf(__uint_as_float(g1.y & 0xFFFF0000u), __uint_as_float(y1.y & 0xFFFF0000u), a.w);
+          b.x = fmaf(__uint_as_float(g1.z << 16), __uint_as_float(y1.z << 16), b.x);
+          b.y = fmaf(__uint_as_float(g1.z & 0xFFFF0000u), __uint_as_float(y1.z & 0xFFFF0000u), b.y);
+          b.z = fmaf(__uint_as_float(g1.w << 16), __uint_as_float(y1.w << 16), b.z);
+          b.w = fmaf(__uint_as_float(g1.w & 0xFFFF0000u), __uint_as_float(y1.w & 0xFFFF0000u), b.w);
+        }
         a.x += __uint_as_float(gw[0] << 16) * bf16_round_f(v[8 * j + 0]);
         a.y += __uint_as_float(gw[0] & 0xFFFF0000u) * bf16_round_f(v[8 * j + 1]);
         a.z += __uint_as_float(gw[1] << 16) * bf16_round_f(v[8 * j + 2]);

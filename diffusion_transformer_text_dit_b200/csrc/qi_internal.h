@@ -77,6 +77,12 @@ struct GemmParams {
   int ldyf;
   const uint16_t* gate;   // bf16: gate of row set r at gate + r * gate_ld
   int gate_ld;
+  // EPI_GATED: if res_y is set, each residual value x first becomes
+  // x + gate1 * res_y (one rounding; gate1 rows like gate's): the mid-block
+  // residual the LayerNorm before this Linear used without storing it
+  const uint16_t* res_y;  // bf16 [M, ld_res_y] or null
+  int ld_res_y;
+  const uint16_t* gate1;
   GroupTable groups;      // row sets of global tokens
   int row0;               // global token index of row 0
   int32_t* acc_debug;     // optional raw int32 accumulators [M, N]
@@ -143,9 +149,11 @@ struct QuantParams {
   int32_t* zp;            // [M]
   uint16_t* u_bf16;       // if non-null: write bf16(u) [M, ldq] instead of quantizing ...
   int quant_too;          // ... or as well as quantizing (LN variant)
-  // LN variant: residual add before the LayerNorm, x += gate[row set] * y
+  // LN variant: residual add before the LayerNorm, x + gate[row set] * y,
+  // written to res_out (fp32 [M, ldx]) if that is set
   const uint16_t* res_y;  // bf16 [M, K] or null
   const uint16_t* res_gate;   // gate row of set r at res_gate + r * mod_ld
+  float* res_out;
   uint32_t* zero_range;   // if non-null: rows' [2] range words set to 0 (for a later producer)
   uint32_t* zero_words;   // LN variant, if non-null: n_zero_words words set to 0 (by the first row)
   int n_zero_words;

@@ -177,7 +177,8 @@ __device__ __forceinline__ void unit_pairs(const uint4 u, uint64_t (&d)[XBF16 ? 
 // instruction of a warp reads one contiguous segment of the row.  The values
 // are used by three passes (sums, modulate + range, codes), so they stay in
 // registers.  Optionally the gated residual of the preceding Linear is added
-// first (x += gate * y, written back to the fp32 stream).
+// first (x + gate * y, one rounding; written out only if asked: the Linear
+// after the LayerNorm can recompute it where it updates the stream).
 constexpr int LN_CH = 4;
 
 template <bool XBF16>
@@ -216,7 +217,7 @@ __global__ void __launch_bounds__(512) quant_ln_kernel(const QuantParams p) {
   const int rs = p.groups.row_set[group_of(p.groups, p.row0 + row)];
   if (!XBF16 && p.res_y) {
     const uint16_t* gt = p.res_gate + static_cast<int64_t>(rs) * p.mod_ld;
-    float* xw = const_cast<float*>(static_cast<const float*>(p.x)) + static_cast<int64_t>(row) * p.ldx;
+    float* xw = p.res_out ? p.res_out + static_cast<int64_t>(row) * p.ldx : nullptr;
 #pragma unroll
     for (int c = 0; c < LN_CH; ++c) {
       const int ch = tid + c * nt;
@@ -226,6 +227,7 @@ __global__ void __launch_bounds__(512) quant_ln_kernel(const QuantParams p) {
       load_bf16_pairs<4>(gt + ch * 8, fg);
 #pragma unroll
       for (int i = 0; i < 4; ++i) v[c][i] = f2_fma(fg[i], fy[i], v[c][i]);
+      if (!xw) continue;
       float e[8];
 #pragma unroll
       for (int i = 0; i < 4; ++i) f2_unpack(v[c][i], e[2 * i], e[2 * i + 1]);
@@ -464,7 +466,7 @@ int launch_quant(const QuantParams& p, cudaStream_t st) {
   if (p.M == 0) return 0;
   if (p.K <= 0 || p.K % 8 != 0 || p.K > 16384) return -1;
   if (p.ln && p.range) return -1;                 // LN computes its own range
-  if (p.res_y && (!p.ln || p.x_bf16)) return -1;  // the residual add writes the fp32 stream
+  if (p.res_y && (!p.ln || p.x_bf16)) return -1;  // the residual add is on the fp32 stream
   if (p.ln) return p.x_bf16 ? launch_quant_ln_t<true>(p, st) : launch_quant_ln_t<false>(p, st);
   // the row copy needs 16-byte aligned rows
   const int esz = p.x_bf16 ? 2 : 4;

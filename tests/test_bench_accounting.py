@@ -106,3 +106,13 @@ def test_clock_summary_without_a_window_uses_every_sample():
                 "Not Active, Not Active", "garbage"]
     out = cs.stop()
     assert out["samples"] == 1 and not out["in_timed_region"] and out["reasons"] == []
+
+
+def test_quantizer_bytes_of_the_1024px_step():
+    """Per row and block: LN1 4H + H + 8, attention-output quantizer
+    3H + 8, LN2 6H + H + 8 (residual and output projection in, codes out),
+    GELU-output quantizer 3F + 8; plus the final LayerNorm 6H per target row."""
+    w = bench.algorithmic_work(synth.STEP1024)
+    S = 4608
+    per_row = (5 * H + 8) + (3 * H + 8) + (7 * H + 8) + (3 * F + 8)
+    assert w["quant_bytes_per_step"] == S * per_row * 32 + 4096 * 6 * H
