@@ -74,13 +74,15 @@ int launch_qk_norm_rope(const QkNormRopeParams& p, cudaStream_t st) {
 
 // y[r][j] = sum_k act(x[r][k]) * W[j][k] + b[j] for every row j of every job.
 // x (R <= 2 rows) is staged in shared memory as fp32 (SiLU applied on load
-// when requested).  One warp handles 4 consecutive weight rows at a time:
-// every lane streams 4 x 16 bytes of weights per step and reuses the x values
-// it read from shared memory for all 4 rows; 8 independent accumulators keep
+// when requested).  One warp handles 8 consecutive weight rows at a time:
+// every lane streams 8 x 16 bytes of weights per step and reuses the x values
+// it read from shared memory for all 8 rows; 16 independent accumulators keep
 // the FMA chains short.  The weights are read once: the kernel is bound by
-// HBM bandwidth (6.4 GB of adaLN weights per 32-block step).
+// HBM bandwidth (6.4 GB of adaLN weights per 32-block step).  8 rows a warp
+// keep 128 bytes a lane in flight: 1.08 ms per 1024^2 step against 1.18 with
+// 4 rows (each row's sum is the same sequence of operations either way).
 constexpr int GEMV_THREADS = 256;
-constexpr int GEMV_ROWS = 4;
+constexpr int GEMV_ROWS = 8;
 
 __device__ __forceinline__ float dot8(const uint4 w, const float4 a, const float4 b, float acc) {
   acc = fmaf(__uint_as_float(w.x << 16), a.x, acc);
@@ -121,7 +123,7 @@ __global__ void __launch_bounds__(GEMV_THREADS) gemv_kernel(const GemvParams p) 
     const GemvJob& J = p.jobs[job];
     const int row0 = grp * GEMV_ROWS;
     const uint16_t* w0 = J.w + static_cast<int64_t>(row0) * p.k;
-    float a0[GEMV_ROWS] = {0.f, 0.f, 0.f, 0.f}, a1[GEMV_ROWS] = {0.f, 0.f, 0.f, 0.f};
+    float a0[GEMV_ROWS] = {}, a1[GEMV_ROWS] = {};
 #pragma unroll 2
     for (int kk = lane * 8; kk < p.k; kk += 256) {
       uint4 w[GEMV_ROWS];
